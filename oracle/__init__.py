@@ -1,0 +1,249 @@
+"""CPU oracle for the binary (+1/-1) matrix product -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  It shares no code with the CUDA path
+(``xnor_popcount_gemm_bnn_b200``) and never imports it.
+
+What it computes is the plain definition of the method, with +1/-1 values
+materialised and integers multiplied and added (``bnn_oracle.c``), and the
+real-valued epilogues evaluated in float64 here with numpy:
+
+* sign -- "Extreme Quantization: Binary, Ternary & 1-bit LLMs", Notation
+  (sign(x) = +1 for x >= 0, -1 for x < 0) and eq. (4) of the XNOR-Net section.
+* packed encoding -- "First Principles: Why Binary Ops Can Be Exponentially
+  Faster", section "1. Arithmetic: MAC -> XNOR + popcount" (bit 0 is +1,
+  bit 1 is -1, pad bits encode +1).
+* alpha and the scaled product -- "Extreme Quantization ...", Binary Neural
+  Networks section, eq. (1): y = alpha * (w_b^T x), alpha = (1/n) sum |w_i|.
+* BatchNorm before re-binarisation -- "Binary Neural Network (BNN)" glossary
+  page, the BatchNorm paragraph (BN stabilises the inputs to each binarised
+  layer; per-filter alpha multiplies the binary product).  The pages give no
+  BN formula; the oracle uses standard inference BatchNorm on alpha*s,
+  evaluated in float64 in the order ((alpha*s - mean) / sqrt(var + eps)) *
+  gamma + beta, and maps a result >= 0 to +1 (the same tie rule as sign).
+
+Readings of the pages made here (all listed with reasons in the design notes):
+sign(-0.0) = +1, sign(NaN) = +1, bit j of word w is element 32*w + j, rows
+padded to a multiple of 4 words, alpha over the true K from the real weights,
+convolution padding value +1, BN decisions taken with alpha rounded to fp32
+(the precision the product stores alpha in).
+
+Parity pins for every function live in ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        i64, p = ctypes.c_int64, ctypes.c_void_p
+        lib.oracle_ld_words.argtypes = [i64]
+        lib.oracle_ld_words.restype = i64
+        lib.oracle_sign_f32.argtypes = [p, i64, p]
+        lib.oracle_pack_pm1.argtypes = [p, i64, i64, p, i64]
+        lib.oracle_alpha_f32.argtypes = [p, i64, i64, p]
+        lib.oracle_matmul_pm1.argtypes = [p, p, i64, i64, i64, p]
+        lib.oracle_conv2d_pm1.argtypes = [p, i64, i64, i64, i64, p, i64, i64, i64, i64, p]
+        lib.oracle_num_threads.restype = ctypes.c_int
+        for name in ("oracle_sign_f32", "oracle_pack_pm1", "oracle_alpha_f32",
+                     "oracle_matmul_pm1", "oracle_conv2d_pm1"):
+            getattr(lib, name).restype = None
+        _LIB = lib
+    return _LIB
+
+
+def _f32(x) -> np.ndarray:
+    """Accept numpy arrays or CPU torch tensors (fp32 or bf16; bf16 widens exactly)."""
+    if hasattr(x, "detach"):
+        import torch
+        t = x.detach().cpu()
+        if t.dtype != torch.float32:
+            t = t.to(torch.float32)
+        x = t.numpy()
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    return int(_lib().oracle_num_threads())
+
+
+def ld_words(K: int) -> int:
+    """Words per packed row: ceil(K/32) rounded up to a multiple of 4."""
+    return int(_lib().oracle_ld_words(int(K)))
+
+
+def sign_pm1(x) -> np.ndarray:
+    """int8 +1/-1 of the same shape: -1 exactly where x < 0 (Notation, eq. (4))."""
+    xf = _f32(x)
+    out = np.empty(xf.shape, dtype=np.int8)
+    _lib().oracle_sign_f32(_ptr(xf), xf.size, _ptr(out))
+    return out
+
+
+def pack_pm1(b: np.ndarray, ld: int | None = None) -> np.ndarray:
+    """Pack a [rows, K] int8 +1/-1 matrix into uint32 [rows, ld] words."""
+    b = np.ascontiguousarray(b, dtype=np.int8)
+    if b.ndim == 1:
+        b = b[None, :]
+    rows, K = b.shape
+    ld = ld_words(K) if ld is None else int(ld)
+    out = np.empty((rows, ld), dtype=np.uint32)
+    _lib().oracle_pack_pm1(_ptr(b), rows, K, _ptr(out), ld)
+    return out
+
+
+def pack_real(x, ld: int | None = None) -> np.ndarray:
+    """sign() then pack, for a real [rows, K] matrix."""
+    return pack_pm1(sign_pm1(x), ld)
+
+
+def alpha(w) -> np.ndarray:
+    """float64 [rows]: mean |w| over each row's true K (eq. (1))."""
+    wf = _f32(w)
+    if wf.ndim == 1:
+        wf = wf[None, :]
+    rows, K = wf.shape
+    out = np.empty(rows, dtype=np.float64)
+    _lib().oracle_alpha_f32(_ptr(wf), rows, K, _ptr(out))
+    return out
+
+
+def alpha_f32(w) -> np.ndarray:
+    """alpha rounded once to fp32 (round to nearest)."""
+    return alpha(w).astype(np.float32)
+
+
+def matmul_pm1(a: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """int32 [M, N] = a @ w^T for int8 +1/-1 a [M, K] and w [N, K]."""
+    a = np.ascontiguousarray(a, dtype=np.int8)
+    w = np.ascontiguousarray(w, dtype=np.int8)
+    if a.ndim == 1:
+        a = a[None, :]
+    M, K = a.shape
+    N, K2 = w.shape
+    assert K == K2, (K, K2)
+    s = np.empty((M, N), dtype=np.int32)
+    _lib().oracle_matmul_pm1(_ptr(a), _ptr(w), M, N, K, _ptr(s))
+    return s
+
+
+def gemv_pm1(w: np.ndarray, x: np.ndarray) -> np.ndarray:
+    """int32 [N] = w @ x for int8 +1/-1 w [N, K] and x [K]."""
+    return matmul_pm1(np.asarray(x, dtype=np.int8)[None, :], w)[0]
+
+
+def conv2d_pm1(x: np.ndarray, f: np.ndarray, stride: int = 1, pad: int = 1) -> np.ndarray:
+    """int32 NCHW output of a square-kernel convolution on +1/-1 tensors,
+    padded taps reading +1."""
+    x = np.ascontiguousarray(x, dtype=np.int8)
+    f = np.ascontiguousarray(f, dtype=np.int8)
+    n, c, h, wd = x.shape
+    cout, c2, kk, kk2 = f.shape
+    assert c == c2 and kk == kk2
+    oh = (h + 2 * pad - kk) // stride + 1
+    ow = (wd + 2 * pad - kk) // stride + 1
+    out = np.empty((n, cout, oh, ow), dtype=np.int32)
+    _lib().oracle_conv2d_pm1(_ptr(x), n, c, h, wd, _ptr(f), cout, kk, stride, pad, _ptr(out))
+    return out
+
+
+# ---------------------------------------------------------------------------
+# epilogues, float64
+# ---------------------------------------------------------------------------
+
+def scaled(s: np.ndarray, alpha_n: np.ndarray) -> np.ndarray:
+    """alpha_n * s_mn in float64; alpha indexes the last axis (output channel)."""
+    return np.asarray(alpha_n, dtype=np.float64) * np.asarray(s, dtype=np.float64)
+
+
+def affine(s: np.ndarray, alpha_n, gamma, beta) -> np.ndarray:
+    """gamma_n * (alpha_n * s) + beta_n in float64 (last axis = channel)."""
+    a = np.asarray(alpha_n, dtype=np.float64)
+    g = np.asarray(gamma, dtype=np.float64)
+    b = np.asarray(beta, dtype=np.float64)
+    return g * (a * np.asarray(s, dtype=np.float64)) + b
+
+
+def bn_value(s: np.ndarray, alpha_n_f32, gamma, beta, mean, var, eps: float) -> np.ndarray:
+    """Inference BatchNorm of alpha*s in float64: ((alpha*s - mean)/sqrt(var+eps))*gamma + beta."""
+    a = np.asarray(alpha_n_f32, dtype=np.float32).astype(np.float64)
+    x = a * np.asarray(s, dtype=np.float64)
+    mu = np.asarray(mean, dtype=np.float32).astype(np.float64)
+    v = np.asarray(var, dtype=np.float32).astype(np.float64)
+    g = np.asarray(gamma, dtype=np.float32).astype(np.float64)
+    b = np.asarray(beta, dtype=np.float32).astype(np.float64)
+    return (x - mu) / np.sqrt(v + float(eps)) * g + b
+
+
+def bn_sign(s, alpha_n_f32, gamma, beta, mean, var, eps: float) -> np.ndarray:
+    """int8 +1/-1: +1 where the BatchNorm value is >= 0 (tie goes to +1, as sign(0))."""
+    y = bn_value(s, alpha_n_f32, gamma, beta, mean, var, eps)
+    return np.where(y >= 0.0, 1, -1).astype(np.int8)
+
+
+# ---------------------------------------------------------------------------
+# whole layers, composed from the definitions above
+# ---------------------------------------------------------------------------
+
+def binary_linear(x_real, w_real):
+    """XNOR-Net linear layer: s = sign(x) sign(W)^T, alpha from the real W.
+
+    Returns (s int32 [M, N], alpha float64 [N])."""
+    a = sign_pm1(x_real)
+    if a.ndim == 1:
+        a = a[None, :]
+    wb = sign_pm1(w_real)
+    return matmul_pm1(a, wb), alpha(w_real)
+
+
+def conv3x3_affine(x_real, w_real, gamma, beta, stride: int = 1, pad: int = 1):
+    """Binary 3x3 convolution with per-output-channel alpha and an affine epilogue.
+
+    Returns (s int32 NCHW, y float64 NCHW)."""
+    xb = sign_pm1(x_real)
+    fb = sign_pm1(w_real)
+    cout = fb.shape[0]
+    s = conv2d_pm1(xb, fb, stride, pad)
+    a = alpha(_f32(w_real).reshape(cout, -1))
+    y = affine(np.moveaxis(s, 1, -1), a, gamma, beta)
+    return s, np.moveaxis(y, -1, 1)
+
+
+def mlp_forward(x0_real, ws_real, bns):
+    """Fully binary MLP: sign the input, then for each layer the +1/-1 product
+    with sign(W_l); layers before the last re-binarise through BatchNorm of
+    alpha*s; the last layer returns alpha*s in float64.
+
+    ``bns`` is a list of (gamma, beta, mean, var, eps), one per hidden layer.
+    Returns (list of int8 +1/-1 activations entering each layer, logits)."""
+    a = sign_pm1(x0_real)
+    if a.ndim == 1:
+        a = a[None, :]
+    acts = [a]
+    L = len(ws_real)
+    logits = None
+    for l, w in enumerate(ws_real):
+        s = matmul_pm1(a, sign_pm1(w))
+        al = alpha(w)
+        if l < L - 1:
+            g, b, mu, var, eps = bns[l]
+            a = bn_sign(s, al.astype(np.float32), g, b, mu, var, eps)
+            acts.append(a)
+        else:
+            logits = scaled(s, al)
+    return acts, logits

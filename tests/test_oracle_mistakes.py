@@ -1,0 +1,171 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and show that the pins
+of ``test_oracle_pins.py`` catch every one of them.
+
+Each mutant is the oracle with one function replaced by a numpy version that
+carries a single slip: a wrong tie rule, a reversed bit order, a dropped term,
+a transposed operand, a wrong pad value, a wrong divisor...
+"""
+import types
+
+import numpy as np
+import pytest
+
+import oracle
+from test_oracle_pins import ALL_CHECKS
+
+
+def _mutant(**overrides):
+    ns = types.SimpleNamespace(**{k: getattr(oracle, k) for k in dir(oracle) if not k.startswith("_")})
+    for k, v in overrides.items():
+        setattr(ns, k, v)
+    # composite helpers must see the mutated primitives
+    ns.mlp_forward = lambda x0, ws, bns: _mlp_with(ns, x0, ws, bns)
+    return ns
+
+
+def _mlp_with(o, x0, ws, bns):
+    a = o.sign_pm1(x0)
+    acts = [a]
+    logits = None
+    for l, w in enumerate(ws):
+        s = o.matmul_pm1(a, o.sign_pm1(w))
+        al = o.alpha(w)
+        if l < len(ws) - 1:
+            g, b, mu, var, eps = bns[l]
+            a = o.bn_sign(s, al.astype(np.float32), g, b, mu, var, eps)
+            acts.append(a)
+        else:
+            logits = o.scaled(s, al)
+    return acts, logits
+
+
+def _sign_gt(x):                       # 0 -> -1 (the glossary's reading)
+    x = oracle._f32(x)
+    return np.where(x > 0, 1, -1).astype(np.int8)
+
+
+def _sign_bit(x):                      # sign-bit test: -0.0 -> -1
+    x = oracle._f32(x)
+    return np.where(np.signbit(x), -1, 1).astype(np.int8)
+
+
+def _pack_msb(b, ld=None):             # bit order reversed inside a word
+    b = np.atleast_2d(np.asarray(b, np.int8))
+    rows, K = b.shape
+    ld = oracle.ld_words(K) if ld is None else ld
+    out = np.zeros((rows, ld), np.uint32)
+    for r in range(rows):
+        for k in range(K):
+            if b[r, k] == -1:
+                out[r, k // 32] |= np.uint32(1 << (31 - k % 32))
+    return out
+
+
+def _pack_inverted(b, ld=None):        # bit 1 for +1
+    b = np.atleast_2d(np.asarray(b, np.int8))
+    return oracle.pack_pm1((-b).astype(np.int8), ld)
+
+
+def _ld_no_round(K):                   # rows not padded to 4 words
+    return (int(K) + 31) // 32
+
+
+def _alpha_padded(w):                  # divides by the padded length
+    w = np.atleast_2d(oracle._f32(w)).astype(np.float64)
+    K = w.shape[1]
+    return np.abs(w).sum(axis=1) / (32 * oracle.ld_words(K))
+
+
+def _alpha_noabs(w):                   # mean of w, not of |w|
+    w = np.atleast_2d(oracle._f32(w)).astype(np.float64)
+    return np.abs(w.sum(axis=1)) / w.shape[1]
+
+
+def _matmul_transposed(a, w):          # reads w as [K, N] storage
+    a = np.atleast_2d(np.asarray(a, np.int64))
+    w = np.asarray(w, np.int64)
+    N, K = w.shape
+    wt = w.reshape(-1)[: N * K].reshape(K, N).T
+    return (a @ wt.T).astype(np.int32)
+
+
+def _matmul_drop_first(a, w):          # loop starts at k = 1
+    a = np.atleast_2d(np.asarray(a, np.int64))
+    w = np.asarray(w, np.int64)
+    return (a[:, 1:] @ w[:, 1:].T).astype(np.int32)
+
+
+def _conv_pad_minus(x, f, stride=1, pad=1):   # padded taps read -1
+    import torch
+    import torch.nn.functional as F
+    xt = F.pad(torch.from_numpy(np.asarray(x, np.float64)), (pad,) * 4, value=-1.0)
+    return F.conv2d(xt, torch.from_numpy(np.asarray(f, np.float64)), stride=stride).numpy().astype(np.int32)
+
+
+def _conv_flipped(x, f, stride=1, pad=1):     # true convolution (flipped kernel)
+    return oracle.conv2d_pm1(x, np.ascontiguousarray(np.asarray(f)[:, :, ::-1, ::-1]), stride, pad)
+
+
+def _bn_value_no_gamma(s, a, g, b, mu, var, eps):
+    return oracle.bn_value(s, a, np.ones_like(np.asarray(g)), b, mu, var, eps)
+
+
+def _bn_value_mean_sign(s, a, g, b, mu, var, eps):
+    return oracle.bn_value(s, a, g, b, -np.asarray(mu), var, eps)
+
+
+def _bn_sign_strict(s, a, g, b, mu, var, eps):   # tie (value 0) goes to -1
+    y = oracle.bn_value(s, a, g, b, mu, var, eps)
+    return np.where(y > 0, 1, -1).astype(np.int8)
+
+
+MUTANTS = {
+    "sign_zero_negative": dict(sign_pm1=_sign_gt),
+    "sign_bit_test": dict(sign_pm1=_sign_bit),
+    "pack_msb_first": dict(pack_pm1=_pack_msb),
+    "pack_inverted_encoding": dict(pack_pm1=_pack_inverted),
+    "ld_not_rounded": dict(ld_words=_ld_no_round),
+    "alpha_padded_divisor": dict(alpha=_alpha_padded),
+    "alpha_without_abs": dict(alpha=_alpha_noabs),
+    "matmul_transposed_operand": dict(matmul_pm1=_matmul_transposed),
+    "matmul_dropped_term": dict(matmul_pm1=_matmul_drop_first),
+    "conv_pad_minus_one": dict(conv2d_pm1=_conv_pad_minus),
+    "conv_flipped_kernel": dict(conv2d_pm1=_conv_flipped),
+    "bn_missing_gamma": dict(bn_value=_bn_value_no_gamma),
+    "bn_mean_sign": dict(bn_value=_bn_value_mean_sign),
+}
+
+
+def _bn_sign_from_value(o):
+    def f(s, a, g, b, mu, var, eps):
+        y = o.bn_value(s, a, g, b, mu, var, eps)
+        return np.where(y >= 0.0, 1, -1).astype(np.int8)
+    return f
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(name, golden_dir):
+    o = _mutant(**MUTANTS[name])
+    if "bn_value" in MUTANTS[name]:
+        o.bn_sign = _bn_sign_from_value(o)
+    failed = []
+    for check_name, check in ALL_CHECKS:
+        try:
+            check(o, golden_dir)
+        except AssertionError:
+            failed.append(check_name)
+        except (ValueError, IndexError):
+            failed.append(check_name)
+    assert failed, f"planted mistake {name!r} passed every pin"
+
+
+def test_tie_rule_mistake_is_caught():
+    """A BN decision that sends an exact 0 to -1 contradicts the sign tie rule
+    (sign(0) = +1): an exact zero is reachable when mean = alpha*s and beta = 0."""
+    s = np.array([[4]], np.int32)
+    a = np.array([0.5], np.float32)
+    one = np.ones(1, np.float32)
+    zero = np.zeros(1, np.float32)
+    mu = np.array([2.0], np.float32)
+    assert oracle.bn_sign(s, a, one, zero, mu, one, 0.0)[0, 0] == 1
+    assert _bn_sign_strict(s, a, one, zero, mu, one, 0.0)[0, 0] == -1

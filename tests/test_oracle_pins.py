@@ -1,0 +1,315 @@
+"""Pins for the CPU oracle: checks against what the pages and the mathematics fix.
+
+None of these compares the oracle with itself.  Each check is one of: a value
+the pages fix (or a hand-computed answer to an exercise they pose), a closed
+form, an invariant, brute force on tiny inputs, or a special case that reduces
+to an independent library routine (torch float64 matmul / conv2d /
+batch_norm, numpy mean).
+
+The checks are written as functions of the oracle's functions so that
+``test_oracle_mistakes.py`` can run them against oracles with a planted
+mistake and show that every plausible slip fails at least one pin.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+import workloads
+
+
+def _popcount_u32(a: np.ndarray) -> np.ndarray:
+    """Per-element popcount of a uint32 array (test-side, independent of the oracle)."""
+    a = a.astype(np.uint64)
+    return np.array([int(v).bit_count() for v in a.ravel()], dtype=np.int64).reshape(a.shape)
+
+
+def all_pm1_vectors(K: int) -> np.ndarray:
+    """All 2^K vectors in {-1, +1}^K as int8 rows."""
+    rows = np.array(list(itertools.product([1, -1], repeat=K)), dtype=np.int8)
+    return rows
+
+
+# ---------------------------------------------------------------------------
+# pin checks (each returns normally or raises AssertionError)
+# ---------------------------------------------------------------------------
+
+def check_identity_bruteforce(o, Ks=range(1, 11)):
+    """eq. (6) of 'Extreme Quantization ...' (XNOR-Net) and the identity of
+    'First Principles ...', section 1: <w,x> = K - 2 popcount(w xor x),
+    over every pair of +1/-1 vectors for K = 1..10."""
+    for K in Ks:
+        V = all_pm1_vectors(K)
+        s = o.matmul_pm1(V, V)                       # plain sum of products
+        P = o.pack_pm1(V)                            # packed words
+        d = np.zeros((len(V), len(V)), dtype=np.int64)
+        for w in range(P.shape[1]):
+            x = P[:, w][:, None] ^ P[:, w][None, :]
+            d += _popcount_u32(x)
+        assert np.array_equal(s.astype(np.int64), K - 2 * d), f"identity fails at K={K}"
+
+
+def check_elementwise_xnor_form(o):
+    """eq. (5): w_b x_b = 2 XNOR(w~, x~) - 1 with w~ = (w_b + 1)/2, all four cases."""
+    for wb, xb in itertools.product([1, -1], repeat=2):
+        s = o.matmul_pm1(np.array([[xb]], np.int8), np.array([[wb]], np.int8))[0, 0]
+        wt, xt = (wb + 1) // 2, (xb + 1) // 2
+        xnor = 1 if wt == xt else 0
+        assert s == 2 * xnor - 1, (wb, xb, s)
+
+
+def check_exercise1(o, golden):
+    """Exercise 1 of 'Extreme Quantization ...' (hand-computed answer)."""
+    g = json.load(open(os.path.join(golden, "exercise1.json")))
+    w = np.array(g["w_b"], np.int8)
+    x = np.array(g["x_b"], np.int8)
+    assert o.matmul_pm1(x[None, :], w[None, :])[0, 0] == g["dot"]
+    pw, px = o.pack_pm1(w[None, :]), o.pack_pm1(x[None, :])
+    assert int(pw[0, 0]) == g["w_word"] and int(px[0, 0]) == g["x_word"]
+    assert int(pw[0, 0] ^ px[0, 0]) == g["xor_word"]
+    assert int(pw[0, 0] ^ px[0, 0]).bit_count() == g["popcount"]
+    K = len(g["w_b"])
+    assert K - 2 * g["popcount"] == g["dot"]
+
+
+def check_pack_examples(o, golden):
+    """Hand-computed packed words ('First Principles ...', section 1)."""
+    g = json.load(open(os.path.join(golden, "pack_examples.json")))
+    for case in g["cases"]:
+        K = case["K"]
+        b = np.ones((1, K), np.int8)
+        b[0, case["negative_positions"]] = -1
+        got = o.pack_pm1(b)
+        assert got.shape[1] == len(case["words"]), (K, got.shape)
+        assert [int(v) for v in got[0]] == case["words"], (K, got[0])
+
+
+def check_sign_rule(o, golden):
+    """Notation section of 'Extreme Quantization ...': +1 for x >= 0, -1 for x < 0."""
+    g = json.load(open(os.path.join(golden, "sign_rule.json")))
+    vals = np.array([float(v) for v, _ in g["cases"]], dtype=np.float32)
+    want = np.array([e for _, e in g["cases"]], dtype=np.int8)
+    assert np.array_equal(o.sign_pm1(vals), want), (o.sign_pm1(vals), want)
+    # bf16 inputs are taken as stored (widened exactly)
+    tb = torch.tensor(vals).to(torch.bfloat16)
+    wb = np.where(np.isnan(tb.float().numpy()) | (tb.float().numpy() >= 0), 1, -1)
+    assert np.array_equal(o.sign_pm1(tb), wb.astype(np.int8))
+
+
+def check_pad_rule(o, Ks=(1, 31, 33, 63, 65, 1000), seed=0):
+    """Pad bits encode +1 ('First Principles ...', section 1): pad bits are
+    0 and the identity uses the true K whatever the padding width."""
+    rng = np.random.default_rng(seed)
+    for K in Ks:
+        a = rng.choice(np.array([-1, 1], np.int8), size=(5, K))
+        w = rng.choice(np.array([-1, 1], np.int8), size=(7, K))
+        s = o.matmul_pm1(a, w).astype(np.int64)
+        for extra in (0, 4, 8):
+            ld = o.ld_words(K) + extra
+            pa, pw = o.pack_pm1(a, ld), o.pack_pm1(w, ld)
+            # pad bits of the last partial word and every pad word are zero
+            nbits = ld * 32
+            for r in range(pa.shape[0]):
+                bits = sum(int(v) << (32 * i) for i, v in enumerate(pa[r]))
+                assert bits >> K == 0, (K, extra)
+            d = np.zeros((5, 7), np.int64)
+            for i in range(ld):
+                d += _popcount_u32(pa[:, i][:, None] ^ pw[:, i][None, :])
+            assert np.array_equal(s, K - 2 * d), (K, extra)
+            assert nbits >= K
+        # 64-bit words see the same bytes (little-endian view of the uint32 rows)
+        p64 = o.pack_pm1(a).view(np.uint64)
+        d64 = np.zeros((5, 5), np.int64)
+        for i in range(p64.shape[1]):
+            x = p64[:, i][:, None] ^ p64[:, i][None, :]
+            d64 += np.array([int(v).bit_count() for v in x.ravel()]).reshape(5, 5)
+        assert np.array_equal(o.matmul_pm1(a, a).astype(np.int64), K - 2 * d64)
+
+
+def check_ld_words(o):
+    """ceil(K/32) words rounded up to a multiple of 4 (16-byte rows)."""
+    table = {1: 4, 31: 4, 32: 4, 33: 4, 128: 4, 129: 8, 576: 20, 1000: 32, 4096: 128, 8192: 256}
+    for K, want in table.items():
+        assert o.ld_words(K) == want, (K, o.ld_words(K), want)
+
+
+def check_memory_ratio(o):
+    """32x memory ('Binary Neural Network (BNN)' glossary; 'First Principles ...',
+    section 2 table: 0.125 bytes per binary weight vs 4 for FP32)."""
+    for K in (128, 1024, 4096, 8192):
+        packed_bytes = o.pack_pm1(np.ones((1, K), np.int8)).nbytes
+        assert packed_bytes * 8 == K          # 0.125 B per weight
+        assert (4 * K) // packed_bytes == 32
+
+
+def check_alpha(o, seed=0):
+    """alpha = (1/n) sum |w_i| (eq. (1) of 'Extreme Quantization ...'):
+    closed form for constant magnitude, a hand value, and numpy's mean."""
+    rng = np.random.default_rng(seed)
+    for K in (1, 7, 1000):
+        for c in (0.25, 3.0):
+            w = (c * rng.choice([-1.0, 1.0], size=(3, K))).astype(np.float32)
+            assert np.allclose(o.alpha(w), c, rtol=0, atol=0), (K, c)
+    w = np.array([[1.0, -2.0, 3.0, -4.0]], np.float32)
+    assert o.alpha(w)[0] == 2.5
+    w = rng.standard_normal((17, 333)).astype(np.float32)
+    ref = np.abs(w.astype(np.float64)).mean(axis=1)
+    assert np.allclose(o.alpha(w), ref, rtol=1e-14, atol=0)
+
+
+def check_matmul_library(o, seed=0):
+    """Special case that reduces to a library routine: torch float64 matmul on
+    the +1/-1 tensors is exact (|s| <= K < 2^53)."""
+    rng = np.random.default_rng(seed)
+    for (M, N, K) in [(1, 1, 1), (3, 5, 7), (64, 256, 1000), (33, 17, 65), (8, 9, 4096)]:
+        a = rng.choice(np.array([-1, 1], np.int8), size=(M, K))
+        w = rng.choice(np.array([-1, 1], np.int8), size=(N, K))
+        ref = torch.from_numpy(a.astype(np.float64)) @ torch.from_numpy(w.astype(np.float64)).T
+        assert np.array_equal(o.matmul_pm1(a, w), ref.numpy().astype(np.int32)), (M, N, K)
+    # asymmetric operands so a transposed operand cannot pass
+    a = rng.choice(np.array([-1, 1], np.int8), size=(4, 9))
+    w = rng.choice(np.array([-1, 1], np.int8), size=(6, 9))
+    s = o.matmul_pm1(a, w)
+    for m in range(4):
+        for n in range(6):
+            assert s[m, n] == int(np.dot(a[m].astype(np.int64), w[n].astype(np.int64)))
+
+
+def check_closed_forms(o, seed=0):
+    """W = X gives K on the diagonal; W = -X gives -K; all +1 gives K;
+    Sylvester-Hadamard rows are orthogonal (0 off the diagonal)."""
+    rng = np.random.default_rng(seed)
+    K = 77
+    x = rng.choice(np.array([-1, 1], np.int8), size=(6, K))
+    s = o.matmul_pm1(x, x)
+    assert np.all(np.diag(s) == K)
+    assert np.all(np.diag(o.matmul_pm1(x, (-x).astype(np.int8))) == -K)
+    assert np.all(o.matmul_pm1(np.ones((2, K), np.int8), np.ones((3, K), np.int8)) == K)
+    H = np.array([[1]], np.int64)
+    for _ in range(6):                                   # 64 x 64
+        H = np.block([[H, H], [H, -H]])
+    s = o.matmul_pm1(H.astype(np.int8), H.astype(np.int8))
+    assert np.array_equal(s, 64 * np.eye(64, dtype=np.int32))
+
+
+def check_conv_library(o, seed=0):
+    """Binary convolution against torch float64 conv2d on +1/-1 tensors, the
+    input padded with +1 (zero-padded real input, then sign)."""
+    rng = np.random.default_rng(seed)
+    for (n, c, h, w, co, stride, pad) in [(2, 3, 5, 6, 4, 1, 1), (1, 64, 9, 7, 5, 1, 1),
+                                          (2, 33, 8, 8, 3, 2, 1), (1, 2, 4, 4, 2, 1, 0)]:
+        x = rng.choice(np.array([-1, 1], np.int8), size=(n, c, h, w))
+        f = rng.choice(np.array([-1, 1], np.int8), size=(co, c, 3, 3))
+        xt = F.pad(torch.from_numpy(x.astype(np.float64)), (pad, pad, pad, pad), value=1.0)
+        ref = F.conv2d(xt, torch.from_numpy(f.astype(np.float64)), stride=stride)
+        got = o.conv2d_pm1(x, f, stride, pad)
+        assert np.array_equal(got, ref.numpy().astype(np.int32)), (n, c, h, w, co, stride, pad)
+    # closed form: all +1 input and filters give 9*c everywhere, padding included
+    x = np.ones((1, 5, 4, 4), np.int8)
+    f = np.ones((2, 5, 3, 3), np.int8)
+    assert np.all(o.conv2d_pm1(x, f, 1, 1) == 45)
+
+
+def check_bn(o, seed=0):
+    """BatchNorm before re-binarisation ('Binary Neural Network (BNN)' glossary,
+    BatchNorm paragraph): identity parameters reduce to sign(alpha*s); a
+    negative gamma flips the decision; values agree with torch's inference
+    batch_norm in float64."""
+    rng = np.random.default_rng(seed)
+    N, K = 64, 99
+    s = (K - 2 * rng.integers(0, K + 1, size=(10, N))).astype(np.int32)
+    a = rng.uniform(0.5, 1.5, N).astype(np.float32)
+    one, zero = np.ones(N, np.float32), np.zeros(N, np.float32)
+    # gamma=1, beta=0, mean=0, var+eps=1 -> alpha*s; s is odd so never 0
+    got = o.bn_sign(s, a, one, zero, zero, one - np.float32(0.0), 0.0)
+    assert np.array_equal(got, np.where(s >= 0, 1, -1).astype(np.int8))
+    g = rng.uniform(0.5, 1.5, N).astype(np.float32)
+    b = (0.1 * rng.standard_normal(N)).astype(np.float32)
+    mu = rng.standard_normal(N).astype(np.float32)
+    var = rng.uniform(0.5, 2.0, N).astype(np.float32)
+    eps = 1e-5
+    v = o.bn_value(s, a, g, b, mu, var, eps)
+    x = torch.from_numpy(a.astype(np.float64) * s.astype(np.float64))
+    ref = F.batch_norm(x, torch.from_numpy(mu.astype(np.float64)),
+                       torch.from_numpy(var.astype(np.float64)),
+                       torch.from_numpy(g.astype(np.float64)),
+                       torch.from_numpy(b.astype(np.float64)), training=False, eps=eps)
+    assert np.allclose(v, ref.numpy(), rtol=1e-12, atol=1e-12)
+    flip = o.bn_sign(s, a, -g, -b, mu, var, eps)
+    base = o.bn_sign(s, a, g, b, mu, var, eps)
+    vv = o.bn_value(s, a, g, b, mu, var, eps)
+    nz = vv != 0
+    assert np.array_equal(flip[nz], -base[nz])
+
+
+def check_mlp_library(o, seed=0):
+    """A small fully binary MLP against a torch float64 composition of sign,
+    matmul, inference batch_norm and the alpha scale."""
+    rng = np.random.default_rng(seed)
+    B, D = 16, 96
+    x0 = rng.standard_normal((B, D)).astype(np.float32)
+    ws = [rng.standard_normal((D, D)).astype(np.float32) for _ in range(3)]
+    bns = []
+    for _ in range(2):
+        bns.append((rng.uniform(0.5, 1.5, D).astype(np.float32),
+                    (0.1 * rng.standard_normal(D)).astype(np.float32),
+                    rng.standard_normal(D).astype(np.float32),
+                    rng.uniform(0.5, 2.0, D).astype(np.float32), 1e-5))
+    acts, logits = o.mlp_forward(x0, ws, bns)
+
+    def tsign(t):
+        return torch.where(t >= 0, 1.0, -1.0).to(torch.float64)
+
+    h = tsign(torch.from_numpy(x0))
+    for l, w in enumerate(ws):
+        wt = torch.from_numpy(w)
+        al = wt.double().abs().mean(dim=1)
+        s = h @ tsign(wt).T
+        if l < len(ws) - 1:
+            g, b, mu, var, eps = bns[l]
+            y = F.batch_norm(al.float().double() * s, torch.from_numpy(mu).double(),
+                             torch.from_numpy(var).double(), torch.from_numpy(g).double(),
+                             torch.from_numpy(b).double(), training=False, eps=eps)
+            h = tsign(y)
+            assert np.array_equal(acts[l + 1], h.numpy().astype(np.int8)), l
+        else:
+            assert np.allclose(logits, (al * s).numpy(), rtol=1e-13, atol=0)
+
+
+ALL_CHECKS = [
+    ("identity_bruteforce", lambda o, g: check_identity_bruteforce(o)),
+    ("elementwise_xnor_form", lambda o, g: check_elementwise_xnor_form(o)),
+    ("exercise1", check_exercise1),
+    ("pack_examples", check_pack_examples),
+    ("sign_rule", check_sign_rule),
+    ("pad_rule", lambda o, g: check_pad_rule(o)),
+    ("ld_words", lambda o, g: check_ld_words(o)),
+    ("memory_ratio", lambda o, g: check_memory_ratio(o)),
+    ("alpha", lambda o, g: check_alpha(o)),
+    ("matmul_library", lambda o, g: check_matmul_library(o)),
+    ("closed_forms", lambda o, g: check_closed_forms(o)),
+    ("conv_library", lambda o, g: check_conv_library(o)),
+    ("bn", lambda o, g: check_bn(o)),
+    ("mlp_library", lambda o, g: check_mlp_library(o)),
+]
+
+
+@pytest.mark.parametrize("name,check", ALL_CHECKS, ids=[c[0] for c in ALL_CHECKS])
+def test_oracle_pin(name, check, golden_dir):
+    check(oracle, golden_dir)
+
+
+def test_oracle_on_workload_shapes():
+    """The tiny workload end to end through the oracle: shapes, ranges, parity of s."""
+    t = workloads.tiny()
+    s, al = oracle.binary_linear(t.X, t.W)
+    assert s.shape == (64, 256) and al.shape == (256,)
+    assert np.all(np.abs(s) <= t.K) and np.all((s - t.K) % 2 == 0)
+    y = oracle.scaled(s, al)
+    assert np.all(np.sign(y) == np.sign(s))

@@ -1,0 +1,187 @@
+"""Seeded synthetic inputs for the binary (±1) matrix-product workloads.
+
+This module only draws random numbers and builds tensors of the right shape,
+dtype and distribution.  It holds none of the method's arithmetic (no sign,
+no packing, no popcount, no scaling), so both the CUDA path and the CPU oracle
+can take their inputs from here without sharing any of the computation.
+
+All draws use a CPU ``torch.Generator`` with a fixed seed, so the oracle and
+the GPU see identical bytes: tensors are generated on the host and copied to
+the device by the caller.  ``N(0, s)`` means mean 0, standard deviation ``s``.
+bf16 tensors are the fp32 draws cast to bf16 (round to nearest even).
+
+Workloads (shapes from the binary-network pages: an XNOR-Net style layer, a
+batch-1 LLM decode projection, a ResNet-18-class hidden 3x3 convolution and a
+fully binary MLP):
+
+* ``tiny``   X fp32 [64, 1000], W fp32 [256, 1000], both N(0, 1), seed 1.
+* ``gemv``   W fp32 [11008, 4096] N(0, 0.02) seed 2; x bf16 [4096] N(0, 1) seed 3.
+* ``square`` A, W fp32 [8192, 8192] N(0, 1), seeds 4 and 5.
+* ``conv``   X bf16 [64, 64, 56, 56] N(0, 1) seed 6; W fp32 [64, 64, 3, 3]
+             N(0, 0.1) seed 7; gamma U(0.5, 1.5), beta N(0, 0.1) [64] seed 8.
+* ``mlp``    X0 fp32 [4096, 4096] N(0, 1) seed 9; W_l fp32 [4096, 4096] N(0, 1)
+             seeds 10..13; BatchNorm after layers 1..3 with gamma U(0.5, 1.5),
+             beta N(0, 0.1), running mean N(0, 1), running var U(0.5, 2),
+             seeds 14..16; eps 1e-5.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import torch
+
+BN_EPS = 1e-5
+
+
+def _gen(seed: int) -> torch.Generator:
+    return torch.Generator().manual_seed(int(seed))
+
+
+def normal(shape, std: float, seed: int, dtype=torch.float32) -> torch.Tensor:
+    """N(0, std) draws in fp32 from ``seed``, optionally cast to ``dtype``."""
+    t = torch.randn(*shape, generator=_gen(seed), dtype=torch.float32)
+    if std != 1.0:
+        t.mul_(std)
+    return t.to(dtype) if dtype != torch.float32 else t
+
+
+def uniform(shape, lo: float, hi: float, seed: int) -> torch.Tensor:
+    t = torch.rand(*shape, generator=_gen(seed), dtype=torch.float32)
+    return t.mul_(hi - lo).add_(lo)
+
+
+@dataclass
+class BatchNormParams:
+    gamma: torch.Tensor
+    beta: torch.Tensor
+    mean: torch.Tensor
+    var: torch.Tensor
+    eps: float = BN_EPS
+
+
+def batchnorm_params(n: int, seed: int) -> BatchNormParams:
+    g = _gen(seed)
+    gamma = torch.rand(n, generator=g).mul_(1.0).add_(0.5)           # U(0.5, 1.5)
+    beta = torch.randn(n, generator=g).mul_(0.1)                       # N(0, 0.1)
+    mean = torch.randn(n, generator=g)                                 # N(0, 1)
+    var = torch.rand(n, generator=g).mul_(1.5).add_(0.5)               # U(0.5, 2)
+    return BatchNormParams(gamma, beta, mean, var, BN_EPS)
+
+
+# --------------------------------------------------------------------------
+# the five workloads
+# --------------------------------------------------------------------------
+
+@dataclass
+class Tiny:
+    M: int = 64
+    N: int = 256
+    K: int = 1000
+    X: torch.Tensor = None
+    W: torch.Tensor = None
+
+
+def tiny(M=64, N=256, K=1000, seed=1) -> Tiny:
+    g = _gen(seed)
+    X = torch.randn(M, K, generator=g)
+    W = torch.randn(N, K, generator=g)
+    return Tiny(M, N, K, X, W)
+
+
+@dataclass
+class Gemv:
+    N: int
+    K: int
+    W: torch.Tensor      # fp32 [N, K]
+    x: torch.Tensor      # bf16 [K]
+
+
+def gemv(N=11008, K=4096, w_seed=2, x_seed=3, x_dtype=torch.bfloat16) -> Gemv:
+    W = normal((N, K), 0.02, w_seed)
+    x = normal((K,), 1.0, x_seed, dtype=x_dtype)
+    return Gemv(N, K, W, x)
+
+
+@dataclass
+class Square:
+    M: int
+    N: int
+    K: int
+    A: torch.Tensor
+    W: torch.Tensor
+
+
+def square(M=8192, N=8192, K=8192, a_seed=4, w_seed=5) -> Square:
+    A = normal((M, K), 1.0, a_seed)
+    W = normal((N, K), 1.0, w_seed)
+    return Square(M, N, K, A, W)
+
+
+@dataclass
+class Conv:
+    X: torch.Tensor      # bf16 [n, c, h, w]
+    W: torch.Tensor      # fp32 [cout, cin, 3, 3]
+    gamma: torch.Tensor  # fp32 [cout]
+    beta: torch.Tensor   # fp32 [cout]
+    stride: int = 1
+    pad: int = 1
+
+
+def conv(n=64, c=64, h=56, w=56, cout=64, x_seed=6, w_seed=7, bn_seed=8,
+         stride=1, pad=1, x_dtype=torch.bfloat16) -> Conv:
+    X = normal((n, c, h, w), 1.0, x_seed, dtype=x_dtype)
+    W = normal((cout, c, 3, 3), 0.1, w_seed)
+    g = _gen(bn_seed)
+    gamma = torch.rand(cout, generator=g).add_(0.5)
+    beta = torch.randn(cout, generator=g).mul_(0.1)
+    return Conv(X, W, gamma, beta, stride, pad)
+
+
+@dataclass
+class Mlp:
+    X0: torch.Tensor                    # fp32 [batch, width]
+    Ws: list = field(default_factory=list)   # 4 x fp32 [width, width]
+    bns: list = field(default_factory=list)  # 3 x BatchNormParams
+
+
+def mlp(batch=4096, width=4096, layers=4, x_seed=9, w_seed0=10, bn_seed0=14) -> Mlp:
+    X0 = normal((batch, width), 1.0, x_seed)
+    Ws = [normal((width, width), 1.0, w_seed0 + l) for l in range(layers)]
+    bns = [batchnorm_params(width, bn_seed0 + l) for l in range(layers - 1)]
+    return Mlp(X0, Ws, bns)
+
+
+# --------------------------------------------------------------------------
+# edge-case values for the sign rule
+# --------------------------------------------------------------------------
+
+def sign_edge_values(dtype=torch.float32) -> torch.Tensor:
+    """Values at which a sign rule is easy to get wrong: signed zeros,
+    denormals, infinities, NaN, and the smallest normals of both signs."""
+    vals = [0.0, -0.0, 1e-45, -1e-45, 1e-40, -1e-40, 1.17549435e-38,
+            -1.17549435e-38, float("inf"), float("-inf"), float("nan"),
+            1.0, -1.0, 3.0e38, -3.0e38]
+    t = torch.tensor(vals, dtype=torch.float32)
+    if dtype == torch.bfloat16:
+        t = t.to(torch.bfloat16)
+    return t
+
+
+def random_with_edges(rows: int, K: int, seed: int, dtype=torch.float32,
+                      edge_fraction: float = 0.05, finite: bool = True) -> torch.Tensor:
+    """N(0, 1) matrix with a seeded fraction of entries replaced by edge values.
+
+    With ``finite`` (the default) infinities and NaN are left out, so a
+    per-row mean magnitude stays finite; the non-finite values are drawn in
+    only when ``finite=False``."""
+    g = _gen(seed)
+    t = torch.randn(rows, K, generator=g)
+    edges = sign_edge_values(torch.float32)
+    if finite:
+        edges = edges[torch.isfinite(edges)]
+    mask = torch.rand(rows, K, generator=g) < edge_fraction
+    idx = torch.randint(0, edges.numel(), (rows, K), generator=g)
+    t = torch.where(mask, edges[idx], t)
+    if dtype == torch.bfloat16:
+        t = t.to(torch.bfloat16)
+    return t
