@@ -1,0 +1,624 @@
+#!/usr/bin/env python
+"""Benchmark of the packed binary (+1/-1) matrix product on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--no-rows] [--no-cpu-baseline] [--no-e2e]
+
+Headline (one JSON line on rank 0): the batch-1 LLM-decode binary GEMV,
+packed +1/-1 weights [11008, 4096] (from N(0, 0.02)), activation x bf16 [4096]
+binarised and packed inside the kernel, alpha-scaled fp32 output; metric =
+algorithmic GB/s.  One step = one GEMV (x pack + XOR/popcount + alpha
+epilogue) through the C ABI.  K steps are captured in CUDA graphs and timed
+with CUDA events on the launching stream; steps rotate over 48 copies of the
+packed weights (270 MB, more than the 126 MB L2), so every step streams its
+weights from HBM.
+
+Also on the line:
+  roofline      the GEMV kernel against the measured HBM copy bandwidth.
+  cpu_baseline  the CPU oracle on a bounded sample of the same workload.
+  e2e           the same metric through the public API with host buffers: per
+                step, pinned x -> device, GEMV, y -> pinned host.
+  rows          the other hot-path rows, each timed the same way: weight pack
+                + alpha (HBM GB/s), the square 8192^3 GEMM, the ResNet-class
+                3x3 binary convolution and the 4-layer binary MLP (binary MAC/s
+                against the integer-pipe roofline).
+Under torchrun (N > 1) every rank runs its own replica of the workload (the
+path has no data exchange), timing is the max over ranks, and value is the
+whole job's bytes / that time ("weak" scaling).
+
+--impl reference times the CPU oracle (the plain +1/-1 integer definition)
+on the host cores on the same workload and metric; rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "binary GMAC/s (TOPS) for packed XNOR-popcount GEMM; GEMV GB/s vs HBM peak"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+SM_COUNT = 148
+# 32-bit population count: 16 per clock per SM (CUDA arithmetic-instruction
+# throughput table); one POPC covers 32 binary multiply-accumulates.
+POPC_PER_CLK_PER_SM = 16
+
+
+# ---------------------------------------------------------------------------
+# process setup
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "sm_max_mhz": float(d.get("sm_max_mhz", 1965.0)),
+                "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+def alu_peak_mac_s(sm_mhz: float) -> float:
+    """Binary MAC/s when every SM retires 16 POPC per clock, 32 MACs each."""
+    return SM_COUNT * POPC_PER_CLK_PER_SM * 32 * sm_mhz * 1e6
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "xnor_popcount_gemm_bnn_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(kernel)
+    if not e or e.get("source_hash") != source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """SM clock and throttle reasons, sampled with NVML during the timed region."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nvml = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+                r = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nvml is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# device timing helpers
+# ---------------------------------------------------------------------------
+
+def _graph(torch, fn, n):
+    """Capture n calls of fn(i) into one CUDA graph (launch-bound inner loop)."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn(0)                                    # warm the stream and library once
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(n):
+            fn(i)
+    return g
+
+
+def time_steps(torch, fn, steps, warmup, period, sync):
+    """Run `warmup` untimed steps, then time exactly `steps` steps with CUDA
+    events on the current stream.  fn(i) launches step i.  Steps are replayed
+    from CUDA graphs of `period` launches (plus one graph for the remainder).
+    Returns milliseconds for the timed steps (max over ranks)."""
+    full = _graph(torch, fn, period) if steps >= period or warmup >= period else None
+    rem = steps % period
+    tail = _graph(torch, fn, rem) if rem else None
+    # warm-up: graphs of the same shapes
+    w = warmup
+    while w > 0:
+        if full is not None and w >= period:
+            full.replay(); w -= period
+        else:
+            g = _graph(torch, fn, w); g.replay(); w = 0
+    torch.cuda.synchronize()
+    sync()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps // period):
+        full.replay()
+    if tail is not None:
+        tail.replay()
+    end.record()
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end)
+    sync()
+    return ms
+
+
+# ---------------------------------------------------------------------------
+# the headline: LLM-decode binary GEMV
+# ---------------------------------------------------------------------------
+
+GEMV_N, GEMV_K = 11008, 4096
+
+
+def gemv_bytes(N=GEMV_N, K=GEMV_K) -> int:
+    kw = ((K + 31) // 32 + 3) // 4 * 4
+    return N * kw * 4 + N * 4 + K * 2 + N * 4     # packed W + alpha + bf16 x + fp32 y
+
+
+def gemv_setup(torch, bnn, workloads, dev, copies):
+    g = workloads.gemv()
+    W_p = bnn.empty_packed(g.N, g.K, dev)
+    alpha = torch.empty(g.N, dtype=torch.float32, device=dev)
+    bnn.bnn_pack_sign(g.W.to(dev), W_p, alpha)
+    Ws = [W_p] + [W_p.clone() for _ in range(copies - 1)]
+    x = g.x.to(dev)
+    y = torch.empty(g.N, dtype=torch.float32, device=dev)
+    return g, Ws, alpha, x, y
+
+
+def run_ours(args, torch, dist):
+    import workloads
+    import xnor_popcount_gemm_bnn_b200 as bnn
+
+    ws, rank, local = dist_env()
+    dev = torch.device("cuda", local)
+    pk = peaks()
+
+    def sync():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    copies = max(2, math.ceil(2 * L2_BYTES / gemv_bytes()) + 1)
+    copies = (copies + 7) // 8 * 8                       # 48
+    g, Ws, alpha, x, y = gemv_setup(torch, bnn, workloads, dev, copies)
+
+    def step(i):
+        bnn.bnn_xnor_gemv(Ws[i % copies], x, g.K, alpha, None, y)
+
+    with ClockSampler(local) as clk:
+        ms = time_steps(torch, step, args.steps, args.warmup, copies, sync)
+    ms = max_over_ranks(ms)
+    if bnn.bnn_device_error() != 0:
+        raise RuntimeError("a kernel reported a device-side timeout")
+    per_step_bytes = gemv_bytes()
+    value = ws * args.steps * per_step_bytes / (ms * 1e-3) / 1e9
+    launch_s = ms * 1e-3 / args.steps
+    achieved = per_step_bytes / launch_s / 1e9
+
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "u32",
+        "data": "synthetic",
+        "config": {
+            "workload": "LLM-decode binary GEMV: packed +1/-1 W [11008, 4096] from N(0,0.02), "
+                        "x bf16 [4096] N(0,1) sign-packed in-kernel, per-row alpha, fp32 y",
+            "N": g.N, "K": g.K,
+            "algorithmic_bytes_per_step": per_step_bytes,
+            "l2": f"inputs larger than L2: {copies} rotating packed weight copies "
+                  f"({copies * Ws[0].numel() * 4 / 1e6:.0f} MB > 126 MB L2)",
+            "timing": f"CUDA graphs of {copies} launches, CUDA events on the launching stream",
+            "parallelism": "replicas" if ws == 1 else f"replicas x{ws}",
+        },
+        "roofline": {
+            "bound": "hbm",
+            "achieved": round(achieved, 1),
+            "peak": pk["hbm_gbs"],
+            "unit": "GB/s",
+            "frac": round(achieved / pk["hbm_gbs"], 4),
+            "traffic": recorded_traffic("xnor_gemv_kernel"),
+            "peak_source": pk["source"],
+            "kernel": "xnor_gemv_kernel",
+        },
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+
+    # e2e: the public API with host buffers
+    if not args.no_e2e:
+        result["e2e"] = e2e_gemv(torch, bnn, g, Ws, alpha, dev, min(args.steps, 2000), sync, max_over_ranks, ws)
+
+    if not args.no_rows:
+        result["rows"] = bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws)
+
+    del Ws
+    torch.cuda.empty_cache()
+    if rank == 0 and not args.no_cpu_baseline and ws == 1:
+        result["cpu_baseline"] = cpu_baseline_gemv(args.cpu_seconds)
+    return result
+
+
+def e2e_gemv(torch, bnn, g, Ws, alpha, dev, steps, sync, max_over_ranks, ws):
+    x_host = g.x.clone().pin_memory()
+    y_host = torch.empty(g.N, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(g.x, device=dev)
+    y_dev = torch.empty(g.N, dtype=torch.float32, device=dev)
+    copies = len(Ws)
+
+    def one(i):
+        x_dev.copy_(x_host, non_blocking=True)
+        bnn.bnn_xnor_gemv(Ws[i % copies], x_dev, g.K, alpha, None, y_dev)
+        y_host.copy_(y_dev, non_blocking=True)
+
+    for i in range(5):
+        one(i)
+    torch.cuda.synchronize()
+    sync()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(steps):
+        one(i)
+    end.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(start.elapsed_time(end))
+    return {"value": round(ws * steps * gemv_bytes() / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+            "d2h_bytes_per_step": y_host.numel() * y_host.element_size(),
+            "steps": steps, "ms_per_step": ms / steps,
+            "path": "eager Python calls of bnn_xnor_gemv with pinned-host copies each step"}
+
+
+# ---------------------------------------------------------------------------
+# the other rows
+# ---------------------------------------------------------------------------
+
+def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws):
+    rows = {}
+    steps = max(3, args.row_steps)
+    warm = max(3, args.warmup)
+    clk_mhz = pk["sm_max_mhz"]
+    alu_peak = alu_peak_mac_s(clk_mhz)
+
+    def timed(fn, n=steps, period=None):
+        return max_over_ranks(time_steps(torch, fn, n, warm, period or n, sync))
+
+    # --- a1: weight pack + alpha, fp32 [11008, 4096] (HBM) ---
+    g = workloads.gemv()
+    Wd = g.W.to(dev)
+    W_p = bnn.empty_packed(g.N, g.K, dev)
+    alpha = torch.empty(g.N, dtype=torch.float32, device=dev)
+    ms = timed(lambda i: bnn.bnn_pack_sign(Wd, W_p, alpha))
+    b = g.N * g.K * 4 + W_p.numel() * 4 + g.N * 4
+    ach = b * steps / (ms * 1e-3) / 1e9
+    rows["pack_sign_weights"] = {"workload": "fp32 W [11008, 4096] -> packed bits + alpha",
+                                 "value": round(ws * ach, 1), "unit": "GB/s", "ms_per_step": ms / steps,
+                                 "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"],
+                                              "frac": round(ach / pk["hbm_gbs"], 4),
+                                              "traffic": recorded_traffic("pack_sign_rows_kernel")}}
+    del Wd, W_p, alpha, g
+    torch.cuda.empty_cache()
+
+    # --- a2+a3+a6: square GEMM 8192^3, int32 + alpha-scaled fp32 outputs ---
+    sq = workloads.square()
+    Ad = sq.A.to(dev)
+    A_p = bnn.empty_packed(sq.M, sq.K, dev)
+    Wsq = bnn.empty_packed(sq.N, sq.K, dev)
+    al = torch.empty(sq.N, dtype=torch.float32, device=dev)
+    bnn.bnn_pack_sign(sq.W.to(dev), Wsq, al)
+    Ci = torch.empty(sq.M, sq.N, dtype=torch.int32, device=dev)
+    Cf = torch.empty(sq.M, sq.N, dtype=torch.float32, device=dev)
+    macs = sq.M * sq.N * sq.K
+    ms_g = timed(lambda i: bnn.bnn_xnor_gemm(A_p, Wsq, sq.K, al, Ci, Cf))
+    bnn.bnn_pack_sign(Ad, A_p)
+    ms_s = timed(lambda i: (bnn.bnn_pack_sign(Ad, A_p), bnn.bnn_xnor_gemm(A_p, Wsq, sq.K, al, Ci, Cf)))
+    mac_s = macs * steps / (ms_g * 1e-3)
+    rows["square_gemm"] = {
+        "workload": "M=N=K=8192 packed A x packed W^T, int32 s + alpha*s fp32 out",
+        "value": round(ws * mac_s / 1e9, 1), "unit": "binary GMAC/s", "tops": round(ws * 2 * mac_s / 1e12, 2),
+        "ms_per_step": ms_g / steps,
+        "with_activation_pack": {"value": round(ws * macs * steps / (ms_s * 1e-3) / 1e9, 1),
+                                 "unit": "binary GMAC/s", "ms_per_step": ms_s / steps},
+        "roofline": {"bound": "alu", "achieved": round(mac_s / 1e12, 2), "peak": round(alu_peak / 1e12, 2),
+                     "unit": "binary TMAC/s", "frac": round(mac_s / alu_peak, 4),
+                     "peak_derivation": f"{SM_COUNT} SMs x {POPC_PER_CLK_PER_SM} POPC/clk x 32 MAC x {clk_mhz:.0f} MHz",
+                     "traffic": recorded_traffic("xnor_gemm_popc_kernel")}}
+    del sq, Ad, A_p, Wsq, al, Ci, Cf
+    torch.cuda.empty_cache()
+
+    # --- a2 (NCHW) + a5 + a6: ResNet-class binary 3x3 conv with affine epilogue ---
+    cv = workloads.conv()
+    n, c, h, w = cv.X.shape
+    Xd = cv.X.to(dev)
+    Xb = bnn.empty_packed_nhwc(n, c, h, w, dev)
+    Wc = bnn.empty_conv3x3_weights(64, c, dev)
+    alc = torch.empty(64, dtype=torch.float32, device=dev)
+    bnn.bnn_pack_conv3x3_weights(cv.W.to(dev), Wc, alc)
+    gam, bet = cv.gamma.to(dev), cv.beta.to(dev)
+    out = torch.empty(n, 64, h, w, dtype=torch.float32, device=dev)
+    ep = bnn.make_epilogue(bnn.BNN_OUT_AFFINE_F32, alpha=alc, gamma=gam, beta=bet)
+
+    def conv_step(i):
+        bnn.bnn_pack_sign_nchw(Xd, Xb)
+        bnn.bnn_binary_conv3x3_fused(Xb, c, Wc, ep, out, 1, 1)
+
+    ms_c = timed(conv_step)
+    bnn.bnn_pack_sign_nchw(Xd, Xb)
+    ms_ck = timed(lambda i: bnn.bnn_binary_conv3x3_fused(Xb, c, Wc, ep, out, 1, 1))
+    cmacs = n * h * w * 64 * 9 * c
+    cmac_s = cmacs * steps / (ms_ck * 1e-3)
+    rows["conv3x3"] = {
+        "workload": "bf16 [64,64,56,56] -> pack NCHW -> binary 3x3 conv (64 filters, stride 1, pad 1), "
+                    "alpha + affine epilogue, fp32 NCHW out",
+        "value": round(ws * cmacs * steps / (ms_c * 1e-3) / 1e9, 1), "unit": "binary GMAC/s",
+        "ms_per_step": ms_c / steps, "conv_kernel_ms": ms_ck / steps,
+        "roofline": {"bound": "alu", "achieved": round(cmac_s / 1e12, 2), "peak": round(alu_peak / 1e12, 2),
+                     "unit": "binary TMAC/s", "frac": round(cmac_s / alu_peak, 4),
+                     "traffic": recorded_traffic("xnor_conv3x3_kernel")}}
+    del cv, Xd, Xb, Wc, alc, gam, bet, out
+    torch.cuda.empty_cache()
+
+    # --- MLP: pack input, 3 x (GEMM + folded-BN re-pack), GEMM + alpha ---
+    m = workloads.mlp()
+    B, D = m.X0.shape
+    X0 = m.X0.to(dev)
+    A0 = bnn.empty_packed(B, D, dev)
+    acts = [bnn.empty_packed(B, D, dev) for _ in range(3)]
+    eps_ = []
+    Wps = []
+    for l, W in enumerate(m.Ws):
+        Wp = bnn.empty_packed(D, D, dev)
+        a = torch.empty(D, dtype=torch.float32, device=dev)
+        bnn.bnn_pack_sign(W.to(dev), Wp, a)
+        Wps.append(Wp)
+        if l < 3:
+            bn = m.bns[l]
+            thr, mode = bnn.bnn_fold_bn_threshold(a.cpu(), bn.gamma, bn.beta, bn.mean, bn.var, bn.eps, D)
+            thr, mode = thr.to(dev), mode.to(dev)
+            eps_.append((bnn.make_epilogue(bnn.BNN_OUT_THRESHOLD_PACK, popc_thresh=thr, thresh_mode=mode), thr, mode))
+        else:
+            eps_.append((bnn.make_epilogue(bnn.BNN_OUT_SCALED_F32, alpha=a), a))
+    logits = torch.empty(B, D, dtype=torch.float32, device=dev)
+
+    def mlp_step(i):
+        bnn.bnn_pack_sign(X0, A0)
+        A = A0
+        for l in range(4):
+            o = acts[l] if l < 3 else logits
+            bnn.bnn_binary_linear_fused(A, Wps[l], D, eps_[l][0], o)
+            A = o
+
+    ms_m = timed(mlp_step)
+    mmacs = 4 * B * D * D
+    rows["mlp4"] = {
+        "workload": "fully binary MLP, batch 4096, width 4096, 4 layers: pack fp32 input, "
+                    "3 x (GEMM + folded BatchNorm sign re-pack), GEMM + alpha fp32 logits",
+        "value": round(ws * mmacs * steps / (ms_m * 1e-3) / 1e9, 1), "unit": "binary GMAC/s",
+        "ms_per_step": ms_m / steps,
+        "roofline": {"bound": "alu", "achieved": round(mmacs * steps / (ms_m * 1e-3) / 1e12, 2),
+                     "peak": round(alu_peak / 1e12, 2), "unit": "binary TMAC/s",
+                     "frac": round(mmacs * steps / (ms_m * 1e-3) / alu_peak, 4)}}
+    del m, X0, A0, acts, eps_, Wps, logits
+    torch.cuda.empty_cache()
+    if bnn.bnn_device_error() != 0:
+        raise RuntimeError("a kernel reported a device-side timeout")
+    return rows
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (the baseline, never the product path)
+# ---------------------------------------------------------------------------
+
+def cpu_oracle_gemv_steps(seconds: float, max_steps: int | None = None):
+    """Time the oracle on the decode GEMV: sign(x), the int8 +1/-1 product
+    with the pre-binarised W (the oracle's analogue of pre-packed weights),
+    and alpha*s in float64.  Runs whole steps until `seconds` have passed (or
+    max_steps).  Returns (steps, elapsed_s, threads)."""
+    import oracle
+    import workloads
+
+    g = workloads.gemv()
+    wb = oracle.sign_pm1(g.W)
+    al = oracle.alpha(g.W)
+    x = g.x
+    done = 0
+    t0 = time.perf_counter()
+    while True:
+        xb = oracle.sign_pm1(x)
+        s = oracle.gemv_pm1(wb, xb)
+        oracle.scaled(s, al)
+        done += 1
+        el = time.perf_counter() - t0
+        if (max_steps is not None and done >= max_steps) or (max_steps is None and el >= seconds):
+            break
+    return done, el, 1          # one output row: the oracle's outer loop runs on one thread
+
+
+def cpu_baseline_gemv(seconds: float):
+    n, el, threads = cpu_oracle_gemv_steps(seconds)
+    return {"value": round(n * gemv_bytes() / el / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{n} whole GEMV steps of the same workload ({el:.1f} s): sign(x), int8 +1/-1 "
+                      f"product with the pre-binarised W, alpha*s in float64",
+            "host_cpus": os.cpu_count()}
+
+
+def run_reference(args):
+    """The CPU oracle on the headline workload.  Each step is a bounded sample:
+    the GEMV over the first `rows` output rows, with `rows` chosen so that the
+    whole --warmup + --steps run takes about two minutes of host time."""
+    import oracle
+    import workloads
+
+    g = workloads.gemv()
+    wb = oracle.sign_pm1(g.W)
+    al = oracle.alpha(g.W)
+    t0 = time.perf_counter()
+    oracle.scaled(oracle.gemv_pm1(wb, oracle.sign_pm1(g.x)), al)
+    t_full = time.perf_counter() - t0
+    total = max(1, args.steps + args.warmup)
+    rows = int(max(1, min(GEMV_N, GEMV_N * 120.0 / (total * t_full))))
+    wbs, als = wb[:rows], al[:rows]
+
+    def step():
+        oracle.scaled(oracle.gemv_pm1(wbs, oracle.sign_pm1(g.x)), als)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    kw = ((GEMV_K + 31) // 32 + 3) // 4 * 4
+    step_bytes = rows * kw * 4 + rows * 4 + GEMV_K * 2 + rows * 4
+    value = args.steps * step_bytes / el / 1e9
+    sample = (f"each step the GEMV over the first {rows} of {GEMV_N} output rows "
+              f"(sign(x), int8 +1/-1 product with the pre-binarised W, alpha*s in float64); "
+              f"{args.steps} timed steps, {el:.1f} s")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": "GB/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": el * 1e3 / max(1, args.steps),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int32",
+        "data": "synthetic",
+        "config": {"workload": "LLM-decode binary GEMV: packed +1/-1 W [11008, 4096] from N(0,0.02), "
+                               "x bf16 [4096] N(0,1), per-row alpha, fp32 y",
+                   "N": GEMV_N, "K": GEMV_K, "algorithmic_bytes_per_step": gemv_bytes()},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample, "host_cpus": os.cpu_count()},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=192000)
+    ap.add_argument("--warmup", type=int, default=480)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--row-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-rows", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    ws, rank, local = dist_env()
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    import torch
+    dist = None
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist_mod
+        torch.cuda.set_device(local)
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        dist = dist_mod
+    else:
+        torch.cuda.set_device(local)
+    try:
+        result = run_ours(args, torch, dist)
+        if rank == 0:
+            print(json.dumps(result), flush=True)
+    finally:
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

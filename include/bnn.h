@@ -1,0 +1,252 @@
+/*
+ * bnn.h -- C ABI of libbnn.so: the binary (+1/-1 weights, +1/-1 activations)
+ * matrix product on bit-packed operands, on NVIDIA B200 (sm_100a).
+ *
+ * What is computed (page title, section / equation):
+ *  - "Extreme Quantization: Binary, Ternary & 1-bit LLMs", XNOR-Net section,
+ *    eq. (4) and eq. (6): w_b = sign(w), x_b = sign(x),
+ *    w_b^T x_b = K - 2 * popcount(w~ XOR x~).
+ *  - same page, Notation: sign(x) = +1 for x >= 0, -1 for x < 0.
+ *  - same page, Binary Neural Networks section, eq. (1):
+ *    y = alpha * (w_b^T x), alpha = (1/n) * sum_i |w_i| (one alpha per filter,
+ *    i.e. per output channel, as in the "Binary Neural Network (BNN)" glossary
+ *    paragraph on BatchNorm and scaling factors).
+ *  - "First Principles: Why Binary Ops Can Be Exponentially Faster",
+ *    section "1. Arithmetic: MAC -> XNOR + popcount": encoding bit 0 -> +1,
+ *    bit 1 -> -1; bits packed into machine words; pad bits encode +1.
+ *
+ * PACKED LAYOUT (used by every call).  A packed row of K elements is an array
+ * of uint32 words; bit j of word w is element 32*w + j (least significant bit
+ * first), 1 meaning -1 and 0 meaning +1.  The row holds
+ * bnn_packed_ld_words(K) = ceil(K/32) rounded up to a multiple of 4 words, so
+ * each row is a whole number of 16-byte units; the bits past element K-1 and
+ * the words past ceil(K/32) are 0 (they encode +1 in both operands, so they
+ * never add to the popcount).  The uint64 view of the same bytes (little
+ * endian) is the 64-bit packing.  Row r of a packed matrix starts at word
+ * r * ld, where ld (the row stride, in words) is >= bnn_packed_ld_words(K)
+ * and a multiple of 4.  Words between bnn_packed_ld_words(K) and ld are never
+ * read or written.
+ *
+ * CONVENTIONS.
+ *  - Device pointers are CUDA device (or managed) memory on the current
+ *    device, owned by the caller; the library keeps no pointer after a call
+ *    returns and allocates no device memory.  Host pointers are named so.
+ *  - Every device call is asynchronous on `stream` (NULL = legacy default
+ *    stream).  It returns after the launch; results are visible to later
+ *    work on the same stream.
+ *  - Arguments are checked on the host before anything is launched; a failed
+ *    check returns an error status and writes nothing.  Launch failures
+ *    return BNN_ERR_CUDA.  No exception crosses the ABI, nothing traps on the
+ *    device, and there is no CPU fallback.
+ *  - Packed operands and all vector loads need 16-byte aligned pointers.
+ *  - A kernel that waits on an asynchronous copy gives up after about one
+ *    second, records BNN_ERR_DEVICE_TIMEOUT in a device-side flag and returns;
+ *    bnn_device_error() reads and clears that flag.
+ */
+#ifndef BNN_H_
+#define BNN_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+struct CUstream_st;
+typedef struct CUstream_st* bnn_stream_t;
+
+typedef enum bnn_status {
+    BNN_OK = 0,
+    BNN_ERR_INVALID_ARG = 1,     /* null pointer, negative or too-large size, bad mode */
+    BNN_ERR_ALIGNMENT = 2,       /* pointer or leading dimension not 16-byte aligned */
+    BNN_ERR_UNSUPPORTED = 3,     /* valid but not implemented (e.g. dtype/mode combination) */
+    BNN_ERR_CUDA = 4,            /* a CUDA runtime call or kernel launch failed */
+    BNN_ERR_DEVICE_TIMEOUT = 5   /* a kernel gave up waiting (reported by bnn_device_error) */
+} bnn_status;
+
+typedef enum bnn_dtype {
+    BNN_F32 = 0,                 /* IEEE binary32 */
+    BNN_BF16 = 1                 /* bfloat16, taken as stored */
+} bnn_dtype;
+
+/* Output of a binary product (the epilogue).  s = K - 2 d is the +1/-1 dot
+ * product, d the popcount of the XOR (eq. (6)). */
+typedef enum bnn_out_mode {
+    BNN_OUT_INT32 = 1,           /* int32 s */
+    BNN_OUT_SCALED_F32 = 2,      /* fp32 alpha_n * s                    (eq. (1)) */
+    BNN_OUT_AFFINE_F32 = 4,      /* fp32 gamma_n * (alpha_n * s) + beta_n */
+    BNN_OUT_THRESHOLD_PACK = 8   /* packed sign of a folded BatchNorm, see bnn_fold_bn_threshold */
+} bnn_out_mode;
+
+/* Per-output-channel epilogue parameters (device pointers, length = number of
+ * output channels).  Unused fields may be NULL.
+ *   INT32:           none.
+ *   SCALED_F32:      alpha.
+ *   AFFINE_F32:      alpha, gamma, beta.
+ *   THRESHOLD_PACK:  popc_thresh, thresh_mode (from bnn_fold_bn_threshold):
+ *                    thresh_mode 0 -> output bit = (d > popc_thresh),
+ *                    thresh_mode 1 -> output bit = (d < popc_thresh);
+ *                    bit 1 means -1. */
+typedef struct bnn_epilogue {
+    int32_t mode;                /* one bnn_out_mode value */
+    const float* alpha;
+    const float* gamma;
+    const float* beta;
+    const int32_t* popc_thresh;
+    const int8_t* thresh_mode;
+} bnn_epilogue;
+
+/* Words in one packed row of K elements: ceil(K/32) rounded up to a multiple
+ * of 4 ("First Principles ...", section 1: pack bits into words).  Returns -1
+ * for K < 1. */
+int64_t bnn_packed_ld_words(int64_t K);
+
+/* Words in one packed 3x3 filter row for `cin` input channels: the 9 taps in
+ * (kh, kw) order, each ceil(cin/32) words, rounded up to a multiple of 4.
+ * Returns -1 for cin < 1. */
+int64_t bnn_conv3x3_ld_words(int64_t cin);
+
+/* Static text for a status code. */
+const char* bnn_status_string(int status);
+
+/* Reads and clears the device-side error flag set by a kernel that gave up
+ * waiting (BNN_OK if none).  Synchronises the current device first.  Writes
+ * the flag value to *code_out (host pointer). */
+bnn_status bnn_device_error(int32_t* code_out);
+
+/* bnn_pack_sign -- sign-binarise and bit-pack a real matrix along K, and
+ * optionally compute alpha per row.
+ *   Passage: "Extreme Quantization ...", Notation (sign) and eq. (4);
+ *   "First Principles ...", section 1 (encoding, packing, pad = +1);
+ *   eq. (1) (alpha = mean |w| over the row).
+ *   x        device, [rows, K] row-major, dtype `dt`, row stride ld_x elements
+ *            (ld_x >= K).
+ *   packed   device, uint32 [rows, ld_words]; ld_words >= bnn_packed_ld_words(K),
+ *            a multiple of 4.  Words [0, bnn_packed_ld_words(K)) of every row
+ *            are written, pad bits and pad words as 0.
+ *   alpha_out device fp32 [rows] or NULL: (sum_k |x_rk|) / K accumulated in
+ *            fp64 over the true K, rounded once to fp32.
+ *   Bit k of a row is 1 exactly when x_rk < 0 (so -0.0 and NaN give +1).
+ *   rows may be 0 (nothing launched).  K >= 1.
+ *   Errors: INVALID_ARG (null, K < 1, ld_x < K, ld_words too small or not a
+ *   multiple of 4), ALIGNMENT (packed not 16-byte aligned). */
+bnn_status bnn_pack_sign(const void* x, bnn_dtype dt, int64_t rows, int64_t K, int64_t ld_x,
+                         uint32_t* packed, int64_t ld_words, float* alpha_out,
+                         bnn_stream_t stream);
+
+/* bnn_pack_sign_nchw -- sign-binarise and pack an NCHW activation tensor into
+ * per-pixel channel words, the operand layout of bnn_binary_conv3x3_fused.
+ *   Passage: as bnn_pack_sign (eq. (4): activations are binarised too).
+ *   x          device, [n, c, h, w] contiguous, dtype `dt`.
+ *   packed_nhwc device, uint32 [n, h, w, cw] contiguous with cw = ceil(c/32):
+ *              bit q of word j of pixel (n, y, x) is channel 32*j + q; bits for
+ *              channels >= c are 0.
+ *   Errors: INVALID_ARG, ALIGNMENT (packed_nhwc not 4-byte aligned). */
+bnn_status bnn_pack_sign_nchw(const void* x, bnn_dtype dt, int64_t n, int64_t c, int64_t h,
+                              int64_t w, uint32_t* packed_nhwc, bnn_stream_t stream);
+
+/* bnn_pack_conv3x3_weights -- pack OIHW 3x3 filters into rows of K = 9 * cin
+ * elements in (kh, kw, c) order, and compute alpha per output channel.
+ *   Passage: eq. (1) and the glossary's "scaling factors for each weight
+ *   filter"; encoding and padding as bnn_pack_sign.
+ *   w_oihw   device, [cout, cin, 3, 3] contiguous, dtype `dt`.
+ *   packed   device, uint32 [cout, ld_words], ld_words >= bnn_conv3x3_ld_words(cin),
+ *            multiple of 4.  Word t*cw + j (t = kh*3 + kw, cw = ceil(cin/32))
+ *            holds channels 32*j .. 32*j+31 of tap t; unused channel bits and
+ *            words [9*cw, bnn_conv3x3_ld_words(cin)) are 0.
+ *   alpha_out device fp32 [cout] or NULL: mean |w| over the 9*cin true weights.
+ *   Errors: INVALID_ARG, ALIGNMENT. */
+bnn_status bnn_pack_conv3x3_weights(const void* w_oihw, bnn_dtype dt, int64_t cout, int64_t cin,
+                                    uint32_t* packed, int64_t ld_words, float* alpha_out,
+                                    bnn_stream_t stream);
+
+/* bnn_xnor_gemm -- C[m, n] = K - 2 * popcount(A[m, :] XOR W[n, :]) for packed
+ * A [M, K] and W [N, K]; optionally also the alpha-scaled fp32 product.
+ *   Passage: eq. (6) of "Extreme Quantization ..." (XNOR-Net), eq. (1) for
+ *   the scale; "First Principles ...", section 1.
+ *   A, W     device, packed rows (layout above), strides lda, ldw words.
+ *   alpha    device fp32 [N]; required when C_f32 is given.
+ *   C_i32    device int32 [M, ldc] or NULL: s.
+ *   C_f32    device fp32 [M, ldf] or NULL: alpha[n] * s in fp32.
+ *   At least one of C_i32, C_f32.  M, N >= 0, K >= 1.
+ *   Errors: INVALID_ARG, ALIGNMENT (A, W not 16-byte aligned, lda/ldw not a
+ *   multiple of 4). */
+bnn_status bnn_xnor_gemm(const uint32_t* A, int64_t lda, const uint32_t* W, int64_t ldw,
+                         int64_t M, int64_t N, int64_t K, const float* alpha,
+                         int32_t* C_i32, int64_t ldc, float* C_f32, int64_t ldf,
+                         bnn_stream_t stream);
+
+/* bnn_xnor_gemv -- batch-1 product y[n] = K - 2 * popcount(W[n, :] XOR
+ * pack(sign(x))), the real activation vector binarised and packed inside the
+ * kernel.  Memory-bound: the packed W is streamed once.
+ *   Passage: eq. (4) and eq. (6); "First Principles ...", "Bandwidth math"
+ *   (batch-1 y = Wx moves MN/8 bytes when packed).
+ *   W        device, packed [N, ldw] (layout above).
+ *   x        device, [K] of dtype x_dt.
+ *   alpha    device fp32 [N]; required when y_f32 is given.
+ *   y_i32    device int32 [N] or NULL; y_f32 device fp32 [N] or NULL (alpha * s);
+ *            at least one.
+ *   Errors: INVALID_ARG, ALIGNMENT. */
+bnn_status bnn_xnor_gemv(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt,
+                         int64_t N, int64_t K, const float* alpha,
+                         int32_t* y_i32, float* y_f32, bnn_stream_t stream);
+
+/* bnn_binary_linear_fused -- packed binary GEMM with one fused epilogue.
+ *   Passage: eq. (6) (product), eq. (1) (alpha), the glossary's BatchNorm
+ *   paragraph (normalise, then binarise for the next layer).
+ *   A, W, lda, ldw, M, N, K as bnn_xnor_gemm.
+ *   ep       host pointer to the epilogue (mode + device parameter arrays of
+ *            length N).
+ *   out      device: int32 or fp32 [M, ld_out] (ld_out in elements) for the
+ *            INT32 / SCALED_F32 / AFFINE_F32 modes; for THRESHOLD_PACK a
+ *            packed uint32 [M, ld_out] matrix of N elements per row (ld_out in
+ *            words, >= bnn_packed_ld_words(N), multiple of 4; pad bits and
+ *            pad words written as 0), i.e. directly the A operand of the next
+ *            layer with K_next = N.
+ *   Errors: INVALID_ARG (incl. missing parameter for the mode), ALIGNMENT. */
+bnn_status bnn_binary_linear_fused(const uint32_t* A, int64_t lda, const uint32_t* W, int64_t ldw,
+                                   int64_t M, int64_t N, int64_t K, const bnn_epilogue* ep,
+                                   void* out, int64_t ld_out, bnn_stream_t stream);
+
+/* bnn_binary_conv3x3_fused -- binary 3x3 convolution as an implicit GEMM over
+ * packed per-pixel channel words, with a fused epilogue.  Output pixel
+ * (n, y, x) gathers the 9 taps (kh, kw); a tap outside the image reads all-0
+ * words (+1: zero-padded real input, then sign).  K = 9 * c.
+ *   Passage: eq. (4), eq. (6), eq. (1) per filter; glossary BatchNorm paragraph.
+ *   X_nhwc_bits device, from bnn_pack_sign_nchw: [n, h, w, ceil(c/32)] words.
+ *   W_packed device, from bnn_pack_conv3x3_weights: [cout, ldw] words.
+ *   stride >= 1, pad >= 0; output spatial size (h + 2 pad - 3)/stride + 1 by
+ *   (w + 2 pad - 3)/stride + 1, both >= 1.
+ *   ep       host pointer; modes INT32, SCALED_F32, AFFINE_F32.
+ *   out_nchw device int32/fp32 [n, cout, oh, ow] contiguous.
+ *   Supports c <= 128.  Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED. */
+bnn_status bnn_binary_conv3x3_fused(const uint32_t* X_nhwc_bits, int64_t n, int64_t c, int64_t h,
+                                    int64_t w, const uint32_t* W_packed, int64_t ldw, int64_t cout,
+                                    int64_t stride, int64_t pad, const bnn_epilogue* ep,
+                                    void* out_nchw, bnn_stream_t stream);
+
+/* bnn_fold_bn_threshold -- HOST function: fold inference BatchNorm of
+ * alpha * s followed by sign() into an integer popcount threshold per channel.
+ *   Passage: glossary "Binary Neural Network (BNN)", BatchNorm paragraph (BN
+ *   before binarisation, alpha per filter); the pages give no BN formula.
+ *   The decision folded is, in IEEE double with each fp32 input widened:
+ *     v(s) = ((alpha*s - mean) / sqrt(var + eps)) * gamma + beta,
+ *     output +1 (bit 0) iff v(s) >= 0,
+ *   for every reachable s = K - 2d, d = 0..K.  The result reproduces that
+ *   decision exactly for every d: thresh_mode 0 -> bit = (d > popc_thresh),
+ *   thresh_mode 1 -> bit = (d < popc_thresh).  A constant decision is
+ *   encoded as mode 0 with popc_thresh = K (always +1) or -1 (always -1).
+ *   alpha, gamma, beta, mean, var: host fp32 [N]; popc_thresh: host int32 [N];
+ *   thresh_mode: host int8 [N].
+ *   Errors: INVALID_ARG (null, N < 0, K < 1, a non-finite parameter,
+ *   var + eps <= 0, alpha < 0). */
+bnn_status bnn_fold_bn_threshold(const float* alpha, const float* gamma, const float* beta,
+                                 const float* mean, const float* var, double eps, int64_t N,
+                                 int64_t K, int32_t* popc_thresh, int8_t* thresh_mode);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BNN_H_ */

@@ -1,0 +1,139 @@
+"""The C ABI without a GPU: the library loads, exports every symbol that
+include/bnn.h declares, and rejects bad arguments on the host before any CUDA
+call (so these checks run on a machine without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+import xnor_popcount_gemm_bnn_b200 as bnn
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "bnn.h")
+FAKE = ctypes.c_void_p(0x10000)        # aligned, never dereferenced: validation fails first
+FAKE_ODD = ctypes.c_void_p(0x10004)    # 4-byte but not 16-byte aligned
+NULL = None
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bnn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declarations_match_binding():
+    assert declared_functions() == sorted(bnn.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(bnn.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_packed_ld_words_matches_layout_reading():
+    for K in (1, 31, 32, 33, 127, 128, 129, 576, 1000, 4095, 4096, 4097, 8192, 123457):
+        assert bnn.bnn_packed_ld_words(K) == oracle.ld_words(K)
+    assert bnn.bnn_packed_ld_words(0) == -1
+    assert bnn.bnn_conv3x3_ld_words(64) == 20      # 9 taps x 2 words, rounded to 4
+    assert bnn.bnn_conv3x3_ld_words(1) == 12
+    assert bnn.bnn_conv3x3_ld_words(128) == 36
+    assert bnn.bnn_conv3x3_ld_words(0) == -1
+
+
+def test_status_strings():
+    for s in range(6):
+        assert isinstance(bnn.bnn_status_string(s), str) and bnn.bnn_status_string(s)
+    assert bnn.bnn_status_string(99) == "unknown status"
+
+
+L = bnn.lib
+
+
+def test_pack_sign_rejects_bad_arguments():
+    st = L.bnn_pack_sign
+    assert st(NULL, 0, 4, 32, 32, FAKE, 4, NULL, NULL) == bnn.BNN_ERR_INVALID_ARG
+    assert st(FAKE, 0, 4, 0, 32, FAKE, 4, NULL, NULL) == bnn.BNN_ERR_INVALID_ARG      # K < 1
+    assert st(FAKE, 0, 4, 64, 32, FAKE, 4, NULL, NULL) == bnn.BNN_ERR_INVALID_ARG     # ld_x < K
+    assert st(FAKE, 0, 4, 200, 200, FAKE, 4, NULL, NULL) == bnn.BNN_ERR_INVALID_ARG   # ld too small
+    assert st(FAKE, 0, 4, 32, 32, FAKE, 6, NULL, NULL) == bnn.BNN_ERR_ALIGNMENT       # ld % 4
+    assert st(FAKE, 0, 4, 32, 32, FAKE_ODD, 4, NULL, NULL) == bnn.BNN_ERR_ALIGNMENT
+    assert st(FAKE, 7, 4, 32, 32, FAKE, 4, NULL, NULL) == bnn.BNN_ERR_INVALID_ARG     # dtype
+    assert st(FAKE, 0, -1, 32, 32, FAKE, 4, NULL, NULL) == bnn.BNN_ERR_INVALID_ARG
+    assert st(FAKE, 0, 0, 32, 32, FAKE, 4, NULL, NULL) == bnn.BNN_OK                  # empty: no launch
+
+
+def test_gemm_rejects_bad_arguments():
+    g = L.bnn_xnor_gemm
+    ok = dict()
+    assert g(NULL, 4, FAKE, 4, 8, 8, 32, NULL, FAKE, 8, NULL, 0, NULL) == bnn.BNN_ERR_INVALID_ARG
+    assert g(FAKE, 4, FAKE, 4, 8, 8, 0, NULL, FAKE, 8, NULL, 0, NULL) == bnn.BNN_ERR_INVALID_ARG
+    assert g(FAKE, 4, FAKE, 4, 8, 8, 32, NULL, NULL, 0, NULL, 0, NULL) == bnn.BNN_ERR_INVALID_ARG  # no output
+    assert g(FAKE, 4, FAKE, 4, 8, 8, 32, NULL, NULL, 0, FAKE, 8, NULL) == bnn.BNN_ERR_INVALID_ARG  # f32 w/o alpha
+    assert g(FAKE, 4, FAKE, 4, 8, 8, 32, NULL, FAKE, 7, NULL, 0, NULL) == bnn.BNN_ERR_INVALID_ARG  # ldc < N
+    assert g(FAKE, 2, FAKE, 4, 8, 8, 32, NULL, FAKE, 8, NULL, 0, NULL) == bnn.BNN_ERR_INVALID_ARG  # lda < kw
+    assert g(FAKE, 6, FAKE, 4, 8, 8, 32, NULL, FAKE, 8, NULL, 0, NULL) == bnn.BNN_ERR_ALIGNMENT    # lda % 4
+    assert g(FAKE_ODD, 4, FAKE, 4, 8, 8, 32, NULL, FAKE, 8, NULL, 0, NULL) == bnn.BNN_ERR_ALIGNMENT
+    assert g(FAKE, 4, FAKE, 4, -1, 8, 32, NULL, FAKE, 8, NULL, 0, NULL) == bnn.BNN_ERR_INVALID_ARG
+    assert g(FAKE, 4, FAKE, 4, 0, 8, 32, NULL, FAKE, 8, NULL, 0, NULL) == bnn.BNN_OK               # M = 0
+    assert g(FAKE, 4, FAKE, 4, 8, 0, 32, NULL, FAKE, 8, NULL, 0, NULL) == bnn.BNN_OK               # N = 0
+    del ok
+
+
+def test_linear_fused_rejects_bad_epilogues():
+    f = L.bnn_binary_linear_fused
+    def ep(mode, **kw):
+        e = bnn.bnn_epilogue(mode, None, None, None, None, None)
+        for k, v in kw.items():
+            setattr(e, k, v)
+        return ctypes.byref(e)
+    args = (FAKE, 4, FAKE, 4, 8, 8, 32)
+    assert f(*args, NULL, FAKE, 8, NULL) == bnn.BNN_ERR_INVALID_ARG
+    assert f(*args, ep(99), FAKE, 8, NULL) == bnn.BNN_ERR_INVALID_ARG
+    assert f(*args, ep(bnn.BNN_OUT_SCALED_F32), FAKE, 8, NULL) == bnn.BNN_ERR_INVALID_ARG
+    assert f(*args, ep(bnn.BNN_OUT_AFFINE_F32, alpha=0x10000), FAKE, 8, NULL) == bnn.BNN_ERR_INVALID_ARG
+    assert f(*args, ep(bnn.BNN_OUT_THRESHOLD_PACK), FAKE, 4, NULL) == bnn.BNN_ERR_INVALID_ARG
+    assert f(*args, ep(bnn.BNN_OUT_THRESHOLD_PACK, popc_thresh=0x10000, thresh_mode=0x10000),
+             FAKE, 2, NULL) == bnn.BNN_ERR_INVALID_ARG     # ld_out < ld_words(N)
+    assert f(*args, ep(bnn.BNN_OUT_THRESHOLD_PACK, popc_thresh=0x10000, thresh_mode=0x10000),
+             FAKE, 6, NULL) == bnn.BNN_ERR_ALIGNMENT
+    assert f(*args, ep(bnn.BNN_OUT_INT32), FAKE, 7, NULL) == bnn.BNN_ERR_INVALID_ARG
+
+
+def test_gemv_rejects_bad_arguments():
+    g = L.bnn_xnor_gemv
+    assert g(FAKE, 4, NULL, 0, 8, 32, NULL, FAKE, NULL, NULL) == bnn.BNN_ERR_INVALID_ARG
+    assert g(FAKE, 4, FAKE, 0, 8, 32, NULL, NULL, NULL, NULL) == bnn.BNN_ERR_INVALID_ARG
+    assert g(FAKE, 4, FAKE, 0, 8, 32, NULL, NULL, FAKE, NULL) == bnn.BNN_ERR_INVALID_ARG   # f32 w/o alpha
+    assert g(FAKE, 4, FAKE, 0, 8, 129, NULL, FAKE, NULL, NULL) == bnn.BNN_ERR_INVALID_ARG  # ldw < kw
+    assert g(FAKE_ODD, 4, FAKE, 0, 8, 32, NULL, FAKE, NULL, NULL) == bnn.BNN_ERR_ALIGNMENT
+    assert g(FAKE, 4, FAKE, 5, 8, 32, NULL, FAKE, NULL, NULL) == bnn.BNN_ERR_INVALID_ARG
+    assert g(FAKE, 4, FAKE, 0, 0, 32, NULL, FAKE, NULL, NULL) == bnn.BNN_OK
+
+
+def test_conv_rejects_bad_arguments():
+    c = L.bnn_binary_conv3x3_fused
+    e = bnn.bnn_epilogue(bnn.BNN_OUT_INT32, None, None, None, None, None)
+    E = ctypes.byref(e)
+    assert c(NULL, 1, 64, 8, 8, FAKE, 20, 4, 1, 1, E, FAKE, NULL) == bnn.BNN_ERR_INVALID_ARG
+    assert c(FAKE, 1, 64, 8, 8, FAKE, 17, 4, 1, 1, E, FAKE, NULL) == bnn.BNN_ERR_INVALID_ARG   # ldw < 18
+    assert c(FAKE, 1, 64, 8, 8, FAKE, 20, 4, 0, 1, E, FAKE, NULL) == bnn.BNN_ERR_INVALID_ARG   # stride
+    assert c(FAKE, 1, 64, 1, 1, FAKE, 20, 4, 1, 0, E, FAKE, NULL) == bnn.BNN_ERR_INVALID_ARG   # no output
+    assert c(FAKE, 1, 160, 8, 8, FAKE, 48, 4, 1, 1, E, FAKE, NULL) == bnn.BNN_ERR_UNSUPPORTED  # c > 128
+    e2 = bnn.bnn_epilogue(bnn.BNN_OUT_THRESHOLD_PACK, None, None, None, None, None)
+    assert c(FAKE, 1, 64, 8, 8, FAKE, 20, 4, 1, 1, ctypes.byref(e2), FAKE, NULL) == bnn.BNN_ERR_UNSUPPORTED
+    assert c(FAKE, 0, 64, 8, 8, FAKE, 20, 4, 1, 1, E, FAKE, NULL) == bnn.BNN_OK
+
+
+def test_fold_rejects_bad_arguments():
+    import torch
+    a = torch.ones(4)
+    with pytest.raises(bnn.BnnError):
+        bnn.bnn_fold_bn_threshold(a, a, a, a, a * 0 - 1.0, 0.0, 16)         # var + eps <= 0
+    with pytest.raises(bnn.BnnError):
+        bnn.bnn_fold_bn_threshold(a * float("nan"), a, a, a, a, 1e-5, 16)   # non-finite
+    with pytest.raises(bnn.BnnError):
+        bnn.bnn_fold_bn_threshold(-a, a, a, a, a, 1e-5, 16)                 # alpha < 0
+    with pytest.raises(bnn.BnnError):
+        bnn.bnn_fold_bn_threshold(a, a, a, a, a, 1e-5, 0)                   # K < 1

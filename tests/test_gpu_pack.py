@@ -1,0 +1,124 @@
+"""Sign-and-pack kernels against the oracle: packed words bit-exact (pad bits
+and pad words included), alpha within 1e-6 relative."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import xnor_popcount_gemm_bnn_b200 as bnn
+from gpu_util import assert_no_device_error, dev, u32
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(1, 1), (5, 31), (7, 32), (3, 33), (2, 65), (9, 129), (64, 1000), (256, 1000),
+          (4, 4096), (3, 8192), (33, 4097), (1, 12345)]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("rows,K", SHAPES)
+def test_pack_sign_rows(rows, K, dtype):
+    x = workloads.random_with_edges(rows, K, seed=rows * 7919 + K, dtype=dtype)
+    xd = x.to(dev())
+    packed = bnn.empty_packed(rows, K, dev())
+    alpha = torch.empty(rows, dtype=torch.float32, device=dev())
+    bnn.bnn_pack_sign(xd, packed, alpha)
+    assert np.array_equal(u32(packed), oracle.pack_real(x))
+    a_ref = oracle.alpha(x)
+    a = alpha.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(a - a_ref) <= 1e-6 * np.abs(a_ref))
+    assert_no_device_error()
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_pack_sign_nonfinite_and_signed_zero(dtype):
+    edges = workloads.sign_edge_values(dtype)
+    x = edges.repeat(3, 11)[:, :150].contiguous()          # NaN, +-inf, -0.0, denormals ...
+    packed = bnn.empty_packed(x.shape[0], x.shape[1], dev())
+    bnn.bnn_pack_sign(x.to(dev()), packed)                   # no alpha
+    assert np.array_equal(u32(packed), oracle.pack_real(x))
+
+
+def test_pack_sign_strided_and_wide_ld():
+    """Row stride ld_x > K that breaks 16-byte alignment (scalar path), and an
+    output stride wider than needed: words past the padded row stay untouched."""
+    rows, K, ldx = 17, 999, 1003
+    base = workloads.normal((rows, ldx), 1.0, 42)
+    x = base[:, :K]
+    packed = torch.full((rows, bnn.bnn_packed_ld_words(K) + 8), -1, dtype=torch.int32, device=dev())
+    alpha = torch.empty(rows, dtype=torch.float32, device=dev())
+    bnn.bnn_pack_sign(base.to(dev())[:, :K], packed, alpha)
+    got = u32(packed)
+    kw = bnn.bnn_packed_ld_words(K)
+    assert np.array_equal(got[:, :kw], oracle.pack_real(x))
+    assert np.all(got[:, kw:] == 0xFFFFFFFF)
+    a_ref = oracle.alpha(x)
+    assert np.all(np.abs(alpha.cpu().numpy() - a_ref) <= 1e-6 * a_ref)
+
+
+def test_pack_sign_alpha_closed_form():
+    rows, K = 8, 1000
+    c = 0.375
+    sgn = torch.where(workloads.normal((rows, K), 1.0, 5) < 0, -1.0, 1.0)
+    x = (c * sgn).to(torch.float32)
+    packed = bnn.empty_packed(rows, K, dev())
+    alpha = torch.empty(rows, dtype=torch.float32, device=dev())
+    bnn.bnn_pack_sign(x.to(dev()), packed, alpha)
+    assert torch.all(alpha.cpu() == c)
+
+
+def test_pack_sign_gemv_weights_full_size():
+    """The LLM-decode weight matrix [11008, 4096] fp32 N(0, 0.02)."""
+    g = workloads.gemv()
+    packed = bnn.empty_packed(g.N, g.K, dev())
+    alpha = torch.empty(g.N, dtype=torch.float32, device=dev())
+    bnn.bnn_pack_sign(g.W.to(dev()), packed, alpha)
+    assert np.array_equal(u32(packed), oracle.pack_real(g.W))
+    a_ref = oracle.alpha(g.W)
+    assert np.all(np.abs(alpha.cpu().numpy() - a_ref) <= 1e-6 * a_ref)
+    assert_no_device_error()
+
+
+def expected_nhwc(x):
+    """Oracle words per pixel: sign of the channel vector, packed (first cw words)."""
+    n, c, h, w = x.shape
+    cw = (c + 31) // 32
+    xs = x.float().permute(0, 2, 3, 1).reshape(-1, c)
+    return oracle.pack_real(xs)[:, :cw].reshape(n, h, w, cw)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("shape", [(2, 64, 5, 7), (2, 33, 8, 8), (1, 1, 3, 3), (3, 100, 4, 6),
+                                   (2, 64, 56, 56)])
+def test_pack_sign_nchw(shape, dtype):
+    n, c, h, w = shape
+    x = workloads.random_with_edges(n * c, h * w, seed=sum(shape), dtype=dtype).reshape(shape).contiguous()
+    out = bnn.empty_packed_nhwc(n, c, h, w, dev())
+    bnn.bnn_pack_sign_nchw(x.to(dev()), out)
+    assert np.array_equal(u32(out), expected_nhwc(x))
+
+
+def expected_conv_weights(wt):
+    """Oracle rows in (kh, kw, c) order, channels padded to whole words per tap."""
+    cout, cin = wt.shape[:2]
+    cw = (cin + 31) // 32
+    t = wt.float().permute(0, 2, 3, 1)                                 # co, kh, kw, c
+    tp = torch.zeros(cout, 3, 3, 32 * cw)
+    tp[..., :cin] = t
+    packed = oracle.pack_real(tp.reshape(cout, -1))                    # zeros pack as +1
+    ldk = bnn.bnn_conv3x3_ld_words(cin)
+    out = np.zeros((cout, ldk), np.uint32)
+    out[:, :9 * cw] = packed[:, :9 * cw]
+    return out
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("cout,cin", [(64, 64), (5, 3), (7, 33), (16, 128)])
+def test_pack_conv3x3_weights(cout, cin, dtype):
+    wt = workloads.normal((cout, cin, 3, 3), 0.1, cout * 100 + cin).to(dtype)
+    packed = bnn.empty_conv3x3_weights(cout, cin, dev())
+    alpha = torch.empty(cout, dtype=torch.float32, device=dev())
+    bnn.bnn_pack_conv3x3_weights(wt.to(dev()).contiguous(), packed, alpha)
+    assert np.array_equal(u32(packed), expected_conv_weights(wt))
+    a_ref = oracle.alpha(wt.float().reshape(cout, -1))
+    assert np.all(np.abs(alpha.cpu().numpy() - a_ref) <= 1e-6 * a_ref)

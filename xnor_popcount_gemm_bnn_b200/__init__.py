@@ -1,0 +1,252 @@
+"""Python binding of libbnn.so: the binary (+1/-1) matrix product on packed bits.
+
+Thin ``ctypes`` marshalling over the C ABI in ``include/bnn.h``; the functions
+keep the C names.  Tensors are torch tensors (device memory on the current
+CUDA device, host memory for ``bnn_fold_bn_threshold``); every device call is
+launched on ``torch.cuda.current_stream()`` unless a stream is given.  All
+computation happens in the library's CUDA kernels; nothing here computes.
+There is no CPU fallback: importing the package fails if ``libbnn.so`` has
+not been built (``python -m xnor_popcount_gemm_bnn_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbnn.so")
+
+BNN_OK = 0
+BNN_ERR_INVALID_ARG = 1
+BNN_ERR_ALIGNMENT = 2
+BNN_ERR_UNSUPPORTED = 3
+BNN_ERR_CUDA = 4
+BNN_ERR_DEVICE_TIMEOUT = 5
+
+BNN_F32 = 0
+BNN_BF16 = 1
+
+BNN_OUT_INT32 = 1
+BNN_OUT_SCALED_F32 = 2
+BNN_OUT_AFFINE_F32 = 4
+BNN_OUT_THRESHOLD_PACK = 8
+
+# Every symbol declared in include/bnn.h.
+EXPORTS = (
+    "bnn_packed_ld_words", "bnn_conv3x3_ld_words", "bnn_status_string", "bnn_device_error",
+    "bnn_pack_sign", "bnn_pack_sign_nchw", "bnn_pack_conv3x3_weights", "bnn_xnor_gemm",
+    "bnn_xnor_gemv", "bnn_binary_linear_fused", "bnn_binary_conv3x3_fused",
+    "bnn_fold_bn_threshold",
+)
+
+
+class BnnError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} failed: status {status} ({msg})")
+        self.status = status
+
+
+class bnn_epilogue(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int32), ("alpha", ctypes.c_void_p), ("gamma", ctypes.c_void_p),
+                ("beta", ctypes.c_void_p), ("popc_thresh", ctypes.c_void_p),
+                ("thresh_mode", ctypes.c_void_p)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m xnor_popcount_gemm_bnn_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    i64, p, i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int32
+    sig = {
+        "bnn_packed_ld_words": (i64, [i64]),
+        "bnn_conv3x3_ld_words": (i64, [i64]),
+        "bnn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "bnn_device_error": (i32, [p]),
+        "bnn_pack_sign": (i32, [p, i32, i64, i64, i64, p, i64, p, p]),
+        "bnn_pack_sign_nchw": (i32, [p, i32, i64, i64, i64, i64, p, p]),
+        "bnn_pack_conv3x3_weights": (i32, [p, i32, i64, i64, p, i64, p, p]),
+        "bnn_xnor_gemm": (i32, [p, i64, p, i64, i64, i64, i64, p, p, i64, p, i64, p]),
+        "bnn_xnor_gemv": (i32, [p, i64, p, i32, i64, i64, p, p, p, p]),
+        "bnn_binary_linear_fused": (i32, [p, i64, p, i64, i64, i64, i64,
+                                          ctypes.POINTER(bnn_epilogue), p, i64, p]),
+        "bnn_binary_conv3x3_fused": (i32, [p, i64, i64, i64, i64, p, i64, i64, i64, i64,
+                                           ctypes.POINTER(bnn_epilogue), p, p]),
+        "bnn_fold_bn_threshold": (i32, [p, p, p, p, p, ctypes.c_double, i64, i64, p, p]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+lib = _lib
+
+
+def _check(fn: str, status: int) -> None:
+    if status != BNN_OK:
+        raise BnnError(fn, status, _lib.bnn_status_string(status).decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return BNN_F32
+    if t.dtype == torch.bfloat16:
+        return BNN_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; expected float32 or bfloat16")
+
+
+def _ld(t: torch.Tensor) -> int:
+    return t.stride(0) if t.dim() >= 2 else t.shape[-1]
+
+
+# --------------------------------------------------------------------------
+# sizes and status
+# --------------------------------------------------------------------------
+
+def bnn_packed_ld_words(K: int) -> int:
+    return int(_lib.bnn_packed_ld_words(int(K)))
+
+
+def bnn_conv3x3_ld_words(cin: int) -> int:
+    return int(_lib.bnn_conv3x3_ld_words(int(cin)))
+
+
+def bnn_status_string(status: int) -> str:
+    return _lib.bnn_status_string(int(status)).decode()
+
+
+def bnn_device_error() -> int:
+    code = ctypes.c_int32(0)
+    _check("bnn_device_error", _lib.bnn_device_error(ctypes.byref(code)))
+    return int(code.value)
+
+
+# --------------------------------------------------------------------------
+# packing
+# --------------------------------------------------------------------------
+
+def bnn_pack_sign(x: torch.Tensor, packed: torch.Tensor, alpha_out: Optional[torch.Tensor] = None,
+                  K: Optional[int] = None, stream=None) -> None:
+    """x [rows, K] (fp32/bf16, unit inner stride) -> packed uint32 [rows, ld] (int32 storage)."""
+    if x.dim() == 1:
+        x = x.view(1, -1)
+    assert x.stride(-1) == 1 and packed.stride(-1) == 1
+    rows, Kx = x.shape
+    K = Kx if K is None else int(K)
+    _check("bnn_pack_sign", _lib.bnn_pack_sign(
+        _ptr(x), _dtype(x), rows, K, _ld(x), _ptr(packed), _ld(packed) if packed.dim() >= 2 else packed.shape[-1],
+        _ptr(alpha_out), _stream(stream)))
+
+
+def bnn_pack_sign_nchw(x: torch.Tensor, packed_nhwc: torch.Tensor, stream=None) -> None:
+    assert x.is_contiguous() and packed_nhwc.is_contiguous()
+    n, c, h, w = x.shape
+    _check("bnn_pack_sign_nchw", _lib.bnn_pack_sign_nchw(
+        _ptr(x), _dtype(x), n, c, h, w, _ptr(packed_nhwc), _stream(stream)))
+
+
+def bnn_pack_conv3x3_weights(w_oihw: torch.Tensor, packed: torch.Tensor,
+                             alpha_out: Optional[torch.Tensor] = None, stream=None) -> None:
+    assert w_oihw.is_contiguous() and tuple(w_oihw.shape[2:]) == (3, 3)
+    cout, cin = w_oihw.shape[:2]
+    _check("bnn_pack_conv3x3_weights", _lib.bnn_pack_conv3x3_weights(
+        _ptr(w_oihw), _dtype(w_oihw), cout, cin, _ptr(packed), _ld(packed), _ptr(alpha_out),
+        _stream(stream)))
+
+
+# --------------------------------------------------------------------------
+# products
+# --------------------------------------------------------------------------
+
+def bnn_xnor_gemm(A: torch.Tensor, W: torch.Tensor, K: int, alpha: Optional[torch.Tensor] = None,
+                  C_i32: Optional[torch.Tensor] = None, C_f32: Optional[torch.Tensor] = None,
+                  M: Optional[int] = None, N: Optional[int] = None, stream=None) -> None:
+    M = A.shape[0] if M is None else M
+    N = W.shape[0] if N is None else N
+    _check("bnn_xnor_gemm", _lib.bnn_xnor_gemm(
+        _ptr(A), _ld(A), _ptr(W), _ld(W), M, N, int(K), _ptr(alpha),
+        _ptr(C_i32), _ld(C_i32) if C_i32 is not None else 0,
+        _ptr(C_f32), _ld(C_f32) if C_f32 is not None else 0, _stream(stream)))
+
+
+def bnn_xnor_gemv(W: torch.Tensor, x: torch.Tensor, K: Optional[int] = None,
+                  alpha: Optional[torch.Tensor] = None, y_i32: Optional[torch.Tensor] = None,
+                  y_f32: Optional[torch.Tensor] = None, N: Optional[int] = None, stream=None) -> None:
+    N = W.shape[0] if N is None else N
+    K = x.shape[-1] if K is None else int(K)
+    _check("bnn_xnor_gemv", _lib.bnn_xnor_gemv(
+        _ptr(W), _ld(W), _ptr(x), _dtype(x), N, K, _ptr(alpha), _ptr(y_i32), _ptr(y_f32),
+        _stream(stream)))
+
+
+def make_epilogue(mode: int, alpha=None, gamma=None, beta=None, popc_thresh=None,
+                  thresh_mode=None) -> bnn_epilogue:
+    return bnn_epilogue(int(mode), _ptr(alpha), _ptr(gamma), _ptr(beta), _ptr(popc_thresh),
+                        _ptr(thresh_mode))
+
+
+def bnn_binary_linear_fused(A: torch.Tensor, W: torch.Tensor, K: int, ep: bnn_epilogue,
+                            out: torch.Tensor, M: Optional[int] = None, N: Optional[int] = None,
+                            stream=None) -> None:
+    M = A.shape[0] if M is None else M
+    N = W.shape[0] if N is None else N
+    _check("bnn_binary_linear_fused", _lib.bnn_binary_linear_fused(
+        _ptr(A), _ld(A), _ptr(W), _ld(W), M, N, int(K), ctypes.byref(ep), _ptr(out), _ld(out),
+        _stream(stream)))
+
+
+def bnn_binary_conv3x3_fused(X_bits: torch.Tensor, c: int, W_packed: torch.Tensor,
+                             ep: bnn_epilogue, out_nchw: torch.Tensor, stride: int = 1, pad: int = 1,
+                             stream=None) -> None:
+    n, h, w = X_bits.shape[:3]
+    cout = W_packed.shape[0]
+    _check("bnn_binary_conv3x3_fused", _lib.bnn_binary_conv3x3_fused(
+        _ptr(X_bits), n, int(c), h, w, _ptr(W_packed), _ld(W_packed), cout, int(stride), int(pad),
+        ctypes.byref(ep), _ptr(out_nchw), _stream(stream)))
+
+
+def bnn_fold_bn_threshold(alpha: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor,
+                          mean: torch.Tensor, var: torch.Tensor, eps: float, K: int):
+    """Host call: returns (popc_thresh int32 [N], thresh_mode int8 [N]) as CPU tensors."""
+    ts = [t.detach().to("cpu", torch.float32).contiguous() for t in (alpha, gamma, beta, mean, var)]
+    N = ts[0].numel()
+    thr = torch.empty(N, dtype=torch.int32)
+    mode = torch.empty(N, dtype=torch.int8)
+    _check("bnn_fold_bn_threshold", _lib.bnn_fold_bn_threshold(
+        *[_ptr(t) for t in ts], float(eps), N, int(K), _ptr(thr), _ptr(mode)))
+    return thr, mode
+
+
+# --------------------------------------------------------------------------
+# allocation helpers (torch device memory; the library itself allocates nothing)
+# --------------------------------------------------------------------------
+
+def empty_packed(rows: int, K: int, device="cuda") -> torch.Tensor:
+    """int32-typed storage for a packed [rows, bnn_packed_ld_words(K)] matrix."""
+    return torch.empty(rows, bnn_packed_ld_words(K), dtype=torch.int32, device=device)
+
+
+def empty_packed_nhwc(n: int, c: int, h: int, w: int, device="cuda") -> torch.Tensor:
+    return torch.empty(n, h, w, (c + 31) // 32, dtype=torch.int32, device=device)
+
+
+def empty_conv3x3_weights(cout: int, cin: int, device="cuda") -> torch.Tensor:
+    return torch.empty(cout, bnn_conv3x3_ld_words(cin), dtype=torch.int32, device=device)

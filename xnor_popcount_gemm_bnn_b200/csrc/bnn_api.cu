@@ -1,0 +1,414 @@
+// libbnn.so: the C ABI declared in include/bnn.h.  Host code here only checks
+// arguments, encodes TMA descriptors, picks launch shapes and launches on the
+// caller's stream; every step of the computation runs in the kernels of
+// pack.cuh, gemm_popc.cuh, gemv.cuh and conv.cuh.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <climits>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "bnn.h"
+#include "common.cuh"
+#include "conv.cuh"
+#include "gemm_popc.cuh"
+#include "gemv.cuh"
+#include "pack.cuh"
+
+namespace {
+
+using bnn::packed_ld_words;
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+inline cudaStream_t as_cuda(bnn_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bnn_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? BNN_OK : BNN_ERR_CUDA;
+}
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// cuTensorMapEncodeTiled from the driver, fetched through the runtime so that
+// the library does not link libcuda directly.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D map over a packed matrix: inner dimension = kw words, outer = rows,
+// box 32 words x 128 rows, 128-byte swizzle, zero fill out of range.
+bool encode_packed_map(CUtensorMap* map, const uint32_t* base, int64_t kw, int64_t rows, int64_t ld) {
+    auto enc = tensor_map_encoder();
+    if (enc == nullptr) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)kw, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ld * 4u};
+    cuuint32_t box[2] = {(cuuint32_t)bnn::gemm::BKW, (cuuint32_t)bnn::gemm::BM};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(base), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Opt the GEMM kernel into its dynamic shared memory once per device (the
+// attribute is per device; doing it once keeps it out of captured graphs).
+bool gemm_smem_configured() {
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> done[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+    if (dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return true;
+    if (cudaFuncSetAttribute(bnn::xnor_gemm_popc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bnn::gemm::SMEM_BYTES) != cudaSuccess)
+        return false;
+    if (dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
+    return true;
+}
+
+bnn_status check_packed_operand(const uint32_t* p, int64_t ld, int64_t kw) {
+    if (p == nullptr) return BNN_ERR_INVALID_ARG;
+    if (ld < kw) return BNN_ERR_INVALID_ARG;
+    if ((ld & 3) != 0 || !aligned(p, 16)) return BNN_ERR_ALIGNMENT;
+    return BNN_OK;
+}
+
+bnn_status launch_gemm(const uint32_t* A, int64_t lda, const uint32_t* W, int64_t ldw, int64_t M, int64_t N,
+                       int64_t K, const bnn::GemmEpilogue& ep, cudaStream_t stream) {
+    using namespace bnn::gemm;
+    const int64_t kw = packed_ld_words(K);
+    CUtensorMap tmA, tmW;
+    if (!encode_packed_map(&tmA, A, kw, M, lda) || !encode_packed_map(&tmW, W, kw, N, ldw))
+        return BNN_ERR_CUDA;
+    const int64_t tiles_n = ceil_div(N, BN);
+    const int64_t tiles = ceil_div(M, BM) * tiles_n;
+    if (tiles > INT_MAX) return BNN_ERR_INVALID_ARG;
+    if (!gemm_smem_configured())
+        return BNN_ERR_CUDA;
+    bnn::xnor_gemm_popc_kernel<<<(unsigned)tiles, THREADS, SMEM_BYTES, stream>>>(
+        tmA, tmW, (int)M, (int)N, (int)K, (int)kw, (int)tiles_n, ep);
+    return launch_status();
+}
+
+bnn_status check_gemm_dims(int64_t M, int64_t N, int64_t K) {
+    if (M < 0 || N < 0 || K < 1) return BNN_ERR_INVALID_ARG;
+    if (M > INT_MAX || N > INT_MAX || K > (INT_MAX / 2)) return BNN_ERR_INVALID_ARG;
+    return BNN_OK;
+}
+
+template <typename XT>
+bnn_status launch_gemv_t(const uint32_t* W, int64_t ldw, const XT* x, int64_t N, int64_t K, int64_t kw,
+                         const float* alpha, int32_t* y_i32, float* y_f32, bool weights_static,
+                         cudaStream_t stream) {
+    using namespace bnn::gemv;
+    const int64_t nchunks = kw / 4;
+    int lpr = 1;
+    while (lpr < 32 && lpr < nchunks) lpr <<= 1;
+    const int64_t rows_per_block = (int64_t)WARPS * U * (32 / lpr);
+    const int64_t blocks = ceil_div(N, rows_per_block);
+    const size_t smem = (size_t)kw * 4;
+
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = weights_static ? 1 : 0;
+
+    cudaError_t e = cudaSuccess;
+    const int iN = (int)N, iK = (int)K, ikw = (int)kw;
+#define BNN_GEMV_CASE(L)                                                                           \
+    case L: {                                                                                      \
+        auto kern = bnn::xnor_gemv_kernel<XT, L>;                                                  \
+        if (smem > 48 * 1024 &&                                                                    \
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=  \
+                cudaSuccess)                                                                       \
+            return BNN_ERR_CUDA;                                                                   \
+        e = cudaLaunchKernelEx(&cfg, kern, W, ldw, x, iN, iK, ikw, alpha, y_i32, y_f32,            \
+                               weights_static);                                                    \
+        break;                                                                                     \
+    }
+    switch (lpr) {
+        BNN_GEMV_CASE(1)
+        BNN_GEMV_CASE(2)
+        BNN_GEMV_CASE(4)
+        BNN_GEMV_CASE(8)
+        BNN_GEMV_CASE(16)
+        BNN_GEMV_CASE(32)
+        default: return BNN_ERR_UNSUPPORTED;
+    }
+#undef BNN_GEMV_CASE
+    if (e != cudaSuccess) return BNN_ERR_CUDA;
+    return launch_status();
+}
+
+constexpr int64_t kGemvMaxWords = 48 * 1024;   // packed x in shared memory: <= 192 KiB
+
+bnn_status gemv_impl(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt, int64_t N, int64_t K,
+                     const float* alpha, int32_t* y_i32, float* y_f32, bool weights_static,
+                     bnn_stream_t stream) {
+    if (N < 0 || K < 1 || N > INT_MAX || K > INT_MAX / 2) return BNN_ERR_INVALID_ARG;
+    if (x == nullptr || (y_i32 == nullptr && y_f32 == nullptr)) return BNN_ERR_INVALID_ARG;
+    if (y_f32 != nullptr && alpha == nullptr) return BNN_ERR_INVALID_ARG;
+    if (x_dt != BNN_F32 && x_dt != BNN_BF16) return BNN_ERR_INVALID_ARG;
+    const int64_t kw = packed_ld_words(K);
+    bnn_status st = check_packed_operand(W, ldw, kw);
+    if (st != BNN_OK) return st;
+    if (kw > kGemvMaxWords) return BNN_ERR_UNSUPPORTED;
+    if (!aligned(x, x_dt == BNN_F32 ? 4 : 2)) return BNN_ERR_ALIGNMENT;
+    if (N == 0) return BNN_OK;
+    if (x_dt == BNN_F32)
+        return launch_gemv_t(W, ldw, static_cast<const float*>(x), N, K, kw, alpha, y_i32, y_f32,
+                             weights_static, as_cuda(stream));
+    return launch_gemv_t(W, ldw, static_cast<const __nv_bfloat16*>(x), N, K, kw, alpha, y_i32, y_f32,
+                         weights_static, as_cuda(stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t bnn_packed_ld_words(int64_t K) { return K < 1 ? -1 : packed_ld_words(K); }
+
+int64_t bnn_conv3x3_ld_words(int64_t cin) {
+    if (cin < 1) return -1;
+    return (9 * ((cin + 31) / 32) + 3) / 4 * 4;
+}
+
+const char* bnn_status_string(int status) {
+    switch (status) {
+        case BNN_OK: return "ok";
+        case BNN_ERR_INVALID_ARG: return "invalid argument";
+        case BNN_ERR_ALIGNMENT: return "pointer or leading dimension not aligned";
+        case BNN_ERR_UNSUPPORTED: return "unsupported shape, dtype or mode";
+        case BNN_ERR_CUDA: return "CUDA error";
+        case BNN_ERR_DEVICE_TIMEOUT: return "a kernel gave up waiting on an asynchronous copy";
+        default: return "unknown status";
+    }
+}
+
+bnn_status bnn_device_error(int32_t* code_out) {
+    if (code_out == nullptr) return BNN_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return BNN_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, bnn::g_device_error, sizeof(int)) != cudaSuccess) return BNN_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(bnn::g_device_error, &zero, sizeof(int)) != cudaSuccess) return BNN_ERR_CUDA;
+    }
+    *code_out = v;
+    return BNN_OK;
+}
+
+bnn_status bnn_pack_sign(const void* x, bnn_dtype dt, int64_t rows, int64_t K, int64_t ld_x, uint32_t* packed,
+                         int64_t ld_words, float* alpha_out, bnn_stream_t stream) {
+    if (x == nullptr || packed == nullptr) return BNN_ERR_INVALID_ARG;
+    if (rows < 0 || K < 1 || ld_x < K) return BNN_ERR_INVALID_ARG;
+    if (dt != BNN_F32 && dt != BNN_BF16) return BNN_ERR_INVALID_ARG;
+    const int64_t kw = packed_ld_words(K);
+    if (ld_words < kw) return BNN_ERR_INVALID_ARG;
+    if ((ld_words & 3) != 0 || !aligned(packed, 16)) return BNN_ERR_ALIGNMENT;
+    const size_t es = dt == BNN_F32 ? 4 : 2;
+    if (!aligned(x, es) || (alpha_out != nullptr && !aligned(alpha_out, 4))) return BNN_ERR_ALIGNMENT;
+    if (rows == 0) return BNN_OK;
+    const bool vec_ok = aligned(x, 16) && ((ld_x * (int64_t)es) % 16 == 0);
+    const int64_t blocks = ceil_div(rows, 8);
+    if (blocks > INT_MAX) return BNN_ERR_INVALID_ARG;
+    cudaStream_t s = as_cuda(stream);
+    if (dt == BNN_F32)
+        bnn::pack_sign_rows_kernel<float, 4><<<(unsigned)blocks, 256, 0, s>>>(
+            static_cast<const float*>(x), rows, K, ld_x, packed, ld_words, alpha_out, kw, vec_ok);
+    else
+        bnn::pack_sign_rows_kernel<__nv_bfloat16, 4><<<(unsigned)blocks, 256, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(x), rows, K, ld_x, packed, ld_words, alpha_out, kw, vec_ok);
+    return launch_status();
+}
+
+bnn_status bnn_pack_sign_nchw(const void* x, bnn_dtype dt, int64_t n, int64_t c, int64_t h, int64_t w,
+                              uint32_t* packed_nhwc, bnn_stream_t stream) {
+    if (x == nullptr || packed_nhwc == nullptr) return BNN_ERR_INVALID_ARG;
+    if (n < 0 || c < 1 || h < 1 || w < 1) return BNN_ERR_INVALID_ARG;
+    if (dt != BNN_F32 && dt != BNN_BF16) return BNN_ERR_INVALID_ARG;
+    const size_t es = dt == BNN_F32 ? 4 : 2;
+    if (!aligned(x, es) || !aligned(packed_nhwc, 4)) return BNN_ERR_ALIGNMENT;
+    if (n == 0) return BNN_OK;
+    const int64_t hw = h * w, cw = (c + 31) / 32;
+    const int64_t threads = n * ceil_div(hw, 8) * cw;
+    const int64_t blocks = ceil_div(threads, 256);
+    if (blocks > INT_MAX) return BNN_ERR_INVALID_ARG;
+    const bool vec_ok = aligned(x, 16) && (hw % 8 == 0);
+    cudaStream_t s = as_cuda(stream);
+    if (dt == BNN_F32)
+        bnn::pack_sign_nchw_kernel<float><<<(unsigned)blocks, 256, 0, s>>>(static_cast<const float*>(x), n, c, hw,
+                                                                           cw, packed_nhwc, vec_ok);
+    else
+        bnn::pack_sign_nchw_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(x), n, c, hw, cw, packed_nhwc, vec_ok);
+    return launch_status();
+}
+
+bnn_status bnn_pack_conv3x3_weights(const void* w_oihw, bnn_dtype dt, int64_t cout, int64_t cin,
+                                    uint32_t* packed, int64_t ld_words, float* alpha_out, bnn_stream_t stream) {
+    if (w_oihw == nullptr || packed == nullptr) return BNN_ERR_INVALID_ARG;
+    if (cout < 0 || cin < 1) return BNN_ERR_INVALID_ARG;
+    if (dt != BNN_F32 && dt != BNN_BF16) return BNN_ERR_INVALID_ARG;
+    if (ld_words < bnn_conv3x3_ld_words(cin)) return BNN_ERR_INVALID_ARG;
+    if ((ld_words & 3) != 0 || !aligned(packed, 16)) return BNN_ERR_ALIGNMENT;
+    if (!aligned(w_oihw, dt == BNN_F32 ? 4 : 2)) return BNN_ERR_ALIGNMENT;
+    if (cout == 0) return BNN_OK;
+    const int64_t blocks = ceil_div(cout, 8);
+    if (blocks > INT_MAX) return BNN_ERR_INVALID_ARG;
+    cudaStream_t s = as_cuda(stream);
+    if (dt == BNN_F32)
+        bnn::pack_conv3x3_weights_kernel<float><<<(unsigned)blocks, 256, 0, s>>>(
+            static_cast<const float*>(w_oihw), cout, cin, packed, ld_words, alpha_out);
+    else
+        bnn::pack_conv3x3_weights_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(w_oihw), cout, cin, packed, ld_words, alpha_out);
+    return launch_status();
+}
+
+bnn_status bnn_xnor_gemm(const uint32_t* A, int64_t lda, const uint32_t* W, int64_t ldw, int64_t M, int64_t N,
+                         int64_t K, const float* alpha, int32_t* C_i32, int64_t ldc, float* C_f32, int64_t ldf,
+                         bnn_stream_t stream) {
+    bnn_status st = check_gemm_dims(M, N, K);
+    if (st != BNN_OK) return st;
+    const int64_t kw = packed_ld_words(K);
+    if ((st = check_packed_operand(A, lda, kw)) != BNN_OK) return st;
+    if ((st = check_packed_operand(W, ldw, kw)) != BNN_OK) return st;
+    if (C_i32 == nullptr && C_f32 == nullptr) return BNN_ERR_INVALID_ARG;
+    if (C_i32 != nullptr && ldc < N) return BNN_ERR_INVALID_ARG;
+    if (C_f32 != nullptr && (ldf < N || alpha == nullptr)) return BNN_ERR_INVALID_ARG;
+    if ((C_i32 && !aligned(C_i32, 4)) || (C_f32 && !aligned(C_f32, 4))) return BNN_ERR_ALIGNMENT;
+    if (M == 0 || N == 0) return BNN_OK;
+    bnn::GemmEpilogue ep{};
+    ep.c_i32 = C_i32;
+    ep.ldc = ldc;
+    ep.c_f32 = C_f32;
+    ep.ldf = ldf;
+    ep.alpha = alpha;
+    return launch_gemm(A, lda, W, ldw, M, N, K, ep, as_cuda(stream));
+}
+
+bnn_status bnn_xnor_gemv(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt, int64_t N, int64_t K,
+                         const float* alpha, int32_t* y_i32, float* y_f32, bnn_stream_t stream) {
+    return gemv_impl(W, ldw, x, x_dt, N, K, alpha, y_i32, y_f32, false, stream);
+}
+
+bnn_status bnn_binary_linear_fused(const uint32_t* A, int64_t lda, const uint32_t* W, int64_t ldw, int64_t M,
+                                   int64_t N, int64_t K, const bnn_epilogue* epi, void* out, int64_t ld_out,
+                                   bnn_stream_t stream) {
+    bnn_status st = check_gemm_dims(M, N, K);
+    if (st != BNN_OK) return st;
+    if (epi == nullptr || out == nullptr) return BNN_ERR_INVALID_ARG;
+    const int64_t kw = packed_ld_words(K);
+    if ((st = check_packed_operand(A, lda, kw)) != BNN_OK) return st;
+    if ((st = check_packed_operand(W, ldw, kw)) != BNN_OK) return st;
+    if (!aligned(out, 4)) return BNN_ERR_ALIGNMENT;
+    bnn::GemmEpilogue ep{};
+    switch (epi->mode) {
+        case BNN_OUT_INT32:
+            if (ld_out < N) return BNN_ERR_INVALID_ARG;
+            ep.c_i32 = static_cast<int32_t*>(out);
+            ep.ldc = ld_out;
+            break;
+        case BNN_OUT_SCALED_F32:
+        case BNN_OUT_AFFINE_F32:
+            if (ld_out < N || epi->alpha == nullptr) return BNN_ERR_INVALID_ARG;
+            if (epi->mode == BNN_OUT_AFFINE_F32 && (epi->gamma == nullptr || epi->beta == nullptr))
+                return BNN_ERR_INVALID_ARG;
+            ep.c_f32 = static_cast<float*>(out);
+            ep.ldf = ld_out;
+            ep.alpha = epi->alpha;
+            if (epi->mode == BNN_OUT_AFFINE_F32) {
+                ep.gamma = epi->gamma;
+                ep.beta = epi->beta;
+            }
+            break;
+        case BNN_OUT_THRESHOLD_PACK:
+            if (epi->popc_thresh == nullptr || epi->thresh_mode == nullptr) return BNN_ERR_INVALID_ARG;
+            if (N > 0 && ld_out < packed_ld_words(N)) return BNN_ERR_INVALID_ARG;
+            if ((ld_out & 3) != 0) return BNN_ERR_ALIGNMENT;
+            ep.c_bits = static_cast<uint32_t*>(out);
+            ep.ldb = ld_out;
+            ep.thresh = epi->popc_thresh;
+            ep.thresh_mode = epi->thresh_mode;
+            break;
+        default:
+            return BNN_ERR_INVALID_ARG;
+    }
+    if (M == 0 || N == 0) return BNN_OK;
+    return launch_gemm(A, lda, W, ldw, M, N, K, ep, as_cuda(stream));
+}
+
+bnn_status bnn_binary_conv3x3_fused(const uint32_t* X_nhwc_bits, int64_t n, int64_t c, int64_t h, int64_t w,
+                                    const uint32_t* W_packed, int64_t ldw, int64_t cout, int64_t stride, int64_t pad,
+                                    const bnn_epilogue* epi, void* out_nchw, bnn_stream_t stream) {
+    if (X_nhwc_bits == nullptr || W_packed == nullptr || epi == nullptr || out_nchw == nullptr)
+        return BNN_ERR_INVALID_ARG;
+    if (n < 0 || c < 1 || h < 1 || w < 1 || cout < 0 || stride < 1 || pad < 0) return BNN_ERR_INVALID_ARG;
+    if (h > INT_MAX / 4 || w > INT_MAX / 4 || c > INT_MAX / 16 || cout > INT_MAX || pad > 1024 || stride > 1024)
+        return BNN_ERR_INVALID_ARG;
+    const int64_t oh = (h + 2 * pad - 3) / stride + 1, ow = (w + 2 * pad - 3) / stride + 1;
+    if (h + 2 * pad < 3 || w + 2 * pad < 3 || oh < 1 || ow < 1) return BNN_ERR_INVALID_ARG;
+    const int64_t cw = (c + 31) / 32;
+    if (ldw < 9 * cw) return BNN_ERR_INVALID_ARG;
+    switch (epi->mode) {
+        case BNN_OUT_INT32: break;
+        case BNN_OUT_SCALED_F32:
+            if (epi->alpha == nullptr) return BNN_ERR_INVALID_ARG;
+            break;
+        case BNN_OUT_AFFINE_F32:
+            if (epi->alpha == nullptr || epi->gamma == nullptr || epi->beta == nullptr) return BNN_ERR_INVALID_ARG;
+            break;
+        case BNN_OUT_THRESHOLD_PACK: return BNN_ERR_UNSUPPORTED;
+        default: return BNN_ERR_INVALID_ARG;
+    }
+    if (!aligned(X_nhwc_bits, 4) || !aligned(W_packed, 16) || !aligned(out_nchw, 4)) return BNN_ERR_ALIGNMENT;
+    if (cw > 4) return BNN_ERR_UNSUPPORTED;
+    const int64_t kwp = (9 * cw + 3) / 4 * 4;
+    const size_t smem = (size_t)cout * kwp * 4;
+    if (smem > 200 * 1024) return BNN_ERR_UNSUPPORTED;
+    if (n == 0 || cout == 0) return BNN_OK;
+    const int64_t npix = n * oh * ow;
+    const int64_t blocks = ceil_div(npix, (int64_t)bnn::conv::WARPS * 32 * bnn::conv::P);
+    if (blocks > INT_MAX) return BNN_ERR_INVALID_ARG;
+    bnn::ConvEpilogue ep{epi->mode, epi->alpha, epi->gamma, epi->beta, out_nchw};
+    cudaStream_t s = as_cuda(stream);
+#define BNN_CONV_CASE(CWV)                                                                                 \
+    case CWV: {                                                                                            \
+        auto kern = bnn::xnor_conv3x3_kernel<CWV>;                                                         \
+        if (smem > 48 * 1024 &&                                                                            \
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) \
+            return BNN_ERR_CUDA;                                                                           \
+        kern<<<(unsigned)blocks, bnn::conv::THREADS, smem, s>>>(X_nhwc_bits, (int)n, (int)c, (int)h, (int)w,  \
+                                                                W_packed, ldw, (int)cout, (int)stride,     \
+                                                                (int)pad, (int)oh, (int)ow, ep);           \
+        break;                                                                                             \
+    }
+    switch (cw) {
+        BNN_CONV_CASE(1)
+        BNN_CONV_CASE(2)
+        BNN_CONV_CASE(3)
+        BNN_CONV_CASE(4)
+        default: return BNN_ERR_UNSUPPORTED;
+    }
+#undef BNN_CONV_CASE
+    return launch_status();
+}
+
+}  // extern "C"

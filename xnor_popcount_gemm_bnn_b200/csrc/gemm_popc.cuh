@@ -1,0 +1,200 @@
+// Packed binary GEMM on the integer pipes: d[m, n] = sum_w popcount(A[m, w]
+// XOR W[n, w]), s = K - 2 d ("Extreme Quantization: Binary, Ternary & 1-bit
+// LLMs", XNOR-Net eq. (6); "First Principles: Why Binary Ops Can Be
+// Exponentially Faster", section 1), with a fused epilogue: int32 s, alpha*s
+// (eq. (1)), gamma*(alpha*s)+beta, or a popcount threshold re-packed into
+// sign bits for the next layer (folded BatchNorm).
+//
+// Design (sm_100a):
+//  * CTA tile 128 x 128 outputs, K staged 32 words (1024 binary elements) at
+//    a time.  One producer warp issues TMA tile loads (no multicast) into a
+//    4-stage ring of 128B-swizzled shared-memory tiles; completion is tracked
+//    with mbarriers (full: TMA bytes landed; empty: all 8 compute warps are
+//    done with the stage).  Every wait is bounded (about 1 s) and reports
+//    BNN_ERR_DEVICE_TIMEOUT instead of hanging.
+//  * 8 compute warps; thread (tx, ty) of a 16 x 16 grid owns rows ty + 16 i
+//    and columns tx + 16 j (i, j < 8): 64 int32 accumulators.  Per 16-byte
+//    chunk (4 words) it loads 8 A vectors and 8 W vectors and does 256
+//    XOR + POPC + ADD.  The 128B swizzle makes the 8 rows read by a quarter
+//    warp fall on 8 distinct 16-byte bank groups.
+//  * Zero-filled out-of-range TMA boxes make ragged M, N and K (pad words)
+//    contribute nothing to d.
+#pragma once
+
+#include "common.cuh"
+
+namespace bnn {
+namespace gemm {
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int BKW = 32;                      // words per K stage (128 bytes per row)
+constexpr int STAGES = 4;
+constexpr int COMPUTE_WARPS = 8;
+constexpr int THREADS = (COMPUTE_WARPS + 1) * 32;
+constexpr int A_TILE_BYTES = BM * BKW * 4;   // 16 KiB
+constexpr int W_TILE_BYTES = BN * BKW * 4;   // 16 KiB
+constexpr int STAGE_BYTES = A_TILE_BYTES + W_TILE_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 2 * STAGES * 8 + 1024;
+}  // namespace gemm
+
+struct GemmEpilogue {
+    int32_t* c_i32;           // int32 s, or null
+    int64_t ldc;
+    float* c_f32;             // alpha*s (or gamma*(alpha*s)+beta when gamma != null), or null
+    int64_t ldf;
+    const float* alpha;
+    const float* gamma;
+    const float* beta;
+    uint32_t* c_bits;         // THRESHOLD_PACK output, or null
+    int64_t ldb;              // words
+    const int32_t* thresh;
+    const int8_t* thresh_mode;
+};
+
+__global__ void __launch_bounds__(gemm::THREADS, 1)
+xnor_gemm_popc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
+                      int M, int N, int K, int kw, int tiles_n, GemmEpilogue ep) {
+    using namespace gemm;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    uint64_t* empty = full + STAGES;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int tile_m = blockIdx.x / tiles_n;
+    const int tile_n = blockIdx.x % tiles_n;
+    const int m0 = tile_m * BM;
+    const int n0 = tile_n * BN;
+    const int nk = (kw + BKW - 1) / BKW;
+
+    if (threadIdx.x == 0) {
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmW);
+        #pragma unroll
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], COMPUTE_WARPS);
+        }
+        fence_mbarrier_init();
+    }
+    __syncthreads();
+
+    if (warp == COMPUTE_WARPS) {
+        // ---------------- producer warp ----------------
+        if (lane == 0) {
+            int issued = 0;
+            for (int kt = 0; kt < nk; ++kt) {
+                const int s = kt % STAGES;
+                const uint32_t ph = (kt / STAGES) & 1;
+                if (kt >= STAGES && !mbar_wait_bounded(&empty[s], ph ^ 1)) break;
+                uint8_t* sa = smem + s * STAGE_BYTES;
+                mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+                tma_load_2d(sa, &tmA, kt * BKW, m0, &full[s]);
+                tma_load_2d(sa + A_TILE_BYTES, &tmW, kt * BKW, n0, &full[s]);
+                ++issued;
+            }
+            // Do not let the CTA retire while copies are still landing.
+            for (int kt = max(0, issued - STAGES); kt < issued; ++kt)
+                if (!mbar_wait_bounded(&full[kt % STAGES], (kt / STAGES) & 1)) break;
+        }
+        return;
+    }
+
+    // ---------------- compute warps ----------------
+    const int t = threadIdx.x;
+    const int tx = t & 15;
+    const int ty = t >> 4;
+    const int swa = ty & 7;   // (ty + 16 i) & 7
+    const int swb = tx & 7;   // (tx + 16 j) & 7
+    uint32_t acc[8][8];
+    #pragma unroll
+    for (int i = 0; i < 8; ++i)
+        #pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0u;
+
+    for (int kt = 0; kt < nk; ++kt) {
+        const int s = kt % STAGES;
+        // Warp-uniform decision, so that no lane leaves while others reach a ballot.
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (kt / STAGES) & 1))) return;
+        const uint8_t* As = smem + s * STAGE_BYTES;
+        const uint8_t* Ws = As + A_TILE_BYTES;
+        #pragma unroll 2
+        for (int c = 0; c < BKW / 4; ++c) {
+            uint4 a[8], b[8];
+            #pragma unroll
+            for (int i = 0; i < 8; ++i)
+                a[i] = *reinterpret_cast<const uint4*>(As + (ty + 16 * i) * 128 + ((c ^ swa) << 4));
+            #pragma unroll
+            for (int j = 0; j < 8; ++j)
+                b[j] = *reinterpret_cast<const uint4*>(Ws + (tx + 16 * j) * 128 + ((c ^ swb) << 4));
+            #pragma unroll
+            for (int i = 0; i < 8; ++i)
+                #pragma unroll
+                for (int j = 0; j < 8; ++j) acc[i][j] += popc_xor4(a[i], b[j]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+    }
+
+    // ---------------- epilogue ----------------
+    if (ep.c_i32 != nullptr || ep.c_f32 != nullptr) {
+        float al[8], ga[8], be[8];
+        #pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int n = n0 + tx + 16 * j;
+            const bool in = n < N;
+            al[j] = (ep.alpha != nullptr && in) ? ep.alpha[n] : 0.0f;
+            ga[j] = (ep.gamma != nullptr && in) ? ep.gamma[n] : 0.0f;
+            be[j] = (ep.beta != nullptr && in) ? ep.beta[n] : 0.0f;
+        }
+        #pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int m = m0 + ty + 16 * i;
+            if (m >= M) continue;
+            #pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int n = n0 + tx + 16 * j;
+                if (n >= N) continue;
+                const int32_t sv = K - 2 * (int32_t)acc[i][j];
+                if (ep.c_i32 != nullptr) ep.c_i32[(int64_t)m * ep.ldc + n] = sv;
+                if (ep.c_f32 != nullptr) {
+                    float y = al[j] * (float)sv;
+                    if (ep.gamma != nullptr) y = fmaf(ga[j], y, be[j]);
+                    ep.c_f32[(int64_t)m * ep.ldf + n] = y;
+                }
+            }
+        }
+    }
+    if (ep.c_bits != nullptr) {
+        int32_t th[8];
+        int8_t md[8];
+        #pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int n = n0 + tx + 16 * j;
+            th[j] = (n < N) ? ep.thresh[n] : 0;
+            md[j] = (n < N) ? ep.thresh_mode[n] : (int8_t)-1;   // -1: column past N, bit 0
+        }
+        #pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int m_even = m0 + 2 * warp + 16 * i;   // lanes 0..15 hold row ty = 2*warp
+            #pragma unroll
+            for (int q = 0; q < 4; ++q) {                 // word q of the 128-column tile
+                const int j0 = 2 * q, j1 = 2 * q + 1;
+                const int32_t d0 = (int32_t)acc[i][j0], d1 = (int32_t)acc[i][j1];
+                const bool bit0 = md[j0] == 0 ? (d0 > th[j0]) : (md[j0] == 1 ? (d0 < th[j0]) : false);
+                const bool bit1 = md[j1] == 0 ? (d1 > th[j1]) : (md[j1] == 1 ? (d1 < th[j1]) : false);
+                const uint32_t b0 = __ballot_sync(0xffffffffu, bit0);
+                const uint32_t b1 = __ballot_sync(0xffffffffu, bit1);
+                const int64_t word = n0 / 32 + q;
+                if (lane == 0 && m_even < M)
+                    ep.c_bits[(int64_t)m_even * ep.ldb + word] = (b0 & 0xffffu) | (b1 << 16);
+                if (lane == 16 && m_even + 1 < M)
+                    ep.c_bits[(int64_t)(m_even + 1) * ep.ldb + word] = (b0 >> 16) | (b1 & 0xffff0000u);
+            }
+        }
+    }
+}
+
+}  // namespace bnn
