@@ -251,12 +251,19 @@ def run_ours(args, torch, dist):
     copies = (copies + 7) // 8 * 8                       # 48
     g, Ws, alpha, x, y = gemv_setup(torch, bnn, workloads, dev, copies)
 
+    # Decode: the weights are resident model parameters, so the GEMV may start
+    # streaming them before the previous step's kernel has finished.
     def step(i):
+        bnn.bnn_xnor_gemv_ex(Ws[i % copies], x, g.K, alpha, None, y, flags=bnn.BNN_GEMV_WEIGHTS_STATIC)
+
+    def step_plain(i):
         bnn.bnn_xnor_gemv(Ws[i % copies], x, g.K, alpha, None, y)
 
     with ClockSampler(local) as clk:
         ms = time_steps(torch, step, args.steps, args.warmup, copies, sync)
     ms = max_over_ranks(ms)
+    plain_steps = min(args.steps, 48 * copies)
+    ms_plain = max_over_ranks(time_steps(torch, step_plain, plain_steps, args.warmup, copies, sync))
     if bnn.bnn_device_error() != 0:
         raise RuntimeError("a kernel reported a device-side timeout")
     per_step_bytes = gemv_bytes()
@@ -299,6 +306,10 @@ def run_ours(args, torch, dist):
         },
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
+        "gemv_default_flags": {
+            "value": round(ws * plain_steps * per_step_bytes / (ms_plain * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "steps": plain_steps, "ms_per_step": ms_plain / plain_steps,
+            "note": "bnn_xnor_gemv without the static-weights flag: W is read after the dependency wait"},
     }
 
     # e2e: the public API with host buffers
@@ -315,6 +326,23 @@ def run_ours(args, torch, dist):
     return result
 
 
+def run_only_rows(args, torch, dist):
+    import workloads
+    import xnor_popcount_gemm_bnn_b200 as bnn
+    ws, rank, local = dist_env()
+    dev = torch.device("cuda", local)
+
+    def sync():
+        if dist is not None:
+            dist.barrier()
+
+    names = [n for n in args.only_rows.split(",") if n]
+    for n in names:
+        if n not in ROW_NAMES:
+            raise SystemExit(f"unknown row {n!r}; choose from {ROW_NAMES}")
+    return {"rows": bench_rows(torch, bnn, workloads, dev, peaks(), args, sync, lambda v: v, ws, names)}
+
+
 def e2e_gemv(torch, bnn, g, Ws, alpha, dev, steps, sync, max_over_ranks, ws):
     x_host = g.x.clone().pin_memory()
     y_host = torch.empty(g.N, dtype=torch.float32).pin_memory()
@@ -324,7 +352,7 @@ def e2e_gemv(torch, bnn, g, Ws, alpha, dev, steps, sync, max_over_ranks, ws):
 
     def one(i):
         x_dev.copy_(x_host, non_blocking=True)
-        bnn.bnn_xnor_gemv(Ws[i % copies], x_dev, g.K, alpha, None, y_dev)
+        bnn.bnn_xnor_gemv_ex(Ws[i % copies], x_dev, g.K, alpha, None, y_dev, flags=bnn.BNN_GEMV_WEIGHTS_STATIC)
         y_host.copy_(y_dev, non_blocking=True)
 
     for i in range(5):
@@ -343,15 +371,19 @@ def e2e_gemv(torch, bnn, g, Ws, alpha, dev, steps, sync, max_over_ranks, ws):
             "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
             "d2h_bytes_per_step": y_host.numel() * y_host.element_size(),
             "steps": steps, "ms_per_step": ms / steps,
-            "path": "eager Python calls of bnn_xnor_gemv with pinned-host copies each step"}
+            "path": "eager Python calls of bnn_xnor_gemv_ex with pinned-host copies each step"}
 
 
 # ---------------------------------------------------------------------------
 # the other rows
 # ---------------------------------------------------------------------------
 
-def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws):
+ROW_NAMES = ("pack_sign_weights", "square_gemm", "conv3x3", "mlp4")
+
+
+def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws, only=None):
     rows = {}
+    want = set(only or ROW_NAMES)
     steps = max(3, args.row_steps)
     warm = max(3, args.warmup)
     clk_mhz = pk["sm_max_mhz"]
@@ -361,6 +393,20 @@ def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws):
         return max_over_ranks(time_steps(torch, fn, n, warm, period or n, sync))
 
     # --- a1: weight pack + alpha, fp32 [11008, 4096] (HBM) ---
+    if "pack_sign_weights" in want:
+        _row_pack(torch, bnn, workloads, dev, pk, rows, timed, steps, ws)
+    if "square_gemm" in want:
+        _row_square(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, clk_mhz)
+    if "conv3x3" in want:
+        _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak)
+    if "mlp4" in want:
+        _row_mlp(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak)
+    if bnn.bnn_device_error() != 0:
+        raise RuntimeError("a kernel reported a device-side timeout")
+    return rows
+
+
+def _row_pack(torch, bnn, workloads, dev, pk, rows, timed, steps, ws):
     g = workloads.gemv()
     Wd = g.W.to(dev)
     W_p = bnn.empty_packed(g.N, g.K, dev)
@@ -376,6 +422,8 @@ def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws):
     del Wd, W_p, alpha, g
     torch.cuda.empty_cache()
 
+
+def _row_square(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, clk_mhz):
     # --- a2+a3+a6: square GEMM 8192^3, int32 + alpha-scaled fp32 outputs ---
     sq = workloads.square()
     Ad = sq.A.to(dev)
@@ -403,6 +451,8 @@ def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws):
     del sq, Ad, A_p, Wsq, al, Ci, Cf
     torch.cuda.empty_cache()
 
+
+def _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak):
     # --- a2 (NCHW) + a5 + a6: ResNet-class binary 3x3 conv with affine epilogue ---
     cv = workloads.conv()
     n, c, h, w = cv.X.shape
@@ -435,6 +485,8 @@ def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws):
     del cv, Xd, Xb, Wc, alc, gam, bet, out
     torch.cuda.empty_cache()
 
+
+def _row_mlp(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak):
     # --- MLP: pack input, 3 x (GEMM + folded-BN re-pack), GEMM + alpha ---
     m = workloads.mlp()
     B, D = m.X0.shape
@@ -477,9 +529,6 @@ def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws):
                      "frac": round(mmacs * steps / (ms_m * 1e-3) / alu_peak, 4)}}
     del m, X0, A0, acts, eps_, Wps, logits
     torch.cuda.empty_cache()
-    if bnn.bnn_device_error() != 0:
-        raise RuntimeError("a kernel reported a device-side timeout")
-    return rows
 
 
 # ---------------------------------------------------------------------------
@@ -589,6 +638,9 @@ def main():
     ap.add_argument("--no-rows", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only-rows", default=None,
+                    help="comma-separated rows to time alone (no headline line); for profiling: "
+                         + ",".join(ROW_NAMES))
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -611,7 +663,10 @@ def main():
     else:
         torch.cuda.set_device(local)
     try:
-        result = run_ours(args, torch, dist)
+        if args.only_rows:
+            result = run_only_rows(args, torch, dist)
+        else:
+            result = run_ours(args, torch, dist)
         if rank == 0:
             print(json.dumps(result), flush=True)
     finally:

@@ -192,6 +192,25 @@ bnn_status bnn_xnor_gemv(const uint32_t* W, int64_t ldw, const void* x, bnn_dtyp
                          int64_t N, int64_t K, const float* alpha,
                          int32_t* y_i32, float* y_f32, bnn_stream_t stream);
 
+/* Flags of bnn_xnor_gemv_ex. */
+typedef enum bnn_gemv_flags {
+    BNN_GEMV_WEIGHTS_STATIC = 1   /* W is not written by any work still in flight on the stream */
+} bnn_gemv_flags;
+
+/* bnn_xnor_gemv_ex -- bnn_xnor_gemv with flags.  Both calls launch the kernel
+ * with programmatic dependent launch: it may be scheduled while the previous
+ * kernel on the stream is still running, and it waits for that kernel to
+ * complete before it reads x or alpha or writes y.  With
+ * BNN_GEMV_WEIGHTS_STATIC the loads of W are issued before that wait, so
+ * consecutive GEMVs over resident weights (one decode step through many
+ * layers) stream their weights back to back.  The caller guarantees that no
+ * earlier work on the stream that may still be running writes W; otherwise
+ * pass 0 (then equivalent to bnn_xnor_gemv).
+ *   Errors: as bnn_xnor_gemv; INVALID_ARG for unknown flag bits. */
+bnn_status bnn_xnor_gemv_ex(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt,
+                            int64_t N, int64_t K, const float* alpha,
+                            int32_t* y_i32, float* y_f32, uint32_t flags, bnn_stream_t stream);
+
 /* bnn_binary_linear_fused -- packed binary GEMM with one fused epilogue.
  *   Passage: eq. (6) (product), eq. (1) (alpha), the glossary's BatchNorm
  *   paragraph (normalise, then binarise for the next layer).

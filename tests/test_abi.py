@@ -112,6 +112,12 @@ def test_gemv_rejects_bad_arguments():
     assert g(FAKE, 4, FAKE, 0, 0, 32, NULL, FAKE, NULL, NULL) == bnn.BNN_OK
 
 
+def test_gemv_ex_rejects_bad_flags():
+    g = L.bnn_xnor_gemv_ex
+    assert g(FAKE, 4, FAKE, 0, 8, 32, NULL, FAKE, NULL, 2, NULL) == bnn.BNN_ERR_INVALID_ARG
+    assert g(FAKE, 4, FAKE, 0, 0, 32, NULL, FAKE, NULL, 1, NULL) == bnn.BNN_OK
+
+
 def test_conv_rejects_bad_arguments():
     c = L.bnn_binary_conv3x3_fused
     e = bnn.bnn_epilogue(bnn.BNN_OUT_INT32, None, None, None, None, None)

@@ -81,3 +81,71 @@ def test_gemv_equals_gemm_row():
     y_v = torch.empty(N, dtype=torch.int32, device=d)
     bnn.bnn_xnor_gemv(W_p, x.to(d), K, None, y_v)
     assert torch.equal(y_g[0], y_v)
+
+
+def _chain_reference(Ws, x0):
+    """Oracle chain: x_{l+1} = alpha_l * s_l (float64), s_l from sign(W_l), sign(x_l)."""
+    x = np.asarray(x0, dtype=np.float64)
+    out = []
+    for W in Ws:
+        s = oracle.gemv_pm1(oracle.sign_pm1(W), oracle.sign_pm1(x.astype(np.float32)))
+        y = oracle.scaled(s, oracle.alpha(W))
+        out.append((s, y))
+        x = y
+    return out
+
+
+@pytest.mark.parametrize("use_graph", [False, True])
+def test_static_weights_chain_orders_dependent_gemvs(use_graph):
+    """Eight GEMVs back to back on one stream with BNN_GEMV_WEIGHTS_STATIC,
+    each reading the previous one's fp32 output as its x: the dependency wait
+    must order every read of x after the previous kernel's writes."""
+    D, L = 4096, 8
+    d = dev()
+    Ws = [workloads.normal((D, D), 1.0, 500 + l) for l in range(L)]
+    x0 = workloads.normal((D,), 1.0, 499)
+    Wp, al = [], []
+    for W in Ws:
+        p = bnn.empty_packed(D, D, d)
+        a = torch.empty(D, dtype=torch.float32, device=d)
+        bnn.bnn_pack_sign(W.to(d), p, a)
+        Wp.append(p)
+        al.append(a)
+    xs = [x0.to(d)] + [torch.empty(D, dtype=torch.float32, device=d) for _ in range(L)]
+    ys = [torch.empty(D, dtype=torch.int32, device=d) for _ in range(L)]
+    torch.cuda.synchronize()
+
+    def chain():
+        for l in range(L):
+            bnn.bnn_xnor_gemv_ex(Wp[l], xs[l], D, al[l], ys[l], xs[l + 1], flags=bnn.BNN_GEMV_WEIGHTS_STATIC)
+
+    if use_graph:
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            chain()
+        torch.cuda.current_stream().wait_stream(s)
+        for t in xs[1:]:
+            t.fill_(float("nan"))
+        with torch.cuda.graph(g):
+            chain()
+        for t in xs[1:]:
+            t.fill_(float("nan"))
+        g.replay()
+    else:
+        chain()
+    torch.cuda.synchronize()
+    ref = _chain_reference(Ws, x0.numpy())
+    for l in range(L):
+        assert np.array_equal(ys[l].cpu().numpy(), ref[l][0]), f"layer {l}"
+        assert_scaled_close(xs[l + 1], ref[l][1])
+    assert_no_device_error()
+
+
+def test_gemv_ex_rejects_unknown_flags():
+    W = bnn.empty_packed(8, 64, dev())
+    x = torch.zeros(64, device=dev())
+    y = torch.empty(8, dtype=torch.int32, device=dev())
+    with pytest.raises(bnn.BnnError):
+        bnn.bnn_xnor_gemv_ex(W, x, 64, None, y, None, flags=2)

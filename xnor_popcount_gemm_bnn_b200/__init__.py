@@ -6,7 +6,7 @@ CUDA device, host memory for ``bnn_fold_bn_threshold``); every device call is
 launched on ``torch.cuda.current_stream()`` unless a stream is given.  All
 computation happens in the library's CUDA kernels; nothing here computes.
 There is no CPU fallback: importing the package fails if ``libbnn.so`` has
-not been built (``python -m xnor_popcount_gemm_bnn_b200.build``).
+not been built (``python xnor_popcount_gemm_bnn_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -34,11 +34,13 @@ BNN_OUT_SCALED_F32 = 2
 BNN_OUT_AFFINE_F32 = 4
 BNN_OUT_THRESHOLD_PACK = 8
 
+BNN_GEMV_WEIGHTS_STATIC = 1
+
 # Every symbol declared in include/bnn.h.
 EXPORTS = (
     "bnn_packed_ld_words", "bnn_conv3x3_ld_words", "bnn_status_string", "bnn_device_error",
     "bnn_pack_sign", "bnn_pack_sign_nchw", "bnn_pack_conv3x3_weights", "bnn_xnor_gemm",
-    "bnn_xnor_gemv", "bnn_binary_linear_fused", "bnn_binary_conv3x3_fused",
+    "bnn_xnor_gemv", "bnn_xnor_gemv_ex", "bnn_binary_linear_fused", "bnn_binary_conv3x3_fused",
     "bnn_fold_bn_threshold",
 )
 
@@ -58,7 +60,7 @@ class bnn_epilogue(ctypes.Structure):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m xnor_popcount_gemm_bnn_b200.build` (nvcc, sm_100a)")
+                          "`python xnor_popcount_gemm_bnn_b200/build.py` (nvcc, sm_100a)")
     lib = ctypes.CDLL(LIB_PATH)
     i64, p, i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int32
     sig = {
@@ -71,6 +73,7 @@ def _load() -> ctypes.CDLL:
         "bnn_pack_conv3x3_weights": (i32, [p, i32, i64, i64, p, i64, p, p]),
         "bnn_xnor_gemm": (i32, [p, i64, p, i64, i64, i64, i64, p, p, i64, p, i64, p]),
         "bnn_xnor_gemv": (i32, [p, i64, p, i32, i64, i64, p, p, p, p]),
+        "bnn_xnor_gemv_ex": (i32, [p, i64, p, i32, i64, i64, p, p, p, ctypes.c_uint32, p]),
         "bnn_binary_linear_fused": (i32, [p, i64, p, i64, i64, i64, i64,
                                           ctypes.POINTER(bnn_epilogue), p, i64, p]),
         "bnn_binary_conv3x3_fused": (i32, [p, i64, i64, i64, i64, p, i64, i64, i64, i64,
@@ -195,6 +198,17 @@ def bnn_xnor_gemv(W: torch.Tensor, x: torch.Tensor, K: Optional[int] = None,
     _check("bnn_xnor_gemv", _lib.bnn_xnor_gemv(
         _ptr(W), _ld(W), _ptr(x), _dtype(x), N, K, _ptr(alpha), _ptr(y_i32), _ptr(y_f32),
         _stream(stream)))
+
+
+def bnn_xnor_gemv_ex(W: torch.Tensor, x: torch.Tensor, K: Optional[int] = None,
+                     alpha: Optional[torch.Tensor] = None, y_i32: Optional[torch.Tensor] = None,
+                     y_f32: Optional[torch.Tensor] = None, flags: int = 0, N: Optional[int] = None,
+                     stream=None) -> None:
+    N = W.shape[0] if N is None else N
+    K = x.shape[-1] if K is None else int(K)
+    _check("bnn_xnor_gemv_ex", _lib.bnn_xnor_gemv_ex(
+        _ptr(W), _ld(W), _ptr(x), _dtype(x), N, K, _ptr(alpha), _ptr(y_i32), _ptr(y_f32),
+        int(flags), _stream(stream)))
 
 
 def make_epilogue(mode: int, alpha=None, gamma=None, beta=None, popc_thresh=None,

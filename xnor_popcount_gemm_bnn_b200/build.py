@@ -1,6 +1,8 @@
 """Build ``libbnn.so`` in-tree with nvcc for sm_100a.
 
-    python -m xnor_popcount_gemm_bnn_b200.build [--force] [--ptxas-v]
+    python xnor_popcount_gemm_bnn_b200/build.py [--force] [--ptxas-v]
+
+(Run as a file: importing the package loads the library this script builds.)
 
 The library links the CUDA runtime statically, so loading it needs no CUDA
 shared library; the first CUDA call needs a driver and a GPU.

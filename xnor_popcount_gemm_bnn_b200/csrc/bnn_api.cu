@@ -127,7 +127,7 @@ bnn_status launch_gemv_t(const uint32_t* W, int64_t ldw, const XT* x, int64_t N,
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = weights_static ? 1 : 0;
+    cfg.numAttrs = 1;
 
     cudaError_t e = cudaSuccess;
     const int iN = (int)N, iK = (int)K, ikw = (int)kw;
@@ -307,6 +307,14 @@ bnn_status bnn_xnor_gemm(const uint32_t* A, int64_t lda, const uint32_t* W, int6
 bnn_status bnn_xnor_gemv(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt, int64_t N, int64_t K,
                          const float* alpha, int32_t* y_i32, float* y_f32, bnn_stream_t stream) {
     return gemv_impl(W, ldw, x, x_dt, N, K, alpha, y_i32, y_f32, false, stream);
+}
+
+bnn_status bnn_xnor_gemv_ex(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt, int64_t N, int64_t K,
+                            const float* alpha, int32_t* y_i32, float* y_f32, uint32_t flags,
+                            bnn_stream_t stream) {
+    if ((flags & ~(uint32_t)BNN_GEMV_WEIGHTS_STATIC) != 0) return BNN_ERR_INVALID_ARG;
+    return gemv_impl(W, ldw, x, x_dt, N, K, alpha, y_i32, y_f32, (flags & BNN_GEMV_WEIGHTS_STATIC) != 0,
+                     stream);
 }
 
 bnn_status bnn_binary_linear_fused(const uint32_t* A, int64_t lda, const uint32_t* W, int64_t ldw, int64_t M,

@@ -15,10 +15,12 @@
 //    row groups before using any of them, keeping U * 512 bytes per warp in
 //    flight.
 //  * Row sums: redux.sync (one instruction) when LPR = 32, else a shuffle tree.
-//  * The loads of W do not depend on earlier kernels' results only when the
-//    caller says so (weights_static): then they are issued before the
-//    programmatic-launch wait, overlapping the previous kernel's tail; x and
-//    the outputs are always touched after the wait.
+//  * Launched with programmatic dependent launch: the grid may start while
+//    the previous kernel on the stream finishes, and waits for it
+//    (griddepcontrol.wait) before reading x or alpha and before writing y.
+//    When the caller declares the weights static (nothing still in flight on
+//    the stream writes W), the W loads are issued before that wait, so the
+//    weight stream of consecutive GEMVs runs back to back.
 #pragma once
 
 #include "common.cuh"
@@ -37,6 +39,7 @@ xnor_gemv_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restri
                  float* __restrict__ y_f32, bool weights_static) {
     using namespace gemv;
     constexpr int RPI = 32 / LPR;  // rows per warp-wide load
+    constexpr int XB = 16;         // x words packed per warp per batch (all loads in flight)
     extern __shared__ __align__(16) uint32_t xs[];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -48,13 +51,9 @@ xnor_gemv_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restri
     #pragma unroll
     for (int u = 0; u < U; ++u) rows[u] = (int)((gw * U + u) * RPI + sub);
 
+    // Let the next kernel on the stream start its own prologue now; it waits
+    // for this grid to finish before it touches anything this grid writes.
     grid_dependents_launch();
-
-    // Chunk loop (a single pass when nchunks <= LPR).
-    uint32_t d[U];
-    #pragma unroll
-    for (int u = 0; u < U; ++u) d[u] = 0u;
-    const int passes = (nchunks + LPR - 1) / LPR;
 
     uint4 v[U];
     auto load_pass = [&](int t) {
@@ -66,19 +65,36 @@ xnor_gemv_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restri
                        : make_uint4(0u, 0u, 0u, 0u);
     };
 
+    // The weight stream does not depend on x.  With static weights it starts
+    // before the dependency wait (overlapping the previous kernel's tail);
+    // otherwise right after it, still ahead of the x loads.
     if (weights_static) load_pass(0);
     grid_dependency_wait();
+    if (!weights_static) load_pass(0);
 
     // Pack x into shared memory: word wd <- ballot over elements 32*wd + lane.
-    for (int wd = warp; wd < kw; wd += WARPS) {
-        const int e = 32 * wd + lane;
-        const float xv = (e < K) ? to_float(x[e]) : 0.0f;
-        const uint32_t word = __ballot_sync(0xffffffffu, xv < 0.0f);
-        if (lane == 0) xs[wd] = word;
+    // XB words per warp per batch, all loads issued before the first ballot.
+    for (int wd0 = warp; wd0 < kw; wd0 += WARPS * XB) {
+        float xv[XB];
+        #pragma unroll
+        for (int j = 0; j < XB; ++j) {
+            const int wd = wd0 + WARPS * j;
+            const int e = 32 * wd + lane;
+            xv[j] = (wd < kw && e < K) ? to_float(x[e]) : 0.0f;
+        }
+        #pragma unroll
+        for (int j = 0; j < XB; ++j) {
+            const int wd = wd0 + WARPS * j;
+            const uint32_t word = __ballot_sync(0xffffffffu, xv[j] < 0.0f);
+            if (lane == 0 && wd < kw) xs[wd] = word;
+        }
     }
     __syncthreads();
 
-    if (!weights_static) load_pass(0);
+    uint32_t d[U];
+    #pragma unroll
+    for (int u = 0; u < U; ++u) d[u] = 0u;
+    const int passes = (nchunks + LPR - 1) / LPR;
     for (int t = 0; t < passes; ++t) {
         if (t > 0) load_pass(t);
         const int c = li + LPR * t;
