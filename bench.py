@@ -32,7 +32,6 @@ on the host cores on the same workload and metric; rank 0 only.
 from __future__ import annotations
 
 import argparse
-import glob
 import hashlib
 import json
 import math
@@ -66,6 +65,21 @@ def dist_env():
     return ws, rank, local
 
 
+def reduce_max(torch, dist, v: float, device) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    if dist is None:
+        return float(v)
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world_size: int, steps: int, units_per_step: float, ms_max: float) -> float:
+    """Whole-job units/s: every rank processes `steps` steps of its own replica,
+    timed as the slowest rank (weak scaling)."""
+    return world_size * steps * units_per_step / (ms_max * 1e-3)
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -80,22 +94,31 @@ def alu_peak_mac_s(sm_mhz: float) -> float:
     return SM_COUNT * POPC_PER_CLK_PER_SM * 32 * sm_mhz * 1e6
 
 
-def source_hash() -> str:
+# Source files that determine each kernel's code (its own header + shared helpers).
+KERNEL_SOURCES = {
+    "xnor_gemv_kernel": ("gemv.cuh", "common.cuh"),
+    "xnor_gemm_popc_kernel": ("gemm_popc.cuh", "common.cuh"),
+    "xnor_conv3x3_kernel": ("conv.cuh", "common.cuh"),
+    "pack_sign_rows_kernel": ("pack.cuh", "common.cuh"),
+}
+
+
+def source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "xnor_popcount_gemm_bnn_b200", "csrc", "*"))):
-        h.update(open(f, "rb").read())
+    for f in KERNEL_SOURCES[kernel]:
+        h.update(open(os.path.join(ROOT, "xnor_popcount_gemm_bnn_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources; else None."""
+    """DRAM bytes per launch (read + write) from the committed ncu summary, if it
+    was captured on the kernel's current sources; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
     e = d.get(kernel)
-    if not e or e.get("source_hash") != source_hash():
+    if not e or e.get("source_hash") != source_hash(kernel):
         return None
     return e.get("bytes_per_launch")
 
@@ -241,11 +264,7 @@ def run_ours(args, torch, dist):
             dist.barrier()
 
     def max_over_ranks(v):
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(torch, dist, v, dev)
 
     copies = max(2, math.ceil(2 * L2_BYTES / gemv_bytes()) + 1)
     copies = (copies + 7) // 8 * 8                       # 48
@@ -267,7 +286,7 @@ def run_ours(args, torch, dist):
     if bnn.bnn_device_error() != 0:
         raise RuntimeError("a kernel reported a device-side timeout")
     per_step_bytes = gemv_bytes()
-    value = ws * args.steps * per_step_bytes / (ms * 1e-3) / 1e9
+    value = job_throughput(ws, args.steps, per_step_bytes, ms) / 1e9
     launch_s = ms * 1e-3 / args.steps
     achieved = per_step_bytes / launch_s / 1e9
 

@@ -161,6 +161,28 @@ bnn_status bnn_pack_conv3x3_weights(const void* w_oihw, bnn_dtype dt, int64_t co
                                     uint32_t* packed, int64_t ld_words, float* alpha_out,
                                     bnn_stream_t stream);
 
+/* Engine used by bnn_xnor_gemm and bnn_binary_linear_fused.  Both engines
+ * return identical results (the product is exact integer arithmetic):
+ *   POPCOUNT: XOR + population count on the integer pipes, with carry-save
+ *             compression (any shape).
+ *   TENSOR:   the sign bits expanded to +1/-1 bytes in shared memory and
+ *             multiplied on the tensor cores (tcgen05.mma kind::i8, int32
+ *             accumulators in tensor memory); for large products.
+ *   AUTO:     TENSOR when M >= 128, N >= 128 and K >= 512, else POPCOUNT
+ *             (the default). */
+typedef enum bnn_gemm_engine {
+    BNN_GEMM_ENGINE_AUTO = 0,
+    BNN_GEMM_ENGINE_POPCOUNT = 1,
+    BNN_GEMM_ENGINE_TENSOR = 2
+} bnn_gemm_engine;
+
+/* Selects the GEMM engine for later calls from every thread of the process
+ * (one process-wide setting).  Errors: INVALID_ARG for an unknown engine. */
+bnn_status bnn_set_gemm_engine(int engine);
+
+/* The current process-wide GEMM engine setting. */
+int bnn_get_gemm_engine(void);
+
 /* bnn_xnor_gemm -- C[m, n] = K - 2 * popcount(A[m, :] XOR W[n, :]) for packed
  * A [M, K] and W [N, K]; optionally also the alpha-scaled fp32 product.
  *   Passage: eq. (6) of "Extreme Quantization ..." (XNOR-Net), eq. (1) for

@@ -143,3 +143,11 @@ def test_fold_rejects_bad_arguments():
         bnn.bnn_fold_bn_threshold(-a, a, a, a, a, 1e-5, 16)                 # alpha < 0
     with pytest.raises(bnn.BnnError):
         bnn.bnn_fold_bn_threshold(a, a, a, a, a, 1e-5, 0)                   # K < 1
+
+
+def test_gemm_engine_setting_on_host():
+    prev = bnn.bnn_get_gemm_engine()
+    assert L.bnn_set_gemm_engine(3) == bnn.BNN_ERR_INVALID_ARG
+    assert L.bnn_set_gemm_engine(bnn.BNN_GEMM_ENGINE_TENSOR) == bnn.BNN_OK
+    assert bnn.bnn_get_gemm_engine() == bnn.BNN_GEMM_ENGINE_TENSOR
+    bnn.bnn_set_gemm_engine(prev)

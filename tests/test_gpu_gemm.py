@@ -13,6 +13,16 @@ from gpu_util import assert_affine_close, assert_no_device_error, assert_scaled_
 
 pytestmark = pytest.mark.gpu
 
+ENGINES = [bnn.BNN_GEMM_ENGINE_POPCOUNT, bnn.BNN_GEMM_ENGINE_TENSOR]
+ENGINE_IDS = ["popcount", "tensor"]
+
+
+@pytest.fixture(params=ENGINES, ids=ENGINE_IDS)
+def engine(request):
+    """Run the test body with one GEMM engine forced (both must agree with the oracle)."""
+    with bnn.gemm_engine(request.param):
+        yield request.param
+
 
 def packed_operands(X, W):
     d = dev()
@@ -26,7 +36,7 @@ def packed_operands(X, W):
     return A_p, W_p, alpha
 
 
-def test_tiny_workload():
+def test_tiny_workload(engine):
     """X [64, 1000], W [256, 1000] N(0, 1): K not a multiple of 32."""
     t = workloads.tiny()
     A_p, W_p, alpha = packed_operands(t.X, t.W)
@@ -40,11 +50,12 @@ def test_tiny_workload():
 
 
 RAGGED = [(1, 1, 1), (3, 5, 7), (129, 130, 1000), (200, 300, 65), (128, 128, 4096),
-          (77, 255, 2049), (256, 384, 1024), (130, 129, 8192), (513, 33, 31), (64, 1000, 97)]
+          (77, 255, 2049), (256, 384, 1024), (130, 129, 8192), (513, 33, 31), (64, 1000, 97),
+          (300, 520, 700), (1000, 257, 5000)]
 
 
 @pytest.mark.parametrize("M,N,K", RAGGED)
-def test_ragged_shapes(M, N, K):
+def test_ragged_shapes(M, N, K, engine):
     X = workloads.normal((M, K), 1.0, M * 31 + K)
     W = workloads.normal((N, K), 1.0, N * 37 + K + 1)
     A_p, W_p, alpha = packed_operands(X, W)
@@ -56,7 +67,7 @@ def test_ragged_shapes(M, N, K):
     assert_scaled_close(C_f32, oracle.scaled(s_ref, a_ref))
 
 
-def test_output_strides_and_single_outputs():
+def test_output_strides_and_single_outputs(engine):
     M, N, K = 70, 90, 300
     X = workloads.normal((M, K), 1.0, 1)
     W = workloads.normal((N, K), 1.0, 2)
@@ -72,7 +83,7 @@ def test_output_strides_and_single_outputs():
     assert torch.all(big_f[:, N:] == 5.0)
 
 
-def test_closed_forms_on_gpu():
+def test_closed_forms_on_gpu(engine):
     """W = X gives K on the diagonal, W = -X gives -K, Sylvester-Hadamard rows
     give 0 off the diagonal (eq. (6) identities with no oracle needed)."""
     K = 4096
@@ -88,7 +99,7 @@ def test_closed_forms_on_gpu():
     assert torch.equal(torch.diagonal(C.cpu()), torch.full((256,), -K, dtype=torch.int32))
 
 
-def test_affine_epilogue():
+def test_affine_epilogue(engine):
     M, N, K = 150, 200, 576
     X = workloads.normal((M, K), 1.0, 3)
     W = workloads.normal((N, K), 0.1, 4)
@@ -110,8 +121,9 @@ def test_affine_epilogue():
     assert_scaled_close(out_s, oracle.scaled(s_ref, a_ref))
 
 
-@pytest.mark.parametrize("M,N,K", [(64, 256, 1000), (130, 100, 4096), (1, 33, 64), (257, 513, 97)])
-def test_threshold_pack_epilogue(M, N, K):
+@pytest.mark.parametrize("M,N,K", [(64, 256, 1000), (130, 100, 4096), (1, 33, 64), (257, 513, 97),
+                                   (200, 40, 300), (129, 300, 2000)])
+def test_threshold_pack_epilogue(M, N, K, engine):
     """Folded BatchNorm + sign, re-packed along N: bit-exact against the
     oracle's direct float64 BatchNorm decision, pad bits and pad words 0."""
     X = workloads.normal((M, K), 1.0, M + 11)
@@ -132,7 +144,7 @@ def test_threshold_pack_epilogue(M, N, K):
     assert_no_device_error()
 
 
-def test_square_workload_sampled_rows():
+def test_square_workload_sampled_rows(engine):
     """M = N = K = 8192 (the square workload) on the GPU, checked on 48 sampled
     rows against the oracle (every column of those rows)."""
     sq = workloads.square()
@@ -149,4 +161,32 @@ def test_square_workload_sampled_rows():
     # properties that hold at any size: parity of s and |s| <= K on the whole output
     C = C_i32.cpu()
     assert bool(((C - sq.K) % 2 == 0).all()) and int(C.abs().max()) <= sq.K
+    assert_no_device_error()
+
+
+def test_engine_setting_roundtrip():
+    prev = bnn.bnn_get_gemm_engine()
+    for e in (bnn.BNN_GEMM_ENGINE_TENSOR, bnn.BNN_GEMM_ENGINE_POPCOUNT, bnn.BNN_GEMM_ENGINE_AUTO):
+        bnn.bnn_set_gemm_engine(e)
+        assert bnn.bnn_get_gemm_engine() == e
+    with pytest.raises(bnn.BnnError):
+        bnn.bnn_set_gemm_engine(7)
+    bnn.bnn_set_gemm_engine(prev)
+
+
+def test_engines_agree_bit_for_bit():
+    """Both engines on the same operands: identical int32 and identical fp32."""
+    M, N, K = 384, 512, 3000
+    X = workloads.normal((M, K), 1.0, 77)
+    W = workloads.normal((N, K), 1.0, 78)
+    A_p, W_p, alpha = packed_operands(X, W)
+    outs = []
+    for e in ENGINES:
+        with bnn.gemm_engine(e):
+            Ci = torch.empty(M, N, dtype=torch.int32, device=dev())
+            Cf = torch.empty(M, N, dtype=torch.float32, device=dev())
+            bnn.bnn_xnor_gemm(A_p, W_p, K, alpha, Ci, Cf)
+            outs.append((Ci.cpu(), Cf.cpu()))
+    assert torch.equal(outs[0][0], outs[1][0])
+    assert torch.equal(outs[0][1], outs[1][1])
     assert_no_device_error()

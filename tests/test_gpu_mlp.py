@@ -13,6 +13,12 @@ from gpu_util import assert_no_device_error, assert_scaled_close, dev, u32
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(params=[bnn.BNN_GEMM_ENGINE_POPCOUNT, bnn.BNN_GEMM_ENGINE_TENSOR], ids=["popcount", "tensor"])
+def engine(request):
+    with bnn.gemm_engine(request.param):
+        yield request.param
+
+
 def gpu_mlp(m: workloads.Mlp):
     """Pack input and weights, fold BN on the host once, run the layers."""
     d = dev()
@@ -48,7 +54,7 @@ def oracle_mlp(m: workloads.Mlp, rows=None):
 
 
 @pytest.mark.parametrize("batch,width", [(64, 256), (100, 300), (33, 4096)])
-def test_small_mlp_all_rows(batch, width):
+def test_small_mlp_all_rows(batch, width, engine):
     m = workloads.mlp(batch=batch, width=width)
     acts, logits = gpu_mlp(m)
     acts_ref, logits_ref = oracle_mlp(m)
@@ -58,7 +64,7 @@ def test_small_mlp_all_rows(batch, width):
     assert_no_device_error()
 
 
-def test_mlp_workload_sampled_rows():
+def test_mlp_workload_sampled_rows(engine):
     """Batch 4096, width 4096, 4 layers; rows are independent, so 24 sampled
     rows are checked through all layers against the oracle."""
     m = workloads.mlp()

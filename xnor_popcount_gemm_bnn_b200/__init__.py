@@ -36,12 +36,16 @@ BNN_OUT_THRESHOLD_PACK = 8
 
 BNN_GEMV_WEIGHTS_STATIC = 1
 
+BNN_GEMM_ENGINE_AUTO = 0
+BNN_GEMM_ENGINE_POPCOUNT = 1
+BNN_GEMM_ENGINE_TENSOR = 2
+
 # Every symbol declared in include/bnn.h.
 EXPORTS = (
     "bnn_packed_ld_words", "bnn_conv3x3_ld_words", "bnn_status_string", "bnn_device_error",
     "bnn_pack_sign", "bnn_pack_sign_nchw", "bnn_pack_conv3x3_weights", "bnn_xnor_gemm",
     "bnn_xnor_gemv", "bnn_xnor_gemv_ex", "bnn_binary_linear_fused", "bnn_binary_conv3x3_fused",
-    "bnn_fold_bn_threshold",
+    "bnn_fold_bn_threshold", "bnn_set_gemm_engine", "bnn_get_gemm_engine",
 )
 
 
@@ -79,6 +83,8 @@ def _load() -> ctypes.CDLL:
         "bnn_binary_conv3x3_fused": (i32, [p, i64, i64, i64, i64, p, i64, i64, i64, i64,
                                            ctypes.POINTER(bnn_epilogue), p, p]),
         "bnn_fold_bn_threshold": (i32, [p, p, p, p, p, ctypes.c_double, i64, i64, p, p]),
+        "bnn_set_gemm_engine": (i32, [ctypes.c_int]),
+        "bnn_get_gemm_engine": (ctypes.c_int, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -134,6 +140,29 @@ def bnn_conv3x3_ld_words(cin: int) -> int:
 
 def bnn_status_string(status: int) -> str:
     return _lib.bnn_status_string(int(status)).decode()
+
+
+def bnn_set_gemm_engine(engine: int) -> None:
+    _check("bnn_set_gemm_engine", _lib.bnn_set_gemm_engine(int(engine)))
+
+
+def bnn_get_gemm_engine() -> int:
+    return int(_lib.bnn_get_gemm_engine())
+
+
+class gemm_engine:
+    """Context manager: run the enclosed calls with one GEMM engine."""
+
+    def __init__(self, engine: int):
+        self.engine = int(engine)
+
+    def __enter__(self):
+        self.prev = bnn_get_gemm_engine()
+        bnn_set_gemm_engine(self.engine)
+        return self
+
+    def __exit__(self, *exc):
+        bnn_set_gemm_engine(self.prev)
 
 
 def bnn_device_error() -> int:

@@ -8,12 +8,14 @@
 #include <climits>
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include "bnn.h"
 #include "common.cuh"
 #include "conv.cuh"
 #include "gemm_popc.cuh"
+#include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "pack.cuh"
 
@@ -47,16 +49,18 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // 2-D map over a packed matrix: inner dimension = kw words, outer = rows,
-// box 32 words x 128 rows, 128-byte swizzle, zero fill out of range.
-bool encode_packed_map(CUtensorMap* map, const uint32_t* base, int64_t kw, int64_t rows, int64_t ld) {
+// box 32 words x box_rows rows, 128-byte swizzle, zero fill out of range.
+bool encode_packed_map(CUtensorMap* map, const uint32_t* base, int64_t kw, int64_t rows, int64_t ld,
+                       int box_rows, int box_words = bnn::gemm::BKW,
+                       CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     auto enc = tensor_map_encoder();
     if (enc == nullptr) return false;
     cuuint64_t dims[2] = {(cuuint64_t)kw, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)ld * 4u};
-    cuuint32_t box[2] = {(cuuint32_t)bnn::gemm::BKW, (cuuint32_t)bnn::gemm::BM};
+    cuuint32_t box[2] = {(cuuint32_t)box_words, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(base), dims, strides,
-                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -69,11 +73,33 @@ bool gemm_smem_configured() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
     if (dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return true;
-    if (cudaFuncSetAttribute(bnn::xnor_gemm_popc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             bnn::gemm::SMEM_BYTES) != cudaSuccess)
+    if (cudaFuncSetAttribute(bnn::xnor_gemm_popc_kernel<bnn::gemm::TN, bnn::gemm::CSA>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, bnn::gemm::SMEM_BYTES) != cudaSuccess)
         return false;
     if (dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
     return true;
+}
+
+// Per-device one-time opt-in to the tensor-core GEMM's shared memory.
+bool gemm_tc_smem_configured() {
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> done[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+    if (dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return true;
+    if (cudaFuncSetAttribute(bnn::xnor_gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bnn::tc::SMEM_BYTES) != cudaSuccess)
+        return false;
+    if (dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
+    return true;
+}
+
+std::atomic<int> g_gemm_engine{BNN_GEMM_ENGINE_AUTO};
+
+int sm_count() {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
 }
 
 bnn_status check_packed_operand(const uint32_t* p, int64_t ld, int64_t kw) {
@@ -88,16 +114,48 @@ bnn_status launch_gemm(const uint32_t* A, int64_t lda, const uint32_t* W, int64_
     using namespace bnn::gemm;
     const int64_t kw = packed_ld_words(K);
     CUtensorMap tmA, tmW;
-    if (!encode_packed_map(&tmA, A, kw, M, lda) || !encode_packed_map(&tmW, W, kw, N, ldw))
+    if (!encode_packed_map(&tmA, A, kw, M, lda, BM) || !encode_packed_map(&tmW, W, kw, N, ldw, BN))
         return BNN_ERR_CUDA;
     const int64_t tiles_n = ceil_div(N, BN);
     const int64_t tiles = ceil_div(M, BM) * tiles_n;
     if (tiles > INT_MAX) return BNN_ERR_INVALID_ARG;
     if (!gemm_smem_configured())
         return BNN_ERR_CUDA;
-    bnn::xnor_gemm_popc_kernel<<<(unsigned)tiles, THREADS, SMEM_BYTES, stream>>>(
-        tmA, tmW, (int)M, (int)N, (int)K, (int)kw, (int)tiles_n, ep);
+    bnn::GemmEpilogue e = ep;
+    e.bits_words = packed_ld_words(N);
+    bnn::xnor_gemm_popc_kernel<TN, CSA><<<(unsigned)tiles, THREADS, SMEM_BYTES, stream>>>(
+        tmA, tmW, (int)M, (int)N, (int)K, (int)kw, (int)tiles_n, e);
     return launch_status();
+}
+
+bnn_status launch_gemm_tc(const uint32_t* A, int64_t lda, const uint32_t* W, int64_t ldw, int64_t M, int64_t N,
+                          int64_t K, const bnn::GemmEpilogue& ep, cudaStream_t stream) {
+    using namespace bnn::tc;
+    const int64_t kw = packed_ld_words(K);
+    CUtensorMap tmA, tmW;
+    if (!encode_packed_map(&tmA, A, kw, M, lda, BM, BKW, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_packed_map(&tmW, W, kw, N, ldw, BN, BKW, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return BNN_ERR_CUDA;
+    const int64_t tiles_m = ceil_div(M, BM), tiles_n = ceil_div(N, BN);
+    if (tiles_m * tiles_n > INT_MAX) return BNN_ERR_INVALID_ARG;
+    if (!gemm_tc_smem_configured()) return BNN_ERR_CUDA;
+    const int64_t grid = std::min<int64_t>(tiles_m * tiles_n, sm_count());
+    bnn::GemmEpilogue e = ep;
+    e.bits_words = packed_ld_words(N);
+    bnn::xnor_gemm_tc_kernel<<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(
+        tmA, tmW, (int)M, (int)N, (int)K, (int)kw, (int)tiles_m, (int)tiles_n, e);
+    return launch_status();
+}
+
+// Engine for one product: the tensor cores once the tile is reasonably
+// filled (M >= 128, N >= 128, K >= 512); the integer pipes otherwise.
+bnn_status dispatch_gemm(const uint32_t* A, int64_t lda, const uint32_t* W, int64_t ldw, int64_t M, int64_t N,
+                         int64_t K, const bnn::GemmEpilogue& ep, cudaStream_t stream) {
+    int engine = g_gemm_engine.load(std::memory_order_relaxed);
+    if (engine == BNN_GEMM_ENGINE_AUTO)
+        engine = (M >= 128 && N >= 128 && K >= 512) ? BNN_GEMM_ENGINE_TENSOR : BNN_GEMM_ENGINE_POPCOUNT;
+    if (engine == BNN_GEMM_ENGINE_TENSOR) return launch_gemm_tc(A, lda, W, ldw, M, N, K, ep, stream);
+    return launch_gemm(A, lda, W, ldw, M, N, K, ep, stream);
 }
 
 bnn_status check_gemm_dims(int64_t M, int64_t N, int64_t K) {
@@ -131,17 +189,26 @@ bnn_status launch_gemv_t(const uint32_t* W, int64_t ldw, const XT* x, int64_t N,
 
     cudaError_t e = cudaSuccess;
     const int iN = (int)N, iK = (int)K, ikw = (int)kw;
-#define BNN_GEMV_CASE(L)                                                                           \
-    case L: {                                                                                      \
-        auto kern = bnn::xnor_gemv_kernel<XT, L>;                                                  \
-        if (smem > 48 * 1024 &&                                                                    \
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=  \
-                cudaSuccess)                                                                       \
-            return BNN_ERR_CUDA;                                                                   \
-        e = cudaLaunchKernelEx(&cfg, kern, W, ldw, x, iN, iK, ikw, alpha, y_i32, y_f32,            \
-                               weights_static);                                                    \
-        break;                                                                                     \
-    }
+    const bool single = nchunks <= lpr;
+    if ((int64_t)blocks * rows_per_block > (int64_t)INT_MAX) return BNN_ERR_INVALID_ARG;
+    auto launch = [&](auto kern) -> bnn_status {
+        if (smem > 48 * 1024 &&
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return BNN_ERR_CUDA;
+        e = cudaLaunchKernelEx(&cfg, kern, W, ldw, x, iN, iK, ikw, alpha, y_i32, y_f32);
+        return BNN_OK;
+    };
+    bnn_status st = BNN_OK;
+    const bool vec = aligned(x, 16);
+#define BNN_GEMV_PICK(L, S, P)                                                                      \
+    (vec ? launch(bnn::xnor_gemv_kernel<XT, L, S, P, true>) : launch(bnn::xnor_gemv_kernel<XT, L, S, P, false>))
+#define BNN_GEMV_CASE(L)                                                                            \
+    case L:                                                                                         \
+        if (single)                                                                                 \
+            st = weights_static ? BNN_GEMV_PICK(L, true, true) : BNN_GEMV_PICK(L, true, false);     \
+        else                                                                                        \
+            st = weights_static ? BNN_GEMV_PICK(L, false, true) : BNN_GEMV_PICK(L, false, false);   \
+        break;
     switch (lpr) {
         BNN_GEMV_CASE(1)
         BNN_GEMV_CASE(2)
@@ -151,7 +218,9 @@ bnn_status launch_gemv_t(const uint32_t* W, int64_t ldw, const XT* x, int64_t N,
         BNN_GEMV_CASE(32)
         default: return BNN_ERR_UNSUPPORTED;
     }
+    if (st != BNN_OK) return st;
 #undef BNN_GEMV_CASE
+#undef BNN_GEMV_PICK
     if (e != cudaSuccess) return BNN_ERR_CUDA;
     return launch_status();
 }
@@ -181,6 +250,15 @@ bnn_status gemv_impl(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_
 }  // namespace
 
 extern "C" {
+
+bnn_status bnn_set_gemm_engine(int engine) {
+    if (engine != BNN_GEMM_ENGINE_AUTO && engine != BNN_GEMM_ENGINE_POPCOUNT && engine != BNN_GEMM_ENGINE_TENSOR)
+        return BNN_ERR_INVALID_ARG;
+    g_gemm_engine.store(engine, std::memory_order_relaxed);
+    return BNN_OK;
+}
+
+int bnn_get_gemm_engine(void) { return g_gemm_engine.load(std::memory_order_relaxed); }
 
 int64_t bnn_packed_ld_words(int64_t K) { return K < 1 ? -1 : packed_ld_words(K); }
 
@@ -301,7 +379,7 @@ bnn_status bnn_xnor_gemm(const uint32_t* A, int64_t lda, const uint32_t* W, int6
     ep.c_f32 = C_f32;
     ep.ldf = ldf;
     ep.alpha = alpha;
-    return launch_gemm(A, lda, W, ldw, M, N, K, ep, as_cuda(stream));
+    return dispatch_gemm(A, lda, W, ldw, M, N, K, ep, as_cuda(stream));
 }
 
 bnn_status bnn_xnor_gemv(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt, int64_t N, int64_t K,
@@ -360,7 +438,7 @@ bnn_status bnn_binary_linear_fused(const uint32_t* A, int64_t lda, const uint32_
             return BNN_ERR_INVALID_ARG;
     }
     if (M == 0 || N == 0) return BNN_OK;
-    return launch_gemm(A, lda, W, ldw, M, N, K, ep, as_cuda(stream));
+    return dispatch_gemm(A, lda, W, ldw, M, N, K, ep, as_cuda(stream));
 }
 
 bnn_status bnn_binary_conv3x3_fused(const uint32_t* X_nhwc_bits, int64_t n, int64_t c, int64_t h, int64_t w,
@@ -389,12 +467,20 @@ bnn_status bnn_binary_conv3x3_fused(const uint32_t* X_nhwc_bits, int64_t n, int6
     if (!aligned(X_nhwc_bits, 4) || !aligned(W_packed, 16) || !aligned(out_nchw, 4)) return BNN_ERR_ALIGNMENT;
     if (cw > 4) return BNN_ERR_UNSUPPORTED;
     const int64_t kwp = (9 * cw + 3) / 4 * 4;
-    const size_t smem = (size_t)cout * kwp * 4;
+    const size_t smem = (size_t)cout * kwp * 4 + (size_t)cout * 3 * 4;   // filters + alpha/gamma/beta
     if (smem > 200 * 1024) return BNN_ERR_UNSUPPORTED;
     if (n == 0 || cout == 0) return BNN_OK;
     const int64_t npix = n * oh * ow;
-    const int64_t blocks = ceil_div(npix, (int64_t)bnn::conv::WARPS * 32 * bnn::conv::P);
-    if (blocks > INT_MAX) return BNN_ERR_INVALID_ARG;
+    const int64_t tasks = ceil_div(npix, (int64_t)32) * ceil_div(cout, (int64_t)bnn::conv::FB);
+    int sms = 148;
+    {
+        int dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    // A whole number of CTAs per SM (the kernel strides over warp tasks), no
+    // more CTAs than there are tasks.
+    const int64_t blocks = std::max<int64_t>(
+        1, std::min<int64_t>(ceil_div(tasks, bnn::conv::WARPS), (int64_t)sms * bnn::conv::CTAS_PER_SM));
     bnn::ConvEpilogue ep{epi->mode, epi->alpha, epi->gamma, epi->beta, out_nchw};
     cudaStream_t s = as_cuda(stream);
 #define BNN_CONV_CASE(CWV)                                                                                 \

@@ -1,0 +1,393 @@
+// Packed binary GEMM on the 5th-generation tensor cores (tcgen05, kind::i8).
+//
+// Same product as gemm_popc.cuh -- s[m, n] = sum_k a_mk * w_nk over +1/-1
+// values ("Extreme Quantization: Binary, Ternary & 1-bit LLMs", eq. (1), (4)
+// and (6)) -- computed by expanding the packed sign bits to signed bytes
+// (bit 0 -> +1 = 0x01, bit 1 -> -1 = 0xFF) in shared memory and multiplying
+// them with tcgen05.mma kind::i8 into int32 accumulators in tensor memory.
+// Every product is +1 or -1 and the accumulation is exact in int32, so the
+// result is bit-identical to K - 2 * popcount(A XOR W).  Pad positions (bits
+// past K inside the packed rows, and zero-filled words past the row end) are
+// 0 bits in both operands, i.e. (+1)(+1) = +1 each; the epilogue subtracts
+// their count, (K rounded up to a whole stage) - K.
+//
+// Design (sm_100a, one persistent CTA per SM, 14 warps):
+//  * warp 0   : TMA producer.  Packed tiles (128 A rows x 4 words, 256 W rows
+//               x 4 words = 128 binary elements of K) into an 8-stage ring.
+//  * warps 2-9: unpack.  Each packed word becomes 32 signed bytes in the
+//               K-major 128B-swizzled layout the tensor core reads (chunk c of
+//               row r at (c ^ (r & 7)) * 16); four ops per 4 bytes (PRMT picks
+//               a nibble, IMAD spreads its bits into bytes, LOP3 masks, IMAD
+//               maps {0,1} to {+1,-1}).  fence.proxy.async, then an mbarrier
+//               arrive hands the stage to the MMA warp.
+//  * warp 1   : allocates 512 TMEM columns (two 128 x 256 int32 accumulators);
+//               one thread issues 4 tcgen05.mma (M=128, N=256, K=32) per stage
+//               and commits them to the stage's "empty" barrier, and to the
+//               accumulator's "full" barrier after the last stage of a tile.
+//  * warps 10-13: epilogue.  Warp q reads TMEM lanes 32q..32q+31 (one output
+//               row per thread) 32 columns at a time with tcgen05.ld, releases
+//               the accumulator, and writes int32 / alpha*s / affine outputs or
+//               the folded-BatchNorm sign bits (32 columns = one packed word,
+//               all in one thread).  Double buffering lets the epilogue of tile
+//               i overlap the MMAs of tile i+1.
+//  * Every mbarrier wait is bounded (about 1 s): on time-out the CTA records
+//    BNN_ERR_DEVICE_TIMEOUT, the other roles stop at their next wait, the MMA
+//    thread waits (bounded) for its last MMAs, and TMEM is freed before exit.
+#pragma once
+
+#include "common.cuh"
+#include "gemm_popc.cuh"   // GemmEpilogue
+
+namespace bnn {
+namespace tc {
+constexpr int BM = 128;                    // tile rows  = TMEM lanes = UMMA M
+constexpr int BN = 256;                    // tile cols  = UMMA N
+constexpr int BKE = 128;                   // binary elements of K per stage (4 packed words)
+constexpr int BKW = BKE / 32;
+constexpr int UMMA_K = 32;                 // int8 K per tcgen05.mma
+constexpr int PSTAGES = 8;                 // packed ring
+constexpr int USTAGES = 3;                 // unpacked (int8) ring
+constexpr int P_A_BYTES = BM * BKW * 4;    // 2 KiB
+constexpr int P_B_BYTES = BN * BKW * 4;    // 4 KiB
+constexpr int P_STAGE = P_A_BYTES + P_B_BYTES;
+constexpr int U_A_BYTES = BM * BKE;        // 16 KiB
+constexpr int U_B_BYTES = BN * BKE;        // 32 KiB
+constexpr int U_STAGE = U_A_BYTES + U_B_BYTES;
+constexpr int UNPACK_WARPS = 8;
+constexpr int EPI_WARPS = 4;
+constexpr int WARP_PRODUCER = 0, WARP_MMA = 1, WARP_UNPACK0 = 2, WARP_EPI0 = WARP_UNPACK0 + UNPACK_WARPS;
+constexpr int THREADS = (WARP_EPI0 + EPI_WARPS) * 32;   // 448
+constexpr int TMEM_COLS = 2 * BN;          // two accumulators
+constexpr int NUM_BARS = 2 * PSTAGES + 2 * USTAGES + 2 * 2 + 1;
+constexpr int SMEM_BYTES = USTAGES * U_STAGE + PSTAGES * P_STAGE + NUM_BARS * 8 + 16 + 1024;
+// kind::i8 instruction descriptor: D s32 (bits 4-5 = 2), A s8 (bits 7-9 = 1),
+// B s8 (bits 10-12 = 1), both K-major, N >> 3 at bits 17-22, M >> 4 at 24-28.
+constexpr uint32_t IDESC = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                           ((uint32_t)(BM >> 4) << 24);
+}  // namespace tc
+
+// Shared-memory matrix descriptor for a K-major, 128B-swizzled operand tile
+// whose rows are 128 bytes (8-row groups 1024 bytes apart): start address,
+// leading offset 16 B (unused for this layout), stride offset 1024 B,
+// descriptor version 1, layout type 2 (SWIZZLE_128B).
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr) {
+    return (uint64_t)((smem_addr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
+           ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(tc::IDESC), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on `bar` once every tcgen05.mma issued so far by this thread is done.
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Bounded wait that also gives up as soon as another role of the CTA aborted.
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    while (true) {
+        #pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+            flag_device_error(BNN_ERR_DEVICE_TIMEOUT);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+// 4 signed bytes (+1 / -1) from the 4 low bits of n (bit j -> byte j).
+__device__ __forceinline__ uint32_t pm1_bytes(uint32_t n) {
+    const uint32_t t = (n * 0x00204081u) & 0x01010101u;   // bit j -> bit 8j (no carries for n < 16)
+    return t * 0xFEu + 0x01010101u;                        // 0x01 -> 0xFF (-1), 0x00 -> 0x01 (+1)
+}
+
+__global__ void __launch_bounds__(tc::THREADS, 1)
+xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW, int M, int N,
+                    int K, int kw, int tiles_m, int tiles_n, GemmEpilogue ep) {
+    using namespace tc;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* uring = smem;                                   // USTAGES x (A 16 KiB | W 32 KiB)
+    uint8_t* pring = smem + USTAGES * U_STAGE;               // PSTAGES x (A 2 KiB | W 4 KiB)
+    uint64_t* bars = reinterpret_cast<uint64_t*>(pring + PSTAGES * P_STAGE);
+    uint64_t* pfull = bars;
+    uint64_t* pempty = pfull + PSTAGES;
+    uint64_t* ufull = pempty + PSTAGES;
+    uint64_t* uempty = ufull + USTAGES;
+    uint64_t* afull = uempty + USTAGES;
+    uint64_t* aempty = afull + 2;
+    uint64_t* drain = aempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int nk = kw / BKW;                                  // kw is a multiple of 4
+    const int tiles = tiles_m * tiles_n;
+
+    if (threadIdx.x == 0) {
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmW);
+        for (int s = 0; s < PSTAGES; ++s) {
+            mbar_init(&pfull[s], 1);
+            mbar_init(&pempty[s], UNPACK_WARPS);
+        }
+        for (int s = 0; s < USTAGES; ++s) {
+            mbar_init(&ufull[s], UNPACK_WARPS);
+            mbar_init(&uempty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&afull[b], 1);
+            mbar_init(&aempty[b], EPI_WARPS);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == WARP_MMA) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == WARP_PRODUCER) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0) {
+            uint32_t g = 0, issued = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+                const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
+                for (int ks = 0; ks < nk; ++ks, ++g) {
+                    const uint32_t s = g % PSTAGES;
+                    if (g >= PSTAGES && !tc_wait(&pempty[s], ((g / PSTAGES) - 1) & 1, abort_flag)) { ok = false; break; }
+                    uint8_t* dst = pring + s * P_STAGE;
+                    mbar_arrive_expect_tx(&pfull[s], P_STAGE);
+                    tma_load_2d(dst, &tmA, ks * BKW, m0, &pfull[s]);
+                    tma_load_2d(dst + P_A_BYTES, &tmW, ks * BKW, n0, &pfull[s]);
+                    ++issued;
+                }
+            }
+            // Let the copies still in flight land before the CTA can retire
+            // (also after an abort).
+            for (uint32_t q = issued > PSTAGES ? issued - PSTAGES : 0; q < issued; ++q)
+                if (!mbar_wait_bounded(&pfull[q % PSTAGES], (q / PSTAGES) & 1)) break;
+        }
+    } else if (warp == WARP_MMA) {
+        // ------------------------------ MMA issuer ------------------------------
+        if (lane == 0) {
+            uint32_t g = 0;
+            int lt = 0;
+            bool ok = true;
+            const uint32_t ubase = smem_u32(uring);
+            for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++lt) {
+                const int b = lt & 1;
+                if (lt >= 2 && !tc_wait(&aempty[b], ((lt >> 1) - 1) & 1, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(b * BN);
+                for (int ks = 0; ks < nk; ++ks, ++g) {
+                    const uint32_t s = g % USTAGES;
+                    if (!tc_wait(&ufull[s], (g / USTAGES) & 1, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_addr = ubase + s * U_STAGE;
+                    const uint32_t b_addr = a_addr + U_A_BYTES;
+                    #pragma unroll
+                    for (int kk = 0; kk < BKE / UMMA_K; ++kk) {
+                        // Advancing the start address by 32 B steps through K inside the swizzle atom.
+                        mma_i8(d_tmem, umma_desc_sw128(a_addr + kk * UMMA_K), umma_desc_sw128(b_addr + kk * UMMA_K),
+                               (ks | kk) != 0 ? 1u : 0u);
+                    }
+                    mma_commit(&uempty[s]);
+                }
+                if (ok) mma_commit(&afull[b]);
+            }
+            // Every MMA issued above is complete once this arrives (waited for
+            // even after an abort: TMEM is freed only after the last MMA).
+            mma_commit(drain);
+            mbar_wait_bounded(drain, 0);
+        }
+        __syncwarp();
+    } else if (warp < WARP_EPI0) {
+        // ------------------------------ unpack warps ------------------------------
+        const int u = threadIdx.x - WARP_UNPACK0 * 32;               // 0..255
+        const uint32_t* pw = reinterpret_cast<const uint32_t*>(pring);
+        uint32_t g = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+            for (int ks = 0; ks < nk; ++ks, ++g) {
+                const uint32_t ps = g % PSTAGES, us = g % USTAGES;
+                bool w1 = tc_wait(&pfull[ps], (g / PSTAGES) & 1, abort_flag);
+                bool w2 = w1 && (g < USTAGES || tc_wait(&uempty[us], ((g / USTAGES) - 1) & 1, abort_flag));
+                if (!__all_sync(0xffffffffu, w1 && w2)) { ok = false; break; }
+                const uint32_t* src = pw + ps * (P_STAGE / 4);
+                uint8_t* dstA = uring + us * U_STAGE;
+                uint8_t* dstB = dstA + U_A_BYTES;
+                uint32_t words[6];
+                #pragma unroll
+                for (int i = 0; i < 6; ++i) words[i] = src[u + 256 * i];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&pempty[ps]);             // packed stage consumed
+                #pragma unroll
+                for (int i = 0; i < 6; ++i) {
+                    const int v = u + 256 * i;                        // word index: A rows first, then W rows
+                    const int r = v < BM * BKW ? (v >> 2) : ((v - BM * BKW) >> 2);
+                    const int q = v & 3;
+                    uint8_t* row = (v < BM * BKW ? dstA : dstB) + r * 128;
+                    const uint32_t w = words[i];
+                    const uint32_t lo = w & 0x0F0F0F0Fu;              // nibbles 0, 2, 4, 6 (one per byte)
+                    const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;       // nibbles 1, 3, 5, 7
+                    uint4 c0, c1;
+                    c0.x = pm1_bytes(__byte_perm(lo, 0u, 0x4440u));
+                    c0.y = pm1_bytes(__byte_perm(hi, 0u, 0x4440u));
+                    c0.z = pm1_bytes(__byte_perm(lo, 0u, 0x4441u));
+                    c0.w = pm1_bytes(__byte_perm(hi, 0u, 0x4441u));
+                    c1.x = pm1_bytes(__byte_perm(lo, 0u, 0x4442u));
+                    c1.y = pm1_bytes(__byte_perm(hi, 0u, 0x4442u));
+                    c1.z = pm1_bytes(__byte_perm(lo, 0u, 0x4443u));
+                    c1.w = pm1_bytes(__byte_perm(hi, 0u, 0x4443u));
+                    const int sw = r & 7;
+                    *reinterpret_cast<uint4*>(row + (((2 * q) ^ sw) << 4)) = c0;
+                    *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ sw) << 4)) = c1;
+                }
+                fence_proxy_async_shared();                           // make the bytes visible to the tensor core
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ufull[us]);
+            }
+        }
+    } else {
+        // ------------------------------ epilogue warps ------------------------------
+        const int quad = warp & 3;                                    // TMEM lanes 32*quad .. 32*quad + 31
+        const int pad = nk * BKE - K;                                 // (+1)(+1) pad positions per output
+        int lt = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++lt) {
+            const int b = lt & 1;
+            if (!__all_sync(0xffffffffu, tc_wait(&afull[b], (lt >> 1) & 1, abort_flag))) break;
+            tc_fence_after();
+            const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
+            const int m = m0 + 32 * quad + lane;
+            #pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * BN + 32 * c), r);
+                tmem_ld_wait();
+                if (c == BN / 32 - 1) {
+                    // Whole accumulator read: hand it back to the MMA warp.
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&aempty[b]);
+                }
+                const int nb = n0 + 32 * c;
+                if (nb >= N) {
+                    // Past the last column: a packed output still has pad words here.
+                    if (ep.c_bits != nullptr && m < M && nb / 32 < ep.bits_words)
+                        ep.c_bits[(int64_t)m * ep.ldb + nb / 32] = 0u;
+                    continue;
+                }
+                const bool full_chunk = nb + 32 <= N;
+                if (ep.c_bits != nullptr) {
+                    uint32_t word = 0;
+                    #pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int n = nb + j;
+                        const int32_t d = (K - ((int32_t)r[j] - pad)) / 2;   // popcount of the XOR
+                        bool bit = false;
+                        if (n < N) {
+                            const int md = ep.thresh_mode[n];
+                            const int th = ep.thresh[n];
+                            bit = md == 0 ? (d > th) : (md == 1 ? (d < th) : false);
+                        }
+                        word |= (bit ? 1u : 0u) << j;
+                    }
+                    if (m < M && nb / 32 < ep.bits_words) ep.c_bits[(int64_t)m * ep.ldb + nb / 32] = word;
+                }
+                if (m < M && ep.c_i32 != nullptr) {
+                    int32_t* dst = ep.c_i32 + (int64_t)m * ep.ldc + nb;
+                    if (full_chunk && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0)) {
+                        #pragma unroll
+                        for (int j = 0; j < 32; j += 4)
+                            *reinterpret_cast<int4*>(dst + j) =
+                                make_int4((int32_t)r[j] - pad, (int32_t)r[j + 1] - pad, (int32_t)r[j + 2] - pad,
+                                          (int32_t)r[j + 3] - pad);
+                    } else {
+                        for (int j = 0; j < 32 && nb + j < N; ++j) dst[j] = (int32_t)r[j] - pad;
+                    }
+                }
+                if (m < M && ep.c_f32 != nullptr) {
+                    float* dst = ep.c_f32 + (int64_t)m * ep.ldf + nb;
+                    float y[32];
+                    #pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int n = min(nb + j, N - 1);
+                        float v = __ldg(ep.alpha + n) * (float)((int32_t)r[j] - pad);
+                        if (ep.gamma != nullptr) v = fmaf(__ldg(ep.gamma + n), v, __ldg(ep.beta + n));
+                        y[j] = v;
+                    }
+                    if (full_chunk && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0)) {
+                        #pragma unroll
+                        for (int j = 0; j < 32; j += 4)
+                            *reinterpret_cast<float4*>(dst + j) = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
+                    } else {
+                        for (int j = 0; j < 32 && nb + j < N; ++j) dst[j] = y[j];
+                    }
+                }
+            }
+            // The last column tile also zeroes pad words of the packed output that no tile covers.
+            if (ep.c_bits != nullptr && (t % tiles_n) == tiles_n - 1 && m < M) {
+                for (int64_t wd = (int64_t)(n0 + BN) / 32; wd < ep.bits_words; ++wd)
+                    ep.c_bits[(int64_t)m * ep.ldb + wd] = 0u;
+            }
+        }
+    }
+
+    // ------------------------------ teardown ------------------------------
+    tc_fence_before();
+    __syncthreads();
+    if (warp == WARP_MMA) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+}  // namespace bnn

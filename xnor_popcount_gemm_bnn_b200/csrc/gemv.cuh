@@ -12,8 +12,7 @@
 //  * The packed rows are read as 16-byte non-allocating vectors, LPR lanes per
 //    row (LPR = 32 when a row is >= 512 bytes, i.e. K >= 4096), so a warp-wide
 //    load is one contiguous row segment.  Each warp issues the loads of its U
-//    row groups before using any of them, keeping U * 512 bytes per warp in
-//    flight.
+//    row groups before using any of them; all of W is in flight at once.
 //  * Row sums: redux.sync (one instruction) when LPR = 32, else a shuffle tree.
 //  * Launched with programmatic dependent launch: the grid may start while
 //    the previous kernel on the stream finishes, and waits for it
@@ -27,29 +26,96 @@
 
 namespace bnn {
 namespace gemv {
-constexpr int THREADS = 256;
+// 512 threads x 2 row groups per warp (32 rows of K = 4096 per CTA): the
+// shape with the shortest step time in back-to-back dependent launches, where
+// each grid waits for the previous one (measured against 256 x 4, 256 x 2,
+// 512 x 1..4, 1024 x 1..2).
+constexpr int THREADS = 512;
 constexpr int WARPS = THREADS / 32;
-constexpr int U = 4;   // row groups per warp
+constexpr int U = 2;   // row groups per warp
+
 }  // namespace gemv
 
-template <typename XT, int LPR>
+// Packs the real vector x (K elements, zero past K up to kw words) into xs[]
+// (shared memory), one bit per element, bit 1 for x < 0.  VEC: x is 16-byte
+// aligned, so each thread loads whole 16-byte vectors (8 bf16 or 4 fp32);
+// all of a thread's loads are issued before any bit is assembled, and the
+// E bits of a vector are OR-combined across the 32/E lanes of a word.
+template <typename XT, bool VEC>
+__device__ __forceinline__ void gemv_pack_x(const XT* __restrict__ x, int K, int kw, uint32_t* xs) {
+    using namespace gemv;
+    const int lane = threadIdx.x & 31;
+    if constexpr (VEC) {
+        constexpr int E = 16 / (int)sizeof(XT);       // elements per vector
+        constexpr int G = 32 / E;                     // lanes per packed word
+        constexpr int VB = 2;                         // vectors per thread per batch
+        const int nvec = kw * 32 / E;                 // vectors covering the padded row
+        for (int v0 = 0; v0 < nvec; v0 += THREADS * VB) {
+            float e[VB][E];
+            #pragma unroll
+            for (int b = 0; b < VB; ++b) {
+                const int vi = v0 + b * THREADS + (int)threadIdx.x;
+                const int base = vi * E;
+                if (base + E <= K) {
+                    const uint4 q = *reinterpret_cast<const uint4*>(x + base);
+                    const XT* el = reinterpret_cast<const XT*>(&q);
+                    #pragma unroll
+                    for (int i = 0; i < E; ++i) e[b][i] = to_float(el[i]);
+                } else {
+                    #pragma unroll
+                    for (int i = 0; i < E; ++i) e[b][i] = (vi < nvec && base + i < K) ? to_float(x[base + i]) : 0.0f;
+                }
+            }
+            #pragma unroll
+            for (int b = 0; b < VB; ++b) {
+                const int vi = v0 + b * THREADS + (int)threadIdx.x;
+                uint32_t bits = 0;
+                #pragma unroll
+                for (int i = 0; i < E; ++i) bits |= neg_bit(e[b][i]) << i;
+                bits <<= E * (lane % G);
+                #pragma unroll
+                for (int off = 1; off < G; off <<= 1) bits |= __shfl_xor_sync(0xffffffffu, bits, off);
+                if ((lane % G) == 0 && vi < nvec) xs[vi / G] = bits;
+            }
+        }
+    } else {
+        constexpr int XB = 8;                         // words per warp per batch, loads first
+        const int warp = threadIdx.x >> 5;
+        for (int wd0 = warp; wd0 < kw; wd0 += WARPS * XB) {
+            float xv[XB];
+            #pragma unroll
+            for (int j = 0; j < XB; ++j) {
+                const int wd = wd0 + WARPS * j;
+                const int e = 32 * wd + lane;
+                xv[j] = (wd < kw && e < K) ? to_float(x[e]) : 0.0f;
+            }
+            #pragma unroll
+            for (int j = 0; j < XB; ++j) {
+                const int wd = wd0 + WARPS * j;
+                const uint32_t word = __ballot_sync(0xffffffffu, xv[j] < 0.0f);
+                if (lane == 0 && wd < kw) xs[wd] = word;
+            }
+        }
+    }
+}
+
+// SINGLE: every row fits in one warp-wide pass (nchunks <= LPR).
+// PREFETCH: issue the W loads before the programmatic-launch wait.
+// VEC: x is 16-byte aligned (vector loads for the x pack).
+template <typename XT, int LPR, bool SINGLE, bool PREFETCH, bool VEC>
 __global__ void __launch_bounds__(gemv::THREADS)
 xnor_gemv_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restrict__ x, int N,
                  int K, int kw, const float* __restrict__ alpha, int32_t* __restrict__ y_i32,
-                 float* __restrict__ y_f32, bool weights_static) {
+                 float* __restrict__ y_f32) {
     using namespace gemv;
     constexpr int RPI = 32 / LPR;  // rows per warp-wide load
-    constexpr int XB = 16;         // x words packed per warp per batch (all loads in flight)
     extern __shared__ __align__(16) uint32_t xs[];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int nchunks = kw / 4;                       // 16-byte chunks per row
-    const int64_t gw = (int64_t)blockIdx.x * WARPS + warp;
     const int sub = lane / LPR;                       // row within a warp-wide load
     const int li = lane % LPR;                        // lane within the row
-    int rows[U];
-    #pragma unroll
-    for (int u = 0; u < U; ++u) rows[u] = (int)((gw * U + u) * RPI + sub);
+    const int row0 = (blockIdx.x * WARPS + warp) * U * RPI + sub;   // rows row0 + u * RPI
 
     // Let the next kernel on the stream start its own prologue now; it waits
     // for this grid to finish before it touches anything this grid writes.
@@ -59,49 +125,41 @@ xnor_gemv_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restri
     auto load_pass = [&](int t) {
         const int c = li + LPR * t;
         #pragma unroll
-        for (int u = 0; u < U; ++u)
-            v[u] = (rows[u] < N && c < nchunks)
-                       ? ldg_stream_v4(W + (int64_t)rows[u] * ldw + 4 * c)
-                       : make_uint4(0u, 0u, 0u, 0u);
+        for (int u = 0; u < U; ++u) {
+            const int r = row0 + u * RPI;
+            v[u] = (r < N && c < nchunks) ? ldg_stream_v4(W + (int64_t)r * ldw + 4 * c)
+                                          : make_uint4(0u, 0u, 0u, 0u);
+        }
     };
 
     // The weight stream does not depend on x.  With static weights it starts
     // before the dependency wait (overlapping the previous kernel's tail);
     // otherwise right after it, still ahead of the x loads.
-    if (weights_static) load_pass(0);
+    if constexpr (PREFETCH) load_pass(0);
     grid_dependency_wait();
-    if (!weights_static) load_pass(0);
+    if constexpr (!PREFETCH) load_pass(0);
 
-    // Pack x into shared memory: word wd <- ballot over elements 32*wd + lane.
-    // XB words per warp per batch, all loads issued before the first ballot.
-    for (int wd0 = warp; wd0 < kw; wd0 += WARPS * XB) {
-        float xv[XB];
-        #pragma unroll
-        for (int j = 0; j < XB; ++j) {
-            const int wd = wd0 + WARPS * j;
-            const int e = 32 * wd + lane;
-            xv[j] = (wd < kw && e < K) ? to_float(x[e]) : 0.0f;
-        }
-        #pragma unroll
-        for (int j = 0; j < XB; ++j) {
-            const int wd = wd0 + WARPS * j;
-            const uint32_t word = __ballot_sync(0xffffffffu, xv[j] < 0.0f);
-            if (lane == 0 && wd < kw) xs[wd] = word;
-        }
-    }
+    gemv_pack_x<XT, VEC>(x, K, kw, xs);
     __syncthreads();
 
     uint32_t d[U];
-    #pragma unroll
-    for (int u = 0; u < U; ++u) d[u] = 0u;
-    const int passes = (nchunks + LPR - 1) / LPR;
-    for (int t = 0; t < passes; ++t) {
-        if (t > 0) load_pass(t);
-        const int c = li + LPR * t;
-        const uint4 xv = (c < nchunks) ? *reinterpret_cast<const uint4*>(xs + 4 * c)
-                                       : make_uint4(0u, 0u, 0u, 0u);
+    if constexpr (SINGLE) {
+        const uint4 xq = li < nchunks ? *reinterpret_cast<const uint4*>(xs + 4 * li)
+                                      : make_uint4(0u, 0u, 0u, 0u);
         #pragma unroll
-        for (int u = 0; u < U; ++u) d[u] += popc_xor4(v[u], xv);
+        for (int u = 0; u < U; ++u) d[u] = popc_xor4(v[u], xq);
+    } else {
+        #pragma unroll
+        for (int u = 0; u < U; ++u) d[u] = 0u;
+        const int passes = (nchunks + LPR - 1) / LPR;
+        for (int t = 0; t < passes; ++t) {
+            if (t > 0) load_pass(t);
+            const int c = li + LPR * t;
+            const uint4 xq = (c < nchunks) ? *reinterpret_cast<const uint4*>(xs + 4 * c)
+                                           : make_uint4(0u, 0u, 0u, 0u);
+            #pragma unroll
+            for (int u = 0; u < U; ++u) d[u] += popc_xor4(v[u], xq);
+        }
     }
 
     #pragma unroll
@@ -113,11 +171,11 @@ xnor_gemv_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restri
             #pragma unroll
             for (int off = LPR / 2; off >= 1; off >>= 1) dd += __shfl_xor_sync(0xffffffffu, dd, off);
         }
-        const int r = rows[u];
+        const int r = row0 + u * RPI;
         if (li == 0 && r < N) {
-            const int32_t s = K - 2 * (int32_t)dd;
-            if (y_i32 != nullptr) y_i32[r] = s;
-            if (y_f32 != nullptr) y_f32[r] = alpha[r] * (float)s;
+            const int32_t sv = K - 2 * (int32_t)dd;
+            if (y_i32 != nullptr) y_i32[r] = sv;
+            if (y_f32 != nullptr) y_f32[r] = alpha[r] * (float)sv;
         }
     }
 }
