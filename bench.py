@@ -48,6 +48,10 @@ if ROOT not in sys.path:
 METRIC = "binary GMAC/s (TOPS) for packed XNOR-popcount GEMM; GEMV GB/s vs HBM peak"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+# Dense int8 tensor throughput is twice dense bf16 (4.5 vs 2.25 PFLOP/s nominal);
+# the int8 peak used here is the measured bf16 peak times that ratio.
+INT8_PER_BF16 = 2.0
 SM_COUNT = 148
 # 32-bit population count: 16 per clock per SM (CUDA arithmetic-instruction
 # throughput table); one POPC covers 32 binary multiply-accumulates.
@@ -85,8 +89,11 @@ def peaks():
     if os.path.exists(p):
         d = json.load(open(p))
         return {"hbm_gbs": float(d["hbm_gbs"]), "sm_max_mhz": float(d.get("sm_max_mhz", 1965.0)),
+                "bf16_tflops": float(d.get("bf16_tflops", FALLBACK_BF16_TFLOPS)),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", 1400.0)),
                 "source": "measured"}
-    return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": 1965.0, "source": "fallback"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": 1965.0, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
 def alu_peak_mac_s(sm_mhz: float) -> float:
@@ -97,6 +104,7 @@ def alu_peak_mac_s(sm_mhz: float) -> float:
 # Source files that determine each kernel's code (its own header + shared helpers).
 KERNEL_SOURCES = {
     "xnor_gemv_kernel": ("gemv.cuh", "common.cuh"),
+    "xnor_gemm_tc_kernel": ("gemm_tc.cuh", "gemm_popc.cuh", "common.cuh"),
     "xnor_gemm_popc_kernel": ("gemm_popc.cuh", "common.cuh"),
     "xnor_conv3x3_kernel": ("conv.cuh", "common.cuh"),
     "pack_sign_rows_kernel": ("pack.cuh", "common.cuh"),
@@ -415,11 +423,11 @@ def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws, o
     if "pack_sign_weights" in want:
         _row_pack(torch, bnn, workloads, dev, pk, rows, timed, steps, ws)
     if "square_gemm" in want:
-        _row_square(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, clk_mhz)
+        _row_square(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, clk_mhz, pk)
     if "conv3x3" in want:
         _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak)
     if "mlp4" in want:
-        _row_mlp(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak)
+        _row_mlp(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk)
     if bnn.bnn_device_error() != 0:
         raise RuntimeError("a kernel reported a device-side timeout")
     return rows
@@ -442,31 +450,53 @@ def _row_pack(torch, bnn, workloads, dev, pk, rows, timed, steps, ws):
     torch.cuda.empty_cache()
 
 
-def _row_square(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, clk_mhz):
-    # --- a2+a3+a6: square GEMM 8192^3, int32 + alpha-scaled fp32 outputs ---
+def _tensor_roofline(pk, macs_per_s, sustained):
+    """The tensor-core engine against the int8 tensor peak (one binary MAC is
+    one int8 MAC there): measured bf16 dense TFLOP/s x 2, as int8 TOPS."""
+    bf16 = pk["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    peak_tops = bf16 * INT8_PER_BF16
+    achieved = 2 * macs_per_s / 1e12
+    return {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak_tops, 1), "unit": "TOPS (int8)",
+            "frac": round(achieved / peak_tops, 4),
+            "peak_derivation": f"measured bf16 {'sustained' if sustained else 'burst'} {bf16} TFLOP/s x {INT8_PER_BF16} (dense int8 / bf16)",
+            "traffic": recorded_traffic("xnor_gemm_tc_kernel")}
+
+
+def _row_square(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, clk_mhz, pk=None):
+    # --- a2+a3+a6: square GEMM 8192^3, int32 + alpha-scaled fp32 outputs, both engines ---
     sq = workloads.square()
     Ad = sq.A.to(dev)
     A_p = bnn.empty_packed(sq.M, sq.K, dev)
     Wsq = bnn.empty_packed(sq.N, sq.K, dev)
     al = torch.empty(sq.N, dtype=torch.float32, device=dev)
     bnn.bnn_pack_sign(sq.W.to(dev), Wsq, al)
+    bnn.bnn_pack_sign(Ad, A_p)
     Ci = torch.empty(sq.M, sq.N, dtype=torch.int32, device=dev)
     Cf = torch.empty(sq.M, sq.N, dtype=torch.float32, device=dev)
     macs = sq.M * sq.N * sq.K
-    ms_g = timed(lambda i: bnn.bnn_xnor_gemm(A_p, Wsq, sq.K, al, Ci, Cf))
-    bnn.bnn_pack_sign(Ad, A_p)
-    ms_s = timed(lambda i: (bnn.bnn_pack_sign(Ad, A_p), bnn.bnn_xnor_gemm(A_p, Wsq, sq.K, al, Ci, Cf)))
-    mac_s = macs * steps / (ms_g * 1e-3)
-    rows["square_gemm"] = {
-        "workload": "M=N=K=8192 packed A x packed W^T, int32 s + alpha*s fp32 out",
-        "value": round(ws * mac_s / 1e9, 1), "unit": "binary GMAC/s", "tops": round(ws * 2 * mac_s / 1e12, 2),
-        "ms_per_step": ms_g / steps,
-        "with_activation_pack": {"value": round(ws * macs * steps / (ms_s * 1e-3) / 1e9, 1),
-                                 "unit": "binary GMAC/s", "ms_per_step": ms_s / steps},
-        "roofline": {"bound": "alu", "achieved": round(mac_s / 1e12, 2), "peak": round(alu_peak / 1e12, 2),
-                     "unit": "binary TMAC/s", "frac": round(mac_s / alu_peak, 4),
-                     "peak_derivation": f"{SM_COUNT} SMs x {POPC_PER_CLK_PER_SM} POPC/clk x 32 MAC x {clk_mhz:.0f} MHz",
-                     "traffic": recorded_traffic("xnor_gemm_popc_kernel")}}
+    for name, engine in (("square_gemm", bnn.BNN_GEMM_ENGINE_TENSOR), ("square_gemm_popcount", bnn.BNN_GEMM_ENGINE_POPCOUNT)):
+        with bnn.gemm_engine(engine):
+            ms_g = timed(lambda i: bnn.bnn_xnor_gemm(A_p, Wsq, sq.K, al, Ci, Cf))
+            ms_s = timed(lambda i: (bnn.bnn_pack_sign(Ad, A_p), bnn.bnn_xnor_gemm(A_p, Wsq, sq.K, al, Ci, Cf)))
+        mac_s = macs * steps / (ms_g * 1e-3)
+        if engine == bnn.BNN_GEMM_ENGINE_TENSOR:
+            roof = _tensor_roofline(pk, mac_s, sustained=False)
+            kernel = "xnor_gemm_tc_kernel"
+        else:
+            roof = {"bound": "alu", "achieved": round(mac_s / 1e12, 2), "peak": round(alu_peak / 1e12, 2),
+                    "unit": "binary TMAC/s", "frac": round(mac_s / alu_peak, 4),
+                    "peak_derivation": f"{SM_COUNT} SMs x {POPC_PER_CLK_PER_SM} POPC/clk x 32 MAC x {clk_mhz:.0f} MHz",
+                    "traffic": recorded_traffic("xnor_gemm_popc_kernel")}
+            kernel = "xnor_gemm_popc_kernel"
+        rows[name] = {
+            "workload": "M=N=K=8192 packed A x packed W^T, int32 s + alpha*s fp32 out",
+            "engine": "tensor (tcgen05 kind::i8)" if engine == bnn.BNN_GEMM_ENGINE_TENSOR else "popcount (XOR + POPC, carry-save)",
+            "kernel": kernel,
+            "value": round(ws * mac_s / 1e9, 1), "unit": "binary GMAC/s", "tops": round(ws * 2 * mac_s / 1e12, 2),
+            "ms_per_step": ms_g / steps,
+            "with_activation_pack": {"value": round(ws * macs * steps / (ms_s * 1e-3) / 1e9, 1),
+                                     "unit": "binary GMAC/s", "ms_per_step": ms_s / steps},
+            "roofline": roof}
     del sq, Ad, A_p, Wsq, al, Ci, Cf
     torch.cuda.empty_cache()
 
@@ -505,7 +535,7 @@ def _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak):
     torch.cuda.empty_cache()
 
 
-def _row_mlp(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak):
+def _row_mlp(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk=None):
     # --- MLP: pack input, 3 x (GEMM + folded-BN re-pack), GEMM + alpha ---
     m = workloads.mlp()
     B, D = m.X0.shape
@@ -536,16 +566,20 @@ def _row_mlp(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak):
             bnn.bnn_binary_linear_fused(A, Wps[l], D, eps_[l][0], o)
             A = o
 
-    ms_m = timed(mlp_step)
     mmacs = 4 * B * D * D
-    rows["mlp4"] = {
-        "workload": "fully binary MLP, batch 4096, width 4096, 4 layers: pack fp32 input, "
-                    "3 x (GEMM + folded BatchNorm sign re-pack), GEMM + alpha fp32 logits",
-        "value": round(ws * mmacs * steps / (ms_m * 1e-3) / 1e9, 1), "unit": "binary GMAC/s",
-        "ms_per_step": ms_m / steps,
-        "roofline": {"bound": "alu", "achieved": round(mmacs * steps / (ms_m * 1e-3) / 1e12, 2),
-                     "peak": round(alu_peak / 1e12, 2), "unit": "binary TMAC/s",
-                     "frac": round(mmacs * steps / (ms_m * 1e-3) / alu_peak, 4)}}
+    for name, engine in (("mlp4", bnn.BNN_GEMM_ENGINE_TENSOR), ("mlp4_popcount", bnn.BNN_GEMM_ENGINE_POPCOUNT)):
+        with bnn.gemm_engine(engine):
+            ms_m = timed(mlp_step)
+        mac_s = mmacs * steps / (ms_m * 1e-3)
+        roof = (_tensor_roofline(pk, mac_s, sustained=False) if engine == bnn.BNN_GEMM_ENGINE_TENSOR else
+                {"bound": "alu", "achieved": round(mac_s / 1e12, 2), "peak": round(alu_peak / 1e12, 2),
+                 "unit": "binary TMAC/s", "frac": round(mac_s / alu_peak, 4)})
+        rows[name] = {
+            "workload": "fully binary MLP, batch 4096, width 4096, 4 layers: pack fp32 input, "
+                        "3 x (GEMM + folded BatchNorm sign re-pack), GEMM + alpha fp32 logits",
+            "engine": "tensor" if engine == bnn.BNN_GEMM_ENGINE_TENSOR else "popcount",
+            "value": round(ws * mac_s / 1e9, 1), "unit": "binary GMAC/s",
+            "ms_per_step": ms_m / steps, "roofline": roof}
     del m, X0, A0, acts, eps_, Wps, logits
     torch.cuda.empty_cache()
 

@@ -195,11 +195,18 @@ bnn_status launch_gemv_t(const uint32_t* W, int64_t ldw, const XT* x, int64_t N,
         if (smem > 48 * 1024 &&
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
             return BNN_ERR_CUDA;
-        e = cudaLaunchKernelEx(&cfg, kern, W, ldw, x, iN, iK, ikw, alpha, y_i32, y_f32);
+        e = cudaLaunchKernelEx(&cfg, kern, W, ldw, x, iN, iK, ikw, alpha, y_i32, y_f32, 1);
         return BNN_OK;
     };
     bnn_status st = BNN_OK;
     const bool vec = aligned(x, 16);
+    if (lpr == 32 && single && vec) {
+        // Rows of 97..128 words: the dedicated one-chunk-per-lane kernel.
+        auto kern = bnn::xnor_gemv_row128_kernel<XT>;
+        e = cudaLaunchKernelEx(&cfg, kern, W, ldw, x, iN, iK, ikw, alpha, y_i32, y_f32, weights_static ? 1 : 0, 1);
+        if (e != cudaSuccess) return BNN_ERR_CUDA;
+        return launch_status();
+    }
 #define BNN_GEMV_PICK(L, S, P)                                                                      \
     (vec ? launch(bnn::xnor_gemv_kernel<XT, L, S, P, true>) : launch(bnn::xnor_gemv_kernel<XT, L, S, P, false>))
 #define BNN_GEMV_CASE(L)                                                                            \

@@ -101,8 +101,9 @@ xnor_gemm_popc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
     constexpr int W_BYTES = BN_ * BKW * 4;
     constexpr int STAGE = A_TILE_BYTES + W_BYTES;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~uintptr_t(1023));
+    // 1024-byte aligned base, derived by offset from the __shared__ array so
+    // that the compiler keeps every access in the shared address space.
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE);
     uint64_t* empty = full + STAGES;
 

@@ -11,10 +11,11 @@
 // 0 bits in both operands, i.e. (+1)(+1) = +1 each; the epilogue subtracts
 // their count, (K rounded up to a whole stage) - K.
 //
-// Design (sm_100a, one persistent CTA per SM, 14 warps):
+// Design (sm_100a, one persistent CTA per SM, 18 warps):
 //  * warp 0   : TMA producer.  Packed tiles (128 A rows x 4 words, 256 W rows
 //               x 4 words = 128 binary elements of K) into an 8-stage ring.
-//  * warps 2-9: unpack.  Each packed word becomes 32 signed bytes in the
+//  * warps 2-13: unpack, one thread per packed row of the stage (128 A rows,
+//               256 W rows).  Each packed word becomes 32 signed bytes in the
 //               K-major 128B-swizzled layout the tensor core reads (chunk c of
 //               row r at (c ^ (r & 7)) * 16); four ops per 4 bytes (PRMT picks
 //               a nibble, IMAD spreads its bits into bytes, LOP3 masks, IMAD
@@ -24,7 +25,7 @@
 //               one thread issues 4 tcgen05.mma (M=128, N=256, K=32) per stage
 //               and commits them to the stage's "empty" barrier, and to the
 //               accumulator's "full" barrier after the last stage of a tile.
-//  * warps 10-13: epilogue.  Warp q reads TMEM lanes 32q..32q+31 (one output
+//  * warps 14-17: epilogue.  Warp q reads TMEM lanes 32q..32q+31 (one output
 //               row per thread) 32 columns at a time with tcgen05.ld, releases
 //               the accumulator, and writes int32 / alpha*s / affine outputs or
 //               the folded-BatchNorm sign bits (32 columns = one packed word,
@@ -53,10 +54,10 @@ constexpr int P_STAGE = P_A_BYTES + P_B_BYTES;
 constexpr int U_A_BYTES = BM * BKE;        // 16 KiB
 constexpr int U_B_BYTES = BN * BKE;        // 32 KiB
 constexpr int U_STAGE = U_A_BYTES + U_B_BYTES;
-constexpr int UNPACK_WARPS = 8;
+constexpr int UNPACK_WARPS = 12;           // one thread per packed row of a stage (128 + 256)
 constexpr int EPI_WARPS = 4;
 constexpr int WARP_PRODUCER = 0, WARP_MMA = 1, WARP_UNPACK0 = 2, WARP_EPI0 = WARP_UNPACK0 + UNPACK_WARPS;
-constexpr int THREADS = (WARP_EPI0 + EPI_WARPS) * 32;   // 448
+constexpr int THREADS = (WARP_EPI0 + EPI_WARPS) * 32;   // 576
 constexpr int TMEM_COLS = 2 * BN;          // two accumulators
 constexpr int NUM_BARS = 2 * PSTAGES + 2 * USTAGES + 2 * 2 + 1;
 constexpr int SMEM_BYTES = USTAGES * U_STAGE + PSTAGES * P_STAGE + NUM_BARS * 8 + 16 + 1024;
@@ -146,7 +147,9 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     int K, int kw, int tiles_m, int tiles_n, GemmEpilogue ep) {
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base, derived by offset from the __shared__ array so
+    // that the compiler keeps every access in the shared address space.
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* uring = smem;                                   // USTAGES x (A 16 KiB | W 32 KiB)
     uint8_t* pring = smem + USTAGES * U_STAGE;               // PSTAGES x (A 2 KiB | W 4 KiB)
     uint64_t* bars = reinterpret_cast<uint64_t*>(pring + PSTAGES * P_STAGE);
@@ -251,8 +254,12 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         __syncwarp();
     } else if (warp < WARP_EPI0) {
         // ------------------------------ unpack warps ------------------------------
-        const int u = threadIdx.x - WARP_UNPACK0 * 32;               // 0..255
-        const uint32_t* pw = reinterpret_cast<const uint32_t*>(pring);
+        // Thread u expands packed row u of the stage (A rows 0..127, then W rows):
+        // one 16-byte load of its 4 words, eight 16-byte stores of its 128 bytes.
+        const int u = threadIdx.x - WARP_UNPACK0 * 32;               // 0..383
+        const bool is_a = u < BM;
+        const int r = is_a ? u : u - BM;
+        const int sw = r & 7;
         uint32_t g = 0;
         bool ok = true;
         for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
@@ -261,21 +268,14 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 bool w1 = tc_wait(&pfull[ps], (g / PSTAGES) & 1, abort_flag);
                 bool w2 = w1 && (g < USTAGES || tc_wait(&uempty[us], ((g / USTAGES) - 1) & 1, abort_flag));
                 if (!__all_sync(0xffffffffu, w1 && w2)) { ok = false; break; }
-                const uint32_t* src = pw + ps * (P_STAGE / 4);
-                uint8_t* dstA = uring + us * U_STAGE;
-                uint8_t* dstB = dstA + U_A_BYTES;
-                uint32_t words[6];
-                #pragma unroll
-                for (int i = 0; i < 6; ++i) words[i] = src[u + 256 * i];
+                const uint4 pk = *reinterpret_cast<const uint4*>(pring + ps * P_STAGE + u * 16);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&pempty[ps]);             // packed stage consumed
+                uint8_t* row = uring + us * U_STAGE + (is_a ? 0 : U_A_BYTES) + r * 128;
+                const uint32_t wq[4] = {pk.x, pk.y, pk.z, pk.w};
                 #pragma unroll
-                for (int i = 0; i < 6; ++i) {
-                    const int v = u + 256 * i;                        // word index: A rows first, then W rows
-                    const int r = v < BM * BKW ? (v >> 2) : ((v - BM * BKW) >> 2);
-                    const int q = v & 3;
-                    uint8_t* row = (v < BM * BKW ? dstA : dstB) + r * 128;
-                    const uint32_t w = words[i];
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t w = wq[q];
                     const uint32_t lo = w & 0x0F0F0F0Fu;              // nibbles 0, 2, 4, 6 (one per byte)
                     const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;       // nibbles 1, 3, 5, 7
                     uint4 c0, c1;
@@ -287,7 +287,6 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     c1.y = pm1_bytes(__byte_perm(hi, 0u, 0x4442u));
                     c1.z = pm1_bytes(__byte_perm(lo, 0u, 0x4443u));
                     c1.w = pm1_bytes(__byte_perm(hi, 0u, 0x4443u));
-                    const int sw = r & 7;
                     *reinterpret_cast<uint4*>(row + (((2 * q) ^ sw) << 4)) = c0;
                     *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ sw) << 4)) = c1;
                 }
@@ -344,32 +343,41 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 }
                 if (m < M && ep.c_i32 != nullptr) {
                     int32_t* dst = ep.c_i32 + (int64_t)m * ep.ldc + nb;
-                    if (full_chunk && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0)) {
-                        #pragma unroll
-                        for (int j = 0; j < 32; j += 4)
-                            *reinterpret_cast<int4*>(dst + j) =
-                                make_int4((int32_t)r[j] - pad, (int32_t)r[j + 1] - pad, (int32_t)r[j + 2] - pad,
-                                          (int32_t)r[j + 3] - pad);
-                    } else {
-                        for (int j = 0; j < 32 && nb + j < N; ++j) dst[j] = (int32_t)r[j] - pad;
+                    const bool vec = full_chunk && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0);
+                    #pragma unroll
+                    for (int j = 0; j < 32; j += 4) {
+                        const int4 o = make_int4((int32_t)r[j] - pad, (int32_t)r[j + 1] - pad,
+                                                 (int32_t)r[j + 2] - pad, (int32_t)r[j + 3] - pad);
+                        if (vec) {
+                            *reinterpret_cast<int4*>(dst + j) = o;
+                        } else {
+                            if (nb + j < N) dst[j] = o.x;
+                            if (nb + j + 1 < N) dst[j + 1] = o.y;
+                            if (nb + j + 2 < N) dst[j + 2] = o.z;
+                            if (nb + j + 3 < N) dst[j + 3] = o.w;
+                        }
                     }
                 }
                 if (m < M && ep.c_f32 != nullptr) {
                     float* dst = ep.c_f32 + (int64_t)m * ep.ldf + nb;
-                    float y[32];
+                    const bool vec = full_chunk && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0);
                     #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int n = min(nb + j, N - 1);
-                        float v = __ldg(ep.alpha + n) * (float)((int32_t)r[j] - pad);
-                        if (ep.gamma != nullptr) v = fmaf(__ldg(ep.gamma + n), v, __ldg(ep.beta + n));
-                        y[j] = v;
-                    }
-                    if (full_chunk && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0)) {
+                    for (int j = 0; j < 32; j += 4) {
+                        float y[4];
                         #pragma unroll
-                        for (int j = 0; j < 32; j += 4)
-                            *reinterpret_cast<float4*>(dst + j) = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
-                    } else {
-                        for (int j = 0; j < 32 && nb + j < N; ++j) dst[j] = y[j];
+                        for (int k = 0; k < 4; ++k) {
+                            const int n = min(nb + j + k, N - 1);
+                            float v = __ldg(ep.alpha + n) * (float)((int32_t)r[j + k] - pad);
+                            if (ep.gamma != nullptr) v = fmaf(__ldg(ep.gamma + n), v, __ldg(ep.beta + n));
+                            y[k] = v;
+                        }
+                        if (vec) {
+                            *reinterpret_cast<float4*>(dst + j) = make_float4(y[0], y[1], y[2], y[3]);
+                        } else {
+                            #pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                if (nb + j + k < N) dst[j + k] = y[k];
+                        }
                     }
                 }
             }
