@@ -103,7 +103,7 @@ def alu_peak_mac_s(sm_mhz: float) -> float:
 
 # Source files that determine each kernel's code (its own header + shared helpers).
 KERNEL_SOURCES = {
-    "xnor_gemv_kernel": ("gemv.cuh", "common.cuh"),
+    "xnor_gemv_row128_kernel": ("gemv.cuh", "common.cuh"),
     "xnor_gemm_tc_kernel": ("gemm_tc.cuh", "gemm_popc.cuh", "common.cuh"),
     "xnor_gemm_popc_kernel": ("gemm_popc.cuh", "common.cuh"),
     "xnor_conv3x3_kernel": ("conv.cuh", "common.cuh"),
@@ -327,9 +327,9 @@ def run_ours(args, torch, dist):
             "peak": pk["hbm_gbs"],
             "unit": "GB/s",
             "frac": round(achieved / pk["hbm_gbs"], 4),
-            "traffic": recorded_traffic("xnor_gemv_kernel"),
+            "traffic": recorded_traffic("xnor_gemv_row128_kernel"),
             "peak_source": pk["source"],
-            "kernel": "xnor_gemv_kernel",
+            "kernel": "xnor_gemv_row128_kernel",
         },
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
