@@ -107,6 +107,7 @@ KERNEL_SOURCES = {
     "xnor_gemm_tc_kernel": ("gemm_tc.cuh", "gemm_popc.cuh", "common.cuh"),
     "xnor_gemm_popc_kernel": ("gemm_popc.cuh", "common.cuh"),
     "xnor_conv3x3_kernel": ("conv.cuh", "common.cuh"),
+    "xnor_conv3x3_tc_kernel": ("conv_tc.cuh", "conv.cuh", "gemm_tc.cuh", "gemm_popc.cuh", "common.cuh"),
     "pack_sign_rows_kernel": ("pack.cuh", "common.cuh"),
 }
 
@@ -425,7 +426,7 @@ def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws, o
     if "square_gemm" in want:
         _row_square(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, clk_mhz, pk)
     if "conv3x3" in want:
-        _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak)
+        _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk)
     if "mlp4" in want:
         _row_mlp(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk)
     if bnn.bnn_device_error() != 0:
@@ -501,7 +502,7 @@ def _row_square(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, cl
     torch.cuda.empty_cache()
 
 
-def _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak):
+def _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk):
     # --- a2 (NCHW) + a5 + a6: ResNet-class binary 3x3 conv with affine epilogue ---
     cv = workloads.conv()
     n, c, h, w = cv.X.shape
@@ -518,19 +519,36 @@ def _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak):
         bnn.bnn_pack_sign_nchw(Xd, Xb)
         bnn.bnn_binary_conv3x3_fused(Xb, c, Wc, ep, out, 1, 1)
 
-    ms_c = timed(conv_step)
-    bnn.bnn_pack_sign_nchw(Xd, Xb)
-    ms_ck = timed(lambda i: bnn.bnn_binary_conv3x3_fused(Xb, c, Wc, ep, out, 1, 1))
     cmacs = n * h * w * 64 * 9 * c
-    cmac_s = cmacs * steps / (ms_ck * 1e-3)
-    rows["conv3x3"] = {
-        "workload": "bf16 [64,64,56,56] -> pack NCHW -> binary 3x3 conv (64 filters, stride 1, pad 1), "
-                    "alpha + affine epilogue, fp32 NCHW out",
-        "value": round(ws * cmacs * steps / (ms_c * 1e-3) / 1e9, 1), "unit": "binary GMAC/s",
-        "ms_per_step": ms_c / steps, "conv_kernel_ms": ms_ck / steps,
-        "roofline": {"bound": "alu", "achieved": round(cmac_s / 1e12, 2), "peak": round(alu_peak / 1e12, 2),
-                     "unit": "binary TMAC/s", "frac": round(cmac_s / alu_peak, 4),
-                     "traffic": recorded_traffic("xnor_conv3x3_kernel")}}
+    # Algorithmic bytes of one conv launch: packed activations and filters in,
+    # fp32 NCHW out (alpha/gamma/beta are 768 B).
+    cbytes = Xb.numel() * 4 + Wc.numel() * 4 + out.numel() * 4
+    for name, engine in (("conv3x3", bnn.BNN_GEMM_ENGINE_POPCOUNT), ("conv3x3_tensor", bnn.BNN_GEMM_ENGINE_TENSOR)):
+        with bnn.gemm_engine(engine):
+            ms_c = timed(conv_step)
+            bnn.bnn_pack_sign_nchw(Xd, Xb)
+            ms_ck = timed(lambda i: bnn.bnn_binary_conv3x3_fused(Xb, c, Wc, ep, out, 1, 1))
+        cmac_s = cmacs * steps / (ms_ck * 1e-3)
+        if engine == bnn.BNN_GEMM_ENGINE_TENSOR:
+            # The fp32 output write bounds this kernel: 51 MB out against 7.4 G
+            # binary MACs, 8 us of HBM time versus under 5 us of int8 tensor time.
+            ach = cbytes * steps / (ms_ck * 1e-3) / 1e9
+            roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(ach / pk["hbm_gbs"], 4), "algorithmic_bytes": cbytes,
+                    "tensor": _tensor_roofline(pk, cmac_s, sustained=False),
+                    "traffic": recorded_traffic("xnor_conv3x3_tc_kernel")}
+            roof["tensor"].pop("traffic")
+        else:
+            roof = {"bound": "alu", "achieved": round(cmac_s / 1e12, 2), "peak": round(alu_peak / 1e12, 2),
+                    "unit": "binary TMAC/s", "frac": round(cmac_s / alu_peak, 4),
+                    "traffic": recorded_traffic("xnor_conv3x3_kernel")}
+        rows[name] = {
+            "workload": "bf16 [64,64,56,56] -> pack NCHW -> binary 3x3 conv (64 filters, stride 1, pad 1), "
+                        "alpha + affine epilogue, fp32 NCHW out"
+                        + (" (tensor-core engine)" if engine == bnn.BNN_GEMM_ENGINE_TENSOR else " (popcount engine)"),
+            "value": round(ws * cmacs * steps / (ms_c * 1e-3) / 1e9, 1), "unit": "binary GMAC/s",
+            "ms_per_step": ms_c / steps, "conv_kernel_ms": ms_ck / steps,
+            "conv_kernel_binary_tmac_s": round(cmac_s / 1e12, 2), "roofline": roof}
     del cv, Xd, Xb, Wc, alc, gam, bet, out
     torch.cuda.empty_cache()
 

@@ -115,6 +115,18 @@ const char* bnn_status_string(int status);
  * the flag value to *code_out (host pointer). */
 bnn_status bnn_device_error(int32_t* code_out);
 
+/* bnn_selftest_wait_timeout -- diagnostic for the bounded waits.  Runs one
+ * kernel that waits on an mbarrier nothing arrives on, with a limit of
+ * timeout_ns (1 .. 1e10); the wait must give up, record
+ * BNN_ERR_DEVICE_TIMEOUT in the device-side flag (read it with
+ * bnn_device_error) and return, leaving the context usable.  Synchronous
+ * (it synchronises the current device); allocates nothing.
+ * *waited_out (host) is 1 when the wait ran out, 0 if it completed.
+ * The pages have no counterpart: it exists to test the library's failure
+ * detection without faulting or hanging the GPU.
+ *   Errors: INVALID_ARG, CUDA. */
+bnn_status bnn_selftest_wait_timeout(int64_t timeout_ns, int32_t* waited_out);
+
 /* bnn_pack_sign -- sign-binarise and bit-pack a real matrix along K, and
  * optionally compute alpha per row.
  *   Passage: "Extreme Quantization ...", Notation (sign) and eq. (4);
@@ -161,15 +173,19 @@ bnn_status bnn_pack_conv3x3_weights(const void* w_oihw, bnn_dtype dt, int64_t co
                                     uint32_t* packed, int64_t ld_words, float* alpha_out,
                                     bnn_stream_t stream);
 
-/* Engine used by bnn_xnor_gemm and bnn_binary_linear_fused.  Both engines
- * return identical results (the product is exact integer arithmetic):
+/* Engine used by bnn_xnor_gemm, bnn_binary_linear_fused and
+ * bnn_binary_conv3x3_fused.  Both engines return identical results (the
+ * product is exact integer arithmetic):
  *   POPCOUNT: XOR + population count on the integer pipes, with carry-save
  *             compression (any shape).
  *   TENSOR:   the sign bits expanded to +1/-1 bytes in shared memory and
  *             multiplied on the tensor cores (tcgen05.mma kind::i8, int32
  *             accumulators in tensor memory); for large products.
  *   AUTO:     TENSOR when M >= 128, N >= 128 and K >= 512, else POPCOUNT
- *             (the default). */
+ *             (the default); the convolution uses POPCOUNT under AUTO.
+ * The convolution uses the tensor cores only under TENSOR, and only where
+ * c <= 64, cout <= 256 and its shared memory fits (c <= 32: every cout;
+ * 33..64: up to 96 filters); other shapes use the popcount kernel. */
 typedef enum bnn_gemm_engine {
     BNN_GEMM_ENGINE_AUTO = 0,
     BNN_GEMM_ENGINE_POPCOUNT = 1,

@@ -12,6 +12,14 @@ from gpu_util import assert_affine_close, assert_no_device_error, assert_scaled_
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(params=[bnn.BNN_GEMM_ENGINE_POPCOUNT, bnn.BNN_GEMM_ENGINE_TENSOR], ids=["popcount", "tensor"])
+def engine(request):
+    """TENSOR runs the tcgen05 convolution where it applies (c <= 64,
+    cout <= 256); other shapes stay on the popcount kernel."""
+    with bnn.gemm_engine(request.param):
+        yield request.param
+
+
 def run_conv(X, Wt, gamma, beta, stride, pad, mode):
     d = dev()
     n, c, h, w = X.shape
@@ -32,11 +40,14 @@ def run_conv(X, Wt, gamma, beta, stride, pad, mode):
 
 
 CASES = [(2, 64, 9, 7, 5, 1, 1), (1, 3, 5, 6, 4, 1, 1), (2, 33, 8, 8, 3, 2, 1), (1, 2, 4, 4, 2, 1, 0),
-         (3, 100, 7, 9, 17, 1, 1), (1, 128, 6, 6, 8, 1, 1), (2, 64, 56, 56, 64, 1, 1), (1, 40, 11, 13, 6, 2, 0)]
+         (3, 100, 7, 9, 17, 1, 1), (1, 128, 6, 6, 8, 1, 1), (2, 64, 56, 56, 64, 1, 1), (1, 40, 11, 13, 6, 2, 0),
+         # tensor-core shapes: filter counts off the 16/32 grid, 256 filters, ragged last tile
+         (3, 50, 19, 17, 40, 1, 1), (1, 20, 9, 9, 48, 1, 1), (2, 32, 12, 12, 256, 1, 1), (1, 64, 10, 10, 200, 1, 1),
+         (1, 1, 5, 5, 1, 1, 1), (5, 64, 33, 31, 96, 2, 1)]
 
 
 @pytest.mark.parametrize("n,c,h,w,cout,stride,pad", CASES)
-def test_conv_modes(n, c, h, w, cout, stride, pad):
+def test_conv_modes(n, c, h, w, cout, stride, pad, engine):
     X = workloads.normal((n, c, h, w), 1.0, n + c + h, dtype=torch.bfloat16)
     Wt = workloads.normal((cout, c, 3, 3), 0.1, cout + c)
     g = workloads.uniform((cout,), 0.5, 1.5, cout)
@@ -58,7 +69,7 @@ def test_conv_modes(n, c, h, w, cout, stride, pad):
     assert_no_device_error()
 
 
-def test_resnet_layer_workload_sampled_images():
+def test_resnet_layer_workload_sampled_images(engine):
     """The ResNet-18-class layer: input bf16 [64, 64, 56, 56], filters
     [64, 64, 3, 3], stride 1, pad 1, affine epilogue; images 0, 31 and 63
     checked against the oracle (each image is independent)."""

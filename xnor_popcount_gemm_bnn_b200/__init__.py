@@ -45,7 +45,7 @@ EXPORTS = (
     "bnn_packed_ld_words", "bnn_conv3x3_ld_words", "bnn_status_string", "bnn_device_error",
     "bnn_pack_sign", "bnn_pack_sign_nchw", "bnn_pack_conv3x3_weights", "bnn_xnor_gemm",
     "bnn_xnor_gemv", "bnn_xnor_gemv_ex", "bnn_binary_linear_fused", "bnn_binary_conv3x3_fused",
-    "bnn_fold_bn_threshold", "bnn_set_gemm_engine", "bnn_get_gemm_engine",
+    "bnn_fold_bn_threshold", "bnn_set_gemm_engine", "bnn_get_gemm_engine", "bnn_selftest_wait_timeout",
 )
 
 
@@ -85,6 +85,7 @@ def _load() -> ctypes.CDLL:
         "bnn_fold_bn_threshold": (i32, [p, p, p, p, p, ctypes.c_double, i64, i64, p, p]),
         "bnn_set_gemm_engine": (i32, [ctypes.c_int]),
         "bnn_get_gemm_engine": (ctypes.c_int, []),
+        "bnn_selftest_wait_timeout": (i32, [i64, p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -163,6 +164,13 @@ class gemm_engine:
 
     def __exit__(self, *exc):
         bnn_set_gemm_engine(self.prev)
+
+
+def bnn_selftest_wait_timeout(timeout_ns: int) -> bool:
+    """Run the bounded-wait diagnostic; True when the wait ran out (expected)."""
+    out = ctypes.c_int32(-1)
+    _check("bnn_selftest_wait_timeout", _lib.bnn_selftest_wait_timeout(int(timeout_ns), ctypes.byref(out)))
+    return bool(out.value)
 
 
 def bnn_device_error() -> int:

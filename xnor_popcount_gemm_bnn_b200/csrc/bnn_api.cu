@@ -14,6 +14,7 @@
 #include "bnn.h"
 #include "common.cuh"
 #include "conv.cuh"
+#include "conv_tc.cuh"
 #include "gemm_popc.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
@@ -299,6 +300,17 @@ bnn_status bnn_device_error(int32_t* code_out) {
     return BNN_OK;
 }
 
+bnn_status bnn_selftest_wait_timeout(int64_t timeout_ns, int32_t* waited_out) {
+    if (timeout_ns < 1 || timeout_ns > 10000000000LL || waited_out == nullptr) return BNN_ERR_INVALID_ARG;
+    bnn::wait_timeout_selftest_kernel<<<1, 32>>>((unsigned long long)timeout_ns);
+    int h = -1;
+    if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess ||
+        cudaMemcpyFromSymbol(&h, bnn::g_selftest_result, sizeof(int)) != cudaSuccess)
+        return BNN_ERR_CUDA;
+    *waited_out = (h == 0) ? 1 : 0;
+    return BNN_OK;
+}
+
 bnn_status bnn_pack_sign(const void* x, bnn_dtype dt, int64_t rows, int64_t K, int64_t ld_x, uint32_t* packed,
                          int64_t ld_words, float* alpha_out, bnn_stream_t stream) {
     if (x == nullptr || packed == nullptr) return BNN_ERR_INVALID_ARG;
@@ -478,6 +490,31 @@ bnn_status bnn_binary_conv3x3_fused(const uint32_t* X_nhwc_bits, int64_t n, int6
     if (smem > 200 * 1024) return BNN_ERR_UNSUPPORTED;
     if (n == 0 || cout == 0) return BNN_OK;
     const int64_t npix = n * oh * ow;
+    bnn::ConvEpilogue ep{epi->mode, epi->alpha, epi->gamma, epi->beta, out_nchw};
+    cudaStream_t s = as_cuda(stream);
+    // Tensor-core engine (when forced): up to 2 words per pixel per tap
+    // (c <= 64) and 256 filters, when the resident filters and two A tiles fit
+    // in shared memory.
+    const int engine = g_gemm_engine.load(std::memory_order_relaxed);
+    const int64_t n_mma = std::max<int64_t>(16, ceil_div(cout, (int64_t)16) * 16);
+    if (engine == BNN_GEMM_ENGINE_TENSOR && cw <= 2 && cout <= bnn::ctc::MAX_N &&
+        bnn::conv_tc_smem_bytes((int)cw, (int)n_mma) <= 227 * 1024) {
+        const int smem_tc = bnn::conv_tc_smem_bytes((int)cw, (int)n_mma);
+        const uint32_t idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n_mma >> 3) << 17) |
+                               ((uint32_t)(bnn::ctc::BM >> 4) << 24);
+        const int64_t tiles = ceil_div(npix, (int64_t)bnn::ctc::BM);
+        if (tiles > INT_MAX) return BNN_ERR_INVALID_ARG;
+        const int64_t grid = std::min<int64_t>(tiles, sm_count());
+        auto launch_tc = [&](auto kern) -> bnn_status {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_tc) != cudaSuccess)
+                return BNN_ERR_CUDA;
+            kern<<<(unsigned)grid, bnn::ctc::THREADS, smem_tc, s>>>(X_nhwc_bits, (int)n, (int)c, (int)h, (int)w,
+                                                                    W_packed, ldw, (int)cout, (int)n_mma, idesc,
+                                                                    (int)stride, (int)pad, (int)oh, (int)ow, ep);
+            return launch_status();
+        };
+        return cw == 1 ? launch_tc(bnn::xnor_conv3x3_tc_kernel<1>) : launch_tc(bnn::xnor_conv3x3_tc_kernel<2>);
+    }
     const int64_t tasks = ceil_div(npix, (int64_t)32) * ceil_div(cout, (int64_t)bnn::conv::FB);
     int sms = 148;
     {
@@ -488,8 +525,6 @@ bnn_status bnn_binary_conv3x3_fused(const uint32_t* X_nhwc_bits, int64_t n, int6
     // more CTAs than there are tasks.
     const int64_t blocks = std::max<int64_t>(
         1, std::min<int64_t>(ceil_div(tasks, bnn::conv::WARPS), (int64_t)sms * bnn::conv::CTAS_PER_SM));
-    bnn::ConvEpilogue ep{epi->mode, epi->alpha, epi->gamma, epi->beta, out_nchw};
-    cudaStream_t s = as_cuda(stream);
 #define BNN_CONV_CASE(CWV)                                                                                 \
     case CWV: {                                                                                            \
         auto kern = bnn::xnor_conv3x3_kernel<CWV>;                                                         \

@@ -84,19 +84,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase of parity `parity` to complete, for at most
-// kWaitTimeoutNs.  On time-out, flags BNN_ERR_DEVICE_TIMEOUT and returns false.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+// `timeout_ns` (about one second by default).  On time-out, flags
+// BNN_ERR_DEVICE_TIMEOUT and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  unsigned long long timeout_ns = kWaitTimeoutNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     while (true) {
         #pragma unroll 1
         for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        if (globaltimer_ns() - t0 > timeout_ns) {
             flag_device_error(BNN_ERR_DEVICE_TIMEOUT);
             return false;
         }
     }
+}
+
+// Diagnostic: one thread waits on an mbarrier that nothing ever arrives on,
+// so the bounded wait runs out after `timeout_ns`; records how it ended in
+// g_selftest_result (1 = completed, 0 = ran out).
+__device__ int g_selftest_result = -1;
+
+__global__ void wait_timeout_selftest_kernel(unsigned long long timeout_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbarrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) g_selftest_result = mbar_wait_bounded(&bar, 0, timeout_ns) ? 1 : 0;
 }
 
 // ---------------------------------------------------------------------------

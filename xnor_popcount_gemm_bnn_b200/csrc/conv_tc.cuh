@@ -1,0 +1,250 @@
+// Binary 3x3 convolution on the tensor cores: the implicit GEMM of conv.cuh
+// (M = output pixels, N = filters, K = 9 taps x C channels; "Extreme
+// Quantization: Binary, Ternary & 1-bit LLMs", eq. (4), (6), eq. (1) per
+// filter) computed with tcgen05.mma kind::i8 on +1/-1 bytes.
+//
+// Every product is +1 or -1 and the int32 accumulation is exact, so the
+// result equals 9*C - 2 * popcount over the gathered words.  Positions that
+// are padding in both operands -- channels past C inside a tap's words and
+// the words that round the row up to whole 128-element stages -- hold 0 bits
+// (+1) on both sides; each adds (+1)(+1), and the epilogue subtracts their
+// count KPAD - 9*C.  A tap outside the image is the all-zero word in the
+// activation only (+1 times the filter bit): a real term, as in conv.cuh.
+//
+// Design (sm_100a, one persistent CTA per SM, 9 warps):
+//  * The filters (N <= 256 rows of 9*CW words) are expanded once per CTA into
+//    shared memory in the K-major 128B-swizzled layout and stay resident.
+//  * warps 1-4: gather + unpack.  Thread r owns output pixel r of the tile:
+//    it loads its 9 taps x CW words from the packed NHWC activations (L2
+//    resident; padded taps read 0), then writes NS stages of 128 signed bytes
+//    into the tile's A buffer (two buffers: the next tile is gathered while
+//    the tensor cores work on this one).
+//  * warp 0: allocates TMEM (two 128 x N int32 accumulators) and one thread
+//    issues NS x 4 tcgen05.mma (M = 128, N, K = 32) per tile.
+//  * warps 5-8: epilogue.  Thread = output pixel, 32 filters per tcgen05.ld;
+//    the NCHW stores of a warp are 32 consecutive pixels of one filter plane.
+//  * Every wait is bounded; on time-out the CTA records BNN_ERR_DEVICE_TIMEOUT,
+//    the roles stop, the MMAs drain and TMEM is freed before exit.
+#pragma once
+
+#include "common.cuh"
+#include "conv.cuh"      // ConvEpilogue
+#include "gemm_tc.cuh"   // tcgen05 helpers, pm1_bytes, umma_desc_sw128
+
+namespace bnn {
+namespace ctc {
+constexpr int BM = 128;                    // output pixels per tile (TMEM lanes)
+constexpr int MAX_N = 256;
+constexpr int GATHER_WARPS = 4;
+constexpr int EPI_WARPS = 4;
+constexpr int WARP_MMA = 0, WARP_GATHER0 = 1, WARP_EPI0 = WARP_GATHER0 + GATHER_WARPS;
+constexpr int THREADS = (WARP_EPI0 + EPI_WARPS) * 32;   // 288
+constexpr int STAGE_A_BYTES = BM * 128;    // 16 KiB per 128-element stage
+}  // namespace ctc
+
+// Shared-memory bytes for CW words per tap and N (a multiple of 16) filter rows.
+__host__ __device__ constexpr int conv_tc_stages(int cw) { return (9 * cw + 3) / 4; }
+__host__ __device__ inline int conv_tc_smem_bytes(int cw, int n) {
+    const int ns = conv_tc_stages(cw);
+    return 2 * ns * ctc::STAGE_A_BYTES + ns * n * 128 + 16 * 8 + 16 + 1024;
+}
+
+// Writes 32 sign bits of a packed word as 32 signed bytes (+1 / -1) into two
+// 16-byte chunks (2q, 2q+1) of a 128-byte swizzled row.
+__device__ __forceinline__ void expand_word_sw128(uint8_t* row, int q, int sw, uint32_t w) {
+    const uint32_t lo = w & 0x0F0F0F0Fu;
+    const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;
+    uint4 c0, c1;
+    c0.x = pm1_bytes(__byte_perm(lo, 0u, 0x4440u));
+    c0.y = pm1_bytes(__byte_perm(hi, 0u, 0x4440u));
+    c0.z = pm1_bytes(__byte_perm(lo, 0u, 0x4441u));
+    c0.w = pm1_bytes(__byte_perm(hi, 0u, 0x4441u));
+    c1.x = pm1_bytes(__byte_perm(lo, 0u, 0x4442u));
+    c1.y = pm1_bytes(__byte_perm(hi, 0u, 0x4442u));
+    c1.z = pm1_bytes(__byte_perm(lo, 0u, 0x4443u));
+    c1.w = pm1_bytes(__byte_perm(hi, 0u, 0x4443u));
+    *reinterpret_cast<uint4*>(row + (((2 * q) ^ sw) << 4)) = c0;
+    *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ sw) << 4)) = c1;
+}
+
+template <int CW>
+__global__ void __launch_bounds__(ctc::THREADS, 1)
+xnor_conv3x3_tc_kernel(const uint32_t* __restrict__ X, int n, int c, int h, int w,
+                       const uint32_t* __restrict__ Wp, int64_t ldw, int cout, int n_mma, uint32_t idesc,
+                       int stride, int pad, int oh, int ow, ConvEpilogue ep) {
+    using namespace ctc;
+    constexpr int KW = 9 * CW;                  // real words per row
+    constexpr int NS = conv_tc_stages(CW);      // 128-element stages
+    constexpr int KWP = 4 * NS;                 // words per row incl. pad words
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t* abuf = smem;                                          // 2 x NS x 16 KiB
+    uint8_t* bsm = smem + 2 * NS * STAGE_A_BYTES;                  // NS x n_mma x 128 B
+    uint64_t* bars = reinterpret_cast<uint64_t*>(bsm + NS * n_mma * 128);
+    uint64_t* afill = bars;            // [2] A buffer gathered (count: gather warps)
+    uint64_t* accfull = afill + 2;     // [2] MMAs of the tile done (tcgen05.commit)
+    uint64_t* accempty = accfull + 2;  // [2] accumulator drained (count: epilogue warps)
+    uint64_t* drain = accempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t plane = (int64_t)oh * ow;
+    const int64_t npix = (int64_t)n * plane;
+    const int tiles = (int)((npix + BM - 1) / BM);
+    // Two accumulators at 32-column aligned offsets; the allocation is a power of 2.
+    const int acc_stride = (n_mma + 31) / 32 * 32;
+    const uint32_t tmem_cols = acc_stride <= 64 ? 128u : (acc_stride <= 128 ? 256u : 512u);
+
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&afill[b], GATHER_WARPS);
+            mbar_init(&accfull[b], 1);
+            mbar_init(&accempty[b], EPI_WARPS);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == WARP_MMA) {
+        tmem_alloc(tmem_slot, tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == WARP_MMA) {
+        // ------------------------------ MMA issuer ------------------------------
+        if (lane == 0) {
+            int lt = 0;
+            const uint32_t a0 = smem_u32(abuf), b0 = smem_u32(bsm);
+            for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++lt) {
+                const int b = lt & 1;
+                if (!tc_wait(&afill[b], (lt >> 1) & 1, abort_flag)) break;
+                if (lt >= 2 && !tc_wait(&accempty[b], ((lt >> 1) - 1) & 1, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(b * acc_stride);
+                #pragma unroll
+                for (int s = 0; s < NS; ++s) {
+                    #pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t ad = umma_desc_sw128(a0 + (b * NS + s) * STAGE_A_BYTES + kk * 32);
+                        const uint64_t bd = umma_desc_sw128(b0 + s * n_mma * 128 + kk * 32);
+                        asm volatile(
+                            "{\n\t.reg .pred p;\n\t"
+                            "setp.ne.b32 p, %4, 0;\n\t"
+                            "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+                            "l"(ad), "l"(bd), "r"(idesc), "r"((s | kk) != 0 ? 1u : 0u)
+                            : "memory");
+                    }
+                }
+                mma_commit(&accfull[b]);
+            }
+            mma_commit(drain);
+            mbar_wait_bounded(drain, 0);       // every MMA done before TMEM is freed
+        }
+        __syncwarp();
+    } else if (warp < WARP_EPI0) {
+        // --------------------------- gather + unpack warps ---------------------------
+        const int r = threadIdx.x - WARP_GATHER0 * 32;             // tile row 0..127
+        const int sw = r & 7;
+        // Filters first: rows r (and r + 128) of B, all stages, once per CTA.
+        for (int fr = r; fr < n_mma; fr += BM) {
+            uint32_t wd[KWP];
+            #pragma unroll
+            for (int k = 0; k < KWP; ++k) wd[k] = (fr < cout && k < KW) ? __ldg(Wp + (int64_t)fr * ldw + k) : 0u;
+            #pragma unroll
+            for (int s = 0; s < NS; ++s) {
+                uint8_t* row = bsm + s * n_mma * 128 + fr * 128;
+                #pragma unroll
+                for (int q = 0; q < 4; ++q) expand_word_sw128(row, q, fr & 7, wd[4 * s + q]);
+            }
+        }
+        int lt = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++lt) {
+            const int b = lt & 1;
+            // The A buffer is free once the MMAs of tile lt - 2 are done.
+            const bool ok = lt < 2 || tc_wait(&accfull[b], ((lt >> 1) - 1) & 1, abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            const int64_t q = (int64_t)t * BM + r;
+            int64_t bi = 0, oy = 0, ox = 0;
+            if (q < npix) {
+                bi = q / plane;
+                const int64_t rem = q % plane;
+                oy = rem / ow;
+                ox = rem % ow;
+            }
+            uint32_t wd[KWP];
+            #pragma unroll
+            for (int tap = 0; tap < 9; ++tap) {
+                const int iy = (int)oy * stride - pad + tap / 3;
+                const int ix = (int)ox * stride - pad + tap % 3;
+                const bool in = q < npix && iy >= 0 && iy < h && ix >= 0 && ix < w;
+                const int64_t off = in ? ((bi * h + iy) * (int64_t)w + ix) * CW : 0;
+                #pragma unroll
+                for (int j = 0; j < CW; ++j) wd[tap * CW + j] = in ? __ldg(X + off + j) : 0u;
+            }
+            #pragma unroll
+            for (int k = KW; k < KWP; ++k) wd[k] = 0u;
+            #pragma unroll
+            for (int s = 0; s < NS; ++s) {
+                uint8_t* row = abuf + (b * NS + s) * STAGE_A_BYTES + r * 128;
+                #pragma unroll
+                for (int qq = 0; qq < 4; ++qq) expand_word_sw128(row, qq, sw, wd[4 * s + qq]);
+            }
+            fence_proxy_async_shared();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&afill[b]);
+        }
+    } else {
+        // ------------------------------ epilogue warps ------------------------------
+        const int quad = warp & 3;
+        const int padc = NS * 128 - 9 * c;           // (+1)(+1) pad positions per output
+        int lt = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++lt) {
+            const int b = lt & 1;
+            if (!__all_sync(0xffffffffu, tc_wait(&accfull[b], (lt >> 1) & 1, abort_flag))) break;
+            tc_fence_after();
+            const int64_t q = (int64_t)t * BM + 32 * quad + lane;
+            const bool valid = q < npix;
+            const int64_t obase = valid ? (q / plane) * cout * plane + q % plane : 0;
+            for (int c0 = 0; c0 < n_mma; c0 += 32) {
+                uint32_t rr[32];
+                tmem_ld32(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * acc_stride + c0), rr);
+                tmem_ld_wait();
+                if (c0 + 32 >= n_mma) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&accempty[b]);
+                }
+                if (!valid) continue;
+                #pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int co = c0 + j;
+                    if (co >= cout) break;
+                    const int32_t sv = (int32_t)rr[j] - padc;
+                    const int64_t o = obase + (int64_t)co * plane;
+                    if (ep.mode == BNN_OUT_INT32) {
+                        static_cast<int32_t*>(ep.out)[o] = sv;
+                    } else {
+                        float y = __ldg(ep.alpha + co) * (float)sv;
+                        if (ep.mode == BNN_OUT_AFFINE_F32) y = fmaf(__ldg(ep.gamma + co), y, __ldg(ep.beta + co));
+                        static_cast<float*>(ep.out)[o] = y;
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == WARP_MMA) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, tmem_cols);
+    }
+}
+
+}  // namespace bnn
