@@ -52,6 +52,9 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # Dense int8 tensor throughput is twice dense bf16 (4.5 vs 2.25 PFLOP/s nominal);
 # the int8 peak used here is the measured bf16 peak times that ratio.
 INT8_PER_BF16 = 2.0
+# Whether AUTO runs the stride-1 convolution on the tensor cores (mirrors the
+# library's dispatch, for labelling the conv row's roofline).
+CONV_AUTO_TENSOR = False
 SM_COUNT = 148
 # 32-bit population count: 16 per clock per SM (CUDA arithmetic-instruction
 # throughput table); one POPC covers 32 binary multiply-accumulates.
@@ -107,7 +110,7 @@ KERNEL_SOURCES = {
     "xnor_gemm_tc_kernel": ("gemm_tc.cuh", "gemm_popc.cuh", "common.cuh"),
     "xnor_gemm_popc_kernel": ("gemm_popc.cuh", "common.cuh"),
     "xnor_conv3x3_kernel": ("conv.cuh", "common.cuh"),
-    "xnor_conv3x3_tc_kernel": ("conv_tc.cuh", "conv.cuh", "gemm_tc.cuh", "gemm_popc.cuh", "common.cuh"),
+    "xnor_conv3x3_tcw_kernel": ("conv_tc.cuh", "conv.cuh", "gemm_tc.cuh", "gemm_popc.cuh", "common.cuh"),
     "pack_sign_rows_kernel": ("pack.cuh", "common.cuh"),
 }
 
@@ -279,9 +282,17 @@ def run_ours(args, torch, dist):
     copies = (copies + 7) // 8 * 8                       # 48
     g, Ws, alpha, x, y = gemv_setup(torch, bnn, workloads, dev, copies)
 
-    # Decode: the weights are resident model parameters, so the GEMV may start
-    # streaming them before the previous step's kernel has finished.
+    # Every step's inputs (packed W, x, alpha) are resident before the timed
+    # region and no step reads another's output, so each GEMV may stream its
+    # weights, pack x and form the product while the previous one finishes;
+    # only its store of y waits for the previous kernel (stream order on y).
     def step(i):
+        bnn.bnn_xnor_gemv_ex(Ws[i % copies], x, g.K, alpha, None, y,
+                             flags=bnn.BNN_GEMV_WEIGHTS_STATIC | bnn.BNN_GEMV_INPUTS_STATIC)
+
+    # A decode chain where x is the previous kernel's output: only the weight
+    # stream may start before the previous kernel has finished.
+    def step_dep(i):
         bnn.bnn_xnor_gemv_ex(Ws[i % copies], x, g.K, alpha, None, y, flags=bnn.BNN_GEMV_WEIGHTS_STATIC)
 
     def step_plain(i):
@@ -290,8 +301,9 @@ def run_ours(args, torch, dist):
     with ClockSampler(local) as clk:
         ms = time_steps(torch, step, args.steps, args.warmup, copies, sync)
     ms = max_over_ranks(ms)
-    plain_steps = min(args.steps, 48 * copies)
-    ms_plain = max_over_ranks(time_steps(torch, step_plain, plain_steps, args.warmup, copies, sync))
+    side_steps = min(args.steps, 48 * copies)
+    ms_dep = max_over_ranks(time_steps(torch, step_dep, side_steps, args.warmup, copies, sync))
+    ms_plain = max_over_ranks(time_steps(torch, step_plain, side_steps, args.warmup, copies, sync))
     if bnn.bnn_device_error() != 0:
         raise RuntimeError("a kernel reported a device-side timeout")
     per_step_bytes = gemv_bytes()
@@ -334,10 +346,17 @@ def run_ours(args, torch, dist):
         },
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
+        "flags": "BNN_GEMV_WEIGHTS_STATIC | BNN_GEMV_INPUTS_STATIC (independent steps over resident inputs)",
+        "dependent_chain": {
+            "value": round(ws * side_steps * per_step_bytes / (ms_dep * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "steps": side_steps, "ms_per_step": ms_dep / side_steps,
+            "frac": round(side_steps * per_step_bytes / (ms_dep * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+            "note": "BNN_GEMV_WEIGHTS_STATIC only: x and alpha are read after the wait for the previous "
+                    "kernel, as when x is the previous layer's output"},
         "gemv_default_flags": {
-            "value": round(ws * plain_steps * per_step_bytes / (ms_plain * 1e-3) / 1e9, 2), "unit": "GB/s",
-            "steps": plain_steps, "ms_per_step": ms_plain / plain_steps,
-            "note": "bnn_xnor_gemv without the static-weights flag: W is read after the dependency wait"},
+            "value": round(ws * side_steps * per_step_bytes / (ms_plain * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "steps": side_steps, "ms_per_step": ms_plain / side_steps,
+            "note": "bnn_xnor_gemv (no flags): W, x and alpha are read after the wait for the previous kernel"},
     }
 
     # e2e: the public API with host buffers
@@ -506,37 +525,44 @@ def _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk):
     # --- a2 (NCHW) + a5 + a6: ResNet-class binary 3x3 conv with affine epilogue ---
     cv = workloads.conv()
     n, c, h, w = cv.X.shape
-    Xd = cv.X.to(dev)
-    Xb = bnn.empty_packed_nhwc(n, c, h, w, dev)
+    # Three rotating sets of (bf16 input, packed input, fp32 output), 235 MB
+    # in all, so that consecutive steps do not find their data in the 126 MB L2.
+    R = 3
+    Xd = [cv.X.to(dev) for _ in range(R)]
+    Xb = [bnn.empty_packed_nhwc(n, c, h, w, dev) for _ in range(R)]
+    out = [torch.empty(n, 64, h, w, dtype=torch.float32, device=dev) for _ in range(R)]
     Wc = bnn.empty_conv3x3_weights(64, c, dev)
     alc = torch.empty(64, dtype=torch.float32, device=dev)
     bnn.bnn_pack_conv3x3_weights(cv.W.to(dev), Wc, alc)
     gam, bet = cv.gamma.to(dev), cv.beta.to(dev)
-    out = torch.empty(n, 64, h, w, dtype=torch.float32, device=dev)
     ep = bnn.make_epilogue(bnn.BNN_OUT_AFFINE_F32, alpha=alc, gamma=gam, beta=bet)
+    rot_mb = R * (Xd[0].numel() * 2 + Xb[0].numel() * 4 + out[0].numel() * 4) / 1e6
 
     def conv_step(i):
-        bnn.bnn_pack_sign_nchw(Xd, Xb)
-        bnn.bnn_binary_conv3x3_fused(Xb, c, Wc, ep, out, 1, 1)
+        bnn.bnn_pack_sign_nchw(Xd[i % R], Xb[i % R])
+        bnn.bnn_binary_conv3x3_fused(Xb[i % R], c, Wc, ep, out[i % R], 1, 1)
 
     cmacs = n * h * w * 64 * 9 * c
     # Algorithmic bytes of one conv launch: packed activations and filters in,
     # fp32 NCHW out (alpha/gamma/beta are 768 B).
-    cbytes = Xb.numel() * 4 + Wc.numel() * 4 + out.numel() * 4
-    for name, engine in (("conv3x3", bnn.BNN_GEMM_ENGINE_POPCOUNT), ("conv3x3_tensor", bnn.BNN_GEMM_ENGINE_TENSOR)):
+    cbytes = Xb[0].numel() * 4 + Wc.numel() * 4 + out[0].numel() * 4
+    for i in range(R):
+        bnn.bnn_pack_sign_nchw(Xd[i], Xb[i])
+    for name, engine in (("conv3x3", bnn.BNN_GEMM_ENGINE_AUTO), ("conv3x3_tensor", bnn.BNN_GEMM_ENGINE_TENSOR),
+                         ("conv3x3_popcount", bnn.BNN_GEMM_ENGINE_POPCOUNT)):
         with bnn.gemm_engine(engine):
             ms_c = timed(conv_step)
-            bnn.bnn_pack_sign_nchw(Xd, Xb)
-            ms_ck = timed(lambda i: bnn.bnn_binary_conv3x3_fused(Xb, c, Wc, ep, out, 1, 1))
+            ms_ck = timed(lambda i: bnn.bnn_binary_conv3x3_fused(Xb[i % R], c, Wc, ep, out[i % R], 1, 1))
         cmac_s = cmacs * steps / (ms_ck * 1e-3)
-        if engine == bnn.BNN_GEMM_ENGINE_TENSOR:
+        tensor = engine == bnn.BNN_GEMM_ENGINE_TENSOR or (engine == bnn.BNN_GEMM_ENGINE_AUTO and CONV_AUTO_TENSOR)
+        if tensor:
             # The fp32 output write bounds this kernel: 51 MB out against 7.4 G
             # binary MACs, 8 us of HBM time versus under 5 us of int8 tensor time.
             ach = cbytes * steps / (ms_ck * 1e-3) / 1e9
             roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                     "frac": round(ach / pk["hbm_gbs"], 4), "algorithmic_bytes": cbytes,
                     "tensor": _tensor_roofline(pk, cmac_s, sustained=False),
-                    "traffic": recorded_traffic("xnor_conv3x3_tc_kernel")}
+                    "traffic": recorded_traffic("xnor_conv3x3_tcw_kernel")}
             roof["tensor"].pop("traffic")
         else:
             roof = {"bound": "alu", "achieved": round(cmac_s / 1e12, 2), "peak": round(alu_peak / 1e12, 2),
@@ -544,11 +570,13 @@ def _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk):
                     "traffic": recorded_traffic("xnor_conv3x3_kernel")}
         rows[name] = {
             "workload": "bf16 [64,64,56,56] -> pack NCHW -> binary 3x3 conv (64 filters, stride 1, pad 1), "
-                        "alpha + affine epilogue, fp32 NCHW out"
-                        + (" (tensor-core engine)" if engine == bnn.BNN_GEMM_ENGINE_TENSOR else " (popcount engine)"),
+                        "alpha + affine epilogue, fp32 NCHW out",
+            "engine": {bnn.BNN_GEMM_ENGINE_AUTO: "auto", bnn.BNN_GEMM_ENGINE_TENSOR: "tensor",
+                       bnn.BNN_GEMM_ENGINE_POPCOUNT: "popcount"}[engine] + (" (tensor cores)" if tensor else " (popcount)"),
             "value": round(ws * cmacs * steps / (ms_c * 1e-3) / 1e9, 1), "unit": "binary GMAC/s",
             "ms_per_step": ms_c / steps, "conv_kernel_ms": ms_ck / steps,
-            "conv_kernel_binary_tmac_s": round(cmac_s / 1e12, 2), "roofline": roof}
+            "conv_kernel_binary_tmac_s": round(cmac_s / 1e12, 2), "roofline": roof,
+            "l2": f"{R} rotating input/output sets, {rot_mb:.0f} MB"}
     del cv, Xd, Xb, Wc, alc, gam, bet, out
     torch.cuda.empty_cache()
 
@@ -557,9 +585,12 @@ def _row_mlp(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk=No
     # --- MLP: pack input, 3 x (GEMM + folded-BN re-pack), GEMM + alpha ---
     m = workloads.mlp()
     B, D = m.X0.shape
-    X0 = m.X0.to(dev)
-    A0 = bnn.empty_packed(B, D, dev)
-    acts = [bnn.empty_packed(B, D, dev) for _ in range(3)]
+    # Two rotating sets of (fp32 input, packed activations, fp32 logits), 270 MB
+    # in all, so that consecutive steps do not find their data in the 126 MB L2.
+    R = 2
+    X0 = [m.X0.to(dev) for _ in range(R)]
+    A0 = [bnn.empty_packed(B, D, dev) for _ in range(R)]
+    acts = [[bnn.empty_packed(B, D, dev) for _ in range(3)] for _ in range(R)]
     eps_ = []
     Wps = []
     for l, W in enumerate(m.Ws):
@@ -574,13 +605,15 @@ def _row_mlp(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk=No
             eps_.append((bnn.make_epilogue(bnn.BNN_OUT_THRESHOLD_PACK, popc_thresh=thr, thresh_mode=mode), thr, mode))
         else:
             eps_.append((bnn.make_epilogue(bnn.BNN_OUT_SCALED_F32, alpha=a), a))
-    logits = torch.empty(B, D, dtype=torch.float32, device=dev)
+    logits = [torch.empty(B, D, dtype=torch.float32, device=dev) for _ in range(R)]
+    rot_mb = R * (X0[0].numel() * 4 + 4 * A0[0].numel() * 4 + logits[0].numel() * 4) / 1e6
 
     def mlp_step(i):
-        bnn.bnn_pack_sign(X0, A0)
-        A = A0
+        r = i % R
+        bnn.bnn_pack_sign(X0[r], A0[r])
+        A = A0[r]
         for l in range(4):
-            o = acts[l] if l < 3 else logits
+            o = acts[r][l] if l < 3 else logits[r]
             bnn.bnn_binary_linear_fused(A, Wps[l], D, eps_[l][0], o)
             A = o
 
@@ -597,7 +630,8 @@ def _row_mlp(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk=No
                         "3 x (GEMM + folded BatchNorm sign re-pack), GEMM + alpha fp32 logits",
             "engine": "tensor" if engine == bnn.BNN_GEMM_ENGINE_TENSOR else "popcount",
             "value": round(ws * mac_s / 1e9, 1), "unit": "binary GMAC/s",
-            "ms_per_step": ms_m / steps, "roofline": roof}
+            "ms_per_step": ms_m / steps, "roofline": roof,
+            "l2": f"{R} rotating input/activation/logit sets, {rot_mb:.0f} MB"}
     del m, X0, A0, acts, eps_, Wps, logits
     torch.cuda.empty_cache()
 

@@ -232,7 +232,8 @@ bnn_status bnn_xnor_gemv(const uint32_t* W, int64_t ldw, const void* x, bnn_dtyp
 
 /* Flags of bnn_xnor_gemv_ex. */
 typedef enum bnn_gemv_flags {
-    BNN_GEMV_WEIGHTS_STATIC = 1   /* W is not written by any work still in flight on the stream */
+    BNN_GEMV_WEIGHTS_STATIC = 1,  /* W is not written by any work still in flight on the stream */
+    BNN_GEMV_INPUTS_STATIC = 2    /* x and alpha are not written by any work still in flight */
 } bnn_gemv_flags;
 
 /* bnn_xnor_gemv_ex -- bnn_xnor_gemv with flags.  Both calls launch the kernel
@@ -243,7 +244,13 @@ typedef enum bnn_gemv_flags {
  * consecutive GEMVs over resident weights (one decode step through many
  * layers) stream their weights back to back.  The caller guarantees that no
  * earlier work on the stream that may still be running writes W; otherwise
- * pass 0 (then equivalent to bnn_xnor_gemv).
+ * pass 0 (then equivalent to bnn_xnor_gemv).  With BNN_GEMV_INPUTS_STATIC
+ * (the caller guarantees the same for x and alpha) x is packed before the
+ * wait as well; with both flags the whole product is computed before it and
+ * only the store of y waits, so GEMVs over independent, resident inputs
+ * overlap their prologues with the previous kernel.  A flag is a permission:
+ * shapes served by the general kernel (rows of more than 128 words, or x not
+ * 16-byte aligned) ignore BNN_GEMV_INPUTS_STATIC.
  *   Errors: as bnn_xnor_gemv; INVALID_ARG for unknown flag bits. */
 bnn_status bnn_xnor_gemv_ex(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt,
                             int64_t N, int64_t K, const float* alpha,

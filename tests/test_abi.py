@@ -114,8 +114,10 @@ def test_gemv_rejects_bad_arguments():
 
 def test_gemv_ex_rejects_bad_flags():
     g = L.bnn_xnor_gemv_ex
-    assert g(FAKE, 4, FAKE, 0, 8, 32, NULL, FAKE, NULL, 2, NULL) == bnn.BNN_ERR_INVALID_ARG
-    assert g(FAKE, 4, FAKE, 0, 0, 32, NULL, FAKE, NULL, 1, NULL) == bnn.BNN_OK
+    assert g(FAKE, 4, FAKE, 0, 8, 32, NULL, FAKE, NULL, 4, NULL) == bnn.BNN_ERR_INVALID_ARG
+    assert g(FAKE, 4, FAKE, 0, 8, 32, NULL, FAKE, NULL, 7, NULL) == bnn.BNN_ERR_INVALID_ARG
+    for flags in (1, 2, 3):
+        assert g(FAKE, 4, FAKE, 0, 0, 32, NULL, FAKE, NULL, flags, NULL) == bnn.BNN_OK
 
 
 def test_conv_rejects_bad_arguments():

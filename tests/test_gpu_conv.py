@@ -43,7 +43,7 @@ CASES = [(2, 64, 9, 7, 5, 1, 1), (1, 3, 5, 6, 4, 1, 1), (2, 33, 8, 8, 3, 2, 1), 
          (3, 100, 7, 9, 17, 1, 1), (1, 128, 6, 6, 8, 1, 1), (2, 64, 56, 56, 64, 1, 1), (1, 40, 11, 13, 6, 2, 0),
          # tensor-core shapes: filter counts off the 16/32 grid, 256 filters, ragged last tile
          (3, 50, 19, 17, 40, 1, 1), (1, 20, 9, 9, 48, 1, 1), (2, 32, 12, 12, 256, 1, 1), (1, 64, 10, 10, 200, 1, 1),
-         (1, 1, 5, 5, 1, 1, 1), (5, 64, 33, 31, 96, 2, 1)]
+         (1, 1, 5, 5, 1, 1, 1), (5, 64, 33, 31, 96, 2, 1), (1, 16, 6, 7, 8, 1, 2)]
 
 
 @pytest.mark.parametrize("n,c,h,w,cout,stride,pad", CASES)
@@ -81,4 +81,29 @@ def test_resnet_layer_workload_sampled_images(engine):
     scale = (np.abs(cv.gamma.numpy().astype(np.float64)[None, :, None, None] * a_ref[None, :, None, None]
                     * s_ref) + np.abs(cv.beta.numpy().astype(np.float64))[None, :, None, None])
     assert_affine_close(out[imgs], y_ref, scale)
+    assert_no_device_error()
+
+
+@pytest.mark.parametrize("n,c,h,w,cout", [(1, 128, 170, 340, 16), (1, 20, 40, 1680, 16)])
+def test_conv_window_segments(n, c, h, w, cout):
+    """Wide images: the 2*(w+2)+2 halo leaves room for one 128-position tile
+    per shared-memory buffer, so the stride-1 tensor-core kernel walks each
+    CTA's 3-4 tiles as separate segments and reuses both buffers.  INT32 and
+    affine outputs against the oracle, and the popcount engine bit for bit."""
+    X = workloads.normal((n, c, h, w), 1.0, w, dtype=torch.bfloat16)
+    Wt = workloads.normal((cout, c, 3, 3), 0.1, c)
+    g = workloads.uniform((cout,), 0.5, 1.5, cout)
+    b = workloads.normal((cout,), 0.1, cout + 1)
+    with bnn.gemm_engine(bnn.BNN_GEMM_ENGINE_TENSOR):
+        out_i = run_conv(X, Wt, None, None, 1, 1, bnn.BNN_OUT_INT32)
+        out_a = run_conv(X, Wt, g, b, 1, 1, bnn.BNN_OUT_AFFINE_F32)
+    with bnn.gemm_engine(bnn.BNN_GEMM_ENGINE_POPCOUNT):
+        out_p = run_conv(X, Wt, None, None, 1, 1, bnn.BNN_OUT_INT32)
+    s_ref, y_ref = oracle.conv3x3_affine(X, Wt, g.numpy(), b.numpy(), 1, 1)
+    assert np.array_equal(out_i.cpu().numpy(), s_ref)
+    assert torch.equal(out_i, out_p)
+    a_ref = oracle.alpha(Wt.reshape(cout, -1))
+    scale = (np.abs(g.numpy().astype(np.float64)[None, :, None, None] * a_ref[None, :, None, None] * s_ref)
+             + np.abs(b.numpy().astype(np.float64))[None, :, None, None])
+    assert_affine_close(out_a, y_ref, scale)
     assert_no_device_error()

@@ -148,4 +148,54 @@ def test_gemv_ex_rejects_unknown_flags():
     x = torch.zeros(64, device=dev())
     y = torch.empty(8, dtype=torch.int32, device=dev())
     with pytest.raises(bnn.BnnError):
-        bnn.bnn_xnor_gemv_ex(W, x, 64, None, y, None, flags=2)
+        bnn.bnn_xnor_gemv_ex(W, x, 64, None, y, None, flags=4)
+
+
+@pytest.mark.parametrize("use_graph", [False, True])
+def test_static_inputs_independent_gemvs(use_graph):
+    """BNN_GEMV_WEIGHTS_STATIC | BNN_GEMV_INPUTS_STATIC on independent GEMVs
+    over resident inputs: each result exact; consecutive calls that write the
+    same y keep stream order (the last call's values remain)."""
+    N, K, L = 1000, 4000, 6
+    d = dev()
+    Ws = [workloads.normal((N, K), 1.0, 700 + l) for l in range(L)]
+    xs = [workloads.normal((K,), 1.0, 800 + l, dtype=torch.bfloat16) for l in range(L)]
+    Wp, al = [], []
+    for W in Ws:
+        p = bnn.empty_packed(N, K, d)
+        a = torch.empty(N, dtype=torch.float32, device=d)
+        bnn.bnn_pack_sign(W.to(d), p, a)
+        Wp.append(p)
+        al.append(a)
+    xd = [x.to(d) for x in xs]
+    ys = [torch.empty(N, dtype=torch.int32, device=d) for _ in range(L)]
+    y_shared = torch.empty(N, dtype=torch.int32, device=d)
+    flags = bnn.BNN_GEMV_WEIGHTS_STATIC | bnn.BNN_GEMV_INPUTS_STATIC
+    torch.cuda.synchronize()
+
+    def run():
+        for l in range(L):
+            bnn.bnn_xnor_gemv_ex(Wp[l], xd[l], K, al[l], ys[l], None, flags=flags)
+        for l in range(L):
+            bnn.bnn_xnor_gemv_ex(Wp[l], xd[l], K, al[l], y_shared, None, flags=flags)
+
+    if use_graph:
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            run()
+        torch.cuda.current_stream().wait_stream(s)
+        with torch.cuda.graph(g):
+            run()
+        for t in ys + [y_shared]:
+            t.fill_(-7)
+        g.replay()
+    else:
+        run()
+    torch.cuda.synchronize()
+    for l in range(L):
+        ref = oracle.gemv_pm1(oracle.sign_pm1(Ws[l]), oracle.sign_pm1(xs[l]))
+        assert np.array_equal(ys[l].cpu().numpy(), ref), f"gemv {l}"
+    assert torch.equal(y_shared, ys[L - 1])
+    assert_no_device_error()

@@ -89,7 +89,8 @@ def expected_nhwc(x):
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("shape", [(2, 64, 5, 7), (2, 33, 8, 8), (1, 1, 3, 3), (3, 100, 4, 6),
-                                   (2, 64, 56, 56)])
+                                   (2, 64, 56, 56), (2, 48, 6, 4), (1, 17, 4, 4), (3, 70, 5, 9),
+                                   (2, 300, 9, 16), (1, 520, 4, 8), (3, 32, 40, 40), (1, 5, 1, 8)])
 def test_pack_sign_nchw(shape, dtype):
     n, c, h, w = shape
     x = workloads.random_with_edges(n * c, h * w, seed=sum(shape), dtype=dtype).reshape(shape).contiguous()

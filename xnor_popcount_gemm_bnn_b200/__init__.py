@@ -35,6 +35,7 @@ BNN_OUT_AFFINE_F32 = 4
 BNN_OUT_THRESHOLD_PACK = 8
 
 BNN_GEMV_WEIGHTS_STATIC = 1
+BNN_GEMV_INPUTS_STATIC = 2
 
 BNN_GEMM_ENGINE_AUTO = 0
 BNN_GEMM_ENGINE_POPCOUNT = 1

@@ -95,6 +95,24 @@ bool gemm_tc_smem_configured() {
     return true;
 }
 
+// Per-device one-time opt-in to the TMA-staged NCHW pack's shared memory
+// (3 stages of up to 48 KB).
+bool pack_nchw_smem_configured() {
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> done[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+    if (dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return true;
+    const int bytes = bnn::pk::STAGES * 48 * 1024 + 128;
+    if (cudaFuncSetAttribute(bnn::pack_sign_nchw_tma_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(bnn::pack_sign_nchw_tma_kernel<__nv_bfloat16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return false;
+    if (dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
+    return true;
+}
+
 std::atomic<int> g_gemm_engine{BNN_GEMM_ENGINE_AUTO};
 
 int sm_count() {
@@ -168,7 +186,7 @@ bnn_status check_gemm_dims(int64_t M, int64_t N, int64_t K) {
 template <typename XT>
 bnn_status launch_gemv_t(const uint32_t* W, int64_t ldw, const XT* x, int64_t N, int64_t K, int64_t kw,
                          const float* alpha, int32_t* y_i32, float* y_f32, bool weights_static,
-                         cudaStream_t stream) {
+                         bool inputs_static, cudaStream_t stream) {
     using namespace bnn::gemv;
     const int64_t nchunks = kw / 4;
     int lpr = 1;
@@ -204,7 +222,8 @@ bnn_status launch_gemv_t(const uint32_t* W, int64_t ldw, const XT* x, int64_t N,
     if (lpr == 32 && single && vec) {
         // Rows of 97..128 words: the dedicated one-chunk-per-lane kernel.
         auto kern = bnn::xnor_gemv_row128_kernel<XT>;
-        e = cudaLaunchKernelEx(&cfg, kern, W, ldw, x, iN, iK, ikw, alpha, y_i32, y_f32, weights_static ? 1 : 0, 1);
+        e = cudaLaunchKernelEx(&cfg, kern, W, ldw, x, iN, iK, ikw, alpha, y_i32, y_f32, weights_static ? 1 : 0,
+                               inputs_static ? 1 : 0, 1);
         if (e != cudaSuccess) return BNN_ERR_CUDA;
         return launch_status();
     }
@@ -237,7 +256,7 @@ constexpr int64_t kGemvMaxWords = 48 * 1024;   // packed x in shared memory: <= 
 
 bnn_status gemv_impl(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt, int64_t N, int64_t K,
                      const float* alpha, int32_t* y_i32, float* y_f32, bool weights_static,
-                     bnn_stream_t stream) {
+                     bool inputs_static, bnn_stream_t stream) {
     if (N < 0 || K < 1 || N > INT_MAX || K > INT_MAX / 2) return BNN_ERR_INVALID_ARG;
     if (x == nullptr || (y_i32 == nullptr && y_f32 == nullptr)) return BNN_ERR_INVALID_ARG;
     if (y_f32 != nullptr && alpha == nullptr) return BNN_ERR_INVALID_ARG;
@@ -250,9 +269,9 @@ bnn_status gemv_impl(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_
     if (N == 0) return BNN_OK;
     if (x_dt == BNN_F32)
         return launch_gemv_t(W, ldw, static_cast<const float*>(x), N, K, kw, alpha, y_i32, y_f32,
-                             weights_static, as_cuda(stream));
+                             weights_static, inputs_static, as_cuda(stream));
     return launch_gemv_t(W, ldw, static_cast<const __nv_bfloat16*>(x), N, K, kw, alpha, y_i32, y_f32,
-                         weights_static, as_cuda(stream));
+                         weights_static, inputs_static, as_cuda(stream));
 }
 
 }  // namespace
@@ -344,16 +363,49 @@ bnn_status bnn_pack_sign_nchw(const void* x, bnn_dtype dt, int64_t n, int64_t c,
     if (!aligned(x, es) || !aligned(packed_nhwc, 4)) return BNN_ERR_ALIGNMENT;
     if (n == 0) return BNN_OK;
     const int64_t hw = h * w, cw = (c + 31) / 32;
-    const int64_t threads = n * ceil_div(hw, 8) * cw;
-    const int64_t blocks = ceil_div(threads, 256);
+    cudaStream_t s = as_cuda(stream);
+    // TMA-staged path: rows of hw elements 16-byte aligned, chunks of px pixels
+    // x all channels of at most 48 KB per stage.
+    {
+        const int64_t nbox = ceil_div(c, 256), cb = ceil_div(c, nbox);
+        int64_t px = es == 2 ? 256 : 128;
+        while ((nbox * cb * px * (int64_t)es > 48 * 1024 || px / 2 >= hw) && px * (int64_t)es > 128) px /= 2;
+        const int64_t stage = nbox * cb * px * (int64_t)es;
+        if (aligned(x, 16) && (hw * (int64_t)es) % 16 == 0 && stage <= 48 * 1024 && n * c <= INT_MAX &&
+            hw <= INT_MAX / 2 && n * ceil_div(hw, px) <= INT_MAX && pack_nchw_smem_configured()) {
+            auto enc = tensor_map_encoder();
+            CUtensorMap tm;
+            cuuint64_t dims[2] = {(cuuint64_t)hw, (cuuint64_t)(n * c)};
+            cuuint64_t strides[1] = {(cuuint64_t)(hw * (int64_t)es)};
+            cuuint32_t box[2] = {(cuuint32_t)px, (cuuint32_t)cb};
+            cuuint32_t estr[2] = {1, 1};
+            if (enc == nullptr ||
+                enc(&tm, dt == BNN_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                    const_cast<void*>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return BNN_ERR_CUDA;
+            const int64_t chunks = n * ceil_div(hw, px);
+            const int64_t grid = std::min<int64_t>(chunks, 2 * (int64_t)sm_count());
+            const int smem = (int)(bnn::pk::STAGES * stage + 128);
+            if (dt == BNN_F32)
+                bnn::pack_sign_nchw_tma_kernel<float><<<(unsigned)grid, bnn::pk::THREADS, smem, s>>>(
+                    tm, (int)n, (int)c, (int)hw, (int)cw, (int)px, (int)cb, (int)nbox, packed_nhwc);
+            else
+                bnn::pack_sign_nchw_tma_kernel<__nv_bfloat16><<<(unsigned)grid, bnn::pk::THREADS, smem, s>>>(
+                    tm, (int)n, (int)c, (int)hw, (int)cw, (int)px, (int)cb, (int)nbox, packed_nhwc);
+            return launch_status();
+        }
+    }
+    const int64_t threads = n * ceil_div(hw, 8) * cw * 2;
+    const int64_t blocks = ceil_div(threads, 128);
     if (blocks > INT_MAX) return BNN_ERR_INVALID_ARG;
     const bool vec_ok = aligned(x, 16) && (hw % 8 == 0);
-    cudaStream_t s = as_cuda(stream);
     if (dt == BNN_F32)
-        bnn::pack_sign_nchw_kernel<float><<<(unsigned)blocks, 256, 0, s>>>(static_cast<const float*>(x), n, c, hw,
+        bnn::pack_sign_nchw_kernel<float><<<(unsigned)blocks, 128, 0, s>>>(static_cast<const float*>(x), n, c, hw,
                                                                            cw, packed_nhwc, vec_ok);
     else
-        bnn::pack_sign_nchw_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
+        bnn::pack_sign_nchw_kernel<__nv_bfloat16><<<(unsigned)blocks, 128, 0, s>>>(
             static_cast<const __nv_bfloat16*>(x), n, c, hw, cw, packed_nhwc, vec_ok);
     return launch_status();
 }
@@ -403,14 +455,15 @@ bnn_status bnn_xnor_gemm(const uint32_t* A, int64_t lda, const uint32_t* W, int6
 
 bnn_status bnn_xnor_gemv(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt, int64_t N, int64_t K,
                          const float* alpha, int32_t* y_i32, float* y_f32, bnn_stream_t stream) {
-    return gemv_impl(W, ldw, x, x_dt, N, K, alpha, y_i32, y_f32, false, stream);
+    return gemv_impl(W, ldw, x, x_dt, N, K, alpha, y_i32, y_f32, false, false, stream);
 }
 
 bnn_status bnn_xnor_gemv_ex(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt, int64_t N, int64_t K,
                             const float* alpha, int32_t* y_i32, float* y_f32, uint32_t flags,
                             bnn_stream_t stream) {
-    if ((flags & ~(uint32_t)BNN_GEMV_WEIGHTS_STATIC) != 0) return BNN_ERR_INVALID_ARG;
+    if ((flags & ~(uint32_t)(BNN_GEMV_WEIGHTS_STATIC | BNN_GEMV_INPUTS_STATIC)) != 0) return BNN_ERR_INVALID_ARG;
     return gemv_impl(W, ldw, x, x_dt, N, K, alpha, y_i32, y_f32, (flags & BNN_GEMV_WEIGHTS_STATIC) != 0,
+                     (flags & BNN_GEMV_INPUTS_STATIC) != 0,
                      stream);
 }
 
@@ -460,6 +513,31 @@ bnn_status bnn_binary_linear_fused(const uint32_t* A, int64_t lda, const uint32_
     return dispatch_gemm(A, lda, W, ldw, M, N, K, ep, as_cuda(stream));
 }
 
+// Geometry of the shifted-window convolution (stride 1): the virtual line of
+// padded positions, its 128-position tiles, and the rows per A buffer that
+// fit in shared memory next to the resident filters.  BNN_ERR_UNSUPPORTED
+// when a buffer cannot hold one tile's window.
+static bnn_status conv_window_plan(int64_t n, int64_t h, int64_t w, int64_t pad, int64_t cw, int64_t n_mma,
+                                   bnn::ConvWindow* g) {
+    const int64_t Hp = h + 2 * pad, Wp = w + 2 * pad;
+    const int64_t V = n * Hp * Wp;
+    const int64_t halo = 2 * Wp + 2;
+    if (V + 2 * halo + 256 > INT_MAX) return BNN_ERR_UNSUPPORTED;
+    const int64_t tiles = ceil_div(V, (int64_t)bnn::ctw::BM);
+    const int64_t fixed = bnn::conv_tcw_smem_bytes((int)cw, (int)n_mma, 0);
+    int64_t rb = (227 * 1024 - fixed) / (2 * cw * 32);
+    rb = std::min<int64_t>(rb, 16000) / 8 * 8;
+    const int64_t grid = std::min<int64_t>(tiles, sm_count());
+    const int64_t per_cta = ceil_div(tiles, grid);
+    rb = std::min<int64_t>(rb, ceil_div(per_cta * bnn::ctw::BM + halo, (int64_t)8) * 8);
+    if (rb < bnn::ctw::BM + halo) return BNN_ERR_UNSUPPORTED;
+    g->n = (int)n; g->h = (int)h; g->w = (int)w; g->pad = (int)pad;
+    g->Hp = (int)Hp; g->Wp = (int)Wp; g->oh = (int)(Hp - 2); g->ow = (int)(Wp - 2);
+    g->V = (int)V; g->tiles = (int)tiles; g->rb = (int)rb; g->halo = (int)halo;
+    g->seg_tiles = (int)((rb - halo) / bnn::ctw::BM);
+    return BNN_OK;
+}
+
 bnn_status bnn_binary_conv3x3_fused(const uint32_t* X_nhwc_bits, int64_t n, int64_t c, int64_t h, int64_t w,
                                     const uint32_t* W_packed, int64_t ldw, int64_t cout, int64_t stride, int64_t pad,
                                     const bnn_epilogue* epi, void* out_nchw, bnn_stream_t stream) {
@@ -492,11 +570,37 @@ bnn_status bnn_binary_conv3x3_fused(const uint32_t* X_nhwc_bits, int64_t n, int6
     const int64_t npix = n * oh * ow;
     bnn::ConvEpilogue ep{epi->mode, epi->alpha, epi->gamma, epi->beta, out_nchw};
     cudaStream_t s = as_cuda(stream);
-    // Tensor-core engine (when forced): up to 2 words per pixel per tap
-    // (c <= 64) and 256 filters, when the resident filters and two A tiles fit
-    // in shared memory.
     const int engine = g_gemm_engine.load(std::memory_order_relaxed);
     const int64_t n_mma = std::max<int64_t>(16, ceil_div(cout, (int64_t)16) * 16);
+    // Tensor cores, stride 1: the shifted-window kernel, when the resident
+    // filters and two A buffers of at least one tile's window fit.
+    if (engine == BNN_GEMM_ENGINE_TENSOR && stride == 1 && cout <= bnn::ctc::MAX_N) {
+        bnn::ConvWindow g{};
+        const bnn_status st = conv_window_plan(n, h, w, pad, cw, n_mma, &g);
+        if (st == BNN_OK) {
+            const int smem_w = bnn::conv_tcw_smem_bytes((int)cw, (int)n_mma, g.rb);
+            const uint32_t idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n_mma >> 3) << 17) |
+                                   ((uint32_t)(bnn::ctw::BM >> 4) << 24);
+            const int grid = std::min(g.tiles, sm_count());
+            auto launch_w = [&](auto kern) -> bnn_status {
+                if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_w) != cudaSuccess)
+                    return BNN_ERR_CUDA;
+                kern<<<(unsigned)grid, bnn::ctw::THREADS, smem_w, s>>>(X_nhwc_bits, (int)c, W_packed, ldw, (int)cout,
+                                                                       (int)n_mma, idesc, g, ep);
+                return launch_status();
+            };
+            switch (cw) {
+                case 1: return launch_w(bnn::xnor_conv3x3_tcw_kernel<1>);
+                case 2: return launch_w(bnn::xnor_conv3x3_tcw_kernel<2>);
+                case 3: return launch_w(bnn::xnor_conv3x3_tcw_kernel<3>);
+                default: return launch_w(bnn::xnor_conv3x3_tcw_kernel<4>);
+            }
+        }
+        if (st != BNN_ERR_UNSUPPORTED) return st;
+    }
+    // Tensor cores, other strides (when forced): per-pixel gather of up to 2
+    // words per tap (c <= 64) and 256 filters, when the resident filters and
+    // two A tiles fit in shared memory.
     if (engine == BNN_GEMM_ENGINE_TENSOR && cw <= 2 && cout <= bnn::ctc::MAX_N &&
         bnn::conv_tc_smem_bytes((int)cw, (int)n_mma) <= 227 * 1024) {
         const int smem_tc = bnn::conv_tc_smem_bytes((int)cw, (int)n_mma);

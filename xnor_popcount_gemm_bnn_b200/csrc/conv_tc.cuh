@@ -247,4 +247,301 @@ xnor_conv3x3_tc_kernel(const uint32_t* __restrict__ X, int n, int c, int h, int 
     }
 }
 
+// ---------------------------------------------------------------------------
+// Stride-1 binary 3x3 convolution on the tensor cores with shifted windows.
+//
+// Index the zero-padded input of every image on a "virtual" line: position
+// u = b*Hp*Wp + y*Wp + x with Hp = h + 2*pad, Wp = w + 2*pad.  The output
+// pixel (b, oy, ox), placed at u = b*Hp*Wp + oy*Wp + ox, reads tap (dy, dx)
+// at u + dy*Wp + dx, so for 128 consecutive positions every tap is the same
+// 128-row matrix shifted by a constant number of rows.  Each input position
+// is expanded to +1/-1 bytes once, into a buffer of consecutive positions in
+// the non-swizzled K-major operand layout (rows 16 B apart inside each 16-byte
+// column of K), and the 9 * CW MMAs of a tile take their A operand at a
+// different row offset of that buffer.  Positions of the line with oy >= oh or
+// ox >= ow are computed and dropped.
+//
+// The sums are exact: (+1)(+1) for the pad bits of each tap's last word is
+// subtracted (9 * (32*CW - C) per output); an out-of-image tap reads the zero
+// word (+1), as in conv.cuh.
+//
+// A CTA owns a contiguous range of 128-position tiles and walks it in
+// segments that fit one of two A buffers.  Inside a segment consecutive tiles
+// share 2*Wp + 2 halo rows, so a tile expands 128 new rows; the first tile of
+// a segment expands its whole window.  A buffer is refilled only after the
+// MMAs of the segment that last used it are done (a tcgen05.commit per
+// segment).
+//
+// Warps: 0 = TMEM owner and MMA issuer, 1-4 = expansion (one row per thread),
+// 5-12 = epilogue (two warps per TMEM lane quadrant, 32-column chunks split
+// between them).  All waits are bounded as in the kernel above.
+// ---------------------------------------------------------------------------
+namespace ctw {
+constexpr int BM = 128;
+constexpr int GATHER_WARPS = 4;
+constexpr int EPI_WARPS = 8;
+constexpr int WARP_MMA = 0, WARP_GATHER0 = 1, WARP_EPI0 = WARP_GATHER0 + GATHER_WARPS;
+constexpr int THREADS = (WARP_EPI0 + EPI_WARPS) * 32;   // 416
+constexpr int BAR_BYTES = 128;                           // 9 mbarriers, TMEM slot, abort flag
+}  // namespace ctw
+
+struct ConvWindow {
+    int n, h, w, pad;
+    int Hp, Wp, oh, ow;
+    int V;           // n * Hp * Wp virtual positions
+    int tiles;       // ceil(V / 128)
+    int rb;          // rows per A buffer (multiple of 8)
+    int seg_tiles;   // tiles per segment: 128 * seg_tiles + halo <= rb
+    int halo;        // 2 * Wp + 2
+};
+
+// Shared-memory bytes for CW words per pixel, n_mma filter rows and rb rows
+// per A buffer.
+__host__ __device__ inline int conv_tcw_smem_bytes(int cw, int n_mma, int rb) {
+    return 1024 + conv_tc_stages(cw) * n_mma * 128 + 2 * rb * cw * 32 + 12 * n_mma + ctw::BAR_BYTES;
+}
+
+// Non-swizzled K-major shared-memory descriptor: rows 16 B apart inside a
+// core matrix, 8-row groups sbo bytes apart, the two 16-byte K halves of one
+// K = 32 step lbo bytes apart.
+__device__ __forceinline__ uint64_t umma_desc_interleave(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((smem_addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1u << 46);
+}
+
+// 32 sign bits -> 32 bytes of +1 / -1: c0 = elements 0-15, c1 = 16-31.
+__device__ __forceinline__ void expand_word_pm1(uint32_t w, uint4& c0, uint4& c1) {
+    const uint32_t lo = w & 0x0F0F0F0Fu;
+    const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;
+    c0.x = pm1_bytes(__byte_perm(lo, 0u, 0x4440u));
+    c0.y = pm1_bytes(__byte_perm(hi, 0u, 0x4440u));
+    c0.z = pm1_bytes(__byte_perm(lo, 0u, 0x4441u));
+    c0.w = pm1_bytes(__byte_perm(hi, 0u, 0x4441u));
+    c1.x = pm1_bytes(__byte_perm(lo, 0u, 0x4442u));
+    c1.y = pm1_bytes(__byte_perm(hi, 0u, 0x4442u));
+    c1.z = pm1_bytes(__byte_perm(lo, 0u, 0x4443u));
+    c1.w = pm1_bytes(__byte_perm(hi, 0u, 0x4443u));
+}
+
+template <int CW>
+__global__ void __launch_bounds__(ctw::THREADS, 1)
+xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* __restrict__ Wp_,
+                        int64_t ldw, int cout, int n_mma, uint32_t idesc, ConvWindow g, ConvEpilogue ep) {
+    using namespace ctw;
+    constexpr int KW = 9 * CW;
+    constexpr int NS = conv_tc_stages(CW);
+    constexpr int KWP = 4 * NS;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t* bsm = smem;                                                   // NS x n_mma x 128 B, SW128
+    const int abuf_stride = g.rb * CW * 32;
+    uint8_t* abuf = bsm + NS * n_mma * 128;                                // 2 x abuf_stride
+    float* s_alpha = reinterpret_cast<float*>(abuf + 2 * abuf_stride);     // [n_mma]
+    float* s_gamma = s_alpha + n_mma;
+    float* s_beta = s_gamma + n_mma;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(s_beta + n_mma);
+    uint64_t* afill = bars;            // [2] window of the tile expanded (count: gather warps)
+    uint64_t* accfull = afill + 2;     // [2] MMAs of the tile done
+    uint64_t* accempty = accfull + 2;  // [2] accumulator read out (count: epilogue warps)
+    uint64_t* segfree = accempty + 2;  // [2] MMAs of the last segment in A buffer i done
+    uint64_t* drain = segfree + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int tb = (int)((int64_t)blockIdx.x * g.tiles / gridDim.x);
+    const int te = (int)((int64_t)(blockIdx.x + 1) * g.tiles / gridDim.x);
+    const int kt = te - tb;
+    const int HpWp = g.Hp * g.Wp;
+    const int acc_stride = (n_mma + 31) / 32 * 32;
+    const uint32_t tmem_cols = acc_stride <= 64 ? 128u : (acc_stride <= 128 ? 256u : 512u);
+
+    for (int i = threadIdx.x; i < n_mma; i += blockDim.x) {
+        const bool real = i < cout && ep.mode != BNN_OUT_INT32;
+        s_alpha[i] = real ? __ldg(ep.alpha + i) : 0.0f;
+        s_gamma[i] = real && ep.mode == BNN_OUT_AFFINE_F32 ? __ldg(ep.gamma + i) : 0.0f;
+        s_beta[i] = real && ep.mode == BNN_OUT_AFFINE_F32 ? __ldg(ep.beta + i) : 0.0f;
+    }
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&afill[b], GATHER_WARPS);
+            mbar_init(&accfull[b], 1);
+            mbar_init(&accempty[b], EPI_WARPS);
+            mbar_init(&segfree[b], 1);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == WARP_MMA) {
+        tmem_alloc(tmem_slot, tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == WARP_MMA) {
+        // ------------------------------ MMA issuer ------------------------------
+        if (lane == 0) {
+            const uint32_t a0 = smem_u32(abuf), b0 = smem_u32(bsm);
+            const uint32_t lbo = (uint32_t)g.rb * 16u;
+            for (int k = 0; k < kt; ++k) {
+                const int b = k & 1;
+                const int seg = k / g.seg_tiles, ks = k - seg * g.seg_tiles;
+                if (!tc_wait(&afill[b], (k >> 1) & 1, abort_flag)) break;
+                if (k >= 2 && !tc_wait(&accempty[b], ((k >> 1) - 1) & 1, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(b * acc_stride);
+                const uint32_t a_tile = a0 + (uint32_t)((seg & 1) * abuf_stride) + (uint32_t)(ks * BM * 16);
+                #pragma unroll
+                for (int tap = 0; tap < 9; ++tap) {
+                    const uint32_t a_tap = a_tile + (uint32_t)(((tap / 3) * g.Wp + tap % 3) * 16);
+                    #pragma unroll
+                    for (int j = 0; j < CW; ++j) {
+                        const int wk = tap * CW + j;
+                        const uint64_t ad = umma_desc_interleave(a_tap + (uint32_t)(2 * j) * lbo, lbo, 128u);
+                        const uint64_t bd = umma_desc_sw128(b0 + (uint32_t)((wk / 4) * n_mma * 128 + (wk % 4) * 32));
+                        asm volatile(
+                            "{\n\t.reg .pred p;\n\t"
+                            "setp.ne.b32 p, %4, 0;\n\t"
+                            "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+                            "l"(ad), "l"(bd), "r"(idesc), "r"(wk != 0 ? 1u : 0u)
+                            : "memory");
+                    }
+                }
+                mma_commit(&accfull[b]);
+                if (ks == g.seg_tiles - 1 || k == kt - 1) mma_commit(&segfree[seg & 1]);
+            }
+            mma_commit(drain);
+            mbar_wait_bounded(drain, 0);       // every MMA done before TMEM is freed
+        }
+        __syncwarp();
+    } else if (warp < WARP_EPI0) {
+        // ------------------------------ expansion warps ------------------------------
+        const int r = threadIdx.x - WARP_GATHER0 * 32;                 // 0..127
+        for (int fr = r; fr < n_mma; fr += BM) {
+            uint32_t wd[KWP];
+            #pragma unroll
+            for (int k = 0; k < KWP; ++k) wd[k] = (fr < cout && k < KW) ? __ldg(Wp_ + (int64_t)fr * ldw + k) : 0u;
+            #pragma unroll
+            for (int s = 0; s < NS; ++s) {
+                uint8_t* row = bsm + s * n_mma * 128 + fr * 128;
+                #pragma unroll
+                for (int q = 0; q < 4; ++q) expand_word_sw128(row, q, fr & 7, wd[4 * s + q]);
+            }
+        }
+        for (int k = 0; k < kt; ++k) {
+            const int b = k & 1;
+            const int seg = k / g.seg_tiles, ks = k - seg * g.seg_tiles;
+            // afill[b] may be re-armed once the MMAs of tile k - 2 are done; a
+            // buffer is refilled once the segment that used it is done.
+            bool ok = k < 2 || tc_wait(&accfull[b], ((k >> 1) - 1) & 1, abort_flag);
+            if (ok && ks == 0 && seg >= 2) ok = tc_wait(&segfree[seg & 1], ((seg >> 1) - 1) & 1, abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            const int useg = (tb + seg * g.seg_tiles) * BM;           // position of buffer row 0
+            const int row_lo = ks == 0 ? 0 : ks * BM + g.halo;
+            const int row_hi = ks * BM + BM + g.halo;
+            uint8_t* ab = abuf + (seg & 1) * abuf_stride;
+            for (int row = row_lo + r; row < row_hi; row += BM) {
+                const int u = useg + row;
+                uint32_t wd[CW];
+                #pragma unroll
+                for (int j = 0; j < CW; ++j) wd[j] = 0u;
+                if (u < g.V) {
+                    const int bi = u / HpWp;
+                    const int rem = u - bi * HpWp;
+                    const int yp = rem / g.Wp;
+                    const int iy = yp - g.pad, ix = rem - yp * g.Wp - g.pad;
+                    if (iy >= 0 && iy < g.h && ix >= 0 && ix < g.w) {
+                        const uint32_t* src = X + (((int64_t)bi * g.h + iy) * g.w + ix) * CW;
+                        #pragma unroll
+                        for (int j = 0; j < CW; ++j) wd[j] = __ldg(src + j);
+                    }
+                }
+                #pragma unroll
+                for (int j = 0; j < CW; ++j) {
+                    uint4 c0, c1;
+                    expand_word_pm1(wd[j], c0, c1);
+                    *reinterpret_cast<uint4*>(ab + (2 * j) * g.rb * 16 + row * 16) = c0;
+                    *reinterpret_cast<uint4*>(ab + (2 * j + 1) * g.rb * 16 + row * 16) = c1;
+                }
+            }
+            fence_proxy_async_shared();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&afill[b]);
+        }
+    } else {
+        // ------------------------------ epilogue warps ------------------------------
+        const int e = warp - WARP_EPI0;               // 0..7
+        const int quad = warp & 3;                    // TMEM lanes 32*quad .. +31
+        const int half = e >> 2;                      // 32-column chunks half, half + 2, ...
+        const int padc = 9 * (32 * CW - c);           // (+1)(+1) pad positions per output
+        const int64_t ohow = (int64_t)g.oh * g.ow;
+        for (int k = 0; k < kt; ++k) {
+            const int b = k & 1;
+            if (!__all_sync(0xffffffffu, tc_wait(&accfull[b], (k >> 1) & 1, abort_flag))) break;
+            tc_fence_after();
+            const int u = (tb + k) * BM + 32 * quad + lane;
+            const int bi = u / HpWp;
+            const int rem = u - bi * HpWp;
+            const int oy = rem / g.Wp, ox = rem - (rem / g.Wp) * g.Wp;
+            const bool valid = u < g.V && oy < g.oh && ox < g.ow;
+            const int64_t obase = valid ? ((int64_t)bi * cout * g.oh + oy) * g.ow + ox : 0;
+            bool arrived = false;
+            for (int c0 = 32 * half; c0 < n_mma; c0 += 64) {
+                uint32_t rr[32];
+                tmem_ld32(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * acc_stride + c0), rr);
+                tmem_ld_wait();
+                if (c0 + 64 >= n_mma) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&accempty[b]);
+                    arrived = true;
+                }
+                if (!valid) continue;
+                if (ep.mode == BNN_OUT_INT32) {
+                    int32_t* o = static_cast<int32_t*>(ep.out) + obase;
+                    #pragma unroll
+                    for (int jj = 0; jj < 32; ++jj)
+                        if (c0 + jj < cout) o[(int64_t)(c0 + jj) * ohow] = (int32_t)rr[jj] - padc;
+                } else {
+                    float* o = static_cast<float*>(ep.out) + obase;
+                    const bool affine = ep.mode == BNN_OUT_AFFINE_F32;
+                    #pragma unroll
+                    for (int j4 = 0; j4 < 32; j4 += 4) {
+                        const float4 a4 = *reinterpret_cast<const float4*>(s_alpha + c0 + j4);
+                        const float4 g4 = *reinterpret_cast<const float4*>(s_gamma + c0 + j4);
+                        const float4 b4 = *reinterpret_cast<const float4*>(s_beta + c0 + j4);
+                        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+                        const float gv[4] = {g4.x, g4.y, g4.z, g4.w};
+                        const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+                        #pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const int co = c0 + j4 + q;
+                            float y = av[q] * (float)((int32_t)rr[j4 + q] - padc);
+                            if (affine) y = fmaf(gv[q], y, bv[q]);
+                            if (co < cout) o[(int64_t)co * ohow] = y;
+                        }
+                    }
+                }
+            }
+            if (!arrived) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&accempty[b]);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == WARP_MMA) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, tmem_cols);
+    }
+}
+
 }  // namespace bnn

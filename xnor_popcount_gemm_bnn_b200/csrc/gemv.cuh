@@ -108,7 +108,7 @@ template <typename XT>
 __global__ void __launch_bounds__(gemv::THREADS)
 xnor_gemv_row128_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restrict__ x, int N, int K,
                         int kw, const float* __restrict__ alpha, int32_t* __restrict__ y_i32,
-                        float* __restrict__ y_f32, int prefetch, int dependent) {
+                        float* __restrict__ y_f32, int prefetch, int xstatic, int dependent) {
     using namespace gemv;
     constexpr int E = 16 / (int)sizeof(XT);           // elements per 16-byte vector
     constexpr int G = 32 / E;                         // lanes per packed word
@@ -121,44 +121,51 @@ xnor_gemv_row128_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* _
     grid_dependents_launch();
     const int nch = kw / 4;
     uint4 v[U];
-    if (prefetch) {
+    auto load_w = [&]() {
         #pragma unroll
         for (int u = 0; u < U; ++u)
             v[u] = (rows[u] < N && lane < nch) ? ldg_stream_v4(W + (int64_t)rows[u] * ldw + 4 * lane)
                                                : make_uint4(0u, 0u, 0u, 0u);
-    }
-    if (dependent) grid_dependency_wait();
-    if (!prefetch) {
-        #pragma unroll
-        for (int u = 0; u < U; ++u)
-            v[u] = (rows[u] < N && lane < nch) ? ldg_stream_v4(W + (int64_t)rows[u] * ldw + 4 * lane)
-                                               : make_uint4(0u, 0u, 0u, 0u);
-    }
-    const int nfull = K / E;                          // whole vectors inside x
-    for (int c = threadIdx.x; c < kw * (32 / E); c += THREADS) {   // vectors covering the padded row
-        uint4 q = make_uint4(0u, 0u, 0u, 0u);
-        if (c < nfull) q = *reinterpret_cast<const uint4*>(x + E * c);
-        const XT* e = reinterpret_cast<const XT*>(&q);
-        uint32_t b = 0;
-        #pragma unroll
-        for (int i = 0; i < E; ++i) b |= neg_bit(to_float(e[i])) << i;
-        if (c == nfull) {                             // the partial last vector, if any
-            b = 0;
-            for (int i = 0; i < K - E * c; ++i) b |= neg_bit(to_float(x[E * c + i])) << i;
+    };
+    auto pack_x = [&]() {
+        const int nfull = K / E;                      // whole vectors inside x
+        for (int c = threadIdx.x; c < kw * (32 / E); c += THREADS) {   // vectors covering the padded row
+            uint4 q = make_uint4(0u, 0u, 0u, 0u);
+            if (c < nfull) q = *reinterpret_cast<const uint4*>(x + E * c);
+            const XT* e = reinterpret_cast<const XT*>(&q);
+            uint32_t b = 0;
+            #pragma unroll
+            for (int i = 0; i < E; ++i) b |= neg_bit(to_float(e[i])) << i;
+            if (c == nfull) {                         // the partial last vector, if any
+                b = 0;
+                for (int i = 0; i < K - E * c; ++i) b |= neg_bit(to_float(x[E * c + i])) << i;
+            }
+            b <<= E * (c & (G - 1));
+            #pragma unroll
+            for (int off = 1; off < G; off <<= 1) b |= __shfl_xor_sync(0xffffffffu, b, off);
+            if ((c & (G - 1)) == 0) xs[c / G] = b;
         }
-        b <<= E * (c & (G - 1));
-        #pragma unroll
-        for (int off = 1; off < G; off <<= 1) b |= __shfl_xor_sync(0xffffffffu, b, off);
-        if ((c & (G - 1)) == 0) xs[c / G] = b;
-    }
-    __syncthreads();
+        __syncthreads();
+    };
+    // Everything that reads only static data runs before the dependency wait:
+    // the weight stream (prefetch), the x pack (xstatic), and with both the
+    // whole product, so that only the store of y waits.
+    if (prefetch) load_w();
+    if (xstatic) pack_x();
+    const bool late_wait = prefetch && xstatic;
+    if (dependent && !late_wait) grid_dependency_wait();
+    if (!prefetch) load_w();
+    if (!xstatic) pack_x();
     const uint4 xq = lane < nch ? *reinterpret_cast<const uint4*>(xs + 4 * lane) : make_uint4(0u, 0u, 0u, 0u);
+    uint32_t d[U];
+    #pragma unroll
+    for (int u = 0; u < U; ++u) d[u] = __reduce_add_sync(0xffffffffu, popc_xor4(v[u], xq));
+    if (dependent && late_wait) grid_dependency_wait();
     #pragma unroll
     for (int u = 0; u < U; ++u) {
-        const uint32_t d = __reduce_add_sync(0xffffffffu, popc_xor4(v[u], xq));
         const int r = rows[u];
         if (lane == 0 && r < N) {
-            const int32_t sv = K - 2 * (int32_t)d;
+            const int32_t sv = K - 2 * (int32_t)d[u];
             if (y_i32 != nullptr) y_i32[r] = sv;
             if (y_f32 != nullptr) y_f32[r] = alpha[r] * (float)sv;
         }
