@@ -95,24 +95,6 @@ bool gemm_tc_smem_configured() {
     return true;
 }
 
-// Per-device one-time opt-in to the TMA-staged NCHW pack's shared memory
-// (3 stages of up to 48 KB).
-bool pack_nchw_smem_configured() {
-    constexpr int kMaxDevices = 64;
-    static std::atomic<int> done[kMaxDevices];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
-    if (dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return true;
-    const int bytes = bnn::pk::STAGES * 48 * 1024 + 128;
-    if (cudaFuncSetAttribute(bnn::pack_sign_nchw_tma_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             bytes) != cudaSuccess ||
-        cudaFuncSetAttribute(bnn::pack_sign_nchw_tma_kernel<__nv_bfloat16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
-        return false;
-    if (dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
-    return true;
-}
-
 std::atomic<int> g_gemm_engine{BNN_GEMM_ENGINE_AUTO};
 
 int sm_count() {
@@ -364,48 +346,15 @@ bnn_status bnn_pack_sign_nchw(const void* x, bnn_dtype dt, int64_t n, int64_t c,
     if (n == 0) return BNN_OK;
     const int64_t hw = h * w, cw = (c + 31) / 32;
     cudaStream_t s = as_cuda(stream);
-    // TMA-staged path: rows of hw elements 16-byte aligned, chunks of px pixels
-    // x all channels of at most 48 KB per stage.
-    {
-        const int64_t nbox = ceil_div(c, 256), cb = ceil_div(c, nbox);
-        int64_t px = es == 2 ? 256 : 128;
-        while ((nbox * cb * px * (int64_t)es > 48 * 1024 || px / 2 >= hw) && px * (int64_t)es > 128) px /= 2;
-        const int64_t stage = nbox * cb * px * (int64_t)es;
-        if (aligned(x, 16) && (hw * (int64_t)es) % 16 == 0 && stage <= 48 * 1024 && n * c <= INT_MAX &&
-            hw <= INT_MAX / 2 && n * ceil_div(hw, px) <= INT_MAX && pack_nchw_smem_configured()) {
-            auto enc = tensor_map_encoder();
-            CUtensorMap tm;
-            cuuint64_t dims[2] = {(cuuint64_t)hw, (cuuint64_t)(n * c)};
-            cuuint64_t strides[1] = {(cuuint64_t)(hw * (int64_t)es)};
-            cuuint32_t box[2] = {(cuuint32_t)px, (cuuint32_t)cb};
-            cuuint32_t estr[2] = {1, 1};
-            if (enc == nullptr ||
-                enc(&tm, dt == BNN_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
-                    const_cast<void*>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-                return BNN_ERR_CUDA;
-            const int64_t chunks = n * ceil_div(hw, px);
-            const int64_t grid = std::min<int64_t>(chunks, 2 * (int64_t)sm_count());
-            const int smem = (int)(bnn::pk::STAGES * stage + 128);
-            if (dt == BNN_F32)
-                bnn::pack_sign_nchw_tma_kernel<float><<<(unsigned)grid, bnn::pk::THREADS, smem, s>>>(
-                    tm, (int)n, (int)c, (int)hw, (int)cw, (int)px, (int)cb, (int)nbox, packed_nhwc);
-            else
-                bnn::pack_sign_nchw_tma_kernel<__nv_bfloat16><<<(unsigned)grid, bnn::pk::THREADS, smem, s>>>(
-                    tm, (int)n, (int)c, (int)hw, (int)cw, (int)px, (int)cb, (int)nbox, packed_nhwc);
-            return launch_status();
-        }
-    }
-    const int64_t threads = n * ceil_div(hw, 8) * cw * 2;
-    const int64_t blocks = ceil_div(threads, 128);
+    const int64_t warps = n * ceil_div(hw, 32) * cw;            // one warp per (image, 32 pixels, word)
+    const int64_t blocks = ceil_div(warps, 8);
     if (blocks > INT_MAX) return BNN_ERR_INVALID_ARG;
-    const bool vec_ok = aligned(x, 16) && (hw % 8 == 0);
+    const bool vec_ok = aligned(x, 16) && (hw % (int64_t)(16 / es) == 0);
     if (dt == BNN_F32)
-        bnn::pack_sign_nchw_kernel<float><<<(unsigned)blocks, 128, 0, s>>>(static_cast<const float*>(x), n, c, hw,
+        bnn::pack_sign_nchw_kernel<float><<<(unsigned)blocks, 256, 0, s>>>(static_cast<const float*>(x), n, c, hw,
                                                                            cw, packed_nhwc, vec_ok);
     else
-        bnn::pack_sign_nchw_kernel<__nv_bfloat16><<<(unsigned)blocks, 128, 0, s>>>(
+        bnn::pack_sign_nchw_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
             static_cast<const __nv_bfloat16*>(x), n, c, hw, cw, packed_nhwc, vec_ok);
     return launch_status();
 }
