@@ -29,7 +29,7 @@
 
 #include "common.cuh"
 #include "conv.cuh"      // ConvEpilogue
-#include "gemm_tc.cuh"   // tcgen05 helpers, pm1_bytes, umma_desc_sw128
+#include "gemm_tc.cuh"   // tcgen05 helpers, expand_word_pm1, umma_desc_sw128
 
 namespace bnn {
 namespace ctc {
@@ -50,19 +50,11 @@ __host__ __device__ inline int conv_tc_smem_bytes(int cw, int n) {
 }
 
 // Writes 32 sign bits of a packed word as 32 signed bytes (+1 / -1) into two
-// 16-byte chunks (2q, 2q+1) of a 128-byte swizzled row.
+// 16-byte chunks (2q, 2q+1) of a 128-byte swizzled row (expand_word_pm1's
+// element order, shared by both operands).
 __device__ __forceinline__ void expand_word_sw128(uint8_t* row, int q, int sw, uint32_t w) {
-    const uint32_t lo = w & 0x0F0F0F0Fu;
-    const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;
     uint4 c0, c1;
-    c0.x = pm1_bytes(__byte_perm(lo, 0u, 0x4440u));
-    c0.y = pm1_bytes(__byte_perm(hi, 0u, 0x4440u));
-    c0.z = pm1_bytes(__byte_perm(lo, 0u, 0x4441u));
-    c0.w = pm1_bytes(__byte_perm(hi, 0u, 0x4441u));
-    c1.x = pm1_bytes(__byte_perm(lo, 0u, 0x4442u));
-    c1.y = pm1_bytes(__byte_perm(hi, 0u, 0x4442u));
-    c1.z = pm1_bytes(__byte_perm(lo, 0u, 0x4443u));
-    c1.w = pm1_bytes(__byte_perm(hi, 0u, 0x4443u));
+    expand_word_pm1(w, c0, c1);
     *reinterpret_cast<uint4*>(row + (((2 * q) ^ sw) << 4)) = c0;
     *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ sw) << 4)) = c1;
 }
@@ -307,20 +299,6 @@ __host__ __device__ inline int conv_tcw_smem_bytes(int cw, int n_mma, int rb) {
 __device__ __forceinline__ uint64_t umma_desc_interleave(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
     return (uint64_t)((smem_addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1u << 46);
-}
-
-// 32 sign bits -> 32 bytes of +1 / -1: c0 = elements 0-15, c1 = 16-31.
-__device__ __forceinline__ void expand_word_pm1(uint32_t w, uint4& c0, uint4& c1) {
-    const uint32_t lo = w & 0x0F0F0F0Fu;
-    const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;
-    c0.x = pm1_bytes(__byte_perm(lo, 0u, 0x4440u));
-    c0.y = pm1_bytes(__byte_perm(hi, 0u, 0x4440u));
-    c0.z = pm1_bytes(__byte_perm(lo, 0u, 0x4441u));
-    c0.w = pm1_bytes(__byte_perm(hi, 0u, 0x4441u));
-    c1.x = pm1_bytes(__byte_perm(lo, 0u, 0x4442u));
-    c1.y = pm1_bytes(__byte_perm(hi, 0u, 0x4442u));
-    c1.z = pm1_bytes(__byte_perm(lo, 0u, 0x4443u));
-    c1.w = pm1_bytes(__byte_perm(hi, 0u, 0x4443u));
 }
 
 template <int CW>

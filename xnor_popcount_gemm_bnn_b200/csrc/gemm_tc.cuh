@@ -136,10 +136,24 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
     }
 }
 
-// 4 signed bytes (+1 / -1) from the 4 low bits of n (bit j -> byte j).
-__device__ __forceinline__ uint32_t pm1_bytes(uint32_t n) {
-    const uint32_t t = (n * 0x00204081u) & 0x01010101u;   // bit j -> bit 8j (no carries for n < 16)
-    return t * 0xFEu + 0x01010101u;                        // 0x01 -> 0xFF (-1), 0x00 -> 0x01 (+1)
+// 32 sign bits -> 32 signed bytes (+1 / -1), as two 16-byte chunks.
+// Register s (0..7) of the 32 bytes holds elements 7-s, 15-s, 23-s and 31-s:
+// shifting the word left by s puts those bits at the sign positions of its 4
+// bytes, a PRMT with sign-replicating selectors turns each byte into 0x00 or
+// 0xFF, and one LOP3 maps 0x00 -> 0x01 (+1), 0xFF -> 0xFF (-1).  Three
+// operations per 4 bytes.  The element order inside a word's 32 bytes is
+// therefore a fixed permutation; both operands of a product are expanded by
+// this same function, so every K-sum pairs the same elements.
+__device__ __forceinline__ void expand_word_pm1(uint32_t w, uint4& c0, uint4& c1) {
+    uint32_t r[8];
+    #pragma unroll
+    for (int s = 0; s < 8; ++s) {
+        uint32_t m;
+        asm("prmt.b32 %0, %1, 0, 0xBA98;" : "=r"(m) : "r"(w << s));
+        r[s] = (m & 0xFEFEFEFEu) | 0x01010101u;
+    }
+    c0 = make_uint4(r[0], r[1], r[2], r[3]);
+    c1 = make_uint4(r[4], r[5], r[6], r[7]);
 }
 
 __global__ void __launch_bounds__(tc::THREADS, 1)
@@ -275,18 +289,8 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 const uint32_t wq[4] = {pk.x, pk.y, pk.z, pk.w};
                 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const uint32_t w = wq[q];
-                    const uint32_t lo = w & 0x0F0F0F0Fu;              // nibbles 0, 2, 4, 6 (one per byte)
-                    const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;       // nibbles 1, 3, 5, 7
                     uint4 c0, c1;
-                    c0.x = pm1_bytes(__byte_perm(lo, 0u, 0x4440u));
-                    c0.y = pm1_bytes(__byte_perm(hi, 0u, 0x4440u));
-                    c0.z = pm1_bytes(__byte_perm(lo, 0u, 0x4441u));
-                    c0.w = pm1_bytes(__byte_perm(hi, 0u, 0x4441u));
-                    c1.x = pm1_bytes(__byte_perm(lo, 0u, 0x4442u));
-                    c1.y = pm1_bytes(__byte_perm(hi, 0u, 0x4442u));
-                    c1.z = pm1_bytes(__byte_perm(lo, 0u, 0x4443u));
-                    c1.w = pm1_bytes(__byte_perm(hi, 0u, 0x4443u));
+                    expand_word_pm1(wq[q], c0, c1);
                     *reinterpret_cast<uint4*>(row + (((2 * q) ^ sw) << 4)) = c0;
                     *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ sw) << 4)) = c1;
                 }
