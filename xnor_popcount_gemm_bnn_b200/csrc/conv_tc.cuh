@@ -265,15 +265,18 @@ xnor_conv3x3_tc_kernel(const uint32_t* __restrict__ X, int n, int c, int h, int 
 // segment).
 //
 // Warps: 0 = TMEM owner and MMA issuer, 1-4 = expansion (one row per thread),
-// 5-12 = epilogue (two warps per TMEM lane quadrant, 32-column chunks split
-// between them).  All waits are bounded as in the kernel above.
+// 5-20 = epilogue: four warps per TMEM lane quadrant, 16-column slices dealt
+// round-robin, so that sixteen warps keep NCHW stores in flight (the fp32
+// output is the largest stream of the kernel).  All waits are bounded as in
+// the kernel above.
 // ---------------------------------------------------------------------------
 namespace ctw {
 constexpr int BM = 128;
 constexpr int GATHER_WARPS = 4;
-constexpr int EPI_WARPS = 8;
+constexpr int EPI_WARPS = 16;
+constexpr int EPI_COLS = 16;                             // columns per tcgen05.ld slice
 constexpr int WARP_MMA = 0, WARP_GATHER0 = 1, WARP_EPI0 = WARP_GATHER0 + GATHER_WARPS;
-constexpr int THREADS = (WARP_EPI0 + EPI_WARPS) * 32;   // 416
+constexpr int THREADS = (WARP_EPI0 + EPI_WARPS) * 32;   // 672
 constexpr int BAR_BYTES = 128;                           // 9 mbarriers, TMEM slot, abort flag
 }  // namespace ctw
 
@@ -453,27 +456,28 @@ xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* _
         }
     } else {
         // ------------------------------ epilogue warps ------------------------------
-        const int e = warp - WARP_EPI0;               // 0..7
+        const int e = warp - WARP_EPI0;               // 0..15
         const int quad = warp & 3;                    // TMEM lanes 32*quad .. +31
-        const int half = e >> 2;                      // 32-column chunks half, half + 2, ...
+        const int slice0 = EPI_COLS * (e >> 2);       // slices slice0, slice0 + 64, ...
         const int padc = 9 * (32 * CW - c);           // (+1)(+1) pad positions per output
         const int64_t ohow = (int64_t)g.oh * g.ow;
+        const int lane_pos = 32 * quad + lane;        // this thread's row of every tile
         for (int k = 0; k < kt; ++k) {
             const int b = k & 1;
             if (!__all_sync(0xffffffffu, tc_wait(&accfull[b], (k >> 1) & 1, abort_flag))) break;
             tc_fence_after();
-            const int u = (tb + k) * BM + 32 * quad + lane;
+            const int u = (tb + k) * BM + lane_pos;
             const int bi = u / HpWp;
             const int rem = u - bi * HpWp;
             const int oy = rem / g.Wp, ox = rem - (rem / g.Wp) * g.Wp;
             const bool valid = u < g.V && oy < g.oh && ox < g.ow;
             const int64_t obase = valid ? ((int64_t)bi * cout * g.oh + oy) * g.ow + ox : 0;
             bool arrived = false;
-            for (int c0 = 32 * half; c0 < n_mma; c0 += 64) {
-                uint32_t rr[32];
-                tmem_ld32(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * acc_stride + c0), rr);
+            for (int c0 = slice0; c0 < n_mma; c0 += 4 * EPI_COLS) {
+                uint32_t rr[EPI_COLS];
+                tmem_ld16(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * acc_stride + c0), rr);
                 tmem_ld_wait();
-                if (c0 + 64 >= n_mma) {
+                if (c0 + 4 * EPI_COLS >= n_mma) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&accempty[b]);
@@ -483,13 +487,13 @@ xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* _
                 if (ep.mode == BNN_OUT_INT32) {
                     int32_t* o = static_cast<int32_t*>(ep.out) + obase;
                     #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj)
+                    for (int jj = 0; jj < EPI_COLS; ++jj)
                         if (c0 + jj < cout) o[(int64_t)(c0 + jj) * ohow] = (int32_t)rr[jj] - padc;
                 } else {
                     float* o = static_cast<float*>(ep.out) + obase;
                     const bool affine = ep.mode == BNN_OUT_AFFINE_F32;
                     #pragma unroll
-                    for (int j4 = 0; j4 < 32; j4 += 4) {
+                    for (int j4 = 0; j4 < EPI_COLS; j4 += 4) {
                         const float4 a4 = *reinterpret_cast<const float4*>(s_alpha + c0 + j4);
                         const float4 g4 = *reinterpret_cast<const float4*>(s_gamma + c0 + j4);
                         const float4 b4 = *reinterpret_cast<const float4*>(s_beta + c0 + j4);
