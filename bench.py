@@ -54,7 +54,7 @@ FALLBACK_BF16_TFLOPS = 1590.0
 INT8_PER_BF16 = 2.0
 # Whether AUTO runs the stride-1 convolution on the tensor cores (mirrors the
 # library's dispatch, for labelling the conv row's roofline).
-CONV_AUTO_TENSOR = False
+CONV_AUTO_TENSOR = True
 SM_COUNT = 148
 # 32-bit population count: 16 per clock per SM (CUDA arithmetic-instruction
 # throughput table); one POPC covers 32 binary multiply-accumulates.
@@ -283,10 +283,18 @@ def run_ours(args, torch, dist):
     g, Ws, alpha, x, y = gemv_setup(torch, bnn, workloads, dev, copies)
 
     # Every step's inputs (packed W, x, alpha) are resident before the timed
-    # region and no step reads another's output, so each GEMV may stream its
-    # weights, pack x and form the product while the previous one finishes;
-    # only its store of y waits for the previous kernel (stream order on y).
+    # region, and each step writes its own output (the y buffers rotate with
+    # the weights), so no step depends on another: each GEMV streams its
+    # weights, packs x, forms the product and stores y while the previous one
+    # may still run, and waits for it only before exiting.
+    ys = [torch.empty(g.N, dtype=torch.float32, device=dev) for _ in range(copies)]
+    all_flags = bnn.BNN_GEMV_WEIGHTS_STATIC | bnn.BNN_GEMV_INPUTS_STATIC | bnn.BNN_GEMV_OUTPUT_FREE
+
     def step(i):
+        bnn.bnn_xnor_gemv_ex(Ws[i % copies], x, g.K, alpha, None, ys[i % copies], flags=all_flags)
+
+    # The same steps with one shared y: the store waits for the previous kernel.
+    def step_ordered(i):
         bnn.bnn_xnor_gemv_ex(Ws[i % copies], x, g.K, alpha, None, y,
                              flags=bnn.BNN_GEMV_WEIGHTS_STATIC | bnn.BNN_GEMV_INPUTS_STATIC)
 
@@ -302,6 +310,7 @@ def run_ours(args, torch, dist):
         ms = time_steps(torch, step, args.steps, args.warmup, copies, sync)
     ms = max_over_ranks(ms)
     side_steps = min(args.steps, 48 * copies)
+    ms_ord = max_over_ranks(time_steps(torch, step_ordered, side_steps, args.warmup, copies, sync))
     ms_dep = max_over_ranks(time_steps(torch, step_dep, side_steps, args.warmup, copies, sync))
     ms_plain = max_over_ranks(time_steps(torch, step_plain, side_steps, args.warmup, copies, sync))
     if bnn.bnn_device_error() != 0:
@@ -346,7 +355,14 @@ def run_ours(args, torch, dist):
         },
         "gpu_launches": args.steps,
         "clocks": clk.summary(),
-        "flags": "BNN_GEMV_WEIGHTS_STATIC | BNN_GEMV_INPUTS_STATIC (independent steps over resident inputs)",
+        "flags": "BNN_GEMV_WEIGHTS_STATIC | BNN_GEMV_INPUTS_STATIC | BNN_GEMV_OUTPUT_FREE "
+                 "(independent steps: resident inputs, one output buffer per step)",
+        "store_ordered": {
+            "value": round(ws * side_steps * per_step_bytes / (ms_ord * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "steps": side_steps, "ms_per_step": ms_ord / side_steps,
+            "frac": round(side_steps * per_step_bytes / (ms_ord * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+            "note": "BNN_GEMV_WEIGHTS_STATIC | BNN_GEMV_INPUTS_STATIC with one shared y: each store waits for "
+                    "the previous kernel"},
         "dependent_chain": {
             "value": round(ws * side_steps * per_step_bytes / (ms_dep * 1e-3) / 1e9, 2), "unit": "GB/s",
             "steps": side_steps, "ms_per_step": ms_dep / side_steps,
@@ -548,6 +564,9 @@ def _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk):
     cbytes = Xb[0].numel() * 4 + Wc.numel() * 4 + out[0].numel() * 4
     for i in range(R):
         bnn.bnn_pack_sign_nchw(Xd[i], Xb[i])
+    ms_pack = timed(lambda i: bnn.bnn_pack_sign_nchw(Xd[i % R], Xb[i % R]))
+    pbytes = Xd[0].numel() * 2 + Xb[0].numel() * 4
+    pack_gbs = pbytes * steps / (ms_pack * 1e-3) / 1e9
     for name, engine in (("conv3x3", bnn.BNN_GEMM_ENGINE_AUTO), ("conv3x3_tensor", bnn.BNN_GEMM_ENGINE_TENSOR),
                          ("conv3x3_popcount", bnn.BNN_GEMM_ENGINE_POPCOUNT)):
         with bnn.gemm_engine(engine):
@@ -576,6 +595,8 @@ def _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk):
             "value": round(ws * cmacs * steps / (ms_c * 1e-3) / 1e9, 1), "unit": "binary GMAC/s",
             "ms_per_step": ms_c / steps, "conv_kernel_ms": ms_ck / steps,
             "conv_kernel_binary_tmac_s": round(cmac_s / 1e12, 2), "roofline": roof,
+            "pack_nchw": {"ms": ms_pack / steps, "achieved_gbs": round(pack_gbs, 1),
+                          "frac": round(pack_gbs / pk["hbm_gbs"], 4), "bytes": pbytes},
             "l2": f"{R} rotating input/output sets, {rot_mb:.0f} MB"}
     del cv, Xd, Xb, Wc, alc, gam, bet, out
     torch.cuda.empty_cache()

@@ -182,10 +182,13 @@ bnn_status bnn_pack_conv3x3_weights(const void* w_oihw, bnn_dtype dt, int64_t co
  *             multiplied on the tensor cores (tcgen05.mma kind::i8, int32
  *             accumulators in tensor memory); for large products.
  *   AUTO:     TENSOR when M >= 128, N >= 128 and K >= 512, else POPCOUNT
- *             (the default); the convolution uses POPCOUNT under AUTO.
- * The convolution uses the tensor cores only under TENSOR, and only where
- * c <= 64, cout <= 256 and its shared memory fits (c <= 32: every cout;
- * 33..64: up to 96 filters); other shapes use the popcount kernel. */
+ *             (the default).  Convolutions: the stride-1 tensor-core kernel
+ *             when cout >= 64, c <= 64 and n*oh*ow >= 16384, else POPCOUNT.
+ * Under TENSOR the convolution uses the tensor cores where its shared memory
+ * fits: stride 1 with cout <= 256 (the filters stay resident next to two
+ * input buffers of at least one 128-pixel window); other strides with
+ * c <= 64 and cout <= 256 when the filters and two gathered tiles fit.  Other
+ * shapes use the popcount kernel. */
 typedef enum bnn_gemm_engine {
     BNN_GEMM_ENGINE_AUTO = 0,
     BNN_GEMM_ENGINE_POPCOUNT = 1,
@@ -233,7 +236,8 @@ bnn_status bnn_xnor_gemv(const uint32_t* W, int64_t ldw, const void* x, bnn_dtyp
 /* Flags of bnn_xnor_gemv_ex. */
 typedef enum bnn_gemv_flags {
     BNN_GEMV_WEIGHTS_STATIC = 1,  /* W is not written by any work still in flight on the stream */
-    BNN_GEMV_INPUTS_STATIC = 2    /* x and alpha are not written by any work still in flight */
+    BNN_GEMV_INPUTS_STATIC = 2,   /* x and alpha are not written by any work still in flight */
+    BNN_GEMV_OUTPUT_FREE = 4      /* y is neither read nor written by any work still in flight */
 } bnn_gemv_flags;
 
 /* bnn_xnor_gemv_ex -- bnn_xnor_gemv with flags.  Both calls launch the kernel
@@ -248,9 +252,14 @@ typedef enum bnn_gemv_flags {
  * (the caller guarantees the same for x and alpha) x is packed before the
  * wait as well; with both flags the whole product is computed before it and
  * only the store of y waits, so GEMVs over independent, resident inputs
- * overlap their prologues with the previous kernel.  A flag is a permission:
- * shapes served by the general kernel (rows of more than 128 words, or x not
- * 16-byte aligned) ignore BNN_GEMV_INPUTS_STATIC.
+ * overlap their prologues with the previous kernel.  With all three flags
+ * the call depends on nothing still in flight: it computes and stores y
+ * while the previous kernel may still run, and waits for that kernel only
+ * before it exits (so stream order stays transitive for later work); GEMVs
+ * over independent inputs and outputs then run concurrently.  A flag is a
+ * permission: shapes served by the general kernel (rows of more than 128
+ * words, or x not 16-byte aligned) ignore BNN_GEMV_INPUTS_STATIC and
+ * BNN_GEMV_OUTPUT_FREE.
  *   Errors: as bnn_xnor_gemv; INVALID_ARG for unknown flag bits. */
 bnn_status bnn_xnor_gemv_ex(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt,
                             int64_t N, int64_t K, const float* alpha,

@@ -114,9 +114,9 @@ def test_gemv_rejects_bad_arguments():
 
 def test_gemv_ex_rejects_bad_flags():
     g = L.bnn_xnor_gemv_ex
-    assert g(FAKE, 4, FAKE, 0, 8, 32, NULL, FAKE, NULL, 4, NULL) == bnn.BNN_ERR_INVALID_ARG
-    assert g(FAKE, 4, FAKE, 0, 8, 32, NULL, FAKE, NULL, 7, NULL) == bnn.BNN_ERR_INVALID_ARG
-    for flags in (1, 2, 3):
+    assert g(FAKE, 4, FAKE, 0, 8, 32, NULL, FAKE, NULL, 8, NULL) == bnn.BNN_ERR_INVALID_ARG
+    assert g(FAKE, 4, FAKE, 0, 8, 32, NULL, FAKE, NULL, 15, NULL) == bnn.BNN_ERR_INVALID_ARG
+    for flags in range(8):
         assert g(FAKE, 4, FAKE, 0, 0, 32, NULL, FAKE, NULL, flags, NULL) == bnn.BNN_OK
 
 

@@ -148,7 +148,7 @@ def test_gemv_ex_rejects_unknown_flags():
     x = torch.zeros(64, device=dev())
     y = torch.empty(8, dtype=torch.int32, device=dev())
     with pytest.raises(bnn.BnnError):
-        bnn.bnn_xnor_gemv_ex(W, x, 64, None, y, None, flags=4)
+        bnn.bnn_xnor_gemv_ex(W, x, 64, None, y, None, flags=8)
 
 
 @pytest.mark.parametrize("use_graph", [False, True])
@@ -198,4 +198,55 @@ def test_static_inputs_independent_gemvs(use_graph):
         ref = oracle.gemv_pm1(oracle.sign_pm1(Ws[l]), oracle.sign_pm1(xs[l]))
         assert np.array_equal(ys[l].cpu().numpy(), ref), f"gemv {l}"
     assert torch.equal(y_shared, ys[L - 1])
+    assert_no_device_error()
+
+
+@pytest.mark.parametrize("use_graph", [False, True])
+def test_independent_gemvs_all_flags(use_graph):
+    """All three flags on GEMVs over distinct resident inputs and distinct
+    outputs: they may run concurrently; every result exact, and a kernel
+    queued after them (a torch copy) sees all of them finished."""
+    N, K, L = 777, 4096, 8
+    d = dev()
+    Ws = [workloads.normal((N, K), 1.0, 900 + l) for l in range(L)]
+    xs = [workloads.normal((K,), 1.0, 950 + l, dtype=torch.bfloat16) for l in range(L)]
+    Wp, al = [], []
+    for W in Ws:
+        p = bnn.empty_packed(N, K, d)
+        a = torch.empty(N, dtype=torch.float32, device=d)
+        bnn.bnn_pack_sign(W.to(d), p, a)
+        Wp.append(p)
+        al.append(a)
+    xd = [x.to(d) for x in xs]
+    ys = [torch.empty(N, dtype=torch.int32, device=d) for _ in range(L)]
+    yf = [torch.empty(N, dtype=torch.float32, device=d) for _ in range(L)]
+    flags = bnn.BNN_GEMV_WEIGHTS_STATIC | bnn.BNN_GEMV_INPUTS_STATIC | bnn.BNN_GEMV_OUTPUT_FREE
+    torch.cuda.synchronize()
+
+    def run():
+        for l in range(L):
+            bnn.bnn_xnor_gemv_ex(Wp[l], xd[l], K, al[l], ys[l], yf[l], flags=flags)
+        return torch.stack(ys)
+
+    if use_graph:
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            run()
+        torch.cuda.current_stream().wait_stream(s)
+        with torch.cuda.graph(g):
+            stacked = run()
+        for t in ys:
+            t.fill_(-7)
+        g.replay()
+    else:
+        stacked = run()
+    torch.cuda.synchronize()
+    for l in range(L):
+        wb, xb = oracle.sign_pm1(Ws[l]), oracle.sign_pm1(xs[l])
+        ref = oracle.gemv_pm1(wb, xb)
+        assert np.array_equal(ys[l].cpu().numpy(), ref), f"gemv {l}"
+        assert np.array_equal(stacked[l].cpu().numpy(), ref), f"stacked {l}"
+        assert_scaled_close(yf[l], oracle.scaled(ref, oracle.alpha(Ws[l])))
     assert_no_device_error()

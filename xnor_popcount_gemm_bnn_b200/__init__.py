@@ -36,6 +36,7 @@ BNN_OUT_THRESHOLD_PACK = 8
 
 BNN_GEMV_WEIGHTS_STATIC = 1
 BNN_GEMV_INPUTS_STATIC = 2
+BNN_GEMV_OUTPUT_FREE = 4
 
 BNN_GEMM_ENGINE_AUTO = 0
 BNN_GEMM_ENGINE_POPCOUNT = 1

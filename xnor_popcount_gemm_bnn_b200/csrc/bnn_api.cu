@@ -168,7 +168,7 @@ bnn_status check_gemm_dims(int64_t M, int64_t N, int64_t K) {
 template <typename XT>
 bnn_status launch_gemv_t(const uint32_t* W, int64_t ldw, const XT* x, int64_t N, int64_t K, int64_t kw,
                          const float* alpha, int32_t* y_i32, float* y_f32, bool weights_static,
-                         bool inputs_static, cudaStream_t stream) {
+                         bool inputs_static, bool independent, cudaStream_t stream) {
     using namespace bnn::gemv;
     const int64_t nchunks = kw / 4;
     int lpr = 1;
@@ -205,7 +205,7 @@ bnn_status launch_gemv_t(const uint32_t* W, int64_t ldw, const XT* x, int64_t N,
         // Rows of 97..128 words: the dedicated one-chunk-per-lane kernel.
         auto kern = bnn::xnor_gemv_row128_kernel<XT>;
         e = cudaLaunchKernelEx(&cfg, kern, W, ldw, x, iN, iK, ikw, alpha, y_i32, y_f32, weights_static ? 1 : 0,
-                               inputs_static ? 1 : 0, 1);
+                               inputs_static ? 1 : 0, independent ? 2 : 1);
         if (e != cudaSuccess) return BNN_ERR_CUDA;
         return launch_status();
     }
@@ -238,7 +238,7 @@ constexpr int64_t kGemvMaxWords = 48 * 1024;   // packed x in shared memory: <= 
 
 bnn_status gemv_impl(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt, int64_t N, int64_t K,
                      const float* alpha, int32_t* y_i32, float* y_f32, bool weights_static,
-                     bool inputs_static, bnn_stream_t stream) {
+                     bool inputs_static, bool independent, bnn_stream_t stream) {
     if (N < 0 || K < 1 || N > INT_MAX || K > INT_MAX / 2) return BNN_ERR_INVALID_ARG;
     if (x == nullptr || (y_i32 == nullptr && y_f32 == nullptr)) return BNN_ERR_INVALID_ARG;
     if (y_f32 != nullptr && alpha == nullptr) return BNN_ERR_INVALID_ARG;
@@ -251,9 +251,9 @@ bnn_status gemv_impl(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_
     if (N == 0) return BNN_OK;
     if (x_dt == BNN_F32)
         return launch_gemv_t(W, ldw, static_cast<const float*>(x), N, K, kw, alpha, y_i32, y_f32,
-                             weights_static, inputs_static, as_cuda(stream));
+                             weights_static, inputs_static, independent, as_cuda(stream));
     return launch_gemv_t(W, ldw, static_cast<const __nv_bfloat16*>(x), N, K, kw, alpha, y_i32, y_f32,
-                         weights_static, inputs_static, as_cuda(stream));
+                         weights_static, inputs_static, independent, as_cuda(stream));
 }
 
 }  // namespace
@@ -346,7 +346,7 @@ bnn_status bnn_pack_sign_nchw(const void* x, bnn_dtype dt, int64_t n, int64_t c,
     if (n == 0) return BNN_OK;
     const int64_t hw = h * w, cw = (c + 31) / 32;
     cudaStream_t s = as_cuda(stream);
-    const int64_t warps = n * ceil_div(hw, 32) * cw;            // one warp per (image, 32 pixels, word)
+    const int64_t warps = n * ceil_div(hw, 8 * (int64_t)(16 / es)) * cw;   // (image, 8 vectors of pixels, word)
     const int64_t blocks = ceil_div(warps, 8);
     if (blocks > INT_MAX) return BNN_ERR_INVALID_ARG;
     const bool vec_ok = aligned(x, 16) && (hw % (int64_t)(16 / es) == 0);
@@ -404,16 +404,16 @@ bnn_status bnn_xnor_gemm(const uint32_t* A, int64_t lda, const uint32_t* W, int6
 
 bnn_status bnn_xnor_gemv(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt, int64_t N, int64_t K,
                          const float* alpha, int32_t* y_i32, float* y_f32, bnn_stream_t stream) {
-    return gemv_impl(W, ldw, x, x_dt, N, K, alpha, y_i32, y_f32, false, false, stream);
+    return gemv_impl(W, ldw, x, x_dt, N, K, alpha, y_i32, y_f32, false, false, false, stream);
 }
 
 bnn_status bnn_xnor_gemv_ex(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt, int64_t N, int64_t K,
                             const float* alpha, int32_t* y_i32, float* y_f32, uint32_t flags,
                             bnn_stream_t stream) {
-    if ((flags & ~(uint32_t)(BNN_GEMV_WEIGHTS_STATIC | BNN_GEMV_INPUTS_STATIC)) != 0) return BNN_ERR_INVALID_ARG;
+    constexpr uint32_t kAll = BNN_GEMV_WEIGHTS_STATIC | BNN_GEMV_INPUTS_STATIC | BNN_GEMV_OUTPUT_FREE;
+    if ((flags & ~kAll) != 0) return BNN_ERR_INVALID_ARG;
     return gemv_impl(W, ldw, x, x_dt, N, K, alpha, y_i32, y_f32, (flags & BNN_GEMV_WEIGHTS_STATIC) != 0,
-                     (flags & BNN_GEMV_INPUTS_STATIC) != 0,
-                     stream);
+                     (flags & BNN_GEMV_INPUTS_STATIC) != 0, flags == kAll, stream);
 }
 
 bnn_status bnn_binary_linear_fused(const uint32_t* A, int64_t lda, const uint32_t* W, int64_t ldw, int64_t M,
@@ -522,8 +522,13 @@ bnn_status bnn_binary_conv3x3_fused(const uint32_t* X_nhwc_bits, int64_t n, int6
     const int engine = g_gemm_engine.load(std::memory_order_relaxed);
     const int64_t n_mma = std::max<int64_t>(16, ceil_div(cout, (int64_t)16) * 16);
     // Tensor cores, stride 1: the shifted-window kernel, when the resident
-    // filters and two A buffers of at least one tile's window fit.
-    if (engine == BNN_GEMM_ENGINE_TENSOR && stride == 1 && cout <= bnn::ctc::MAX_N) {
+    // filters and two A buffers of at least one tile's window fit.  AUTO takes
+    // it where it was measured to win clearly (the ResNet-class layer: 64
+    // filters, c = 64, 200k output pixels: 29 us against 62 us): at least 64
+    // filters, c <= 64 and 16384 output pixels.
+    const bool tc_window = engine == BNN_GEMM_ENGINE_TENSOR ||
+                           (engine == BNN_GEMM_ENGINE_AUTO && cout >= 64 && cw <= 2 && npix >= 16384);
+    if (tc_window && stride == 1 && cout <= bnn::ctc::MAX_N) {
         bnn::ConvWindow g{};
         const bnn_status st = conv_window_plan(n, h, w, pad, cw, n_mma, &g);
         if (st == BNN_OK) {

@@ -265,19 +265,23 @@ xnor_conv3x3_tc_kernel(const uint32_t* __restrict__ X, int n, int c, int h, int 
 // segment).
 //
 // Warps: 0 = TMEM owner and MMA issuer, 1-4 = expansion (one row per thread),
-// 5-20 = epilogue: four warps per TMEM lane quadrant, 16-column slices dealt
-// round-robin, so that sixteen warps keep NCHW stores in flight (the fp32
-// output is the largest stream of the kernel).  All waits are bounded as in
+// 5-20 = epilogue in two groups of eight: group i drains the accumulator of
+// tiles k = i (mod 2), i.e. always TMEM buffer i, so one group's stores run
+// while the other waits for its MMAs and TMEM load.  Inside a group, two warps
+// per TMEM lane quadrant take alternate 16-column slices.  The fp32 NCHW
+// output is the largest stream of the kernel.  All waits are bounded as in
 // the kernel above.
 // ---------------------------------------------------------------------------
 namespace ctw {
 constexpr int BM = 128;
 constexpr int GATHER_WARPS = 4;
-constexpr int EPI_WARPS = 16;
+constexpr int EPI_WARPS = 16;                            // two groups of 8
+constexpr int EPI_GROUP = 8;
 constexpr int EPI_COLS = 16;                             // columns per tcgen05.ld slice
 constexpr int WARP_MMA = 0, WARP_GATHER0 = 1, WARP_EPI0 = WARP_GATHER0 + GATHER_WARPS;
 constexpr int THREADS = (WARP_EPI0 + EPI_WARPS) * 32;   // 672
-constexpr int BAR_BYTES = 128;                           // 9 mbarriers, TMEM slot, abort flag
+constexpr int AHEAD = 4;                                 // tiles the expansion may run ahead
+constexpr int BAR_BYTES = 192;                           // 15 mbarriers, TMEM slot, abort flag
 }  // namespace ctw
 
 struct ConvWindow {
@@ -321,8 +325,9 @@ xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* _
     float* s_gamma = s_alpha + n_mma;
     float* s_beta = s_gamma + n_mma;
     uint64_t* bars = reinterpret_cast<uint64_t*>(s_beta + n_mma);
-    uint64_t* afill = bars;            // [2] window of the tile expanded (count: gather warps)
-    uint64_t* accfull = afill + 2;     // [2] MMAs of the tile done
+    uint64_t* afill = bars;               // [AHEAD] window of the tile expanded (count: gather warps)
+    uint64_t* aconsumed = afill + AHEAD;  // [AHEAD] the MMA thread has seen that afill phase
+    uint64_t* accfull = aconsumed + AHEAD;  // [2] MMAs of the tile done
     uint64_t* accempty = accfull + 2;  // [2] accumulator read out (count: epilogue warps)
     uint64_t* segfree = accempty + 2;  // [2] MMAs of the last segment in A buffer i done
     uint64_t* drain = segfree + 2;
@@ -345,10 +350,13 @@ xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* _
         s_beta[i] = real && ep.mode == BNN_OUT_AFFINE_F32 ? __ldg(ep.beta + i) : 0.0f;
     }
     if (threadIdx.x == 0) {
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < AHEAD; ++b) {
             mbar_init(&afill[b], GATHER_WARPS);
+            mbar_init(&aconsumed[b], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
             mbar_init(&accfull[b], 1);
-            mbar_init(&accempty[b], EPI_WARPS);
+            mbar_init(&accempty[b], EPI_GROUP);
             mbar_init(&segfree[b], 1);
         }
         mbar_init(drain, 1);
@@ -367,24 +375,36 @@ xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* _
     if (warp == WARP_MMA) {
         // ------------------------------ MMA issuer ------------------------------
         if (lane == 0) {
-            const uint32_t a0 = smem_u32(abuf), b0 = smem_u32(bsm);
-            const uint32_t lbo = (uint32_t)g.rb * 16u;
+            // Descriptors are built once; per MMA only the start-address field
+            // (bits 0-13, in 16-byte units) moves, and every smem address here
+            // is below 256 KB, so a 32-bit add on the low word cannot carry
+            // into the other fields.  This keeps the issuing thread short: it
+            // shares its SM sub-partition with expansion and epilogue warps.
+            const uint64_t ad0 = umma_desc_interleave(smem_u32(abuf), (uint32_t)g.rb * 16u, 128u);
+            const uint64_t bd0 = umma_desc_sw128(smem_u32(bsm));
+            const uint32_t ad_lo = (uint32_t)ad0, ad_hi = (uint32_t)(ad0 >> 32);
+            const uint32_t bd_lo = (uint32_t)bd0, bd_hi = (uint32_t)(bd0 >> 32);
+            const uint32_t row_dy[3] = {0u, (uint32_t)g.Wp, 2u * (uint32_t)g.Wp};   // tap row shift, in rows
+            const uint32_t khalf = 2u * (uint32_t)g.rb;                           // one 32-byte K step, in 16-B units
+            const uint32_t bstage = (uint32_t)n_mma * 8u;                          // one B stage, in 16-B units
             for (int k = 0; k < kt; ++k) {
                 const int b = k & 1;
                 const int seg = k / g.seg_tiles, ks = k - seg * g.seg_tiles;
-                if (!tc_wait(&afill[b], (k >> 1) & 1, abort_flag)) break;
+                if (!tc_wait(&afill[k % AHEAD], (k / AHEAD) & 1, abort_flag)) break;
+                mbar_arrive(&aconsumed[k % AHEAD]);
                 if (k >= 2 && !tc_wait(&accempty[b], ((k >> 1) - 1) & 1, abort_flag)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(b * acc_stride);
-                const uint32_t a_tile = a0 + (uint32_t)((seg & 1) * abuf_stride) + (uint32_t)(ks * BM * 16);
+                const uint32_t a_tile = ad_lo + (uint32_t)(((seg & 1) * abuf_stride) >> 4) + (uint32_t)(ks * BM);
                 #pragma unroll
                 for (int tap = 0; tap < 9; ++tap) {
-                    const uint32_t a_tap = a_tile + (uint32_t)(((tap / 3) * g.Wp + tap % 3) * 16);
+                    const uint32_t a_tap = a_tile + row_dy[tap / 3] + (uint32_t)(tap % 3);
                     #pragma unroll
                     for (int j = 0; j < CW; ++j) {
                         const int wk = tap * CW + j;
-                        const uint64_t ad = umma_desc_interleave(a_tap + (uint32_t)(2 * j) * lbo, lbo, 128u);
-                        const uint64_t bd = umma_desc_sw128(b0 + (uint32_t)((wk / 4) * n_mma * 128 + (wk % 4) * 32));
+                        const uint64_t ad = ((uint64_t)ad_hi << 32) | (a_tap + (uint32_t)j * khalf);
+                        const uint64_t bd = ((uint64_t)bd_hi << 32) |
+                                            (bd_lo + (uint32_t)(wk / 4) * bstage + (uint32_t)((wk % 4) * 2));
                         asm volatile(
                             "{\n\t.reg .pred p;\n\t"
                             "setp.ne.b32 p, %4, 0;\n\t"
@@ -415,12 +435,11 @@ xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* _
             }
         }
         for (int k = 0; k < kt; ++k) {
-            const int b = k & 1;
             const int seg = k / g.seg_tiles, ks = k - seg * g.seg_tiles;
-            // afill[b] may be re-armed once the MMAs of tile k - 2 are done; a
-            // buffer is refilled once the segment that used it is done.
-            bool ok = k < 2 || tc_wait(&accfull[b], ((k >> 1) - 1) & 1, abort_flag);
-            if (ok && ks == 0 && seg >= 2) ok = tc_wait(&segfree[seg & 1], ((seg >> 1) - 1) & 1, abort_flag);
+            // Inside a segment rows are only appended, so the expansion runs up
+            // to AHEAD tiles ahead of the MMAs; a buffer is refilled once the
+            // MMAs of the segment that used it before are done.
+            const bool ok = ks != 0 || seg < 2 || tc_wait(&segfree[seg & 1], ((seg >> 1) - 1) & 1, abort_flag);
             if (!__all_sync(0xffffffffu, ok)) break;
             const int useg = (tb + seg * g.seg_tiles) * BM;           // position of buffer row 0
             const int row_lo = ks == 0 ? 0 : ks * BM + g.halo;
@@ -451,19 +470,24 @@ xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* _
                 }
             }
             fence_proxy_async_shared();
+            // afill[k % AHEAD] is re-armed only after the MMA thread has seen
+            // its previous phase (tile k - AHEAD).
+            const bool ok2 = k < AHEAD || tc_wait(&aconsumed[k % AHEAD], ((k / AHEAD) - 1) & 1, abort_flag);
+            if (!__all_sync(0xffffffffu, ok2)) break;
             __syncwarp();
-            if (lane == 0) mbar_arrive(&afill[b]);
+            if (lane == 0) mbar_arrive(&afill[k % AHEAD]);
         }
     } else {
         // ------------------------------ epilogue warps ------------------------------
         const int e = warp - WARP_EPI0;               // 0..15
+        const int grp = e / EPI_GROUP;                // tiles k = grp (mod 2): TMEM buffer grp
         const int quad = warp & 3;                    // TMEM lanes 32*quad .. +31
-        const int slice0 = EPI_COLS * (e >> 2);       // slices slice0, slice0 + 64, ...
+        const int slice0 = EPI_COLS * ((e % EPI_GROUP) >> 2);   // slices slice0, slice0 + 32, ...
         const int padc = 9 * (32 * CW - c);           // (+1)(+1) pad positions per output
         const int64_t ohow = (int64_t)g.oh * g.ow;
         const int lane_pos = 32 * quad + lane;        // this thread's row of every tile
-        for (int k = 0; k < kt; ++k) {
-            const int b = k & 1;
+        for (int k = grp; k < kt; k += 2) {
+            const int b = grp;
             if (!__all_sync(0xffffffffu, tc_wait(&accfull[b], (k >> 1) & 1, abort_flag))) break;
             tc_fence_after();
             const int u = (tb + k) * BM + lane_pos;
@@ -473,11 +497,11 @@ xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* _
             const bool valid = u < g.V && oy < g.oh && ox < g.ow;
             const int64_t obase = valid ? ((int64_t)bi * cout * g.oh + oy) * g.ow + ox : 0;
             bool arrived = false;
-            for (int c0 = slice0; c0 < n_mma; c0 += 4 * EPI_COLS) {
+            for (int c0 = slice0; c0 < n_mma; c0 += 2 * EPI_COLS) {
                 uint32_t rr[EPI_COLS];
                 tmem_ld16(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * acc_stride + c0), rr);
                 tmem_ld_wait();
-                if (c0 + 4 * EPI_COLS >= n_mma) {
+                if (c0 + 2 * EPI_COLS >= n_mma) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&accempty[b]);

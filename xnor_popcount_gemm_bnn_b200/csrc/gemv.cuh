@@ -153,14 +153,14 @@ xnor_gemv_row128_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* _
     if (prefetch) load_w();
     if (xstatic) pack_x();
     const bool late_wait = prefetch && xstatic;
-    if (dependent && !late_wait) grid_dependency_wait();
+    if (dependent == 1 && !late_wait) grid_dependency_wait();
     if (!prefetch) load_w();
     if (!xstatic) pack_x();
     const uint4 xq = lane < nch ? *reinterpret_cast<const uint4*>(xs + 4 * lane) : make_uint4(0u, 0u, 0u, 0u);
     uint32_t d[U];
     #pragma unroll
     for (int u = 0; u < U; ++u) d[u] = __reduce_add_sync(0xffffffffu, popc_xor4(v[u], xq));
-    if (dependent && late_wait) grid_dependency_wait();
+    if (dependent == 1 && late_wait) grid_dependency_wait();
     #pragma unroll
     for (int u = 0; u < U; ++u) {
         const int r = rows[u];
@@ -170,6 +170,10 @@ xnor_gemv_row128_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* _
             if (y_f32 != nullptr) y_f32[r] = alpha[r] * (float)sv;
         }
     }
+    // dependent == 2: the call touches nothing that work in flight uses; it
+    // still waits for the previous grid before it exits, so that its own
+    // completion implies that grid's (stream order stays transitive).
+    if (dependent == 2) grid_dependency_wait();
 }
 
 // SINGLE: every row fits in one warp-wide pass (nchunks <= LPR).

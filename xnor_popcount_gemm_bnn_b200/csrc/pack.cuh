@@ -74,58 +74,103 @@ pack_sign_rows_kernel(const T* __restrict__ x, int64_t rows, int64_t K, int64_t 
     }
 }
 
+// Raw bits of one element, and element p of a 16-byte vector as float.
+__device__ __forceinline__ uint32_t raw_bits(float v) { return __float_as_uint(v); }
+__device__ __forceinline__ uint32_t raw_bits(__nv_bfloat16 v) { return (uint32_t)__bfloat16_as_ushort(v); }
+template <typename T>
+__device__ __forceinline__ float vec_elem(const uint32_t (&w)[4], int p) {
+    if constexpr (sizeof(T) == 4) {
+        return __uint_as_float(w[p]);
+    } else {
+        const uint32_t x = w[p >> 1];
+        return __uint_as_float((p & 1) ? (x & 0xFFFF0000u) : (x << 16));   // bf16 -> fp32 is exact
+    }
+}
+
 // NCHW real activations -> per-pixel channel words [n, h, w, cw].
-// One warp task = word j of 32 consecutive pixels of one image.  Lane q reads
-// channel 32*j + q over those pixels (64 contiguous bytes of bf16, 128 of
-// fp32, as 16-byte vectors all in flight together), and one __ballot_sync
-// per pixel collects the word: bit q = sign of channel 32*j + q, which is
-// exactly the packed layout (LSB = lowest channel).  Lane p keeps the word
-// of pixel p and stores it.  Tasks are ordered (image, pixel group, word),
-// so consecutive warps stream consecutive stretches of the same channel rows.
+// A warp task is word j of 8*E consecutive pixels of one image (E = pixels
+// per 16-byte vector: 8 bf16, 4 fp32).  Lane (g, q) = (lane / 4, lane % 4)
+// owns pixels [g*E, g*E + E) of the task and channels 32j + 8q .. + 7: eight
+// 16-byte loads, issued together by one asm statement so that all eight are
+// in flight before any is used.  For one channel the 32 lanes read 4 rows x
+// 128 contiguous bytes, so every load instruction is 4 full lines.  Each lane
+// sets bits 8q .. 8q+7 of its E pixels' words; two shuffles OR the four
+// quarters together, and lane q stores the pixels p = q (mod 4).
 template <typename T>
 __global__ void __launch_bounds__(256)
 pack_sign_nchw_kernel(const T* __restrict__ x, int64_t n, int64_t c, int64_t hw, int64_t cw,
                       uint32_t* __restrict__ out, bool vec_ok) {
-    constexpr int PX = 32;                        // pixels per task
-    constexpr int E = 16 / (int)sizeof(T);        // elements per 16-byte vector
-    constexpr int NV = PX / E;                    // vectors per lane
+    constexpr int E = 16 / (int)sizeof(T);
+    constexpr int PX = 8 * E;                     // pixels per task
     const int lane = threadIdx.x & 31;
+    const int g = lane >> 2, q = lane & 3;
     const int64_t groups = (hw + PX - 1) / PX;
     const int64_t task = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (task >= n * groups * cw) return;          // whole warps leave together
     const int64_t j = task % cw;
-    const int64_t g = (task / cw) % groups;
+    const int64_t gi = (task / cw) % groups;
     const int64_t b = task / (cw * groups);
-    const int64_t p0 = g * PX;
-    const int np = (int)(hw - p0 < PX ? hw - p0 : PX);
-    const int64_t ch = 32 * j + lane;
-    const bool live = ch < c;
-    const T* src = x + ((b * c + (live ? ch : 0)) * hw + p0);
-    uint4 v[NV];
-    if (vec_ok && np == PX) {
-        #pragma unroll
-        for (int i = 0; i < NV; ++i)
-            v[i] = live ? __ldg(reinterpret_cast<const uint4*>(src + i * E)) : make_uint4(0u, 0u, 0u, 0u);
+    const int64_t p0 = gi * PX + g * E;           // this lane's first pixel
+    const int np = (int)(hw - p0 <= 0 ? 0 : (hw - p0 < E ? hw - p0 : E));
+    const int64_t ch0 = 32 * j + 8 * q;           // this lane's first channel
+    const int nc = (int)(c - ch0 <= 0 ? 0 : (c - ch0 < 8 ? c - ch0 : 8));
+    const T* src = x + ((b * c + (nc > 0 ? ch0 : 0)) * hw + (np > 0 ? p0 : 0));
+    uint32_t v[8][4];                             // raw 16-byte vectors, one per channel
+    if (vec_ok && np == E && nc == 8) {
+        const size_t rs = (size_t)hw * sizeof(T);     // one channel row, in bytes
+        const char* a = reinterpret_cast<const char*>(src);
+        asm volatile(
+            "ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%32];\n\t"
+            "ld.global.nc.v4.u32 {%4, %5, %6, %7}, [%33];\n\t"
+            "ld.global.nc.v4.u32 {%8, %9, %10, %11}, [%34];\n\t"
+            "ld.global.nc.v4.u32 {%12, %13, %14, %15}, [%35];\n\t"
+            "ld.global.nc.v4.u32 {%16, %17, %18, %19}, [%36];\n\t"
+            "ld.global.nc.v4.u32 {%20, %21, %22, %23}, [%37];\n\t"
+            "ld.global.nc.v4.u32 {%24, %25, %26, %27}, [%38];\n\t"
+            "ld.global.nc.v4.u32 {%28, %29, %30, %31}, [%39];"
+            : "=r"(v[0][0]), "=r"(v[0][1]), "=r"(v[0][2]), "=r"(v[0][3]),
+              "=r"(v[1][0]), "=r"(v[1][1]), "=r"(v[1][2]), "=r"(v[1][3]),
+              "=r"(v[2][0]), "=r"(v[2][1]), "=r"(v[2][2]), "=r"(v[2][3]),
+              "=r"(v[3][0]), "=r"(v[3][1]), "=r"(v[3][2]), "=r"(v[3][3]),
+              "=r"(v[4][0]), "=r"(v[4][1]), "=r"(v[4][2]), "=r"(v[4][3]),
+              "=r"(v[5][0]), "=r"(v[5][1]), "=r"(v[5][2]), "=r"(v[5][3]),
+              "=r"(v[6][0]), "=r"(v[6][1]), "=r"(v[6][2]), "=r"(v[6][3]),
+              "=r"(v[7][0]), "=r"(v[7][1]), "=r"(v[7][2]), "=r"(v[7][3])
+            : "l"(a), "l"(a + rs), "l"(a + 2 * rs), "l"(a + 3 * rs), "l"(a + 4 * rs), "l"(a + 5 * rs),
+              "l"(a + 6 * rs), "l"(a + 7 * rs));
     } else {
+        // Ragged pixels or channels: element loads, zeros (+1) elsewhere.
         #pragma unroll
-        for (int i = 0; i < NV; ++i) {
-            union { uint4 u; T e[E]; } t;
+        for (int i = 0; i < 8; ++i) {
             #pragma unroll
-            for (int k = 0; k < E; ++k) t.e[k] = (live && i * E + k < np) ? src[i * E + k] : T(0.0f);
-            v[i] = t.u;
+            for (int k = 0; k < 4; ++k) {
+                uint32_t w = 0;
+                #pragma unroll
+                for (int t = 0; t < E / 4; ++t) {
+                    const int pp = k * (E / 4) + t;
+                    const uint32_t raw = (i < nc && pp < np) ? raw_bits(src[(int64_t)i * hw + pp]) : 0u;
+                    w |= raw << (32 / (E / 4) * t);
+                }
+                v[i][k] = w;
+            }
         }
     }
-    uint32_t mine = 0;
+    uint32_t bits[E];
     #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-        const T* e = reinterpret_cast<const T*>(&v[i]);
+    for (int p = 0; p < E; ++p) {
+        uint32_t w = 0;
         #pragma unroll
-        for (int k = 0; k < E; ++k) {
-            const uint32_t word = __ballot_sync(0xffffffffu, to_float(e[k]) < 0.0f);
-            if (lane == i * E + k) mine = word;
-        }
+        for (int i = 0; i < 8; ++i) w |= neg_bit(vec_elem<T>(v[i], p)) << i;
+        bits[p] = w << (8 * q);
     }
-    if (lane < np) out[(b * hw + p0 + lane) * cw + j] = mine;
+    #pragma unroll
+    for (int p = 0; p < E; ++p) {
+        bits[p] |= __shfl_xor_sync(0xffffffffu, bits[p], 1);
+        bits[p] |= __shfl_xor_sync(0xffffffffu, bits[p], 2);
+    }
+    #pragma unroll
+    for (int p = 0; p < E; ++p)
+        if ((p & 3) == q && p < np) out[(b * hw + p0 + p) * cw + j] = bits[p];
 }
 
 // OIHW 3x3 filters -> packed rows in (kh, kw, c) order, one warp per output
