@@ -202,12 +202,25 @@ bnn_status launch_gemv_t(const uint32_t* W, int64_t ldw, const XT* x, int64_t N,
     bnn_status st = BNN_OK;
     const bool vec = aligned(x, 16);
     if (lpr == 32 && single && vec) {
-        // Rows of 97..128 words: the dedicated one-chunk-per-lane kernel.
-        auto kern = bnn::xnor_gemv_row128_kernel<XT>;
-        e = cudaLaunchKernelEx(&cfg, kern, W, ldw, x, iN, iK, ikw, alpha, y_i32, y_f32, weights_static ? 1 : 0,
-                               inputs_static ? 1 : 0, independent ? 2 : 1);
-        if (e != cudaSuccess) return BNN_ERR_CUDA;
-        return launch_status();
+        // Rows of 97..128 words: the dedicated one-chunk-per-lane kernel.  Its
+        // block shape depends on what the launch may overlap; each was the
+        // fastest of ~30 shapes on the 11008 x 4096 decode GEMV in back-to-back
+        // launches (steps of 1.10 / 1.39 / 2.18 us):
+        //   all three flags (nothing to wait for):  256 threads x 12 rows per warp
+        //   static W and x, ordered store:          128 threads x 8 rows per warp
+        //   x (or W) read after the wait:           768 threads x 2 rows per warp
+        auto go = [&](auto kern, int th, int u) -> bnn_status {
+            const int64_t rows = (int64_t)(th / 32) * u;
+            cfg.gridDim = dim3((unsigned)ceil_div(N, rows));
+            cfg.blockDim = dim3((unsigned)th);
+            e = cudaLaunchKernelEx(&cfg, kern, W, ldw, x, iN, iK, ikw, alpha, y_i32, y_f32, weights_static ? 1 : 0,
+                                   inputs_static ? 1 : 0, independent ? 2 : 1);
+            if (e != cudaSuccess) return BNN_ERR_CUDA;
+            return launch_status();
+        };
+        if (independent) return go(bnn::xnor_gemv_row128_kernel<XT, 256, 12>, 256, 12);
+        if (weights_static && inputs_static) return go(bnn::xnor_gemv_row128_kernel<XT, 128, 8>, 128, 8);
+        return go(bnn::xnor_gemv_row128_kernel<XT, 768, 2>, 768, 2);
     }
 #define BNN_GEMV_PICK(L, S, P)                                                                      \
     (vec ? launch(bnn::xnor_gemv_kernel<XT, L, S, P, true>) : launch(bnn::xnor_gemv_kernel<XT, L, S, P, false>))

@@ -46,8 +46,8 @@ constexpr int BN = 256;                    // tile cols  = UMMA N
 constexpr int BKE = 128;                   // binary elements of K per stage (4 packed words)
 constexpr int BKW = BKE / 32;
 constexpr int UMMA_K = 32;                 // int8 K per tcgen05.mma
-constexpr int PSTAGES = 8;                 // packed ring
-constexpr int USTAGES = 3;                 // unpacked (int8) ring
+constexpr int PSTAGES = 4;                 // packed ring
+constexpr int USTAGES = 4;                 // unpacked (int8) ring
 constexpr int P_A_BYTES = BM * BKW * 4;    // 2 KiB
 constexpr int P_B_BYTES = BN * BKW * 4;    // 4 KiB
 constexpr int P_STAGE = P_A_BYTES + P_B_BYTES;

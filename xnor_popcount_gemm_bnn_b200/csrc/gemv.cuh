@@ -26,10 +26,9 @@
 
 namespace bnn {
 namespace gemv {
-// 512 threads x 2 row groups per warp (32 rows of K = 4096 per CTA): the
-// shape with the shortest step time in back-to-back dependent launches, where
-// each grid waits for the previous one (measured against 256 x 4, 256 x 2,
-// 512 x 1..4, 1024 x 1..2).
+// Block shape of the general kernel: 512 threads x 2 row groups per warp.
+// (The one-chunk-per-lane kernel below takes its shape as template
+// parameters, chosen per dependency mode by the launcher.)
 constexpr int THREADS = 512;
 constexpr int WARPS = THREADS / 32;
 constexpr int U = 2;   // row groups per warp
@@ -104,12 +103,16 @@ __device__ __forceinline__ void gemv_pack_x(const XT* __restrict__ x, int K, int
 // x pack is one vector per thread per round (E elements; 32/E lanes OR their
 // bits into a word).  Measured about 20% shorter steps than the generic
 // kernel in dependent back-to-back launches.
-template <typename XT>
-__global__ void __launch_bounds__(gemv::THREADS)
+//
+// The block shape (TH threads, U rows per warp) is a template parameter: the
+// launcher picks it per dependency mode (see row128_shape in the library).
+template <typename XT, int TH, int U>
+__global__ void __launch_bounds__(TH)
 xnor_gemv_row128_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restrict__ x, int N, int K,
                         int kw, const float* __restrict__ alpha, int32_t* __restrict__ y_i32,
                         float* __restrict__ y_f32, int prefetch, int xstatic, int dependent) {
-    using namespace gemv;
+    constexpr int THREADS = TH;
+    constexpr int WARPS = TH / 32;
     constexpr int E = 16 / (int)sizeof(XT);           // elements per 16-byte vector
     constexpr int G = 32 / E;                         // lanes per packed word
     extern __shared__ __align__(16) uint32_t xs[];
