@@ -46,8 +46,8 @@ constexpr int BN = 256;                    // tile cols  = UMMA N
 constexpr int BKE = 128;                   // binary elements of K per stage (4 packed words)
 constexpr int BKW = BKE / 32;
 constexpr int UMMA_K = 32;                 // int8 K per tcgen05.mma
-constexpr int PSTAGES = 4;                 // packed ring
-constexpr int USTAGES = 4;                 // unpacked (int8) ring
+constexpr int PSTAGES = 8;                 // packed ring
+constexpr int USTAGES = 3;                 // unpacked (int8) ring
 constexpr int P_A_BYTES = BM * BKW * 4;    // 2 KiB
 constexpr int P_B_BYTES = BN * BKW * 4;    // 4 KiB
 constexpr int P_STAGE = P_A_BYTES + P_B_BYTES;
@@ -60,7 +60,10 @@ constexpr int WARP_PRODUCER = 0, WARP_MMA = 1, WARP_UNPACK0 = 2, WARP_EPI0 = WAR
 constexpr int THREADS = (WARP_EPI0 + EPI_WARPS) * 32;   // 576
 constexpr int TMEM_COLS = 2 * BN;          // two accumulators
 constexpr int NUM_BARS = 2 * PSTAGES + 2 * USTAGES + 2 * 2 + 1;
-constexpr int SMEM_BYTES = USTAGES * U_STAGE + PSTAGES * P_STAGE + NUM_BARS * 8 + 16 + 1024;
+// Per-tile epilogue column parameters, two buffers (by tile parity): float4
+// {alpha, gamma, beta, -} and int2 {c1, len2} of the threshold test per column.
+constexpr int COLP_BYTES = 2 * BN * (16 + 8);
+constexpr int SMEM_BYTES = USTAGES * U_STAGE + PSTAGES * P_STAGE + COLP_BYTES + NUM_BARS * 8 + 16 + 1024;
 // kind::i8 instruction descriptor: D s32 (bits 4-5 = 2), A s8 (bits 7-9 = 1),
 // B s8 (bits 10-12 = 1), both K-major, N >> 3 at bits 17-22, M >> 4 at 24-28.
 constexpr uint32_t IDESC = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
@@ -174,7 +177,9 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* uring = smem;                                   // USTAGES x (A 16 KiB | W 32 KiB)
     uint8_t* pring = smem + USTAGES * U_STAGE;               // PSTAGES x (A 2 KiB | W 4 KiB)
-    uint64_t* bars = reinterpret_cast<uint64_t*>(pring + PSTAGES * P_STAGE);
+    float4* colf = reinterpret_cast<float4*>(pring + PSTAGES * P_STAGE);      // [2][BN]
+    int2* colt = reinterpret_cast<int2*>(colf + 2 * BN);                       // [2][BN]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(colt + 2 * BN);
     uint64_t* pfull = bars;
     uint64_t* pempty = pfull + PSTAGES;
     uint64_t* ufull = pempty + PSTAGES;
@@ -309,15 +314,58 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
     } else {
         // ------------------------------ epilogue warps ------------------------------
+        // Per tile, the 128 epilogue threads first stage the tile's column
+        // parameters in shared memory (alpha/gamma/beta and the threshold test
+        // as one unsigned range check on the raw accumulator), then each thread
+        // turns its row's 256 accumulators into outputs with broadcast shared
+        // loads instead of per-column global loads.
         const int quad = warp & 3;                                    // TMEM lanes 32*quad .. 32*quad + 31
-        const int pad = nk * BKE - K;                                 // (+1)(+1) pad positions per output
+        const int etid = threadIdx.x - WARP_EPI0 * 32;                // 0..127
+        const int kp = nk * BKE;                                      // padded K: acc = kp - 2 * popcount
+        const int pad = kp - K;                                       // (+1)(+1) pad positions per output
+        const bool affine = ep.gamma != nullptr;
         int lt = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++lt) {
             const int b = lt & 1;
+            const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
+            // Stage this tile's columns into buffer b (its previous reader, tile
+            // lt - 2, finished before every epilogue warp passed tile lt - 1's
+            // barrier below).
+            for (int i = etid; i < BN; i += EPI_WARPS * 32) {
+                const int n = n0 + i;
+                float4 f = make_float4(0.f, 1.f, 0.f, 0.f);
+                int2 th = make_int2(0, 0);                            // len2 = 0: bit never set
+                if (n < N) {
+                    if (ep.alpha != nullptr) f.x = __ldg(ep.alpha + n);
+                    if (affine) { f.y = __ldg(ep.gamma + n); f.z = __ldg(ep.beta + n); }
+                    if (ep.c_bits != nullptr) {
+                        // d = popcount = (kp - acc) / 2 lies in [0, K].  mode 0: bit = d > T,
+                        // the interval [max(T+1, 0), K]; mode 1: bit = d < T, the interval
+                        // [0, min(T-1, K)]; other modes: empty.  With lo and len of the
+                        // interval, bit = (unsigned)(d - lo) < len, which is
+                        // (unsigned)(c1 - acc) < 2*len for c1 = kp - 2*lo (kp - acc is even).
+                        const long long T = __ldg(ep.thresh + n);
+                        const int md = ep.thresh_mode[n];
+                        long long lo = 0, len = 0;
+                        if (md == 0) {
+                            lo = T + 1 > 0 ? T + 1 : 0;
+                            len = K - lo + 1 > 0 ? K - lo + 1 : 0;
+                        } else if (md == 1) {
+                            len = T < K + 1 ? T : K + 1;
+                            if (len < 0) len = 0;
+                        }
+                        th = make_int2((int)(uint32_t)(kp - 2 * lo), (int)(uint32_t)(2 * len));
+                    }
+                }
+                colf[b * BN + i] = f;
+                colt[b * BN + i] = th;
+            }
+            asm volatile("bar.sync 1, %0;" ::"r"(EPI_WARPS * 32) : "memory");
             if (!__all_sync(0xffffffffu, tc_wait(&afull[b], (lt >> 1) & 1, abort_flag))) break;
             tc_fence_after();
-            const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
             const int m = m0 + 32 * quad + lane;
+            const float4* cf = colf + b * BN;
+            const int2* ct = colt + b * BN;
             #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t r[32];
@@ -341,15 +389,8 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     uint32_t word = 0;
                     #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        const int n = nb + j;
-                        const int32_t d = (K - ((int32_t)r[j] - pad)) / 2;   // popcount of the XOR
-                        bool bit = false;
-                        if (n < N) {
-                            const int md = ep.thresh_mode[n];
-                            const int th = ep.thresh[n];
-                            bit = md == 0 ? (d > th) : (md == 1 ? (d < th) : false);
-                        }
-                        word |= (bit ? 1u : 0u) << j;
+                        const int2 q = ct[32 * c + j];
+                        word |= ((uint32_t)(q.x - (int32_t)r[j]) < (uint32_t)q.y ? 1u : 0u) << j;
                     }
                     if (m < M && nb / 32 < ep.bits_words) ep.c_bits[(int64_t)m * ep.ldb + nb / 32] = word;
                 }
@@ -378,9 +419,9 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         float y[4];
                         #pragma unroll
                         for (int k = 0; k < 4; ++k) {
-                            const int n = min(nb + j + k, N - 1);
-                            float v = __ldg(ep.alpha + n) * (float)((int32_t)r[j + k] - pad);
-                            if (ep.gamma != nullptr) v = fmaf(__ldg(ep.gamma + n), v, __ldg(ep.beta + n));
+                            const float4 f = cf[32 * c + j + k];
+                            float v = f.x * (float)((int32_t)r[j + k] - pad);
+                            if (affine) v = fmaf(f.y, v, f.z);
                             y[k] = v;
                         }
                         if (vec) {
