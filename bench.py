@@ -112,6 +112,7 @@ KERNEL_SOURCES = {
     "xnor_conv3x3_kernel": ("conv.cuh", "common.cuh"),
     "xnor_conv3x3_tcw_kernel": ("conv_tc.cuh", "conv.cuh", "gemm_tc.cuh", "gemm_popc.cuh", "common.cuh"),
     "pack_sign_rows_kernel": ("pack.cuh", "common.cuh"),
+    "pack_sign_nchw_kernel": ("pack.cuh", "common.cuh"),
 }
 
 
@@ -602,7 +603,8 @@ def _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk):
             "ms_per_step": ms_c / steps, "conv_kernel_ms": ms_ck / steps,
             "conv_kernel_binary_tmac_s": round(cmac_s / 1e12, 2), "roofline": roof,
             "pack_nchw": {"ms": ms_pack / steps, "achieved_gbs": round(pack_gbs, 1),
-                          "frac": round(pack_gbs / pk["hbm_gbs"], 4), "bytes": pbytes},
+                          "frac": round(pack_gbs / pk["hbm_gbs"], 4), "bytes": pbytes,
+                          "traffic": recorded_traffic("pack_sign_nchw_kernel")},
             "l2": f"{R} rotating input/output sets, {rot_mb:.0f} MB"}
     del cv, Xd, Xb, Wc, alc, gam, bet, out
     torch.cuda.empty_cache()
