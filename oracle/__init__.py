@@ -147,6 +147,26 @@ def gemv_pm1(w: np.ndarray, x: np.ndarray) -> np.ndarray:
     return matmul_pm1(np.asarray(x, dtype=np.int8)[None, :], w)[0]
 
 
+def binary_weight_product(w: np.ndarray, x) -> np.ndarray:
+    """float64 [N]: sum_i sign(w_ni) * x_i for int8 +1/-1 w [N, K] and a real
+    x [K] -- "Extreme Quantization: Binary, Ternary & 1-bit LLMs", Binary
+    Neural Networks, eq. (1) without alpha, with eq. (2): each term is +x_i
+    where the weight is +1 and -x_i where it is -1 (no multiplication).  The
+    terms are added in float64."""
+    w = np.asarray(w, dtype=np.int8)
+    xd = np.asarray(x, dtype=np.float64)
+    return np.where(w > 0, xd[None, :], -xd[None, :]).sum(axis=1)
+
+
+def binary_weight_gemv(w_real, x_real) -> tuple[np.ndarray, np.ndarray]:
+    """eq. (1): y = alpha * (w_b^T x) per output row with binary weights and
+    real activations; returns (alpha float64, y float64).  x is taken as
+    stored (bf16 inputs widened exactly)."""
+    wb = sign_pm1(w_real)
+    a = alpha(w_real)
+    return a, scaled(binary_weight_product(wb, _f32(x_real)), a)
+
+
 def conv2d_pm1(x: np.ndarray, f: np.ndarray, stride: int = 1, pad: int = 1) -> np.ndarray:
     """int32 NCHW output of a square-kernel convolution on +1/-1 tensors,
     padded taps reading +1."""

@@ -119,7 +119,28 @@ def _bn_sign_strict(s, a, g, b, mu, var, eps):   # tie (value 0) goes to -1
     return np.where(y > 0, 1, -1).astype(np.int8)
 
 
+def _bw_sign_swapped(w, x):            # +x where the weight is -1 (encoding read backwards)
+    w = np.asarray(w, np.int8)
+    xd = np.asarray(x, np.float64)
+    return np.where(w > 0, -xd[None, :], xd[None, :]).sum(axis=1)
+
+
+def _bw_drop_last(w, x):               # the last term is lost
+    w = np.asarray(w, np.int8)
+    xd = np.asarray(x, np.float64)
+    return np.where(w > 0, xd[None, :], -xd[None, :])[:, :-1].sum(axis=1)
+
+
+def _bw_abs_x(w, x):                   # adds |x| instead of x
+    w = np.asarray(w, np.int8)
+    xd = np.abs(np.asarray(x, np.float64))
+    return np.where(w > 0, xd[None, :], -xd[None, :]).sum(axis=1)
+
+
 MUTANTS = {
+    "bw_sign_swapped": dict(binary_weight_product=_bw_sign_swapped),
+    "bw_dropped_term": dict(binary_weight_product=_bw_drop_last),
+    "bw_abs_activation": dict(binary_weight_product=_bw_abs_x),
     "sign_zero_negative": dict(sign_pm1=_sign_gt),
     "sign_bit_test": dict(sign_pm1=_sign_bit),
     "pack_msb_first": dict(pack_pm1=_pack_msb),

@@ -282,6 +282,32 @@ def check_mlp_library(o, seed=0):
             assert np.allclose(logits, (al * s).numpy(), rtol=1e-13, atol=0)
 
 
+def check_binary_weight_product(o):
+    """eq. (1)-(2) of 'Extreme Quantization ...' (binary weights, real x):
+    brute force by the case split of eq. (2) for K <= 6, the closed form for a
+    constant x, torch float64 matmul, and the reduction to the binary product
+    when x itself is +1/-1."""
+    rng = np.random.default_rng(11)
+    for K in range(1, 7):
+        V = all_pm1_vectors(K)
+        x = rng.standard_normal(K)
+        y = o.binary_weight_product(V, x)
+        for r, w in enumerate(V):
+            ref = 0.0
+            for i in range(K):
+                ref = ref + (x[i] if w[i] == 1 else -x[i])      # eq. (2), term by term
+            assert abs(y[r] - ref) <= 1e-12 * np.abs(x).sum(), (K, r)
+    w = np.where(rng.random((9, 300)) < 0.4, -1, 1).astype(np.int8)
+    c = 0.75
+    y = o.binary_weight_product(w, np.full(300, c))
+    assert np.array_equal(y, c * (300 - 2 * (w == -1).sum(axis=1)))
+    x = rng.standard_normal(300)
+    ref = (torch.from_numpy(w).double() @ torch.from_numpy(x)).numpy()
+    assert np.allclose(o.binary_weight_product(w, x), ref, rtol=0, atol=1e-12 * np.abs(x).sum())
+    xb = np.where(rng.random(300) < 0.5, -1, 1).astype(np.int8)
+    assert np.array_equal(o.binary_weight_product(w, xb).astype(np.int64), o.gemv_pm1(w, xb).astype(np.int64))
+
+
 ALL_CHECKS = [
     ("identity_bruteforce", lambda o, g: check_identity_bruteforce(o)),
     ("elementwise_xnor_form", lambda o, g: check_elementwise_xnor_form(o)),
@@ -297,6 +323,7 @@ ALL_CHECKS = [
     ("conv_library", lambda o, g: check_conv_library(o)),
     ("bn", lambda o, g: check_bn(o)),
     ("mlp_library", lambda o, g: check_mlp_library(o)),
+    ("binary_weight_product", lambda o, g: check_binary_weight_product(o)),
 ]
 
 
