@@ -113,6 +113,7 @@ KERNEL_SOURCES = {
     "xnor_conv3x3_tcw_kernel": ("conv_tc.cuh", "conv.cuh", "gemm_tc.cuh", "gemm_popc.cuh", "common.cuh"),
     "pack_sign_rows_kernel": ("pack.cuh", "common.cuh"),
     "pack_sign_nchw_kernel": ("pack.cuh", "common.cuh"),
+    "bw_gemv_kernel": ("bwgemv.cuh", "common.cuh"),
 }
 
 
@@ -448,7 +449,7 @@ def e2e_gemv(torch, bnn, g, Ws, alpha, dev, steps, sync, max_over_ranks, ws):
 # the other rows
 # ---------------------------------------------------------------------------
 
-ROW_NAMES = ("pack_sign_weights", "square_gemm", "conv3x3", "mlp4")
+ROW_NAMES = ("pack_sign_weights", "square_gemm", "conv3x3", "mlp4", "bw_gemv")
 
 
 def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws, only=None):
@@ -471,6 +472,8 @@ def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws, o
         _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk)
     if "mlp4" in want:
         _row_mlp(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk)
+    if "bw_gemv" in want:
+        _row_bw_gemv(torch, bnn, workloads, dev, pk, rows, timed, ws)
     if bnn.bnn_device_error() != 0:
         raise RuntimeError("a kernel reported a device-side timeout")
     return rows
@@ -607,6 +610,39 @@ def _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk):
                           "traffic": recorded_traffic("pack_sign_nchw_kernel")},
             "l2": f"{R} rotating input/output sets, {rot_mb:.0f} MB"}
     del cv, Xd, Xb, Wc, alc, gam, bet, out
+    torch.cuda.empty_cache()
+
+
+def _row_bw_gemv(torch, bnn, workloads, dev, pk, rows, timed, ws):
+    # --- next row: binary weights x real (bf16) activations, the decode shape ---
+    g = workloads.gemv()
+    copies = max(2, math.ceil(2 * L2_BYTES / gemv_bytes()) + 1)
+    copies = (copies + 7) // 8 * 8
+    W_p = bnn.empty_packed(g.N, g.K, dev)
+    alpha = torch.empty(g.N, dtype=torch.float32, device=dev)
+    bnn.bnn_pack_sign(g.W.to(dev), W_p, alpha)
+    Ws = [W_p] + [W_p.clone() for _ in range(copies - 1)]
+    ys = [torch.empty(g.N, dtype=torch.float32, device=dev) for _ in range(copies)]
+    x = g.x.to(dev)
+    steps = 48 * copies
+    all_flags = bnn.BNN_GEMV_WEIGHTS_STATIC | bnn.BNN_GEMV_INPUTS_STATIC | bnn.BNN_GEMV_OUTPUT_FREE
+    ms = timed(lambda i: bnn.bnn_binary_weight_gemv(Ws[i % copies], x, g.K, alpha, ys[i % copies], flags=all_flags),
+               n=steps, period=copies)
+    ms_dep = timed(lambda i: bnn.bnn_binary_weight_gemv(Ws[i % copies], x, g.K, alpha, ys[0],
+                                                        flags=bnn.BNN_GEMV_WEIGHTS_STATIC), n=steps, period=copies)
+    b = gemv_bytes()
+    ach = b * steps / (ms * 1e-3) / 1e9
+    ach_dep = b * steps / (ms_dep * 1e-3) / 1e9
+    rows["bw_gemv"] = {
+        "workload": "binary weights x real activations (eq. (1)): packed W [11008, 4096], x bf16 [4096] "
+                    "not binarised, alpha-scaled fp32 y; independent steps over 48 rotating weight copies",
+        "value": round(ws * ach, 1), "unit": "GB/s", "ms_per_step": ms / steps,
+        "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"],
+                     "frac": round(ach / pk["hbm_gbs"], 4), "algorithmic_bytes": b,
+                     "traffic": recorded_traffic("bw_gemv_kernel")},
+        "dependent_chain": {"value": round(ws * ach_dep, 1), "unit": "GB/s", "ms_per_step": ms_dep / steps,
+                            "frac": round(ach_dep / pk["hbm_gbs"], 4)}}
+    del Ws, ys, W_p, x, g
     torch.cuda.empty_cache()
 
 

@@ -265,6 +265,26 @@ bnn_status bnn_xnor_gemv_ex(const uint32_t* W, int64_t ldw, const void* x, bnn_d
                             int64_t N, int64_t K, const float* alpha,
                             int32_t* y_i32, float* y_f32, uint32_t flags, bnn_stream_t stream);
 
+/* bnn_binary_weight_gemv -- binary weights times a REAL activation vector:
+ *   y[n] = alpha[n] * sum_k sign(W[n,k]) * x[k]
+ * ("Extreme Quantization: Binary, Ternary & 1-bit LLMs", Binary Neural
+ * Networks, eq. (1)-(2): every term is +x_k or -x_k, no multiplication).
+ * Unlike bnn_xnor_gemv, x is not binarised.
+ *   W        device, packed [N, ldw] as produced by bnn_pack_sign (16-B aligned,
+ *            ldw % 4 == 0, pad bits zero).  kw = bnn_packed_ld_words(K) <= 384
+ *            (K <= 12288; the per-block add table lives in shared memory).
+ *   x        device fp32 or bf16 [K] (x_dt).
+ *   alpha    device fp32 [N], required; y device fp32 [N].
+ *   flags    as for bnn_xnor_gemv_ex (BNN_GEMV_WEIGHTS_STATIC,
+ *            BNN_GEMV_INPUTS_STATIC, BNN_GEMV_OUTPUT_FREE).
+ * Accumulation is fp32: a 16-entry table of +-x0 +-x1 +-x2 +-x3 per group
+ * of 4 elements, then one lookup and one add per 4 weights, 32 adds per
+ * partial sum at K = 4096, and 8 partial sums per row.
+ *   Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (K too large), CUDA. */
+bnn_status bnn_binary_weight_gemv(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt,
+                                  int64_t N, int64_t K, const float* alpha, float* y,
+                                  uint32_t flags, bnn_stream_t stream);
+
 /* bnn_binary_linear_fused -- packed binary GEMM with one fused epilogue.
  *   Passage: eq. (6) (product), eq. (1) (alpha), the glossary's BatchNorm
  *   paragraph (normalise, then binarise for the next layer).

@@ -153,3 +153,16 @@ def test_gemm_engine_setting_on_host():
     assert L.bnn_set_gemm_engine(bnn.BNN_GEMM_ENGINE_TENSOR) == bnn.BNN_OK
     assert bnn.bnn_get_gemm_engine() == bnn.BNN_GEMM_ENGINE_TENSOR
     bnn.bnn_set_gemm_engine(prev)
+
+
+def test_binary_weight_gemv_rejects_bad_arguments():
+    f = L.bnn_binary_weight_gemv
+    assert f(FAKE, 4, FAKE, 0, 8, 32, FAKE, FAKE, 8, NULL) == bnn.BNN_ERR_INVALID_ARG       # unknown flag
+    assert f(FAKE, 4, NULL, 0, 8, 32, FAKE, FAKE, 0, NULL) == bnn.BNN_ERR_INVALID_ARG       # no x
+    assert f(FAKE, 4, FAKE, 0, 8, 32, NULL, FAKE, 0, NULL) == bnn.BNN_ERR_INVALID_ARG       # alpha required
+    assert f(FAKE, 4, FAKE, 0, 8, 32, FAKE, NULL, 0, NULL) == bnn.BNN_ERR_INVALID_ARG       # no y
+    assert f(FAKE, 4, FAKE, 7, 8, 32, FAKE, FAKE, 0, NULL) == bnn.BNN_ERR_INVALID_ARG       # dtype
+    assert f(FAKE, 6, FAKE, 0, 8, 32, FAKE, FAKE, 0, NULL) == bnn.BNN_ERR_ALIGNMENT         # ld % 4
+    assert f(FAKE_ODD, 4, FAKE, 0, 8, 32, FAKE, FAKE, 0, NULL) == bnn.BNN_ERR_ALIGNMENT
+    assert f(FAKE, 388, FAKE, 0, 8, 12289, FAKE, FAKE, 0, NULL) == bnn.BNN_ERR_UNSUPPORTED  # table too large
+    assert f(FAKE, 4, FAKE, 0, 0, 32, FAKE, FAKE, 7, NULL) == bnn.BNN_OK                    # N = 0: nothing to do

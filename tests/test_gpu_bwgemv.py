@@ -1,0 +1,111 @@
+"""Binary weights x real activations GEMV ("Extreme Quantization ...", Binary
+Neural Networks, eq. (1)-(2)) against the oracle's float64 add/sub sum.
+
+Tolerance, derived from the kernel's fp32 arithmetic (u = 2^-24): a table
+entry +-x0 +-x1 +-x2 +-x3 takes 3 roundings, each of the 4 accumulators of a
+lane adds ceil(K/128) entries, the 4 accumulators and the 8 partial sums of a
+row take 9 more additions, and alpha*s one multiplication.  So
+|y - y_ref| <= alpha * (ceil(K/128) + 12) * u * sum|x| + 2u * |y_ref| (the
+second term also covers alpha rounded to fp32)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import xnor_popcount_gemm_bnn_b200 as bnn
+from gpu_util import assert_no_device_error, dev
+
+pytestmark = pytest.mark.gpu
+
+U = 2.0 ** -24
+
+
+def check(y, W, x, K):
+    a, y_ref = oracle.binary_weight_gemv(W, x)
+    sx = np.abs(oracle._f32(x).astype(np.float64)).sum()
+    tol = a * (math.ceil(K / 128) + 12) * U * sx * 1.05 + 2 * U * np.abs(y_ref) * 1.05
+    err = np.abs(y.detach().cpu().numpy().astype(np.float64) - y_ref)
+    bad = np.nonzero(err > tol)[0]
+    assert bad.size == 0, f"{bad.size} rows outside the bound, first {bad[:5]}: err {err[bad[:5]]} tol {tol[bad[:5]]}"
+
+
+def run(W, x, K, flags=0):
+    d = dev()
+    N = W.shape[0]
+    Wp = bnn.empty_packed(N, K, d)
+    al = torch.empty(N, dtype=torch.float32, device=d)
+    bnn.bnn_pack_sign(W.to(d), Wp, al)
+    y = torch.full((N,), float("nan"), dtype=torch.float32, device=d)
+    bnn.bnn_binary_weight_gemv(Wp, x.to(d), K, al, y, flags=flags)
+    torch.cuda.synchronize()
+    return y
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("N,K", [(1, 1), (5, 31), (64, 1000), (65, 33), (300, 4096), (100, 4100),
+                                 (129, 8192), (33, 12288)])
+@pytest.mark.parametrize("flags", [0, 3, 7])
+def test_bw_gemv_shapes(N, K, dtype, flags):
+    W = workloads.normal((N, K), 1.0, N + K)
+    x = workloads.normal((K,), 1.0, K + 7, dtype=dtype)
+    y = run(W, x, K, flags)
+    check(y, W, x, K)
+    assert_no_device_error()
+
+
+def test_bw_gemv_decode_workload():
+    """The decode shape: W [11008, 4096] ~ N(0, 0.02) (the GEMV workload's
+    weights), x bf16 [4096] ~ N(0, 1) used as a real activation."""
+    g = workloads.gemv()
+    y = run(g.W, g.x, g.K, flags=bnn.BNN_GEMV_WEIGHTS_STATIC)
+    check(y, g.W, g.x, g.K)
+    assert_no_device_error()
+
+
+def test_bw_gemv_special_values():
+    """Signed zeros and exact halves of x: every term is exact, and a +1/-1 x
+    reduces to the binary product (K - 2 popcount)."""
+    K, N = 256, 40
+    W = workloads.normal((N, K), 1.0, 5)
+    xb = torch.where(workloads.normal((K,), 1.0, 6) < 0, -1.0, 1.0)
+    y = run(W, xb, K)
+    s_ref = oracle.gemv_pm1(oracle.sign_pm1(W), oracle.sign_pm1(xb))
+    a = oracle.alpha(W)
+    assert np.allclose(y.cpu().numpy(), a * s_ref, rtol=4 * U, atol=0)
+    x0 = torch.zeros(K)
+    x0[::2] = -0.0
+    y0 = run(W, x0, K)
+    assert torch.count_nonzero(y0) == 0
+
+
+def test_bw_gemv_store_order_and_independent_calls():
+    """BNN_GEMV_WEIGHTS_STATIC | BNN_GEMV_INPUTS_STATIC: consecutive calls
+    that write one y keep stream order; with all three flags, calls over
+    separate outputs are each exact."""
+    d = dev()
+    N, K, L = 500, 2048, 5
+    Ws = [workloads.normal((N, K), 1.0, 40 + l) for l in range(L)]
+    xs = [workloads.normal((K,), 1.0, 50 + l, dtype=torch.bfloat16) for l in range(L)]
+    Wp, al = [], []
+    for W in Ws:
+        p = bnn.empty_packed(N, K, d)
+        a = torch.empty(N, dtype=torch.float32, device=d)
+        bnn.bnn_pack_sign(W.to(d), p, a)
+        Wp.append(p)
+        al.append(a)
+    xd = [x.to(d) for x in xs]
+    ys = [torch.empty(N, dtype=torch.float32, device=d) for _ in range(L)]
+    shared = torch.empty(N, dtype=torch.float32, device=d)
+    torch.cuda.synchronize()
+    for l in range(L):
+        bnn.bnn_binary_weight_gemv(Wp[l], xd[l], K, al[l], ys[l], flags=7)
+    for l in range(L):
+        bnn.bnn_binary_weight_gemv(Wp[l], xd[l], K, al[l], shared, flags=3)
+    torch.cuda.synchronize()
+    for l in range(L):
+        check(ys[l], Ws[l], xs[l], K)
+    assert torch.equal(shared, ys[L - 1])
+    assert_no_device_error()

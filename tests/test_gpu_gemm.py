@@ -190,3 +190,29 @@ def test_engines_agree_bit_for_bit():
     assert torch.equal(outs[0][0], outs[1][0])
     assert torch.equal(outs[0][1], outs[1][1])
     assert_no_device_error()
+
+
+def test_tensor_engine_full_matrix_repeated():
+    """Races show up as a few wrong tiles in some launches only, so the square
+    workload runs 8 times on the tensor engine and every one of the 67M int32
+    outputs is compared with the popcount engine's (two independent kernels;
+    the popcount result is itself checked against the oracle above).  Once with
+    fp32 alpha outputs too, whose epilogue parameters come from shared memory."""
+    sq = workloads.square()
+    A_p, W_p, alpha = packed_operands(sq.A, sq.W)
+    ref = torch.empty(sq.M, sq.N, dtype=torch.int32, device=dev())
+    ref_f = torch.empty(sq.M, sq.N, dtype=torch.float32, device=dev())
+    with bnn.gemm_engine(bnn.BNN_GEMM_ENGINE_POPCOUNT):
+        bnn.bnn_xnor_gemm(A_p, W_p, sq.K, alpha, ref, ref_f)
+    C = torch.empty_like(ref)
+    Cf = torch.empty_like(ref_f)
+    with bnn.gemm_engine(bnn.BNN_GEMM_ENGINE_TENSOR):
+        for r in range(8):
+            C.fill_(0x5A5A5A5A)
+            Cf.fill_(float("nan"))
+            bnn.bnn_xnor_gemm(A_p, W_p, sq.K, alpha if r == 0 else None, C, Cf if r == 0 else None)
+            torch.cuda.synchronize()
+            assert torch.equal(C, ref), f"launch {r}: {int((C != ref).sum())} outputs differ"
+            if r == 0:
+                assert torch.equal(Cf, ref_f)
+    assert_no_device_error()

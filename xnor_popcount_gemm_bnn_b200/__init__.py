@@ -48,6 +48,7 @@ EXPORTS = (
     "bnn_pack_sign", "bnn_pack_sign_nchw", "bnn_pack_conv3x3_weights", "bnn_xnor_gemm",
     "bnn_xnor_gemv", "bnn_xnor_gemv_ex", "bnn_binary_linear_fused", "bnn_binary_conv3x3_fused",
     "bnn_fold_bn_threshold", "bnn_set_gemm_engine", "bnn_get_gemm_engine", "bnn_selftest_wait_timeout",
+    "bnn_binary_weight_gemv",
 )
 
 
@@ -80,6 +81,7 @@ def _load() -> ctypes.CDLL:
         "bnn_xnor_gemm": (i32, [p, i64, p, i64, i64, i64, i64, p, p, i64, p, i64, p]),
         "bnn_xnor_gemv": (i32, [p, i64, p, i32, i64, i64, p, p, p, p]),
         "bnn_xnor_gemv_ex": (i32, [p, i64, p, i32, i64, i64, p, p, p, ctypes.c_uint32, p]),
+        "bnn_binary_weight_gemv": (i32, [p, i64, p, i32, i64, i64, p, p, ctypes.c_uint32, p]),
         "bnn_binary_linear_fused": (i32, [p, i64, p, i64, i64, i64, i64,
                                           ctypes.POINTER(bnn_epilogue), p, i64, p]),
         "bnn_binary_conv3x3_fused": (i32, [p, i64, i64, i64, i64, p, i64, i64, i64, i64,
@@ -248,6 +250,15 @@ def bnn_xnor_gemv_ex(W: torch.Tensor, x: torch.Tensor, K: Optional[int] = None,
     _check("bnn_xnor_gemv_ex", _lib.bnn_xnor_gemv_ex(
         _ptr(W), _ld(W), _ptr(x), _dtype(x), N, K, _ptr(alpha), _ptr(y_i32), _ptr(y_f32),
         int(flags), _stream(stream)))
+
+
+def bnn_binary_weight_gemv(W: torch.Tensor, x: torch.Tensor, K: Optional[int], alpha: torch.Tensor,
+                           y: torch.Tensor, flags: int = 0, N: Optional[int] = None, stream=None) -> None:
+    """y = alpha * (sign(W) x) with a real x (fp32 or bf16), W packed."""
+    N = W.shape[0] if N is None else N
+    K = x.shape[-1] if K is None else int(K)
+    _check("bnn_binary_weight_gemv", _lib.bnn_binary_weight_gemv(
+        _ptr(W), _ld(W), _ptr(x), _dtype(x), N, K, _ptr(alpha), _ptr(y), int(flags), _stream(stream)))
 
 
 def make_epilogue(mode: int, alpha=None, gamma=None, beta=None, popc_thresh=None,

@@ -18,6 +18,7 @@
 #include "gemm_popc.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "bwgemv.cuh"
 #include "pack.cuh"
 
 namespace {
@@ -90,6 +91,23 @@ bool gemm_tc_smem_configured() {
     if (dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return true;
     if (cudaFuncSetAttribute(bnn::xnor_gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              bnn::tc::SMEM_BYTES) != cudaSuccess)
+        return false;
+    if (dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
+    return true;
+}
+
+// Per-device one-time opt-in to the add table of the binary-weight GEMV.
+bool bw_gemv_smem_configured() {
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> done[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+    if (dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return true;
+    const int bytes = bnn::bwg::smem_bytes(bnn::bwg::MAX_KW);
+    if (cudaFuncSetAttribute(bnn::bw_gemv_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(bnn::bw_gemv_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bytes) != cudaSuccess)
         return false;
     if (dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
     return true;
@@ -427,6 +445,46 @@ bnn_status bnn_xnor_gemv_ex(const uint32_t* W, int64_t ldw, const void* x, bnn_d
     if ((flags & ~kAll) != 0) return BNN_ERR_INVALID_ARG;
     return gemv_impl(W, ldw, x, x_dt, N, K, alpha, y_i32, y_f32, (flags & BNN_GEMV_WEIGHTS_STATIC) != 0,
                      (flags & BNN_GEMV_INPUTS_STATIC) != 0, flags == kAll, stream);
+}
+
+bnn_status bnn_binary_weight_gemv(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt, int64_t N,
+                                  int64_t K, const float* alpha, float* y, uint32_t flags, bnn_stream_t stream) {
+    constexpr uint32_t kAll = BNN_GEMV_WEIGHTS_STATIC | BNN_GEMV_INPUTS_STATIC | BNN_GEMV_OUTPUT_FREE;
+    if ((flags & ~kAll) != 0) return BNN_ERR_INVALID_ARG;
+    if (x == nullptr || alpha == nullptr || y == nullptr) return BNN_ERR_INVALID_ARG;
+    if (N < 0 || K < 1 || N > INT_MAX || K > INT_MAX / 2) return BNN_ERR_INVALID_ARG;
+    if (x_dt != BNN_F32 && x_dt != BNN_BF16) return BNN_ERR_INVALID_ARG;
+    const int64_t kw = packed_ld_words(K);
+    bnn_status st = check_packed_operand(W, ldw, kw);
+    if (st != BNN_OK) return st;
+    if (kw > bnn::bwg::MAX_KW) return BNN_ERR_UNSUPPORTED;
+    if (!aligned(x, x_dt == BNN_F32 ? 4 : 2) || !aligned(alpha, 4) || !aligned(y, 4)) return BNN_ERR_ALIGNMENT;
+    if (N == 0) return BNN_OK;
+    if (!bw_gemv_smem_configured()) return BNN_ERR_CUDA;
+    const int64_t blocks = ceil_div(N, (int64_t)(bnn::bwg::RG * 32));
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(bnn::bwg::THREADS);
+    cfg.dynamicSmemBytes = (size_t)bnn::bwg::smem_bytes((int)kw);
+    cfg.stream = as_cuda(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const int prefetch = (flags & BNN_GEMV_WEIGHTS_STATIC) ? 1 : 0;
+    const int xstatic = (flags & BNN_GEMV_INPUTS_STATIC) ? 1 : 0;
+    const int dependent = flags == kAll ? 2 : 1;
+    cudaError_t e;
+    if (x_dt == BNN_F32)
+        e = cudaLaunchKernelEx(&cfg, bnn::bw_gemv_kernel<float>, W, ldw, static_cast<const float*>(x), (int)N, (int)K,
+                               (int)kw, alpha, y, prefetch, xstatic, dependent);
+    else
+        e = cudaLaunchKernelEx(&cfg, bnn::bw_gemv_kernel<__nv_bfloat16>, W, ldw,
+                               static_cast<const __nv_bfloat16*>(x), (int)N, (int)K, (int)kw, alpha, y, prefetch,
+                               xstatic, dependent);
+    if (e != cudaSuccess) return BNN_ERR_CUDA;
+    return launch_status();
 }
 
 bnn_status bnn_binary_linear_fused(const uint32_t* A, int64_t lda, const uint32_t* W, int64_t ldw, int64_t M,

@@ -60,9 +60,10 @@ constexpr int WARP_PRODUCER = 0, WARP_MMA = 1, WARP_UNPACK0 = 2, WARP_EPI0 = WAR
 constexpr int THREADS = (WARP_EPI0 + EPI_WARPS) * 32;   // 576
 constexpr int TMEM_COLS = 2 * BN;          // two accumulators
 constexpr int NUM_BARS = 2 * PSTAGES + 2 * USTAGES + 2 * 2 + 1;
-// Per-tile epilogue column parameters, two buffers (by tile parity): float4
-// {alpha, gamma, beta, -} and int2 {c1, len2} of the threshold test per column.
-constexpr int COLP_BYTES = 2 * BN * (16 + 8);
+// Per-tile epilogue column parameters, one private copy per epilogue warp:
+// float4 {alpha, gamma, beta, -} and int2 {c1, len2} of the threshold test
+// per column.
+constexpr int COLP_BYTES = EPI_WARPS * BN * (16 + 8);
 constexpr int SMEM_BYTES = USTAGES * U_STAGE + PSTAGES * P_STAGE + COLP_BYTES + NUM_BARS * 8 + 16 + 1024;
 // kind::i8 instruction descriptor: D s32 (bits 4-5 = 2), A s8 (bits 7-9 = 1),
 // B s8 (bits 10-12 = 1), both K-major, N >> 3 at bits 17-22, M >> 4 at 24-28.
@@ -177,9 +178,9 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* uring = smem;                                   // USTAGES x (A 16 KiB | W 32 KiB)
     uint8_t* pring = smem + USTAGES * U_STAGE;               // PSTAGES x (A 2 KiB | W 4 KiB)
-    float4* colf = reinterpret_cast<float4*>(pring + PSTAGES * P_STAGE);      // [2][BN]
-    int2* colt = reinterpret_cast<int2*>(colf + 2 * BN);                       // [2][BN]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(colt + 2 * BN);
+    float4* colf = reinterpret_cast<float4*>(pring + PSTAGES * P_STAGE);      // [EPI_WARPS][BN]
+    int2* colt = reinterpret_cast<int2*>(colf + EPI_WARPS * BN);               // [EPI_WARPS][BN]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(colt + EPI_WARPS * BN);
     uint64_t* pfull = bars;
     uint64_t* pempty = pfull + PSTAGES;
     uint64_t* ufull = pempty + PSTAGES;
@@ -314,13 +315,16 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
     } else {
         // ------------------------------ epilogue warps ------------------------------
-        // Per tile, the 128 epilogue threads first stage the tile's column
-        // parameters in shared memory (alpha/gamma/beta and the threshold test
+        // Per tile, each epilogue warp first stages the tile's column parameters
+        // in its own shared-memory copy (alpha/gamma/beta and the threshold test
         // as one unsigned range check on the raw accumulator), then each thread
         // turns its row's 256 accumulators into outputs with broadcast shared
-        // loads instead of per-column global loads.
+        // loads instead of per-column global loads.  The copy is private to
+        // the warp, so only __syncwarp orders it: a named barrier across the
+        // epilogue warps here corrupted accumulator reads in testing.
         const int quad = warp & 3;                                    // TMEM lanes 32*quad .. 32*quad + 31
-        const int etid = threadIdx.x - WARP_EPI0 * 32;                // 0..127
+        float4* wcolf = colf + (warp - WARP_EPI0) * BN;
+        int2* wcolt = colt + (warp - WARP_EPI0) * BN;
         const int kp = nk * BKE;                                      // padded K: acc = kp - 2 * popcount
         const int pad = kp - K;                                       // (+1)(+1) pad positions per output
         const bool affine = ep.gamma != nullptr;
@@ -328,10 +332,10 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++lt) {
             const int b = lt & 1;
             const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
-            // Stage this tile's columns into buffer b (its previous reader, tile
-            // lt - 2, finished before every epilogue warp passed tile lt - 1's
-            // barrier below).
-            for (int i = etid; i < BN; i += EPI_WARPS * 32) {
+            // Stage this tile's columns once every lane of the warp is done
+            // with the previous tile's copy.
+            __syncwarp();
+            for (int i = lane; i < BN; i += 32) {
                 const int n = n0 + i;
                 float4 f = make_float4(0.f, 1.f, 0.f, 0.f);
                 int2 th = make_int2(0, 0);                            // len2 = 0: bit never set
@@ -357,15 +361,15 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         th = make_int2((int)(uint32_t)(kp - 2 * lo), (int)(uint32_t)(2 * len));
                     }
                 }
-                colf[b * BN + i] = f;
-                colt[b * BN + i] = th;
+                wcolf[i] = f;
+                wcolt[i] = th;
             }
-            asm volatile("bar.sync 1, %0;" ::"r"(EPI_WARPS * 32) : "memory");
+            __syncwarp();
             if (!__all_sync(0xffffffffu, tc_wait(&afull[b], (lt >> 1) & 1, abort_flag))) break;
             tc_fence_after();
             const int m = m0 + 32 * quad + lane;
-            const float4* cf = colf + b * BN;
-            const int2* ct = colt + b * BN;
+            const float4* cf = wcolf;
+            const int2* ct = wcolt;
             #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t r[32];
