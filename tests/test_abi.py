@@ -166,3 +166,15 @@ def test_binary_weight_gemv_rejects_bad_arguments():
     assert f(FAKE_ODD, 4, FAKE, 0, 8, 32, FAKE, FAKE, 0, NULL) == bnn.BNN_ERR_ALIGNMENT
     assert f(FAKE, 388, FAKE, 0, 8, 12289, FAKE, FAKE, 0, NULL) == bnn.BNN_ERR_UNSUPPORTED  # table too large
     assert f(FAKE, 4, FAKE, 0, 0, 32, FAKE, FAKE, 7, NULL) == bnn.BNN_OK                    # N = 0: nothing to do
+
+
+def test_make_epilogue_keeps_its_tensors_alive():
+    """The struct holds raw pointers; it must keep the tensors it points into
+    alive (e.g. temporaries from ``t.to(device)``)."""
+    import gc
+    import weakref
+    import torch
+    ep = bnn.make_epilogue(bnn.BNN_OUT_AFFINE_F32, alpha=torch.ones(3), gamma=torch.ones(3), beta=torch.zeros(3))
+    refs = [weakref.ref(t) for t in ep._keep if t is not None]
+    gc.collect()
+    assert len(refs) == 3 and all(r() is not None for r in refs)

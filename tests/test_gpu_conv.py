@@ -107,3 +107,28 @@ def test_conv_window_segments(n, c, h, w, cout):
              + np.abs(b.numpy().astype(np.float64))[None, :, None, None])
     assert_affine_close(out_a, y_ref, scale)
     assert_no_device_error()
+
+
+def test_tensor_conv_full_output_repeated():
+    """Races show up as a few wrong tiles in some launches only: the ResNet
+    layer runs 4 times on the tensor-core window kernel (INT32 output) and all
+    12.8M outputs are compared with the popcount kernel's."""
+    cv = workloads.conv()
+    d = dev()
+    n, c, h, w = cv.X.shape
+    Xb = bnn.empty_packed_nhwc(n, c, h, w, d)
+    bnn.bnn_pack_sign_nchw(cv.X.to(d), Xb)
+    Wp = bnn.empty_conv3x3_weights(64, c, d)
+    bnn.bnn_pack_conv3x3_weights(cv.W.to(d), Wp, None)
+    ep = bnn.make_epilogue(bnn.BNN_OUT_INT32)
+    ref = torch.empty(n, 64, h, w, dtype=torch.int32, device=d)
+    with bnn.gemm_engine(bnn.BNN_GEMM_ENGINE_POPCOUNT):
+        bnn.bnn_binary_conv3x3_fused(Xb, c, Wp, ep, ref, 1, 1)
+    out = torch.empty_like(ref)
+    with bnn.gemm_engine(bnn.BNN_GEMM_ENGINE_TENSOR):
+        for r in range(4):
+            out.fill_(0x5A5A5A5A)
+            bnn.bnn_binary_conv3x3_fused(Xb, c, Wp, ep, out, 1, 1)
+            torch.cuda.synchronize()
+            assert torch.equal(out, ref), f"launch {r}: {int((out != ref).sum())} outputs differ"
+    assert_no_device_error()

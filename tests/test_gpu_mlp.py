@@ -76,3 +76,30 @@ def test_mlp_workload_sampled_rows(engine):
         assert np.array_equal(u32(acts[l][ridx]), oracle.pack_pm1(acts_ref[l])), f"layer {l} bits"
     assert_scaled_close(logits[ridx], logits_ref)
     assert_no_device_error()
+
+
+def test_threshold_layer_engines_agree_repeated():
+    """One 4096 x 4096 x 4096 BN-threshold layer, 4 launches on the tensor
+    engine, every packed output word compared with the popcount engine's."""
+    m = workloads.mlp()
+    d = dev()
+    B, D = m.X0.shape
+    A = bnn.empty_packed(B, D, d)
+    bnn.bnn_pack_sign(m.X0.to(d), A)
+    W_p = bnn.empty_packed(D, D, d)
+    alpha = torch.empty(D, dtype=torch.float32, device=d)
+    bnn.bnn_pack_sign(m.Ws[0].to(d), W_p, alpha)
+    bn = m.bns[0]
+    thr, mode = bnn.bnn_fold_bn_threshold(alpha.cpu(), bn.gamma, bn.beta, bn.mean, bn.var, bn.eps, D)
+    ep = bnn.make_epilogue(bnn.BNN_OUT_THRESHOLD_PACK, popc_thresh=thr.to(d), thresh_mode=mode.to(d))
+    ref = bnn.empty_packed(B, D, d)
+    with bnn.gemm_engine(bnn.BNN_GEMM_ENGINE_POPCOUNT):
+        bnn.bnn_binary_linear_fused(A, W_p, D, ep, ref)
+    out = bnn.empty_packed(B, D, d)
+    with bnn.gemm_engine(bnn.BNN_GEMM_ENGINE_TENSOR):
+        for r in range(4):
+            out.fill_(0x5A5A5A5A)
+            bnn.bnn_binary_linear_fused(A, W_p, D, ep, out)
+            torch.cuda.synchronize()
+            assert torch.equal(out, ref), f"launch {r}: {int((out != ref).sum())} words differ"
+    assert_no_device_error()

@@ -263,8 +263,13 @@ def bnn_binary_weight_gemv(W: torch.Tensor, x: torch.Tensor, K: Optional[int], a
 
 def make_epilogue(mode: int, alpha=None, gamma=None, beta=None, popc_thresh=None,
                   thresh_mode=None) -> bnn_epilogue:
-    return bnn_epilogue(int(mode), _ptr(alpha), _ptr(gamma), _ptr(beta), _ptr(popc_thresh),
-                        _ptr(thresh_mode))
+    """The epilogue struct with raw device pointers.  It keeps references to
+    the tensors it points into, so that temporaries (``t.to(device)``) stay
+    alive for as long as the struct does."""
+    ep = bnn_epilogue(int(mode), _ptr(alpha), _ptr(gamma), _ptr(beta), _ptr(popc_thresh),
+                      _ptr(thresh_mode))
+    ep._keep = (alpha, gamma, beta, popc_thresh, thresh_mode)
+    return ep
 
 
 def bnn_binary_linear_fused(A: torch.Tensor, W: torch.Tensor, K: int, ep: bnn_epilogue,

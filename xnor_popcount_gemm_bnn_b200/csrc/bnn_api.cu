@@ -461,7 +461,7 @@ bnn_status bnn_binary_weight_gemv(const uint32_t* W, int64_t ldw, const void* x,
     if (!aligned(x, x_dt == BNN_F32 ? 4 : 2) || !aligned(alpha, 4) || !aligned(y, 4)) return BNN_ERR_ALIGNMENT;
     if (N == 0) return BNN_OK;
     if (!bw_gemv_smem_configured()) return BNN_ERR_CUDA;
-    const int64_t blocks = ceil_div(N, (int64_t)(bnn::bwg::RG * 32));
+    const int64_t blocks = std::min<int64_t>(ceil_div(N, (int64_t)32), sm_count());
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)blocks);
     cfg.blockDim = dim3(bnn::bwg::THREADS);

@@ -10,12 +10,14 @@
 // elements are 0).  A row's sum is then one table lookup and one add per 4
 // weights.
 //
-// Work split.  A CTA owns RG groups of 32 rows.  Warp w takes the 16-byte
-// chunks w, w + 8, w + 16, ... of each row (K split 8 ways) and lane l is row
-// l of a group, so the 32 lanes of a warp always look up the same table row
-// (16 consecutive floats): no bank conflicts.  The weight loads of the first
-// chunks are issued before the table is built, so they overlap it.  The 8
-// partial sums of a row meet in shared memory.
+// Work split.  One CTA per SM walks groups of 32 rows, and the table is
+// built once per CTA.  Warp w takes the 16-byte chunks w, w + 16, w + 32, ...
+// of each row (K split 16 ways) and lane l is row l of the group, so the 32
+// lanes of a warp always look up the same table row (16 consecutive floats):
+// no bank conflicts.  The first weight batch is loaded before the table is
+// built, and the next group's batch while the current one is summed.  The 16
+// partial sums of a row meet in shared memory.  A CTA holds 66 KB of shared
+// memory at K = 4096, so two consecutive launches fit on one SM.
 //
 // Launched with programmatic dependent launch, like the XNOR GEMV: with static
 // weights the W loads precede the wait for the previous grid, with static
@@ -27,12 +29,11 @@
 
 namespace bnn {
 namespace bwg {
-constexpr int WARPS = 8;                  // K slices
+constexpr int WARPS = 16;                 // K slices
 constexpr int THREADS = WARPS * 32;
-constexpr int RG = 2;                     // row groups of 32 per CTA
-constexpr int NB = 4;                     // chunks per lane per batch (loads in flight)
+constexpr int NB = 2;                     // chunks per lane per batch (loads in flight)
 constexpr int MAX_KW = 384;               // table of MAX_KW * 8 groups x 64 B = 192 KiB
-__host__ __device__ constexpr int smem_bytes(int kw) { return kw * 8 * 64 + RG * WARPS * 32 * 4; }
+__host__ __device__ constexpr int smem_bytes(int kw) { return 64 + kw * 8 * 64 + WARPS * 32 * 4; }
 }  // namespace bwg
 
 template <typename XT>
@@ -41,22 +42,27 @@ bw_gemv_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restrict
                const float* __restrict__ alpha, float* __restrict__ y, int prefetch, int xstatic, int dependent) {
     using namespace bwg;
     extern __shared__ __align__(16) float bw_smem[];
-    float* table = bw_smem;                                   // [kw * 8][16]
-    float* part = bw_smem + kw * 8 * 16;                      // [RG][WARPS][32]
+    // [kw * 8][16] with 64-byte aligned rows: the entry of group g, nibble n is
+    // at byte offset (g * 64) | (n * 4).
+    float* table = bw_smem + (((64u - (smem_u32(bw_smem) & 63u)) & 63u) >> 2);
+    const char* tbytes = reinterpret_cast<const char*>(table);
+    float* part = table + kw * 8 * 16;                        // [WARPS][32]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nch = kw / 4;                                   // 16-byte chunks per row
-    const int row0 = blockIdx.x * (RG * 32);
+    const int groups = (N + 31) / 32;                         // row groups of 32
     grid_dependents_launch();
 
-    // First batch of weight chunks for every row group (K = 4096: all of them).
-    uint4 v[RG][NB];
-    auto load_batch = [&](int rg, int cb) {
-        const int row = row0 + rg * 32 + lane;
+    // A CTA walks the row groups blockIdx.x, + gridDim.x, ...; the table is
+    // built once per CTA and the first weight batch of the next row group is
+    // loaded while the current one is summed.
+    uint4 v[NB], vn[NB];
+    auto load_batch = [&](uint4 (&dst)[NB], int rgi, int cb) {
+        const int row = rgi * 32 + lane;
         #pragma unroll
         for (int i = 0; i < NB; ++i) {
             const int c = cb + WARPS * i;
-            v[rg][i] = (row < N && c < nch) ? ldg_stream_v4(W + (int64_t)row * ldw + 4 * c)
-                                            : make_uint4(0u, 0u, 0u, 0u);
+            dst[i] = (rgi < groups && row < N && c < nch) ? ldg_stream_v4(W + (int64_t)row * ldw + 4 * c)
+                                                          : make_uint4(0u, 0u, 0u, 0u);
         }
     };
     auto build_table = [&]() {
@@ -80,48 +86,50 @@ bw_gemv_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restrict
         }
     };
     const bool late_wait = prefetch && xstatic;
-    if (prefetch) {
-        #pragma unroll
-        for (int rg = 0; rg < RG; ++rg) load_batch(rg, warp);
-    }
+    if (prefetch) load_batch(v, blockIdx.x, warp);
     if (xstatic) build_table();
     if (dependent == 1 && !late_wait) grid_dependency_wait();
-    if (!prefetch) {
-        #pragma unroll
-        for (int rg = 0; rg < RG; ++rg) load_batch(rg, warp);
-    }
+    if (!prefetch) load_batch(v, blockIdx.x, warp);
     if (!xstatic) build_table();
     __syncthreads();
 
-    #pragma unroll
-    for (int rg = 0; rg < RG; ++rg) {
+    bool first = true;
+    for (int rgi = blockIdx.x; rgi < groups; rgi += gridDim.x) {
+        load_batch(vn, rgi + gridDim.x, warp);                // next row group, first batch
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         for (int cb = warp; cb < nch; cb += WARPS * NB) {
-            if (cb != warp) load_batch(rg, cb);               // later batches (K > 4096)
+            if (cb != warp) load_batch(v, rgi, cb);           // later batches (K > 4096)
             #pragma unroll
             for (int i = 0; i < NB; ++i) {
                 const int c = cb + WARPS * i;
                 if (c >= nch) break;
-                const uint32_t wq[4] = {v[rg][i].x, v[rg][i].y, v[rg][i].z, v[rg][i].w};
+                const uint32_t wq[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
                 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const float* tg = table + (size_t)((4 * c + q) * 8) * 16;   // 8 nibble groups of this word
+                    const uint32_t grow = (uint32_t)((4 * c + q) * 8) * 64u;   // byte offset of the word's groups
                     #pragma unroll
-                    for (int j = 0; j < 8; ++j) acc[j & 3] += tg[j * 16 + ((wq[q] >> (4 * j)) & 15u)];
+                    for (int j = 0; j < 8; ++j) {
+                        // nibble j moved to bits 2..5 (byte offset nibble * 4)
+                        const uint32_t nib4 = j == 0 ? (wq[q] << 2) : (wq[q] >> (4 * j - 2));
+                        acc[j & 3] += *reinterpret_cast<const float*>(tbytes + ((grow + 64u * j) | (nib4 & 0x3Cu)));
+                    }
                 }
             }
         }
-        part[(rg * WARPS + warp) * 32 + lane] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-    }
-    __syncthreads();
-    if (dependent == 1 && late_wait) grid_dependency_wait();
-    if (threadIdx.x < RG * 32) {
-        const int rg = threadIdx.x >> 5;
-        const int row = row0 + threadIdx.x;
-        float s = 0.0f;
+        part[warp * 32 + lane] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            const int row = rgi * 32 + lane;
+            float s = 0.0f;
+            #pragma unroll
+            for (int w = 0; w < WARPS; ++w) s += part[w * 32 + lane];
+            if (first && dependent == 1 && late_wait) grid_dependency_wait();
+            if (row < N) y[row] = alpha[row] * s;
+        }
+        __syncthreads();                                      // part[] is rewritten next round
+        first = false;
         #pragma unroll
-        for (int w = 0; w < WARPS; ++w) s += part[(rg * WARPS + w) * 32 + lane];
-        if (row < N) y[row] = alpha[row] * s;
+        for (int i = 0; i < NB; ++i) v[i] = vn[i];
     }
     if (dependent == 2) grid_dependency_wait();
 }
