@@ -15,6 +15,11 @@ real-valued epilogues evaluated in float64 here with numpy:
   bit 1 is -1, pad bits encode +1).
 * alpha and the scaled product -- "Extreme Quantization ...", Binary Neural
   Networks section, eq. (1): y = alpha * (w_b^T x), alpha = (1/n) sum |w_i|.
+* ternary weights -- "Extreme Quantization ...", eq. (7) (threshold Delta)
+  and eq. (9) (BitNet b1.58: RoundClip(W / gamma, -1, 1), gamma = mean |W|
+  over the matrix); "First Principles ...", the op-per-element table
+  (ternary: add / skip / sub), with int8 activations (the BitNet section:
+  activations quantised to INT8).
 * BatchNorm before re-binarisation -- "Binary Neural Network (BNN)" glossary
   page, the BatchNorm paragraph (BN stabilises the inputs to each binarised
   layer; per-filter alpha multiplies the binary product).  The pages give no
@@ -25,7 +30,9 @@ real-valued epilogues evaluated in float64 here with numpy:
 Readings of the pages made here (all listed with reasons in the design notes):
 sign(-0.0) = +1, sign(NaN) = +1, bit j of word w is element 32*w + j, rows
 padded to a multiple of 4 words, alpha over the true K from the real weights,
-convolution padding value +1, BN decisions taken with alpha rounded to fp32
+convolution padding value +1, RoundClip rounding halves to even, ternary
+codes t + 1 packed 2 bits per weight (16 per word, least significant first,
+pad code 1), BN decisions taken with alpha rounded to fp32
 (the precision the product stores alpha in).
 
 Parity pins for every function live in ``tests/test_oracle_pins.py``.
@@ -165,6 +172,100 @@ def binary_weight_gemv(w_real, x_real) -> tuple[np.ndarray, np.ndarray]:
     wb = sign_pm1(w_real)
     a = alpha(w_real)
     return a, scaled(binary_weight_product(wb, _f32(x_real)), a)
+
+
+
+# ---------------------------------------------------------------------------
+# ternary weights (BitNet b1.58) times int8 activations
+# ---------------------------------------------------------------------------
+
+def ternary_ld_words(K: int) -> int:
+    """Words per packed ternary row: 2 bits per weight, 16 weights per uint32
+    word, rounded up to a multiple of 4 words (whole 16-byte units, as the
+    binary rows)."""
+    K = int(K)
+    if K < 1:
+        return -1
+    words = -(-K // 16)
+    return -(-words // 4) * 4
+
+
+def ternary_gamma(w) -> float:
+    """eq. (9) of "Extreme Quantization: Binary, Ternary & 1-bit LLMs", BitNet
+    b1.58: gamma = ||W||_1 / (n m), the mean absolute value over every entry
+    of the matrix (one scale per tensor), in float64."""
+    wd = _f32(w).astype(np.float64)
+    return float(np.abs(wd).sum() / wd.size)
+
+
+def round_clip(v, lo: float, hi: float) -> np.ndarray:
+    """RoundClip(v, lo, hi) of eq. (9): round to the nearest integer, then
+    clip to [lo, hi].  The pages do not say how halves round; this takes
+    round half to even (numpy.rint), so +-0.5 go to 0."""
+    return np.clip(np.rint(np.asarray(v, dtype=np.float64)), lo, hi)
+
+
+def ternary_quantize(w, delta: float | None = None) -> tuple[np.ndarray, float]:
+    """Ternary weights in {-1, 0, +1} (int8, same shape as w) and gamma.
+
+    delta None -- eq. (9), BitNet b1.58: W_t = RoundClip(W / gamma, -1, 1) with
+    gamma = ternary_gamma(W), the division and rounding in float64.  An all-
+    zero W has gamma = 0; its weights are all 0.
+    delta given -- eq. (7), ternary quantisation with threshold Delta:
+    +1 where w > Delta, 0 where |w| <= Delta, -1 where w < -Delta.
+    gamma is returned in both cases (the scale of eq. (9))."""
+    wd = _f32(w).astype(np.float64)
+    g = ternary_gamma(w)
+    if delta is None:
+        if g == 0.0:
+            return np.zeros(wd.shape, dtype=np.int8), g
+        return round_clip(wd / g, -1, 1).astype(np.int8), g
+    d = float(delta)
+    t = np.where(wd > d, 1, np.where(wd < -d, -1, 0))
+    return t.astype(np.int8), g
+
+
+def pack_ternary(t: np.ndarray, ld: int | None = None) -> np.ndarray:
+    """Pack a [rows, K] matrix of ternary weights into uint32 [rows, ld].
+    Weight k of a row is the 2-bit code t + 1 (0 for -1, 1 for 0, 2 for +1)
+    at bits 2k, 2k+1 of the row's bit string, least significant bit first:
+    bits 2(k mod 16) of word k // 16.  Positions past K hold code 1 (weight
+    0).  The pages give the density (about 0.2 bytes per weight, log2(3) =
+    1.58 bits) but no layout; this is the plainest addressable one."""
+    t = np.ascontiguousarray(t, dtype=np.int8)
+    if t.ndim == 1:
+        t = t[None, :]
+    rows, K = t.shape
+    ld = ternary_ld_words(K) if ld is None else int(ld)
+    codes = np.ones((rows, ld * 16), dtype=np.uint64)
+    codes[:, :K] = (t.astype(np.int64) + 1).astype(np.uint64)
+    shifts = (2 * np.arange(16, dtype=np.uint64))[None, None, :]
+    words = (codes.reshape(rows, ld, 16) << shifts).sum(axis=2)
+    return words.astype(np.uint32)
+
+
+def ternary_product(t: np.ndarray, x) -> np.ndarray:
+    """int64 [N]: sum_k t_nk * x_k for ternary t [N, K] and integer x [K], by
+    the rule of the op-per-element table in "First Principles: Why Binary Ops
+    Can Be Exponentially Faster" (ternary: add / skip / sub): x_k is added
+    where the weight is +1, skipped where it is 0, subtracted where it is -1."""
+    t = np.asarray(t, dtype=np.int8)
+    if t.ndim == 1:
+        t = t[None, :]
+    xi = np.asarray(x, dtype=np.int64)
+    terms = np.where(t > 0, xi[None, :], np.where(t < 0, -xi[None, :], 0))
+    return terms.sum(axis=1)
+
+
+def ternary_gemv_i8(t: np.ndarray, x_q, w_scale: float = 1.0, x_scale: float = 1.0):
+    """Ternary weights times an int8 activation vector ("Extreme Quantization
+    ...", BitNet: activations quantised to INT8; BitNet b1.58: ternary
+    weights).  Returns (acc int64 [N], y float64 [N]) with
+    y = w_scale * x_scale * acc, the dequantised product (w_scale is gamma of
+    eq. (9); x_scale the activation's quantisation step, which the pages
+    leave to the caller)."""
+    acc = ternary_product(t, x_q)
+    return acc, float(w_scale) * float(x_scale) * acc.astype(np.float64)
 
 
 def conv2d_pm1(x: np.ndarray, f: np.ndarray, stride: int = 1, pad: int = 1) -> np.ndarray:

@@ -137,7 +137,80 @@ def _bw_abs_x(w, x):                   # adds |x| instead of x
     return np.where(w > 0, xd[None, :], -xd[None, :]).sum(axis=1)
 
 
+
+def _tern_gamma_noabs(w, delta=None):  # gamma from the mean of w, not of |w|
+    wd = oracle._f32(w).astype(np.float64)
+    g = abs(float(wd.mean())) or 1.0
+    return oracle.round_clip(wd / g, -1, 1).astype(np.int8), g
+
+
+def _tern_round_half_away(w, delta=None):   # halves round away from zero
+    wd = oracle._f32(w).astype(np.float64)
+    g = oracle.ternary_gamma(w)
+    if g == 0.0:
+        return np.zeros(wd.shape, np.int8), g
+    q = wd / g
+    return np.clip(np.sign(q) * np.floor(np.abs(q) + 0.5), -1, 1).astype(np.int8), g
+
+
+def _tern_no_clip(w, delta=None):      # RoundClip without the clip
+    wd = oracle._f32(w).astype(np.float64)
+    g = oracle.ternary_gamma(w)
+    if g == 0.0:
+        return np.zeros(wd.shape, np.int8), g
+    return np.rint(wd / g).astype(np.int8), g
+
+
+def _tern_per_row_gamma(w, delta=None):     # one gamma per row instead of per matrix
+    wd = np.atleast_2d(oracle._f32(w).astype(np.float64))
+    g = np.abs(wd).mean(axis=1, keepdims=True)
+    g[g == 0] = 1.0
+    return oracle.round_clip(wd / g, -1, 1).astype(np.int8).reshape(np.shape(w)), float(g.mean())
+
+
+def _tern_pack_codes_t(t, ld=None):    # stores t itself (two's complement bits), not t + 1
+    t = np.atleast_2d(np.asarray(t, np.int8))
+    rows, K = t.shape
+    ld = oracle.ternary_ld_words(K) if ld is None else ld
+    out = np.zeros((rows, ld), np.uint32)
+    for r in range(rows):
+        for k in range(K):
+            out[r, k // 16] |= np.uint32((int(t[r, k]) & 3) << (2 * (k % 16)))
+    return out
+
+
+def _tern_pack_msb(t, ld=None):        # codes placed from the top of the word down
+    t = np.atleast_2d(np.asarray(t, np.int8))
+    rows, K = t.shape
+    ld = oracle.ternary_ld_words(K) if ld is None else ld
+    out = np.full((rows, ld), 0x55555555, np.uint32)
+    for r in range(rows):
+        for k in range(K):
+            sh = 30 - 2 * (k % 16)
+            w = int(out[r, k // 16]) & ~(3 << sh)
+            out[r, k // 16] = np.uint32(w | ((int(t[r, k]) + 1) << sh))
+    return out
+
+
+def _tern_minus_as_skip(t, x):         # -1 weights skipped instead of subtracted
+    t = np.atleast_2d(np.asarray(t, np.int8))
+    xi = np.asarray(x, np.int64)
+    return np.where(t > 0, xi[None, :], 0).sum(axis=1)
+
+
+def _tern_sign_swapped(t, x):          # add where -1, subtract where +1
+    return -oracle.ternary_product(t, x)
+
+
 MUTANTS = {
+    "ternary_gamma_without_abs": dict(ternary_quantize=_tern_gamma_noabs),
+    "ternary_round_half_away": dict(ternary_quantize=_tern_round_half_away),
+    "ternary_no_clip": dict(ternary_quantize=_tern_no_clip),
+    "ternary_per_row_gamma": dict(ternary_quantize=_tern_per_row_gamma),
+    "ternary_pack_codes_t": dict(pack_ternary=_tern_pack_codes_t),
+    "ternary_pack_msb_first": dict(pack_ternary=_tern_pack_msb),
+    "ternary_minus_as_skip": dict(ternary_product=_tern_minus_as_skip),
+    "ternary_sign_swapped": dict(ternary_product=_tern_sign_swapped),
     "bw_sign_swapped": dict(binary_weight_product=_bw_sign_swapped),
     "bw_dropped_term": dict(binary_weight_product=_bw_drop_last),
     "bw_abs_activation": dict(binary_weight_product=_bw_abs_x),

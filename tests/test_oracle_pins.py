@@ -308,6 +308,93 @@ def check_binary_weight_product(o):
     assert np.array_equal(o.binary_weight_product(w, xb).astype(np.int64), o.gemv_pm1(w, xb).astype(np.int64))
 
 
+
+def check_ternary_examples(o, golden):
+    """Hand-computed ternary quantisation, packing and add/skip/sub sums
+    ('Extreme Quantization ...', eq. (7) and eq. (9); 'First Principles ...',
+    the op-per-element and memory tables)."""
+    g = json.load(open(os.path.join(golden, "ternary_examples.json")))
+    for c in g["quantize_eq9"]:
+        t, _ = o.ternary_quantize(np.array(c["w"], np.float32))
+        assert t.tolist() == c["t"], (c["w"], t)
+    for c in g["quantize_eq7"]:
+        t, _ = o.ternary_quantize(np.array(c["w"], np.float32), c["delta"])
+        assert t.tolist() == c["t"], (c["w"], t)
+    for c in g["pack"]:
+        K = c["K"]
+        t = np.zeros(K, np.int8)
+        if "t" in c:
+            t[:] = c["t"]
+        else:
+            for k, v in c["t_nonzero"].items():
+                t[int(k)] = v
+        got = o.pack_ternary(t)
+        assert [int(v) for v in got[0]] == c["words"], (K, [hex(int(v)) for v in got[0]])
+    for c in g["product"]:
+        got = o.ternary_product(np.array([c["t"]], np.int8), np.array(c["x"]))
+        assert int(got[0]) == c["sum"], (c, got)
+
+
+def check_ternary_quantizer(o):
+    """eq. (9) against closed forms, a library mean and eq. (7):
+    * gamma is the entrywise mean |w| of the whole matrix (torch float64 mean);
+    * weights of equal magnitude quantise to their signs (w / gamma = +-1);
+    * eq. (9) equals eq. (7) with Delta = gamma / 2 on random matrices (the
+      threshold form and the round-and-clip form agree away from exact ties);
+    * scaling W by a power of two changes nothing (gamma scales with it);
+    * RoundClip closed forms: halves to even, clipping at +-1;
+    * packed row length: the fewest multiples of 4 words holding 2 K bits."""
+    rng = np.random.default_rng(21)
+    w = (rng.standard_normal((7, 333)) * np.array([1, 0.01, 3, 1, 1, 0.5, 2])[:, None]).astype(np.float32)
+    gl = torch.from_numpy(w).double().abs().mean().item()
+    assert abs(o.ternary_gamma(w) - gl) <= 1e-15 * gl
+    t9, g9 = o.ternary_quantize(w)
+    assert abs(g9 - gl) <= 1e-15 * gl
+    t7, _ = o.ternary_quantize(w, delta=g9 / 2)
+    assert np.array_equal(t9, t7)
+    assert set(np.unique(t9).tolist()) == {-1, 0, 1}
+    assert np.all(t9[np.abs(w) > 1.5 * g9] == np.sign(w[np.abs(w) > 1.5 * g9]))     # clipped
+    for e in (-3, 5):
+        assert np.array_equal(o.ternary_quantize(w * np.float32(2.0 ** e))[0], t9)
+    c = np.float32(0.3)
+    ws = np.where(rng.random((5, 50)) < 0.5, -c, c).astype(np.float32)
+    ts, gs = o.ternary_quantize(ws)
+    assert abs(gs - float(c)) <= 1e-15 and np.array_equal(ts, np.sign(ws).astype(np.int8))
+    v = np.array([0.5, -0.5, 1.5, -1.5, 2.5, -2.5, 0.49, -0.51, 0.0, 7.0])
+    assert o.round_clip(v, -1, 1).tolist() == [0, 0, 1, -1, 1, -1, 0, -1, 0, 1]
+    for K in range(1, 300):
+        words = 4
+        while words * 32 < 2 * K:
+            words += 4
+        assert o.ternary_ld_words(K) == words, K
+    assert o.ternary_ld_words(4096) * 4 / 4096 == 0.25    # 2 bits per weight (pages: ~0.2 B at 1.58 bits)
+
+
+def check_ternary_product(o):
+    """The add/skip/sub sum against brute force over every ternary vector for
+    K <= 4 (as a sum of products), torch int64 matmul, the binary product
+    when no weight is 0, and the dequantised output's scale."""
+    rng = np.random.default_rng(23)
+    for K in range(1, 5):
+        T = np.array(list(itertools.product([-1, 0, 1], repeat=K)), dtype=np.int8)
+        x = rng.integers(-128, 128, K)
+        got = o.ternary_product(T, x)
+        for r in range(len(T)):
+            ref = 0
+            for k in range(K):
+                ref += int(T[r, k]) * int(x[k])
+            assert int(got[r]) == ref, (K, T[r], x)
+    t = rng.integers(-1, 2, (40, 1000)).astype(np.int8)
+    x = rng.integers(-128, 128, 1000)
+    ref = (torch.from_numpy(t).long() @ torch.from_numpy(x).long()).numpy()
+    assert np.array_equal(o.ternary_product(t, x), ref)
+    tb = np.where(rng.random((9, 300)) < 0.5, -1, 1).astype(np.int8)
+    xb = np.where(rng.random(300) < 0.5, -1, 1).astype(np.int8)
+    assert np.array_equal(o.ternary_product(tb, xb), o.gemv_pm1(tb, xb).astype(np.int64))
+    acc, y = o.ternary_gemv_i8(t, x, 0.25, 8.0)
+    assert np.array_equal(acc, ref) and np.array_equal(y, 2.0 * ref.astype(np.float64))
+
+
 ALL_CHECKS = [
     ("identity_bruteforce", lambda o, g: check_identity_bruteforce(o)),
     ("elementwise_xnor_form", lambda o, g: check_elementwise_xnor_form(o)),
@@ -324,6 +411,9 @@ ALL_CHECKS = [
     ("bn", lambda o, g: check_bn(o)),
     ("mlp_library", lambda o, g: check_mlp_library(o)),
     ("binary_weight_product", lambda o, g: check_binary_weight_product(o)),
+    ("ternary_examples", check_ternary_examples),
+    ("ternary_quantizer", lambda o, g: check_ternary_quantizer(o)),
+    ("ternary_product", lambda o, g: check_ternary_product(o)),
 ]
 
 
