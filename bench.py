@@ -114,6 +114,8 @@ KERNEL_SOURCES = {
     "pack_sign_rows_kernel": ("pack.cuh", "common.cuh"),
     "pack_sign_nchw_kernel": ("pack.cuh", "common.cuh"),
     "bw_gemv_kernel": ("bwgemv.cuh", "common.cuh"),
+    "ternary_gemv_i8_staged_kernel": ("ternary.cuh", "common.cuh"),
+    "pack_ternary_kernel": ("ternary.cuh", "common.cuh"),
 }
 
 
@@ -449,7 +451,7 @@ def e2e_gemv(torch, bnn, g, Ws, alpha, dev, steps, sync, max_over_ranks, ws):
 # the other rows
 # ---------------------------------------------------------------------------
 
-ROW_NAMES = ("pack_sign_weights", "square_gemm", "conv3x3", "mlp4", "bw_gemv")
+ROW_NAMES = ("pack_sign_weights", "square_gemm", "conv3x3", "mlp4", "bw_gemv", "ternary")
 
 
 def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws, only=None):
@@ -474,6 +476,8 @@ def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws, o
         _row_mlp(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk)
     if "bw_gemv" in want:
         _row_bw_gemv(torch, bnn, workloads, dev, pk, rows, timed, ws)
+    if "ternary" in want:
+        _row_ternary(torch, bnn, workloads, dev, pk, rows, timed, steps, ws)
     if bnn.bnn_device_error() != 0:
         raise RuntimeError("a kernel reported a device-side timeout")
     return rows
@@ -643,6 +647,55 @@ def _row_bw_gemv(torch, bnn, workloads, dev, pk, rows, timed, ws):
         "dependent_chain": {"value": round(ws * ach_dep, 1), "unit": "GB/s", "ms_per_step": ms_dep / steps,
                             "frac": round(ach_dep / pk["hbm_gbs"], 4)}}
     del Ws, ys, W_p, x, g
+    torch.cuda.empty_cache()
+
+
+
+def _row_ternary(torch, bnn, workloads, dev, pk, rows, timed, steps, ws):
+    # --- next row: ternary (b1.58) weights: eq. (9) quantise + pack, then the int8 GEMV ---
+    g = workloads.ternary()
+    Wd = g.W.to(dev)
+    codes = bnn.empty_ternary(g.N, g.K, dev)
+    gam = torch.empty(1, dtype=torch.float32, device=dev)
+    wsp = torch.empty(bnn.bnn_ternary_workspace_bytes(g.N) // 8, dtype=torch.float64, device=dev)
+    ms_p = timed(lambda i: bnn.bnn_ternary_pack(Wd, codes, gamma_out=gam, workspace=wsp))
+    q_bytes = codes.numel() * 4
+    pb = 2 * g.N * g.K * 4 + q_bytes          # W read twice (gamma first, then the codes) + codes
+    ach_p = pb * steps / (ms_p * 1e-3) / 1e9
+    del Wd
+    torch.cuda.empty_cache()
+    copies = max(2, math.ceil(2 * L2_BYTES / q_bytes) + 1)
+    copies = (copies + 7) // 8 * 8
+    Qs = [codes] + [codes.clone() for _ in range(copies - 1)]
+    ys = [torch.empty(g.N, dtype=torch.float32, device=dev) for _ in range(copies)]
+    x = g.x.to(dev)
+    xsc = torch.full((1,), 1.0 / 64, dtype=torch.float32, device=dev)
+    n = 48 * copies
+    all_flags = bnn.BNN_GEMV_WEIGHTS_STATIC | bnn.BNN_GEMV_INPUTS_STATIC | bnn.BNN_GEMV_OUTPUT_FREE
+    ms = timed(lambda i: bnn.bnn_ternary_gemv_i8(Qs[i % copies], x, g.K, y_f32=ys[i % copies], w_scale=gam,
+                                                 x_scale=xsc, flags=all_flags), n=n, period=copies)
+    ms_dep = timed(lambda i: bnn.bnn_ternary_gemv_i8(Qs[i % copies], x, g.K, y_f32=ys[0], w_scale=gam, x_scale=xsc,
+                                                     flags=bnn.BNN_GEMV_WEIGHTS_STATIC), n=n, period=copies)
+    b = q_bytes + g.K + 4 * g.N + 8           # codes + int8 x + fp32 y + two scales
+    ach = b * n / (ms * 1e-3) / 1e9
+    ach_dep = b * n / (ms_dep * 1e-3) / 1e9
+    rows["ternary_gemv"] = {
+        "workload": f"ternary (b1.58) weights x int8 activations: codes [11008, 4096] at 2 bits, x int8 [4096], "
+                    f"fp32 y = gamma * x_scale * acc; independent steps over {copies} rotating code copies",
+        "value": round(ws * ach, 1), "unit": "GB/s", "ms_per_step": ms / n,
+        "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"],
+                     "frac": round(ach / pk["hbm_gbs"], 4), "algorithmic_bytes": b,
+                     "traffic": recorded_traffic("ternary_gemv_i8_staged_kernel")},
+        "dependent_chain": {"value": round(ws * ach_dep, 1), "unit": "GB/s", "ms_per_step": ms_dep / n,
+                            "frac": round(ach_dep / pk["hbm_gbs"], 4)}}
+    rows["ternary_pack"] = {
+        "workload": "fp32 W [11008, 4096] -> eq. (9) gamma (fp64 row sums, fixed-order total) + 2-bit codes; "
+                    "3 launches",
+        "value": round(ws * ach_p, 1), "unit": "GB/s", "ms_per_step": ms_p / steps,
+        "roofline": {"bound": "hbm", "achieved": round(ach_p, 1), "peak": pk["hbm_gbs"],
+                     "frac": round(ach_p / pk["hbm_gbs"], 4), "algorithmic_bytes": pb,
+                     "traffic": recorded_traffic("pack_ternary_kernel")}}
+    del Qs, ys, codes, x, g, wsp
     torch.cuda.empty_cache()
 
 

@@ -30,7 +30,8 @@
  * CONVENTIONS.
  *  - Device pointers are CUDA device (or managed) memory on the current
  *    device, owned by the caller; the library keeps no pointer after a call
- *    returns and allocates no device memory.  Host pointers are named so.
+ *    returns and allocates no device memory (a call that needs scratch
+ *    space takes a caller-owned workspace).  Host pointers are named so.
  *  - Every device call is asynchronous on `stream` (NULL = legacy default
  *    stream).  It returns after the launch; results are visible to later
  *    work on the same stream.
@@ -278,12 +279,82 @@ bnn_status bnn_xnor_gemv_ex(const uint32_t* W, int64_t ldw, const void* x, bnn_d
  *   flags    as for bnn_xnor_gemv_ex (BNN_GEMV_WEIGHTS_STATIC,
  *            BNN_GEMV_INPUTS_STATIC, BNN_GEMV_OUTPUT_FREE).
  * Accumulation is fp32: a 16-entry table of +-x0 +-x1 +-x2 +-x3 per group
- * of 4 elements, then one lookup and one add per 4 weights, 32 adds per
- * partial sum at K = 4096, and 8 partial sums per row.
+ * of 4 elements, then one lookup and one add per 4 weights, 4 accumulators
+ * per lane, and 16 partial sums per row.
  *   Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (K too large), CUDA. */
 bnn_status bnn_binary_weight_gemv(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt,
                                   int64_t N, int64_t K, const float* alpha, float* y,
                                   uint32_t flags, bnn_stream_t stream);
+
+/* TERNARY LAYOUT (bnn_ternary_pack, bnn_ternary_gemv_i8).  A ternary weight
+ * t in {-1, 0, +1} is stored as the 2-bit code t + 1 (0 = -1, 1 = 0, 2 = +1;
+ * code 3 is not a weight and must not occur).  Weight k of a row sits at bits
+ * 2(k mod 16), 2(k mod 16)+1 of uint32 word k / 16 (least significant first).
+ * A row holds bnn_ternary_ld_words(K) = ceil(K/16) rounded up to a multiple of
+ * 4 words; positions past K hold code 1.  Row r starts at word r * ldq, ldq a
+ * multiple of 4 and >= bnn_ternary_ld_words(K).  2 bits per weight: the pages
+ * give ~1.58 bits (log2 3) as the information content and ~0.2 bytes per
+ * weight for packed ternary; the 2-bit code is the densest layout whose
+ * weights can be addressed with shifts and masks. */
+
+/* Words in one ternary row of K weights; -1 for K < 1. */
+int64_t bnn_ternary_ld_words(int64_t K);
+
+/* Bytes of device workspace bnn_ternary_pack needs for `rows` rows when it
+ * computes gamma: 8 * (rows + 1).  -1 for rows < 0. */
+int64_t bnn_ternary_workspace_bytes(int64_t rows);
+
+/* bnn_ternary_pack -- quantise a real matrix to ternary weights and pack them.
+ *   Passage: "Extreme Quantization: Binary, Ternary & 1-bit LLMs",
+ *   Ternary Quantization, eq. (7), and BitNet b1.58, eq. (9).
+ *   delta < 0  -- eq. (9): W_t = RoundClip(W / gamma, -1, 1),
+ *                 gamma = sum |w| / (rows * K) over the whole matrix.
+ *                 Halves round to even, so the weight is +-1 exactly where
+ *                 |w| > gamma / 2 and 0 elsewhere; that comparison is made in
+ *                 fp64 with gamma summed in fp64 (per row, then the rows in a
+ *                 fixed order: the same codes on every run).  All-zero W gives
+ *                 gamma = 0 and all weights 0.
+ *   delta >= 0 -- eq. (7) with Delta = delta: +1 where w > delta, -1 where
+ *                 w < -delta, 0 otherwise (compared in fp64).
+ *   NaN weights quantise to 0.
+ *   w         device, [rows, K] row-major, dtype dt, row stride ld_w >= K.
+ *   codes     device, uint32 [rows, ldq] (TERNARY LAYOUT, 16-byte aligned);
+ *             words [0, bnn_ternary_ld_words(K)) of each row are written.
+ *   gamma_out device fp32 [1] or NULL: gamma rounded once to fp32 (the scale
+ *             of eq. (9): W is approximated by gamma * W_t).
+ *   workspace device, >= bnn_ternary_workspace_bytes(rows) bytes, 8-byte
+ *             aligned, owned by the caller; required when delta < 0 or
+ *             gamma_out is given, else may be NULL.  Its contents on entry do
+ *             not matter; it must not be used by other work until the call's
+ *             kernels are done (stream order).
+ *   Launches up to three kernels (row sums of |w|, gamma, pack).
+ *   Errors: INVALID_ARG (null, sizes, NaN delta, workspace missing or too
+ *   small), ALIGNMENT. */
+bnn_status bnn_ternary_pack(const void* w, bnn_dtype dt, int64_t rows, int64_t K, int64_t ld_w,
+                            double delta, uint32_t* codes, int64_t ldq, float* gamma_out,
+                            void* workspace, int64_t workspace_bytes, bnn_stream_t stream);
+
+/* bnn_ternary_gemv_i8 -- ternary weights times an int8 activation vector:
+ *   acc[n]   = sum_k t_nk * x_k                    (exact, int32)
+ *   y_f32[n] = fp32( fp32(w_scale * x_scale) * fp32(acc[n]) )
+ * ("Extreme Quantization ...", BitNet: INT8 activations; BitNet b1.58:
+ * ternary weights; "First Principles ...", op-per-element table: add / skip /
+ * sub).  The pages do not define the activation quantiser: x arrives
+ * quantised, with its scale.
+ *   codes    device, [N, ldq] words (TERNARY LAYOUT), 16-byte aligned.
+ *   x        device int8 [K] (any alignment; 16-byte aligned is faster).
+ *   w_scale, x_scale  device fp32 [1] each, or NULL for 1.0 (read only when
+ *            y_f32 is given).  w_scale is typically gamma from
+ *            bnn_ternary_pack.
+ *   y_i32    device int32 [N] or NULL; y_f32 device fp32 [N] or NULL; at
+ *            least one.  fp32(acc) is exact for K <= 65536.
+ *   flags    as for bnn_xnor_gemv_ex (the x vector and both scales are the
+ *            inputs of BNN_GEMV_INPUTS_STATIC).
+ *   K <= 98304 (x is staged in shared memory).
+ *   Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (K too large), CUDA. */
+bnn_status bnn_ternary_gemv_i8(const uint32_t* codes, int64_t ldq, const int8_t* x, int64_t N, int64_t K,
+                               const float* w_scale, const float* x_scale, int32_t* y_i32, float* y_f32,
+                               uint32_t flags, bnn_stream_t stream);
 
 /* bnn_binary_linear_fused -- packed binary GEMM with one fused epilogue.
  *   Passage: eq. (6) (product), eq. (1) (alpha), the glossary's BatchNorm

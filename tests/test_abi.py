@@ -178,3 +178,45 @@ def test_make_epilogue_keeps_its_tensors_alive():
     refs = [weakref.ref(t) for t in ep._keep if t is not None]
     gc.collect()
     assert len(refs) == 3 and all(r() is not None for r in refs)
+
+
+def test_ternary_layout_sizes():
+    """Ternary row length and workspace size match the layout reading (2 bits
+    per weight, rows of whole 16-byte units) as the oracle states it."""
+    for K in (1, 15, 16, 17, 64, 65, 1000, 4096, 11008):
+        assert bnn.bnn_ternary_ld_words(K) == oracle.ternary_ld_words(K)
+    assert bnn.bnn_ternary_ld_words(0) == -1
+    assert bnn.bnn_ternary_workspace_bytes(11008) == 8 * 11009
+    assert bnn.bnn_ternary_workspace_bytes(-1) == -1
+
+
+def test_ternary_pack_rejects_bad_arguments():
+    f = L.bnn_ternary_pack
+    ws = 8 * 9
+    assert f(NULL, 0, 8, 32, 32, -1.0, FAKE, 4, NULL, FAKE, ws, NULL) == bnn.BNN_ERR_INVALID_ARG    # no w
+    assert f(FAKE, 0, 8, 32, 32, -1.0, NULL, 4, NULL, FAKE, ws, NULL) == bnn.BNN_ERR_INVALID_ARG    # no codes
+    assert f(FAKE, 0, 8, 32, 31, -1.0, FAKE, 4, NULL, FAKE, ws, NULL) == bnn.BNN_ERR_INVALID_ARG    # ld_w < K
+    assert f(FAKE, 5, 8, 32, 32, -1.0, FAKE, 4, NULL, FAKE, ws, NULL) == bnn.BNN_ERR_INVALID_ARG    # dtype
+    assert f(FAKE, 0, 8, 32, 32, float("nan"), FAKE, 4, NULL, NULL, 0, NULL) == bnn.BNN_ERR_INVALID_ARG
+    assert f(FAKE, 0, 8, 100, 100, -1.0, FAKE, 4, NULL, FAKE, ws, NULL) == bnn.BNN_ERR_INVALID_ARG  # ldq < 8
+    assert f(FAKE, 0, 8, 32, 32, -1.0, FAKE, 4, NULL, NULL, 0, NULL) == bnn.BNN_ERR_INVALID_ARG     # eq. (9) needs ws
+    assert f(FAKE, 0, 8, 32, 32, -1.0, FAKE, 4, NULL, FAKE, ws - 8, NULL) == bnn.BNN_ERR_INVALID_ARG  # ws too small
+    assert f(FAKE, 0, 8, 32, 32, 0.5, FAKE, 4, FAKE, NULL, 0, NULL) == bnn.BNN_ERR_INVALID_ARG      # gamma_out needs ws
+    assert f(FAKE, 0, 8, 32, 32, -1.0, FAKE, 6, NULL, FAKE, ws, NULL) == bnn.BNN_ERR_ALIGNMENT      # ldq % 4
+    assert f(FAKE, 0, 8, 32, 32, -1.0, FAKE_ODD, 4, NULL, FAKE, ws, NULL) == bnn.BNN_ERR_ALIGNMENT
+    assert f(FAKE, 0, 8, 32, 32, -1.0, FAKE, 4, NULL, ctypes.c_void_p(0x10004), ws, NULL) == bnn.BNN_ERR_ALIGNMENT
+    assert f(FAKE, 0, 0, 32, 32, 0.5, FAKE, 4, NULL, NULL, 0, NULL) == bnn.BNN_OK                  # rows = 0
+
+
+def test_ternary_gemv_rejects_bad_arguments():
+    f = L.bnn_ternary_gemv_i8
+    assert f(FAKE, 4, FAKE, 8, 32, NULL, NULL, FAKE, NULL, 8, NULL) == bnn.BNN_ERR_INVALID_ARG   # unknown flag
+    assert f(NULL, 4, FAKE, 8, 32, NULL, NULL, FAKE, NULL, 0, NULL) == bnn.BNN_ERR_INVALID_ARG   # no codes
+    assert f(FAKE, 4, NULL, 8, 32, NULL, NULL, FAKE, NULL, 0, NULL) == bnn.BNN_ERR_INVALID_ARG   # no x
+    assert f(FAKE, 4, FAKE, 8, 32, NULL, NULL, NULL, NULL, 0, NULL) == bnn.BNN_ERR_INVALID_ARG   # no output
+    assert f(FAKE, 4, FAKE, 8, 100, NULL, NULL, FAKE, NULL, 0, NULL) == bnn.BNN_ERR_INVALID_ARG  # ldq too small
+    assert f(FAKE, 6, FAKE, 8, 32, NULL, NULL, FAKE, NULL, 0, NULL) == bnn.BNN_ERR_ALIGNMENT     # ldq % 4
+    assert f(FAKE_ODD, 4, FAKE, 8, 32, NULL, NULL, FAKE, NULL, 0, NULL) == bnn.BNN_ERR_ALIGNMENT
+    assert f(FAKE, 4, FAKE, 8, 32, NULL, NULL, ctypes.c_void_p(0x10002), NULL, 0, NULL) == bnn.BNN_ERR_ALIGNMENT
+    assert f(FAKE, 6148, FAKE, 8, 98305, NULL, NULL, FAKE, NULL, 0, NULL) == bnn.BNN_ERR_UNSUPPORTED
+    assert f(FAKE, 4, FAKE, 0, 32, NULL, NULL, FAKE, NULL, 7, NULL) == bnn.BNN_OK                # N = 0

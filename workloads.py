@@ -19,6 +19,8 @@ fully binary MLP):
 * ``square`` A, W fp32 [8192, 8192] N(0, 1), seeds 4 and 5.
 * ``conv``   X bf16 [64, 64, 56, 56] N(0, 1) seed 6; W fp32 [64, 64, 3, 3]
              N(0, 0.1) seed 7; gamma U(0.5, 1.5), beta N(0, 0.1) [64] seed 8.
+* ``ternary`` W fp32 [11008, 4096] N(0, 0.02) seed 2 (the decode weights, to be
+             ternarised); x int8 [4096] uniform over [-128, 127] seed 17.
 * ``mlp``    X0 fp32 [4096, 4096] N(0, 1) seed 9; W_l fp32 [4096, 4096] N(0, 1)
              seeds 10..13; BatchNorm after layers 1..3 with gamma U(0.5, 1.5),
              beta N(0, 0.1), running mean N(0, 1), running var U(0.5, 2),
@@ -100,6 +102,23 @@ def gemv(N=11008, K=4096, w_seed=2, x_seed=3, x_dtype=torch.bfloat16) -> Gemv:
     W = normal((N, K), 0.02, w_seed)
     x = normal((K,), 1.0, x_seed, dtype=x_dtype)
     return Gemv(N, K, W, x)
+
+
+@dataclass
+class Ternary:
+    N: int
+    K: int
+    W: torch.Tensor      # fp32 [N, K]
+    x: torch.Tensor      # int8 [K]
+
+
+def int8_uniform(shape, seed: int) -> torch.Tensor:
+    """int8 draws, uniform over [-128, 127]."""
+    return torch.randint(-128, 128, tuple(shape), generator=_gen(seed), dtype=torch.int8)
+
+
+def ternary(N=11008, K=4096, w_seed=2, x_seed=17) -> Ternary:
+    return Ternary(N, K, normal((N, K), 0.02, w_seed), int8_uniform((K,), x_seed))
 
 
 @dataclass

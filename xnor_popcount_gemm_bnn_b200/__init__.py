@@ -48,7 +48,8 @@ EXPORTS = (
     "bnn_pack_sign", "bnn_pack_sign_nchw", "bnn_pack_conv3x3_weights", "bnn_xnor_gemm",
     "bnn_xnor_gemv", "bnn_xnor_gemv_ex", "bnn_binary_linear_fused", "bnn_binary_conv3x3_fused",
     "bnn_fold_bn_threshold", "bnn_set_gemm_engine", "bnn_get_gemm_engine", "bnn_selftest_wait_timeout",
-    "bnn_binary_weight_gemv",
+    "bnn_binary_weight_gemv", "bnn_ternary_ld_words", "bnn_ternary_workspace_bytes", "bnn_ternary_pack",
+    "bnn_ternary_gemv_i8",
 )
 
 
@@ -90,6 +91,10 @@ def _load() -> ctypes.CDLL:
         "bnn_set_gemm_engine": (i32, [ctypes.c_int]),
         "bnn_get_gemm_engine": (ctypes.c_int, []),
         "bnn_selftest_wait_timeout": (i32, [i64, p]),
+        "bnn_ternary_ld_words": (i64, [i64]),
+        "bnn_ternary_workspace_bytes": (i64, [i64]),
+        "bnn_ternary_pack": (i32, [p, i32, i64, i64, i64, ctypes.c_double, p, i64, p, p, i64, p]),
+        "bnn_ternary_gemv_i8": (i32, [p, i64, p, i64, i64, p, p, p, p, ctypes.c_uint32, p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -141,6 +146,14 @@ def bnn_packed_ld_words(K: int) -> int:
 
 def bnn_conv3x3_ld_words(cin: int) -> int:
     return int(_lib.bnn_conv3x3_ld_words(int(cin)))
+
+
+def bnn_ternary_ld_words(K: int) -> int:
+    return int(_lib.bnn_ternary_ld_words(int(K)))
+
+
+def bnn_ternary_workspace_bytes(rows: int) -> int:
+    return int(_lib.bnn_ternary_workspace_bytes(int(rows)))
 
 
 def bnn_status_string(status: int) -> str:
@@ -261,6 +274,41 @@ def bnn_binary_weight_gemv(W: torch.Tensor, x: torch.Tensor, K: Optional[int], a
         _ptr(W), _ld(W), _ptr(x), _dtype(x), N, K, _ptr(alpha), _ptr(y), int(flags), _stream(stream)))
 
 
+
+def bnn_ternary_pack(w: torch.Tensor, codes: torch.Tensor, gamma_out: Optional[torch.Tensor] = None,
+                     delta: Optional[float] = None, workspace: Optional[torch.Tensor] = None,
+                     K: Optional[int] = None, stream=None) -> None:
+    """w [rows, K] (fp32/bf16) -> ternary codes [rows, ldq] (int32 storage).
+    delta None: eq. (9) (absmean gamma); else eq. (7) with that threshold.
+    The workspace (needed for gamma) is allocated here with torch when not
+    given."""
+    if w.dim() == 1:
+        w = w[None, :]
+    assert w.stride(-1) == 1 and codes.stride(-1) == 1
+    rows, Kw = w.shape
+    K = Kw if K is None else int(K)
+    d = -1.0 if delta is None else float(delta)
+    if workspace is None and (delta is None or gamma_out is not None):
+        workspace = torch.empty(max(1, bnn_ternary_workspace_bytes(rows) // 8), dtype=torch.float64,
+                                device=w.device)
+    wsb = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("bnn_ternary_pack", _lib.bnn_ternary_pack(
+        _ptr(w), _dtype(w), rows, K, _ld(w), d, _ptr(codes), _ld(codes) if codes.dim() >= 2 else codes.shape[-1],
+        _ptr(gamma_out), _ptr(workspace), wsb, _stream(stream)))
+
+
+def bnn_ternary_gemv_i8(codes: torch.Tensor, x: torch.Tensor, K: Optional[int] = None,
+                        y_i32: Optional[torch.Tensor] = None, y_f32: Optional[torch.Tensor] = None,
+                        w_scale: Optional[torch.Tensor] = None, x_scale: Optional[torch.Tensor] = None,
+                        flags: int = 0, N: Optional[int] = None, stream=None) -> None:
+    """acc = t x (int8 x, exact int32) and/or y = w_scale * x_scale * acc."""
+    assert x.dtype == torch.int8
+    N = codes.shape[0] if N is None else N
+    K = x.shape[-1] if K is None else int(K)
+    _check("bnn_ternary_gemv_i8", _lib.bnn_ternary_gemv_i8(
+        _ptr(codes), _ld(codes), _ptr(x), N, K, _ptr(w_scale), _ptr(x_scale), _ptr(y_i32), _ptr(y_f32),
+        int(flags), _stream(stream)))
+
 def make_epilogue(mode: int, alpha=None, gamma=None, beta=None, popc_thresh=None,
                   thresh_mode=None) -> bnn_epilogue:
     """The epilogue struct with raw device pointers.  It keeps references to
@@ -311,6 +359,11 @@ def bnn_fold_bn_threshold(alpha: torch.Tensor, gamma: torch.Tensor, beta: torch.
 def empty_packed(rows: int, K: int, device="cuda") -> torch.Tensor:
     """int32-typed storage for a packed [rows, bnn_packed_ld_words(K)] matrix."""
     return torch.empty(rows, bnn_packed_ld_words(K), dtype=torch.int32, device=device)
+
+
+def empty_ternary(rows: int, K: int, device="cuda") -> torch.Tensor:
+    """int32-typed storage for ternary codes [rows, bnn_ternary_ld_words(K)]."""
+    return torch.empty(rows, bnn_ternary_ld_words(K), dtype=torch.int32, device=device)
 
 
 def empty_packed_nhwc(n: int, c: int, h: int, w: int, device="cuda") -> torch.Tensor:

@@ -1,10 +1,12 @@
 // libbnn.so: the C ABI declared in include/bnn.h.  Host code here only checks
 // arguments, encodes TMA descriptors, picks launch shapes and launches on the
 // caller's stream; every step of the computation runs in the kernels of
-// pack.cuh, gemm_popc.cuh, gemv.cuh and conv.cuh.
+// pack.cuh, gemm_popc.cuh, gemm_tc.cuh, gemv.cuh, bwgemv.cuh, conv.cuh, conv_tc.cuh
+// and ternary.cuh.
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <cmath>
 #include <climits>
 #include <cstdint>
 #include <cstring>
@@ -20,6 +22,7 @@
 #include "gemv.cuh"
 #include "bwgemv.cuh"
 #include "pack.cuh"
+#include "ternary.cuh"
 
 namespace {
 
@@ -111,6 +114,45 @@ bool bw_gemv_smem_configured() {
         return false;
     if (dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
     return true;
+}
+
+bool ternary_gemv_smem_configured() {
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> done[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+    if (dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return true;
+    if (cudaFuncSetAttribute(bnn::ternary_gemv_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(bnn::tgv::MAX_WORDS * 16)) != cudaSuccess)
+        return false;
+    if (dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
+    return true;
+}
+
+// The staged ternary GEMV with UR rows per warp: shared memory opted in (and
+// the carveout set to the largest shared-memory share) once per device.
+template <int UR, int MINB>
+cudaError_t launch_ternary_staged(cudaLaunchConfig_t& cfg, const uint32_t* codes, int64_t ldq, const int8_t* x,
+                                  int N, int K, int nw, bool x_vec, const float* w_scale, const float* x_scale,
+                                  int32_t* y_i32, float* y_f32, int prefetch, int xstatic, int dependent) {
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> done[kMaxDevices];
+    auto kern = bnn::ternary_gemv_i8_staged_kernel<UR, MINB>;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return cudaErrorInvalidDevice;
+    if (dev >= kMaxDevices || !done[dev].load(std::memory_order_acquire)) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     (int)cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+        if (dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
+    }
+    const int rows = bnn::tgv::WARPS * UR;
+    cfg.gridDim = dim3((unsigned)ceil_div(N, (int64_t)rows));
+    cfg.dynamicSmemBytes = (size_t)bnn::tgv::staged_smem_bytes(rows, nw);
+    return cudaLaunchKernelEx(&cfg, kern, codes, ldq, x, N, K, nw, x_vec, w_scale, x_scale, y_i32, y_f32, prefetch,
+                              xstatic, dependent);
 }
 
 std::atomic<int> g_gemm_engine{BNN_GEMM_ENGINE_AUTO};
@@ -483,6 +525,121 @@ bnn_status bnn_binary_weight_gemv(const uint32_t* W, int64_t ldw, const void* x,
         e = cudaLaunchKernelEx(&cfg, bnn::bw_gemv_kernel<__nv_bfloat16>, W, ldw,
                                static_cast<const __nv_bfloat16*>(x), (int)N, (int)K, (int)kw, alpha, y, prefetch,
                                xstatic, dependent);
+    if (e != cudaSuccess) return BNN_ERR_CUDA;
+    return launch_status();
+}
+
+int64_t bnn_ternary_ld_words(int64_t K) { return K < 1 ? -1 : bnn::ternary_ld_words(K); }
+
+int64_t bnn_ternary_workspace_bytes(int64_t rows) { return rows < 0 ? -1 : 8 * (rows + 1); }
+
+bnn_status bnn_ternary_pack(const void* w, bnn_dtype dt, int64_t rows, int64_t K, int64_t ld_w, double delta,
+                            uint32_t* codes, int64_t ldq, float* gamma_out, void* workspace,
+                            int64_t workspace_bytes, bnn_stream_t stream) {
+    if (w == nullptr || codes == nullptr) return BNN_ERR_INVALID_ARG;
+    if (rows < 0 || K < 1 || ld_w < K || std::isnan(delta)) return BNN_ERR_INVALID_ARG;
+    if (dt != BNN_F32 && dt != BNN_BF16) return BNN_ERR_INVALID_ARG;
+    if (rows > ((int64_t)1 << 40) / K) return BNN_ERR_INVALID_ARG;        // rows * K stays exact in fp64
+    const int64_t nw = bnn::ternary_ld_words(K);
+    if (ldq < nw) return BNN_ERR_INVALID_ARG;
+    if ((ldq & 3) != 0 || !aligned(codes, 16)) return BNN_ERR_ALIGNMENT;
+    const size_t es = dt == BNN_F32 ? 4 : 2;
+    if (!aligned(w, es) || (gamma_out != nullptr && !aligned(gamma_out, 4))) return BNN_ERR_ALIGNMENT;
+    const bool need_gamma = delta < 0.0 || gamma_out != nullptr;
+    if (need_gamma) {
+        if (workspace == nullptr || workspace_bytes < bnn_ternary_workspace_bytes(rows)) return BNN_ERR_INVALID_ARG;
+        if (!aligned(workspace, 8)) return BNN_ERR_ALIGNMENT;
+    }
+    if (rows == 0) return BNN_OK;
+    const bool vec_ok = aligned(w, 16) && ((ld_w * (int64_t)es) % 16 == 0);
+    const int64_t blocks = ceil_div(rows, 8);
+    if (blocks > INT_MAX) return BNN_ERR_INVALID_ARG;
+    cudaStream_t s = as_cuda(stream);
+    double* rowsum = static_cast<double*>(workspace);
+    double* gamma_d = need_gamma ? rowsum + rows : nullptr;
+    // Row sums (plain launch: ordered after all earlier work), then gamma and
+    // the pack as programmatic dependents, each waiting for its predecessor
+    // before reading what that one wrote.
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = need_gamma ? 1 : 0;
+    cudaError_t e = cudaSuccess;
+    if (need_gamma) {
+        if (dt == BNN_F32)
+            bnn::ternary_abs_rowsum_kernel<float, 4><<<(unsigned)blocks, 256, 0, s>>>(
+                static_cast<const float*>(w), rows, K, ld_w, vec_ok, rowsum);
+        else
+            bnn::ternary_abs_rowsum_kernel<__nv_bfloat16, 4><<<(unsigned)blocks, 256, 0, s>>>(
+                static_cast<const __nv_bfloat16*>(w), rows, K, ld_w, vec_ok, rowsum);
+        cfg.gridDim = dim3(1);
+        cfg.blockDim = dim3(1024);
+        e = cudaLaunchKernelEx(&cfg, bnn::ternary_gamma_kernel, (const double*)rowsum, rows, K, gamma_d, gamma_out);
+        if (e != cudaSuccess) return BNN_ERR_CUDA;
+    }
+    const double* gsrc = delta < 0.0 ? gamma_d : nullptr;
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(256);
+    if (dt == BNN_F32)
+        e = cudaLaunchKernelEx(&cfg, bnn::pack_ternary_kernel<float, 4>, static_cast<const float*>(w), rows, K, ld_w,
+                               vec_ok, gsrc, delta, codes, ldq);
+    else
+        e = cudaLaunchKernelEx(&cfg, bnn::pack_ternary_kernel<__nv_bfloat16, 4>,
+                               static_cast<const __nv_bfloat16*>(w), rows, K, ld_w, vec_ok, gsrc, delta, codes, ldq);
+    if (e != cudaSuccess) return BNN_ERR_CUDA;
+    return launch_status();
+}
+
+bnn_status bnn_ternary_gemv_i8(const uint32_t* codes, int64_t ldq, const int8_t* x, int64_t N, int64_t K,
+                               const float* w_scale, const float* x_scale, int32_t* y_i32, float* y_f32,
+                               uint32_t flags, bnn_stream_t stream) {
+    constexpr uint32_t kAll = BNN_GEMV_WEIGHTS_STATIC | BNN_GEMV_INPUTS_STATIC | BNN_GEMV_OUTPUT_FREE;
+    if ((flags & ~kAll) != 0) return BNN_ERR_INVALID_ARG;
+    if (codes == nullptr || x == nullptr || (y_i32 == nullptr && y_f32 == nullptr)) return BNN_ERR_INVALID_ARG;
+    if (N < 0 || K < 1 || N > INT_MAX) return BNN_ERR_INVALID_ARG;
+    const int64_t nw = bnn::ternary_ld_words(K);
+    if (ldq < nw) return BNN_ERR_INVALID_ARG;
+    if ((ldq & 3) != 0 || !aligned(codes, 16)) return BNN_ERR_ALIGNMENT;
+    if ((y_i32 != nullptr && !aligned(y_i32, 4)) || (y_f32 != nullptr && !aligned(y_f32, 4)) ||
+        (w_scale != nullptr && !aligned(w_scale, 4)) || (x_scale != nullptr && !aligned(x_scale, 4)))
+        return BNN_ERR_ALIGNMENT;
+    if (nw > bnn::tgv::MAX_WORDS) return BNN_ERR_UNSUPPORTED;
+    if (N == 0) return BNN_OK;
+    if (!ternary_gemv_smem_configured()) return BNN_ERR_CUDA;
+    cudaLaunchConfig_t cfg{};
+    cfg.blockDim = dim3(bnn::tgv::THREADS);
+    cfg.stream = as_cuda(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const int prefetch = (flags & BNN_GEMV_WEIGHTS_STATIC) ? 1 : 0;
+    const int xstatic = (flags & BNN_GEMV_INPUTS_STATIC) ? 1 : 0;
+    const int dependent = flags == kAll ? 2 : 1;
+    const bool x_vec = aligned(x, 16);
+    cudaError_t e;
+    if (nw <= bnn::tgv::STAGED_MAX_WORDS) {
+        // Shared-memory staged kernel: 64 rows per block up to K = 4096, fewer
+        // for longer rows (the codes of a block stay under 64 KiB).
+        if (nw <= 256)
+            e = launch_ternary_staged<8, 3>(cfg, codes, ldq, x, (int)N, (int)K, (int)nw, x_vec, w_scale, x_scale,
+                                            y_i32, y_f32, prefetch, xstatic, dependent);
+        else if (nw <= 512)
+            e = launch_ternary_staged<4, 3>(cfg, codes, ldq, x, (int)N, (int)K, (int)nw, x_vec, w_scale, x_scale,
+                                            y_i32, y_f32, prefetch, xstatic, dependent);
+        else
+            e = launch_ternary_staged<2, 2>(cfg, codes, ldq, x, (int)N, (int)K, (int)nw, x_vec, w_scale, x_scale,
+                                            y_i32, y_f32, prefetch, xstatic, dependent);
+    } else {
+        cfg.gridDim = dim3((unsigned)ceil_div(N, (int64_t)bnn::tgv::ROWS_PER_BLOCK));
+        cfg.dynamicSmemBytes = (size_t)nw * 16;
+        e = cudaLaunchKernelEx(&cfg, bnn::ternary_gemv_i8_kernel, codes, ldq, x, (int)N, (int)K, (int)nw, x_vec,
+                               w_scale, x_scale, y_i32, y_f32, prefetch, xstatic, dependent);
+    }
     if (e != cudaSuccess) return BNN_ERR_CUDA;
     return launch_status();
 }
