@@ -172,8 +172,8 @@ def random_ternary(N, K, seed, p_zero=0.3):
     return np.where(rng.random((N, K)) < p_zero, 0, np.where(rng.random((N, K)) < 0.5, -1, 1)).astype(np.int8)
 
 
-# K <= 16384: the shared-memory staged kernel (64, 32 or 16 rows per block);
-# longer rows: the register kernel.
+# flags 7 launch 4 rows per warp, the other flags 8 rows per warp; both for
+# every shape.
 @pytest.mark.parametrize("N,K", [(1, 1), (5, 17), (64, 1000), (65, 33), (300, 4096), (100, 4100),
                                  (129, 8192), (33, 12288), (40, 11008), (17, 16384), (300, 16400),
                                  (70, 50000), (3, 98304)])

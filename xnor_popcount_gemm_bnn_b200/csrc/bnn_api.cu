@@ -116,43 +116,22 @@ bool bw_gemv_smem_configured() {
     return true;
 }
 
+// Opt the ternary GEMV (x staged in up to 96 KiB of shared memory) in once
+// per device, for both block shapes the launcher uses.
 bool ternary_gemv_smem_configured() {
     constexpr int kMaxDevices = 64;
     static std::atomic<int> done[kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
     if (dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return true;
-    if (cudaFuncSetAttribute(bnn::ternary_gemv_i8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(bnn::tgv::MAX_WORDS * 16)) != cudaSuccess)
+    const int bytes = (int)(bnn::tgv::MAX_WORDS * 16);
+    if (cudaFuncSetAttribute(bnn::ternary_gemv_i8_kernel<256, 4, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bytes) != cudaSuccess ||
+        cudaFuncSetAttribute(bnn::ternary_gemv_i8_kernel<256, 8, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bytes) != cudaSuccess)
         return false;
     if (dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
     return true;
-}
-
-// The staged ternary GEMV with UR rows per warp: shared memory opted in (and
-// the carveout set to the largest shared-memory share) once per device.
-template <int UR, int MINB>
-cudaError_t launch_ternary_staged(cudaLaunchConfig_t& cfg, const uint32_t* codes, int64_t ldq, const int8_t* x,
-                                  int N, int K, int nw, bool x_vec, const float* w_scale, const float* x_scale,
-                                  int32_t* y_i32, float* y_f32, int prefetch, int xstatic, int dependent) {
-    constexpr int kMaxDevices = 64;
-    static std::atomic<int> done[kMaxDevices];
-    auto kern = bnn::ternary_gemv_i8_staged_kernel<UR, MINB>;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return cudaErrorInvalidDevice;
-    if (dev >= kMaxDevices || !done[dev].load(std::memory_order_acquire)) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                     (int)cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess) return e;
-        if (dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
-    }
-    const int rows = bnn::tgv::WARPS * UR;
-    cfg.gridDim = dim3((unsigned)ceil_div(N, (int64_t)rows));
-    cfg.dynamicSmemBytes = (size_t)bnn::tgv::staged_smem_bytes(rows, nw);
-    return cudaLaunchKernelEx(&cfg, kern, codes, ldq, x, N, K, nw, x_vec, w_scale, x_scale, y_i32, y_f32, prefetch,
-                              xstatic, dependent);
 }
 
 std::atomic<int> g_gemm_engine{BNN_GEMM_ENGINE_AUTO};
@@ -610,7 +589,8 @@ bnn_status bnn_ternary_gemv_i8(const uint32_t* codes, int64_t ldq, const int8_t*
     if (N == 0) return BNN_OK;
     if (!ternary_gemv_smem_configured()) return BNN_ERR_CUDA;
     cudaLaunchConfig_t cfg{};
-    cfg.blockDim = dim3(bnn::tgv::THREADS);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = (size_t)nw * 16;
     cfg.stream = as_cuda(stream);
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -619,26 +599,21 @@ bnn_status bnn_ternary_gemv_i8(const uint32_t* codes, int64_t ldq, const int8_t*
     cfg.numAttrs = 1;
     const int prefetch = (flags & BNN_GEMV_WEIGHTS_STATIC) ? 1 : 0;
     const int xstatic = (flags & BNN_GEMV_INPUTS_STATIC) ? 1 : 0;
-    const int dependent = flags == kAll ? 2 : 1;
+    const bool independent = flags == kAll;
+    const int dependent = independent ? 2 : 1;
     const bool x_vec = aligned(x, 16);
+    // Measured at the decode shape (K = 4096): 4 rows per warp for independent
+    // steps (more, smaller blocks overlap consecutive launches), 8 for a
+    // dependent chain.
     cudaError_t e;
-    if (nw <= bnn::tgv::STAGED_MAX_WORDS) {
-        // Shared-memory staged kernel: 64 rows per block up to K = 4096, fewer
-        // for longer rows (the codes of a block stay under 64 KiB).
-        if (nw <= 256)
-            e = launch_ternary_staged<8, 3>(cfg, codes, ldq, x, (int)N, (int)K, (int)nw, x_vec, w_scale, x_scale,
-                                            y_i32, y_f32, prefetch, xstatic, dependent);
-        else if (nw <= 512)
-            e = launch_ternary_staged<4, 3>(cfg, codes, ldq, x, (int)N, (int)K, (int)nw, x_vec, w_scale, x_scale,
-                                            y_i32, y_f32, prefetch, xstatic, dependent);
-        else
-            e = launch_ternary_staged<2, 2>(cfg, codes, ldq, x, (int)N, (int)K, (int)nw, x_vec, w_scale, x_scale,
-                                            y_i32, y_f32, prefetch, xstatic, dependent);
+    if (independent) {
+        cfg.gridDim = dim3((unsigned)ceil_div(N, (int64_t)32));
+        e = cudaLaunchKernelEx(&cfg, bnn::ternary_gemv_i8_kernel<256, 4, 2>, codes, ldq, x, (int)N, (int)K, (int)nw,
+                               x_vec, w_scale, x_scale, y_i32, y_f32, prefetch, xstatic, dependent);
     } else {
-        cfg.gridDim = dim3((unsigned)ceil_div(N, (int64_t)bnn::tgv::ROWS_PER_BLOCK));
-        cfg.dynamicSmemBytes = (size_t)nw * 16;
-        e = cudaLaunchKernelEx(&cfg, bnn::ternary_gemv_i8_kernel, codes, ldq, x, (int)N, (int)K, (int)nw, x_vec,
-                               w_scale, x_scale, y_i32, y_f32, prefetch, xstatic, dependent);
+        cfg.gridDim = dim3((unsigned)ceil_div(N, (int64_t)64));
+        e = cudaLaunchKernelEx(&cfg, bnn::ternary_gemv_i8_kernel<256, 8, 2>, codes, ldq, x, (int)N, (int)K, (int)nw,
+                               x_vec, w_scale, x_scale, y_i32, y_f32, prefetch, xstatic, dependent);
     }
     if (e != cudaSuccess) return BNN_ERR_CUDA;
     return launch_status();

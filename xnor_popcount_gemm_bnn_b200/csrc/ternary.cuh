@@ -198,14 +198,7 @@ pack_ternary_kernel(const T* __restrict__ w, int64_t rows, int64_t K, int64_t ld
 // sum c x - sum x, one warp reduction.
 // ---------------------------------------------------------------------------
 namespace tgv {
-constexpr int THREADS = 256;
-constexpr int WARPS = THREADS / 32;
-constexpr int U = 4;                       // register kernel: rows per warp
-constexpr int P = 2;                       // register kernel: chunks per lane per pass (loads in flight: U * P)
-constexpr int ROWS_PER_BLOCK = WARPS * U;
 constexpr int64_t MAX_WORDS = 6144;        // staged x = 16 bytes per code word: 96 KiB (K <= 98304)
-constexpr int64_t STAGED_MAX_WORDS = 1024; // the staged kernel: codes of K <= 16384 per row
-__host__ __device__ constexpr int staged_smem_bytes(int rows, int nw) { return 16 + rows * nw * 4 + nw * 16; }
 }  // namespace tgv
 
 __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
@@ -217,7 +210,7 @@ __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
 __device__ __forceinline__ void stage_x_transposed(const int8_t* __restrict__ x, int K, int nw, bool vec_ok,
                                                    uint32_t* xs) {
     const int nch = nw / 4;
-    for (int g = threadIdx.x; g < nw; g += tgv::THREADS) {
+    for (int g = threadIdx.x; g < nw; g += blockDim.x) {
         uint32_t a[4];
         if (vec_ok && 16 * g + 16 <= K) {
             const uint4 q = *reinterpret_cast<const uint4*>(x + 16 * g);
@@ -279,17 +272,20 @@ __device__ __forceinline__ int lane_total(const int (&acc)[2], int xsum) {
     return acc[0] + (acc[1] >> 2) - xsum;
 }
 
-// Register kernel (any K up to 98304).  A warp owns U rows; lane l reads the
-// 16-byte chunks l, l + 32, ... of each (a warp-wide load is 512 contiguous
-// bytes of one row) and P chunks per row are in flight before any is used.
-// Programmatic dependent launch as the XNOR GEMV: static weights are loaded
-// before the wait for the previous grid, static inputs staged before it too.
-__global__ void __launch_bounds__(tgv::THREADS)
+// TH threads per block; a warp owns U rows.  Lane l reads the 16-byte chunks
+// l, l + 32, ... of each row (a warp-wide load is 512 contiguous bytes of one
+// row) and P chunks per row are in flight before any is used.  Programmatic
+// dependent launch as the XNOR GEMV: static weights are loaded before the
+// wait for the previous grid, static inputs staged before it too.  The
+// launcher picks U per dependency mode (independent steps: U = 4, 344 blocks
+// at N = 11008; a dependent chain: U = 8, fewer and fuller blocks).
+template <int TH, int U, int P>
+__global__ void __launch_bounds__(TH)
 ternary_gemv_i8_kernel(const uint32_t* __restrict__ Q, int64_t ldq, const int8_t* __restrict__ x, int N, int K,
                        int nw, bool x_vec, const float* __restrict__ w_scale, const float* __restrict__ x_scale,
                        int32_t* __restrict__ y_i32, float* __restrict__ y_f32, int prefetch, int xstatic,
                        int dependent) {
-    using namespace tgv;
+    constexpr int WARPS = TH / 32;
     extern __shared__ __align__(16) uint32_t txs[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row0 = (blockIdx.x * WARPS + warp) * U;
@@ -351,97 +347,6 @@ ternary_gemv_i8_kernel(const uint32_t* __restrict__ Q, int64_t ldq, const int8_t
             if (r < N) {
                 if (y_i32 != nullptr) y_i32[r] = tot[u];
                 if (y_f32 != nullptr) y_f32[r] = scale * (float)tot[u];
-            }
-        }
-    }
-    if (dependent == 2) grid_dependency_wait();
-}
-
-// Staged kernel (K <= 16384).  A block owns R = WARPS * UR consecutive rows
-// (MINB: blocks per SM the register budget is set for);
-// warp 0 copies them into shared memory with one bulk copy per row, all
-// completing on one mbarrier, so the bytes in flight are bounded by shared
-// memory rather than registers and several consecutive launches can keep
-// their copies in flight on one SM.  Warp w then sums rows w*UR .. w*UR+UR-1
-// from shared memory, lane l taking chunks l, l + 32, ...
-// The wait on the copies is bounded: on time-out the kernel records
-// BNN_ERR_DEVICE_TIMEOUT, waits once more (bounded) for the copies it issued
-// and returns without writing y.
-template <int UR, int MINB>
-__global__ void __launch_bounds__(tgv::THREADS, MINB)
-ternary_gemv_i8_staged_kernel(const uint32_t* __restrict__ Q, int64_t ldq, const int8_t* __restrict__ x, int N,
-                              int K, int nw, bool x_vec, const float* __restrict__ w_scale,
-                              const float* __restrict__ x_scale, int32_t* __restrict__ y_i32,
-                              float* __restrict__ y_f32, int prefetch, int xstatic, int dependent) {
-    using namespace tgv;
-    constexpr int R = WARPS * UR;
-    extern __shared__ __align__(128) uint32_t tsm[];
-    uint64_t* bar = reinterpret_cast<uint64_t*>(tsm);
-    uint32_t* cs = tsm + 4;                              // [R][nw] codes
-    uint32_t* xs = cs + R * nw;                          // staged x
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int row0 = blockIdx.x * R;
-    const int nrows = min(R, N - row0);
-    const int nch = nw / 4;
-    grid_dependents_launch();
-    if (threadIdx.x == 0) {
-        mbar_init(bar, 1);
-        fence_mbarrier_init();
-    }
-    __syncthreads();
-    auto issue = [&]() {
-        if (warp == 0) {
-            const uint32_t row_bytes = (uint32_t)nw * 4u;
-            if (lane == 0) mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)nrows);
-            __syncwarp();
-            for (int r = lane; r < nrows; r += 32)
-                bulk_load(cs + r * nw, Q + (int64_t)(row0 + r) * ldq, row_bytes, bar);
-        }
-    };
-    float scale = 1.0f;
-    auto stage = [&]() {
-        stage_x_transposed(x, K, nw, x_vec, xs);
-        if (y_f32 != nullptr) scale = (w_scale != nullptr ? *w_scale : 1.0f) * (x_scale != nullptr ? *x_scale : 1.0f);
-    };
-    const bool late_wait = prefetch && xstatic;
-    if (prefetch) issue();
-    if (xstatic) stage();
-    if (dependent == 1 && !late_wait) grid_dependency_wait();
-    if (!prefetch) issue();
-    if (!xstatic) stage();
-    // Every thread waits on the copies itself; the block leaves together if
-    // any wait ran out (after one more bounded wait for the copies).
-    const bool copied = mbar_wait_bounded(bar, 0);
-    if (!__syncthreads_and(copied)) {
-        if (!copied) mbar_wait_bounded(bar, 0);
-        grid_dependency_wait();
-        return;
-    }
-
-    int acc[UR][2];
-    #pragma unroll
-    for (int u = 0; u < UR; ++u) acc[u][0] = acc[u][1] = 0;
-    int xsum = 0;
-    const uint32_t* wrow = cs + warp * UR * nw;
-    for (int c = lane; c < nch; c += 32) {
-        uint4 X[4];
-        load_x_chunk(xs, nch, c, X);
-        xsum = xsum_chunk(X, xsum);
-        #pragma unroll
-        for (int u = 0; u < UR; ++u)
-            ternary_chunk(*reinterpret_cast<const uint4*>(wrow + u * nw + 4 * c), X, acc[u]);
-    }
-    int tot[UR];
-    #pragma unroll
-    for (int u = 0; u < UR; ++u) tot[u] = __reduce_add_sync(0xffffffffu, lane_total(acc[u], xsum));
-    if (dependent == 1 && late_wait) grid_dependency_wait();
-    if (lane == 0) {
-        #pragma unroll
-        for (int u = 0; u < UR; ++u) {
-            const int lr = warp * UR + u;
-            if (lr < nrows) {
-                if (y_i32 != nullptr) y_i32[row0 + lr] = tot[u];
-                if (y_f32 != nullptr) y_f32[row0 + lr] = scale * (float)tot[u];
             }
         }
     }
