@@ -334,6 +334,36 @@ bnn_status bnn_ternary_pack(const void* w, bnn_dtype dt, int64_t rows, int64_t K
                             double delta, uint32_t* codes, int64_t ldq, float* gamma_out,
                             void* workspace, int64_t workspace_bytes, bnn_stream_t stream);
 
+/* Largest `rows` bnn_ternary_pack_noalloc accepts. */
+#define BNN_TERNARY_PACK_NOALLOC_MAX_ROWS 262144
+
+/* bnn_ternary_pack_noalloc -- bnn_ternary_pack without a caller workspace.
+ * The pages have no counterpart: this entry point exists for callers that
+ * cannot allocate device memory themselves -- code that only receives the
+ * input and output pointers from a host framework (a plugin or custom
+ * operator of another runtime, whose allocator it cannot reach), or a
+ * latency-critical path where cudaMalloc, which may synchronise the device,
+ * is not allowed.  It computes exactly what bnn_ternary_pack computes, with
+ * the same arguments minus the workspace, and allocates nothing: the row sums
+ * and gamma go to one array of BNN_TERNARY_PACK_NOALLOC_MAX_ROWS + 1 doubles
+ * (about 2 MiB) that the library holds in device memory on every GPU that
+ * loads it, for the life of the process.
+ *   rows > BNN_TERNARY_PACK_NOALLOC_MAX_ROWS: BNN_ERR_UNSUPPORTED (use
+ *   bnn_ternary_pack with a workspace).
+ *   The first call on a device looks up that array's device address (one
+ *   cudaGetSymbolAddress, with the device current); make that first call
+ *   before any stream capture.
+ *   Every call on a device shares the one array.  Calls whose kernels may
+ *   overlap on the GPU (on different streams without ordering between them)
+ *   race on it and must not be issued; calls in stream order are safe.
+ *   Nothing in the array needs to start at zero: each call writes every entry
+ *   it reads.
+ *   Errors: as bnn_ternary_pack (INVALID_ARG, ALIGNMENT), UNSUPPORTED (too
+ *   many rows), CUDA (the address look-up failed). */
+bnn_status bnn_ternary_pack_noalloc(const void* w, bnn_dtype dt, int64_t rows, int64_t K, int64_t ld_w,
+                                    double delta, uint32_t* codes, int64_t ldq, float* gamma_out,
+                                    bnn_stream_t stream);
+
 /* bnn_ternary_gemv_i8 -- ternary weights times an int8 activation vector:
  *   acc[n]   = sum_k t_nk * x_k                    (exact, int32)
  *   y_f32[n] = fp32( fp32(w_scale * x_scale) * fp32(acc[n]) )

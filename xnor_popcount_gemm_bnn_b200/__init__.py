@@ -49,7 +49,7 @@ EXPORTS = (
     "bnn_xnor_gemv", "bnn_xnor_gemv_ex", "bnn_binary_linear_fused", "bnn_binary_conv3x3_fused",
     "bnn_fold_bn_threshold", "bnn_set_gemm_engine", "bnn_get_gemm_engine", "bnn_selftest_wait_timeout",
     "bnn_binary_weight_gemv", "bnn_ternary_ld_words", "bnn_ternary_workspace_bytes", "bnn_ternary_pack",
-    "bnn_ternary_gemv_i8",
+    "bnn_ternary_gemv_i8", "bnn_ternary_pack_noalloc",
 )
 
 
@@ -95,6 +95,7 @@ def _load() -> ctypes.CDLL:
         "bnn_ternary_workspace_bytes": (i64, [i64]),
         "bnn_ternary_pack": (i32, [p, i32, i64, i64, i64, ctypes.c_double, p, i64, p, p, i64, p]),
         "bnn_ternary_gemv_i8": (i32, [p, i64, p, i64, i64, p, p, p, p, ctypes.c_uint32, p]),
+        "bnn_ternary_pack_noalloc": (i32, [p, i32, i64, i64, i64, ctypes.c_double, p, i64, p, p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -296,6 +297,25 @@ def bnn_ternary_pack(w: torch.Tensor, codes: torch.Tensor, gamma_out: Optional[t
         _ptr(w), _dtype(w), rows, K, _ld(w), d, _ptr(codes), _ld(codes) if codes.dim() >= 2 else codes.shape[-1],
         _ptr(gamma_out), _ptr(workspace), wsb, _stream(stream)))
 
+
+
+BNN_TERNARY_PACK_NOALLOC_MAX_ROWS = 262144
+
+
+def bnn_ternary_pack_noalloc(w: torch.Tensor, codes: torch.Tensor, gamma_out: Optional[torch.Tensor] = None,
+                             delta: Optional[float] = None, K: Optional[int] = None, stream=None) -> None:
+    """bnn_ternary_pack for callers that cannot allocate device memory: the
+    scratch space lives in the library (rows <= 262144); this wrapper
+    allocates nothing either."""
+    if w.dim() == 1:
+        w = w[None, :]
+    assert w.stride(-1) == 1 and codes.stride(-1) == 1
+    rows, Kw = w.shape
+    K = Kw if K is None else int(K)
+    d = -1.0 if delta is None else float(delta)
+    _check("bnn_ternary_pack_noalloc", _lib.bnn_ternary_pack_noalloc(
+        _ptr(w), _dtype(w), rows, K, _ld(w), d, _ptr(codes), _ld(codes) if codes.dim() >= 2 else codes.shape[-1],
+        _ptr(gamma_out), _stream(stream)))
 
 def bnn_ternary_gemv_i8(codes: torch.Tensor, x: torch.Tensor, K: Optional[int] = None,
                         y_i32: Optional[torch.Tensor] = None, y_f32: Optional[torch.Tensor] = None,

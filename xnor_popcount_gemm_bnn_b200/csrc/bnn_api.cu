@@ -572,6 +572,42 @@ bnn_status bnn_ternary_pack(const void* w, bnn_dtype dt, int64_t rows, int64_t K
     return launch_status();
 }
 
+// ---------------------------------------------------------------------------
+// bnn_ternary_pack_noalloc: bnn_ternary_pack with its workspace in a
+// library-owned device array instead of caller memory.
+// ---------------------------------------------------------------------------
+namespace {
+
+// Row sums (one double per row) plus gamma: BNN_TERNARY_PACK_NOALLOC_MAX_ROWS
+// + 1 doubles, about 2 MiB, held by every GPU that loads the library.
+static __device__ __align__(256) double g_ternary_scratch[BNN_TERNARY_PACK_NOALLOC_MAX_ROWS + 1];
+
+// The device address of g_ternary_scratch on the current device, looked up
+// once per device (host code cannot use the symbol itself as a pointer).
+void* ternary_scratch_address() {
+    constexpr int kMaxDevices = 64;
+    static std::atomic<void*> addr[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    void* p = addr[dev].load(std::memory_order_acquire);
+    if (p != nullptr) return p;
+    if (cudaGetSymbolAddress(&p, g_ternary_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    addr[dev].store(p, std::memory_order_release);
+    return p;
+}
+
+}  // namespace
+
+bnn_status bnn_ternary_pack_noalloc(const void* w, bnn_dtype dt, int64_t rows, int64_t K, int64_t ld_w, double delta,
+                                    uint32_t* codes, int64_t ldq, float* gamma_out, bnn_stream_t stream) {
+    if (rows > BNN_TERNARY_PACK_NOALLOC_MAX_ROWS) return BNN_ERR_UNSUPPORTED;
+    if (rows < 0) return BNN_ERR_INVALID_ARG;
+    void* scratch = ternary_scratch_address();
+    if (scratch == nullptr) return BNN_ERR_CUDA;
+    return bnn_ternary_pack(w, dt, rows, K, ld_w, delta, codes, ldq, gamma_out, scratch,
+                            (int64_t)sizeof(g_ternary_scratch), stream);
+}
+
 bnn_status bnn_ternary_gemv_i8(const uint32_t* codes, int64_t ldq, const int8_t* x, int64_t N, int64_t K,
                                const float* w_scale, const float* x_scale, int32_t* y_i32, float* y_f32,
                                uint32_t flags, bnn_stream_t stream) {
