@@ -114,7 +114,7 @@ KERNEL_SOURCES = {
     "pack_sign_rows_kernel": ("pack.cuh", "common.cuh"),
     "pack_sign_nchw_kernel": ("pack.cuh", "common.cuh"),
     "bw_gemv_kernel": ("bwgemv.cuh", "common.cuh"),
-    "ternary_gemv_i8_staged_kernel": ("ternary.cuh", "common.cuh"),
+    "ternary_gemv_i8_kernel": ("ternary.cuh", "common.cuh"),
     "pack_ternary_kernel": ("ternary.cuh", "common.cuh"),
 }
 
@@ -685,7 +685,7 @@ def _row_ternary(torch, bnn, workloads, dev, pk, rows, timed, steps, ws):
         "value": round(ws * ach, 1), "unit": "GB/s", "ms_per_step": ms / n,
         "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"],
                      "frac": round(ach / pk["hbm_gbs"], 4), "algorithmic_bytes": b,
-                     "traffic": recorded_traffic("ternary_gemv_i8_staged_kernel")},
+                     "traffic": recorded_traffic("ternary_gemv_i8_kernel")},
         "dependent_chain": {"value": round(ws * ach_dep, 1), "unit": "GB/s", "ms_per_step": ms_dep / n,
                             "frac": round(ach_dep / pk["hbm_gbs"], 4)}}
     rows["ternary_pack"] = {
