@@ -15,6 +15,8 @@ real-valued epilogues evaluated in float64 here with numpy:
   bit 1 is -1, pad bits encode +1).
 * alpha and the scaled product -- "Extreme Quantization ...", Binary Neural
   Networks section, eq. (1): y = alpha * (w_b^T x), alpha = (1/n) sum |w_i|.
+* per-channel sign threshold (RSign) -- "State of the Art Survey (2016 ->
+  2026)", classic CNN BNN table (ReActNet): sign(x - beta_c).
 * ternary weights -- "Extreme Quantization ...", eq. (7) (threshold Delta)
   and eq. (9) (BitNet b1.58: RoundClip(W / gamma, -1, 1), gamma = mean |W|
   over the matrix); "First Principles ...", the op-per-element table
@@ -101,6 +103,25 @@ def sign_pm1(x) -> np.ndarray:
     _lib().oracle_sign_f32(_ptr(xf), xf.size, _ptr(out))
     return out
 
+
+
+def rsign_pm1(x, beta, axis: int = -1) -> np.ndarray:
+    """int8 +1/-1: sign(x - beta_c) with a learned threshold beta_c per channel
+    (ReActNet's RSign, "State of the Art Survey (2016 -> 2026)", classic CNN
+    BNN table: a per-channel reshape of the activation distribution before
+    the sign).  beta has one entry per index of x along `axis` and is
+    broadcast over the other axes.  The difference is taken in float64 and
+    mapped by the Notation rule of "Extreme Quantization ..." (-1 exactly
+    where x - beta < 0; so x = beta gives +1, and NaN anywhere gives +1)."""
+    xf = _f32(x).astype(np.float64)
+    b = _f32(beta).astype(np.float64).reshape(-1)
+    ax = axis % xf.ndim
+    assert b.size == xf.shape[ax], (b.size, xf.shape, ax)
+    shape = [1] * xf.ndim
+    shape[ax] = b.size
+    with np.errstate(invalid="ignore"):
+        v = xf - b.reshape(shape)
+        return np.where(v < 0.0, -1, 1).astype(np.int8)
 
 def pack_pm1(b: np.ndarray, ld: int | None = None) -> np.ndarray:
     """Pack a [rows, K] int8 +1/-1 matrix into uint32 [rows, ld] words."""

@@ -202,7 +202,38 @@ def _tern_sign_swapped(t, x):          # add where -1, subtract where +1
     return -oracle.ternary_product(t, x)
 
 
+
+def _rsign_tie_negative(x, beta, axis=-1):      # x = beta mapped to -1
+    xf = oracle._f32(x).astype(np.float64)
+    b = oracle._f32(beta).astype(np.float64).reshape(-1)
+    shape = [1] * xf.ndim
+    shape[axis % xf.ndim] = b.size
+    with np.errstate(invalid="ignore"):
+        return np.where(xf - b.reshape(shape) <= 0.0, -1, 1).astype(np.int8)
+
+
+def _rsign_reversed(x, beta, axis=-1):          # sign(beta - x)
+    xf = oracle._f32(x).astype(np.float64)
+    b = oracle._f32(beta).astype(np.float64).reshape(-1)
+    shape = [1] * xf.ndim
+    shape[axis % xf.ndim] = b.size
+    with np.errstate(invalid="ignore"):
+        return np.where(b.reshape(shape) - xf < 0.0, -1, 1).astype(np.int8)
+
+
+def _rsign_last_axis(x, beta, axis=-1):         # threshold applied along the last axis
+    xf = oracle._f32(x).astype(np.float64)
+    b = oracle._f32(beta).astype(np.float64).reshape(-1)
+    if b.size != xf.shape[-1]:
+        b = np.resize(b, xf.shape[-1])
+    with np.errstate(invalid="ignore"):
+        return np.where(xf - b < 0.0, -1, 1).astype(np.int8)
+
+
 MUTANTS = {
+    "rsign_tie_negative": dict(rsign_pm1=_rsign_tie_negative),
+    "rsign_reversed": dict(rsign_pm1=_rsign_reversed),
+    "rsign_wrong_axis": dict(rsign_pm1=_rsign_last_axis),
     "ternary_gamma_without_abs": dict(ternary_quantize=_tern_gamma_noabs),
     "ternary_round_half_away": dict(ternary_quantize=_tern_round_half_away),
     "ternary_no_clip": dict(ternary_quantize=_tern_no_clip),

@@ -395,6 +395,40 @@ def check_ternary_product(o):
     assert np.array_equal(acc, ref) and np.array_equal(y, 2.0 * ref.astype(np.float64))
 
 
+
+def check_rsign(o, golden):
+    """RSign (the survey's ReActNet row) as sign(x - beta_c): hand-computed
+    cases, the comparison form x < beta on random and special values, beta = 0
+    reducing to the Notation sign, invariance under a common exact shift, and
+    the channel axis against explicit loops."""
+    g = json.load(open(os.path.join(golden, "rsign_rule.json")))
+    x = np.array([float(a) for a, _, _ in g["cases"]], np.float32)
+    b = np.array([float(c) for _, c, _ in g["cases"]], np.float32)
+    want = [e for *_, e in g["cases"]]
+    got = [int(o.rsign_pm1(np.array([xi]), np.array([bi]))[0]) for xi, bi in zip(x, b)]
+    assert got == want, (got, want)
+    rng = np.random.default_rng(31)
+    xs = rng.standard_normal((6, 40)).astype(np.float32)
+    xs[0, :8] = [0.0, -0.0, np.inf, -np.inf, np.nan, 1e-45, -1e-45, 0.25]
+    bs = rng.standard_normal(40).astype(np.float32)
+    bs[:4] = [0.0, 0.0, np.inf, -np.inf]
+    with np.errstate(invalid="ignore"):
+        cmp = np.where(xs < bs[None, :], -1, 1).astype(np.int8)
+    assert np.array_equal(o.rsign_pm1(xs, bs, axis=1), cmp)
+    assert np.array_equal(o.rsign_pm1(xs, np.zeros(40, np.float32), axis=1), o.sign_pm1(xs))
+    xi = rng.integers(-50, 50, (5, 30)).astype(np.float32)
+    bi = rng.integers(-50, 50, 30).astype(np.float32)
+    assert np.array_equal(o.rsign_pm1(xi + 7, bi + 7, axis=1), o.rsign_pm1(xi, bi, axis=1))
+    x4 = rng.standard_normal((2, 3, 4, 5)).astype(np.float32)
+    b4 = rng.standard_normal(3).astype(np.float32)
+    r4 = o.rsign_pm1(x4, b4, axis=1)
+    for n in range(2):
+        for c in range(3):
+            for h in range(4):
+                for w in range(5):
+                    assert r4[n, c, h, w] == (-1 if x4[n, c, h, w] < b4[c] else 1)
+
+
 ALL_CHECKS = [
     ("identity_bruteforce", lambda o, g: check_identity_bruteforce(o)),
     ("elementwise_xnor_form", lambda o, g: check_elementwise_xnor_form(o)),
@@ -414,6 +448,7 @@ ALL_CHECKS = [
     ("ternary_examples", check_ternary_examples),
     ("ternary_quantizer", lambda o, g: check_ternary_quantizer(o)),
     ("ternary_product", lambda o, g: check_ternary_product(o)),
+    ("rsign", check_rsign),
 ]
 
 
