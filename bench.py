@@ -581,6 +581,9 @@ def _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk):
     ms_pack = timed(lambda i: bnn.bnn_pack_sign_nchw(Xd[i % R], Xb[i % R]))
     pbytes = Xd[0].numel() * 2 + Xb[0].numel() * 4
     pack_gbs = pbytes * steps / (ms_pack * 1e-3) / 1e9
+    rbeta = torch.linspace(-0.5, 0.5, c, device=dev)       # a per-channel threshold (RSign)
+    ms_rs = timed(lambda i: bnn.bnn_pack_sign_nchw_rsign(Xd[i % R], rbeta, Xb[i % R]))
+    rs_gbs = (pbytes + c * 4) * steps / (ms_rs * 1e-3) / 1e9
     for name, engine in (("conv3x3", bnn.BNN_GEMM_ENGINE_AUTO), ("conv3x3_tensor", bnn.BNN_GEMM_ENGINE_TENSOR),
                          ("conv3x3_popcount", bnn.BNN_GEMM_ENGINE_POPCOUNT)):
         with bnn.gemm_engine(engine):
@@ -612,6 +615,8 @@ def _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk):
             "pack_nchw": {"ms": ms_pack / steps, "achieved_gbs": round(pack_gbs, 1),
                           "frac": round(pack_gbs / pk["hbm_gbs"], 4), "bytes": pbytes,
                           "traffic": recorded_traffic("pack_sign_nchw_kernel")},
+            "pack_nchw_rsign": {"ms": ms_rs / steps, "achieved_gbs": round(rs_gbs, 1),
+                                "frac": round(rs_gbs / pk["hbm_gbs"], 4), "bytes": pbytes + c * 4},
             "l2": f"{R} rotating input/output sets, {rot_mb:.0f} MB"}
     del cv, Xd, Xb, Wc, alc, gam, bet, out
     torch.cuda.empty_cache()

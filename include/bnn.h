@@ -159,6 +159,24 @@ bnn_status bnn_pack_sign(const void* x, bnn_dtype dt, int64_t rows, int64_t K, i
 bnn_status bnn_pack_sign_nchw(const void* x, bnn_dtype dt, int64_t n, int64_t c, int64_t h,
                               int64_t w, uint32_t* packed_nhwc, bnn_stream_t stream);
 
+/* bnn_pack_sign_rsign, bnn_pack_sign_nchw_rsign -- bnn_pack_sign (without
+ * alpha) and bnn_pack_sign_nchw with a learned threshold per channel:
+ * bit = 1 (-1) exactly where x < beta_c, i.e. sign(x - beta_c) with the
+ * Notation tie rule (x = beta_c gives +1; NaN in x or beta gives +1).
+ *   Passage: "State of the Art Survey (2016 -> 2026)", classic CNN BNN table,
+ *   ReActNet row (RSign: a per-channel reshape of the activation
+ *   distribution before binarisation); the pages give no formula, this
+ *   reading is sign(x - beta_c).
+ *   beta     device fp32, required: [K] per column for bnn_pack_sign_rsign
+ *            (the channels of a [rows, K] activation matrix), [c] per channel
+ *            for bnn_pack_sign_nchw_rsign.  4-byte aligned.
+ *   Other arguments, layouts and errors as bnn_pack_sign / bnn_pack_sign_nchw;
+ *   INVALID_ARG for a NULL beta.  Pad bits and padded channels stay 0 (+1). */
+bnn_status bnn_pack_sign_rsign(const void* x, bnn_dtype dt, int64_t rows, int64_t K, int64_t ld_x,
+                               const float* beta, uint32_t* packed, int64_t ld_words, bnn_stream_t stream);
+bnn_status bnn_pack_sign_nchw_rsign(const void* x, bnn_dtype dt, int64_t n, int64_t c, int64_t h, int64_t w,
+                                    const float* beta, uint32_t* packed_nhwc, bnn_stream_t stream);
+
 /* bnn_pack_conv3x3_weights -- pack OIHW 3x3 filters into rows of K = 9 * cin
  * elements in (kh, kw, c) order, and compute alpha per output channel.
  *   Passage: eq. (1) and the glossary's "scaling factors for each weight

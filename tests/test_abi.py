@@ -220,3 +220,14 @@ def test_ternary_gemv_rejects_bad_arguments():
     assert f(FAKE, 4, FAKE, 8, 32, NULL, NULL, ctypes.c_void_p(0x10002), NULL, 0, NULL) == bnn.BNN_ERR_ALIGNMENT
     assert f(FAKE, 6148, FAKE, 8, 98305, NULL, NULL, FAKE, NULL, 0, NULL) == bnn.BNN_ERR_UNSUPPORTED
     assert f(FAKE, 4, FAKE, 0, 32, NULL, NULL, FAKE, NULL, 7, NULL) == bnn.BNN_OK                # N = 0
+
+
+def test_rsign_packs_reject_bad_arguments():
+    f, g = L.bnn_pack_sign_rsign, L.bnn_pack_sign_nchw_rsign
+    assert f(FAKE, 0, 8, 32, 32, NULL, FAKE, 4, NULL) == bnn.BNN_ERR_INVALID_ARG               # beta required
+    assert f(FAKE, 0, 8, 32, 32, ctypes.c_void_p(0x10002), FAKE, 4, NULL) == bnn.BNN_ERR_ALIGNMENT
+    assert f(FAKE, 0, 8, 32, 31, FAKE, FAKE, 4, NULL) == bnn.BNN_ERR_INVALID_ARG               # ld_x < K
+    assert f(FAKE, 0, 0, 32, 32, FAKE, FAKE, 4, NULL) == bnn.BNN_OK                            # rows = 0
+    assert g(FAKE, 0, 2, 64, 5, 5, NULL, FAKE, NULL) == bnn.BNN_ERR_INVALID_ARG                # beta required
+    assert g(FAKE, 0, 2, 64, 5, 5, ctypes.c_void_p(0x10002), FAKE, NULL) == bnn.BNN_ERR_ALIGNMENT
+    assert g(FAKE, 0, 0, 64, 5, 5, FAKE, FAKE, NULL) == bnn.BNN_OK                             # n = 0

@@ -123,3 +123,66 @@ def test_pack_conv3x3_weights(cout, cin, dtype):
     assert np.array_equal(u32(packed), expected_conv_weights(wt))
     a_ref = oracle.alpha(wt.float().reshape(cout, -1))
     assert np.all(np.abs(alpha.cpu().numpy() - a_ref) <= 1e-6 * a_ref)
+
+
+# ---------------------------------------------------------------------------
+# per-channel threshold (RSign): sign(x - beta_c)
+# ---------------------------------------------------------------------------
+
+def _beta(n, seed):
+    b = workloads.normal((n,), 0.5, seed)
+    b[:3] = torch.tensor([0.0, float("inf"), -float("inf")])[: min(3, n)]
+    return b
+
+
+@pytest.mark.parametrize("rows,K", [(1, 1), (7, 33), (64, 1000), (300, 4096), (5, 4100)])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_pack_sign_rsign_rows(rows, K, dtype):
+    d = dev()
+    x = workloads.normal((rows, K), 1.0, rows + 3 * K).to(dtype)
+    x[0, : min(K, 4)] = torch.tensor([0.0, -0.0, float("nan"), 1.0])[: min(K, 4)].to(dtype)
+    beta = _beta(K, K + 5)
+    if K > 4:
+        x[0, 4] = beta[4].to(dtype)                                   # a tie where bf16 holds beta exactly or not
+    packed = torch.full((rows, bnn.bnn_packed_ld_words(K)), -1, dtype=torch.int32, device=d)
+    bnn.bnn_pack_sign_rsign(x.to(d), beta.to(d), packed)
+    torch.cuda.synchronize()
+    want = oracle.pack_pm1(oracle.rsign_pm1(x, beta, axis=1))
+    assert np.array_equal(u32(packed), want)
+    assert_no_device_error()
+
+
+@pytest.mark.parametrize("shape", [(2, 64, 56, 56), (3, 40, 7, 9), (1, 130, 5, 5), (2, 32, 1, 1)])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_pack_sign_nchw_rsign(shape, dtype):
+    d = dev()
+    n, c, h, w = shape
+    x = workloads.normal(shape, 1.0, n * c + h * w).to(dtype)
+    beta = _beta(c, c + 11)
+    x[0, 3, 0, 0] = beta[3].to(dtype)
+    packed = bnn.empty_packed_nhwc(n, c, h, w, d)
+    bnn.bnn_pack_sign_nchw_rsign(x.to(d), beta.to(d), packed)
+    torch.cuda.synchronize()
+    cw = (c + 31) // 32
+    r = oracle.rsign_pm1(x, beta, axis=1)                               # [n, c, h, w]
+    want = oracle.pack_pm1(np.ascontiguousarray(r.transpose(0, 2, 3, 1)).reshape(-1, c))[:, :cw]
+    assert np.array_equal(u32(packed).reshape(-1, cw), want)
+    assert_no_device_error()
+
+
+def test_pack_sign_rsign_zero_threshold_is_sign():
+    """beta = 0 gives exactly bnn_pack_sign's bits (both layouts)."""
+    d = dev()
+    x = workloads.normal((4, 64, 9, 9), 1.0, 77).to(d)
+    a = bnn.empty_packed_nhwc(4, 64, 9, 9, d)
+    b = bnn.empty_packed_nhwc(4, 64, 9, 9, d)
+    bnn.bnn_pack_sign_nchw(x, a)
+    bnn.bnn_pack_sign_nchw_rsign(x, torch.zeros(64, device=d), b)
+    m = x.reshape(36, -1)
+    pa = bnn.empty_packed(36, m.shape[1], d)
+    pb = bnn.empty_packed(36, m.shape[1], d)
+    bnn.bnn_pack_sign(m, pa)
+    bnn.bnn_pack_sign_rsign(m, torch.zeros(m.shape[1], device=d), pb)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(pa, pb)
+    assert_no_device_error()

@@ -49,7 +49,7 @@ EXPORTS = (
     "bnn_xnor_gemv", "bnn_xnor_gemv_ex", "bnn_binary_linear_fused", "bnn_binary_conv3x3_fused",
     "bnn_fold_bn_threshold", "bnn_set_gemm_engine", "bnn_get_gemm_engine", "bnn_selftest_wait_timeout",
     "bnn_binary_weight_gemv", "bnn_ternary_ld_words", "bnn_ternary_workspace_bytes", "bnn_ternary_pack",
-    "bnn_ternary_gemv_i8", "bnn_ternary_pack_noalloc",
+    "bnn_ternary_gemv_i8", "bnn_ternary_pack_noalloc", "bnn_pack_sign_rsign", "bnn_pack_sign_nchw_rsign",
 )
 
 
@@ -96,6 +96,8 @@ def _load() -> ctypes.CDLL:
         "bnn_ternary_pack": (i32, [p, i32, i64, i64, i64, ctypes.c_double, p, i64, p, p, i64, p]),
         "bnn_ternary_gemv_i8": (i32, [p, i64, p, i64, i64, p, p, p, p, ctypes.c_uint32, p]),
         "bnn_ternary_pack_noalloc": (i32, [p, i32, i64, i64, i64, ctypes.c_double, p, i64, p, p]),
+        "bnn_pack_sign_rsign": (i32, [p, i32, i64, i64, i64, p, p, i64, p]),
+        "bnn_pack_sign_nchw_rsign": (i32, [p, i32, i64, i64, i64, i64, p, p, p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -220,6 +222,27 @@ def bnn_pack_sign_nchw(x: torch.Tensor, packed_nhwc: torch.Tensor, stream=None) 
     _check("bnn_pack_sign_nchw", _lib.bnn_pack_sign_nchw(
         _ptr(x), _dtype(x), n, c, h, w, _ptr(packed_nhwc), _stream(stream)))
 
+
+
+def bnn_pack_sign_rsign(x: torch.Tensor, beta: torch.Tensor, packed: torch.Tensor, K: Optional[int] = None,
+                        stream=None) -> None:
+    """x [rows, K] -> packed bits of sign(x - beta_k), beta fp32 [K] per column."""
+    if x.dim() == 1:
+        x = x[None, :]
+    assert x.stride(-1) == 1 and packed.stride(-1) == 1 and beta.dtype == torch.float32
+    rows, Kx = x.shape
+    K = Kx if K is None else int(K)
+    _check("bnn_pack_sign_rsign", _lib.bnn_pack_sign_rsign(
+        _ptr(x), _dtype(x), rows, K, _ld(x), _ptr(beta), _ptr(packed),
+        _ld(packed) if packed.dim() >= 2 else packed.shape[-1], _stream(stream)))
+
+
+def bnn_pack_sign_nchw_rsign(x: torch.Tensor, beta: torch.Tensor, packed_nhwc: torch.Tensor, stream=None) -> None:
+    """NCHW x -> per-pixel channel words of sign(x - beta_c), beta fp32 [c]."""
+    assert x.is_contiguous() and packed_nhwc.is_contiguous() and beta.dtype == torch.float32
+    n, c, h, w = x.shape
+    _check("bnn_pack_sign_nchw_rsign", _lib.bnn_pack_sign_nchw_rsign(
+        _ptr(x), _dtype(x), n, c, h, w, _ptr(beta), _ptr(packed_nhwc), _stream(stream)))
 
 def bnn_pack_conv3x3_weights(w_oihw: torch.Tensor, packed: torch.Tensor,
                              alpha_out: Optional[torch.Tensor] = None, stream=None) -> None:

@@ -364,8 +364,10 @@ bnn_status bnn_selftest_wait_timeout(int64_t timeout_ns, int32_t* waited_out) {
     return BNN_OK;
 }
 
-bnn_status bnn_pack_sign(const void* x, bnn_dtype dt, int64_t rows, int64_t K, int64_t ld_x, uint32_t* packed,
-                         int64_t ld_words, float* alpha_out, bnn_stream_t stream) {
+namespace {
+
+bnn_status pack_sign_rows(const void* x, bnn_dtype dt, int64_t rows, int64_t K, int64_t ld_x, const float* beta,
+                          uint32_t* packed, int64_t ld_words, float* alpha_out, bnn_stream_t stream) {
     if (x == nullptr || packed == nullptr) return BNN_ERR_INVALID_ARG;
     if (rows < 0 || K < 1 || ld_x < K) return BNN_ERR_INVALID_ARG;
     if (dt != BNN_F32 && dt != BNN_BF16) return BNN_ERR_INVALID_ARG;
@@ -374,27 +376,38 @@ bnn_status bnn_pack_sign(const void* x, bnn_dtype dt, int64_t rows, int64_t K, i
     if ((ld_words & 3) != 0 || !aligned(packed, 16)) return BNN_ERR_ALIGNMENT;
     const size_t es = dt == BNN_F32 ? 4 : 2;
     if (!aligned(x, es) || (alpha_out != nullptr && !aligned(alpha_out, 4))) return BNN_ERR_ALIGNMENT;
+    if (beta != nullptr && !aligned(beta, 4)) return BNN_ERR_ALIGNMENT;
     if (rows == 0) return BNN_OK;
     const bool vec_ok = aligned(x, 16) && ((ld_x * (int64_t)es) % 16 == 0);
     const int64_t blocks = ceil_div(rows, 8);
     if (blocks > INT_MAX) return BNN_ERR_INVALID_ARG;
     cudaStream_t s = as_cuda(stream);
-    if (dt == BNN_F32)
-        bnn::pack_sign_rows_kernel<float, 4><<<(unsigned)blocks, 256, 0, s>>>(
-            static_cast<const float*>(x), rows, K, ld_x, packed, ld_words, alpha_out, kw, vec_ok);
+    const float* xf = static_cast<const float*>(x);
+    const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+    const unsigned g = (unsigned)blocks;
+    if (dt == BNN_F32 && beta == nullptr)
+        bnn::pack_sign_rows_kernel<float, 4, false><<<g, 256, 0, s>>>(xf, rows, K, ld_x, packed, ld_words, alpha_out,
+                                                                      kw, vec_ok, beta);
+    else if (dt == BNN_F32)
+        bnn::pack_sign_rows_kernel<float, 4, true><<<g, 256, 0, s>>>(xf, rows, K, ld_x, packed, ld_words, alpha_out,
+                                                                     kw, vec_ok, beta);
+    else if (beta == nullptr)
+        bnn::pack_sign_rows_kernel<__nv_bfloat16, 4, false><<<g, 256, 0, s>>>(xb, rows, K, ld_x, packed, ld_words,
+                                                                              alpha_out, kw, vec_ok, beta);
     else
-        bnn::pack_sign_rows_kernel<__nv_bfloat16, 4><<<(unsigned)blocks, 256, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(x), rows, K, ld_x, packed, ld_words, alpha_out, kw, vec_ok);
+        bnn::pack_sign_rows_kernel<__nv_bfloat16, 4, true><<<g, 256, 0, s>>>(xb, rows, K, ld_x, packed, ld_words,
+                                                                             alpha_out, kw, vec_ok, beta);
     return launch_status();
 }
 
-bnn_status bnn_pack_sign_nchw(const void* x, bnn_dtype dt, int64_t n, int64_t c, int64_t h, int64_t w,
-                              uint32_t* packed_nhwc, bnn_stream_t stream) {
+bnn_status pack_sign_nchw(const void* x, bnn_dtype dt, int64_t n, int64_t c, int64_t h, int64_t w, const float* beta,
+                          uint32_t* packed_nhwc, bnn_stream_t stream) {
     if (x == nullptr || packed_nhwc == nullptr) return BNN_ERR_INVALID_ARG;
     if (n < 0 || c < 1 || h < 1 || w < 1) return BNN_ERR_INVALID_ARG;
     if (dt != BNN_F32 && dt != BNN_BF16) return BNN_ERR_INVALID_ARG;
     const size_t es = dt == BNN_F32 ? 4 : 2;
     if (!aligned(x, es) || !aligned(packed_nhwc, 4)) return BNN_ERR_ALIGNMENT;
+    if (beta != nullptr && !aligned(beta, 4)) return BNN_ERR_ALIGNMENT;
     if (n == 0) return BNN_OK;
     const int64_t hw = h * w, cw = (c + 31) / 32;
     cudaStream_t s = as_cuda(stream);
@@ -402,13 +415,42 @@ bnn_status bnn_pack_sign_nchw(const void* x, bnn_dtype dt, int64_t n, int64_t c,
     const int64_t blocks = ceil_div(warps, 8);
     if (blocks > INT_MAX) return BNN_ERR_INVALID_ARG;
     const bool vec_ok = aligned(x, 16) && (hw % (int64_t)(16 / es) == 0);
-    if (dt == BNN_F32)
-        bnn::pack_sign_nchw_kernel<float><<<(unsigned)blocks, 256, 0, s>>>(static_cast<const float*>(x), n, c, hw,
-                                                                           cw, packed_nhwc, vec_ok);
+    const float* xf = static_cast<const float*>(x);
+    const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+    const unsigned g = (unsigned)blocks;
+    if (dt == BNN_F32 && beta == nullptr)
+        bnn::pack_sign_nchw_kernel<float, false><<<g, 256, 0, s>>>(xf, n, c, hw, cw, packed_nhwc, vec_ok, beta);
+    else if (dt == BNN_F32)
+        bnn::pack_sign_nchw_kernel<float, true><<<g, 256, 0, s>>>(xf, n, c, hw, cw, packed_nhwc, vec_ok, beta);
+    else if (beta == nullptr)
+        bnn::pack_sign_nchw_kernel<__nv_bfloat16, false><<<g, 256, 0, s>>>(xb, n, c, hw, cw, packed_nhwc, vec_ok, beta);
     else
-        bnn::pack_sign_nchw_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(x), n, c, hw, cw, packed_nhwc, vec_ok);
+        bnn::pack_sign_nchw_kernel<__nv_bfloat16, true><<<g, 256, 0, s>>>(xb, n, c, hw, cw, packed_nhwc, vec_ok, beta);
     return launch_status();
+}
+
+}  // namespace
+
+bnn_status bnn_pack_sign(const void* x, bnn_dtype dt, int64_t rows, int64_t K, int64_t ld_x, uint32_t* packed,
+                         int64_t ld_words, float* alpha_out, bnn_stream_t stream) {
+    return pack_sign_rows(x, dt, rows, K, ld_x, nullptr, packed, ld_words, alpha_out, stream);
+}
+
+bnn_status bnn_pack_sign_rsign(const void* x, bnn_dtype dt, int64_t rows, int64_t K, int64_t ld_x, const float* beta,
+                               uint32_t* packed, int64_t ld_words, bnn_stream_t stream) {
+    if (beta == nullptr) return BNN_ERR_INVALID_ARG;
+    return pack_sign_rows(x, dt, rows, K, ld_x, beta, packed, ld_words, nullptr, stream);
+}
+
+bnn_status bnn_pack_sign_nchw_rsign(const void* x, bnn_dtype dt, int64_t n, int64_t c, int64_t h, int64_t w,
+                                    const float* beta, uint32_t* packed_nhwc, bnn_stream_t stream) {
+    if (beta == nullptr) return BNN_ERR_INVALID_ARG;
+    return pack_sign_nchw(x, dt, n, c, h, w, beta, packed_nhwc, stream);
+}
+
+bnn_status bnn_pack_sign_nchw(const void* x, bnn_dtype dt, int64_t n, int64_t c, int64_t h, int64_t w,
+                              uint32_t* packed_nhwc, bnn_stream_t stream) {
+    return pack_sign_nchw(x, dt, n, c, h, w, nullptr, packed_nhwc, stream);
 }
 
 bnn_status bnn_pack_conv3x3_weights(const void* w_oihw, bnn_dtype dt, int64_t cout, int64_t cin,

@@ -18,11 +18,16 @@ namespace bnn {
 // 16-byte vector; a warp-wide load covers 32*E elements = E words.  Lane l's
 // E sign bits land at bit E*(l % G) of word l / G (G = 32/E lanes per word);
 // an OR-butterfly over those G lanes assembles the word.
-template <typename T, int U>
+//
+// RS: a per-column threshold beta (fp32 [K]), bit = (x < beta_k), i.e.
+// sign(x - beta_k) (RSign, "State of the Art Survey (2016 -> 2026)", ReActNet
+// row); columns past K use -inf, so their bits stay 0 (+1).  Without RS the
+// threshold is 0 (the Notation sign) and beta is not read.
+template <typename T, int U, bool RS>
 __global__ void __launch_bounds__(256)
 pack_sign_rows_kernel(const T* __restrict__ x, int64_t rows, int64_t K, int64_t ld_x,
                       uint32_t* __restrict__ packed, int64_t ldp, float* __restrict__ alpha_out,
-                      int64_t kw, bool vec_ok) {
+                      int64_t kw, bool vec_ok, const float* __restrict__ beta) {
     constexpr int E = 16 / (int)sizeof(T);
     constexpr int G = 32 / E;
     constexpr int CH = 32 * E;  // elements per warp chunk
@@ -55,10 +60,20 @@ pack_sign_rows_kernel(const T* __restrict__ x, int64_t rows, int64_t K, int64_t 
             const int64_t chunk = c0 + u;
             if (chunk >= nchunks) break;
             uint32_t bits = 0;
-            #pragma unroll
-            for (int i = 0; i < E; ++i) {
-                bits |= neg_bit(v[u][i]) << i;
-                asum += fabs((double)v[u][i]);  // elements past K were loaded as 0
+            if constexpr (!RS) {
+                #pragma unroll
+                for (int i = 0; i < E; ++i) {
+                    bits |= neg_bit(v[u][i]) << i;
+                    asum += fabs((double)v[u][i]);  // elements past K were loaded as 0
+                }
+            } else {
+                const int64_t base = chunk * CH + (int64_t)lane * E;
+                #pragma unroll
+                for (int i = 0; i < E; ++i) {
+                    const float b = base + i < K ? __ldg(beta + base + i) : -INFINITY;
+                    bits |= (v[u][i] < b ? 1u : 0u) << i;
+                    asum += fabs((double)v[u][i]);
+                }
             }
             bits <<= E * (lane % G);
             #pragma unroll
@@ -96,10 +111,12 @@ __device__ __forceinline__ float vec_elem(const uint32_t (&w)[4], int p) {
 // 128 contiguous bytes, so every load instruction is 4 full lines.  Each lane
 // sets bits 8q .. 8q+7 of its E pixels' words; two shuffles OR the four
 // quarters together, and lane q stores the pixels p = q (mod 4).
-template <typename T>
+// RS: per-channel threshold beta (fp32 [c]), bit = (x < beta_c) (RSign, as in
+// pack_sign_rows_kernel); channels past c use -inf.
+template <typename T, bool RS>
 __global__ void __launch_bounds__(256)
 pack_sign_nchw_kernel(const T* __restrict__ x, int64_t n, int64_t c, int64_t hw, int64_t cw,
-                      uint32_t* __restrict__ out, bool vec_ok) {
+                      uint32_t* __restrict__ out, bool vec_ok, const float* __restrict__ beta) {
     constexpr int E = 16 / (int)sizeof(T);
     constexpr int PX = 8 * E;                     // pixels per task
     const int lane = threadIdx.x & 31;
@@ -156,12 +173,25 @@ pack_sign_nchw_kernel(const T* __restrict__ x, int64_t n, int64_t c, int64_t hw,
         }
     }
     uint32_t bits[E];
-    #pragma unroll
-    for (int p = 0; p < E; ++p) {
-        uint32_t w = 0;
+    if constexpr (RS) {
+        float th[8];
         #pragma unroll
-        for (int i = 0; i < 8; ++i) w |= neg_bit(vec_elem<T>(v[i], p)) << i;
-        bits[p] = w << (8 * q);
+        for (int i = 0; i < 8; ++i) th[i] = i < nc ? __ldg(beta + ch0 + i) : -INFINITY;
+        #pragma unroll
+        for (int p = 0; p < E; ++p) {
+            uint32_t w = 0;
+            #pragma unroll
+            for (int i = 0; i < 8; ++i) w |= (vec_elem<T>(v[i], p) < th[i] ? 1u : 0u) << i;
+            bits[p] = w << (8 * q);
+        }
+    } else {
+        #pragma unroll
+        for (int p = 0; p < E; ++p) {
+            uint32_t w = 0;
+            #pragma unroll
+            for (int i = 0; i < 8; ++i) w |= neg_bit(vec_elem<T>(v[i], p)) << i;
+            bits[p] = w << (8 * q);
+        }
     }
     #pragma unroll
     for (int p = 0; p < E; ++p) {
