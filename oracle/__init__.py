@@ -353,8 +353,16 @@ def binary_linear(x_real, w_real):
     return matmul_pm1(a, wb), alpha(w_real)
 
 
+def conv_affine(x_real, w_real, gamma, beta, stride: int = 1, pad: int = 1):
+    """Binary convolution (any square kernel in w_real [cout, cin, k, k]) with
+    per-output-channel alpha over the filter's cin*k*k weights and an affine
+    epilogue.  Returns (s int32 NCHW, y float64 NCHW)."""
+    return conv3x3_affine(x_real, w_real, gamma, beta, stride, pad)
+
+
 def conv3x3_affine(x_real, w_real, gamma, beta, stride: int = 1, pad: int = 1):
-    """Binary 3x3 convolution with per-output-channel alpha and an affine epilogue.
+    """Binary 3x3 convolution with per-output-channel alpha and an affine epilogue
+    (the code holds for any square kernel size).
 
     Returns (s int32 NCHW, y float64 NCHW)."""
     xb = sign_pm1(x_real)

@@ -210,6 +210,12 @@ def check_conv_library(o, seed=0):
         ref = F.conv2d(xt, torch.from_numpy(f.astype(np.float64)), stride=stride)
         got = o.conv2d_pm1(x, f, stride, pad)
         assert np.array_equal(got, ref.numpy().astype(np.int32)), (n, c, h, w, co, stride, pad)
+    # 1x1 kernels with stride (the downsampling projection), no padding
+    for (n, c, h, w, co, stride) in [(2, 40, 9, 7, 5, 2), (1, 64, 8, 8, 3, 2), (2, 3, 5, 5, 4, 1), (1, 7, 6, 6, 2, 3)]:
+        x = rng.choice(np.array([-1, 1], np.int8), size=(n, c, h, w))
+        f = rng.choice(np.array([-1, 1], np.int8), size=(co, c, 1, 1))
+        ref = F.conv2d(torch.from_numpy(x.astype(np.float64)), torch.from_numpy(f.astype(np.float64)), stride=stride)
+        assert np.array_equal(o.conv2d_pm1(x, f, stride, 0), ref.numpy().astype(np.int32)), (n, c, h, w, co, stride)
     # closed form: all +1 input and filters give 9*c everywhere, padding included
     x = np.ones((1, 5, 4, 4), np.int8)
     f = np.ones((2, 5, 3, 3), np.int8)
