@@ -115,6 +115,7 @@ KERNEL_SOURCES = {
     "pack_sign_nchw_kernel": ("pack.cuh", "common.cuh"),
     "bw_gemv_kernel": ("bwgemv.cuh", "common.cuh"),
     "ternary_gemv_i8_kernel": ("ternary.cuh", "common.cuh"),
+    "xnor_conv1x1_kernel": ("conv1x1.cuh", "conv.cuh", "gemm_popc.cuh", "common.cuh"),
     "pack_ternary_kernel": ("ternary.cuh", "common.cuh"),
 }
 
@@ -451,7 +452,7 @@ def e2e_gemv(torch, bnn, g, Ws, alpha, dev, steps, sync, max_over_ranks, ws):
 # the other rows
 # ---------------------------------------------------------------------------
 
-ROW_NAMES = ("pack_sign_weights", "square_gemm", "conv3x3", "mlp4", "bw_gemv", "ternary")
+ROW_NAMES = ("pack_sign_weights", "square_gemm", "conv3x3", "mlp4", "bw_gemv", "ternary", "conv1x1")
 
 
 def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws, only=None):
@@ -478,6 +479,8 @@ def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws, o
         _row_bw_gemv(torch, bnn, workloads, dev, pk, rows, timed, ws)
     if "ternary" in want:
         _row_ternary(torch, bnn, workloads, dev, pk, rows, timed, steps, ws)
+    if "conv1x1" in want:
+        _row_conv1x1(torch, bnn, workloads, dev, pk, rows, timed, steps, ws, alu_peak)
     if bnn.bnn_device_error() != 0:
         raise RuntimeError("a kernel reported a device-side timeout")
     return rows
@@ -701,6 +704,44 @@ def _row_ternary(torch, bnn, workloads, dev, pk, rows, timed, steps, ws):
                      "frac": round(ach_p / pk["hbm_gbs"], 4), "algorithmic_bytes": pb,
                      "traffic": recorded_traffic("pack_ternary_kernel")}}
     del Qs, ys, codes, x, g, wsp
+    torch.cuda.empty_cache()
+
+
+
+def _row_conv1x1(torch, bnn, workloads, dev, pk, rows, timed, steps, ws, alu_peak):
+    # --- next row: binary 1x1 stride-2 downsampling projection (ResNet block) ---
+    cv = workloads.downsample()
+    n, c, h, w = cv.X.shape
+    cout = cv.W.shape[0]
+    oh, ow = (h - 1) // 2 + 1, (w - 1) // 2 + 1
+    # Four rotating (packed input, fp32 output) sets, 109 MB, larger than L2 together.
+    R = 4
+    Xd = cv.X.to(dev)
+    Xb = [bnn.empty_packed_nhwc(n, c, h, w, dev) for _ in range(R)]
+    for i in range(R):
+        bnn.bnn_pack_sign_nchw(Xd, Xb[i])
+    Wp = bnn.empty_packed(cout, c, dev)
+    al = torch.empty(cout, dtype=torch.float32, device=dev)
+    bnn.bnn_pack_sign(cv.W.reshape(cout, c).to(dev), Wp, al)
+    gam, bet = cv.gamma.to(dev), cv.beta.to(dev)
+    ep = bnn.make_epilogue(bnn.BNN_OUT_AFFINE_F32, alpha=al, gamma=gam, beta=bet)
+    out = [torch.empty(n, cout, oh, ow, dtype=torch.float32, device=dev) for _ in range(R)]
+    ms = timed(lambda i: bnn.bnn_binary_conv1x1_fused(Xb[i % R], c, Wp, ep, out[i % R], stride=2))
+    cw = (c + 31) // 32
+    # Algorithmic bytes: the strided input pixels, the filters and the fp32 output.
+    b = n * oh * ow * cw * 4 + Wp.numel() * 4 + out[0].numel() * 4
+    ach = b * steps / (ms * 1e-3) / 1e9
+    macs = n * oh * ow * cout * c
+    rows["conv1x1"] = {
+        "workload": "binary 1x1 stride-2 projection: packed [64,56,56,2 words] x 128 filters -> "
+                    "alpha + affine fp32 NCHW [64,128,28,28]",
+        "value": round(ws * ach, 1), "unit": "GB/s", "ms_per_step": ms / steps,
+        "binary_tmac_s": round(macs * steps / (ms * 1e-3) / 1e12, 2),
+        "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"],
+                     "frac": round(ach / pk["hbm_gbs"], 4), "algorithmic_bytes": b,
+                     "traffic": recorded_traffic("xnor_conv1x1_kernel")},
+        "l2": f"{R} rotating packed-input/output sets"}
+    del cv, Xd, Xb, Wp, al, gam, bet, out
     torch.cuda.empty_cache()
 
 

@@ -438,6 +438,24 @@ bnn_status bnn_binary_conv3x3_fused(const uint32_t* X_nhwc_bits, int64_t n, int6
                                     int64_t stride, int64_t pad, const bnn_epilogue* ep,
                                     void* out_nchw, bnn_stream_t stream);
 
+/* bnn_binary_conv1x1_fused -- binary 1x1 convolution with stride (the
+ * downsampling projection of a ResNet-class block), fused epilogue.  Output
+ * pixel (n, y, x) reads input pixel (n, s*y, s*x); no padding.  K = c.
+ *   Passage: eq. (4), eq. (6), eq. (1) per filter of "Extreme Quantization
+ *   ..."; the glossary's BatchNorm paragraph for the affine epilogue.
+ *   X_nhwc_bits device, from bnn_pack_sign_nchw (or its RSign variant):
+ *            [n, h, w, ceil(c/32)] words.
+ *   W_packed device, [cout, ldw] words, ldw >= ceil(c/32): the filters
+ *            [cout, c, 1, 1] packed as rows of c elements, e.g. by
+ *            bnn_pack_sign on the [cout, c] view (which also gives alpha).
+ *   stride >= 1; output spatial size (h - 1)/stride + 1 by (w - 1)/stride + 1.
+ *   ep       host pointer; modes INT32, SCALED_F32, AFFINE_F32.
+ *   out_nchw device int32/fp32 [n, cout, oh, ow] contiguous.
+ *   Supports c <= 512.  Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED. */
+bnn_status bnn_binary_conv1x1_fused(const uint32_t* X_nhwc_bits, int64_t n, int64_t c, int64_t h, int64_t w,
+                                    const uint32_t* W_packed, int64_t ldw, int64_t cout, int64_t stride,
+                                    const bnn_epilogue* ep, void* out_nchw, bnn_stream_t stream);
+
 /* bnn_fold_bn_threshold -- HOST function: fold inference BatchNorm of
  * alpha * s followed by sign() into an integer popcount threshold per channel.
  *   Passage: glossary "Binary Neural Network (BNN)", BatchNorm paragraph (BN

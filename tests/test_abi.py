@@ -231,3 +231,18 @@ def test_rsign_packs_reject_bad_arguments():
     assert g(FAKE, 0, 2, 64, 5, 5, NULL, FAKE, NULL) == bnn.BNN_ERR_INVALID_ARG                # beta required
     assert g(FAKE, 0, 2, 64, 5, 5, ctypes.c_void_p(0x10002), FAKE, NULL) == bnn.BNN_ERR_ALIGNMENT
     assert g(FAKE, 0, 0, 64, 5, 5, FAKE, FAKE, NULL) == bnn.BNN_OK                             # n = 0
+
+
+def test_conv1x1_rejects_bad_arguments():
+    f = L.bnn_binary_conv1x1_fused
+    ep = bnn.make_epilogue(bnn.BNN_OUT_INT32)
+    epb = ctypes.byref(ep)
+    assert f(NULL, 2, 64, 8, 8, FAKE, 4, 16, 2, epb, FAKE, NULL) == bnn.BNN_ERR_INVALID_ARG     # no input
+    assert f(FAKE, 2, 64, 8, 8, FAKE, 4, 16, 0, epb, FAKE, NULL) == bnn.BNN_ERR_INVALID_ARG     # stride 0
+    assert f(FAKE, 2, 64, 8, 8, FAKE, 1, 16, 2, epb, FAKE, NULL) == bnn.BNN_ERR_INVALID_ARG     # ldw < cw
+    assert f(FAKE, 2, 600, 8, 8, FAKE, 20, 16, 2, epb, FAKE, NULL) == bnn.BNN_ERR_UNSUPPORTED   # c > 512
+    thr = bnn.make_epilogue(bnn.BNN_OUT_THRESHOLD_PACK)
+    assert f(FAKE, 2, 64, 8, 8, FAKE, 4, 16, 2, ctypes.byref(thr), FAKE, NULL) == bnn.BNN_ERR_UNSUPPORTED
+    sc = bnn.make_epilogue(bnn.BNN_OUT_SCALED_F32)
+    assert f(FAKE, 2, 64, 8, 8, FAKE, 4, 16, 2, ctypes.byref(sc), FAKE, NULL) == bnn.BNN_ERR_INVALID_ARG  # no alpha
+    assert f(FAKE, 0, 64, 8, 8, FAKE, 4, 16, 2, epb, FAKE, NULL) == bnn.BNN_OK                   # n = 0

@@ -19,6 +19,9 @@ fully binary MLP):
 * ``square`` A, W fp32 [8192, 8192] N(0, 1), seeds 4 and 5.
 * ``conv``   X bf16 [64, 64, 56, 56] N(0, 1) seed 6; W fp32 [64, 64, 3, 3]
              N(0, 0.1) seed 7; gamma U(0.5, 1.5), beta N(0, 0.1) [64] seed 8.
+* ``downsample`` X bf16 [64, 64, 56, 56] N(0, 1) seed 6 (the conv input); W fp32
+             [128, 64, 1, 1] N(0, 0.1) seed 18; gamma U(0.5, 1.5), beta N(0, 0.1)
+             [128] seed 19 (1x1 stride-2 projection to 128 channels).
 * ``ternary`` W fp32 [11008, 4096] N(0, 0.02) seed 2 (the decode weights, to be
              ternarised); x int8 [4096] uniform over [-128, 127] seed 17.
 * ``mlp``    X0 fp32 [4096, 4096] N(0, 1) seed 9; W_l fp32 [4096, 4096] N(0, 1)
@@ -102,6 +105,16 @@ def gemv(N=11008, K=4096, w_seed=2, x_seed=3, x_dtype=torch.bfloat16) -> Gemv:
     W = normal((N, K), 0.02, w_seed)
     x = normal((K,), 1.0, x_seed, dtype=x_dtype)
     return Gemv(N, K, W, x)
+
+
+def downsample(n=64, c=64, h=56, w=56, cout=128, x_seed=6, w_seed=18, bn_seed=19, stride=2,
+               x_dtype=torch.bfloat16) -> Conv:
+    X = normal((n, c, h, w), 1.0, x_seed, dtype=x_dtype)
+    W = normal((cout, c, 1, 1), 0.1, w_seed)
+    g = _gen(bn_seed)
+    gamma = torch.rand(cout, generator=g).add_(0.5)
+    beta = torch.randn(cout, generator=g).mul_(0.1)
+    return Conv(X, W, gamma, beta, stride, 0)
 
 
 @dataclass

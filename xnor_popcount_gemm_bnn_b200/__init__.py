@@ -50,6 +50,7 @@ EXPORTS = (
     "bnn_fold_bn_threshold", "bnn_set_gemm_engine", "bnn_get_gemm_engine", "bnn_selftest_wait_timeout",
     "bnn_binary_weight_gemv", "bnn_ternary_ld_words", "bnn_ternary_workspace_bytes", "bnn_ternary_pack",
     "bnn_ternary_gemv_i8", "bnn_ternary_pack_noalloc", "bnn_pack_sign_rsign", "bnn_pack_sign_nchw_rsign",
+    "bnn_binary_conv1x1_fused",
 )
 
 
@@ -98,6 +99,8 @@ def _load() -> ctypes.CDLL:
         "bnn_ternary_pack_noalloc": (i32, [p, i32, i64, i64, i64, ctypes.c_double, p, i64, p, p]),
         "bnn_pack_sign_rsign": (i32, [p, i32, i64, i64, i64, p, p, i64, p]),
         "bnn_pack_sign_nchw_rsign": (i32, [p, i32, i64, i64, i64, i64, p, p, p]),
+        "bnn_binary_conv1x1_fused": (i32, [p, i64, i64, i64, i64, p, i64, i64, i64,
+                                           ctypes.POINTER(bnn_epilogue), p, p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -382,6 +385,16 @@ def bnn_binary_conv3x3_fused(X_bits: torch.Tensor, c: int, W_packed: torch.Tenso
         _ptr(X_bits), n, int(c), h, w, _ptr(W_packed), _ld(W_packed), cout, int(stride), int(pad),
         ctypes.byref(ep), _ptr(out_nchw), _stream(stream)))
 
+
+
+def bnn_binary_conv1x1_fused(X_bits: torch.Tensor, c: int, W_packed: torch.Tensor, ep: bnn_epilogue,
+                             out_nchw: torch.Tensor, stride: int = 2, stream=None) -> None:
+    """Binary 1x1 convolution (stride, no padding) of packed NHWC words."""
+    n, h, w = X_bits.shape[:3]
+    cout = W_packed.shape[0]
+    _check("bnn_binary_conv1x1_fused", _lib.bnn_binary_conv1x1_fused(
+        _ptr(X_bits), n, int(c), h, w, _ptr(W_packed), _ld(W_packed), cout, int(stride), ctypes.byref(ep),
+        _ptr(out_nchw), _stream(stream)))
 
 def bnn_fold_bn_threshold(alpha: torch.Tensor, gamma: torch.Tensor, beta: torch.Tensor,
                           mean: torch.Tensor, var: torch.Tensor, eps: float, K: int):

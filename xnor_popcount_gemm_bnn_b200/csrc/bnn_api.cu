@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "conv.cuh"
 #include "conv_tc.cuh"
+#include "conv1x1.cuh"
 #include "gemm_popc.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
@@ -884,6 +885,77 @@ bnn_status bnn_binary_conv3x3_fused(const uint32_t* X_nhwc_bits, int64_t n, int6
     }
 #undef BNN_CONV_CASE
     return launch_status();
+}
+
+bnn_status bnn_binary_conv1x1_fused(const uint32_t* X_nhwc_bits, int64_t n, int64_t c, int64_t h, int64_t w,
+                                    const uint32_t* W_packed, int64_t ldw, int64_t cout, int64_t stride,
+                                    const bnn_epilogue* epi, void* out_nchw, bnn_stream_t stream) {
+    if (X_nhwc_bits == nullptr || W_packed == nullptr || epi == nullptr || out_nchw == nullptr)
+        return BNN_ERR_INVALID_ARG;
+    if (n < 0 || c < 1 || h < 1 || w < 1 || cout < 0 || stride < 1) return BNN_ERR_INVALID_ARG;
+    if (h > INT_MAX / 4 || w > INT_MAX / 4 || c > INT_MAX / 16 || cout > INT_MAX || stride > 1024)
+        return BNN_ERR_INVALID_ARG;
+    const int64_t oh = (h - 1) / stride + 1, ow = (w - 1) / stride + 1;
+    const int64_t cw = (c + 31) / 32;
+    if (ldw < cw) return BNN_ERR_INVALID_ARG;
+    switch (epi->mode) {
+        case BNN_OUT_INT32: break;
+        case BNN_OUT_SCALED_F32:
+            if (epi->alpha == nullptr) return BNN_ERR_INVALID_ARG;
+            break;
+        case BNN_OUT_AFFINE_F32:
+            if (epi->alpha == nullptr || epi->gamma == nullptr || epi->beta == nullptr) return BNN_ERR_INVALID_ARG;
+            break;
+        case BNN_OUT_THRESHOLD_PACK: return BNN_ERR_UNSUPPORTED;
+        default: return BNN_ERR_INVALID_ARG;
+    }
+    if (!aligned(X_nhwc_bits, 4) || !aligned(W_packed, 4) || !aligned(out_nchw, 4)) return BNN_ERR_ALIGNMENT;
+    if (cw > 16) return BNN_ERR_UNSUPPORTED;
+    // The kernel instance's word capacity (1, 2, 4, 8, 16) fixes the filter
+    // row stride in shared memory: bnn::xnor_conv1x1_kernel<cwp> uses
+    // (cwp + 3) / 4 * 4 words per row.
+    const int cwp = cw == 1 ? 1 : cw == 2 ? 2 : cw <= 4 ? 4 : cw <= 8 ? 8 : 16;
+    const int64_t kwp = (cwp + 3) / 4 * 4;
+    const size_t smem = (size_t)cout * kwp * 4 + (size_t)cout * 2 * 4;   // filters + gamma*alpha, beta
+    if (smem > 200 * 1024) return BNN_ERR_UNSUPPORTED;
+    if (n == 0 || cout == 0) return BNN_OK;
+    const int64_t npix = n * oh * ow;
+    bnn::ConvEpilogue ep{epi->mode, epi->alpha, epi->gamma, epi->beta, out_nchw};
+    if (npix > INT_MAX - 4096 || cout * oh * ow > INT_MAX) return BNN_ERR_UNSUPPORTED;   // 32-bit pixel indices
+    // One contiguous run of (pixel block, filter) units per warp: 4 CTAs per
+    // SM, fewer when there are fewer than about 16 units per warp.
+    const int64_t units = ceil_div(npix, (int64_t)(32 * bnn::c1x1::pixels_per_lane(cwp))) * cout;
+    const int64_t blocks = std::max<int64_t>(
+        1, std::min<int64_t>(ceil_div(units, (int64_t)bnn::conv::WARPS * 16),
+                             (int64_t)sm_count() * bnn::conv::CTAS_PER_SM));
+    cudaStream_t s = as_cuda(stream);
+    auto launch = [&](auto kern) -> bnn_status {
+        if (smem > 48 * 1024 &&
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return BNN_ERR_CUDA;
+        kern<<<(unsigned)blocks, bnn::conv::THREADS, smem, s>>>(X_nhwc_bits, (int)n, (int)c, (int)h, (int)w, W_packed,
+                                                                ldw, (int)cout, (int)stride, (int)oh, (int)ow, ep);
+        return launch_status();
+    };
+    auto by_mode = [&](auto k_int, auto k_scaled, auto k_affine) -> bnn_status {
+        if (epi->mode == BNN_OUT_INT32) return launch(k_int);
+        if (epi->mode == BNN_OUT_SCALED_F32) return launch(k_scaled);
+        return launch(k_affine);
+    };
+#define BNN_C1_CASE(CWV)                                                                                      \
+    case CWV:                                                                                                 \
+        return by_mode(bnn::xnor_conv1x1_kernel<CWV, BNN_OUT_INT32>, bnn::xnor_conv1x1_kernel<CWV, BNN_OUT_SCALED_F32>, \
+                       bnn::xnor_conv1x1_kernel<CWV, BNN_OUT_AFFINE_F32>);
+    switch (cwp) {
+        BNN_C1_CASE(1)
+        BNN_C1_CASE(2)
+        BNN_C1_CASE(4)
+        BNN_C1_CASE(8)
+        default: return by_mode(bnn::xnor_conv1x1_kernel<16, BNN_OUT_INT32>,
+                                bnn::xnor_conv1x1_kernel<16, BNN_OUT_SCALED_F32>,
+                                bnn::xnor_conv1x1_kernel<16, BNN_OUT_AFFINE_F32>);
+    }
+#undef BNN_C1_CASE
 }
 
 }  // extern "C"
