@@ -22,6 +22,9 @@ real-valued epilogues evaluated in float64 here with numpy:
   over the matrix); "First Principles ...", the op-per-element table
   (ternary: add / skip / sub), with int8 activations (the BitNet section:
   activations quantised to INT8).
+* multi-bit products -- "State of the Art Survey ...", classic CNN BNN table:
+  DoReFa-Net bit planes (unsigned k-bit codes, the integer product) and
+  ABC-Net binary bases (a weighted sum of +1/-1 products).
 * BatchNorm before re-binarisation -- "Binary Neural Network (BNN)" glossary
   page, the BatchNorm paragraph (BN stabilises the inputs to each binarised
   layer; per-filter alpha multiplies the binary product).  The pages give no
@@ -288,6 +291,52 @@ def ternary_gemv_i8(t: np.ndarray, x_q, w_scale: float = 1.0, x_scale: float = 1
     acc = ternary_product(t, x_q)
     return acc, float(w_scale) * float(x_scale) * acc.astype(np.float64)
 
+
+
+# ---------------------------------------------------------------------------
+# multi-bit products: bit planes (DoReFa-Net) and binary bases (ABC-Net)
+# ---------------------------------------------------------------------------
+
+def bit_planes(x_u, k: int) -> np.ndarray:
+    """uint8 [k, *shape]: plane b holds bit b of the unsigned k-bit codes
+    x_u (0 <= x < 2^k), so x = sum_b 2^b * plane_b ("State of the Art Survey
+    (2016 -> 2026)", classic CNN BNN table, DoReFa-Net: low-bit weights and
+    activations, bit-convolution)."""
+    x = np.asarray(x_u, dtype=np.int64)
+    assert k >= 1 and x.min(initial=0) >= 0 and x.max(initial=0) < (1 << k)
+    return np.stack([(x >> b) & 1 for b in range(k)]).astype(np.uint8)
+
+
+def bitserial_product(a_u, w_u) -> np.ndarray:
+    """int64 [M, N]: sum_k a[m, k] * w[n, k] for unsigned integer codes
+    a [M, K] and w [N, K] -- the product a bit-serial kernel computes as
+    sum over plane pairs (b, b') of 2^(b+b') * popcount(a_b AND w_b')
+    (DoReFa-Net's bit-convolution, same table).  Written as the plain sum of
+    products."""
+    a = np.asarray(a_u, dtype=np.int64)
+    w = np.asarray(w_u, dtype=np.int64)
+    return (a[:, None, :] * w[None, :, :]).sum(axis=2)
+
+
+def binary_bases_product(h_pm1, b_pm1, alpha, beta) -> np.ndarray:
+    """float64 [M, N]: sum_j sum_i beta_j * alpha_i[n] * (H_j B_i^T)[m, n]
+    for activations approximated by J binary bases, A ~ sum_j beta_j H_j
+    (H_j in {-1, +1}^[M, K]), and weights by I bases, W ~ sum_i alpha_i B_i
+    (B_i in {-1, +1}^[N, K], alpha_i per output channel) ("State of the Art
+    Survey ...", classic CNN BNN table, ABC-Net: approximate full precision
+    with K binary bases).  Each H_j B_i^T is a +1/-1 product (eq. (6))."""
+    h = np.asarray(h_pm1, dtype=np.int8)
+    b = np.asarray(b_pm1, dtype=np.int8)
+    al = np.asarray(alpha, dtype=np.float64)
+    be = np.asarray(beta, dtype=np.float64).reshape(-1)
+    J, M, K = h.shape
+    I, N, K2 = b.shape
+    assert K == K2 and al.shape == (I, N) and be.shape == (J,)
+    y = np.zeros((M, N), dtype=np.float64)
+    for j in range(J):
+        for i in range(I):
+            y += be[j] * al[i][None, :] * matmul_pm1(h[j], b[i]).astype(np.float64)
+    return y
 
 def conv2d_pm1(x: np.ndarray, f: np.ndarray, stride: int = 1, pad: int = 1) -> np.ndarray:
     """int32 NCHW output of a square-kernel convolution on +1/-1 tensors,

@@ -230,7 +230,39 @@ def _rsign_last_axis(x, beta, axis=-1):         # threshold applied along the la
         return np.where(xf - b < 0.0, -1, 1).astype(np.int8)
 
 
+
+def _planes_msb(x_u, k):                        # plane 0 holds the top bit
+    x = np.asarray(x_u, np.int64)
+    return np.stack([(x >> (k - 1 - b)) & 1 for b in range(k)]).astype(np.uint8)
+
+
+def _bitserial_unweighted(a_u, w_u):            # plane pairs added without 2^(b+b')
+    a = np.asarray(a_u, np.int64)
+    w = np.asarray(w_u, np.int64)
+    ka = max(1, int(a.max()).bit_length())
+    kw = max(1, int(w.max()).bit_length())
+    out = np.zeros((a.shape[0], w.shape[0]), np.int64)
+    for b1 in range(ka):
+        for b2 in range(kw):
+            out += (((a >> b1) & 1)[:, None, :] * ((w >> b2) & 1)[None, :, :]).sum(axis=2)
+    return out
+
+
+def _bases_diagonal_only(h_pm1, b_pm1, alpha, beta):    # only the i == j cross terms
+    h = np.asarray(h_pm1, np.int8)
+    b = np.asarray(b_pm1, np.int8)
+    al = np.asarray(alpha, np.float64)
+    be = np.asarray(beta, np.float64).reshape(-1)
+    y = np.zeros((h.shape[1], b.shape[1]))
+    for j in range(min(h.shape[0], b.shape[0])):
+        y += be[j] * al[j][None, :] * oracle.matmul_pm1(h[j], b[j]).astype(np.float64)
+    return y
+
+
 MUTANTS = {
+    "planes_msb_first": dict(bit_planes=_planes_msb),
+    "bitserial_unweighted_planes": dict(bitserial_product=_bitserial_unweighted),
+    "bases_diagonal_only": dict(binary_bases_product=_bases_diagonal_only),
     "rsign_tie_negative": dict(rsign_pm1=_rsign_tie_negative),
     "rsign_reversed": dict(rsign_pm1=_rsign_reversed),
     "rsign_wrong_axis": dict(rsign_pm1=_rsign_last_axis),

@@ -435,6 +435,55 @@ def check_rsign(o, golden):
                     assert r4[n, c, h, w] == (-1 if x4[n, c, h, w] < b4[c] else 1)
 
 
+
+def check_multibit(o):
+    """Bit planes and the two multi-bit products of the survey's DoReFa-Net and
+    ABC-Net rows: plane reconstruction and a hand example; the integer product
+    against brute force and against the bit-serial identity
+    sum 2^(b+b') popcount(a_b AND w_b') evaluated on Python integers; the
+    all-ones closed form; the binary-bases product against brute force, its
+    single-basis case (the +1/-1 product) and bilinearity in the scales."""
+    assert o.bit_planes(np.array([5, 0, 7]), 3).tolist() == [[1, 0, 1], [0, 0, 1], [1, 0, 1]]
+    rng = np.random.default_rng(41)
+    x = rng.integers(0, 16, (3, 7))
+    pl = o.bit_planes(x, 4)
+    assert np.array_equal(sum((1 << bb) * pl[bb].astype(np.int64) for bb in range(4)), x)
+    for ka, kw, M, N, K in [(1, 1, 3, 4, 9), (2, 3, 4, 3, 33), (4, 2, 2, 5, 70), (8, 8, 2, 2, 40)]:
+        a = rng.integers(0, 1 << ka, (M, K))
+        w = rng.integers(0, 1 << kw, (N, K))
+        got = o.bitserial_product(a, w)
+        for m in range(M):
+            for n in range(N):
+                ref = 0
+                for k in range(K):
+                    ref += int(a[m, k]) * int(w[n, k])
+                assert int(got[m, n]) == ref
+                bits = 0
+                for b1 in range(ka):
+                    for b2 in range(kw):
+                        am = sum(((int(a[m, k]) >> b1) & 1) << k for k in range(K))
+                        wm = sum(((int(w[n, k]) >> b2) & 1) << k for k in range(K))
+                        bits += (1 << (b1 + b2)) * (am & wm).bit_count()
+                assert bits == ref
+    assert np.all(o.bitserial_product(np.full((2, 10), 7), np.full((3, 10), 3)) == 7 * 3 * 10)
+    J, I, M, N, K = 2, 3, 3, 4, 21
+    h = np.where(rng.random((J, M, K)) < 0.5, -1, 1).astype(np.int8)
+    b = np.where(rng.random((I, N, K)) < 0.5, -1, 1).astype(np.int8)
+    al = rng.uniform(0.1, 1.0, (I, N))
+    be = rng.uniform(0.1, 1.0, J)
+    got = o.binary_bases_product(h, b, al, be)
+    for m in range(M):
+        for n in range(N):
+            ref = 0.0
+            for j in range(J):
+                for i in range(I):
+                    ref += be[j] * al[i, n] * sum(int(h[j, m, k]) * int(b[i, n, k]) for k in range(K))
+            assert abs(got[m, n] - ref) <= 1e-12 * (1 + abs(ref))
+    one = o.binary_bases_product(h[:1], b[:1], np.ones((1, N)), np.ones(1))
+    assert np.array_equal(one, o.matmul_pm1(h[0], b[0]).astype(np.float64))
+    assert np.allclose(o.binary_bases_product(h, b, 2 * al, 3 * be), 6 * got, rtol=1e-14, atol=0)
+
+
 ALL_CHECKS = [
     ("identity_bruteforce", lambda o, g: check_identity_bruteforce(o)),
     ("elementwise_xnor_form", lambda o, g: check_elementwise_xnor_form(o)),
@@ -455,6 +504,7 @@ ALL_CHECKS = [
     ("ternary_quantizer", lambda o, g: check_ternary_quantizer(o)),
     ("ternary_product", lambda o, g: check_ternary_product(o)),
     ("rsign", check_rsign),
+    ("multibit", lambda o, g: check_multibit(o)),
 ]
 
 
