@@ -451,7 +451,8 @@ bnn_status bnn_binary_conv3x3_fused(const uint32_t* X_nhwc_bits, int64_t n, int6
  *   stride >= 1; output spatial size (h - 1)/stride + 1 by (w - 1)/stride + 1.
  *   ep       host pointer; modes INT32, SCALED_F32, AFFINE_F32.
  *   out_nchw device int32/fp32 [n, cout, oh, ow] contiguous.
- *   Supports c <= 512.  Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED. */
+ *   Supports c <= 512, n*oh*ow < 2^31 - 4096 and cout*oh*ow < 2^31 (32-bit
+ *   pixel indices).  Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED. */
 bnn_status bnn_binary_conv1x1_fused(const uint32_t* X_nhwc_bits, int64_t n, int64_t c, int64_t h, int64_t w,
                                     const uint32_t* W_packed, int64_t ldw, int64_t cout, int64_t stride,
                                     const bnn_epilogue* ep, void* out_nchw, bnn_stream_t stream);
