@@ -246,3 +246,10 @@ def test_conv1x1_rejects_bad_arguments():
     sc = bnn.make_epilogue(bnn.BNN_OUT_SCALED_F32)
     assert f(FAKE, 2, 64, 8, 8, FAKE, 4, 16, 2, ctypes.byref(sc), FAKE, NULL) == bnn.BNN_ERR_INVALID_ARG  # no alpha
     assert f(FAKE, 0, 64, 8, 8, FAKE, 4, 16, 2, epb, FAKE, NULL) == bnn.BNN_OK                   # n = 0
+
+
+def test_conv1x1_rejects_indices_past_32_bits():
+    """n*oh*ow at or past 2^31 - 4096 is refused before any launch."""
+    ep = bnn.make_epilogue(bnn.BNN_OUT_INT32)
+    st = L.bnn_binary_conv1x1_fused(FAKE, 1 << 22, 64, 64, 64, FAKE, 4, 16, 2, ctypes.byref(ep), FAKE, NULL)
+    assert st == bnn.BNN_ERR_UNSUPPORTED
