@@ -30,3 +30,28 @@ def test_rejects_short_warmup():
     r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "1"],
                        cwd=ROOT, capture_output=True, text=True, timeout=300)
     assert r.returncode != 0 and "warmup" in r.stderr
+
+
+def test_failing_row_is_reported_not_fatal():
+    """A row that raises is recorded as an error in the rows object; the
+    other rows and the headline line still come out."""
+    import types
+
+    import torch
+
+    import bench
+    import workloads
+
+    class Boom(RuntimeError):
+        pass
+
+    def fail(*a, **k):
+        raise Boom("planted failure")
+
+    fake = types.SimpleNamespace(empty_packed=fail, bnn_device_error=lambda: 0)
+    args = types.SimpleNamespace(row_steps=3, warmup=3)
+    pk = {"sm_max_mhz": 1965.0, "hbm_gbs": 6513.5}
+    rows = bench.bench_rows(torch, fake, workloads, torch.device("cpu"), pk, args, lambda: None, lambda v: v, 1,
+                            only=["pack_sign_weights"])
+    assert list(rows) == ["pack_sign_weights"]
+    assert rows["pack_sign_weights"]["error"].startswith("Boom: planted failure")
