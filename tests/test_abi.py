@@ -253,3 +253,17 @@ def test_conv1x1_rejects_indices_past_32_bits():
     ep = bnn.make_epilogue(bnn.BNN_OUT_INT32)
     st = L.bnn_binary_conv1x1_fused(FAKE, 1 << 22, 64, 64, 64, FAKE, 4, 16, 2, ctypes.byref(ep), FAKE, NULL)
     assert st == bnn.BNN_ERR_UNSUPPORTED
+
+
+def test_header_constants_match_binding():
+    """Numeric constants of include/bnn.h (enums, #defines) equal the binding's."""
+    text = open(HEADER).read()
+    m = re.search(r"#define\s+BNN_TERNARY_PACK_NOALLOC_MAX_ROWS\s+(\d+)", text)
+    assert m and int(m.group(1)) == bnn.BNN_TERNARY_PACK_NOALLOC_MAX_ROWS
+    for name in ("BNN_GEMV_WEIGHTS_STATIC", "BNN_GEMV_INPUTS_STATIC", "BNN_GEMV_OUTPUT_FREE", "BNN_OUT_INT32",
+                 "BNN_OUT_SCALED_F32", "BNN_OUT_AFFINE_F32", "BNN_OUT_THRESHOLD_PACK", "BNN_GEMM_ENGINE_AUTO",
+                 "BNN_GEMM_ENGINE_POPCOUNT", "BNN_GEMM_ENGINE_TENSOR", "BNN_F32", "BNN_BF16",
+                 "BNN_ERR_DEVICE_TIMEOUT"):
+        m = re.search(rf"\b{name}\s*=\s*(\d+)", text)
+        assert m, name
+        assert int(m.group(1)) == getattr(bnn, name), name
