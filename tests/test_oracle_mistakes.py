@@ -259,7 +259,44 @@ def _bases_diagonal_only(h_pm1, b_pm1, alpha, beta):    # only the i == j cross 
     return y
 
 
+
+def _affine_no_beta(s, alpha_n, gamma, beta):     # beta dropped
+    return np.asarray(gamma, np.float64) * (np.asarray(alpha_n, np.float64) * np.asarray(s, np.float64))
+
+
+def _scaled_row_axis(s, alpha_n):                 # alpha applied along rows
+    s = np.asarray(s, np.float64)
+    a = np.asarray(alpha_n, np.float64)
+    return a.reshape(-1, 1)[: s.shape[0]] * s if a.size >= s.shape[0] else s * 0
+
+
+def _conv_affine_center_alpha(x_real, w_real, gamma, beta, stride=1, pad=1):   # alpha from the centre tap only
+    xb = oracle.sign_pm1(x_real)
+    fb = oracle.sign_pm1(w_real)
+    wf = oracle._f32(w_real).astype(np.float64)
+    k = wf.shape[2]
+    a = np.abs(wf[:, :, k // 2, k // 2]).mean(axis=1)
+    s = oracle.conv2d_pm1(xb, fb, stride, pad)
+    y = oracle.affine(np.moveaxis(s, 1, -1), a, gamma, beta)
+    return s, np.moveaxis(y, -1, 1)
+
+
+def _binary_linear_alpha_from_x(x_real, w_real):  # alpha taken from the activations
+    s, _ = oracle.binary_linear(x_real, w_real)
+    return s, np.abs(np.atleast_2d(oracle._f32(x_real)).astype(np.float64)).mean()
+
+
+def _bw_gemv_no_alpha(w_real, x_real):            # alpha left out of y
+    a = oracle.alpha(w_real)
+    return a, oracle.binary_weight_product(oracle.sign_pm1(w_real), oracle._f32(x_real))
+
+
 MUTANTS = {
+    "affine_without_beta": dict(affine=_affine_no_beta),
+    "scaled_on_row_axis": dict(scaled=_scaled_row_axis),
+    "conv_alpha_centre_tap": dict(conv_affine=_conv_affine_center_alpha),
+    "linear_alpha_from_activations": dict(binary_linear=_binary_linear_alpha_from_x),
+    "bw_gemv_without_alpha": dict(binary_weight_gemv=_bw_gemv_no_alpha),
     "planes_msb_first": dict(bit_planes=_planes_msb),
     "bitserial_unweighted_planes": dict(bitserial_product=_bitserial_unweighted),
     "bases_diagonal_only": dict(binary_bases_product=_bases_diagonal_only),

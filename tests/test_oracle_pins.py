@@ -484,6 +484,53 @@ def check_multibit(o):
     assert np.allclose(o.binary_bases_product(h, b, 2 * al, 3 * be), 6 * got, rtol=1e-14, atol=0)
 
 
+
+def check_compositions(o):
+    """The layer-level compositions the GPU tests compare against: alpha*s and
+    gamma*(alpha*s) + beta by hand values (alpha on the channel axis), the
+    XNOR-Net linear layer, the convolution with its affine epilogue (3x3 and
+    1x1 strided) and the binary-weight GEMV against torch float64, and alpha
+    rounded once to fp32."""
+    assert o.scaled(np.array([[3, -5, 0]]), np.array([0.5, 2.0, 7.0])).tolist() == [[1.5, -10.0, 0.0]]
+    assert o.scaled(np.array([[1, 1, 1], [2, 2, 2]]), np.array([1.0, 2.0, 3.0])).tolist() == [[1, 2, 3], [2, 4, 6]]
+    assert o.affine(np.array([[4, -2]]), np.array([0.25, 0.5]), np.array([2.0, -1.0]),
+                    np.array([-1.0, 0.5])).tolist() == [[1.0, 1.5]]
+    rng = np.random.default_rng(51)
+
+    def tsign(t):
+        return torch.where(t >= 0, 1.0, -1.0).to(torch.float64)
+
+    x = rng.standard_normal((6, 70)).astype(np.float32)
+    w = rng.standard_normal((9, 70)).astype(np.float32)
+    s, a = o.binary_linear(x, w)
+    xt, wt = torch.from_numpy(x), torch.from_numpy(w)
+    assert np.array_equal(s, (tsign(xt) @ tsign(wt).T).numpy().astype(np.int32))
+    assert np.allclose(a, wt.double().abs().mean(dim=1).numpy(), rtol=1e-15, atol=0)
+    af = o.alpha_f32(w)
+    assert af.dtype == np.float32
+    assert np.all(np.abs(af.astype(np.float64) - a) <= np.spacing(af).astype(np.float64) / 2)
+    for (n, c, h, wd, co, k, stride, pad) in [(2, 5, 7, 6, 4, 3, 1, 1), (1, 40, 9, 8, 3, 1, 2, 0), (2, 3, 6, 6, 2, 3, 2, 1)]:
+        X = rng.standard_normal((n, c, h, wd)).astype(np.float32)
+        Wc = rng.standard_normal((co, c, k, k)).astype(np.float32)
+        g = rng.uniform(0.5, 1.5, co)
+        b = rng.standard_normal(co) * 0.1
+        s_c, y_c = o.conv_affine(X, Wc, g, b, stride, pad)
+        xp = F.pad(tsign(torch.from_numpy(X)), (pad, pad, pad, pad), value=1.0)
+        s_ref = F.conv2d(xp, tsign(torch.from_numpy(Wc)), stride=stride)
+        a_ref = torch.from_numpy(Wc).double().abs().mean(dim=(1, 2, 3))
+        y_ref = torch.from_numpy(g)[None, :, None, None] * (a_ref[None, :, None, None] * s_ref) \
+            + torch.from_numpy(b)[None, :, None, None]
+        assert np.array_equal(s_c, s_ref.numpy().astype(np.int32))
+        assert np.allclose(y_c, y_ref.numpy(), rtol=1e-13, atol=1e-13)
+        if k == 3:
+            assert np.array_equal(o.conv3x3_affine(X, Wc, g, b, stride, pad)[1], y_c)
+    xv = rng.standard_normal(70).astype(np.float32)
+    a_bw, y_bw = o.binary_weight_gemv(w, xv)
+    y_t = wt.double().abs().mean(dim=1) * (tsign(wt) @ torch.from_numpy(xv).double())
+    assert np.allclose(a_bw, a, rtol=0, atol=0)
+    assert np.allclose(y_bw, y_t.numpy(), rtol=1e-13, atol=1e-13 * np.abs(xv).sum())
+
+
 ALL_CHECKS = [
     ("identity_bruteforce", lambda o, g: check_identity_bruteforce(o)),
     ("elementwise_xnor_form", lambda o, g: check_elementwise_xnor_form(o)),
@@ -505,6 +552,7 @@ ALL_CHECKS = [
     ("ternary_product", lambda o, g: check_ternary_product(o)),
     ("rsign", check_rsign),
     ("multibit", lambda o, g: check_multibit(o)),
+    ("compositions", lambda o, g: check_compositions(o)),
 ]
 
 
