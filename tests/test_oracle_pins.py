@@ -495,6 +495,8 @@ def check_compositions(o):
     assert o.scaled(np.array([[1, 1, 1], [2, 2, 2]]), np.array([1.0, 2.0, 3.0])).tolist() == [[1, 2, 3], [2, 4, 6]]
     assert o.affine(np.array([[4, -2]]), np.array([0.25, 0.5]), np.array([2.0, -1.0]),
                     np.array([-1.0, 0.5])).tolist() == [[1.0, 1.5]]
+    # sign then pack: negatives at 0 and 4 (-0.0 is +1) -> bits 0 and 4
+    assert o.pack_real(np.array([[-1.0, 0.0, 2.0, -0.0, -3.0]], np.float32)).tolist() == [[17, 0, 0, 0]]
     rng = np.random.default_rng(51)
 
     def tsign(t):
