@@ -40,7 +40,8 @@ def test_llm_decode_workload():
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("N,K", [(1, 1), (7, 31), (33, 100), (1000, 1000), (300, 4095),
-                                 (257, 4097), (130, 8192), (64, 12345), (5, 129), (100, 576)])
+                                 (257, 4097), (130, 8192), (64, 12345), (5, 129), (100, 576),
+                                 (300, 2100), (301, 2400), (77, 3100)])
 def test_ragged_shapes(N, K, dtype):
     W = workloads.normal((N, K), 0.02, N + K)
     x = workloads.random_with_edges(1, K, seed=K, dtype=dtype)[0]
@@ -48,6 +49,30 @@ def test_ragged_shapes(N, K, dtype):
     s_ref, y_ref = reference(W, x)
     assert np.array_equal(y_i.cpu().numpy(), s_ref)
     assert_scaled_close(y_f, y_ref)
+
+
+@pytest.mark.parametrize("flags", [0, 1, 3, 7])
+@pytest.mark.parametrize("K", [2100, 2400, 3100, 4096])
+def test_row128_kernel_every_block_shape(K, flags):
+    """The one-chunk-per-lane kernel takes rows of 68..128 words; with bf16 x
+    its pack covers 4 vectors per word, so kw * 4 vectors need not fill whole
+    warps (K = 2100, 2400, 3100).  Every dependency mode (each has its own
+    block shape) must give the exact product there."""
+    N = 1234
+    d = dev()
+    W = workloads.normal((N, K), 0.02, 3 * K + flags)
+    x = workloads.random_with_edges(1, K, seed=K + 1, dtype=torch.bfloat16)[0]
+    W_p = bnn.empty_packed(N, K, d)
+    alpha = torch.empty(N, dtype=torch.float32, device=d)
+    bnn.bnn_pack_sign(W.to(d), W_p, alpha)
+    y_i = torch.empty(N, dtype=torch.int32, device=d)
+    y_f = torch.empty(N, dtype=torch.float32, device=d)
+    bnn.bnn_xnor_gemv_ex(W_p, x.to(d), K, alpha, y_i, y_f, flags=flags)
+    torch.cuda.synchronize()
+    s_ref, y_ref = reference(W, x)
+    assert np.array_equal(y_i.cpu().numpy(), s_ref)
+    assert_scaled_close(y_f, y_ref)
+    assert_no_device_error()
 
 
 def test_int32_only_and_f32_only():

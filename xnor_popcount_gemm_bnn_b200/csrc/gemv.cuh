@@ -98,7 +98,7 @@ __device__ __forceinline__ void gemv_pack_x(const XT* __restrict__ x, int K, int
     }
 }
 
-// Fast path for rows of 97..128 words (LPR = 32, one 16-byte chunk per lane,
+// Fast path for rows of 68..128 words (LPR = 32, one 16-byte chunk per lane,
 // K <= 4096) and a 16-byte aligned x: each lane owns one chunk of U rows, the
 // x pack is one vector per thread per round (E elements; 32/E lanes OR their
 // bits into a word).  Measured about 20% shorter steps than the generic
@@ -132,21 +132,26 @@ xnor_gemv_row128_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* _
     };
     auto pack_x = [&]() {
         const int nfull = K / E;                      // whole vectors inside x
-        for (int c = threadIdx.x; c < kw * (32 / E); c += THREADS) {   // vectors covering the padded row
+        const int nvec = kw * (32 / E);               // vectors covering the padded row
+        // The trip count is block-uniform (c0 steps over whole blocks), so
+        // every lane of a warp reaches the full-mask shuffle together even
+        // when nvec is not a multiple of 32; lanes past nvec carry zeros.
+        for (int c0 = 0; c0 < nvec; c0 += THREADS) {
+            const int c = c0 + (int)threadIdx.x;
             uint4 q = make_uint4(0u, 0u, 0u, 0u);
             if (c < nfull) q = *reinterpret_cast<const uint4*>(x + E * c);
             const XT* e = reinterpret_cast<const XT*>(&q);
             uint32_t b = 0;
             #pragma unroll
             for (int i = 0; i < E; ++i) b |= neg_bit(to_float(e[i])) << i;
-            if (c == nfull) {                         // the partial last vector, if any
+            if (c == nfull && c < nvec) {             // the partial last vector, if any
                 b = 0;
                 for (int i = 0; i < K - E * c; ++i) b |= neg_bit(to_float(x[E * c + i])) << i;
             }
             b <<= E * (c & (G - 1));
             #pragma unroll
             for (int off = 1; off < G; off <<= 1) b |= __shfl_xor_sync(0xffffffffu, b, off);
-            if ((c & (G - 1)) == 0) xs[c / G] = b;
+            if ((c & (G - 1)) == 0 && c < nvec) xs[c / G] = b;
         }
         __syncthreads();
     };
