@@ -68,8 +68,9 @@ def _lib():
         lib.oracle_matmul_pm1.argtypes = [p, p, i64, i64, i64, p]
         lib.oracle_conv2d_pm1.argtypes = [p, i64, i64, i64, i64, p, i64, i64, i64, i64, p]
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         for name in ("oracle_sign_f32", "oracle_pack_pm1", "oracle_alpha_f32",
-                     "oracle_matmul_pm1", "oracle_conv2d_pm1"):
+                     "oracle_matmul_pm1", "oracle_conv2d_pm1", "oracle_set_num_threads"):
             getattr(lib, name).restype = None
         _LIB = lib
     return _LIB
@@ -92,6 +93,11 @@ def _ptr(a: np.ndarray):
 
 def num_threads() -> int:
     return int(_lib().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads for the C loops (timing only; no result depends on it)."""
+    _lib().oracle_set_num_threads(int(n))
 
 
 def ld_words(K: int) -> int:

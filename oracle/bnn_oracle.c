@@ -5,8 +5,9 @@
  *
  * Every routine here is the plain definition, written out with +1/-1 values
  * materialised as int8 and integer multiply-accumulate.  No bit tricks, no
- * blocking, no reordering beyond an OpenMP split of the outermost loop (which
- * does not change an integer result).
+ * blocking, no reordering beyond an OpenMP split over independent outputs
+ * (each output is still one thread's plain loop over k, so the split does not
+ * change any result).
  *
  * Sources (page title, section / equation):
  *  - "Extreme Quantization: Binary, Ternary & 1-bit LLMs", Notation:
@@ -77,16 +78,17 @@ void oracle_alpha_f32(const float* w, int64_t rows, int64_t K, double* alpha) {
  * definition of w_b^T x_b (left-hand side of eq. (6)). */
 void oracle_matmul_pm1(const int8_t* a, const int8_t* w, int64_t M, int64_t N,
                        int64_t K, int32_t* s) {
-    int64_t m;
+    int64_t job;
+    /* One job per output (m, n), so that a single row (a GEMV) also spreads
+     * over the threads. */
 #pragma omp parallel for schedule(static)
-    for (m = 0; m < M; ++m) {
+    for (job = 0; job < M * N; ++job) {
+        const int64_t m = job / N, n = job % N;
         const int8_t* arow = a + m * K;
-        for (int64_t n = 0; n < N; ++n) {
-            const int8_t* wrow = w + n * K;
-            int32_t acc = 0;
-            for (int64_t k = 0; k < K; ++k) acc += (int32_t)arow[k] * (int32_t)wrow[k];
-            s[m * N + n] = acc;
-        }
+        const int8_t* wrow = w + n * K;
+        int32_t acc = 0;
+        for (int64_t k = 0; k < K; ++k) acc += (int32_t)arow[k] * (int32_t)wrow[k];
+        s[m * N + n] = acc;
     }
 }
 
@@ -122,6 +124,16 @@ void oracle_conv2d_pm1(const int8_t* x, int64_t n, int64_t c, int64_t h, int64_t
             }
         }
     }
+}
+
+/* Thread count for the OpenMP loops above (timing of the oracle on one core
+ * and on all cores); it changes no result. */
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
 }
 
 int oracle_num_threads(void) {
