@@ -30,8 +30,11 @@
  * CONVENTIONS.
  *  - Device pointers are CUDA device (or managed) memory on the current
  *    device, owned by the caller; the library keeps no pointer after a call
- *    returns and allocates no device memory (a call that needs scratch
- *    space takes a caller-owned workspace).  Host pointers are named so.
+ *    returns and allocates no device memory: a call that needs scratch space
+ *    takes a caller-owned workspace.  The one exception is
+ *    bnn_ternary_pack_noalloc, whose scratch is a fixed library-owned device
+ *    array (about 2 MiB per GPU that loads the library; see there).  Host
+ *    pointers are named so.
  *  - Every device call is asynchronous on `stream` (NULL = legacy default
  *    stream).  It returns after the launch; results are visible to later
  *    work on the same stream.
@@ -115,6 +118,27 @@ const char* bnn_status_string(int status);
  * waiting (BNN_OK if none).  Synchronises the current device first.  Writes
  * the flag value to *code_out (host pointer). */
 bnn_status bnn_device_error(int32_t* code_out);
+
+/* bnn_probe_int_pipes -- measures the integer-pipe rates that bound the
+ * popcount engine ("First Principles: Why Binary Ops Can Be Exponentially
+ * Faster", section "1. Arithmetic: MAC -> XNOR + popcount": one 32-bit XOR +
+ * popcount stands for 32 binary multiply-accumulates, so a word rate times 32
+ * is a binary MAC rate).  Runs, on the current device, one 1024-thread CTA
+ * per SM of register-only chains, timed with the SM clock, and writes (host
+ * pointers) the median over SMs of:
+ *   *popc_per_clk_sm       32-bit population counts per SM clock;
+ *   *lop3_per_clk_sm       three-input logic ops per SM clock;
+ *   *csa_words_per_clk_sm  XOR words per SM clock through the popcount GEMM's
+ *                          own inner step (XOR, 7:3 carry-save counter, 4
+ *                          POPC per 8 words).
+ * `iters` (1 .. 2^24) loop iterations per thread; each does 32 operations
+ * (words in the third mode).  Synchronous: launches on the legacy default
+ * stream and synchronises the device; a diagnostic for roofline
+ * denominators, not part of the product path.  Uses a small library-owned
+ * device array for the per-SM clock counts (no allocation).
+ * Errors: INVALID_ARG, UNSUPPORTED (more than 1024 SMs), CUDA. */
+bnn_status bnn_probe_int_pipes(int64_t iters, double* popc_per_clk_sm, double* lop3_per_clk_sm,
+                               double* csa_words_per_clk_sm);
 
 /* bnn_selftest_wait_timeout -- diagnostic for the bounded waits.  Runs one
  * kernel that waits on an mbarrier nothing arrives on, with a limit of
@@ -369,8 +393,11 @@ bnn_status bnn_ternary_pack(const void* w, bnn_dtype dt, int64_t rows, int64_t K
  *   rows > BNN_TERNARY_PACK_NOALLOC_MAX_ROWS: BNN_ERR_UNSUPPORTED (use
  *   bnn_ternary_pack with a workspace).
  *   The first call on a device looks up that array's device address (one
- *   cudaGetSymbolAddress, with the device current); make that first call
- *   before any stream capture.
+ *   cudaGetSymbolAddress, with the device current) and keeps it for the life
+ *   of the process; make that first call before any stream capture.  After
+ *   cudaDeviceReset() the array may sit at another address while the kept
+ *   one stays: do not call this entry point on a device that was reset
+ *   after its first call (use bnn_ternary_pack there).
  *   Every call on a device shares the one array.  Calls whose kernels may
  *   overlap on the GPU (on different streams without ordering between them)
  *   race on it and must not be issued; calls in stream order are safe.
@@ -475,6 +502,68 @@ bnn_status bnn_binary_conv1x1_fused(const uint32_t* X_nhwc_bits, int64_t n, int6
 bnn_status bnn_fold_bn_threshold(const float* alpha, const float* gamma, const float* beta,
                                  const float* mean, const float* var, double eps, int64_t N,
                                  int64_t K, int32_t* popc_thresh, int8_t* thresh_mode);
+
+/* ------------------------------------------------------------------------
+ * Multi-bit products on bit planes ("State of the Art Survey (2016 -> 2026)",
+ * classic CNN BNN table: DoReFa-Net -- low-bit weights and activations,
+ * bit-convolution; ABC-Net -- several binary bases approximating full
+ * precision).
+ *
+ * PLANE-INTERLEAVED LAYOUT.  An operand of R rows with P planes per row is a
+ * packed matrix (PACKED LAYOUT above) of R * P rows: plane p of row r is
+ * packed row r * P + p, at word (r * P + p) * ld.  Every plane holds K
+ * elements.  A plane of bits (DoReFa) or a +1/-1 base (ABC-Net) uses the
+ * same packed encoding as every other call.
+ * ------------------------------------------------------------------------ */
+
+/* bnn_pack_bit_planes -- unsigned k-bit codes to bit planes.
+ *   codes: device uint8 [rows, ld_codes] (ld_codes >= K); only the low `bits`
+ *   bits of each byte are used.  planes: device, plane-interleaved, `bits`
+ *   planes per row, row stride ld_words (>= bnn_packed_ld_words(K), multiple of
+ *   4, 16-byte aligned): bit j of word w of plane p of row r is bit p of
+ *   codes[r, 32 w + j]; code = sum_p 2^p * bit_p.  Elements past K are 0.
+ *   bits: 1 .. 8.
+ *   Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+bnn_status bnn_pack_bit_planes(const uint8_t* codes, int64_t rows, int64_t K, int64_t ld_codes, int bits,
+                               uint32_t* planes, int64_t ld_words, bnn_stream_t stream);
+
+/* bnn_bitserial_gemm -- the product of unsigned low-bit integer codes:
+ *   C_i32[m, n] = sum_k a[m, k] * w[n, k]      (exact, int32)
+ *   C_f32[m, n] = fp32(alpha[n] * fp32(C_i32[m, n]))
+ * for codes 0 <= a < 2^a_bits and 0 <= w < 2^w_bits given as bit planes
+ * (DoReFa-Net's bit-convolution, which a bit-serial kernel computes as
+ * sum over plane pairs of 2^(b + b') * popcount(a_b AND w_b')).  The
+ * tensor-core kernel folds each row's planes back into one unsigned byte per
+ * element in shared memory and multiplies u8 x u8, so all plane pairs cost
+ * one pass.
+ *   A: plane-interleaved [M rows x a_bits planes], row stride lda words.
+ *   W: plane-interleaved [N rows x w_bits planes], row stride ldw words.
+ *   a_bits, w_bits: 1 .. 4.  K * (2^a_bits - 1) * (2^w_bits - 1) must fit in
+ *   int32.  C_i32 (ldc >= N) and/or C_f32 (ldf >= N, needs alpha [N]); either
+ *   may be NULL, not both.
+ *   Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED, CUDA. */
+bnn_status bnn_bitserial_gemm(const uint32_t* A, int64_t lda, int a_bits, const uint32_t* W, int64_t ldw, int w_bits,
+                              int64_t M, int64_t N, int64_t K, const float* alpha, int32_t* C_i32, int64_t ldc,
+                              float* C_f32, int64_t ldf, bnn_stream_t stream);
+
+/* bnn_binary_bases_gemm -- activations approximated by J binary bases,
+ * A ~ sum_j beta_j H_j, weights by I bases per output channel,
+ * W[n] ~ sum_i alpha_i[n] B_i[n] (ABC-Net):
+ *   Y[m, n] = sum_j sum_i beta_j * alpha_i[n] * s_ji[m, n],
+ *   s_ji[m, n] = <H_j[m, :], B_i[n, :]>  (a +1/-1 product, eq. (6)),
+ * with every s_ji exact and the weighted sum in fp32.  Within a row, v_j =
+ * sum_i alpha_i[n] * s_ji is formed by fused multiply-adds in i order, then
+ * beta_j * v_j, then the J terms are added pairwise (j, j^1), (j, j^2), ...;
+ * |Y - Y_exact| <= (I + J + 2) * 2^-24 * sum_j sum_i |beta_j alpha_i[n] s_ji|.
+ *   H: plane-interleaved +1/-1 bases [M rows x J planes], stride ldh words
+ *   (base j of row m, packed as by bnn_pack_sign, at packed row m * J + j).
+ *   B: plane-interleaved [N rows x I planes], stride ldb words.
+ *   J, I: 1 .. 8.  beta: device fp32 [J]; alpha: device fp32 [I, lda_alpha]
+ *   (alpha_i[n] at i * lda_alpha + n, lda_alpha >= N); Y: device fp32 [M, ldy].
+ *   Errors: INVALID_ARG, ALIGNMENT, CUDA. */
+bnn_status bnn_binary_bases_gemm(const uint32_t* H, int64_t ldh, int J, const uint32_t* B, int64_t ldb, int I,
+                                 int64_t M, int64_t N, int64_t K, const float* beta, const float* alpha,
+                                 int64_t lda_alpha, float* Y, int64_t ldy, bnn_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -2,12 +2,16 @@
 Neural Networks, eq. (1)-(2)) against the oracle's float64 add/sub sum.
 
 Tolerance, derived from the kernel's fp32 arithmetic (u = 2^-24): a table
-entry +-x0 +-x1 +-x2 +-x3 takes 3 roundings; K is split 16 ways over the
-warps, and each of a lane's 4 accumulators adds ceil(K/256) entries in
-sequence; the 4 accumulators meet in a 2-level tree and the 16 per-warp
-partial sums are added in sequence (15 roundings); alpha*s is one
-multiplication.  So |y - y_ref| <= alpha * (ceil(K/256) + 20) * u * sum|x|
-+ 2u * |y_ref| (the second term also covers alpha rounded to fp32)."""
+entry +-x0 +-x1 +-x2 +-x3 takes 3 roundings; a lane sums the 32 groups of
+each of its P = ceil(kw/128) chunks on 4 accumulators (8P - 1 roundings
+each), the 4 meet in a 2-level tree, and the lanes of a row meet in a
+butterfly of at most 5 levels; alpha*s is one multiplication.  That is at
+most 8P + 10 roundings on the path of every term, which the bound below,
+(ceil(K/256) + 20) roundings of alpha * sum|x|, covers at every K (P = 1 for
+K <= 4096, where the bound's count is at least 21; P = 2 needs K > 4096, count
+>= 37; P = 3 needs K > 8192, count >= 53).  So |y - y_ref| <= alpha *
+(ceil(K/256) + 20) * u * sum|x| + 2u * |y_ref| (the second term also covers
+alpha rounded to fp32)."""
 import math
 
 import numpy as np

@@ -28,6 +28,13 @@ fully binary MLP):
              seeds 10..13; BatchNorm after layers 1..3 with gamma U(0.5, 1.5),
              beta N(0, 0.1), running mean N(0, 1), running var U(0.5, 2),
              seeds 14..16; eps 1e-5.
+* ``bitserial`` unsigned codes a uint8 [4096, 4096] (2 bits) seed 20 and w uint8
+             [4096, 4096] (2 bits) seed 21, uniform over [0, 2^bits): DoReFa-style
+             low-bit activations and weights at the MLP's layer shape.
+* ``bases``  J = 3 activation bases and I = 3 weight bases at the same shape: real
+             draws N(0, 1) [J, 4096, 4096] seed 22 and [I, 4096, 4096] seed 23 (their
+             signs are the bases), alpha_i[n] |N(0, 0.3)| + 0.01 seed 24, beta_j
+             |N(0, 0.5)| + 0.05 seed 25 (ABC-Net-style weighted binary bases).
 """
 from __future__ import annotations
 
@@ -181,6 +188,39 @@ def mlp(batch=4096, width=4096, layers=4, x_seed=9, w_seed0=10, bn_seed0=14) -> 
     Ws = [normal((width, width), 1.0, w_seed0 + l) for l in range(layers)]
     bns = [batchnorm_params(width, bn_seed0 + l) for l in range(layers - 1)]
     return Mlp(X0, Ws, bns)
+
+
+def codes(shape, bits: int, seed: int) -> torch.Tensor:
+    """Unsigned integer codes, uniform over [0, 2^bits), as uint8."""
+    return torch.randint(0, 1 << bits, tuple(shape), generator=_gen(seed), dtype=torch.int64).to(torch.uint8)
+
+
+@dataclass
+class Bitserial:
+    a: torch.Tensor      # uint8 [M, K], a_bits-bit codes
+    w: torch.Tensor      # uint8 [N, K], w_bits-bit codes
+    a_bits: int
+    w_bits: int
+
+
+def bitserial(M=4096, N=4096, K=4096, a_bits=2, w_bits=2, a_seed=20, w_seed=21) -> Bitserial:
+    return Bitserial(codes((M, K), a_bits, a_seed), codes((N, K), w_bits, w_seed), a_bits, w_bits)
+
+
+@dataclass
+class Bases:
+    h_real: torch.Tensor  # fp32 [J, M, K]: the activation bases are their signs
+    b_real: torch.Tensor  # fp32 [I, N, K]: the weight bases are their signs
+    alpha: torch.Tensor   # fp32 [I, N]
+    beta: torch.Tensor    # fp32 [J]
+
+
+def bases(M=4096, N=4096, K=4096, J=3, I=3, seed=22) -> Bases:
+    h_real = normal((J, M, K), 1.0, seed)
+    b_real = normal((I, N, K), 1.0, seed + 1)
+    alpha = normal((I, N), 0.3, seed + 2).abs_().add_(0.01)
+    beta = normal((J,), 0.5, seed + 3).abs_().add_(0.05)
+    return Bases(h_real, b_real, alpha, beta)
 
 
 # --------------------------------------------------------------------------

@@ -50,7 +50,8 @@ EXPORTS = (
     "bnn_fold_bn_threshold", "bnn_set_gemm_engine", "bnn_get_gemm_engine", "bnn_selftest_wait_timeout",
     "bnn_binary_weight_gemv", "bnn_ternary_ld_words", "bnn_ternary_workspace_bytes", "bnn_ternary_pack",
     "bnn_ternary_gemv_i8", "bnn_ternary_pack_noalloc", "bnn_pack_sign_rsign", "bnn_pack_sign_nchw_rsign",
-    "bnn_binary_conv1x1_fused",
+    "bnn_binary_conv1x1_fused", "bnn_probe_int_pipes", "bnn_pack_bit_planes", "bnn_bitserial_gemm",
+    "bnn_binary_bases_gemm",
 )
 
 
@@ -101,6 +102,10 @@ def _load() -> ctypes.CDLL:
         "bnn_pack_sign_nchw_rsign": (i32, [p, i32, i64, i64, i64, i64, p, p, p]),
         "bnn_binary_conv1x1_fused": (i32, [p, i64, i64, i64, i64, p, i64, i64, i64,
                                            ctypes.POINTER(bnn_epilogue), p, p]),
+        "bnn_probe_int_pipes": (i32, [i64, p, p, p]),
+        "bnn_pack_bit_planes": (i32, [p, i64, i64, i64, i32, p, i64, p]),
+        "bnn_bitserial_gemm": (i32, [p, i64, i32, p, i64, i32, i64, i64, i64, p, p, i64, p, i64, p]),
+        "bnn_binary_bases_gemm": (i32, [p, i64, i32, p, i64, i32, i64, i64, i64, p, p, i64, p, i64, p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -187,6 +192,15 @@ class gemm_engine:
 
     def __exit__(self, *exc):
         bnn_set_gemm_engine(self.prev)
+
+
+def bnn_probe_int_pipes(iters: int = 4096) -> dict:
+    """Integer-pipe rates of the current device, per SM clock:
+    {"popc": POPC, "lop3": LOP3, "csa_words": XOR words through the carry-save step}."""
+    a, b, c = ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
+    _check("bnn_probe_int_pipes", _lib.bnn_probe_int_pipes(int(iters), ctypes.byref(a), ctypes.byref(b),
+                                                           ctypes.byref(c)))
+    return {"popc": a.value, "lop3": b.value, "csa_words": c.value}
 
 
 def bnn_selftest_wait_timeout(timeout_ns: int) -> bool:
@@ -411,6 +425,39 @@ def bnn_fold_bn_threshold(alpha: torch.Tensor, gamma: torch.Tensor, beta: torch.
 # --------------------------------------------------------------------------
 # allocation helpers (torch device memory; the library itself allocates nothing)
 # --------------------------------------------------------------------------
+
+def bnn_pack_bit_planes(codes: torch.Tensor, bits: int, planes: torch.Tensor, K: Optional[int] = None,
+                        stream=None) -> None:
+    """uint8 codes [rows, K] -> plane-interleaved packed planes [rows * bits, ld]."""
+    assert codes.dtype == torch.uint8 and codes.dim() == 2 and planes.dtype == torch.int32
+    rows = codes.shape[0]
+    K = codes.shape[1] if K is None else int(K)
+    assert planes.shape[0] == rows * bits
+    _check("bnn_pack_bit_planes", _lib.bnn_pack_bit_planes(_ptr(codes), rows, K, _ld(codes), int(bits),
+                                                           _ptr(planes), _ld(planes), _stream(stream)))
+
+
+def bnn_bitserial_gemm(A: torch.Tensor, a_bits: int, W: torch.Tensor, w_bits: int, K: int,
+                       alpha: Optional[torch.Tensor] = None, C_i32: Optional[torch.Tensor] = None,
+                       C_f32: Optional[torch.Tensor] = None, stream=None) -> None:
+    """A, W: plane-interleaved packed planes [M * a_bits, ld], [N * w_bits, ld]."""
+    M, N = A.shape[0] // a_bits, W.shape[0] // w_bits
+    assert A.shape[0] == M * a_bits and W.shape[0] == N * w_bits
+    _check("bnn_bitserial_gemm", _lib.bnn_bitserial_gemm(
+        _ptr(A), _ld(A), int(a_bits), _ptr(W), _ld(W), int(w_bits), M, N, int(K), _ptr(alpha),
+        _ptr(C_i32), _ld(C_i32) if C_i32 is not None else 0, _ptr(C_f32), _ld(C_f32) if C_f32 is not None else 0,
+        _stream(stream)))
+
+
+def bnn_binary_bases_gemm(H: torch.Tensor, J: int, B: torch.Tensor, I: int, K: int, beta: torch.Tensor,
+                          alpha: torch.Tensor, Y: torch.Tensor, stream=None) -> None:
+    """H, B: plane-interleaved packed +1/-1 bases [M * J, ld], [N * I, ld]; beta [J]; alpha [I, N]; Y [M, N]."""
+    M, N = H.shape[0] // J, B.shape[0] // I
+    assert H.shape[0] == M * J and B.shape[0] == N * I and tuple(Y.shape) == (M, N)
+    _check("bnn_binary_bases_gemm", _lib.bnn_binary_bases_gemm(
+        _ptr(H), _ld(H), int(J), _ptr(B), _ld(B), int(I), M, N, int(K), _ptr(beta), _ptr(alpha), _ld(alpha),
+        _ptr(Y), _ld(Y), _stream(stream)))
+
 
 def empty_packed(rows: int, K: int, device="cuda") -> torch.Tensor:
     """int32-typed storage for a packed [rows, bnn_packed_ld_words(K)] matrix."""

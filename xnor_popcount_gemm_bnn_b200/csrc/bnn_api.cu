@@ -23,6 +23,7 @@
 #include "gemv.cuh"
 #include "bwgemv.cuh"
 #include "pack.cuh"
+#include "probe.cuh"
 #include "ternary.cuh"
 
 namespace {
@@ -93,7 +94,11 @@ bool gemm_tc_smem_configured() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
     if (dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return true;
-    if (cudaFuncSetAttribute(bnn::xnor_gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(bnn::xnor_gemm_tc_kernel<bnn::TC_BINARY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bnn::tc::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(bnn::xnor_gemm_tc_kernel<bnn::TC_PLANE_CODES>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, bnn::tc::SMEM_LIMIT) != cudaSuccess ||
+        cudaFuncSetAttribute(bnn::xnor_gemm_tc_kernel<bnn::TC_BASES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              bnn::tc::SMEM_BYTES) != cudaSuccess)
         return false;
     if (dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
@@ -183,9 +188,33 @@ bnn_status launch_gemm_tc(const uint32_t* A, int64_t lda, const uint32_t* W, int
     const int64_t grid = std::min<int64_t>(tiles_m * tiles_n, sm_count());
     bnn::GemmEpilogue e = ep;
     e.bits_words = packed_ld_words(N);
-    bnn::xnor_gemm_tc_kernel<<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(
-        tmA, tmW, (int)M, (int)N, (int)K, (int)kw, (int)tiles_m, (int)tiles_n, e);
+    bnn::xnor_gemm_tc_kernel<bnn::TC_BINARY><<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(
+        tmA, tmW, (int)M, (int)N, (int)K, (int)kw, (int)tiles_m, (int)tiles_n, e, bnn::TcPlanes{});
     return launch_status();
+}
+
+// 3-D map over a plane-interleaved packed matrix (plane p of row r is packed
+// row r * planes + p): dimensions (word, plane, row), box (4 words,
+// box_planes, box_rows), no swizzle.  box_planes > planes reads the missing
+// planes as zero words.
+bool encode_plane_map(CUtensorMap* map, const uint32_t* base, int64_t kw, int64_t planes, int64_t rows, int64_t ld,
+                      int box_planes, int box_rows) {
+    auto enc = tensor_map_encoder();
+    if (enc == nullptr) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)kw, (cuuint64_t)planes, (cuuint64_t)rows};
+    cuuint64_t strides[2] = {(cuuint64_t)ld * 4u, (cuuint64_t)(planes * ld) * 4u};
+    cuuint32_t box[3] = {(cuuint32_t)bnn::tc::BKW, (cuuint32_t)box_planes, (cuuint32_t)box_rows};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int pow2_at_least(int v) {
+    int p = 1;
+    while (p < v) p <<= 1;
+    return p;
 }
 
 // Engine for one product: the tensor cores once the tile is reasonably
@@ -242,7 +271,7 @@ bnn_status launch_gemv_t(const uint32_t* W, int64_t ldw, const XT* x, int64_t N,
     bnn_status st = BNN_OK;
     const bool vec = aligned(x, 16);
     if (lpr == 32 && single && vec) {
-        // Rows of 97..128 words: the dedicated one-chunk-per-lane kernel.  Its
+        // Rows of 68..128 words: the dedicated one-chunk-per-lane kernel.  Its
         // block shape depends on what the launch may overlap; each was the
         // fastest of ~30 shapes on the 11008 x 4096 decode GEMV in back-to-back
         // launches (steps of 1.10 / 1.39 / 2.18 us):
@@ -351,6 +380,36 @@ bnn_status bnn_device_error(int32_t* code_out) {
         if (cudaMemcpyToSymbol(bnn::g_device_error, &zero, sizeof(int)) != cudaSuccess) return BNN_ERR_CUDA;
     }
     *code_out = v;
+    return BNN_OK;
+}
+
+bnn_status bnn_probe_int_pipes(int64_t iters, double* popc_per_clk_sm, double* lop3_per_clk_sm,
+                               double* csa_words_per_clk_sm) {
+    if (iters < 1 || iters > (1 << 24) || popc_per_clk_sm == nullptr || lop3_per_clk_sm == nullptr ||
+        csa_words_per_clk_sm == nullptr)
+        return BNN_ERR_INVALID_ARG;
+    const int sms = sm_count();
+    if (sms < 1 || sms > bnn::probe::MAX_SMS) return BNN_ERR_UNSUPPORTED;
+    void (*kern[bnn::probe::MODES])(int, uint32_t) = {bnn::int_pipe_probe_kernel<0>, bnn::int_pipe_probe_kernel<1>,
+                                                      bnn::int_pipe_probe_kernel<2>};
+    // Operations each thread retires per loop iteration: 4 x 8 POPC, 4 x 8
+    // LOP3, and 4 accumulators x 8 words.
+    const double per_iter[bnn::probe::MODES] = {32.0, 32.0, 32.0};
+    double* out[bnn::probe::MODES] = {popc_per_clk_sm, lop3_per_clk_sm, csa_words_per_clk_sm};
+    unsigned long long cyc[bnn::probe::MAX_SMS];
+    for (int m = 0; m < bnn::probe::MODES; ++m) {
+        if (cudaFuncSetAttribute(kern[m], cudaFuncAttributeMaxDynamicSharedMemorySize, bnn::probe::SMEM_BYTES) !=
+            cudaSuccess)
+            return BNN_ERR_CUDA;
+        kern[m]<<<sms, bnn::probe::THREADS, bnn::probe::SMEM_BYTES>>>((int)iters, 0x2545F491u);
+        if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) return BNN_ERR_CUDA;
+        if (cudaMemcpyFromSymbol(cyc, bnn::g_probe_cycles, sizeof(unsigned long long) * (size_t)sms) != cudaSuccess)
+            return BNN_ERR_CUDA;
+        std::sort(cyc, cyc + sms);
+        const double median = (double)cyc[sms / 2];
+        if (median <= 0.0) return BNN_ERR_CUDA;
+        *out[m] = (double)bnn::probe::THREADS * (double)iters * per_iter[m] / median;
+    }
     return BNN_OK;
 }
 
@@ -525,7 +584,12 @@ bnn_status bnn_binary_weight_gemv(const uint32_t* W, int64_t ldw, const void* x,
     if (!aligned(x, x_dt == BNN_F32 ? 4 : 2) || !aligned(alpha, 4) || !aligned(y, 4)) return BNN_ERR_ALIGNMENT;
     if (N == 0) return BNN_OK;
     if (!bw_gemv_smem_configured()) return BNN_ERR_CUDA;
-    const int64_t blocks = std::min<int64_t>(ceil_div(N, (int64_t)32), sm_count());
+    // One batch of U row groups per warp covers N with this many CTAs; more
+    // rows loop.  Two CTAs fit on an SM, so the grid is capped at two per SM.
+    int64_t lpr = 1;
+    while (lpr < 32 && lpr < kw / 4) lpr <<= 1;
+    const int64_t rows_per_cta = (int64_t)bnn::bwg::WARPS * bnn::bwg::U * (32 / lpr);
+    const int64_t blocks = std::min<int64_t>(ceil_div(N, rows_per_cta), 2 * (int64_t)sm_count());
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)blocks);
     cfg.blockDim = dim3(bnn::bwg::THREADS);
@@ -548,6 +612,113 @@ bnn_status bnn_binary_weight_gemv(const uint32_t* W, int64_t ldw, const void* x,
                                static_cast<const __nv_bfloat16*>(x), (int)N, (int)K, (int)kw, alpha, y, prefetch,
                                xstatic, dependent);
     if (e != cudaSuccess) return BNN_ERR_CUDA;
+    return launch_status();
+}
+
+bnn_status bnn_pack_bit_planes(const uint8_t* codes, int64_t rows, int64_t K, int64_t ld_codes, int bits,
+                               uint32_t* planes, int64_t ld_words, bnn_stream_t stream) {
+    if (codes == nullptr || planes == nullptr) return BNN_ERR_INVALID_ARG;
+    if (rows < 0 || K < 1 || ld_codes < K || bits < 1 || bits > 8) return BNN_ERR_INVALID_ARG;
+    const int64_t kw = packed_ld_words(K);
+    if (ld_words < kw) return BNN_ERR_INVALID_ARG;
+    if ((ld_words & 3) != 0 || !aligned(planes, 16)) return BNN_ERR_ALIGNMENT;
+    if (rows == 0) return BNN_OK;
+    const int64_t blocks = ceil_div(rows, 8);
+    if (blocks > INT_MAX) return BNN_ERR_INVALID_ARG;
+    const bool vec = aligned(codes, 16) && (ld_codes % 16 == 0);
+    bnn::pack_bit_planes_kernel<<<(unsigned)blocks, 256, 0, as_cuda(stream)>>>(codes, rows, K, ld_codes, bits, planes,
+                                                                                ld_words, kw, vec);
+    return launch_status();
+}
+
+bnn_status bnn_bitserial_gemm(const uint32_t* A, int64_t lda, int a_bits, const uint32_t* W, int64_t ldw, int w_bits,
+                              int64_t M, int64_t N, int64_t K, const float* alpha, int32_t* C_i32, int64_t ldc,
+                              float* C_f32, int64_t ldf, bnn_stream_t stream) {
+    using namespace bnn::tc;
+    bnn_status st = check_gemm_dims(M, N, K);
+    if (st != BNN_OK) return st;
+    if (a_bits < 1 || a_bits > MAX_CODE_PLANES || w_bits < 1 || w_bits > MAX_CODE_PLANES) return BNN_ERR_INVALID_ARG;
+    // The int32 accumulator holds K * (2^a - 1) * (2^w - 1) at most.
+    if ((double)K * (double)((1 << a_bits) - 1) * (double)((1 << w_bits) - 1) > (double)INT_MAX)
+        return BNN_ERR_INVALID_ARG;
+    if (M * a_bits > INT_MAX || N * w_bits > INT_MAX) return BNN_ERR_INVALID_ARG;
+    const int64_t kw = packed_ld_words(K);
+    if ((st = check_packed_operand(A, lda, kw)) != BNN_OK) return st;
+    if ((st = check_packed_operand(W, ldw, kw)) != BNN_OK) return st;
+    if (C_i32 == nullptr && C_f32 == nullptr) return BNN_ERR_INVALID_ARG;
+    if (C_i32 != nullptr && ldc < N) return BNN_ERR_INVALID_ARG;
+    if (C_f32 != nullptr && (ldf < N || alpha == nullptr)) return BNN_ERR_INVALID_ARG;
+    if ((C_i32 && !aligned(C_i32, 4)) || (C_f32 && !aligned(C_f32, 4)) || (alpha && !aligned(alpha, 4)))
+        return BNN_ERR_ALIGNMENT;
+    if (M == 0 || N == 0) return BNN_OK;
+    CUtensorMap tmA, tmW;
+    if (!encode_plane_map(&tmA, A, kw, a_bits, M, lda, a_bits, BM) ||
+        !encode_plane_map(&tmW, W, kw, w_bits, N, ldw, w_bits, BN))
+        return BNN_ERR_CUDA;
+    const int64_t tiles_m = ceil_div(M, BM), tiles_n = ceil_div(N, BN);
+    if (tiles_m * tiles_n > INT_MAX) return BNN_ERR_INVALID_ARG;
+    if (!gemm_tc_smem_configured()) return BNN_ERR_CUDA;
+    bnn::TcPlanes pl{};
+    pl.ja = a_bits;
+    pl.jw = w_bits;
+    pl.j_real = a_bits;
+    pl.i_real = w_bits;
+    pl.p_stage = packed_stage_bytes(bnn::TC_PLANE_CODES, a_bits, w_bits);
+    pl.pstages = packed_stages(bnn::TC_PLANE_CODES, a_bits, w_bits);
+    if (pl.pstages < 2) return BNN_ERR_UNSUPPORTED;
+    bnn::GemmEpilogue e{};
+    e.c_i32 = C_i32;
+    e.ldc = ldc;
+    e.c_f32 = C_f32;
+    e.ldf = ldf;
+    e.alpha = alpha;
+    e.bits_words = packed_ld_words(N);
+    const int64_t grid = std::min<int64_t>(tiles_m * tiles_n, sm_count());
+    const size_t smem = (size_t)SMEM_FIXED + (size_t)pl.pstages * (size_t)pl.p_stage;
+    bnn::xnor_gemm_tc_kernel<bnn::TC_PLANE_CODES><<<(unsigned)grid, THREADS, smem, as_cuda(stream)>>>(
+        tmA, tmW, (int)M, (int)N, (int)K, (int)kw, (int)tiles_m, (int)tiles_n, e, pl);
+    return launch_status();
+}
+
+bnn_status bnn_binary_bases_gemm(const uint32_t* H, int64_t ldh, int J, const uint32_t* B, int64_t ldb, int I,
+                                 int64_t M, int64_t N, int64_t K, const float* beta, const float* alpha,
+                                 int64_t lda_alpha, float* Y, int64_t ldy, bnn_stream_t stream) {
+    using namespace bnn::tc;
+    bnn_status st = check_gemm_dims(M, N, K);
+    if (st != BNN_OK) return st;
+    if (J < 1 || J > MAX_BASES || I < 1 || I > MAX_BASES) return BNN_ERR_INVALID_ARG;
+    if (M * J > INT_MAX || N * I > INT_MAX) return BNN_ERR_INVALID_ARG;
+    const int64_t kw = packed_ld_words(K);
+    if ((st = check_packed_operand(H, ldh, kw)) != BNN_OK) return st;
+    if ((st = check_packed_operand(B, ldb, kw)) != BNN_OK) return st;
+    if (beta == nullptr || alpha == nullptr || Y == nullptr) return BNN_ERR_INVALID_ARG;
+    if (lda_alpha < N || ldy < N) return BNN_ERR_INVALID_ARG;
+    if (!aligned(beta, 4) || !aligned(alpha, 4) || !aligned(Y, 4)) return BNN_ERR_ALIGNMENT;
+    if (M == 0 || N == 0) return BNN_OK;
+    const int jp = pow2_at_least(J), ip = pow2_at_least(I);
+    const int rows_per_tile = BM / jp, cols_per_tile = BN / ip;
+    CUtensorMap tmA, tmW;
+    if (!encode_plane_map(&tmA, H, kw, J, M, ldh, jp, rows_per_tile) ||
+        !encode_plane_map(&tmW, B, kw, I, N, ldb, ip, cols_per_tile))
+        return BNN_ERR_CUDA;
+    const int64_t tiles_m = ceil_div(M, rows_per_tile), tiles_n = ceil_div(N, cols_per_tile);
+    if (tiles_m * tiles_n > INT_MAX) return BNN_ERR_INVALID_ARG;
+    if (!gemm_tc_smem_configured()) return BNN_ERR_CUDA;
+    bnn::TcPlanes pl{};
+    pl.ja = jp;
+    pl.jw = ip;
+    pl.j_real = J;
+    pl.i_real = I;
+    pl.p_stage = P_STAGE;
+    pl.pstages = PSTAGES;
+    pl.beta = beta;
+    pl.alpha = alpha;
+    pl.lda_alpha = lda_alpha;
+    pl.y = Y;
+    pl.ldy = ldy;
+    const int64_t grid = std::min<int64_t>(tiles_m * tiles_n, sm_count());
+    bnn::xnor_gemm_tc_kernel<bnn::TC_BASES><<<(unsigned)grid, THREADS, SMEM_BYTES, as_cuda(stream)>>>(
+        tmA, tmW, (int)M, (int)N, (int)K, (int)kw, (int)tiles_m, (int)tiles_n, bnn::GemmEpilogue{}, pl);
     return launch_status();
 }
 
@@ -626,7 +797,9 @@ namespace {
 static __device__ __align__(256) double g_ternary_scratch[BNN_TERNARY_PACK_NOALLOC_MAX_ROWS + 1];
 
 // The device address of g_ternary_scratch on the current device, looked up
-// once per device (host code cannot use the symbol itself as a pointer).
+// once per device (host code cannot use the symbol itself as a pointer) and
+// kept for the life of the process; a cudaDeviceReset() after the look-up
+// would leave the kept address stale (the header says not to do that).
 void* ternary_scratch_address() {
     constexpr int kMaxDevices = 64;
     static std::atomic<void*> addr[kMaxDevices];

@@ -205,8 +205,7 @@ xnor_conv3x3_tc_kernel(const uint32_t* __restrict__ X, int n, int c, int h, int 
             const int64_t obase = valid ? (q / plane) * cout * plane + q % plane : 0;
             for (int c0 = 0; c0 < n_mma; c0 += 32) {
                 uint32_t rr[32];
-                tmem_ld32(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * acc_stride + c0), rr);
-                tmem_ld_wait();
+                tmem_ld32_sync(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * acc_stride + c0), rr);
                 if (c0 + 32 >= n_mma) {
                     tc_fence_before();
                     __syncwarp();
@@ -499,8 +498,7 @@ xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* _
             bool arrived = false;
             for (int c0 = slice0; c0 < n_mma; c0 += 2 * EPI_COLS) {
                 uint32_t rr[EPI_COLS];
-                tmem_ld16(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * acc_stride + c0), rr);
-                tmem_ld_wait();
+                tmem_ld16_sync(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * acc_stride + c0), rr);
                 if (c0 + 2 * EPI_COLS >= n_mma) {
                     tc_fence_before();
                     __syncwarp();

@@ -212,6 +212,10 @@ xnor_gemm_popc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_cons
                     for (int j = 0; j < TN_; ++j) acc[i][j] += popc_xor4(a[i], b[j]);
             }
         }
+        // The stage's words were read through the generic proxy; the
+        // producer refills it with TMA (async proxy) once `empty` completes.
+        // The proxy fence orders those reads before that write.
+        fence_proxy_async_shared();
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
     }

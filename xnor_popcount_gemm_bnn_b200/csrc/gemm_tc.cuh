@@ -43,10 +43,10 @@ namespace bnn {
 namespace tc {
 constexpr int BM = 128;                    // tile rows  = TMEM lanes = UMMA M
 constexpr int BN = 256;                    // tile cols  = UMMA N
-constexpr int BKE = 128;                   // binary elements of K per stage (4 packed words)
+constexpr int BKE = 128;                   // elements of K per stage (4 packed words)
 constexpr int BKW = BKE / 32;
 constexpr int UMMA_K = 32;                 // int8 K per tcgen05.mma
-constexpr int PSTAGES = 8;                 // packed ring
+constexpr int PSTAGES = 8;                 // packed ring (binary and bases modes)
 constexpr int USTAGES = 3;                 // unpacked (int8) ring
 constexpr int P_A_BYTES = BM * BKW * 4;    // 2 KiB
 constexpr int P_B_BYTES = BN * BKW * 4;    // 4 KiB
@@ -64,12 +64,61 @@ constexpr int NUM_BARS = 2 * PSTAGES + 2 * USTAGES + 2 * 2 + 1;
 // float4 {alpha, gamma, beta, -} and int2 {c1, len2} of the threshold test
 // per column.
 constexpr int COLP_BYTES = EPI_WARPS * BN * (16 + 8);
-constexpr int SMEM_BYTES = USTAGES * U_STAGE + PSTAGES * P_STAGE + COLP_BYTES + NUM_BARS * 8 + 16 + 1024;
-// kind::i8 instruction descriptor: D s32 (bits 4-5 = 2), A s8 (bits 7-9 = 1),
-// B s8 (bits 10-12 = 1), both K-major, N >> 3 at bits 17-22, M >> 4 at 24-28.
+constexpr int SMEM_FIXED = USTAGES * U_STAGE + COLP_BYTES + NUM_BARS * 8 + 16 + 1024;
+constexpr int SMEM_BYTES = SMEM_FIXED + PSTAGES * P_STAGE;
+// Shared memory one CTA may use on sm_100 (opt-in maximum).
+constexpr int SMEM_LIMIT = 227 * 1024;
+// Bit planes per operand row in the plane-code mode (unsigned codes of up to
+// this many bits), and bases per operand in the bases mode.
+constexpr int MAX_CODE_PLANES = 4;
+constexpr int MAX_BASES = 8;
+// kind::i8 instruction descriptor: D s32 (bits 4-5 = 2), A and B type at bits
+// 7-9 and 10-12 (1 = s8, 0 = u8), both K-major, N >> 3 at bits 17-22, M >> 4
+// at 24-28.
 constexpr uint32_t IDESC = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                            ((uint32_t)(BM >> 4) << 24);
+constexpr uint32_t IDESC_U8 = (2u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+// Bytes of one packed stage and the packed-ring depth that fits beside the
+// fixed part of shared memory.  Binary and bases modes: 128 + 256 packed rows
+// of 16 bytes.  Plane-code mode: every code row brings its planes.
+__host__ __device__ constexpr int packed_stage_bytes(int mode, int ja, int jw) {
+    return mode == 1 ? (BM * ja + BN * jw) * 16 : P_STAGE;
+}
+__host__ __device__ constexpr int packed_stages(int mode, int ja, int jw) {
+    return (SMEM_LIMIT - SMEM_FIXED) / packed_stage_bytes(mode, ja, jw) < PSTAGES
+               ? (SMEM_LIMIT - SMEM_FIXED) / packed_stage_bytes(mode, ja, jw)
+               : PSTAGES;
+}
 }  // namespace tc
+
+// Kernel modes of xnor_gemm_tc_kernel.
+//  TC_BINARY      +1/-1 operands, one packed row per matrix row (eq. (6)).
+//  TC_PLANE_CODES unsigned integer codes stored as bit planes: plane p of
+//                 code row r is packed row r * planes + p; the unpack folds
+//                 the planes into one byte per element, code = sum_p bit_p
+//                 2^p, and the tensor cores multiply u8 x u8 -- the whole
+//                 multi-bit product sum_k a_k w_k in one pass (DoReFa-Net's
+//                 bit-convolution).
+//  TC_BASES       +1/-1 binary bases stored plane-interleaved the same way;
+//                 each base is expanded like a binary row, so every pair
+//                 (base j of A, base i of W) gets its own +1/-1 product, and
+//                 the epilogue forms sum_j beta_j sum_i alpha_i[n] * s_ji
+//                 (ABC-Net).
+enum TcMode { TC_BINARY = 0, TC_PLANE_CODES = 1, TC_BASES = 2 };
+
+// Plane layout and the bases epilogue's parameters.
+struct TcPlanes {
+    int ja, jw;           // planes per A / W row inside a stage (bases: padded to a power of two)
+    int j_real, i_real;   // bases actually present (the padded ones are zero-filled by the TMA box)
+    int pstages;          // packed-ring depth
+    int p_stage;          // bytes per packed stage
+    const float* beta;    // bases: beta_j, [j_real]
+    const float* alpha;   // bases: alpha_i[n], [i_real][lda_alpha]
+    int64_t lda_alpha;
+    float* y;             // bases: fp32 output [M, N]
+    int64_t ldy;
+};
 
 // Shared-memory matrix descriptor for a K-major, 128B-swizzled operand tile
 // whose rows are 128 bytes (8-row groups 1024 bytes apart): start address,
@@ -95,12 +144,13 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
-__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(tc::IDESC), "r"(accumulate)
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -110,26 +160,37 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                  : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+// TMEM -> registers for one warp: 32 lanes x 32 (or 16) consecutive 32-bit
+// columns, followed by tcgen05.wait::ld in the SAME asm statement.  The load
+// is asynchronous: its destination registers hold the values only after the
+// wait.  With the wait in a separate asm statement nothing ties the uses of
+// those registers to it (the wait names no register), so the compiler may
+// schedule arithmetic on them before the wait and read stale values.
+// Keeping both instructions in one statement defines the outputs at the end
+// of the statement, after the wait.
+__device__ __forceinline__ void tmem_ld32_sync(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
         "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
           "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
           "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
+        : "r"(taddr)
+        : "memory");
 }
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+__device__ __forceinline__ void tmem_ld16_sync(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
+        : "r"(taddr)
+        : "memory");
 }
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Bounded wait that also gives up as soon as another role of the CTA aborted.
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
@@ -168,17 +229,68 @@ __device__ __forceinline__ void expand_word_pm1(uint32_t w, uint4& c0, uint4& c1
     c1 = make_uint4(r[4], r[5], r[6], r[7]);
 }
 
+// Bit planes -> unsigned byte codes.  `w[p]` holds word q of plane p (the
+// same 32 elements in every plane); byte e of the result is sum_p bit_p(e)
+// 2^p.  Per plane and 4 bytes: a shift, a sign-replicating PRMT (byte ->
+// 0x00 / 0xFF as in expand_word_pm1) and one LOP3 that keeps bit p of each
+// byte and ORs it in.  The byte order inside the 32 is expand_word_pm1's
+// permutation, so an A row and a W row expanded by this function pair the
+// same elements.
+__device__ __forceinline__ void expand_planes_u8(const uint32_t (&w)[tc::MAX_CODE_PLANES], int planes, uint4& c0,
+                                                 uint4& c1) {
+    uint32_t r[8];
+    #pragma unroll
+    for (int s = 0; s < 8; ++s) r[s] = 0u;
+    #pragma unroll
+    for (int p = 0; p < tc::MAX_CODE_PLANES; ++p) {
+        if (p < planes) {
+            const uint32_t wp = w[p], mask = 0x01010101u << p;
+            #pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                uint32_t m;
+                asm("prmt.b32 %0, %1, 0, 0xBA98;" : "=r"(m) : "r"(wp << s));
+                asm("lop3.b32 %0, %1, %2, %3, 0xf8;" : "=r"(r[s]) : "r"(r[s]), "r"(m), "r"(mask));   // r | (m & mask)
+            }
+        }
+    }
+    c0 = make_uint4(r[0], r[1], r[2], r[3]);
+    c1 = make_uint4(r[4], r[5], r[6], r[7]);
+}
+
+// Hand a packed stage back to the TMA producer once this warp has read it.
+// The reads are generic-proxy loads; the producer's next fill of the same
+// bytes is an async-proxy (TMA) write issued as soon as the stage's "empty"
+// barrier completes.  The proxy fence orders this thread's reads before any
+// later async-proxy access, so the fill cannot land before a read it would
+// overwrite has taken its value (without it, full-output comparisons caught
+// unpack warps expanding words of a later stage).
+__device__ __forceinline__ void release_packed_stage(uint64_t* empty_bar, int lane) {
+    fence_proxy_async_shared();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty_bar);
+}
+
+template <int MODE>
 __global__ void __launch_bounds__(tc::THREADS, 1)
 xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW, int M, int N,
-                    int K, int kw, int tiles_m, int tiles_n, GemmEpilogue ep) {
+                    int K, int kw, int tiles_m, int tiles_n, GemmEpilogue ep, TcPlanes pl) {
     using namespace tc;
     extern __shared__ uint8_t smem_raw[];
+    // Packed-ring geometry: fixed in the binary and bases modes, set by the
+    // plane counts in the plane-code mode.
+    const int pst = MODE == TC_PLANE_CODES ? pl.pstages : PSTAGES;
+    const int pstage = MODE == TC_PLANE_CODES ? pl.p_stage : P_STAGE;
+    const int pa_bytes = MODE == TC_PLANE_CODES ? BM * pl.ja * 16 : P_A_BYTES;
+    // Rows (and columns) of the output per tile: the bases mode spends ja (jw)
+    // accumulator lanes (columns) on each output row (column).
+    const int rows_per_tile = MODE == TC_BASES ? BM / pl.ja : BM;
+    const int cols_per_tile = MODE == TC_BASES ? BN / pl.jw : BN;
     // 1024-byte aligned base, derived by offset from the __shared__ array so
     // that the compiler keeps every access in the shared address space.
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* uring = smem;                                   // USTAGES x (A 16 KiB | W 32 KiB)
-    uint8_t* pring = smem + USTAGES * U_STAGE;               // PSTAGES x (A 2 KiB | W 4 KiB)
-    float4* colf = reinterpret_cast<float4*>(pring + PSTAGES * P_STAGE);      // [EPI_WARPS][BN]
+    uint8_t* pring = smem + USTAGES * U_STAGE;               // pst x (A | W packed)
+    float4* colf = reinterpret_cast<float4*>(pring + pst * pstage);           // [EPI_WARPS][BN]
     int2* colt = reinterpret_cast<int2*>(colf + EPI_WARPS * BN);               // [EPI_WARPS][BN]
     uint64_t* bars = reinterpret_cast<uint64_t*>(colt + EPI_WARPS * BN);
     uint64_t* pfull = bars;
@@ -199,7 +311,7 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     if (threadIdx.x == 0) {
         prefetch_tensormap(&tmA);
         prefetch_tensormap(&tmW);
-        for (int s = 0; s < PSTAGES; ++s) {
+        for (int s = 0; s < pst; ++s) {
             mbar_init(&pfull[s], 1);
             mbar_init(&pempty[s], UNPACK_WARPS);
         }
@@ -230,21 +342,28 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             uint32_t g = 0, issued = 0;
             bool ok = true;
             for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
-                const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
+                const int m0 = (t / tiles_n) * rows_per_tile, n0 = (t % tiles_n) * cols_per_tile;
                 for (int ks = 0; ks < nk; ++ks, ++g) {
-                    const uint32_t s = g % PSTAGES;
-                    if (g >= PSTAGES && !tc_wait(&pempty[s], ((g / PSTAGES) - 1) & 1, abort_flag)) { ok = false; break; }
-                    uint8_t* dst = pring + s * P_STAGE;
-                    mbar_arrive_expect_tx(&pfull[s], P_STAGE);
-                    tma_load_2d(dst, &tmA, ks * BKW, m0, &pfull[s]);
-                    tma_load_2d(dst + P_A_BYTES, &tmW, ks * BKW, n0, &pfull[s]);
+                    const uint32_t s = g % (uint32_t)pst;
+                    if (g >= (uint32_t)pst && !tc_wait(&pempty[s], ((g / pst) - 1) & 1, abort_flag)) { ok = false; break; }
+                    uint8_t* dst = pring + s * pstage;
+                    mbar_arrive_expect_tx(&pfull[s], pstage);
+                    if constexpr (MODE == TC_BINARY) {
+                        tma_load_2d(dst, &tmA, ks * BKW, m0, &pfull[s]);
+                        tma_load_2d(dst + pa_bytes, &tmW, ks * BKW, n0, &pfull[s]);
+                    } else {
+                        // Boxes of {4 words, all planes, rows}: the planes of
+                        // a row land next to each other, 16 bytes apart.
+                        tma_load_3d(dst, &tmA, ks * BKW, 0, m0, &pfull[s]);
+                        tma_load_3d(dst + pa_bytes, &tmW, ks * BKW, 0, n0, &pfull[s]);
+                    }
                     ++issued;
                 }
             }
             // Let the copies still in flight land before the CTA can retire
             // (also after an abort).
-            for (uint32_t q = issued > PSTAGES ? issued - PSTAGES : 0; q < issued; ++q)
-                if (!mbar_wait_bounded(&pfull[q % PSTAGES], (q / PSTAGES) & 1)) break;
+            for (uint32_t q = issued > (uint32_t)pst ? issued - pst : 0; q < issued; ++q)
+                if (!mbar_wait_bounded(&pfull[q % pst], (q / pst) & 1)) break;
         }
     } else if (warp == WARP_MMA) {
         // ------------------------------ MMA issuer ------------------------------
@@ -253,6 +372,7 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             int lt = 0;
             bool ok = true;
             const uint32_t ubase = smem_u32(uring);
+            const uint32_t idesc = MODE == TC_PLANE_CODES ? IDESC_U8 : IDESC;
             for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++lt) {
                 const int b = lt & 1;
                 if (lt >= 2 && !tc_wait(&aempty[b], ((lt >> 1) - 1) & 1, abort_flag)) break;
@@ -268,7 +388,7 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     for (int kk = 0; kk < BKE / UMMA_K; ++kk) {
                         // Advancing the start address by 32 B steps through K inside the swizzle atom.
                         mma_i8(d_tmem, umma_desc_sw128(a_addr + kk * UMMA_K), umma_desc_sw128(b_addr + kk * UMMA_K),
-                               (ks | kk) != 0 ? 1u : 0u);
+                               idesc, (ks | kk) != 0 ? 1u : 0u);
                     }
                     mma_commit(&uempty[s]);
                 }
@@ -282,51 +402,74 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         __syncwarp();
     } else if (warp < WARP_EPI0) {
         // ------------------------------ unpack warps ------------------------------
-        // Thread u expands packed row u of the stage (A rows 0..127, then W rows):
-        // one 16-byte load of its 4 words, eight 16-byte stores of its 128 bytes.
+        // Thread u expands row u of the stage (A rows 0..127, then W rows) into
+        // 128 bytes: one 16-byte load of its 4 words per plane, eight 16-byte
+        // stores.  Binary and bases modes: a row is one +1/-1 plane.  Plane-code
+        // mode: a row is a code row whose planes sit 16 bytes apart.
         const int u = threadIdx.x - WARP_UNPACK0 * 32;               // 0..383
         const bool is_a = u < BM;
         const int r = is_a ? u : u - BM;
         const int sw = r & 7;
+        const int planes = MODE == TC_PLANE_CODES ? (is_a ? pl.ja : pl.jw) : 1;
         uint32_t g = 0;
         bool ok = true;
         for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
             for (int ks = 0; ks < nk; ++ks, ++g) {
-                const uint32_t ps = g % PSTAGES, us = g % USTAGES;
-                bool w1 = tc_wait(&pfull[ps], (g / PSTAGES) & 1, abort_flag);
+                const uint32_t ps = g % (uint32_t)pst, us = g % USTAGES;
+                bool w1 = tc_wait(&pfull[ps], (g / pst) & 1, abort_flag);
                 bool w2 = w1 && (g < USTAGES || tc_wait(&uempty[us], ((g / USTAGES) - 1) & 1, abort_flag));
                 if (!__all_sync(0xffffffffu, w1 && w2)) { ok = false; break; }
-                const uint4 pk = *reinterpret_cast<const uint4*>(pring + ps * P_STAGE + u * 16);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&pempty[ps]);             // packed stage consumed
                 uint8_t* row = uring + us * U_STAGE + (is_a ? 0 : U_A_BYTES) + r * 128;
-                const uint32_t wq[4] = {pk.x, pk.y, pk.z, pk.w};
-                #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint4 c0, c1;
-                    expand_word_pm1(wq[q], c0, c1);
-                    *reinterpret_cast<uint4*>(row + (((2 * q) ^ sw) << 4)) = c0;
-                    *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ sw) << 4)) = c1;
+                if constexpr (MODE == TC_PLANE_CODES) {
+                    const uint8_t* src = pring + ps * pstage + (is_a ? 0 : pa_bytes) + r * planes * 16;
+                    uint32_t wq[4][MAX_CODE_PLANES];
+                    #pragma unroll
+                    for (int p = 0; p < MAX_CODE_PLANES; ++p) {
+                        const uint4 pk = p < planes ? *reinterpret_cast<const uint4*>(src + p * 16)
+                                                    : make_uint4(0u, 0u, 0u, 0u);
+                        wq[0][p] = pk.x; wq[1][p] = pk.y; wq[2][p] = pk.z; wq[3][p] = pk.w;
+                    }
+                    release_packed_stage(&pempty[ps], lane);
+                    #pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 c0, c1;
+                        expand_planes_u8(wq[q], planes, c0, c1);
+                        *reinterpret_cast<uint4*>(row + (((2 * q) ^ sw) << 4)) = c0;
+                        *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ sw) << 4)) = c1;
+                    }
+                } else {
+                    const uint4 pk = *reinterpret_cast<const uint4*>(pring + ps * pstage + u * 16);
+                    release_packed_stage(&pempty[ps], lane);
+                    const uint32_t wq[4] = {pk.x, pk.y, pk.z, pk.w};
+                    #pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 c0, c1;
+                        expand_word_pm1(wq[q], c0, c1);
+                        *reinterpret_cast<uint4*>(row + (((2 * q) ^ sw) << 4)) = c0;
+                        *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ sw) << 4)) = c1;
+                    }
                 }
                 fence_proxy_async_shared();                           // make the bytes visible to the tensor core
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&ufull[us]);
             }
         }
-    } else {
+    } else if constexpr (MODE != TC_BASES) {
         // ------------------------------ epilogue warps ------------------------------
         // Per tile, each epilogue warp first stages the tile's column parameters
         // in its own shared-memory copy (alpha/gamma/beta and the threshold test
         // as one unsigned range check on the raw accumulator), then each thread
         // turns its row's 256 accumulators into outputs with broadcast shared
         // loads instead of per-column global loads.  The copy is private to
-        // the warp, so only __syncwarp orders it: a named barrier across the
-        // epilogue warps here corrupted accumulator reads in testing.
+        // the warp, so only __syncwarp orders it and no warp waits for
+        // another.
         const int quad = warp & 3;                                    // TMEM lanes 32*quad .. 32*quad + 31
         float4* wcolf = colf + (warp - WARP_EPI0) * BN;
         int2* wcolt = colt + (warp - WARP_EPI0) * BN;
         const int kp = nk * BKE;                                      // padded K: acc = kp - 2 * popcount
-        const int pad = kp - K;                                       // (+1)(+1) pad positions per output
+        // Binary: (+1)(+1) pad positions per output.  Plane codes: a pad
+        // element is code 0 and adds nothing.
+        const int pad = MODE == TC_PLANE_CODES ? 0 : kp - K;
         const bool affine = ep.gamma != nullptr;
         int lt = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++lt) {
@@ -373,8 +516,7 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t r[32];
-                tmem_ld32(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * BN + 32 * c), r);
-                tmem_ld_wait();
+                tmem_ld32_sync(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * BN + 32 * c), r);
                 if (c == BN / 32 - 1) {
                     // Whole accumulator read: hand it back to the MMA warp.
                     tc_fence_before();
@@ -442,6 +584,65 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             if (ep.c_bits != nullptr && (t % tiles_n) == tiles_n - 1 && m < M) {
                 for (int64_t wd = (int64_t)(n0 + BN) / 32; wd < ep.bits_words; ++wd)
                     ep.c_bits[(int64_t)m * ep.ldb + wd] = 0u;
+            }
+        }
+    } else {
+        // ------------------------- epilogue warps, bases mode -------------------------
+        // Accumulator lane L holds base j = L mod ja of output row L / ja;
+        // column c holds base i = c mod jw of output column c / jw.  Each
+        // thread forms v = sum_i alpha_i[n] * s_ji for its base j, scales it by
+        // beta_j, and a butterfly over the ja lanes of the row adds the bases
+        // j (every lane of the group ends with the same total).  Padded bases
+        // have beta_j = 0 or alpha_i[n] = 0, so their products add exactly 0.
+        const int quad = warp & 3;
+        const int ja = pl.ja, jw = pl.jw;
+        float* wcola = reinterpret_cast<float*>(colf + (warp - WARP_EPI0) * BN);   // alpha per column
+        const int kp = nk * BKE;
+        const int pad = kp - K;
+        const int L = 32 * quad + lane;
+        const int jl = L & (ja - 1);
+        const float bj = jl < pl.j_real ? __ldg(pl.beta + jl) : 0.0f;
+        const int outs_per_chunk = 32 / jw;                           // output columns per 32 accumulator columns
+        int lt = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++lt) {
+            const int b = lt & 1;
+            const int m0 = (t / tiles_n) * rows_per_tile, n0 = (t % tiles_n) * cols_per_tile;
+            __syncwarp();
+            for (int i = lane; i < BN; i += 32) {
+                const int n = n0 + i / jw, ib = i & (jw - 1);
+                wcola[i] = (n < N && ib < pl.i_real) ? __ldg(pl.alpha + (int64_t)ib * pl.lda_alpha + n) : 0.0f;
+            }
+            __syncwarp();
+            if (!__all_sync(0xffffffffu, tc_wait(&afull[b], (lt >> 1) & 1, abort_flag))) break;
+            tc_fence_after();
+            const int m = m0 + L / ja;
+            #pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32_sync(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * BN + 32 * c), r);
+                if (c == BN / 32 - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&aempty[b]);
+                }
+                const int nb = n0 + c * outs_per_chunk;
+                if (nb >= N) continue;                                // uniform across the warp
+                // Columns in order; after the last base of each output column
+                // (every jw columns, the same for all lanes) the row total is
+                // formed and stored.  Register indices stay compile-time.
+                float v = 0.0f;
+                #pragma unroll
+                for (int col = 0; col < 32; ++col) {
+                    v = fmaf(wcola[32 * c + col], (float)((int32_t)r[col] - pad), v);
+                    if (((col + 1) & (jw - 1)) == 0) {
+                        float tsum = bj * v;
+                        for (int off = 1; off < ja; off <<= 1) tsum += __shfl_xor_sync(0xffffffffu, tsum, off);
+                        const int o = col / jw;
+                        const int n = nb + o;
+                        if ((o & (ja - 1)) == jl && m < M && n < N) pl.y[(int64_t)m * pl.ldy + n] = tsum;
+                        v = 0.0f;
+                    }
+                }
             }
         }
     }

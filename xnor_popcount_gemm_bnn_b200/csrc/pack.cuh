@@ -235,4 +235,54 @@ pack_conv3x3_weights_kernel(const T* __restrict__ w, int64_t cout, int64_t cin,
     }
 }
 
+// Unsigned k-bit codes -> bit planes ("State of the Art Survey (2016 ->
+// 2026)", classic CNN BNN table, DoReFa-Net: low-bit weights and activations
+// multiplied by bit-convolution).  codes: uint8 [rows, ld_codes], only the low
+// `bits` bits of each byte are used.  planes: plane p of row r is the packed
+// row r * bits + p (stride ldw words), bit j of word w = bit p of code
+// 32 w + j; elements past K and words up to kw are zero.  One warp per row; a
+// lane takes 16 consecutive codes (one 16-byte load when aligned), each plane's
+// 16 bits are gathered 4 codes at a time with a multiply (bits at 0, 8, 16, 24
+// land on 28..31 without carries), and two neighbouring lanes form a word.
+__global__ void __launch_bounds__(256)
+pack_bit_planes_kernel(const uint8_t* __restrict__ codes, int64_t rows, int64_t K, int64_t ldc, int bits,
+                       uint32_t* __restrict__ planes, int64_t ldw, int64_t kw, bool vec) {
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (row >= rows) return;                                  // warp-uniform
+    const uint8_t* src = codes + row * ldc;
+    uint32_t* dst = planes + row * bits * ldw;
+    for (int64_t w0 = 0; w0 < kw; w0 += 16) {                 // 16 words (512 codes) per warp pass
+        const int64_t e0 = 32 * w0 + 16 * (int64_t)lane;      // this lane's first code
+        uint32_t x[4];
+        if (vec && e0 + 16 <= K) {
+            const uint4 q = *reinterpret_cast<const uint4*>(src + e0);
+            x[0] = q.x; x[1] = q.y; x[2] = q.z; x[3] = q.w;
+        } else {
+            #pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t v = 0;
+                #pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int64_t e = e0 + 4 * q + i;
+                    if (e < K) v |= (uint32_t)src[e] << (8 * i);
+                }
+                x[q] = v;
+            }
+        }
+        const int64_t wd = w0 + (lane >> 1);
+        for (int p = 0; p < bits; ++p) {
+            uint32_t b16 = 0;
+            #pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t y = (x[q] >> p) & 0x01010101u;
+                b16 |= ((y * 0x10204080u) >> 28) << (4 * q);
+            }
+            uint32_t word = b16 << (16 * (lane & 1));
+            word |= __shfl_xor_sync(0xffffffffu, word, 1);
+            if ((lane & 1) == 0 && wd < kw) dst[(int64_t)p * ldw + wd] = word;
+        }
+    }
+}
+
 }  // namespace bnn
