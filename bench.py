@@ -56,9 +56,15 @@ INT8_PER_BF16 = 2.0
 # library's dispatch, for labelling the conv row's roofline).
 CONV_AUTO_TENSOR = True
 SM_COUNT = 148
-# 32-bit population count: 16 per clock per SM (CUDA arithmetic-instruction
-# throughput table); one POPC covers 32 binary multiply-accumulates.
+# Nominal integer-pipe rates per SM clock (CUDA arithmetic-instruction
+# throughput table): 32-bit population count 16, logic ops 64.  Used only when
+# the library's probe (bnn_probe_int_pipes) cannot run; the bench measures them.
 POPC_PER_CLK_PER_SM = 16
+LOP3_PER_CLK_PER_SM = 64
+# The carry-save popcount GEMM's instruction mix per XOR word: 8 XOR + 8 LOP3
+# (four full adders) + 1 IADD3 on the ALU pipe and 4 POPC per 8 words.
+CSA_ALU_PER_WORD = 17 / 8
+CSA_POPC_PER_WORD = 4 / 8
 
 
 # ---------------------------------------------------------------------------
@@ -99,9 +105,37 @@ def peaks():
             "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def alu_peak_mac_s(sm_mhz: float) -> float:
-    """Binary MAC/s when every SM retires 16 POPC per clock, 32 MACs each."""
-    return SM_COUNT * POPC_PER_CLK_PER_SM * 32 * sm_mhz * 1e6
+def int_pipe_peaks(bnn, sm_mhz: float, sms: int = SM_COUNT) -> dict:
+    """Integer rooflines in binary MAC/s (one 32-bit word = 32 binary MACs).
+    `popc_only`: every SM retiring POPC at its measured rate (one word each).
+    `combined`: the carry-save GEMM's mix -- a word needs CSA_ALU_PER_WORD ALU
+    ops and CSA_POPC_PER_WORD POPC, so the slower of the two pipes at their
+    measured rates bounds the word rate.  `csa_probe`: the same step measured
+    end to end on registers, for comparison."""
+    try:
+        r = bnn.bnn_probe_int_pipes(4096)
+        src = "measured (bnn_probe_int_pipes)"
+    except Exception as e:            # no device: the nominal table rates, labelled as such
+        r = {"popc": float(POPC_PER_CLK_PER_SM), "lop3": float(LOP3_PER_CLK_PER_SM), "csa_words": None}
+        src = f"nominal table rates ({type(e).__name__})"
+    hz = sms * 32 * sm_mhz * 1e6
+    words = min(r["lop3"] / CSA_ALU_PER_WORD, r["popc"] / CSA_POPC_PER_WORD)
+    return {"popc_per_clk_sm": r["popc"], "lop3_per_clk_sm": r["lop3"], "csa_words_per_clk_sm": r["csa_words"],
+            "popc_only": r["popc"] * hz, "combined": words * hz,
+            "csa_probe": r["csa_words"] * hz if r["csa_words"] else None, "source": src, "sm_mhz": sm_mhz}
+
+
+def alu_roofline(mac_s: float, ip: dict) -> dict:
+    """The popcount engine against the integer pipes (binary TMAC/s)."""
+    out = {"bound": "alu", "achieved": round(mac_s / 1e12, 2), "peak": round(ip["combined"] / 1e12, 2),
+           "unit": "binary TMAC/s", "frac": round(mac_s / ip["combined"], 4),
+           "peak_derivation": (f"{SM_COUNT} SMs x min(LOP3 {ip['lop3_per_clk_sm']:.1f}/clk / {CSA_ALU_PER_WORD}, "
+                               f"POPC {ip['popc_per_clk_sm']:.2f}/clk / {CSA_POPC_PER_WORD}) words/clk x 32 MAC x "
+                               f"{ip['sm_mhz']:.0f} MHz; rates {ip['source']}"),
+           "popc_only_peak": round(ip["popc_only"] / 1e12, 2), "popc_only_frac": round(mac_s / ip["popc_only"], 4)}
+    if ip["csa_probe"]:
+        out["csa_probe_peak"] = round(ip["csa_probe"] / 1e12, 2)
+    return out
 
 
 # Source files that determine each kernel's code (its own header + shared helpers).
@@ -122,19 +156,21 @@ KERNEL_SOURCES = {
 
 def source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES[kernel]:
+    for f in KERNEL_SOURCES[kernel.split("<")[0]]:
         h.update(open(os.path.join(ROOT, "xnor_popcount_gemm_bnn_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str):
-    """DRAM bytes per launch (read + write) from the committed ncu summary, if it
-    was captured on the kernel's current sources; else None."""
+def recorded_traffic(row: str, kernel: str):
+    """DRAM bytes per launch (read + write) of `kernel` on the workload of bench
+    row `row`, from the committed ncu summary of that row's capture, if it was
+    taken on the kernel's current sources; else None.  Entries are keyed by
+    row, so a capture of one workload is never reported for another."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
-    e = d.get(kernel)
+    e = d.get(f"{row}/{kernel}")
     if not e or e.get("source_hash") != source_hash(kernel):
         return None
     return e.get("bytes_per_launch")
@@ -214,31 +250,72 @@ def _graph(torch, fn, n):
     return g
 
 
+# Largest number of timed steps captured in one graph.
+MAX_GRAPH_STEPS = 960
+
+
 def time_steps(torch, fn, steps, warmup, period, sync):
-    """Run `warmup` untimed steps, then time exactly `steps` steps with CUDA
-    events on the current stream.  fn(i) launches step i.  Steps are replayed
-    from CUDA graphs of `period` launches (plus one graph for the remainder).
-    Returns milliseconds for the timed steps (max over ranks)."""
-    full = _graph(torch, fn, period) if steps >= period or warmup >= period else None
-    rem = steps % period
-    tail = _graph(torch, fn, rem) if rem else None
-    # warm-up: graphs of the same shapes
-    w = warmup
-    while w > 0:
-        if full is not None and w >= period:
-            full.replay(); w -= period
-        else:
-            g = _graph(torch, fn, w); g.replay(); w = 0
+    """Run at least `warmup` untimed steps, then time exactly `steps` steps
+    with CUDA events on the device.  fn(i) launches step i.
+
+    The steps run from CUDA graphs.  The first graph holds `lead` untimed
+    steps (max(period, warmup)), then the start event, then the first timed
+    steps; further graphs hold up to MAX_GRAPH_STEPS timed steps each (a
+    multiple of `period`, the rotation of the inputs), and the last one ends
+    with the end event.  The events are graph nodes (external events): the
+    start event sits on a forked branch that waits for the last lead step, so
+    the first timed step keeps its place in the launch chain (a kernel that
+    may start before its predecessor ends still does), and the timed window
+    runs from the completion of the last lead step to the completion of the
+    last timed step.  Every graph is replayed once before the host
+    synchronize and the barrier, so no first-replay upload is timed; then the
+    graphs are replayed back to back and the events read after a synchronize.
+    Returns milliseconds for the timed steps."""
+    lead = max(period, warmup)
+    chunk = max(period, MAX_GRAPH_STEPS // period * period)
+    sizes = []
+    left = steps
+    while left > 0:
+        sizes.append(min(chunk, left))
+        left -= sizes[-1]
+    start = torch.cuda.Event(enable_timing=True, external=True)
+    end = torch.cuda.Event(enable_timing=True, external=True)
+
+    # warm the stream and the library once, outside any graph
+    s0 = torch.cuda.Stream()
+    s0.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s0):
+        fn(0)
+    torch.cuda.current_stream().wait_stream(s0)
+
+    side = torch.cuda.Stream()                 # the start event's branch, created outside capture
+    graphs = []
+    i = 0
+    for gi, n in enumerate(sizes):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            main = torch.cuda.current_stream()
+            if gi == 0:
+                for _ in range(lead):
+                    fn(i)
+                    i += 1
+                side.wait_stream(main)
+                with torch.cuda.stream(side):
+                    start.record()
+            for _ in range(n):
+                fn(i)
+                i += 1
+            if gi == len(sizes) - 1:
+                end.record()
+            if gi == 0:
+                main.wait_stream(side)
+        graphs.append(g)
+    for g in graphs:                           # warm-up: lead + every timed step once, every graph uploaded
+        g.replay()
     torch.cuda.synchronize()
     sync()
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    start.record()
-    for _ in range(steps // period):
-        full.replay()
-    if tail is not None:
-        tail.replay()
-    end.record()
+    for g in graphs:
+        g.replay()
     torch.cuda.synchronize()
     ms = start.elapsed_time(end)
     sync()
@@ -345,7 +422,8 @@ def run_ours(args, torch, dist):
             "algorithmic_bytes_per_step": per_step_bytes,
             "l2": f"inputs larger than L2: {copies} rotating packed weight copies "
                   f"({copies * Ws[0].numel() * 4 / 1e6:.0f} MB > 126 MB L2)",
-            "timing": f"CUDA graphs of {copies} launches, CUDA events on the launching stream",
+            "timing": f"CUDA graphs (first: {max(copies, args.warmup)} untimed lead steps, then the timed steps, up to "
+                      f"{MAX_GRAPH_STEPS} per graph); start and end are CUDA events captured as graph nodes",
             "parallelism": "replicas" if ws == 1 else f"replicas x{ws}",
         },
         "roofline": {
@@ -354,7 +432,7 @@ def run_ours(args, torch, dist):
             "peak": pk["hbm_gbs"],
             "unit": "GB/s",
             "frac": round(achieved / pk["hbm_gbs"], 4),
-            "traffic": recorded_traffic("xnor_gemv_row128_kernel"),
+            "traffic": recorded_traffic("gemv", "xnor_gemv_row128_kernel"),
             "peak_source": pk["source"],
             "kernel": "xnor_gemv_row128_kernel",
         },
@@ -391,6 +469,8 @@ def run_ours(args, torch, dist):
     torch.cuda.empty_cache()
     if rank == 0 and not args.no_cpu_baseline and ws == 1:
         result["cpu_baseline"] = cpu_baseline_gemv(args.cpu_seconds)
+        if "rows" in result:
+            cpu_baseline_rows(result["rows"], args.cpu_row_seconds)
     return result
 
 
@@ -452,7 +532,7 @@ def e2e_gemv(torch, bnn, g, Ws, alpha, dev, steps, sync, max_over_ranks, ws):
 # the other rows
 # ---------------------------------------------------------------------------
 
-ROW_NAMES = ("pack_sign_weights", "square_gemm", "conv3x3", "mlp4", "bw_gemv", "ternary", "conv1x1")
+ROW_NAMES = ("pack_sign_weights", "square_gemm", "conv3x3", "mlp4", "bw_gemv", "ternary", "conv1x1", "multibit")
 
 
 def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws, only=None):
@@ -461,7 +541,9 @@ def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws, o
     steps = max(3, args.row_steps)
     warm = max(3, args.warmup)
     clk_mhz = pk["sm_max_mhz"]
-    alu_peak = alu_peak_mac_s(clk_mhz)
+    alu_peak = int_pipe_peaks(bnn, clk_mhz) if want & {"square_gemm", "conv3x3", "mlp4"} else None
+    if alu_peak is not None:
+        rows["int_pipes"] = {k: (round(v, 3) if isinstance(v, float) else v) for k, v in alu_peak.items()}
 
     def timed(fn, n=steps, period=None):
         return max_over_ranks(time_steps(torch, fn, n, warm, period or n, sync))
@@ -476,6 +558,7 @@ def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws, o
         ("bw_gemv", lambda: _row_bw_gemv(torch, bnn, workloads, dev, pk, rows, timed, ws)),
         ("ternary", lambda: _row_ternary(torch, bnn, workloads, dev, pk, rows, timed, steps, ws)),
         ("conv1x1", lambda: _row_conv1x1(torch, bnn, workloads, dev, pk, rows, timed, steps, ws, alu_peak)),
+        ("multibit", lambda: _row_multibit(torch, bnn, workloads, dev, pk, rows, timed, steps, ws)),
     )
     for name, run in plan:
         if name not in want:
@@ -503,12 +586,12 @@ def _row_pack(torch, bnn, workloads, dev, pk, rows, timed, steps, ws):
                                  "value": round(ws * ach, 1), "unit": "GB/s", "ms_per_step": ms / steps,
                                  "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"],
                                               "frac": round(ach / pk["hbm_gbs"], 4),
-                                              "traffic": recorded_traffic("pack_sign_rows_kernel")}}
+                                              "traffic": recorded_traffic("pack_sign_weights", "pack_sign_rows_kernel")}}
     del Wd, W_p, alpha, g
     torch.cuda.empty_cache()
 
 
-def _tensor_roofline(pk, macs_per_s, sustained):
+def _tensor_roofline(pk, macs_per_s, sustained, row=None):
     """The tensor-core engine against the int8 tensor peak (one binary MAC is
     one int8 MAC there): measured bf16 dense TFLOP/s x 2, as int8 TOPS."""
     bf16 = pk["bf16_tflops_sustained" if sustained else "bf16_tflops"]
@@ -517,7 +600,7 @@ def _tensor_roofline(pk, macs_per_s, sustained):
     return {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak_tops, 1), "unit": "TOPS (int8)",
             "frac": round(achieved / peak_tops, 4),
             "peak_derivation": f"measured bf16 {'sustained' if sustained else 'burst'} {bf16} TFLOP/s x {INT8_PER_BF16} (dense int8 / bf16)",
-            "traffic": recorded_traffic("xnor_gemm_tc_kernel")}
+            "traffic": recorded_traffic(row, "xnor_gemm_tc_kernel<TC_BINARY>") if row else None}
 
 
 def _row_square(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, clk_mhz, pk=None):
@@ -538,13 +621,11 @@ def _row_square(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, cl
             ms_s = timed(lambda i: (bnn.bnn_pack_sign(Ad, A_p), bnn.bnn_xnor_gemm(A_p, Wsq, sq.K, al, Ci, Cf)))
         mac_s = macs * steps / (ms_g * 1e-3)
         if engine == bnn.BNN_GEMM_ENGINE_TENSOR:
-            roof = _tensor_roofline(pk, mac_s, sustained=False)
+            roof = _tensor_roofline(pk, mac_s, sustained=False, row=name)
             kernel = "xnor_gemm_tc_kernel"
         else:
-            roof = {"bound": "alu", "achieved": round(mac_s / 1e12, 2), "peak": round(alu_peak / 1e12, 2),
-                    "unit": "binary TMAC/s", "frac": round(mac_s / alu_peak, 4),
-                    "peak_derivation": f"{SM_COUNT} SMs x {POPC_PER_CLK_PER_SM} POPC/clk x 32 MAC x {clk_mhz:.0f} MHz",
-                    "traffic": recorded_traffic("xnor_gemm_popc_kernel")}
+            roof = alu_roofline(mac_s, alu_peak)
+            roof["traffic"] = recorded_traffic("square_gemm_popcount", "xnor_gemm_popc_kernel")
             kernel = "xnor_gemm_popc_kernel"
         rows[name] = {
             "workload": "M=N=K=8192 packed A x packed W^T, int32 s + alpha*s fp32 out",
@@ -606,12 +687,11 @@ def _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk):
             roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                     "frac": round(ach / pk["hbm_gbs"], 4), "algorithmic_bytes": cbytes,
                     "tensor": _tensor_roofline(pk, cmac_s, sustained=False),
-                    "traffic": recorded_traffic("xnor_conv3x3_tcw_kernel")}
+                    "traffic": recorded_traffic("conv3x3", "xnor_conv3x3_tcw_kernel")}
             roof["tensor"].pop("traffic")
         else:
-            roof = {"bound": "alu", "achieved": round(cmac_s / 1e12, 2), "peak": round(alu_peak / 1e12, 2),
-                    "unit": "binary TMAC/s", "frac": round(cmac_s / alu_peak, 4),
-                    "traffic": recorded_traffic("xnor_conv3x3_kernel")}
+            roof = alu_roofline(cmac_s, alu_peak)
+            roof["traffic"] = recorded_traffic(name, "xnor_conv3x3_kernel")
         rows[name] = {
             "workload": "bf16 [64,64,56,56] -> pack NCHW -> binary 3x3 conv (64 filters, stride 1, pad 1), "
                         "alpha + affine epilogue, fp32 NCHW out",
@@ -622,7 +702,7 @@ def _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk):
             "conv_kernel_binary_tmac_s": round(cmac_s / 1e12, 2), "roofline": roof,
             "pack_nchw": {"ms": ms_pack / steps, "achieved_gbs": round(pack_gbs, 1),
                           "frac": round(pack_gbs / pk["hbm_gbs"], 4), "bytes": pbytes,
-                          "traffic": recorded_traffic("pack_sign_nchw_kernel")},
+                          "traffic": recorded_traffic("conv3x3", "pack_sign_nchw_kernel")},
             "pack_nchw_rsign": {"ms": ms_rs / steps, "achieved_gbs": round(rs_gbs, 1),
                                 "frac": round(rs_gbs / pk["hbm_gbs"], 4), "bytes": pbytes + c * 4},
             "l2": f"{R} rotating input/output sets, {rot_mb:.0f} MB"}
@@ -656,7 +736,7 @@ def _row_bw_gemv(torch, bnn, workloads, dev, pk, rows, timed, ws):
         "value": round(ws * ach, 1), "unit": "GB/s", "ms_per_step": ms / steps,
         "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"],
                      "frac": round(ach / pk["hbm_gbs"], 4), "algorithmic_bytes": b,
-                     "traffic": recorded_traffic("bw_gemv_kernel")},
+                     "traffic": recorded_traffic("bw_gemv", "bw_gemv_kernel")},
         "dependent_chain": {"value": round(ws * ach_dep, 1), "unit": "GB/s", "ms_per_step": ms_dep / steps,
                             "frac": round(ach_dep / pk["hbm_gbs"], 4)}}
     del Ws, ys, W_p, x, g
@@ -698,7 +778,7 @@ def _row_ternary(torch, bnn, workloads, dev, pk, rows, timed, steps, ws):
         "value": round(ws * ach, 1), "unit": "GB/s", "ms_per_step": ms / n,
         "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"],
                      "frac": round(ach / pk["hbm_gbs"], 4), "algorithmic_bytes": b,
-                     "traffic": recorded_traffic("ternary_gemv_i8_kernel")},
+                     "traffic": recorded_traffic("ternary_gemv", "ternary_gemv_i8_kernel")},
         "dependent_chain": {"value": round(ws * ach_dep, 1), "unit": "GB/s", "ms_per_step": ms_dep / n,
                             "frac": round(ach_dep / pk["hbm_gbs"], 4)}}
     rows["ternary_pack"] = {
@@ -707,7 +787,7 @@ def _row_ternary(torch, bnn, workloads, dev, pk, rows, timed, steps, ws):
         "value": round(ws * ach_p, 1), "unit": "GB/s", "ms_per_step": ms_p / steps,
         "roofline": {"bound": "hbm", "achieved": round(ach_p, 1), "peak": pk["hbm_gbs"],
                      "frac": round(ach_p / pk["hbm_gbs"], 4), "algorithmic_bytes": pb,
-                     "traffic": recorded_traffic("pack_ternary_kernel")}}
+                     "traffic": recorded_traffic("ternary_pack", "pack_ternary_kernel")}}
     del Qs, ys, codes, x, g, wsp
     torch.cuda.empty_cache()
 
@@ -744,9 +824,75 @@ def _row_conv1x1(torch, bnn, workloads, dev, pk, rows, timed, steps, ws, alu_pea
         "binary_tmac_s": round(macs * steps / (ms * 1e-3) / 1e12, 2),
         "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"],
                      "frac": round(ach / pk["hbm_gbs"], 4), "algorithmic_bytes": b,
-                     "traffic": recorded_traffic("xnor_conv1x1_kernel")},
+                     "traffic": recorded_traffic("conv1x1", "xnor_conv1x1_kernel")},
         "l2": f"{R} rotating packed-input/output sets"}
     del cv, Xd, Xb, Wp, al, gam, bet, out
+    torch.cuda.empty_cache()
+
+
+def _row_multibit(torch, bnn, workloads, dev, pk, rows, timed, steps, ws):
+    # --- next row: multi-bit products on bit planes (DoReFa codes, ABC-Net bases) ---
+    bs = workloads.bitserial()
+    M, K = bs.a.shape
+    N = bs.w.shape[0]
+    ld = bnn.bnn_packed_ld_words(K)
+    ad, wd = bs.a.to(dev), bs.w.to(dev)
+    A = torch.empty(M * bs.a_bits, ld, dtype=torch.int32, device=dev)
+    W = torch.empty(N * bs.w_bits, ld, dtype=torch.int32, device=dev)
+    bnn.bnn_pack_bit_planes(wd, bs.w_bits, W, K)
+    alpha = torch.full((N,), 0.25, dtype=torch.float32, device=dev)
+    # Two rotating (codes, planes, int32 out) sets, 2 x 100 MB, larger than L2 together.
+    R = 2
+    As = [A] + [A.clone() for _ in range(R - 1)]
+    Cs = [torch.empty(M, N, dtype=torch.int32, device=dev) for _ in range(R)]
+    ms_g = timed(lambda i: bnn.bnn_bitserial_gemm(As[i % R], bs.a_bits, W, bs.w_bits, K, None, Cs[i % R], None))
+    ms_p = timed(lambda i: bnn.bnn_pack_bit_planes(ad, bs.a_bits, As[i % R], K))
+    macs = M * N * K
+    mac_s = macs * steps / (ms_g * 1e-3)
+    pbytes = M * K + A.numel() * 4
+    pack_gbs = pbytes * steps / (ms_p * 1e-3) / 1e9
+    roof = _tensor_roofline(pk, mac_s, sustained=False)
+    roof["traffic"] = recorded_traffic("bitserial_gemm", "xnor_gemm_tc_kernel<TC_PLANE_CODES>")
+    rows["bitserial_gemm"] = {
+        "workload": f"DoReFa-style unsigned codes: a [{M}, {K}] {bs.a_bits}-bit x w [{N}, {K}] {bs.w_bits}-bit as bit "
+                    f"planes -> exact int32 sum_k a*w (planes folded to u8 codes, tcgen05 kind::i8 unsigned)",
+        "value": round(ws * mac_s / 1e9, 1), "unit": "code GMAC/s",
+        "plane_pair_gmac_s": round(ws * mac_s * bs.a_bits * bs.w_bits / 1e9, 1),
+        "ms_per_step": ms_g / steps, "roofline": roof,
+        "pack_bit_planes": {"ms": ms_p / steps, "achieved_gbs": round(pack_gbs, 1),
+                            "frac": round(pack_gbs / pk["hbm_gbs"], 4), "bytes": pbytes},
+        "l2": f"{R} rotating activation-plane / output sets"}
+    del bs, ad, wd, A, W, As, Cs, alpha
+    torch.cuda.empty_cache()
+
+    bb = workloads.bases()
+    J, M, K = bb.h_real.shape
+    I, N, _ = bb.b_real.shape
+    ld = bnn.bnn_packed_ld_words(K)
+    H = torch.empty(M * J, ld, dtype=torch.int32, device=dev)
+    B = torch.empty(N * I, ld, dtype=torch.int32, device=dev)
+    for j in range(J):
+        bnn.bnn_pack_sign(bb.h_real[j].to(dev), H[j::J])
+    for i in range(I):
+        bnn.bnn_pack_sign(bb.b_real[i].to(dev), B[i::I])
+    al, be = bb.alpha.to(dev), bb.beta.to(dev)
+    Ys = [torch.empty(M, N, dtype=torch.float32, device=dev) for _ in range(R)]
+    Hs = [H] + [H.clone() for _ in range(R - 1)]
+    ms_b = timed(lambda i: bnn.bnn_binary_bases_gemm(Hs[i % R], J, B, I, K, be, al, Ys[i % R]))
+    jp, ip = 1 << (J - 1).bit_length(), 1 << (I - 1).bit_length()
+    bmacs = M * N * K * J * I
+    bmac_s = bmacs * steps / (ms_b * 1e-3)
+    roof_b = _tensor_roofline(pk, bmac_s, sustained=False)
+    roof_b["traffic"] = recorded_traffic("binary_bases_gemm", "xnor_gemm_tc_kernel<TC_BASES>")
+    roof_b["note"] = (f"{J} x {I} bases run as {jp} x {ip} (zero bases fill the power-of-two tile): "
+                      f"the tensor pipe does {jp * ip / (J * I):.2f}x the algorithmic MACs")
+    rows["binary_bases_gemm"] = {
+        "workload": f"ABC-Net-style bases: {J} activation bases [{M}, {K}] x {I} weight bases [{N}, {K}], "
+                    f"Y = sum_j sum_i beta_j alpha_i[n] (H_j B_i^T) fp32",
+        "value": round(ws * bmac_s / 1e9, 1), "unit": "binary GMAC/s (all base pairs)",
+        "ms_per_step": ms_b / steps, "roofline": roof_b,
+        "l2": f"{R} rotating activation-base / output sets"}
+    del bb, H, B, Hs, Ys, al, be
     torch.cuda.empty_cache()
 
 
@@ -791,9 +937,8 @@ def _row_mlp(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk=No
         with bnn.gemm_engine(engine):
             ms_m = timed(mlp_step)
         mac_s = mmacs * steps / (ms_m * 1e-3)
-        roof = (_tensor_roofline(pk, mac_s, sustained=False) if engine == bnn.BNN_GEMM_ENGINE_TENSOR else
-                {"bound": "alu", "achieved": round(mac_s / 1e12, 2), "peak": round(alu_peak / 1e12, 2),
-                 "unit": "binary TMAC/s", "frac": round(mac_s / alu_peak, 4)})
+        roof = (_tensor_roofline(pk, mac_s, sustained=False, row=name) if engine == bnn.BNN_GEMM_ENGINE_TENSOR else
+                alu_roofline(mac_s, alu_peak))
         rows[name] = {
             "workload": "fully binary MLP, batch 4096, width 4096, 4 layers: pack fp32 input, "
                         "3 x (GEMM + folded BatchNorm sign re-pack), GEMM + alpha fp32 logits",
@@ -809,38 +954,171 @@ def _row_mlp(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk=No
 # CPU oracle timing (the baseline, never the product path)
 # ---------------------------------------------------------------------------
 
-def cpu_oracle_gemv_steps(seconds: float, max_steps: int | None = None):
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def _time_oracle(step, seconds: float, min_steps: int = 1):
+    """Run step() until `seconds` have passed (at least `min_steps` times);
+    returns (steps, elapsed seconds)."""
+    done = 0
+    t0 = time.perf_counter()
+    while True:
+        step()
+        done += 1
+        el = time.perf_counter() - t0
+        if done >= min_steps and el >= seconds:
+            return done, el
+
+
+def cpu_oracle_gemv_steps(seconds: float, threads: int | None = None):
     """Time the oracle on the decode GEMV: sign(x), the int8 +1/-1 product
     with the pre-binarised W (the oracle's analogue of pre-packed weights),
-    and alpha*s in float64.  Runs whole steps until `seconds` have passed (or
-    max_steps).  Returns (steps, elapsed_s, threads)."""
+    and alpha*s in float64.  Whole steps until `seconds` have passed.
+    Returns (steps, elapsed_s, threads used)."""
     import oracle
     import workloads
 
     g = workloads.gemv()
     wb = oracle.sign_pm1(g.W)
     al = oracle.alpha(g.W)
-    x = g.x
-    done = 0
-    t0 = time.perf_counter()
-    while True:
-        xb = oracle.sign_pm1(x)
-        s = oracle.gemv_pm1(wb, xb)
-        oracle.scaled(s, al)
-        done += 1
-        el = time.perf_counter() - t0
-        if (max_steps is not None and done >= max_steps) or (max_steps is None and el >= seconds):
-            break
-    return done, el, 1          # one output row: the oracle's outer loop runs on one thread
+    full = os.cpu_count() or 1
+    oracle.set_num_threads(threads or full)
+    try:
+        n, el = _time_oracle(lambda: oracle.scaled(oracle.gemv_pm1(wb, oracle.sign_pm1(g.x)), al), seconds)
+        used = oracle.num_threads()
+    finally:
+        oracle.set_num_threads(full)
+    return n, el, used
 
 
 def cpu_baseline_gemv(seconds: float):
+    """The oracle on all host cores (the outputs split over OpenMP threads),
+    and the same on one core beside it."""
     n, el, threads = cpu_oracle_gemv_steps(seconds)
+    n1, el1, _ = cpu_oracle_gemv_steps(max(2.0, seconds / 3), threads=1)
     return {"value": round(n * gemv_bytes() / el / 1e9, 4), "unit": "GB/s", "cores": threads,
             "kind": "oracle",
             "sample": f"{n} whole GEMV steps of the same workload ({el:.1f} s): sign(x), int8 +1/-1 "
                       f"product with the pre-binarised W, alpha*s in float64",
-            "host_cpus": os.cpu_count()}
+            "one_core": {"value": round(n1 * gemv_bytes() / el1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                         "sample": f"{n1} steps ({el1:.1f} s)"},
+            "host_cpus": os.cpu_count(), "cpu_model": cpu_model()}
+
+
+def cpu_baseline_rows(rows: dict, seconds: float) -> None:
+    """Time the oracle on a bounded sample of each measured row's workload, on
+    all host cores, and attach it as rows[name]["cpu_baseline"] in that row's
+    unit.  The samples are stated; each is the oracle's own computation of the
+    same outputs (sign, the plain +1/-1 integer product, the float64 epilogue)."""
+    import oracle
+    import workloads
+
+    full = os.cpu_count() or 1
+    oracle.set_num_threads(full)
+    model = cpu_model()
+
+    def put(name, value, unit, sample, one_core=None, numpy_only=False):
+        # The C loops (products, convolutions) run on the OpenMP threads; the
+        # add/sub GEMVs and the code product are numpy expressions on one core.
+        if name in rows and isinstance(rows[name], dict) and "error" not in rows[name]:
+            d = {"value": value, "unit": unit, "cores": 1 if numpy_only else oracle.num_threads(), "kind": "oracle",
+                 "sample": sample, "host_cpus": os.cpu_count(), "cpu_model": model}
+            if one_core is not None:
+                d["one_core"] = one_core
+            rows[name]["cpu_baseline"] = d
+
+    if "square_gemm" in rows or "square_gemm_popcount" in rows:
+        sq = workloads.square()
+        ab, wb = oracle.sign_pm1(sq.A[:8]), oracle.sign_pm1(sq.W)
+        al = oracle.alpha(sq.W)
+        R = 2
+        n, el = _time_oracle(lambda: oracle.scaled(oracle.matmul_pm1(ab[:R], wb), al), seconds)
+        v = n * R * sq.N * sq.K / el / 1e9
+        oracle.set_num_threads(1)
+        n1, el1 = _time_oracle(lambda: oracle.scaled(oracle.matmul_pm1(ab[:1], wb), al), seconds / 2)
+        oracle.set_num_threads(full)
+        one = {"value": round(n1 * sq.N * sq.K / el1 / 1e9, 4), "unit": "binary GMAC/s", "cores": 1,
+               "sample": f"{n1} x 1 row ({el1:.1f} s)"}
+        for name in ("square_gemm", "square_gemm_popcount"):
+            put(name, round(v, 4), "binary GMAC/s",
+                f"{n} x {R} rows of A (of 8192) against all 8192 rows of W, K = 8192, pre-binarised operands, "
+                f"int32 s and alpha*s in float64 ({el:.1f} s)", one)
+        del sq, ab, wb
+    if "conv3x3" in rows:
+        cv = workloads.conv()
+        x1 = cv.X[:1]
+        n, el = _time_oracle(lambda: oracle.conv3x3_affine(x1, cv.W, cv.gamma.numpy(), cv.beta.numpy()), seconds)
+        macs = 56 * 56 * 64 * 9 * 64
+        for name in ("conv3x3", "conv3x3_tensor", "conv3x3_popcount"):
+            put(name, round(n * macs / el / 1e9, 4), "binary GMAC/s",
+                f"{n} x 1 image (of 64): sign, 7-loop +1/-1 convolution, alpha and affine in float64 ({el:.1f} s)")
+        del cv
+    if "mlp4" in rows:
+        m = workloads.mlp()
+        bns = [(b.gamma.numpy(), b.beta.numpy(), b.mean.numpy(), b.var.numpy(), b.eps) for b in m.bns]
+        R = 4
+        x = m.X0[:R]
+        n, el = _time_oracle(lambda: oracle.mlp_forward(x, m.Ws, bns), seconds)
+        macs = R * 4 * 4096 * 4096
+        for name in ("mlp4", "mlp4_popcount"):
+            put(name, round(n * macs / el / 1e9, 4), "binary GMAC/s",
+                f"{n} x {R} rows (of 4096) through all 4 layers: sign of the input and of every W, +1/-1 "
+                f"products, BatchNorm sign in float64, alpha*s logits ({el:.1f} s)")
+        del m
+    if "bw_gemv" in rows:
+        g = workloads.gemv()
+        wb, al, xf = oracle.sign_pm1(g.W), oracle.alpha(g.W), oracle._f32(g.x)
+        n, el = _time_oracle(lambda: oracle.scaled(oracle.binary_weight_product(wb, xf), al), seconds)
+        put("bw_gemv", round(n * gemv_bytes() / el / 1e9, 4), "GB/s",
+            f"{n} whole steps, pre-binarised W: +x / -x sums in float64, alpha ({el:.1f} s)", numpy_only=True)
+        del g, wb
+    if "ternary_gemv" in rows:
+        t = workloads.ternary()
+        tq, gam = oracle.ternary_quantize(t.W)
+        xq = t.x.numpy()
+        n, el = _time_oracle(lambda: oracle.ternary_gemv_i8(tq, xq, gam, 1.0 / 64), seconds)
+        b = 11008 * bnn_ternary_ld(4096) * 4 + 4096 + 4 * 11008 + 8
+        put("ternary_gemv", round(n * b / el / 1e9, 4), "GB/s",
+            f"{n} whole steps with the pre-quantised ternary W: exact int64 sum of t*x, scaled ({el:.1f} s)",
+            numpy_only=True)
+        del t, tq
+    if "conv1x1" in rows:
+        cv = workloads.downsample()
+        x1 = cv.X[:1]
+        n, el = _time_oracle(lambda: oracle.conv_affine(x1, cv.W, cv.gamma.numpy(), cv.beta.numpy(), stride=2,
+                                                        pad=0), seconds)
+        b1 = 28 * 28 * 2 * 4 + 128 * 4 * 4 + 128 * 28 * 28 * 4
+        put("conv1x1", round(n * b1 / el / 1e9, 4), "GB/s",
+            f"{n} x 1 image (of 64): sign, 1x1 stride-2 +1/-1 convolution, alpha and affine ({el:.1f} s)")
+        del cv
+    if "bitserial_gemm" in rows:
+        bs = workloads.bitserial()
+        a, w = bs.a[:4].numpy(), bs.w.numpy()
+        n, el = _time_oracle(lambda: [oracle.bitserial_product(a[i:i + 1], w) for i in range(4)], seconds)
+        put("bitserial_gemm", round(n * 4 * 4096 * 4096 / el / 1e9, 4), "code GMAC/s",
+            f"{n} x 4 rows (of 4096) of the 2-bit x 2-bit code product, int64 sums of products ({el:.1f} s)",
+            numpy_only=True)
+        del bs
+    if "binary_bases_gemm" in rows:
+        bb = workloads.bases()
+        h = oracle.sign_pm1(bb.h_real[:, :2].numpy())
+        bw = oracle.sign_pm1(bb.b_real.numpy())
+        al, be = bb.alpha.numpy(), bb.beta.numpy()
+        n, el = _time_oracle(lambda: oracle.binary_bases_product(h, bw, al, be), seconds)
+        put("binary_bases_gemm", round(n * 2 * 4096 * 4096 * 9 / el / 1e9, 4), "binary GMAC/s (all base pairs)",
+            f"{n} x 2 rows (of 4096), 3 x 3 base pairs of +1/-1 products, weighted sum in float64 ({el:.1f} s)")
+        del bb
+
+
+def bnn_ternary_ld(K: int) -> int:
+    return ((K + 15) // 16 + 3) // 4 * 4
 
 
 def run_reference(args):
@@ -909,6 +1187,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--row-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--cpu-row-seconds", type=float, default=3.0)
     ap.add_argument("--no-rows", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
