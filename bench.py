@@ -148,6 +148,7 @@ KERNEL_SOURCES = {
     "pack_sign_rows_kernel": ("pack.cuh", "common.cuh"),
     "pack_sign_nchw_kernel": ("pack.cuh", "common.cuh"),
     "bw_gemv_kernel": ("bwgemv.cuh", "common.cuh"),
+    "bw_gemv_i8_kernel": ("bwgemv_i8.cuh", "common.cuh"),
     "ternary_gemv_i8_kernel": ("ternary.cuh", "common.cuh"),
     "xnor_conv1x1_kernel": ("conv1x1.cuh", "conv.cuh", "gemm_popc.cuh", "common.cuh"),
     "pack_ternary_kernel": ("ternary.cuh", "common.cuh"),
@@ -555,7 +556,7 @@ def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws, o
                                             pk)),
         ("conv3x3", lambda: _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk)),
         ("mlp4", lambda: _row_mlp(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk)),
-        ("bw_gemv", lambda: _row_bw_gemv(torch, bnn, workloads, dev, pk, rows, timed, ws)),
+        ("bw_gemv", lambda: _row_bw_gemv(torch, bnn, workloads, dev, pk, rows, timed, ws, steps)),
         ("ternary", lambda: _row_ternary(torch, bnn, workloads, dev, pk, rows, timed, steps, ws)),
         ("conv1x1", lambda: _row_conv1x1(torch, bnn, workloads, dev, pk, rows, timed, steps, ws, alu_peak)),
         ("multibit", lambda: _row_multibit(torch, bnn, workloads, dev, pk, rows, timed, steps, ws)),
@@ -710,7 +711,7 @@ def _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk):
     torch.cuda.empty_cache()
 
 
-def _row_bw_gemv(torch, bnn, workloads, dev, pk, rows, timed, ws):
+def _row_bw_gemv(torch, bnn, workloads, dev, pk, rows, timed, ws, row_steps):
     # --- next row: binary weights x real (bf16) activations, the decode shape ---
     g = workloads.gemv()
     copies = max(2, math.ceil(2 * L2_BYTES / gemv_bytes()) + 1)
@@ -721,7 +722,7 @@ def _row_bw_gemv(torch, bnn, workloads, dev, pk, rows, timed, ws):
     Ws = [W_p] + [W_p.clone() for _ in range(copies - 1)]
     ys = [torch.empty(g.N, dtype=torch.float32, device=dev) for _ in range(copies)]
     x = g.x.to(dev)
-    steps = 48 * copies
+    steps = max(row_steps, 20) * copies            # 960 steps by default: each copy streamed 20 times
     all_flags = bnn.BNN_GEMV_WEIGHTS_STATIC | bnn.BNN_GEMV_INPUTS_STATIC | bnn.BNN_GEMV_OUTPUT_FREE
     ms = timed(lambda i: bnn.bnn_binary_weight_gemv(Ws[i % copies], x, g.K, alpha, ys[i % copies], flags=all_flags),
                n=steps, period=copies)
@@ -739,7 +740,27 @@ def _row_bw_gemv(torch, bnn, workloads, dev, pk, rows, timed, ws):
                      "traffic": recorded_traffic("bw_gemv", "bw_gemv_kernel")},
         "dependent_chain": {"value": round(ws * ach_dep, 1), "unit": "GB/s", "ms_per_step": ms_dep / steps,
                             "frac": round(ach_dep / pk["hbm_gbs"], 4)}}
-    del Ws, ys, W_p, x, g
+    # the same weights x INT8 activations (x of the ternary workload, scale 1/64)
+    t = workloads.ternary()
+    xq = t.x.to(dev)
+    xsc = torch.full((1,), 1.0 / 64, dtype=torch.float32, device=dev)
+    ms8 = timed(lambda i: bnn.bnn_binary_weight_gemv_i8(Ws[i % copies], xq, g.K, alpha, xsc, None, ys[i % copies],
+                                                        flags=all_flags), n=steps, period=copies)
+    ms8_dep = timed(lambda i: bnn.bnn_binary_weight_gemv_i8(Ws[i % copies], xq, g.K, alpha, xsc, None, ys[0],
+                                                            flags=bnn.BNN_GEMV_WEIGHTS_STATIC), n=steps, period=copies)
+    b8 = Ws[0].numel() * 4 + 4 * g.N + g.K + 4 * g.N + 4        # packed W + alpha + int8 x + fp32 y + x scale
+    a8 = b8 * steps / (ms8 * 1e-3) / 1e9
+    a8_dep = b8 * steps / (ms8_dep * 1e-3) / 1e9
+    rows["bw_gemv_i8"] = {
+        "workload": "binary weights x INT8 activations: packed W [11008, 4096], x int8 [4096] with its scale, "
+                    "exact int32 sum of +-x, alpha * x_scale fp32 y; independent steps over 48 rotating weight copies",
+        "value": round(ws * a8, 1), "unit": "GB/s", "ms_per_step": ms8 / steps,
+        "roofline": {"bound": "hbm", "achieved": round(a8, 1), "peak": pk["hbm_gbs"],
+                     "frac": round(a8 / pk["hbm_gbs"], 4), "algorithmic_bytes": b8,
+                     "traffic": recorded_traffic("bw_gemv_i8", "bw_gemv_i8_kernel")},
+        "dependent_chain": {"value": round(ws * a8_dep, 1), "unit": "GB/s", "ms_per_step": ms8_dep / steps,
+                            "frac": round(a8_dep / pk["hbm_gbs"], 4)}}
+    del Ws, ys, W_p, x, g, xq, t
     torch.cuda.empty_cache()
 
 
@@ -763,7 +784,7 @@ def _row_ternary(torch, bnn, workloads, dev, pk, rows, timed, steps, ws):
     ys = [torch.empty(g.N, dtype=torch.float32, device=dev) for _ in range(copies)]
     x = g.x.to(dev)
     xsc = torch.full((1,), 1.0 / 64, dtype=torch.float32, device=dev)
-    n = 48 * copies
+    n = max(steps, 20) * copies
     all_flags = bnn.BNN_GEMV_WEIGHTS_STATIC | bnn.BNN_GEMV_INPUTS_STATIC | bnn.BNN_GEMV_OUTPUT_FREE
     ms = timed(lambda i: bnn.bnn_ternary_gemv_i8(Qs[i % copies], x, g.K, y_f32=ys[i % copies], w_scale=gam,
                                                  x_scale=xsc, flags=all_flags), n=n, period=copies)
@@ -1017,6 +1038,8 @@ def cpu_baseline_rows(rows: dict, seconds: float) -> None:
     all host cores, and attach it as rows[name]["cpu_baseline"] in that row's
     unit.  The samples are stated; each is the oracle's own computation of the
     same outputs (sign, the plain +1/-1 integer product, the float64 epilogue)."""
+    import numpy as np
+
     import oracle
     import workloads
 
@@ -1079,6 +1102,15 @@ def cpu_baseline_rows(rows: dict, seconds: float) -> None:
         put("bw_gemv", round(n * gemv_bytes() / el / 1e9, 4), "GB/s",
             f"{n} whole steps, pre-binarised W: +x / -x sums in float64, alpha ({el:.1f} s)", numpy_only=True)
         del g, wb
+    if "bw_gemv_i8" in rows:
+        g, t = workloads.gemv(), workloads.ternary()
+        wb, al, xq = oracle.sign_pm1(g.W), oracle.alpha(g.W), t.x.numpy().astype(np.float64)
+        n, el = _time_oracle(lambda: al * (1.0 / 64) * oracle.binary_weight_product(wb, xq), seconds)
+        b8 = 11008 * 128 * 4 + 4 * 11008 + 4096 + 4 * 11008 + 4
+        put("bw_gemv_i8", round(n * b8 / el / 1e9, 4), "GB/s",
+            f"{n} whole steps, pre-binarised W: +x / -x sums of the int8 x, alpha * x_scale ({el:.1f} s)",
+            numpy_only=True)
+        del g, t, wb
     if "ternary_gemv" in rows:
         t = workloads.ternary()
         tq, gam = oracle.ternary_quantize(t.W)

@@ -320,10 +320,16 @@ bnn_status bnn_xnor_gemv_ex(const uint32_t* W, int64_t ldw, const void* x, bnn_d
  *   alpha    device fp32 [N], required; y device fp32 [N].
  *   flags    as for bnn_xnor_gemv_ex (BNN_GEMV_WEIGHTS_STATIC,
  *            BNN_GEMV_INPUTS_STATIC, BNN_GEMV_OUTPUT_FREE).
+ *   N        <= 2^30.
  * Accumulation is fp32: a 16-entry table of +-x0 +-x1 +-x2 +-x3 per group
- * of 4 elements, then one lookup and one add per 4 weights, 4 accumulators
- * per lane, and 16 partial sums per row.
- *   Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (K too large), CUDA. */
+ * of 4 elements, then one lookup and one add per 4 weights on 4 accumulators
+ * per lane (each lane holds 128 consecutive weights of a row per pass), and
+ * the lanes of a row added by a butterfly of shuffles.
+ *   Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (K too large), CUDA.  A
+ *   launch whose shared-memory window is laid out where the 32 KiB-aligned
+ *   table does not fit (not expected on sm_100) records
+ *   BNN_ERR_UNSUPPORTED in the device flag (bnn_device_error) and writes
+ *   nothing. */
 bnn_status bnn_binary_weight_gemv(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt,
                                   int64_t N, int64_t K, const float* alpha, float* y,
                                   uint32_t flags, bnn_stream_t stream);
@@ -338,6 +344,29 @@ bnn_status bnn_binary_weight_gemv(const uint32_t* W, int64_t ldw, const void* x,
  * give ~1.58 bits (log2 3) as the information content and ~0.2 bytes per
  * weight for packed ternary; the 2-bit code is the densest layout whose
  * weights can be addressed with shifts and masks. */
+
+/* bnn_binary_weight_gemv_i8 -- binary weights times an INT8 activation vector:
+ *   acc[n]   = sum_k sign(W[n,k]) * x[k]              (exact, int32)
+ *   y_f32[n] = fp32( fp32(a_n * x_scale) * fp32(acc[n]) ),
+ *   a_n = alpha[n] (alpha_per_row = 1, eq. (1): one scale per output row) or
+ *   alpha[0] (alpha_per_row = 0, eq. (8): one scale for the whole matrix).
+ * ("Extreme Quantization: Binary, Ternary & 1-bit LLMs", Binary Neural
+ * Networks, eq. (1)-(2): each term is +x_k or -x_k; BitNet: activations
+ * quantised to INT8, weights binarised with the matrix scale of eq. (8).)
+ * The pages give no activation quantiser: x arrives as int8 with its scale.
+ *   W        device, packed [N, ldw] as produced by bnn_pack_sign (16-B
+ *            aligned, ldw % 4 == 0, pad bits zero); kw = bnn_packed_ld_words(K)
+ *            <= 1536 (K <= 49152).
+ *   x        device int8 [K]; x_scale device fp32 [1] or NULL (1.0).
+ *   alpha    device fp32 [N] or [1] (see alpha_per_row); required with y_f32.
+ *   y_i32, y_f32  device [N]; either may be NULL, not both.  N <= 2^30.
+ *   flags    as for bnn_xnor_gemv_ex.
+ * Per 4 weights the kernel does one shift, one byte permute and one dp4a
+ * against x staged in that byte order; the int32 result is exact.
+ *   Errors: INVALID_ARG, ALIGNMENT, UNSUPPORTED (K too large), CUDA. */
+bnn_status bnn_binary_weight_gemv_i8(const uint32_t* W, int64_t ldw, const int8_t* x, int64_t N, int64_t K,
+                                     const float* alpha, int alpha_per_row, const float* x_scale, int32_t* y_i32,
+                                     float* y_f32, uint32_t flags, bnn_stream_t stream);
 
 /* Words in one ternary row of K weights; -1 for K < 1. */
 int64_t bnn_ternary_ld_words(int64_t K);

@@ -114,3 +114,83 @@ def test_bw_gemv_store_order_and_independent_calls():
         check(ys[l], Ws[l], xs[l], K)
     assert torch.equal(shared, ys[L - 1])
     assert_no_device_error()
+
+
+# ---------------------------------------------------------------------------
+# binary weights x INT8 activations (BitNet section: INT8 activations; eq. (1)
+# per-row alpha, eq. (8) one alpha for the matrix).  acc is exact; y_f32 takes
+# three roundings: fp32(alpha), fp32(alpha * x_scale), the product with
+# fp32(acc) -- |y - y_ref| <= 4u |y_ref| covers them with the fp32 alpha used.
+# ---------------------------------------------------------------------------
+
+def run_i8(W, xq, K, per_row=True, flags=0, x_scale=0.03125, x_dev=None):
+    d = dev()
+    N = W.shape[0]
+    Wp = bnn.empty_packed(N, K, d)
+    al = torch.empty(N, dtype=torch.float32, device=d)
+    bnn.bnn_pack_sign(W.to(d), Wp, al)
+    if not per_row:
+        al = torch.tensor([oracle.ternary_gamma(W)], dtype=torch.float32, device=d)
+    xs = torch.tensor([x_scale], dtype=torch.float32, device=d)
+    yi = torch.full((N,), -7, dtype=torch.int32, device=d)
+    yf = torch.full((N,), float("nan"), dtype=torch.float32, device=d)
+    bnn.bnn_binary_weight_gemv_i8(Wp, xq.to(d) if x_dev is None else x_dev, K, al, xs, yi, yf, flags=flags)
+    torch.cuda.synchronize()
+    return yi, yf, al.cpu().numpy().astype(np.float64)
+
+
+def check_i8(yi, yf, W, xq, alpha_used, x_scale=0.03125):
+    acc = oracle.binary_weight_product(oracle.sign_pm1(W), xq.numpy().astype(np.float64))
+    assert np.array_equal(yi.cpu().numpy().astype(np.float64), acc)
+    a = alpha_used if alpha_used.size == acc.size else np.full(acc.size, alpha_used[0])
+    y_ref = a * x_scale * acc
+    err = np.abs(yf.cpu().numpy().astype(np.float64) - y_ref)
+    assert np.all(err <= 4 * U * np.abs(y_ref)), f"max rel err {np.max(err / np.maximum(np.abs(y_ref), 1e-300))}"
+
+
+@pytest.mark.parametrize("N,K", [(1, 1), (5, 31), (64, 1000), (65, 33), (300, 4096), (100, 4100), (129, 8192),
+                                 (33, 12288), (7, 49152), (1000, 2100)])
+@pytest.mark.parametrize("flags", [0, 1, 3, 7])
+def test_bw_gemv_i8_shapes(N, K, flags):
+    W = workloads.normal((N, K), 1.0, 3 * N + K)
+    xq = workloads.int8_uniform((K,), K + 11)
+    yi, yf, a = run_i8(W, xq, K, flags=flags)
+    check_i8(yi, yf, W, xq, a)
+    assert_no_device_error()
+
+
+def test_bw_gemv_i8_decode_workload():
+    """The decode shape: packed W [11008, 4096] from N(0, 0.02), x int8 [4096]."""
+    g, t = workloads.gemv(), workloads.ternary()
+    yi, yf, a = run_i8(g.W, t.x, g.K, flags=bnn.BNN_GEMV_WEIGHTS_STATIC)
+    check_i8(yi, yf, g.W, t.x, a)
+    assert_no_device_error()
+
+
+def test_bw_gemv_i8_one_alpha_for_the_matrix():
+    """eq. (8): one scale ||W||_1 / (n m) for every row."""
+    N, K = 777, 3000
+    W = workloads.normal((N, K), 0.5, 91)
+    xq = workloads.int8_uniform((K,), 92)
+    yi, yf, a = run_i8(W, xq, K, per_row=False)
+    assert a.size == 1
+    check_i8(yi, yf, W, xq, a)
+
+
+def test_bw_gemv_i8_extremes_and_unaligned_x():
+    """x = -128 everywhere and W all +1 / all -1 rows: |acc| = 128 K; x read
+    from an unaligned address takes the byte path."""
+    N, K = 64, 4096
+    W = torch.ones(N, K)
+    W[1::2] = -1.0
+    xq = torch.full((K,), -128, dtype=torch.int8)
+    yi, yf, a = run_i8(W, xq, K)
+    check_i8(yi, yf, W, xq, a)
+    assert int(yi[0]) == -128 * K and int(yi[1]) == 128 * K
+    xq2 = workloads.int8_uniform((K,), 5)
+    buf = torch.zeros(K + 1, dtype=torch.int8, device=dev())
+    buf[1:] = xq2.to(dev())
+    W2 = workloads.normal((N, K), 1.0, 6)
+    yi2, yf2, a2 = run_i8(W2, xq2, K, x_dev=buf[1:])
+    check_i8(yi2, yf2, W2, xq2, a2)
+    assert_no_device_error()

@@ -51,7 +51,7 @@ EXPORTS = (
     "bnn_binary_weight_gemv", "bnn_ternary_ld_words", "bnn_ternary_workspace_bytes", "bnn_ternary_pack",
     "bnn_ternary_gemv_i8", "bnn_ternary_pack_noalloc", "bnn_pack_sign_rsign", "bnn_pack_sign_nchw_rsign",
     "bnn_binary_conv1x1_fused", "bnn_probe_int_pipes", "bnn_pack_bit_planes", "bnn_bitserial_gemm",
-    "bnn_binary_bases_gemm",
+    "bnn_binary_bases_gemm", "bnn_binary_weight_gemv_i8",
 )
 
 
@@ -106,6 +106,7 @@ def _load() -> ctypes.CDLL:
         "bnn_pack_bit_planes": (i32, [p, i64, i64, i64, i32, p, i64, p]),
         "bnn_bitserial_gemm": (i32, [p, i64, i32, p, i64, i32, i64, i64, i64, p, p, i64, p, i64, p]),
         "bnn_binary_bases_gemm": (i32, [p, i64, i32, p, i64, i32, i64, i64, i64, p, p, i64, p, i64, p]),
+        "bnn_binary_weight_gemv_i8": (i32, [p, i64, p, i64, i64, p, i32, p, p, p, ctypes.c_uint32, p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -314,6 +315,21 @@ def bnn_binary_weight_gemv(W: torch.Tensor, x: torch.Tensor, K: Optional[int], a
     _check("bnn_binary_weight_gemv", _lib.bnn_binary_weight_gemv(
         _ptr(W), _ld(W), _ptr(x), _dtype(x), N, K, _ptr(alpha), _ptr(y), int(flags), _stream(stream)))
 
+
+
+def bnn_binary_weight_gemv_i8(W: torch.Tensor, x: torch.Tensor, K: Optional[int] = None,
+                              alpha: Optional[torch.Tensor] = None, x_scale: Optional[torch.Tensor] = None,
+                              y_i32: Optional[torch.Tensor] = None, y_f32: Optional[torch.Tensor] = None,
+                              flags: int = 0, stream=None) -> None:
+    """Packed binary W [N, ld] x int8 x [K]; alpha [N] (per row) or [1] (one scale for the matrix)."""
+    assert x.dtype == torch.int8
+    K = x.shape[-1] if K is None else int(K)
+    per_row = 1 if (alpha is None or alpha.numel() == W.shape[0]) else 0
+    if alpha is not None and not per_row:
+        assert alpha.numel() == 1
+    _check("bnn_binary_weight_gemv_i8", _lib.bnn_binary_weight_gemv_i8(
+        _ptr(W), _ld(W), _ptr(x), W.shape[0], K, _ptr(alpha), per_row, _ptr(x_scale), _ptr(y_i32), _ptr(y_f32),
+        int(flags), _stream(stream)))
 
 
 def bnn_ternary_pack(w: torch.Tensor, codes: torch.Tensor, gamma_out: Optional[torch.Tensor] = None,

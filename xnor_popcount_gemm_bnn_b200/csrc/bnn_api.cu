@@ -22,6 +22,7 @@
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "bwgemv.cuh"
+#include "bwgemv_i8.cuh"
 #include "pack.cuh"
 #include "probe.cuh"
 #include "ternary.cuh"
@@ -575,7 +576,7 @@ bnn_status bnn_binary_weight_gemv(const uint32_t* W, int64_t ldw, const void* x,
     constexpr uint32_t kAll = BNN_GEMV_WEIGHTS_STATIC | BNN_GEMV_INPUTS_STATIC | BNN_GEMV_OUTPUT_FREE;
     if ((flags & ~kAll) != 0) return BNN_ERR_INVALID_ARG;
     if (x == nullptr || alpha == nullptr || y == nullptr) return BNN_ERR_INVALID_ARG;
-    if (N < 0 || K < 1 || N > INT_MAX || K > INT_MAX / 2) return BNN_ERR_INVALID_ARG;
+    if (N < 0 || K < 1 || N > INT_MAX / 2 || K > INT_MAX / 2) return BNN_ERR_INVALID_ARG;
     if (x_dt != BNN_F32 && x_dt != BNN_BF16) return BNN_ERR_INVALID_ARG;
     const int64_t kw = packed_ld_words(K);
     bnn_status st = check_packed_operand(W, ldw, kw);
@@ -719,6 +720,46 @@ bnn_status bnn_binary_bases_gemm(const uint32_t* H, int64_t ldh, int J, const ui
     const int64_t grid = std::min<int64_t>(tiles_m * tiles_n, sm_count());
     bnn::xnor_gemm_tc_kernel<bnn::TC_BASES><<<(unsigned)grid, THREADS, SMEM_BYTES, as_cuda(stream)>>>(
         tmA, tmW, (int)M, (int)N, (int)K, (int)kw, (int)tiles_m, (int)tiles_n, bnn::GemmEpilogue{}, pl);
+    return launch_status();
+}
+
+bnn_status bnn_binary_weight_gemv_i8(const uint32_t* W, int64_t ldw, const int8_t* x, int64_t N, int64_t K,
+                                     const float* alpha, int alpha_per_row, const float* x_scale, int32_t* y_i32,
+                                     float* y_f32, uint32_t flags, bnn_stream_t stream) {
+    constexpr uint32_t kAll = BNN_GEMV_WEIGHTS_STATIC | BNN_GEMV_INPUTS_STATIC | BNN_GEMV_OUTPUT_FREE;
+    if ((flags & ~kAll) != 0) return BNN_ERR_INVALID_ARG;
+    if (x == nullptr || (y_i32 == nullptr && y_f32 == nullptr)) return BNN_ERR_INVALID_ARG;
+    if (y_f32 != nullptr && alpha == nullptr) return BNN_ERR_INVALID_ARG;
+    if (alpha_per_row != 0 && alpha_per_row != 1) return BNN_ERR_INVALID_ARG;
+    if (N < 0 || K < 1 || N > INT_MAX / 2) return BNN_ERR_INVALID_ARG;
+    const int64_t kw = packed_ld_words(K);
+    bnn_status st = check_packed_operand(W, ldw, kw);
+    if (st != BNN_OK) return st;
+    if (kw > bnn::bwi8::MAX_KW) return BNN_ERR_UNSUPPORTED;
+    if ((y_i32 != nullptr && !aligned(y_i32, 4)) || (y_f32 != nullptr && !aligned(y_f32, 4)) ||
+        (alpha != nullptr && !aligned(alpha, 4)) || (x_scale != nullptr && !aligned(x_scale, 4)))
+        return BNN_ERR_ALIGNMENT;
+    if (N == 0) return BNN_OK;
+    int64_t lpr = 1;
+    while (lpr < 32 && lpr < kw / 4) lpr <<= 1;
+    const int64_t rows_per_cta = (int64_t)bnn::bwi8::WARPS * bnn::bwi8::U * (32 / lpr);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)ceil_div(N, rows_per_cta));
+    cfg.blockDim = dim3(bnn::bwi8::THREADS);
+    cfg.dynamicSmemBytes = (size_t)kw * 32;
+    cfg.stream = as_cuda(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const int prefetch = (flags & BNN_GEMV_WEIGHTS_STATIC) ? 1 : 0;
+    const int xstatic = (flags & BNN_GEMV_INPUTS_STATIC) ? 1 : 0;
+    const int dependent = flags == kAll ? 2 : 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, bnn::bw_gemv_i8_kernel<bnn::bwi8::U>, W, ldw, x, (int)N, (int)K,
+                                             (int)kw, alpha, alpha_per_row, x_scale, y_i32, y_f32, prefetch, xstatic,
+                                             dependent);
+    if (e != cudaSuccess) return BNN_ERR_CUDA;
     return launch_status();
 }
 
