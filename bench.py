@@ -451,8 +451,8 @@ def run_ours(args, torch, dist):
             "value": round(ws * side_steps * per_step_bytes / (ms_dep * 1e-3) / 1e9, 2), "unit": "GB/s",
             "steps": side_steps, "ms_per_step": ms_dep / side_steps,
             "frac": round(side_steps * per_step_bytes / (ms_dep * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
-            "note": "BNN_GEMV_WEIGHTS_STATIC only: x and alpha are read after the wait for the previous "
-                    "kernel, as when x is the previous layer's output"},
+            "note": "BNN_GEMV_WEIGHTS_STATIC only: W and alpha are read before, x after the wait for the "
+                    "previous kernel, as when x is the previous layer's output"},
         "gemv_default_flags": {
             "value": round(ws * side_steps * per_step_bytes / (ms_plain * 1e-3) / 1e9, 2), "unit": "GB/s",
             "steps": side_steps, "ms_per_step": ms_plain / side_steps,

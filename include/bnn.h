@@ -278,22 +278,23 @@ bnn_status bnn_xnor_gemv(const uint32_t* W, int64_t ldw, const void* x, bnn_dtyp
 
 /* Flags of bnn_xnor_gemv_ex. */
 typedef enum bnn_gemv_flags {
-    BNN_GEMV_WEIGHTS_STATIC = 1,  /* W is not written by any work still in flight on the stream */
-    BNN_GEMV_INPUTS_STATIC = 2,   /* x and alpha are not written by any work still in flight */
+    BNN_GEMV_WEIGHTS_STATIC = 1,  /* W and its scale (alpha, w_scale) are not written by any work still in flight */
+    BNN_GEMV_INPUTS_STATIC = 2,   /* x (and x_scale) are not written by any work still in flight */
     BNN_GEMV_OUTPUT_FREE = 4      /* y is neither read nor written by any work still in flight */
 } bnn_gemv_flags;
 
 /* bnn_xnor_gemv_ex -- bnn_xnor_gemv with flags.  Both calls launch the kernel
  * with programmatic dependent launch: it may be scheduled while the previous
  * kernel on the stream is still running, and it waits for that kernel to
- * complete before it reads x or alpha or writes y.  With
- * BNN_GEMV_WEIGHTS_STATIC the loads of W are issued before that wait, so
- * consecutive GEMVs over resident weights (one decode step through many
- * layers) stream their weights back to back.  The caller guarantees that no
- * earlier work on the stream that may still be running writes W; otherwise
- * pass 0 (then equivalent to bnn_xnor_gemv).  With BNN_GEMV_INPUTS_STATIC
- * (the caller guarantees the same for x and alpha) x is packed before the
- * wait as well; with both flags the whole product is computed before it and
+ * complete before it reads x, alpha or W or writes y.  With
+ * BNN_GEMV_WEIGHTS_STATIC the loads of W and of alpha (the weights' per-row
+ * scale, eq. (1)) are issued before that wait, so consecutive GEMVs over
+ * resident weights (one decode step through many layers) stream their
+ * weights back to back and only x waits.  The caller guarantees that no
+ * earlier work on the stream that may still be running writes W or alpha;
+ * otherwise pass 0 (then equivalent to bnn_xnor_gemv).  With
+ * BNN_GEMV_INPUTS_STATIC (the caller guarantees the same for x) x is packed
+ * before the wait as well; with both flags the whole product is computed before it and
  * only the store of y waits, so GEMVs over independent, resident inputs
  * overlap their prologues with the previous kernel.  With all three flags
  * the call depends on nothing still in flight: it computes and stores y

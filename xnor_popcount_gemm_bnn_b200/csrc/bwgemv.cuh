@@ -30,9 +30,9 @@
 // and two adds.
 //
 // Launched with programmatic dependent launch, like the XNOR GEMV: with static
-// weights the first W loads precede the wait for the previous grid, with
-// static inputs the table and the product do too (only the store waits), and
-// with all three flags only the exit waits.
+// weights the first W and alpha loads precede the wait for the previous grid,
+// with static inputs the table and the product do too (only the store waits),
+// and with all three flags only the exit waits.
 #pragma once
 
 #include "common.cuh"
@@ -56,11 +56,6 @@ constexpr int TABLE_ALIGN = 32768;
 // window starts below 32 KiB - x slice, checked in the kernel), the table.
 __host__ __device__ constexpr int smem_bytes(int kw) { return TABLE_ALIGN + passes(kw) * PASS_BYTES; }
 
-// Byte offset of entry m of group t (lane 0) inside a pass.
-__device__ __forceinline__ uint32_t entry_offset(int t, int m) {
-    const uint32_t P = (uint32_t)t >> 1;
-    return (t & 1) ? (32768u | (P << 7) | ((uint32_t)m << 11)) : (((uint32_t)m << 7) | (P << 11));
-}
 }  // namespace bwg
 
 // Two lookups of the pair P: v holds nibble 2P at bits 7..10 and nibble 2P+1
@@ -122,13 +117,19 @@ bw_gemv_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restrict
     grid_dependents_launch();
 
     uint4 v[U];
+    float al[U];                                              // alpha of the rows this lane stores (li == 0)
     // Rows of a batch: row0 + u * rpi for row0 = first row of the warp's batch + sub.
+    // The first pass also reads the rows' alpha: the weights and their scale
+    // are read together.
+    const int64_t row_step = (int64_t)rpi * ldw;               // words between the rows of one load pass
     auto load_pass = [&](int row0, int p) {
         const int c = li + lpr * p;
+        const uint32_t* wp = W + (int64_t)row0 * ldw + 4 * c;
         #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int r = row0 + u * rpi;
-            v[u] = (r < N && c < nch) ? ldg_stream_v4(W + (int64_t)r * ldw + 4 * c) : make_uint4(0u, 0u, 0u, 0u);
+            v[u] = (row0 + u * rpi < N && c < nch) ? ldg_stream_v4(wp) : make_uint4(0u, 0u, 0u, 0u);
+            wp += row_step;
+            if (p == 0) al[u] = (li == 0 && row0 + u * rpi < N) ? alpha[row0 + u * rpi] : 0.0f;
         }
     };
     // Per pass: the pass's slice of x -> shared fp32 (coalesced 16-byte loads
@@ -177,9 +178,19 @@ bw_gemv_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restrict
                     p01[b] = ((b & 1) ? -e[0] : e[0]) + ((b & 2) ? -e[1] : e[1]);
                     p23[b] = ((b & 1) ? -e[2] : e[2]) + ((b & 2) ? -e[3] : e[3]);
                 }
-                #pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    *reinterpret_cast<float*>(tp + entry_offset(t, m)) = p01[m & 3] + p23[m >> 2];
+                // Entry m of an even group at (m << 7) | (P << 11), of an odd
+                // group at 32768 | (P << 7) | (m << 11): one base per group and
+                // compile-time offsets per entry.  (t's parity is warp-uniform.)
+                const uint32_t P = (uint32_t)t >> 1;
+                if (t & 1) {
+                    float* ge = reinterpret_cast<float*>(tp + (32768u | (P << 7)));
+                    #pragma unroll
+                    for (int m = 0; m < 16; ++m) ge[m * 512] = p01[m & 3] + p23[m >> 2];
+                } else {
+                    float* ge = reinterpret_cast<float*>(tp + (P << 11));
+                    #pragma unroll
+                    for (int m = 0; m < 16; ++m) ge[m * 32] = p01[m & 3] + p23[m >> 2];
+                }
             }
         }
     };
@@ -216,7 +227,12 @@ bw_gemv_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restrict
         #pragma unroll
         for (int u = 0; u < U; ++u) {
             float s = (acc[u][0] + acc[u][1]) + (acc[u][2] + acc[u][3]);
-            for (int off = lpr >> 1; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+            if (lpr == 32) {                                  // a row spans the warp (K > 2048)
+                #pragma unroll
+                for (int off = 16; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+            } else {
+                for (int off = lpr >> 1; off >= 1; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+            }
             acc[u][0] = s;
         }
         if (first && dependent == 1 && late_wait) grid_dependency_wait();
@@ -225,7 +241,7 @@ bw_gemv_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restrict
             #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int r = row0 + u * rpi;
-                if (r < N) y[r] = alpha[r] * acc[u][0];
+                if (r < N) y[r] = al[u] * acc[u][0];
             }
         }
     }

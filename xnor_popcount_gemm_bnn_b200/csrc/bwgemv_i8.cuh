@@ -53,12 +53,16 @@ bw_gemv_i8_kernel(const uint32_t* __restrict__ W, int64_t ldw, const int8_t* __r
     grid_dependents_launch();
 
     uint4 v[U];
+    float al[U];                                               // alpha of the rows this lane stores (li == 0)
+    // The first pass also reads the rows' alpha (the weights and their scale
+    // are read together).
     auto load_pass = [&](int row0, int p) {
         const int c = li + lpr * p;
         #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int r = row0 + u * rpi;
             v[u] = (r < N && c < nch) ? ldg_stream_v4(W + (int64_t)r * ldw + 4 * c) : make_uint4(0u, 0u, 0u, 0u);
+            if (p == 0) al[u] = (li == 0 && y_f32 != nullptr && r < N) ? alpha[alpha_per_row ? r : 0] : 0.0f;
         }
     };
     // Word w of x (elements 32 w .. 32 w + 31, zero past K) -> 8 permuted
@@ -164,7 +168,7 @@ bw_gemv_i8_kernel(const uint32_t* __restrict__ W, int64_t ldw, const int8_t* __r
                 const int r = row0 + u * rpi;
                 if (r < N) {
                     if (y_i32 != nullptr) y_i32[r] = acc[u];
-                    if (y_f32 != nullptr) y_f32[r] = (alpha[alpha_per_row ? r : 0] * xs) * (float)acc[u];
+                    if (y_f32 != nullptr) y_f32[r] = (al[u] * xs) * (float)acc[u];
                 }
             }
         }

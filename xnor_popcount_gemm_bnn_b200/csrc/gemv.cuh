@@ -16,10 +16,10 @@
 //  * Row sums: redux.sync (one instruction) when LPR = 32, else a shuffle tree.
 //  * Launched with programmatic dependent launch: the grid may start while
 //    the previous kernel on the stream finishes, and waits for it
-//    (griddepcontrol.wait) before reading x or alpha and before writing y.
-//    When the caller declares the weights static (nothing still in flight on
-//    the stream writes W), the W loads are issued before that wait, so the
-//    weight stream of consecutive GEMVs runs back to back.
+//    (griddepcontrol.wait) before reading x and before writing y.  When the
+//    caller declares the weights static (nothing still in flight on the stream
+//    writes W or alpha), the W and alpha loads are issued before that wait, so
+//    the weight stream of consecutive GEMVs runs back to back.
 #pragma once
 
 #include "common.cuh"
@@ -124,11 +124,15 @@ xnor_gemv_row128_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* _
     grid_dependents_launch();
     const int nch = kw / 4;
     uint4 v[U];
+    float al[U];                                      // alpha of the rows this lane stores (lane 0)
+    // The weights and their per-row scale, read together.
     auto load_w = [&]() {
         #pragma unroll
-        for (int u = 0; u < U; ++u)
+        for (int u = 0; u < U; ++u) {
             v[u] = (rows[u] < N && lane < nch) ? ldg_stream_v4(W + (int64_t)rows[u] * ldw + 4 * lane)
                                                : make_uint4(0u, 0u, 0u, 0u);
+            al[u] = (lane == 0 && y_f32 != nullptr && rows[u] < N) ? alpha[rows[u]] : 0.0f;
+        }
     };
     auto pack_x = [&]() {
         const int nfull = K / E;                      // whole vectors inside x
@@ -175,7 +179,7 @@ xnor_gemv_row128_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* _
         if (lane == 0 && r < N) {
             const int32_t sv = K - 2 * (int32_t)d[u];
             if (y_i32 != nullptr) y_i32[r] = sv;
-            if (y_f32 != nullptr) y_f32[r] = alpha[r] * (float)sv;
+            if (y_f32 != nullptr) y_f32[r] = al[u] * (float)sv;
         }
     }
     // dependent == 2: the call touches nothing that work in flight uses; it
@@ -207,6 +211,7 @@ xnor_gemv_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restri
     grid_dependents_launch();
 
     uint4 v[U];
+    float al[U];                                      // alpha of the rows this lane stores (li == 0)
     auto load_pass = [&](int t) {
         const int c = li + LPR * t;
         #pragma unroll
@@ -216,6 +221,13 @@ xnor_gemv_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restri
                                           : make_uint4(0u, 0u, 0u, 0u);
         }
     };
+    auto load_alpha = [&]() {
+        #pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int r = row0 + u * RPI;
+            al[u] = (li == 0 && y_f32 != nullptr && r < N) ? alpha[r] : 0.0f;
+        }
+    };
 
     // The weight stream does not depend on x.  With static weights it starts
     // before the dependency wait (overlapping the previous kernel's tail);
@@ -223,9 +235,15 @@ xnor_gemv_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restri
     // `dependent` is always 1 from the host.  Keeping the wait behind a
     // run-time branch puts it in its own basic block, so the instruction
     // scheduler cannot hoist it above the weight loads issued before it.
-    if constexpr (PREFETCH) load_pass(0);
+    if constexpr (PREFETCH) {
+        load_pass(0);
+        load_alpha();
+    }
     if (dependent) grid_dependency_wait();
-    if constexpr (!PREFETCH) load_pass(0);
+    if constexpr (!PREFETCH) {
+        load_pass(0);
+        load_alpha();
+    }
 
     gemv_pack_x<XT, VEC>(x, K, kw, xs);
     __syncthreads();
@@ -263,7 +281,7 @@ xnor_gemv_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restri
         if (li == 0 && r < N) {
             const int32_t sv = K - 2 * (int32_t)dd;
             if (y_i32 != nullptr) y_i32[r] = sv;
-            if (y_f32 != nullptr) y_f32[r] = alpha[r] * (float)sv;
+            if (y_f32 != nullptr) y_f32[r] = al[u] * (float)sv;
         }
     }
 }

@@ -306,16 +306,21 @@ ternary_gemv_i8_kernel(const uint32_t* __restrict__ Q, int64_t ldq, const int8_t
             }
         }
     };
-    float scale = 1.0f;
+    // w_scale belongs to the weights (read with them), x_scale to x.
+    float scale = 1.0f, wsc = 1.0f;
+    auto load_weights = [&]() {
+        load_pass(0);
+        if (y_f32 != nullptr && w_scale != nullptr) wsc = *w_scale;
+    };
     auto stage = [&]() {
         stage_x_transposed(x, K, nw, x_vec, txs);
-        if (y_f32 != nullptr) scale = (w_scale != nullptr ? *w_scale : 1.0f) * (x_scale != nullptr ? *x_scale : 1.0f);
+        if (y_f32 != nullptr) scale = wsc * (x_scale != nullptr ? *x_scale : 1.0f);
     };
     const bool late_wait = prefetch && xstatic;
-    if (prefetch) load_pass(0);
+    if (prefetch) load_weights();
     if (xstatic) stage();
     if (dependent == 1 && !late_wait) grid_dependency_wait();
-    if (!prefetch) load_pass(0);
+    if (!prefetch) load_weights();
     if (!xstatic) stage();
 
     int acc[U][2];
