@@ -298,9 +298,11 @@ typedef enum bnn_gemv_flags {
  * only the store of y waits, so GEMVs over independent, resident inputs
  * overlap their prologues with the previous kernel.  With all three flags
  * the call depends on nothing still in flight: it computes and stores y
- * while the previous kernel may still run, and waits for that kernel only
- * before it exits (so stream order stays transitive for later work); GEMVs
- * over independent inputs and outputs then run concurrently.  A flag is a
+ * while the previous kernel may still run; one block of the launch waits for
+ * that kernel before it exits, so the launch completes only after it (stream
+ * order stays transitive for later work), and the other blocks leave as soon
+ * as their rows are stored.  GEMVs over independent inputs and outputs then
+ * run concurrently.  A flag is a
  * permission: shapes served by the general kernel (rows of more than 128
  * words, or x not 16-byte aligned) ignore BNN_GEMV_INPUTS_STATIC and
  * BNN_GEMV_OUTPUT_FREE.

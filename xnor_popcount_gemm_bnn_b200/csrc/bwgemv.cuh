@@ -32,7 +32,7 @@
 // Launched with programmatic dependent launch, like the XNOR GEMV: with static
 // weights the first W and alpha loads precede the wait for the previous grid,
 // with static inputs the table and the product do too (only the store waits),
-// and with all three flags only the exit waits.
+// and with all three flags only block 0 waits, before it exits.
 #pragma once
 
 #include "common.cuh"
@@ -216,13 +216,15 @@ bw_gemv_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restrict
         for (int p = 0; p < np; ++p) {
             if (!first || p > 0) load_pass(row0, p);
             const uint32_t lb = lane_base + (uint32_t)p * PASS_BYTES;
+            // Rows innermost, so that consecutive adds belong to different rows.
             #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                bw_lookup_word<0>(v[u].x, lb, acc[u]);
-                bw_lookup_word<1>(v[u].y, lb, acc[u]);
-                bw_lookup_word<2>(v[u].z, lb, acc[u]);
-                bw_lookup_word<3>(v[u].w, lb, acc[u]);
-            }
+            for (int u = 0; u < U; ++u) bw_lookup_word<0>(v[u].x, lb, acc[u]);
+            #pragma unroll
+            for (int u = 0; u < U; ++u) bw_lookup_word<1>(v[u].y, lb, acc[u]);
+            #pragma unroll
+            for (int u = 0; u < U; ++u) bw_lookup_word<2>(v[u].z, lb, acc[u]);
+            #pragma unroll
+            for (int u = 0; u < U; ++u) bw_lookup_word<3>(v[u].w, lb, acc[u]);
         }
         #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -245,7 +247,7 @@ bw_gemv_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* __restrict
             }
         }
     }
-    if (dependent == 2) grid_dependency_wait();
+    if (dependent == 2) exit_after_previous_grid();
 }
 
 }  // namespace bnn

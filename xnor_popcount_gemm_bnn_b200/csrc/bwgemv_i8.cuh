@@ -173,7 +173,7 @@ bw_gemv_i8_kernel(const uint32_t* __restrict__ W, int64_t ldw, const int8_t* __r
             }
         }
     }
-    if (dependent == 2) grid_dependency_wait();
+    if (dependent == 2) exit_after_previous_grid();
 }
 
 }  // namespace bnn

@@ -168,6 +168,15 @@ __device__ __forceinline__ void grid_dependency_wait() {
 __device__ __forceinline__ void grid_dependents_launch() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+// End of a launch that depends on nothing still in flight: its completion
+// must still imply the previous grid's, so that stream order stays
+// transitive for later work.  A grid completes when its last block exits, so
+// it is enough that one block (block 0) waits for the previous grid before
+// exiting; the other blocks leave as soon as their work is stored and free
+// their slots for the launches behind them.
+__device__ __forceinline__ void exit_after_previous_grid() {
+    if (blockIdx.x == 0) grid_dependency_wait();
+}
 
 // Real-valued element access for the two input dtypes.
 __device__ __forceinline__ float to_float(float v) { return v; }

@@ -182,10 +182,10 @@ xnor_gemv_row128_kernel(const uint32_t* __restrict__ W, int64_t ldw, const XT* _
             if (y_f32 != nullptr) y_f32[r] = al[u] * (float)sv;
         }
     }
-    // dependent == 2: the call touches nothing that work in flight uses; it
-    // still waits for the previous grid before it exits, so that its own
-    // completion implies that grid's (stream order stays transitive).
-    if (dependent == 2) grid_dependency_wait();
+    // dependent == 2: the call touches nothing that work in flight uses; its
+    // completion must still imply the previous grid's (stream order stays
+    // transitive), which one block waiting before it exits is enough for.
+    if (dependent == 2) exit_after_previous_grid();
 }
 
 // SINGLE: every row fits in one warp-wide pass (nchunks <= LPR).

@@ -355,7 +355,7 @@ ternary_gemv_i8_kernel(const uint32_t* __restrict__ Q, int64_t ldq, const int8_t
             }
         }
     }
-    if (dependent == 2) grid_dependency_wait();
+    if (dependent == 2) exit_after_previous_grid();
 }
 
 }  // namespace bnn
