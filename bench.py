@@ -152,6 +152,8 @@ KERNEL_SOURCES = {
     "ternary_gemv_i8_kernel": ("ternary.cuh", "common.cuh"),
     "xnor_conv1x1_kernel": ("conv1x1.cuh", "conv.cuh", "gemm_popc.cuh", "common.cuh"),
     "pack_ternary_kernel": ("ternary.cuh", "common.cuh"),
+    "pack_bit_planes_kernel": ("pack.cuh", "common.cuh"),
+    "xnor_gemv_chain_kernel": ("chain.cuh", "common.cuh"),
 }
 
 
@@ -533,7 +535,8 @@ def e2e_gemv(torch, bnn, g, Ws, alpha, dev, steps, sync, max_over_ranks, ws):
 # the other rows
 # ---------------------------------------------------------------------------
 
-ROW_NAMES = ("pack_sign_weights", "square_gemm", "conv3x3", "mlp4", "bw_gemv", "ternary", "conv1x1", "multibit")
+ROW_NAMES = ("pack_sign_weights", "square_gemm", "conv3x3", "mlp4", "bw_gemv", "ternary", "conv1x1", "multibit",
+             "decode_chain")
 
 
 def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws, only=None):
@@ -560,6 +563,7 @@ def bench_rows(torch, bnn, workloads, dev, pk, args, sync, max_over_ranks, ws, o
         ("ternary", lambda: _row_ternary(torch, bnn, workloads, dev, pk, rows, timed, steps, ws)),
         ("conv1x1", lambda: _row_conv1x1(torch, bnn, workloads, dev, pk, rows, timed, steps, ws, alu_peak)),
         ("multibit", lambda: _row_multibit(torch, bnn, workloads, dev, pk, rows, timed, steps, ws)),
+        ("decode_chain", lambda: _row_chain(torch, bnn, workloads, dev, pk, rows, timed, steps, ws)),
     )
     for name, run in plan:
         if name not in want:
@@ -917,6 +921,59 @@ def _row_multibit(torch, bnn, workloads, dev, pk, rows, timed, steps, ws):
     torch.cuda.empty_cache()
 
 
+def chain_bytes(c) -> int:
+    """Algorithmic bytes of one decode step through a binary layer chain: every
+    layer's packed W once, thresholds and modes of the hidden layers, alpha of
+    the last, the real input and the fp32 output."""
+    total, L = 0, len(c.Ws)
+    for l, W in enumerate(c.Ws):
+        N, K = W.shape
+        total += N * (((K + 31) // 32 + 3) // 4 * 4) * 4
+        total += N * 5 if l < L - 1 else N * 4
+    return total + c.x0.numel() * c.x0.element_size() + c.Ws[-1].shape[0] * 4
+
+
+def _row_chain(torch, bnn, workloads, dev, pk, rows, timed, steps, ws):
+    # --- next row: one decode step through a fully binary MLP, all layers in one launch ---
+    c = workloads.chain()
+    L = len(c.Ws)
+    packed, layers = [], []
+    for l, W in enumerate(c.Ws):
+        N, K = W.shape
+        Wp = bnn.empty_packed(N, K, dev)
+        alpha = torch.empty(N, dtype=torch.float32, device=dev)
+        bnn.bnn_pack_sign(W.to(dev), Wp, alpha)
+        if l < L - 1:
+            bn = c.bns[l]
+            thr, mode = bnn.bnn_fold_bn_threshold(alpha.cpu(), bn.gamma, bn.beta, bn.mean, bn.var, bn.eps, K)
+            layers.append({"popc_thresh": thr.to(dev), "thresh_mode": mode.to(dev)})
+        else:
+            layers.append({"alpha": alpha})
+        packed.append(Wp)
+    b = chain_bytes(c)
+    copies = max(2, math.ceil(2 * L2_BYTES / b) + 1)
+    sets = []
+    for i in range(copies):
+        sets.append(bnn.chain_layers([dict(ly, W=(Wp if i == 0 else Wp.clone())) for ly, Wp in zip(layers, packed)]))
+    x = c.x0.to(dev)
+    y = torch.empty(c.Ws[-1].shape[0], dtype=torch.float32, device=dev)
+    wsp = bnn.gemv_chain_workspace(dev)
+    n = max(steps, 20) * copies
+    ms = timed(lambda i: bnn.bnn_xnor_gemv_chain(sets[i % copies], x, wsp, y_f32=y), n=n, period=copies)
+    ach = b * n / (ms * 1e-3) / 1e9
+    rows["decode_chain"] = {
+        "workload": "batch-1 decode step through a fully binary MLP in one launch: x bf16 [4096] signed, 8 layers "
+                    "alternating [11008, 4096] / [4096, 11008] packed W, BatchNorm folded into popcount thresholds "
+                    f"between layers, alpha-scaled fp32 out; independent steps over {copies} rotating weight sets",
+        "value": round(ws * ach, 1), "unit": "GB/s", "ms_per_step": ms / n, "layers": L,
+        "us_per_layer": round(ms / n * 1e3 / L, 3),
+        "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": pk["hbm_gbs"],
+                     "frac": round(ach / pk["hbm_gbs"], 4), "algorithmic_bytes": b,
+                     "traffic": recorded_traffic("decode_chain", "xnor_gemv_chain_kernel")}}
+    del sets, packed, layers, x, y
+    torch.cuda.empty_cache()
+
+
 def _row_mlp(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk=None):
     # --- MLP: pack input, 3 x (GEMM + folded-BN re-pack), GEMM + alpha ---
     m = workloads.mlp()
@@ -1147,6 +1204,29 @@ def cpu_baseline_rows(rows: dict, seconds: float) -> None:
         put("binary_bases_gemm", round(n * 2 * 4096 * 4096 * 9 / el / 1e9, 4), "binary GMAC/s (all base pairs)",
             f"{n} x 2 rows (of 4096), 3 x 3 base pairs of +1/-1 products, weighted sum in float64 ({el:.1f} s)")
         del bb
+
+
+    if "decode_chain" in rows:
+        c = workloads.chain()
+        bns = [(b.gamma.numpy(), b.beta.numpy(), b.mean.numpy(), b.var.numpy(), b.eps) for b in c.bns]
+        wb = [oracle.sign_pm1(W) for W in c.Ws]
+        als = [oracle.alpha(W) for W in c.Ws]
+
+        def forward():
+            # the oracle's MLP forward at batch 1, with every W binarised once up front
+            a = oracle.sign_pm1(c.x0)[None, :]
+            for l in range(len(wb)):
+                s_ = oracle.matmul_pm1(a, wb[l])
+                if l < len(wb) - 1:
+                    g_, be, mu, var, eps = bns[l]
+                    a = oracle.bn_sign(s_, als[l].astype(np.float32), g_, be, mu, var, eps)
+                else:
+                    oracle.scaled(s_, als[l])
+        n, el = _time_oracle(forward, seconds)
+        put("decode_chain", round(n * chain_bytes(c) / el / 1e9, 4), "GB/s",
+            f"{n} whole steps through all 8 layers with pre-binarised W: +1/-1 products, BatchNorm sign in "
+            f"float64, alpha*s logits ({el:.1f} s)")
+        del c, wb
 
 
 def bnn_ternary_ld(K: int) -> int:

@@ -597,6 +597,58 @@ bnn_status bnn_binary_bases_gemm(const uint32_t* H, int64_t ldh, int J, const ui
                                  int64_t M, int64_t N, int64_t K, const float* beta, const float* alpha,
                                  int64_t lda_alpha, float* Y, int64_t ldy, bnn_stream_t stream);
 
+/* One layer of bnn_xnor_gemv_chain.  The layer's K is the previous layer's N
+ * (the first layer's is the call's K). */
+typedef struct bnn_chain_layer {
+    const uint32_t* W;            /* device, packed [N, ldw] as by bnn_pack_sign (16-B aligned, ldw % 4 == 0) */
+    int64_t ldw;                  /* >= bnn_packed_ld_words(K) */
+    int64_t N;                    /* outputs, 1 .. 2^24; a hidden layer's N is <= 16384 */
+    const int32_t* popc_thresh;   /* hidden layers: device int32 [N] (bnn_fold_bn_threshold) */
+    const int8_t* thresh_mode;    /* hidden layers: device int8 [N] */
+    const float* alpha;           /* last layer: device fp32 [N], needed for y_f32 */
+} bnn_chain_layer;
+
+/* Size, in uint32 words, of the workspace of bnn_xnor_gemv_chain. */
+int64_t bnn_gemv_chain_workspace_words(void);
+
+/* bnn_xnor_gemv_chain -- a batch-1 fully binary layer chain, the decode step
+ * of a binary network, in ONE launch:
+ *   a_0 = sign(x)                                  (bit 1 = x < 0)
+ *   d_l = popcount(W_l[n, :] XOR a_l)              (eq. (6): s = K_l - 2 d_l)
+ *   a_{l+1}[n] = THRESHOLD_PACK bit of d_l[n]      (hidden layers: BatchNorm of
+ *                alpha * s followed by sign, folded by bnn_fold_bn_threshold)
+ *   last layer: y_i32[n] = s, y_f32[n] = alpha[n] * s (eq. (1)).
+ * Each layer is the XNOR GEMV of bnn_xnor_gemv ("Extreme Quantization:
+ * Binary, Ternary & 1-bit LLMs", eq. (4) and (6); "First Principles: Why
+ * Binary Ops Can Be Exponentially Faster", "Bandwidth math": a batch-1 layer
+ * streams its packed weights once).  The layers run in one cooperative launch
+ * (every block resident): no launch or grid barrier between layers, the
+ * weights of later layers are fetched into L2 while earlier layers run, and
+ * a layer's blocks start as soon as the previous layer's output words are
+ * complete.  Results are those of the same chain of bnn_binary_linear_fused
+ * calls at M = 1 (THRESHOLD_PACK for hidden layers).
+ *   layers    HOST array [L] of bnn_chain_layer; 1 <= L <= 16.
+ *   x         device [K] fp32 or bf16 (x_dt), element-aligned; 1 <= K <= 16384,
+ *             and every layer's K <= 16384 (packed rows of at most 512 words).
+ *   y_i32     device int32 [N_{L-1}] or NULL; y_f32 device fp32 [N_{L-1}] or
+ *             NULL; at least one.
+ *   acts      device uint32 [L-1, ld_acts] or NULL: the packed input of every
+ *             layer after the first (row l-1 = a_l, bnn_pack_sign layout);
+ *             ld_acts >= bnn_packed_ld_words of every hidden N.
+ *   workspace device uint32 [bnn_gemv_chain_workspace_words()], 16-byte
+ *             aligned, ZERO before its first use; every call leaves it zero
+ *             again (also after a timeout).  Calls that may run concurrently
+ *             need separate workspaces.
+ *   A block that waits more than about a second for the previous layer's
+ *   output gives up and sets the device error flag (bnn_device_error then
+ *   reports BNN_ERR_DEVICE_TIMEOUT); outputs are then undefined.
+ *   Errors: INVALID_ARG (null or out-of-range argument, missing thresholds
+ *   or alpha, small ld_acts), ALIGNMENT, UNSUPPORTED (a layer K > 16384),
+ *   CUDA (launch failed, e.g. the grid cannot be co-resident). */
+bnn_status bnn_xnor_gemv_chain(const bnn_chain_layer* layers, int32_t L, const void* x, bnn_dtype x_dt, int64_t K,
+                               int32_t* y_i32, float* y_f32, uint32_t* acts, int64_t ld_acts, uint32_t* workspace,
+                               bnn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -267,3 +267,41 @@ def test_header_constants_match_binding():
         m = re.search(rf"\b{name}\s*=\s*(\d+)", text)
         assert m, name
         assert int(m.group(1)) == getattr(bnn, name), name
+
+
+def test_gemv_chain_rejects_bad_arguments():
+    f = L.bnn_xnor_gemv_chain
+    assert bnn.bnn_gemv_chain_workspace_words() == 16 + 4 * 512 * 2
+
+    def layers(*specs):       # (W, ldw, N, popc_thresh, thresh_mode, alpha)
+        arr = (bnn.bnn_chain_layer * len(specs))()
+        for i, s in enumerate(specs):
+            arr[i] = bnn.bnn_chain_layer(*s)
+        return arr
+
+    W, T, M, A = 0x10000, 0x20000, 0x30000, 0x40000
+    good = layers((W, 32, 64, T, M, None), (W, 4, 10, None, None, A))   # K = 1000 -> 64 -> 10
+    INV, ALN, UNS = bnn.BNN_ERR_INVALID_ARG, bnn.BNN_ERR_ALIGNMENT, bnn.BNN_ERR_UNSUPPORTED
+
+    def call(arr=good, n=2, x=FAKE, dt=0, K=1000, yi=FAKE, yf=FAKE, acts=NULL, ld_acts=0, ws=FAKE):
+        return f(arr, n, x, dt, K, yi, yf, acts, ld_acts, ws, NULL)
+
+    assert call(arr=NULL) == INV
+    assert call(n=0) == INV
+    assert call(n=17) == INV
+    assert call(x=NULL) == INV
+    assert call(dt=7) == INV
+    assert call(K=0) == INV
+    assert call(yi=NULL, yf=NULL) == INV
+    assert call(ws=NULL) == INV
+    assert call(ws=FAKE_ODD) == ALN
+    assert call(acts=FAKE, ld_acts=2) == INV                                  # hidden N = 64 needs 4 words
+    assert call(arr=layers((W, 32, 0, T, M, None), (W, 4, 10, None, None, A))) == INV       # N = 0
+    assert call(arr=layers((W, 32, 64, NULL, M, None), (W, 4, 10, None, None, A))) == INV   # no thresholds
+    assert call(arr=layers((W, 32, 64, T, NULL, None), (W, 4, 10, None, None, A))) == INV
+    assert call(arr=layers((W, 32, 64, T, M, None), (W, 4, 10, None, None, None))) == INV   # y_f32 needs alpha
+    assert call(arr=layers((W, 28, 64, T, M, None), (W, 4, 10, None, None, A))) == INV      # ldw < words of K
+    assert call(arr=layers((W, 34, 64, T, M, None), (W, 4, 10, None, None, A))) == ALN      # ldw % 4
+    assert call(arr=layers((0x10008, 32, 64, T, M, None), (W, 4, 10, None, None, A))) == ALN
+    assert call(arr=layers((W, 516, 64, T, M, None), (W, 4, 10, None, None, A)), K=16385) == UNS
+    assert call(arr=layers((W, 32, 16385, T, M, None), (W, 516, 10, None, None, A))) == UNS  # hidden N > 16384

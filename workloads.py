@@ -35,6 +35,10 @@ fully binary MLP):
              draws N(0, 1) [J, 4096, 4096] seed 22 and [I, 4096, 4096] seed 23 (their
              signs are the bases), alpha_i[n] |N(0, 0.3)| + 0.01 seed 24, beta_j
              |N(0, 0.5)| + 0.05 seed 25 (ABC-Net-style weighted binary bases).
+* ``chain``  a batch-1 decode step through a fully binary MLP: x bf16 [4096] N(0, 1)
+             seed 30; 8 layers alternating up [11008, 4096] and down [4096, 11008]
+             (the decode projection's shape and weight law, N(0, 0.02), seeds 31..);
+             BatchNorm after every hidden layer drawn as for ``mlp`` (seeds 50..).
 """
 from __future__ import annotations
 
@@ -257,3 +261,21 @@ def random_with_edges(rows: int, K: int, seed: int, dtype=torch.float32,
     if dtype == torch.bfloat16:
         t = t.to(torch.bfloat16)
     return t
+
+
+@dataclass
+class Chain:
+    x0: torch.Tensor                    # [K0] real input (bf16 or fp32)
+    Ws: list = field(default_factory=list)   # fp32 [N_l, K_l], K_l = N_{l-1}
+    bns: list = field(default_factory=list)  # BatchNormParams after each hidden layer
+
+
+def chain(widths=(11008, 4096) * 4, K0=4096, x_seed=30, w_seed0=31, bn_seed0=50, w_std=0.02,
+          x_dtype=torch.bfloat16) -> Chain:
+    x0 = normal((K0,), 1.0, x_seed, dtype=x_dtype)
+    Ws, k = [], K0
+    for l, n in enumerate(widths):
+        Ws.append(normal((n, k), w_std, w_seed0 + l))
+        k = n
+    bns = [batchnorm_params(n, bn_seed0 + l) for l, n in enumerate(widths[:-1])]
+    return Chain(x0, Ws, bns)

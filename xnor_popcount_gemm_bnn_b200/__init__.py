@@ -51,7 +51,8 @@ EXPORTS = (
     "bnn_binary_weight_gemv", "bnn_ternary_ld_words", "bnn_ternary_workspace_bytes", "bnn_ternary_pack",
     "bnn_ternary_gemv_i8", "bnn_ternary_pack_noalloc", "bnn_pack_sign_rsign", "bnn_pack_sign_nchw_rsign",
     "bnn_binary_conv1x1_fused", "bnn_probe_int_pipes", "bnn_pack_bit_planes", "bnn_bitserial_gemm",
-    "bnn_binary_bases_gemm", "bnn_binary_weight_gemv_i8",
+    "bnn_binary_bases_gemm", "bnn_binary_weight_gemv_i8", "bnn_gemv_chain_workspace_words",
+    "bnn_xnor_gemv_chain",
 )
 
 
@@ -65,6 +66,11 @@ class bnn_epilogue(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("alpha", ctypes.c_void_p), ("gamma", ctypes.c_void_p),
                 ("beta", ctypes.c_void_p), ("popc_thresh", ctypes.c_void_p),
                 ("thresh_mode", ctypes.c_void_p)]
+
+
+class bnn_chain_layer(ctypes.Structure):
+    _fields_ = [("W", ctypes.c_void_p), ("ldw", ctypes.c_int64), ("N", ctypes.c_int64),
+                ("popc_thresh", ctypes.c_void_p), ("thresh_mode", ctypes.c_void_p), ("alpha", ctypes.c_void_p)]
 
 
 def _load() -> ctypes.CDLL:
@@ -107,6 +113,8 @@ def _load() -> ctypes.CDLL:
         "bnn_bitserial_gemm": (i32, [p, i64, i32, p, i64, i32, i64, i64, i64, p, p, i64, p, i64, p]),
         "bnn_binary_bases_gemm": (i32, [p, i64, i32, p, i64, i32, i64, i64, i64, p, p, i64, p, i64, p]),
         "bnn_binary_weight_gemv_i8": (i32, [p, i64, p, i64, i64, p, i32, p, p, p, ctypes.c_uint32, p]),
+        "bnn_gemv_chain_workspace_words": (i64, []),
+        "bnn_xnor_gemv_chain": (i32, [ctypes.POINTER(bnn_chain_layer), i32, p, i32, i64, p, p, p, i64, p, p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -384,6 +392,42 @@ def bnn_ternary_gemv_i8(codes: torch.Tensor, x: torch.Tensor, K: Optional[int] =
     _check("bnn_ternary_gemv_i8", _lib.bnn_ternary_gemv_i8(
         _ptr(codes), _ld(codes), _ptr(x), N, K, _ptr(w_scale), _ptr(x_scale), _ptr(y_i32), _ptr(y_f32),
         int(flags), _stream(stream)))
+
+def bnn_gemv_chain_workspace_words() -> int:
+    return int(_lib.bnn_gemv_chain_workspace_words())
+
+
+def gemv_chain_workspace(device) -> torch.Tensor:
+    """A zeroed workspace for bnn_xnor_gemv_chain (each call leaves it zero)."""
+    return torch.zeros(bnn_gemv_chain_workspace_words(), dtype=torch.int32, device=device)
+
+
+def chain_layers(layers) -> ctypes.Array:
+    """bnn_chain_layer array from dicts with keys W (packed [N, ld]), and
+    popc_thresh / thresh_mode (hidden layers) or alpha (last layer); N defaults
+    to W.shape[0].  The array keeps references to the tensors."""
+    arr = (bnn_chain_layer * len(layers))()
+    keep = []
+    for i, ly in enumerate(layers):
+        W = ly["W"]
+        arr[i] = bnn_chain_layer(W.data_ptr(), _ld(W), int(ly.get("N", W.shape[0])), _ptr(ly.get("popc_thresh")),
+                                 _ptr(ly.get("thresh_mode")), _ptr(ly.get("alpha")))
+        keep.append(ly)
+    arr._keep = keep
+    return arr
+
+
+def bnn_xnor_gemv_chain(layers, x: torch.Tensor, workspace: torch.Tensor, K: Optional[int] = None,
+                        y_i32: Optional[torch.Tensor] = None, y_f32: Optional[torch.Tensor] = None,
+                        acts: Optional[torch.Tensor] = None, stream=None) -> None:
+    """A batch-1 fully binary layer chain in one launch; ``layers`` is a list
+    of dicts (see chain_layers) or an array it returned."""
+    arr = layers if isinstance(layers, ctypes.Array) else chain_layers(layers)
+    K = x.shape[-1] if K is None else int(K)
+    _check("bnn_xnor_gemv_chain", _lib.bnn_xnor_gemv_chain(
+        arr, len(arr), _ptr(x), _dtype(x), K, _ptr(y_i32), _ptr(y_f32), _ptr(acts),
+        _ld(acts) if acts is not None else 0, _ptr(workspace), _stream(stream)))
+
 
 def make_epilogue(mode: int, alpha=None, gamma=None, beta=None, popc_thresh=None,
                   thresh_mode=None) -> bnn_epilogue:

@@ -1,8 +1,8 @@
 // libbnn.so: the C ABI declared in include/bnn.h.  Host code here only checks
 // arguments, encodes TMA descriptors, picks launch shapes and launches on the
 // caller's stream; every step of the computation runs in the kernels of
-// pack.cuh, gemm_popc.cuh, gemm_tc.cuh, gemv.cuh, bwgemv.cuh, conv.cuh, conv_tc.cuh
-// and ternary.cuh.
+// pack.cuh, gemm_popc.cuh, gemm_tc.cuh, gemv.cuh, chain.cuh, bwgemv.cuh, conv.cuh,
+// conv_tc.cuh and ternary.cuh.
 #include <cudaTypedefs.h>
 
 #include <atomic>
@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "bnn.h"
+#include "chain.cuh"
 #include "common.cuh"
 #include "conv.cuh"
 #include "conv_tc.cuh"
@@ -1170,6 +1171,101 @@ bnn_status bnn_binary_conv1x1_fused(const uint32_t* X_nhwc_bits, int64_t n, int6
                                 bnn::xnor_conv1x1_kernel<16, BNN_OUT_AFFINE_F32>);
     }
 #undef BNN_C1_CASE
+}
+
+int64_t bnn_gemv_chain_workspace_words(void) { return bnn::chain::WORKSPACE_WORDS; }
+
+bnn_status bnn_xnor_gemv_chain(const bnn_chain_layer* layers, int32_t L, const void* x, bnn_dtype x_dt, int64_t K,
+                               int32_t* y_i32, float* y_f32, uint32_t* acts, int64_t ld_acts, uint32_t* workspace,
+                               bnn_stream_t stream) {
+    using namespace bnn::chain;
+    if (layers == nullptr || L < 1 || L > MAX_LAYERS || x == nullptr || workspace == nullptr) return BNN_ERR_INVALID_ARG;
+    if (x_dt != BNN_F32 && x_dt != BNN_BF16) return BNN_ERR_INVALID_ARG;
+    if (y_i32 == nullptr && y_f32 == nullptr) return BNN_ERR_INVALID_ARG;
+    if (K < 1) return BNN_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16) || !aligned(x, x_dt == BNN_F32 ? 4 : 2)) return BNN_ERR_ALIGNMENT;
+    if (acts != nullptr && !aligned(acts, 4)) return BNN_ERR_ALIGNMENT;
+
+    // every argument is checked before the first CUDA call
+    int64_t k = K, hidden_kw = 0;
+    for (int l = 0; l < L; ++l) {
+        const bnn_chain_layer& c = layers[l];
+        const bool hidden = l < L - 1;
+        if (c.N < 1 || c.N > (int64_t(1) << 24)) return BNN_ERR_INVALID_ARG;
+        if (k > (int64_t)MAX_KW * 32) return BNN_ERR_UNSUPPORTED;
+        const bnn_status st = check_packed_operand(c.W, c.ldw, packed_ld_words(k));
+        if (st != BNN_OK) return st;
+        if (hidden && (c.popc_thresh == nullptr || c.thresh_mode == nullptr)) return BNN_ERR_INVALID_ARG;
+        if (!hidden && y_f32 != nullptr && c.alpha == nullptr) return BNN_ERR_INVALID_ARG;
+        if (hidden) hidden_kw = std::max(hidden_kw, packed_ld_words(c.N));
+        k = c.N;
+    }
+    if (acts != nullptr && ld_acts < hidden_kw) return BNN_ERR_INVALID_ARG;
+
+    auto kern = x_dt == BNN_F32 ? bnn::xnor_gemv_chain_kernel<float> : bnn::xnor_gemv_chain_kernel<__nv_bfloat16>;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, THREADS, 0) != cudaSuccess || per_sm < 1)
+        return BNN_ERR_CUDA;
+    const int64_t G = (int64_t)std::min(per_sm, 2) * sm_count();
+
+    bnn::ChainArgs args{};
+    k = K;
+    for (int l = 0; l < L; ++l) {
+        const bnn_chain_layer& c = layers[l];
+        const int64_t kw = packed_ld_words(k);
+        bnn::ChainLayer& ly = args.layer[l];
+        ly.W = c.W;
+        ly.thr = c.popc_thresh;
+        ly.mode = c.thresh_mode;
+        ly.alpha = c.alpha;
+        ly.ldw = c.ldw;
+        ly.N = (int)c.N;
+        ly.K = (int)k;
+        ly.kw = (int)kw;
+        ly.rc = (int)ceil_div(c.N, G);
+        ly.active = (int)ceil_div(c.N, ly.rc);
+        const int nch = (int)(kw / 4);
+        int lpr = 1;
+        while (lpr < 32 && lpr < nch) lpr <<= 1;
+        ly.lpr = lpr;
+        ly.lpr_log2 = 0;
+        while ((1 << ly.lpr_log2) < lpr) ++ly.lpr_log2;
+        ly.np = (int)ceil_div(nch, lpr);                 // 1 .. 4 for kw <= 512
+        k = c.N;
+    }
+    // Layer l zeroes the slots layer l + 2 writes; the zeroing blocks own rows
+    // of layer l + 1 too (their adds there order the zeroes before layer l + 2).
+    for (int l = 0; l < L; ++l) {
+        bnn::ChainLayer& ly = args.layer[l];
+        ly.zero_blocks = l + 2 <= L - 2 ? std::min(ly.active, args.layer[l + 1].active) : 0;
+        ly.zero_words = ly.zero_blocks > 0 ? (int)ceil_div(args.layer[l + 2].N, 32) : 0;
+        ly.zero_per = ly.zero_blocks > 0 ? (int)ceil_div(ly.zero_words, ly.zero_blocks) : 0;
+    }
+    args.x = x;
+    args.y_i32 = y_i32;
+    args.y_f32 = y_f32;
+    args.acts = acts;
+    args.ld_acts = ld_acts;
+    args.slots = reinterpret_cast<unsigned long long*>(workspace + HEADER_WORDS);
+    args.finished = workspace;
+    args.L = L;
+    args.x_vec = aligned(x, 16) ? 1 : 0;
+
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)G);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = as_cuda(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, args) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return BNN_ERR_CUDA;
+    }
+    return launch_status();
 }
 
 }  // extern "C"
