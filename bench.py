@@ -147,6 +147,7 @@ KERNEL_SOURCES = {
     "xnor_conv3x3_tcw_kernel": ("conv_tc.cuh", "conv.cuh", "gemm_tc.cuh", "gemm_popc.cuh", "common.cuh"),
     "pack_sign_rows_kernel": ("pack.cuh", "common.cuh"),
     "pack_sign_nchw_kernel": ("pack.cuh", "common.cuh"),
+    "pack_sign_nchw_tma_kernel": ("pack.cuh", "common.cuh"),
     "bw_gemv_kernel": ("bwgemv.cuh", "common.cuh"),
     "bw_gemv_i8_kernel": ("bwgemv_i8.cuh", "common.cuh"),
     "ternary_gemv_i8_kernel": ("ternary.cuh", "common.cuh"),
@@ -707,7 +708,8 @@ def _row_conv(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk):
             "conv_kernel_binary_tmac_s": round(cmac_s / 1e12, 2), "roofline": roof,
             "pack_nchw": {"ms": ms_pack / steps, "achieved_gbs": round(pack_gbs, 1),
                           "frac": round(pack_gbs / pk["hbm_gbs"], 4), "bytes": pbytes,
-                          "traffic": recorded_traffic("conv3x3", "pack_sign_nchw_kernel")},
+                          "traffic": recorded_traffic("conv3x3", "pack_sign_nchw_tma_kernel"),
+                          "kernel": "pack_sign_nchw_tma_kernel"},
             "pack_nchw_rsign": {"ms": ms_rs / steps, "achieved_gbs": round(rs_gbs, 1),
                                 "frac": round(rs_gbs / pk["hbm_gbs"], 4), "bytes": pbytes + c * 4},
             "l2": f"{R} rotating input/output sets, {rot_mb:.0f} MB"}

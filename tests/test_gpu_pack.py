@@ -186,3 +186,58 @@ def test_pack_sign_rsign_zero_threshold_is_sign():
     torch.cuda.synchronize()
     assert torch.equal(a, b) and torch.equal(pa, pb)
     assert_no_device_error()
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_pack_sign_nchw_many_tiles_per_warp(dtype):
+    """A tensor of more 4 KiB tiles than the grid's warps x stages, so every
+    warp of the TMA-streamed pack refills its stages; checked against the
+    oracle and against the register kernel (taken for an unaligned view)."""
+    d = dev()
+    n, c, h, w = 96, 64, 56, 56
+    x = workloads.normal((n, c, h, w), 1.0, 4242).to(dtype)
+    xd = x.to(d)
+    out = bnn.empty_packed_nhwc(n, c, h, w, d)
+    bnn.bnn_pack_sign_nchw(xd, out)
+    buf = torch.empty(xd.numel() + 8, dtype=dtype, device=d)
+    xu = buf[1:1 + xd.numel()].view(n, c, h, w)                      # 2 or 4 bytes off: the other kernel
+    xu.copy_(xd)
+    out_u = bnn.empty_packed_nhwc(n, c, h, w, d)
+    bnn.bnn_pack_sign_nchw(xu, out_u)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out_u)
+    assert np.array_equal(u32(out), expected_nhwc(x))
+    assert_no_device_error()
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_pack_sign_nchw_rsign_ragged_channels_streamed(dtype):
+    """RSign on the TMA-streamed pack: 40 channels (the second word holds 8),
+    72 pixels per image (whole 16-byte rows for both dtypes)."""
+    d = dev()
+    shape = (3, 40, 8, 9)
+    n, c, h, w = shape
+    x = workloads.normal(shape, 1.0, 977).to(dtype)
+    beta = _beta(c, 131)
+    x[1, 3, 0, 0] = beta[3].to(dtype)
+    packed = bnn.empty_packed_nhwc(n, c, h, w, d)
+    bnn.bnn_pack_sign_nchw_rsign(x.to(d), beta.to(d), packed)
+    torch.cuda.synchronize()
+    cw = (c + 31) // 32
+    r = oracle.rsign_pm1(x, beta, axis=1)
+    want = oracle.pack_pm1(np.ascontiguousarray(r.transpose(0, 2, 3, 1)).reshape(-1, c))[:, :cw]
+    assert np.array_equal(u32(packed).reshape(-1, cw), want)
+    assert_no_device_error()
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("shape", [(2, 64, 8, 8), (3, 40, 6, 6), (1, 33, 5, 7)])
+def test_pack_sign_nchw_nonfinite(shape, dtype):
+    """NaN -> +1, +inf -> +1, -inf -> -1, signed zeros and subnormals, on the
+    streamed pack (whole 16-byte rows) and the register kernel (the rest)."""
+    n, c, h, w = shape
+    x = workloads.random_with_edges(n * c, h * w, seed=7 * sum(shape), dtype=dtype, edge_fraction=0.3,
+                                    finite=False).reshape(shape).contiguous()
+    out = bnn.empty_packed_nhwc(n, c, h, w, dev())
+    bnn.bnn_pack_sign_nchw(x.to(dev()), out)
+    assert np.array_equal(u32(out), expected_nhwc(x))

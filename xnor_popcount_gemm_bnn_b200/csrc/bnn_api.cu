@@ -462,6 +462,60 @@ bnn_status pack_sign_rows(const void* x, bnn_dtype dt, int64_t rows, int64_t K, 
     return launch_status();
 }
 
+// The TMA-streamed NCHW pack (pack_sign_nchw_tma_kernel): a 2-D map over
+// the tensor as [n*c rows, hw pixels], box 32 rows x 128 bytes, zero fill
+// past either end.  Returns UNSUPPORTED when the map cannot be encoded, so
+// the caller falls back to the register kernel.
+bnn_status pack_sign_nchw_tma(const void* x, bnn_dtype dt, int64_t n, int64_t c, int64_t hw, int64_t cw,
+                              const float* beta, uint32_t* packed_nhwc, cudaStream_t s) {
+    using namespace bnn::nchw_tma;
+    auto enc = tensor_map_encoder();
+    if (enc == nullptr) return BNN_ERR_UNSUPPORTED;
+    const int64_t es = dt == BNN_F32 ? 4 : 2;
+    const int64_t P = 128 / es;
+    CUtensorMap map;
+    cuuint64_t dims[2] = {(cuuint64_t)hw, (cuuint64_t)(n * c)};
+    cuuint64_t strides[1] = {(cuuint64_t)(hw * es)};
+    cuuint32_t box[2] = {(cuuint32_t)P, 32u};
+    cuuint32_t estr[2] = {1, 1};
+    if (enc(&map, dt == BNN_F32 ? CU_TENSOR_MAP_DATA_TYPE_UINT32 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
+            const_cast<void*>(x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return BNN_ERR_UNSUPPORTED;
+    const int64_t tiles_per_plane = ceil_div(hw, P);
+    const int64_t total = n * cw * tiles_per_plane;
+    const int64_t blocks = std::min<int64_t>(sm_count(), ceil_div(total, WARPS));
+    // one-time opt-in to the shared memory per device (kept out of captured graphs)
+    {
+        constexpr int kMaxDevices = 64;
+        static std::atomic<int> done[kMaxDevices];
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return BNN_ERR_CUDA;
+        if (dev >= kMaxDevices || !done[dev].load(std::memory_order_acquire)) {
+            if (cudaFuncSetAttribute(bnn::pack_sign_nchw_tma_kernel<float, false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess ||
+                cudaFuncSetAttribute(bnn::pack_sign_nchw_tma_kernel<float, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess ||
+                cudaFuncSetAttribute(bnn::pack_sign_nchw_tma_kernel<__nv_bfloat16, false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess ||
+                cudaFuncSetAttribute(bnn::pack_sign_nchw_tma_kernel<__nv_bfloat16, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+                return BNN_ERR_CUDA;
+            if (dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
+        }
+    }
+    auto go = [&](auto kern) -> bnn_status {
+        kern<<<(unsigned)blocks, THREADS, SMEM_BYTES, s>>>(map, n, c, hw, cw, tiles_per_plane, packed_nhwc, beta);
+        return launch_status();
+    };
+    if (dt == BNN_F32)
+        return beta == nullptr ? go(bnn::pack_sign_nchw_tma_kernel<float, false>)
+                               : go(bnn::pack_sign_nchw_tma_kernel<float, true>);
+    return beta == nullptr ? go(bnn::pack_sign_nchw_tma_kernel<__nv_bfloat16, false>)
+                           : go(bnn::pack_sign_nchw_tma_kernel<__nv_bfloat16, true>);
+}
+
 bnn_status pack_sign_nchw(const void* x, bnn_dtype dt, int64_t n, int64_t c, int64_t h, int64_t w, const float* beta,
                           uint32_t* packed_nhwc, bnn_stream_t stream) {
     if (x == nullptr || packed_nhwc == nullptr) return BNN_ERR_INVALID_ARG;
@@ -473,6 +527,12 @@ bnn_status pack_sign_nchw(const void* x, bnn_dtype dt, int64_t n, int64_t c, int
     if (n == 0) return BNN_OK;
     const int64_t hw = h * w, cw = (c + 31) / 32;
     cudaStream_t s = as_cuda(stream);
+    // TMA-streamed kernel: needs a 16-byte aligned tensor whose channel rows
+    // are whole 16-byte units (TMA's stride rule) and coordinates in int32.
+    if (aligned(x, 16) && (hw * (int64_t)es) % 16 == 0 && n * c < (int64_t)INT_MAX && hw < (int64_t)INT_MAX) {
+        const bnn_status st = pack_sign_nchw_tma(x, dt, n, c, hw, cw, beta, packed_nhwc, s);
+        if (st != BNN_ERR_UNSUPPORTED) return st;
+    }
     const int64_t warps = n * ceil_div(hw, 8 * (int64_t)(16 / es)) * cw;   // (image, 8 vectors of pixels, word)
     const int64_t blocks = ceil_div(warps, 8);
     if (blocks > INT_MAX) return BNN_ERR_INVALID_ARG;

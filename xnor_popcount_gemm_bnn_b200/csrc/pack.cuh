@@ -203,6 +203,134 @@ pack_sign_nchw_kernel(const T* __restrict__ x, int64_t n, int64_t c, int64_t hw,
         if ((p & 3) == q && p < np) out[(b * hw + p0 + p) * cw + j] = bits[p];
 }
 
+// The same NCHW -> per-pixel channel words, streamed by TMA.  A tile is 32
+// channel rows x 128 bytes of pixels (64 bf16 or 32 fp32) of one image:
+// channels 32j .. 32j+31 of pixels [t*P, t*P + P), 4 KiB.  Every warp is its
+// own pipeline over the tiles gw, gw + W, gw + 2W, ... (W = warps in the
+// grid) with STAGES tiles in flight in its own part of shared memory, so with
+// one 512-thread block per SM the whole activation tensor of a ResNet layer
+// is requested at once and HBM streams without waves or register limits.
+// Lane l reads 4 bytes of each of the 32 rows (pixels 2l, 2l+1 for bf16, l
+// for fp32; a warp reads one 128-byte row per load, no bank conflicts) and
+// builds the whole 32-bit channel word of its pixels itself.  Rows past c
+// belong to the next image (or lie past the tensor, zero-filled) and are
+// masked; pixels past hw are zero-filled and not stored.
+// RS: per-channel threshold beta (fp32 [c]), bit = (x < beta_c).
+namespace nchw_tma {
+constexpr int WARPS = 16;
+constexpr int THREADS = 32 * WARPS;
+constexpr int STAGES = 3;
+constexpr int TILE_BYTES = 32 * 128;
+constexpr int SMEM_BYTES = WARPS * STAGES * TILE_BYTES + WARPS * STAGES * 8;
+}  // namespace nchw_tma
+
+template <typename T, bool RS>
+__global__ void __launch_bounds__(nchw_tma::THREADS, 1)
+pack_sign_nchw_tma_kernel(const __grid_constant__ CUtensorMap map, int64_t n, int64_t c, int64_t hw, int64_t cw,
+                          int64_t tiles_per_plane, uint32_t* __restrict__ out, const float* __restrict__ beta) {
+    using namespace nchw_tma;
+    constexpr int P = 128 / (int)sizeof(T);       // pixels per tile
+    constexpr int PPL = P / 32;                   // pixels per lane
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint8_t* tiles = smem + warp * STAGES * TILE_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + WARPS * STAGES * TILE_BYTES) + warp * STAGES;
+    const int64_t total = n * cw * tiles_per_plane;
+    const int64_t gw = (int64_t)blockIdx.x * WARPS + warp;
+    const int64_t nw = (int64_t)gridDim.x * WARPS;
+    if (lane == 0) {
+        prefetch_tensormap(&map);
+        #pragma unroll
+        for (int s = 0; s < STAGES; ++s) mbar_init(&bars[s], 1);
+        fence_mbarrier_init();
+    }
+    __syncwarp();
+    auto issue = [&](int64_t u, int s) {
+        const int64_t t = u % tiles_per_plane, bj = u / tiles_per_plane;
+        const int64_t j = bj % cw, b = bj / cw;
+        mbar_arrive_expect_tx(&bars[s], TILE_BYTES);
+        tma_load_2d(tiles + s * TILE_BYTES, &map, (int32_t)(t * P), (int32_t)(b * c + 32 * j), &bars[s]);
+    };
+    if (lane == 0) {
+        #pragma unroll
+        for (int s = 0; s < STAGES; ++s)
+            if (gw + s * nw < total) issue(gw + s * nw, s);
+    }
+    const int64_t mine = gw < total ? (total - gw + nw - 1) / nw : 0;   // tiles of this warp
+    int k = 0;
+    for (int64_t u = gw; u < total; u += nw, ++k) {
+        const int s = k % STAGES;
+        const bool ok = mbar_wait_bounded(&bars[s], (uint32_t)((k / STAGES) & 1));
+        if (!__all_sync(0xffffffffu, ok)) {
+            // gave up (the error flag is set): wait, bounded, for the tiles
+            // still in flight into this warp's stages before leaving
+            const int64_t issued = min(mine, (int64_t)k + STAGES);
+            for (int64_t i = k + 1; i < issued; ++i) mbar_wait_bounded(&bars[i % STAGES], (uint32_t)((i / STAGES) & 1));
+            break;
+        }
+        const int64_t t = u % tiles_per_plane, bj = u / tiles_per_plane;
+        const int64_t j = bj % cw, b = bj / cw;
+        const int64_t cvalid = c - 32 * j;
+        const uint32_t mask = cvalid >= 32 ? 0xffffffffu : ((1u << cvalid) - 1u);
+        const uint8_t* tile = tiles + s * TILE_BYTES;
+        uint32_t wd[PPL];
+        // Each row costs one compare that writes a mask register and one LOP3
+        // that keeps that row's bit: x < th as an ordered compare, so -0.0 and
+        // NaN give 0 and negative subnormals give 1, as in the other packs.
+        if constexpr (sizeof(T) == 2) {
+            // Two pixels per lane as one bf16x2.  For a bf16 x and an fp32
+            // threshold b, x < b exactly when x < (b rounded up to bf16), so
+            // the compare runs in bf16x2 with no loss.  Rows 0..15 gather in
+            // acc0 (pixel 2l in bits 0..15, pixel 2l+1 in bits 16..31), rows
+            // 16..31 in acc1.
+            uint32_t th_lane = 0u;
+            if constexpr (RS) {
+                const __nv_bfloat16 tb =
+                    __float2bfloat16_ru((32 * j + lane < c) ? __ldg(beta + 32 * j + lane) : 0.0f);
+                const uint32_t h = (uint32_t)__bfloat16_as_ushort(tb);
+                th_lane = h | (h << 16);
+            }
+            uint32_t acc0 = 0u, acc1 = 0u;
+            #pragma unroll
+            for (int r = 0; r < 32; ++r) {
+                const uint32_t raw = *reinterpret_cast<const uint32_t*>(tile + r * 128 + lane * 4);
+                uint32_t tb2 = 0u;
+                if constexpr (RS) tb2 = __shfl_sync(0xffffffffu, th_lane, r);
+                const uint32_t m = __hlt2_mask(*reinterpret_cast<const __nv_bfloat162*>(&raw),
+                                               *reinterpret_cast<const __nv_bfloat162*>(&tb2));
+                if (r < 16) acc0 |= m & (0x00010001u << r);
+                else        acc1 |= m & (0x00010001u << (r - 16));
+            }
+            wd[0] = (acc0 & 0xFFFFu) | (acc1 << 16);
+            wd[PPL - 1] = (acc0 >> 16) | (acc1 & 0xFFFF0000u);
+        } else {
+            float th_lane = 0.0f;
+            if constexpr (RS) th_lane = (32 * j + lane < c) ? __ldg(beta + 32 * j + lane) : 0.0f;
+            uint32_t acc = 0u;
+            #pragma unroll
+            for (int r = 0; r < 32; ++r) {
+                const float v = *reinterpret_cast<const float*>(tile + r * 128 + lane * 4);
+                float th = 0.0f;
+                if constexpr (RS) th = __shfl_sync(0xffffffffu, th_lane, r);
+                uint32_t m;
+                asm("set.lt.u32.f32 %0, %1, %2;" : "=r"(m) : "f"(v), "f"(th));
+                acc |= m & (1u << r);
+            }
+            wd[0] = acc;
+        }
+        // the stage's bytes were read through the generic proxy; order those
+        // reads before the next TMA write into the same bytes
+        fence_proxy_async_shared();
+        __syncwarp();
+        if (lane == 0 && u + STAGES * nw < total) issue(u + STAGES * nw, s);
+        #pragma unroll
+        for (int q = 0; q < PPL; ++q) {
+            const int64_t p = t * P + lane * PPL + q;
+            if (p < hw) out[(b * hw + p) * cw + j] = wd[q] & mask;
+        }
+    }
+}
+
 // OIHW 3x3 filters -> packed rows in (kh, kw, c) order, one warp per output
 // channel; lane = channel within a 32-channel word.  alpha over the 9*cin
 // true weights (eq. (1): one scale per filter).
