@@ -52,6 +52,8 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # Dense int8 tensor throughput is twice dense bf16 (4.5 vs 2.25 PFLOP/s nominal);
 # the int8 peak used here is the measured bf16 peak times that ratio.
 INT8_PER_BF16 = 2.0
+# Dense fp4 (e2m1) over dense bf16 tensor throughput, nominal (9 / 2.25 PFLOP/s).
+FP4_PER_BF16 = 4.0
 # Whether AUTO runs the stride-1 convolution on the tensor cores (mirrors the
 # library's dispatch, for labelling the conv row's roofline).
 CONV_AUTO_TENSOR = True
@@ -142,6 +144,7 @@ def alu_roofline(mac_s: float, ip: dict) -> dict:
 KERNEL_SOURCES = {
     "xnor_gemv_row128_kernel": ("gemv.cuh", "common.cuh"),
     "xnor_gemm_tc_kernel": ("gemm_tc.cuh", "gemm_popc.cuh", "common.cuh"),
+    "xnor_gemm_f4_kernel": ("gemm_f4.cuh", "gemm_tc.cuh", "gemm_popc.cuh", "common.cuh"),
     "xnor_gemm_popc_kernel": ("gemm_popc.cuh", "common.cuh"),
     "xnor_conv3x3_kernel": ("conv.cuh", "common.cuh"),
     "xnor_conv3x3_tcw_kernel": ("conv_tc.cuh", "conv.cuh", "gemm_tc.cuh", "gemm_popc.cuh", "common.cuh"),
@@ -597,16 +600,19 @@ def _row_pack(torch, bnn, workloads, dev, pk, rows, timed, steps, ws):
     torch.cuda.empty_cache()
 
 
-def _tensor_roofline(pk, macs_per_s, sustained, row=None):
-    """The tensor-core engine against the int8 tensor peak (one binary MAC is
-    one int8 MAC there): measured bf16 dense TFLOP/s x 2, as int8 TOPS."""
+def _tensor_roofline(pk, macs_per_s, sustained, row=None, operand="int8", kernel="xnor_gemm_tc_kernel<TC_BINARY>"):
+    """A tensor-core engine against the dense peak of its operand type (one
+    binary MAC is one MAC there): measured bf16 dense TFLOP/s x 2 for int8
+    operands, x 4 for e2m1 (fp4) operands, in TOPS of that type."""
     bf16 = pk["bf16_tflops_sustained" if sustained else "bf16_tflops"]
-    peak_tops = bf16 * INT8_PER_BF16
+    ratio = FP4_PER_BF16 if operand == "e2m1" else INT8_PER_BF16
+    peak_tops = bf16 * ratio
     achieved = 2 * macs_per_s / 1e12
-    return {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak_tops, 1), "unit": "TOPS (int8)",
-            "frac": round(achieved / peak_tops, 4),
-            "peak_derivation": f"measured bf16 {'sustained' if sustained else 'burst'} {bf16} TFLOP/s x {INT8_PER_BF16} (dense int8 / bf16)",
-            "traffic": recorded_traffic(row, "xnor_gemm_tc_kernel<TC_BINARY>") if row else None}
+    return {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak_tops, 1),
+            "unit": f"TOPS ({operand})", "frac": round(achieved / peak_tops, 4),
+            "peak_derivation": f"measured bf16 {'sustained' if sustained else 'burst'} {bf16} TFLOP/s x {ratio} "
+                               f"(dense {operand} / bf16, nominal)",
+            "traffic": recorded_traffic(row, kernel) if row else None}
 
 
 def _row_square(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, clk_mhz, pk=None):
@@ -621,21 +627,29 @@ def _row_square(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, cl
     Ci = torch.empty(sq.M, sq.N, dtype=torch.int32, device=dev)
     Cf = torch.empty(sq.M, sq.N, dtype=torch.float32, device=dev)
     macs = sq.M * sq.N * sq.K
-    for name, engine in (("square_gemm", bnn.BNN_GEMM_ENGINE_TENSOR), ("square_gemm_popcount", bnn.BNN_GEMM_ENGINE_POPCOUNT)):
+    engines = (("square_gemm", bnn.BNN_GEMM_ENGINE_TENSOR), ("square_gemm_i8", bnn.BNN_GEMM_ENGINE_TENSOR_I8),
+               ("square_gemm_popcount", bnn.BNN_GEMM_ENGINE_POPCOUNT))
+    for name, engine in engines:
         with bnn.gemm_engine(engine):
             ms_g = timed(lambda i: bnn.bnn_xnor_gemm(A_p, Wsq, sq.K, al, Ci, Cf))
             ms_s = timed(lambda i: (bnn.bnn_pack_sign(Ad, A_p), bnn.bnn_xnor_gemm(A_p, Wsq, sq.K, al, Ci, Cf)))
         mac_s = macs * steps / (ms_g * 1e-3)
         if engine == bnn.BNN_GEMM_ENGINE_TENSOR:
-            roof = _tensor_roofline(pk, mac_s, sustained=False, row=name)
+            kernel = "xnor_gemm_f4_kernel"
+            roof = _tensor_roofline(pk, mac_s, sustained=False, row=name, operand="e2m1", kernel=kernel)
+            label = "tensor (tcgen05 kind::mxf4, e2m1 +1/-1, unit scales)"
+        elif engine == bnn.BNN_GEMM_ENGINE_TENSOR_I8:
             kernel = "xnor_gemm_tc_kernel"
+            roof = _tensor_roofline(pk, mac_s, sustained=False, row="square_gemm")
+            label = "tensor (tcgen05 kind::i8)"
         else:
             roof = alu_roofline(mac_s, alu_peak)
             roof["traffic"] = recorded_traffic("square_gemm_popcount", "xnor_gemm_popc_kernel")
             kernel = "xnor_gemm_popc_kernel"
+            label = "popcount (XOR + POPC, carry-save)"
         rows[name] = {
             "workload": "M=N=K=8192 packed A x packed W^T, int32 s + alpha*s fp32 out",
-            "engine": "tensor (tcgen05 kind::i8)" if engine == bnn.BNN_GEMM_ENGINE_TENSOR else "popcount (XOR + POPC, carry-save)",
+            "engine": label,
             "kernel": kernel,
             "value": round(ws * mac_s / 1e9, 1), "unit": "binary GMAC/s", "tops": round(ws * 2 * mac_s / 1e12, 2),
             "ms_per_step": ms_g / steps,
@@ -1013,16 +1027,22 @@ def _row_mlp(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk=No
             A = o
 
     mmacs = 4 * B * D * D
-    for name, engine in (("mlp4", bnn.BNN_GEMM_ENGINE_TENSOR), ("mlp4_popcount", bnn.BNN_GEMM_ENGINE_POPCOUNT)):
+    for name, engine in (("mlp4", bnn.BNN_GEMM_ENGINE_TENSOR), ("mlp4_i8", bnn.BNN_GEMM_ENGINE_TENSOR_I8),
+                         ("mlp4_popcount", bnn.BNN_GEMM_ENGINE_POPCOUNT)):
         with bnn.gemm_engine(engine):
             ms_m = timed(mlp_step)
         mac_s = mmacs * steps / (ms_m * 1e-3)
-        roof = (_tensor_roofline(pk, mac_s, sustained=False, row=name) if engine == bnn.BNN_GEMM_ENGINE_TENSOR else
-                alu_roofline(mac_s, alu_peak))
+        if engine == bnn.BNN_GEMM_ENGINE_TENSOR:
+            roof = _tensor_roofline(pk, mac_s, sustained=False, row=name, operand="e2m1", kernel="xnor_gemm_f4_kernel")
+        elif engine == bnn.BNN_GEMM_ENGINE_TENSOR_I8:
+            roof = _tensor_roofline(pk, mac_s, sustained=False, row="mlp4")
+        else:
+            roof = alu_roofline(mac_s, alu_peak)
         rows[name] = {
             "workload": "fully binary MLP, batch 4096, width 4096, 4 layers: pack fp32 input, "
                         "3 x (GEMM + folded BatchNorm sign re-pack), GEMM + alpha fp32 logits",
-            "engine": "tensor" if engine == bnn.BNN_GEMM_ENGINE_TENSOR else "popcount",
+            "engine": {bnn.BNN_GEMM_ENGINE_TENSOR: "tensor (e2m1)", bnn.BNN_GEMM_ENGINE_TENSOR_I8: "tensor (int8)",
+                       bnn.BNN_GEMM_ENGINE_POPCOUNT: "popcount"}[engine],
             "value": round(ws * mac_s / 1e9, 1), "unit": "binary GMAC/s",
             "ms_per_step": ms_m / steps, "roofline": roof,
             "l2": f"{R} rotating input/activation/logit sets, {rot_mb:.0f} MB"}

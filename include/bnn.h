@@ -221,9 +221,14 @@ bnn_status bnn_pack_conv3x3_weights(const void* w_oihw, bnn_dtype dt, int64_t co
  * product is exact integer arithmetic):
  *   POPCOUNT: XOR + population count on the integer pipes, with carry-save
  *             compression (any shape).
- *   TENSOR:   the sign bits expanded to +1/-1 bytes in shared memory and
- *             multiplied on the tensor cores (tcgen05.mma kind::i8, int32
- *             accumulators in tensor memory); for large products.
+ *   TENSOR:   the sign bits expanded to +1/-1 values in shared memory and
+ *             multiplied on the tensor cores: as 4-bit e2m1 values
+ *             (tcgen05.mma kind::mxf4 with unit block scales, fp32
+ *             accumulators holding exact integers) while K rounded up to a
+ *             multiple of 256 is at most 2^20, as int8 bytes (kind::i8,
+ *             int32 accumulators) beyond that; for large products.
+ *   TENSOR_I8: the int8 tensor-core kernel at every K (the convolutions
+ *             take it as TENSOR).
  *   AUTO:     TENSOR when M >= 128, N >= 128 and K >= 512, else POPCOUNT
  *             (the default).  Convolutions: the stride-1 tensor-core kernel
  *             when cout >= 64, c <= 64 and n*oh*ow >= 16384, else POPCOUNT.
@@ -235,7 +240,8 @@ bnn_status bnn_pack_conv3x3_weights(const void* w_oihw, bnn_dtype dt, int64_t co
 typedef enum bnn_gemm_engine {
     BNN_GEMM_ENGINE_AUTO = 0,
     BNN_GEMM_ENGINE_POPCOUNT = 1,
-    BNN_GEMM_ENGINE_TENSOR = 2
+    BNN_GEMM_ENGINE_TENSOR = 2,
+    BNN_GEMM_ENGINE_TENSOR_I8 = 3
 } bnn_gemm_engine;
 
 /* Selects the GEMM engine for later calls from every thread of the process

@@ -149,9 +149,12 @@ def test_fold_rejects_bad_arguments():
 
 def test_gemm_engine_setting_on_host():
     prev = bnn.bnn_get_gemm_engine()
-    assert L.bnn_set_gemm_engine(3) == bnn.BNN_ERR_INVALID_ARG
+    assert L.bnn_set_gemm_engine(4) == bnn.BNN_ERR_INVALID_ARG
+    assert L.bnn_set_gemm_engine(-1) == bnn.BNN_ERR_INVALID_ARG
     assert L.bnn_set_gemm_engine(bnn.BNN_GEMM_ENGINE_TENSOR) == bnn.BNN_OK
     assert bnn.bnn_get_gemm_engine() == bnn.BNN_GEMM_ENGINE_TENSOR
+    assert L.bnn_set_gemm_engine(bnn.BNN_GEMM_ENGINE_TENSOR_I8) == bnn.BNN_OK
+    assert bnn.bnn_get_gemm_engine() == bnn.BNN_GEMM_ENGINE_TENSOR_I8
     bnn.bnn_set_gemm_engine(prev)
 
 
@@ -262,7 +265,7 @@ def test_header_constants_match_binding():
     assert m and int(m.group(1)) == bnn.BNN_TERNARY_PACK_NOALLOC_MAX_ROWS
     for name in ("BNN_GEMV_WEIGHTS_STATIC", "BNN_GEMV_INPUTS_STATIC", "BNN_GEMV_OUTPUT_FREE", "BNN_OUT_INT32",
                  "BNN_OUT_SCALED_F32", "BNN_OUT_AFFINE_F32", "BNN_OUT_THRESHOLD_PACK", "BNN_GEMM_ENGINE_AUTO",
-                 "BNN_GEMM_ENGINE_POPCOUNT", "BNN_GEMM_ENGINE_TENSOR", "BNN_F32", "BNN_BF16",
+                 "BNN_GEMM_ENGINE_POPCOUNT", "BNN_GEMM_ENGINE_TENSOR", "BNN_GEMM_ENGINE_TENSOR_I8", "BNN_F32", "BNN_BF16",
                  "BNN_ERR_DEVICE_TIMEOUT"):
         m = re.search(rf"\b{name}\s*=\s*(\d+)", text)
         assert m, name

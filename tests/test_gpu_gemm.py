@@ -13,8 +13,8 @@ from gpu_util import assert_affine_close, assert_no_device_error, assert_scaled_
 
 pytestmark = pytest.mark.gpu
 
-ENGINES = [bnn.BNN_GEMM_ENGINE_POPCOUNT, bnn.BNN_GEMM_ENGINE_TENSOR]
-ENGINE_IDS = ["popcount", "tensor"]
+ENGINES = [bnn.BNN_GEMM_ENGINE_POPCOUNT, bnn.BNN_GEMM_ENGINE_TENSOR, bnn.BNN_GEMM_ENGINE_TENSOR_I8]
+ENGINE_IDS = ["popcount", "tensor", "tensor_i8"]
 
 
 @pytest.fixture(params=ENGINES, ids=ENGINE_IDS)
@@ -166,7 +166,8 @@ def test_square_workload_sampled_rows(engine):
 
 def test_engine_setting_roundtrip():
     prev = bnn.bnn_get_gemm_engine()
-    for e in (bnn.BNN_GEMM_ENGINE_TENSOR, bnn.BNN_GEMM_ENGINE_POPCOUNT, bnn.BNN_GEMM_ENGINE_AUTO):
+    for e in (bnn.BNN_GEMM_ENGINE_TENSOR, bnn.BNN_GEMM_ENGINE_TENSOR_I8, bnn.BNN_GEMM_ENGINE_POPCOUNT,
+              bnn.BNN_GEMM_ENGINE_AUTO):
         bnn.bnn_set_gemm_engine(e)
         assert bnn.bnn_get_gemm_engine() == e
     with pytest.raises(bnn.BnnError):
@@ -175,7 +176,7 @@ def test_engine_setting_roundtrip():
 
 
 def test_engines_agree_bit_for_bit():
-    """Both engines on the same operands: identical int32 and identical fp32."""
+    """Every engine on the same operands: identical int32 and identical fp32."""
     M, N, K = 384, 512, 3000
     X = workloads.normal((M, K), 1.0, 77)
     W = workloads.normal((N, K), 1.0, 78)
@@ -187,14 +188,17 @@ def test_engines_agree_bit_for_bit():
             Cf = torch.empty(M, N, dtype=torch.float32, device=dev())
             bnn.bnn_xnor_gemm(A_p, W_p, K, alpha, Ci, Cf)
             outs.append((Ci.cpu(), Cf.cpu()))
-    assert torch.equal(outs[0][0], outs[1][0])
-    assert torch.equal(outs[0][1], outs[1][1])
+    for o in outs[1:]:
+        assert torch.equal(outs[0][0], o[0])
+        assert torch.equal(outs[0][1], o[1])
     assert_no_device_error()
 
 
-def test_tensor_engine_full_matrix_repeated():
+@pytest.mark.parametrize("tensor_engine,launches", [(bnn.BNN_GEMM_ENGINE_TENSOR, 8), (bnn.BNN_GEMM_ENGINE_TENSOR_I8, 4)],
+                         ids=["tensor", "tensor_i8"])
+def test_tensor_engine_full_matrix_repeated(tensor_engine, launches):
     """Races show up as a few wrong tiles in some launches only, so the square
-    workload runs 8 times on the tensor engine and every one of the 67M int32
+    workload runs several times on a tensor engine and every one of the 67M int32
     outputs is compared with the popcount engine's (two independent kernels;
     the popcount result is itself checked against the oracle above).  Once with
     fp32 alpha outputs too, whose epilogue parameters come from shared memory."""
@@ -206,8 +210,8 @@ def test_tensor_engine_full_matrix_repeated():
         bnn.bnn_xnor_gemm(A_p, W_p, sq.K, alpha, ref, ref_f)
     C = torch.empty_like(ref)
     Cf = torch.empty_like(ref_f)
-    with bnn.gemm_engine(bnn.BNN_GEMM_ENGINE_TENSOR):
-        for r in range(8):
+    with bnn.gemm_engine(tensor_engine):
+        for r in range(launches):
             C.fill_(0x5A5A5A5A)
             Cf.fill_(float("nan"))
             bnn.bnn_xnor_gemm(A_p, W_p, sq.K, alpha if r == 0 else None, C, Cf if r == 0 else None)
@@ -215,4 +219,32 @@ def test_tensor_engine_full_matrix_repeated():
             assert torch.equal(C, ref), f"launch {r}: {int((C != ref).sum())} outputs differ"
             if r == 0:
                 assert torch.equal(Cf, ref_f)
+    assert_no_device_error()
+
+
+def test_e2m1_engine_exact_at_the_largest_k():
+    """The 4-bit tensor engine accumulates in fp32; its partial sums are
+    integers of magnitude up to the padded K (2^20 at most), which fp32 holds
+    exactly.  K = 1,048,000 (padded 1,048,064, the top of its range): W rows
+    0..129 are the A rows with 1 in 64 elements negated, so s[m, m] = K - 2 f_m
+    (about 0.97 K, closed form), and every output must equal the popcount
+    engine's exact integer."""
+    M, N, K = 130, 140, 1_048_000
+    d = dev()
+    X = workloads.normal((M, K), 1.0, 2024)
+    flip = workloads.uniform((M, K), 0.0, 1.0, 2025) < (1.0 / 64)
+    Wt = torch.cat([torch.where(flip, -X, X), workloads.normal((N - M, K), 1.0, 2026)])
+    # sign(-x) differs from sign(x) unless x == 0 (then both are +1)
+    f = (flip & (X != 0)).sum(1)
+    A_p, W_p, _ = packed_operands(X, Wt)
+    del X, Wt, flip
+    out = {}
+    for e in (bnn.BNN_GEMM_ENGINE_TENSOR, bnn.BNN_GEMM_ENGINE_POPCOUNT):
+        with bnn.gemm_engine(e):
+            C = torch.empty(M, N, dtype=torch.int32, device=d)
+            bnn.bnn_xnor_gemm(A_p, W_p, K, None, C)
+            out[e] = C.cpu()
+    diag = torch.diagonal(out[bnn.BNN_GEMM_ENGINE_TENSOR][:, :M])
+    assert torch.equal(diag, (K - 2 * f).to(torch.int32))
+    assert torch.equal(out[bnn.BNN_GEMM_ENGINE_TENSOR], out[bnn.BNN_GEMM_ENGINE_POPCOUNT])
     assert_no_device_error()

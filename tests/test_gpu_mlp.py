@@ -13,7 +13,8 @@ from gpu_util import assert_no_device_error, assert_scaled_close, dev, u32
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(params=[bnn.BNN_GEMM_ENGINE_POPCOUNT, bnn.BNN_GEMM_ENGINE_TENSOR], ids=["popcount", "tensor"])
+@pytest.fixture(params=[bnn.BNN_GEMM_ENGINE_POPCOUNT, bnn.BNN_GEMM_ENGINE_TENSOR, bnn.BNN_GEMM_ENGINE_TENSOR_I8],
+                ids=["popcount", "tensor", "tensor_i8"])
 def engine(request):
     with bnn.gemm_engine(request.param):
         yield request.param

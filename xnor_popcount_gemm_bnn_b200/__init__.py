@@ -41,6 +41,7 @@ BNN_GEMV_OUTPUT_FREE = 4
 BNN_GEMM_ENGINE_AUTO = 0
 BNN_GEMM_ENGINE_POPCOUNT = 1
 BNN_GEMM_ENGINE_TENSOR = 2
+BNN_GEMM_ENGINE_TENSOR_I8 = 3
 
 # Every symbol declared in include/bnn.h.
 EXPORTS = (

@@ -1,7 +1,7 @@
 // libbnn.so: the C ABI declared in include/bnn.h.  Host code here only checks
 // arguments, encodes TMA descriptors, picks launch shapes and launches on the
 // caller's stream; every step of the computation runs in the kernels of
-// pack.cuh, gemm_popc.cuh, gemm_tc.cuh, gemv.cuh, chain.cuh, bwgemv.cuh, conv.cuh,
+// pack.cuh, gemm_popc.cuh, gemm_tc.cuh, gemm_f4.cuh, gemv.cuh, chain.cuh, bwgemv.cuh, conv.cuh,
 // conv_tc.cuh and ternary.cuh.
 #include <cudaTypedefs.h>
 
@@ -21,6 +21,7 @@
 #include "conv1x1.cuh"
 #include "gemm_popc.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_f4.cuh"
 #include "gemv.cuh"
 #include "bwgemv.cuh"
 #include "bwgemv_i8.cuh"
@@ -102,6 +103,20 @@ bool gemm_tc_smem_configured() {
                              cudaFuncAttributeMaxDynamicSharedMemorySize, bnn::tc::SMEM_LIMIT) != cudaSuccess ||
         cudaFuncSetAttribute(bnn::xnor_gemm_tc_kernel<bnn::TC_BASES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              bnn::tc::SMEM_BYTES) != cudaSuccess)
+        return false;
+    if (dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
+    return true;
+}
+
+// Per-device one-time opt-in to the 4-bit tensor-core GEMM's shared memory.
+bool gemm_f4_smem_configured() {
+    constexpr int kMaxDevices = 64;
+    static std::atomic<int> done[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+    if (dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return true;
+    if (cudaFuncSetAttribute(bnn::xnor_gemm_f4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bnn::f4::SMEM_BYTES) != cudaSuccess)
         return false;
     if (dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
     return true;
@@ -195,6 +210,73 @@ bnn_status launch_gemm_tc(const uint32_t* A, int64_t lda, const uint32_t* W, int
     return launch_status();
 }
 
+// 2-D map over a row-major fp32 / int32 output [rows, cols] with row stride
+// ld elements, for 32 x 32 tensor stores from 128B-swizzled shared memory.
+// False (store directly) when the pointer or the stride does not suit one.
+bool encode_output_map(CUtensorMap* map, void* base, CUtensorMapDataType dt, int64_t cols, int64_t rows,
+                       int64_t ld) {
+    if (base == nullptr || !aligned(base, 16) || (ld * 4) % 16 != 0 || cols < 1 || rows < 1) return false;
+    auto enc = tensor_map_encoder();
+    if (enc == nullptr) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ld * 4u};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, dt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tile width of the 4-bit kernel: the multiple of 32 up to 224 that
+// minimises (rounds of tiles over the grid) x (rows a stage expands, 128 +
+// bn), the shared-memory traffic that bounds a stage.
+int f4_tile_n(int64_t M, int64_t N, int64_t sms) {
+    const int64_t tiles_m = ceil_div(M, bnn::f4::BM);
+    int best = bnn::f4::BN_MAX;
+    int64_t best_cost = INT64_MAX;
+    for (int bn = bnn::f4::BN_MAX; bn >= 128; bn -= 32) {
+        const int64_t tiles = tiles_m * ceil_div(N, bn);
+        const int64_t cost = ceil_div(tiles, sms) * (bnn::f4::BM + bn);
+        if (cost < best_cost) { best_cost = cost; best = bn; }
+    }
+    return best;
+}
+
+// The +1/-1 product on the tensor cores with e2m1 operands.  Callers check
+// K against MAX_KP (the exact-integer range of the fp32 accumulator).
+bnn_status launch_gemm_f4(const uint32_t* A, int64_t lda, const uint32_t* W, int64_t ldw, int64_t M, int64_t N,
+                          int64_t K, const bnn::GemmEpilogue& ep, cudaStream_t stream) {
+    using namespace bnn::f4;
+    const int64_t kw = packed_ld_words(K);
+    const int64_t sms = sm_count();
+    const int bn = f4_tile_n(M, N, sms);
+    CUtensorMap tmA, tmW;
+    if (!encode_packed_map(&tmA, A, kw, M, lda, BM, BKW, CU_TENSOR_MAP_SWIZZLE_32B) ||
+        !encode_packed_map(&tmW, W, kw, N, ldw, bn, BKW, CU_TENSOR_MAP_SWIZZLE_32B))
+        return BNN_ERR_CUDA;
+    const int64_t tiles_m = ceil_div(M, BM), tiles_n = ceil_div(N, bn);
+    if (tiles_m * tiles_n > INT_MAX) return BNN_ERR_INVALID_ARG;
+    if (!gemm_f4_smem_configured()) return BNN_ERR_CUDA;
+    const int64_t grid = std::min<int64_t>(tiles_m * tiles_n, sms);
+    bnn::GemmEpilogue e = ep;
+    e.bits_words = packed_ld_words(N);
+    // Dense outputs leave through TMA tensor stores where a map fits them.
+    CUtensorMap tmCi, tmCf;
+    std::memset(&tmCi, 0, sizeof(tmCi));
+    std::memset(&tmCf, 0, sizeof(tmCf));
+    int tma_out = 0;
+    if (encode_output_map(&tmCi, e.c_i32, CU_TENSOR_MAP_DATA_TYPE_INT32, N, M, e.ldc)) tma_out |= 1;
+    if (encode_output_map(&tmCf, e.c_f32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, N, M, e.ldf)) tma_out |= 2;
+    bnn::xnor_gemm_f4_kernel<<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(
+        tmA, tmW, tmCi, tmCf, (int)M, (int)N, (int)K, (int)kw, bn, (int)tiles_m, (int)tiles_n, tma_out, e);
+    return launch_status();
+}
+
+// Padded K of the 4-bit kernel (whole 256-element stages).
+inline int64_t f4_padded_k(int64_t K) {
+    return ceil_div(packed_ld_words(K), bnn::f4::BKW) * bnn::f4::BKE;
+}
+
 // 3-D map over a plane-interleaved packed matrix (plane p of row r is packed
 // row r * planes + p): dimensions (word, plane, row), box (4 words,
 // box_planes, box_rows), no swizzle.  box_planes > planes reads the missing
@@ -220,13 +302,18 @@ int pow2_at_least(int v) {
 }
 
 // Engine for one product: the tensor cores once the tile is reasonably
-// filled (M >= 128, N >= 128, K >= 512); the integer pipes otherwise.
+// filled (M >= 128, N >= 128, K >= 512); the integer pipes otherwise.  The
+// tensor engine multiplies e2m1 operands while the padded K keeps every
+// partial sum exact in fp32, and int8 operands beyond (or when forced).
 bnn_status dispatch_gemm(const uint32_t* A, int64_t lda, const uint32_t* W, int64_t ldw, int64_t M, int64_t N,
                          int64_t K, const bnn::GemmEpilogue& ep, cudaStream_t stream) {
     int engine = g_gemm_engine.load(std::memory_order_relaxed);
     if (engine == BNN_GEMM_ENGINE_AUTO)
         engine = (M >= 128 && N >= 128 && K >= 512) ? BNN_GEMM_ENGINE_TENSOR : BNN_GEMM_ENGINE_POPCOUNT;
-    if (engine == BNN_GEMM_ENGINE_TENSOR) return launch_gemm_tc(A, lda, W, ldw, M, N, K, ep, stream);
+    if (engine == BNN_GEMM_ENGINE_TENSOR && f4_padded_k(K) <= bnn::f4::MAX_KP)
+        return launch_gemm_f4(A, lda, W, ldw, M, N, K, ep, stream);
+    if (engine == BNN_GEMM_ENGINE_TENSOR || engine == BNN_GEMM_ENGINE_TENSOR_I8)
+        return launch_gemm_tc(A, lda, W, ldw, M, N, K, ep, stream);
     return launch_gemm(A, lda, W, ldw, M, N, K, ep, stream);
 }
 
@@ -345,7 +432,8 @@ bnn_status gemv_impl(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_
 extern "C" {
 
 bnn_status bnn_set_gemm_engine(int engine) {
-    if (engine != BNN_GEMM_ENGINE_AUTO && engine != BNN_GEMM_ENGINE_POPCOUNT && engine != BNN_GEMM_ENGINE_TENSOR)
+    if (engine != BNN_GEMM_ENGINE_AUTO && engine != BNN_GEMM_ENGINE_POPCOUNT && engine != BNN_GEMM_ENGINE_TENSOR &&
+        engine != BNN_GEMM_ENGINE_TENSOR_I8)
         return BNN_ERR_INVALID_ARG;
     g_gemm_engine.store(engine, std::memory_order_relaxed);
     return BNN_OK;
@@ -1076,7 +1164,8 @@ bnn_status bnn_binary_conv3x3_fused(const uint32_t* X_nhwc_bits, int64_t n, int6
     const int64_t npix = n * oh * ow;
     bnn::ConvEpilogue ep{epi->mode, epi->alpha, epi->gamma, epi->beta, out_nchw};
     cudaStream_t s = as_cuda(stream);
-    const int engine = g_gemm_engine.load(std::memory_order_relaxed);
+    int engine = g_gemm_engine.load(std::memory_order_relaxed);
+    if (engine == BNN_GEMM_ENGINE_TENSOR_I8) engine = BNN_GEMM_ENGINE_TENSOR;   // the conv kernels are int8 only
     const int64_t n_mma = std::max<int64_t>(16, ceil_div(cout, (int64_t)16) * 16);
     // Tensor cores, stride 1: the shifted-window kernel, when the resident
     // filters and two A buffers of at least one tile's window fit.  AUTO takes

@@ -1,0 +1,516 @@
+// Packed binary GEMM on the tensor cores with 4-bit operands
+// (tcgen05.mma kind::mxf4, e2m1 elements, unit block scales).
+//
+// Same product as gemm_popc.cuh and gemm_tc.cuh -- s[m, n] = sum_k a_mk w_nk
+// over +1/-1 values ("Extreme Quantization: Binary, Ternary & 1-bit LLMs",
+// eq. (1), (4) and (6)).  +1 and -1 are exact e2m1 values (0x2 and 0xA: the
+// sign bit is bit 3 of the nibble), so each packed sign bit expands to one
+// nibble instead of one byte: a 128-byte shared-memory row holds 256
+// elements, and the tensor core multiplies 4-bit operands at twice its int8
+// rate.  Every scale factor is 2^0 (ue8m0 127), every product is +1 or -1,
+// and every partial sum is an integer of magnitude at most the padded K
+// (<= 2^20, checked by the host), which fp32 holds exactly; the epilogue
+// reads the fp32 accumulator as that integer.  Pad positions (bits past K
+// and zero-filled words) are +1 in both operands and are subtracted as in
+// the int8 kernel.
+//
+// Roles (sm_100a, one persistent CTA per SM, 17 warps):
+//  * warp 0     : TMA producer, packed tiles of 128 A rows and bn W rows x 8
+//                 words (256 elements of K, 32-byte swizzle) into a ring.
+//  * warps 2-12 : unpack, one thread per packed row (128 + up to 224).  Each
+//                 word becomes 16 bytes: word j of the result is
+//                 ((w << (3 - j)) & 0x88888888) | 0x22222222, i.e. nibble i
+//                 holds element 4i + j -- a fixed permutation of the word's
+//                 32 elements shared by both operands.  One shift and one
+//                 LOP3 per 8 elements.  Chunk q of row r is stored at
+//                 (q ^ (r & 7)) * 16 (the K-major 128B-swizzled layout).
+//  * warp 1     : allocates all 512 TMEM columns (accumulator 0 at column 0,
+//                 accumulator 1 at 256, the scale factors at 480..511); one
+//                 thread issues 4 tcgen05.mma (M = 128, N = bn, K = 64) per
+//                 stage.
+//  * warps 13-16: epilogue: TMEM -> registers -> the fused output modes of
+//                 the int8 kernel; dense int32 / fp32 outputs leave as 32 x 32
+//                 blocks through swizzled shared memory and TMA tensor stores.
+//                 They also fill the scale-factor columns once before the
+//                 first MMA.
+// Every mbarrier wait is bounded (about 1 s) as in gemm_tc.cuh.
+#pragma once
+
+#include "gemm_tc.cuh"
+
+namespace bnn {
+namespace f4 {
+constexpr int BM = 128;
+constexpr int BN_MAX = 224;                 // accumulator columns per tile (bn: a multiple of 32, <= BN_MAX)
+constexpr int BKE = 256;                    // elements of K per stage
+constexpr int BKW = BKE / 32;               // 8 packed words
+constexpr int UMMA_K = 64;                  // e2m1 elements (32 bytes) per tcgen05.mma
+constexpr int USTAGES = 3;                  // unpacked ring
+constexpr int ROW_BYTES = BKE / 2;          // 128: one unpacked row of a stage
+constexpr int U_A_BYTES = BM * ROW_BYTES;   // 16 KiB
+constexpr int U_B_BYTES = BN_MAX * ROW_BYTES;  // 28 KiB
+constexpr int U_STAGE = U_A_BYTES + U_B_BYTES;
+constexpr int P_ROW = BKW * 4;              // 32 bytes of a packed row per stage
+constexpr int P_A_BYTES = BM * P_ROW;       // 4 KiB
+constexpr int P_STAGE = (BM + BN_MAX) * P_ROW;
+constexpr int UNPACK_WARPS = (BM + BN_MAX) / 32;   // 11
+constexpr int EPI_WARPS = 4;
+constexpr int WARP_PRODUCER = 0, WARP_MMA = 1, WARP_UNPACK0 = 2, WARP_EPI0 = WARP_UNPACK0 + UNPACK_WARPS;
+constexpr int THREADS = (WARP_EPI0 + EPI_WARPS) * 32;   // 544
+constexpr int TMEM_COLS = 512;
+constexpr int ACC_STRIDE = 256;             // accumulator b starts at column 256 b
+constexpr int SF_COL = 480;                 // 32 columns of unit scale factors
+constexpr int SFA_COL = SF_COL, SFB_COL = SF_COL + 16;
+constexpr uint32_t SF_ONE = 0x7F7F7F7Fu;    // four ue8m0 bytes of 2^0
+constexpr int MAX_PSTAGES = 8;
+constexpr int NUM_BARS = 2 * MAX_PSTAGES + 2 * USTAGES + 2 * 2 + 1;
+// Output staging for the TMA stores: per epilogue warp one 32 x 32 block of
+// int32 and one of fp32 (4 KiB each, 128B-swizzled rows of 32 values).
+constexpr int OUT_BLOCK = 32 * 32 * 4;
+constexpr int OUT_BYTES = EPI_WARPS * 2 * OUT_BLOCK;
+// Per-tile column parameters, one copy shared by the epilogue warps, double
+// buffered across tiles: float4 {alpha, gamma, beta, -} and int2 {c1, len2}.
+constexpr int COLP_BYTES = 2 * BN_MAX * (16 + 8);
+constexpr int SMEM_FIXED = USTAGES * U_STAGE + OUT_BYTES + COLP_BYTES + NUM_BARS * 8 + 16 + 1024;
+constexpr int PSTAGES = (tc::SMEM_LIMIT - SMEM_FIXED) / P_STAGE < MAX_PSTAGES
+                            ? (tc::SMEM_LIMIT - SMEM_FIXED) / P_STAGE
+                            : MAX_PSTAGES;
+constexpr int SMEM_BYTES = SMEM_FIXED + PSTAGES * P_STAGE;
+static_assert(PSTAGES >= 4, "packed ring too shallow");
+static_assert(U_STAGE % 1024 == 0 && OUT_BLOCK % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+// Named barrier of the epilogue warps (id 0 is __syncthreads).
+constexpr int EPI_BAR = 1;
+static_assert(SMEM_BYTES <= tc::SMEM_LIMIT, "shared memory");
+static_assert(ACC_STRIDE + BN_MAX <= SF_COL, "accumulators overlap the scale factors");
+// Largest padded K: partial sums stay integers of magnitude <= 2^20, exact
+// in fp32 and in the epilogue's float-to-int conversion (valid below 2^22).
+constexpr int64_t MAX_KP = int64_t(1) << 20;
+// Block-scaled instruction descriptor: A and B e2m1 (format 1 of kind::mxf4)
+// at bits 7-9 and 10-12, both K-major, N >> 3 at bits 17-22, scale format
+// ue8m0 (bit 23), M >> 4 at bits 24-28; scale-factor byte ids 0, K = 64.
+__host__ __device__ constexpr uint32_t idesc(int bn) {
+    return (1u << 7) | (1u << 10) | ((uint32_t)(bn >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24);
+}
+}  // namespace f4
+
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+
+// Registers -> TMEM for one warp: the same 32-bit value in 32 consecutive
+// columns of the warp's 32 lanes, then tcgen05.wait::st.
+__device__ __forceinline__ void tmem_fill32(uint32_t taddr, uint32_t v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
+        "%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1};\n\t"
+        "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+        "r"(v)
+        : "memory");
+}
+
+// Shared -> global tensor store of one box (bulk-group completion), and the
+// waits on this thread's outstanding bulk groups.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int32_t x, int32_t y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// 32 sign bits -> 32 e2m1 values (bit 0 -> +1.0 = 0x2, bit 1 -> -1.0 = 0xA)
+// in 16 bytes.  Word j of the result holds element 4i + j in nibble i.
+__device__ __forceinline__ uint4 expand_word_e2m1(uint32_t w) {
+    constexpr uint32_t sign = 0x88888888u, one = 0x22222222u;
+    return make_uint4(((w << 3) & sign) | one, ((w << 2) & sign) | one, ((w << 1) & sign) | one, (w & sign) | one);
+}
+
+// fp32 accumulator holding an integer of magnitude < 2^22 -> that integer
+// (adding 1.5 * 2^23 puts it in the low mantissa bits).
+__device__ __forceinline__ int32_t acc_to_int(uint32_t bits) {
+    return __float_as_int(__uint_as_float(bits) + 12582912.0f) - 0x4B400000;
+}
+
+__global__ void __launch_bounds__(f4::THREADS, 1)
+xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
+                    const __grid_constant__ CUtensorMap tmCi, const __grid_constant__ CUtensorMap tmCf, int M, int N,
+                    int K, int kw, int bn, int tiles_m, int tiles_n, int tma_out, GemmEpilogue ep) {
+    using namespace f4;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t* uring = smem;                                          // USTAGES x (A 16 KiB | W 28 KiB)
+    uint8_t* oring = uring + USTAGES * U_STAGE;                     // [EPI_WARPS][int32 | fp32] 32 x 32 blocks
+    uint8_t* pring = oring + OUT_BYTES;                             // PSTAGES x (A | W packed)
+    float4* colf = reinterpret_cast<float4*>(pring + PSTAGES * P_STAGE);   // [2][BN_MAX]
+    int2* colt = reinterpret_cast<int2*>(colf + 2 * BN_MAX);               // [2][BN_MAX]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(colt + 2 * BN_MAX);
+    uint64_t* pfull = bars;
+    uint64_t* pempty = pfull + MAX_PSTAGES;
+    uint64_t* ufull = pempty + MAX_PSTAGES;
+    uint64_t* uempty = ufull + USTAGES;
+    uint64_t* afull = uempty + USTAGES;
+    uint64_t* aempty = afull + 2;
+    uint64_t* drain = aempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int nk = (kw + BKW - 1) / BKW;
+    const int tiles = tiles_m * tiles_n;
+    const uint32_t stage_tx = (uint32_t)(BM + bn) * P_ROW;
+
+    if (threadIdx.x == 0) {
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmW);
+        if (tma_out & 1) prefetch_tensormap(&tmCi);
+        if (tma_out & 2) prefetch_tensormap(&tmCf);
+        for (int s = 0; s < PSTAGES; ++s) {
+            mbar_init(&pfull[s], 1);
+            mbar_init(&pempty[s], UNPACK_WARPS);
+        }
+        for (int s = 0; s < USTAGES; ++s) {
+            mbar_init(&ufull[s], UNPACK_WARPS);
+            mbar_init(&uempty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&afull[b], 1);
+            mbar_init(&aempty[b], EPI_WARPS);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == WARP_MMA) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    // Unit scale factors: each epilogue warp fills its 32 lanes of the 32
+    // scale-factor columns, so whatever TMEM layout the MMA reads them in,
+    // every factor it finds is 2^0.
+    if (warp >= WARP_EPI0) tmem_fill32(tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + SF_COL, SF_ONE);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    if (warp == WARP_PRODUCER) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0) {
+            uint32_t g = 0, issued = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+                const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * bn;
+                for (int ks = 0; ks < nk; ++ks, ++g) {
+                    const uint32_t s = g % (uint32_t)PSTAGES;
+                    if (g >= (uint32_t)PSTAGES && !tc_wait(&pempty[s], ((g / PSTAGES) - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* dst = pring + s * P_STAGE;
+                    mbar_arrive_expect_tx(&pfull[s], stage_tx);
+                    tma_load_2d(dst, &tmA, ks * BKW, m0, &pfull[s]);
+                    tma_load_2d(dst + P_A_BYTES, &tmW, ks * BKW, n0, &pfull[s]);
+                    ++issued;
+                }
+            }
+            for (uint32_t q = issued > (uint32_t)PSTAGES ? issued - PSTAGES : 0; q < issued; ++q)
+                if (!mbar_wait_bounded(&pfull[q % PSTAGES], (q / PSTAGES) & 1)) break;
+        }
+    } else if (warp == WARP_MMA) {
+        // ------------------------------ MMA issuer ------------------------------
+        if (lane == 0) {
+            uint32_t g = 0;
+            int lt = 0;
+            bool ok = true;
+            const uint32_t ubase = smem_u32(uring);
+            const uint32_t id = idesc(bn);
+            const uint32_t sfa = tmem_base + SFA_COL, sfb = tmem_base + SFB_COL;
+            for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++lt) {
+                const int b = lt & 1;
+                if (lt >= 2 && !tc_wait(&aempty[b], ((lt >> 1) - 1) & 1, abort_flag)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(b * ACC_STRIDE);
+                for (int ks = 0; ks < nk; ++ks, ++g) {
+                    const uint32_t s = g % USTAGES;
+                    if (!tc_wait(&ufull[s], (g / USTAGES) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = ubase + s * U_STAGE;
+                    const uint32_t b_addr = a_addr + U_A_BYTES;
+                    #pragma unroll
+                    for (int kk = 0; kk < BKE / UMMA_K; ++kk) {
+                        // 32 bytes (64 elements) per K step inside the swizzle atom.
+                        mma_mxf4(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32), id, sfa,
+                                 sfb, (ks | kk) != 0 ? 1u : 0u);
+                    }
+                    mma_commit(&uempty[s]);
+                }
+                if (ok) mma_commit(&afull[b]);
+            }
+            mma_commit(drain);
+            mbar_wait_bounded(drain, 0);
+        }
+        __syncwarp();
+    } else if (warp < WARP_EPI0) {
+        // ------------------------------ unpack warps ------------------------------
+        // Thread u expands packed row u of the stage (A rows 0..127, then W
+        // rows 0..bn-1) into 128 bytes.  Rows are 32 bytes apart in the packed
+        // stage, written by the TMA with the 32-byte swizzle: half h of row u
+        // sits at 16 * (h ^ ((u >> 2) & 1)), so the eight lanes of a 16-byte
+        // load phase hit distinct banks, while the words keep their order for
+        // the conflict-free swizzled stores below.
+        const int u = threadIdx.x - WARP_UNPACK0 * 32;               // 0 .. BM + BN_MAX - 1
+        const bool is_a = u < BM;
+        const int r = is_a ? u : u - BM;
+        const bool active = is_a || r < bn;
+        const int sw = r & 7;
+        const int hsw = 16 * ((u >> 2) & 1);
+        uint32_t g = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+            for (int ks = 0; ks < nk; ++ks, ++g) {
+                const uint32_t ps = g % (uint32_t)PSTAGES, us = g % USTAGES;
+                const bool w1 = tc_wait(&pfull[ps], (g / PSTAGES) & 1, abort_flag);
+                const bool w2 = w1 && (g < USTAGES || tc_wait(&uempty[us], ((g / USTAGES) - 1) & 1, abort_flag));
+                if (!__all_sync(0xffffffffu, w1 && w2)) {
+                    ok = false;
+                    break;
+                }
+                uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;      // words 0..3 and 4..7 of the row
+                if (active) {
+                    const uint8_t* src = pring + ps * P_STAGE + u * P_ROW;
+                    lo = *reinterpret_cast<const uint4*>(src + hsw);
+                    hi = *reinterpret_cast<const uint4*>(src + (hsw ^ 16));
+                }
+                release_packed_stage(&pempty[ps], lane);
+                if (active) {
+                    // Chunk q of the row at (q ^ (r & 7)) * 16: the eight lanes of a
+                    // store phase (eight consecutive rows) hit distinct banks.
+                    uint8_t* row = uring + us * U_STAGE + (is_a ? 0 : U_A_BYTES) + r * ROW_BYTES;
+                    *reinterpret_cast<uint4*>(row + ((0 ^ sw) << 4)) = expand_word_e2m1(lo.x);
+                    *reinterpret_cast<uint4*>(row + ((1 ^ sw) << 4)) = expand_word_e2m1(lo.y);
+                    *reinterpret_cast<uint4*>(row + ((2 ^ sw) << 4)) = expand_word_e2m1(lo.z);
+                    *reinterpret_cast<uint4*>(row + ((3 ^ sw) << 4)) = expand_word_e2m1(lo.w);
+                    *reinterpret_cast<uint4*>(row + ((4 ^ sw) << 4)) = expand_word_e2m1(hi.x);
+                    *reinterpret_cast<uint4*>(row + ((5 ^ sw) << 4)) = expand_word_e2m1(hi.y);
+                    *reinterpret_cast<uint4*>(row + ((6 ^ sw) << 4)) = expand_word_e2m1(hi.z);
+                    *reinterpret_cast<uint4*>(row + ((7 ^ sw) << 4)) = expand_word_e2m1(hi.w);
+                }
+                fence_proxy_async_shared();                           // the bytes, visible to the tensor core
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ufull[us]);
+            }
+        }
+    } else {
+        // ------------------------------ epilogue warps ------------------------------
+        // Per tile the four warps stage the tile's column parameters in the
+        // shared copy of this tile's parity (alpha/gamma/beta and the
+        // threshold test as one unsigned range check on the integer
+        // accumulator), meet at a named barrier, then each thread turns its
+        // row's bn accumulators (fp32 integers) into int32 s, alpha * s, the
+        // affine output or the folded-BatchNorm sign bits.  Dense outputs go
+        // out as 32 x 32 blocks: the warp writes a block into its staging
+        // buffer (row = lane, 16-byte chunk q at (q ^ (lane & 7)) * 16, the
+        // TMA's 128-byte swizzle, so no bank conflicts) and lane 0 stores it
+        // with one TMA tensor store, which writes whole lines and clips the
+        // block at M and N.  Outputs whose pointer or stride does not suit a
+        // tensor map are stored directly.  The barrier is reached the same
+        // number of times by every warp, also after a failed wait (the warp
+        // then skips the work), so it cannot hang.
+        const int quad = warp & 3;                                    // TMEM lanes 32*quad .. 32*quad + 31
+        const int ew = warp - WARP_EPI0;                              // 0..3
+        uint8_t* obuf_i = oring + ew * 2 * OUT_BLOCK;                 // this warp's int32 block
+        uint8_t* obuf_f = obuf_i + OUT_BLOCK;                         // and fp32 block
+        const bool tma_i = (tma_out & 1) != 0 && ep.c_i32 != nullptr;
+        const bool tma_f = (tma_out & 2) != 0 && ep.c_f32 != nullptr;
+        const int kp = nk * BKE;                                      // padded K: acc = kp - 2 * popcount
+        const int pad = kp - K;
+        const float padf = (float)pad;
+        const bool affine = ep.gamma != nullptr;
+        const int chunks = bn / 32;
+        const uint32_t sw = (uint32_t)(lane & 7);
+        bool ok = true;
+        int lt = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++lt) {
+            const int b = lt & 1;
+            const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * bn;
+            float4* cf = colf + b * BN_MAX;
+            int2* ct = colt + b * BN_MAX;
+            // Every warp finished tile lt - 2 (the last reader of this copy)
+            // before it reached the barrier of tile lt - 1.
+            for (int i = 32 * ew + lane; i < bn; i += 32 * EPI_WARPS) {
+                const int n = n0 + i;
+                float4 f = make_float4(0.f, 1.f, 0.f, 0.f);
+                int2 th = make_int2(0, 0);                            // len2 = 0: bit never set
+                if (n < N) {
+                    if (ep.alpha != nullptr) f.x = __ldg(ep.alpha + n);
+                    if (affine) { f.y = __ldg(ep.gamma + n); f.z = __ldg(ep.beta + n); }
+                    if (ep.c_bits != nullptr) {
+                        // bit = (unsigned)(c1 - acc) < 2 len for the interval
+                        // [lo, lo + len) of popcounts d = (kp - acc) / 2 that set
+                        // the bit (mode 0: d > T; mode 1: d < T; else none).
+                        const long long T = __ldg(ep.thresh + n);
+                        const int md = ep.thresh_mode[n];
+                        long long lo = 0, len = 0;
+                        if (md == 0) {
+                            lo = T + 1 > 0 ? T + 1 : 0;
+                            len = K - lo + 1 > 0 ? K - lo + 1 : 0;
+                        } else if (md == 1) {
+                            len = T < K + 1 ? T : K + 1;
+                            if (len < 0) len = 0;
+                        }
+                        th = make_int2((int)(uint32_t)(kp - 2 * lo), (int)(uint32_t)(2 * len));
+                    }
+                }
+                cf[i] = f;
+                ct[i] = th;
+            }
+            named_bar_sync(EPI_BAR, EPI_WARPS * 32);
+            ok = ok && __all_sync(0xffffffffu, tc_wait(&afull[b], (lt >> 1) & 1, abort_flag));
+            if (!ok) continue;
+            tc_fence_after();
+            const int mq = m0 + 32 * quad;                            // first row of this warp's quadrant
+            const int m = mq + lane;
+            #pragma unroll 1
+            for (int c = 0; c < chunks; ++c) {
+                uint32_t r[32];
+                tmem_ld32_sync(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * ACC_STRIDE + 32 * c), r);
+                if (c == chunks - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&aempty[b]);
+                }
+                const int nb = n0 + 32 * c;
+                if (nb >= N) {
+                    if (ep.c_bits != nullptr && m < M && nb / 32 < ep.bits_words)
+                        ep.c_bits[(int64_t)m * ep.ldb + nb / 32] = 0u;
+                    continue;
+                }
+                const bool full_chunk = nb + 32 <= N;
+                if (ep.c_bits != nullptr) {
+                    uint32_t word = 0;
+                    #pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int2 q = ct[32 * c + j];
+                        word |= ((uint32_t)(q.x - acc_to_int(r[j])) < (uint32_t)q.y ? 1u : 0u) << j;
+                    }
+                    if (m < M && nb / 32 < ep.bits_words) ep.c_bits[(int64_t)m * ep.ldb + nb / 32] = word;
+                }
+                if (ep.c_i32 != nullptr && tma_i) {
+                    // The block's previous store must have read the buffer
+                    // (the other output's store may still be reading its own).
+                    if (lane == 0) { if (tma_f) bulk_wait_read<1>(); else bulk_wait_read<0>(); }
+                    __syncwarp();
+                    uint8_t* rowp = obuf_i + lane * 128;
+                    #pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        *reinterpret_cast<int4*>(rowp + (((uint32_t)q ^ sw) << 4)) =
+                            make_int4(acc_to_int(r[4 * q]) - pad, acc_to_int(r[4 * q + 1]) - pad,
+                                      acc_to_int(r[4 * q + 2]) - pad, acc_to_int(r[4 * q + 3]) - pad);
+                    fence_proxy_async_shared();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmCi, obuf_i, nb, mq);
+                        bulk_commit();
+                    }
+                } else if (m < M && ep.c_i32 != nullptr) {
+                    int32_t* dst = ep.c_i32 + (int64_t)m * ep.ldc + nb;
+                    const bool vec = full_chunk && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0);
+                    #pragma unroll
+                    for (int j = 0; j < 32; j += 4) {
+                        const int4 o = make_int4(acc_to_int(r[j]) - pad, acc_to_int(r[j + 1]) - pad,
+                                                 acc_to_int(r[j + 2]) - pad, acc_to_int(r[j + 3]) - pad);
+                        if (vec) {
+                            *reinterpret_cast<int4*>(dst + j) = o;
+                        } else {
+                            if (nb + j < N) dst[j] = o.x;
+                            if (nb + j + 1 < N) dst[j + 1] = o.y;
+                            if (nb + j + 2 < N) dst[j + 2] = o.z;
+                            if (nb + j + 3 < N) dst[j + 3] = o.w;
+                        }
+                    }
+                }
+                if (ep.c_f32 != nullptr && (tma_f || m < M)) {
+                    // acc - pad is an integer below 2^21: exact in fp32, so
+                    // f.x * (acc - pad) is alpha * (float)s.
+                    if (tma_f) {
+                        if (lane == 0) { if (tma_i) bulk_wait_read<1>(); else bulk_wait_read<0>(); }
+                        __syncwarp();
+                    }
+                    float* dst = ep.c_f32 + (int64_t)m * ep.ldf + nb;
+                    const bool vec = full_chunk && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0);
+                    #pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        float y[4];
+                        #pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const float4 f = cf[32 * c + 4 * q + k];
+                            float v = f.x * (__uint_as_float(r[4 * q + k]) - padf);
+                            if (affine) v = fmaf(f.y, v, f.z);
+                            y[k] = v;
+                        }
+                        if (tma_f) {
+                            *reinterpret_cast<float4*>(obuf_f + lane * 128 + (((uint32_t)q ^ sw) << 4)) =
+                                make_float4(y[0], y[1], y[2], y[3]);
+                        } else if (vec) {
+                            *reinterpret_cast<float4*>(dst + 4 * q) = make_float4(y[0], y[1], y[2], y[3]);
+                        } else {
+                            #pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                if (nb + 4 * q + k < N) dst[4 * q + k] = y[k];
+                        }
+                    }
+                    if (tma_f) {
+                        fence_proxy_async_shared();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tmCf, obuf_f, nb, mq);
+                            bulk_commit();
+                        }
+                    }
+                }
+            }
+            if (ep.c_bits != nullptr && (t % tiles_n) == tiles_n - 1 && m < M) {
+                for (int64_t wd = (int64_t)(n0 + bn) / 32; wd < ep.bits_words; ++wd)
+                    ep.c_bits[(int64_t)m * ep.ldb + wd] = 0u;
+            }
+        }
+        // The tensor stores must have finished reading shared memory (and
+        // be complete) before the CTA exits.
+        if (lane == 0) bulk_wait_all();
+        __syncwarp();
+    }
+
+    // ------------------------------ teardown ------------------------------
+    tc_fence_before();
+    __syncthreads();
+    if (warp == WARP_MMA) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+}  // namespace bnn
