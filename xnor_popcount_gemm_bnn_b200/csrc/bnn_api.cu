@@ -43,6 +43,9 @@ inline bnn_status launch_status() {
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Resident CTA-pair count that marks the pair mode of the 4-bit GEMM as unavailable.
+constexpr int kNoPairs = 1 << 30;
+
 // cuTensorMapEncodeTiled from the driver, fetched through the runtime so that
 // the library does not link libcuda directly.
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -108,18 +111,43 @@ bool gemm_tc_smem_configured() {
     return true;
 }
 
-// Per-device one-time opt-in to the 4-bit tensor-core GEMM's shared memory.
-bool gemm_f4_smem_configured() {
+// Per-device one-time opt-in to the 4-bit tensor-core GEMM's shared memory
+// (both modes), and the number of CTA pairs that fit on the device at once.
+int gemm_f4_pairs_resident() {
     constexpr int kMaxDevices = 64;
-    static std::atomic<int> done[kMaxDevices];
+    static std::atomic<int> pairs[kMaxDevices];              // 0: not configured yet
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
-    if (dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return true;
-    if (cudaFuncSetAttribute(bnn::xnor_gemm_f4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             bnn::f4::SMEM_BYTES) != cudaSuccess)
-        return false;
-    if (dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
-    return true;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return -1;
+    if (dev < kMaxDevices) {
+        const int p = pairs[dev].load(std::memory_order_acquire);
+        if (p > 0) return p;
+    }
+    using C1 = bnn::f4::Cfg<false>;
+    using C2 = bnn::f4::Cfg<true>;
+    if (cudaFuncSetAttribute(bnn::xnor_gemm_f4_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C1::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(bnn::xnor_gemm_f4_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C2::SMEM_BYTES) != cudaSuccess)
+        return -1;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * 74);
+    cfg.blockDim = dim3(C2::THREADS);
+    cfg.dynamicSmemBytes = C2::SMEM_BYTES;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, bnn::xnor_gemm_f4_kernel<true>, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+    }
+    if (n < 1) n = kNoPairs;                                  // pairs unavailable: f4_plan never picks them
+    if (dev < kMaxDevices) pairs[dev].store(n, std::memory_order_release);
+    return n;
 }
 
 // Per-device one-time opt-in to the add table of the binary-weight GEMV.
@@ -227,17 +255,30 @@ bool encode_output_map(CUtensorMap* map, void* base, CUtensorMapDataType dt, int
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Tile width of the 4-bit kernel: the multiple of 32 up to 224 that
-// minimises (rounds of tiles over the grid) x (rows a stage expands, 128 +
-// bn), the shared-memory traffic that bounds a stage.
-int f4_tile_n(int64_t M, int64_t N, int64_t sms) {
-    const int64_t tiles_m = ceil_div(M, bnn::f4::BM);
-    int best = bnn::f4::BN_MAX;
+// Launch plan of the 4-bit kernel: single CTAs or CTA pairs, and the tile
+// width bn (a multiple of 32 up to 224).  Shared-memory traffic bounds a
+// stage: per SM it moves 128 + bn rows (single) or 128 + bn / 2 rows (pair)
+// for the same 128 x bn x 256 multiply-adds, so the plan minimises (rounds
+// of tiles over the resident CTAs or pairs) x (rows per stage).
+struct F4Plan {
+    bool pair;
+    int bn;
+};
+F4Plan f4_plan(int64_t M, int64_t N, int64_t sms, int64_t pairs) {
+    F4Plan best{false, bnn::f4::BN_MAX};
     int64_t best_cost = INT64_MAX;
-    for (int bn = bnn::f4::BN_MAX; bn >= 128; bn -= 32) {
-        const int64_t tiles = tiles_m * ceil_div(N, bn);
-        const int64_t cost = ceil_div(tiles, sms) * (bnn::f4::BM + bn);
-        if (cost < best_cost) { best_cost = cost; best = bn; }
+    for (int pair = 0; pair < 2; ++pair) {
+        if (pair && (pairs >= kNoPairs || M <= bnn::f4::BM)) continue;
+        const int64_t units = pair ? pairs : sms;
+        const int64_t tiles_m = ceil_div(M, (int64_t)bnn::f4::BM * (pair ? 2 : 1));
+        for (int bn = bnn::f4::BN_MAX; bn >= 128; bn -= 32) {
+            const int64_t tiles = tiles_m * ceil_div(N, bn);
+            const int64_t cost = ceil_div(tiles, units) * (bnn::f4::BM + (pair ? bn / 2 : bn));
+            if (cost < best_cost) {
+                best_cost = cost;
+                best = F4Plan{pair != 0, bn};
+            }
+        }
     }
     return best;
 }
@@ -249,15 +290,16 @@ bnn_status launch_gemm_f4(const uint32_t* A, int64_t lda, const uint32_t* W, int
     using namespace bnn::f4;
     const int64_t kw = packed_ld_words(K);
     const int64_t sms = sm_count();
-    const int bn = f4_tile_n(M, N, sms);
+    const int pairs = gemm_f4_pairs_resident();
+    if (pairs < 0) return BNN_ERR_CUDA;
+    const F4Plan plan = f4_plan(M, N, sms, pairs);
+    const int bn = plan.bn, ctas = plan.pair ? 2 : 1;
     CUtensorMap tmA, tmW;
     if (!encode_packed_map(&tmA, A, kw, M, lda, BM, BKW, CU_TENSOR_MAP_SWIZZLE_32B) ||
-        !encode_packed_map(&tmW, W, kw, N, ldw, bn, BKW, CU_TENSOR_MAP_SWIZZLE_32B))
+        !encode_packed_map(&tmW, W, kw, N, ldw, bn / ctas, BKW, CU_TENSOR_MAP_SWIZZLE_32B))
         return BNN_ERR_CUDA;
-    const int64_t tiles_m = ceil_div(M, BM), tiles_n = ceil_div(N, bn);
+    const int64_t tiles_m = ceil_div(M, (int64_t)BM * ctas), tiles_n = ceil_div(N, bn);
     if (tiles_m * tiles_n > INT_MAX) return BNN_ERR_INVALID_ARG;
-    if (!gemm_f4_smem_configured()) return BNN_ERR_CUDA;
-    const int64_t grid = std::min<int64_t>(tiles_m * tiles_n, sms);
     bnn::GemmEpilogue e = ep;
     e.bits_words = packed_ld_words(N);
     // Dense outputs leave through TMA tensor stores where a map fits them.
@@ -267,8 +309,29 @@ bnn_status launch_gemm_f4(const uint32_t* A, int64_t lda, const uint32_t* W, int
     int tma_out = 0;
     if (encode_output_map(&tmCi, e.c_i32, CU_TENSOR_MAP_DATA_TYPE_INT32, N, M, e.ldc)) tma_out |= 1;
     if (encode_output_map(&tmCf, e.c_f32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, N, M, e.ldf)) tma_out |= 2;
-    bnn::xnor_gemm_f4_kernel<<<(unsigned)grid, THREADS, SMEM_BYTES, stream>>>(
-        tmA, tmW, tmCi, tmCf, (int)M, (int)N, (int)K, (int)kw, bn, (int)tiles_m, (int)tiles_n, tma_out, e);
+    if (!plan.pair) {
+        const int64_t grid = std::min<int64_t>(tiles_m * tiles_n, sms);
+        bnn::xnor_gemm_f4_kernel<false><<<(unsigned)grid, Cfg<false>::THREADS, Cfg<false>::SMEM_BYTES, stream>>>(
+            tmA, tmW, tmCi, tmCf, (int)M, (int)N, (int)K, (int)kw, bn, (int)tiles_m, (int)tiles_n, tma_out, e);
+        return launch_status();
+    }
+    // CTA pairs: clusters of two, as many as are resident at once.
+    const int64_t clusters = std::min<int64_t>(tiles_m * tiles_n, pairs);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)(2 * clusters));
+    cfg.blockDim = dim3(Cfg<true>::THREADS);
+    cfg.dynamicSmemBytes = Cfg<true>::SMEM_BYTES;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, bnn::xnor_gemm_f4_kernel<true>, tmA, tmW, tmCi, tmCf, (int)M, (int)N, (int)K,
+                           (int)kw, bn, (int)tiles_m, (int)tiles_n, tma_out, e) != cudaSuccess)
+        return BNN_ERR_CUDA;
     return launch_status();
 }
 

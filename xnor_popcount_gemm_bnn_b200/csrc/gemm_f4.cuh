@@ -14,7 +14,8 @@
 // and zero-filled words) are +1 in both operands and are subtracted as in
 // the int8 kernel.
 //
-// Roles (sm_100a, one persistent CTA per SM, 17 warps):
+// Roles (sm_100a, one persistent CTA per SM; 17 warps, 14 in the pair mode of
+// the Cfg comment below):
 //  * warp 0     : TMA producer, packed tiles of 128 A rows and bn W rows x 8
 //                 words (256 elements of K, 32-byte swizzle) into a ring.
 //  * warps 2-12 : unpack, one thread per packed row (128 + up to 224).  Each
@@ -40,30 +41,23 @@
 
 namespace bnn {
 namespace f4 {
-constexpr int BM = 128;
+constexpr int BM = 128;                     // A rows per CTA = TMEM lanes
 constexpr int BN_MAX = 224;                 // accumulator columns per tile (bn: a multiple of 32, <= BN_MAX)
 constexpr int BKE = 256;                    // elements of K per stage
 constexpr int BKW = BKE / 32;               // 8 packed words
 constexpr int UMMA_K = 64;                  // e2m1 elements (32 bytes) per tcgen05.mma
-constexpr int USTAGES = 3;                  // unpacked ring
 constexpr int ROW_BYTES = BKE / 2;          // 128: one unpacked row of a stage
-constexpr int U_A_BYTES = BM * ROW_BYTES;   // 16 KiB
-constexpr int U_B_BYTES = BN_MAX * ROW_BYTES;  // 28 KiB
-constexpr int U_STAGE = U_A_BYTES + U_B_BYTES;
 constexpr int P_ROW = BKW * 4;              // 32 bytes of a packed row per stage
 constexpr int P_A_BYTES = BM * P_ROW;       // 4 KiB
-constexpr int P_STAGE = (BM + BN_MAX) * P_ROW;
-constexpr int UNPACK_WARPS = (BM + BN_MAX) / 32;   // 11
+constexpr int U_A_BYTES = BM * ROW_BYTES;   // 16 KiB
 constexpr int EPI_WARPS = 4;
-constexpr int WARP_PRODUCER = 0, WARP_MMA = 1, WARP_UNPACK0 = 2, WARP_EPI0 = WARP_UNPACK0 + UNPACK_WARPS;
-constexpr int THREADS = (WARP_EPI0 + EPI_WARPS) * 32;   // 544
+constexpr int WARP_PRODUCER = 0, WARP_MMA = 1, WARP_UNPACK0 = 2;
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_STRIDE = 256;             // accumulator b starts at column 256 b
 constexpr int SF_COL = 480;                 // 32 columns of unit scale factors
 constexpr int SFA_COL = SF_COL, SFB_COL = SF_COL + 16;
 constexpr uint32_t SF_ONE = 0x7F7F7F7Fu;    // four ue8m0 bytes of 2^0
 constexpr int MAX_PSTAGES = 8;
-constexpr int NUM_BARS = 2 * MAX_PSTAGES + 2 * USTAGES + 2 * 2 + 1;
 // Output staging for the TMA stores: per epilogue warp one 32 x 32 block of
 // int32 and one of fp32 (4 KiB each, 128B-swizzled rows of 32 values).
 constexpr int OUT_BLOCK = 32 * 32 * 4;
@@ -71,36 +65,128 @@ constexpr int OUT_BYTES = EPI_WARPS * 2 * OUT_BLOCK;
 // Per-tile column parameters, one copy shared by the epilogue warps, double
 // buffered across tiles: float4 {alpha, gamma, beta, -} and int2 {c1, len2}.
 constexpr int COLP_BYTES = 2 * BN_MAX * (16 + 8);
-constexpr int SMEM_FIXED = USTAGES * U_STAGE + OUT_BYTES + COLP_BYTES + NUM_BARS * 8 + 16 + 1024;
-constexpr int PSTAGES = (tc::SMEM_LIMIT - SMEM_FIXED) / P_STAGE < MAX_PSTAGES
-                            ? (tc::SMEM_LIMIT - SMEM_FIXED) / P_STAGE
-                            : MAX_PSTAGES;
-constexpr int SMEM_BYTES = SMEM_FIXED + PSTAGES * P_STAGE;
-static_assert(PSTAGES >= 4, "packed ring too shallow");
-static_assert(U_STAGE % 1024 == 0 && OUT_BLOCK % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert(ACC_STRIDE + BN_MAX <= SF_COL, "accumulators overlap the scale factors");
+static_assert(U_A_BYTES % 1024 == 0 && OUT_BLOCK % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 // Named barrier of the epilogue warps (id 0 is __syncthreads).
 constexpr int EPI_BAR = 1;
-static_assert(SMEM_BYTES <= tc::SMEM_LIMIT, "shared memory");
-static_assert(ACC_STRIDE + BN_MAX <= SF_COL, "accumulators overlap the scale factors");
 // Largest padded K: partial sums stay integers of magnitude <= 2^20, exact
 // in fp32 and in the epilogue's float-to-int conversion (valid below 2^22).
 constexpr int64_t MAX_KP = int64_t(1) << 20;
+
+// Geometry of one CTA.  Single: the CTA owns a 128 x bn tile.  Pair
+// (cta_group::2, a cluster of two CTAs on two SMs): the pair owns a 256 x bn
+// tile; each CTA holds its 128 A rows and half of the bn W rows in its
+// shared memory and its 128 x bn accumulator in its tensor memory, and the
+// even CTA issues the MMAs for both.  Per multiply-add the pair moves
+// (128 + bn / 2) instead of (128 + bn) rows through each SM's shared memory.
+template <bool PAIR>
+struct Cfg {
+    static constexpr int CTAS = PAIR ? 2 : 1;
+    static constexpr int BN_CTA_MAX = BN_MAX / CTAS;            // W rows per CTA
+    static constexpr int USTAGES = PAIR ? 4 : 3;                // unpacked ring
+    static constexpr int U_B_BYTES = BN_CTA_MAX * ROW_BYTES;
+    static constexpr int U_STAGE = U_A_BYTES + U_B_BYTES;
+    static constexpr int P_STAGE = (BM + BN_CTA_MAX) * P_ROW;
+    static constexpr int UNPACK_WARPS = (BM + BN_CTA_MAX + 31) / 32;   // 11 single, 8 pair
+    static constexpr int WARP_EPI0 = WARP_UNPACK0 + UNPACK_WARPS;
+    static constexpr int THREADS = (WARP_EPI0 + EPI_WARPS) * 32;       // 544 single, 448 pair
+    static constexpr int NUM_BARS = 2 * MAX_PSTAGES + 2 * USTAGES + 2 * 2 + 1;
+    static constexpr int SMEM_FIXED = USTAGES * U_STAGE + OUT_BYTES + COLP_BYTES + NUM_BARS * 8 + 16 + 1024;
+    static constexpr int PSTAGES = (tc::SMEM_LIMIT - SMEM_FIXED) / P_STAGE < MAX_PSTAGES
+                                       ? (tc::SMEM_LIMIT - SMEM_FIXED) / P_STAGE
+                                       : MAX_PSTAGES;
+    static constexpr int SMEM_BYTES = SMEM_FIXED + PSTAGES * P_STAGE;
+    static_assert(PSTAGES >= 4, "packed ring too shallow");
+    static_assert(SMEM_BYTES <= tc::SMEM_LIMIT, "shared memory");
+    static_assert(U_STAGE % 1024 == 0 && P_STAGE % 256 == 0, "stage alignment (128B / 32B swizzle)");
+    static_assert((WARP_EPI0 & 3) == 0 || EPI_WARPS == 4, "the epilogue warps cover the four TMEM lane quadrants");
+};
 // Block-scaled instruction descriptor: A and B e2m1 (format 1 of kind::mxf4)
 // at bits 7-9 and 10-12, both K-major, N >> 3 at bits 17-22, scale format
-// ue8m0 (bit 23), M >> 4 at bits 24-28; scale-factor byte ids 0, K = 64.
-__host__ __device__ constexpr uint32_t idesc(int bn) {
-    return (1u << 7) | (1u << 10) | ((uint32_t)(bn >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24);
+// ue8m0 (bit 23), M >> 4 at bits 24-28 (M = 128 per CTA of the group);
+// scale-factor byte ids 0, K = 64.
+__host__ __device__ constexpr uint32_t idesc(int bn, int ctas) {
+    return (1u << 7) | (1u << 10) | ((uint32_t)(bn >> 3) << 17) | (1u << 23) | ((uint32_t)((BM * ctas) >> 4) << 24);
 }
 }  // namespace f4
 
+template <bool PAIR>
 __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    if constexpr (PAIR) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %6, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
+                d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %6, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
+                d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+            : "memory");
+    }
+}
+
+// Arrive on `bar` (the same shared-memory offset in every CTA of `mask`)
+// once the MMAs issued so far by this thread are done.
+template <bool PAIR>
+__device__ __forceinline__ void f4_commit(uint64_t* bar, uint16_t mask) {
+    if constexpr (PAIR) {
+        asm volatile(
+            "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                smem_u32(bar)),
+            "h"(mask)
+            : "memory");
+    } else {
+        mma_commit(bar);
+    }
+}
+
+template <bool PAIR>
+__device__ __forceinline__ void f4_tmem_alloc(uint32_t* dst, uint32_t ncols) {
+    if constexpr (PAIR) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
+                     "r"(ncols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+        tmem_alloc(dst, ncols);
+        tmem_relinquish();
+    }
+}
+template <bool PAIR>
+__device__ __forceinline__ void f4_tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    if constexpr (PAIR) {
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+    } else {
+        tmem_dealloc(taddr, ncols);
+    }
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive on the mbarrier at the same shared-memory offset in CTA `rank` of
+// the cluster (release semantics at the default CTA scope: what the arrival
+// publishes -- expanded bytes behind a proxy fence, or TMEM reads behind a
+// tcgen05 fence -- is consumed by the tensor core, which the waiting thread
+// orders after its wait with tcgen05.fence::after_thread_sync).
+__device__ __forceinline__ void mbar_arrive_remote(uint64_t* bar, uint32_t rank) {
     asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %6, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
-            d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        "{\n\t.reg .b32 ra;\n\t"
+        "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+        "mbarrier.arrive.shared::cluster.b64 _, [ra];\n\t}" ::"r"(smem_u32(bar)),
+        "r"(rank)
         : "memory");
 }
 
@@ -148,14 +234,18 @@ __device__ __forceinline__ int32_t acc_to_int(uint32_t bits) {
     return __float_as_int(__uint_as_float(bits) + 12582912.0f) - 0x4B400000;
 }
 
-__global__ void __launch_bounds__(f4::THREADS, 1)
+template <bool PAIR>
+__global__ void __launch_bounds__(f4::Cfg<PAIR>::THREADS, 1)
 xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                     const __grid_constant__ CUtensorMap tmCi, const __grid_constant__ CUtensorMap tmCf, int M, int N,
                     int K, int kw, int bn, int tiles_m, int tiles_n, int tma_out, GemmEpilogue ep) {
     using namespace f4;
+    using C = Cfg<PAIR>;
+    constexpr int CTAS = C::CTAS, USTAGES = C::USTAGES, PSTAGES = C::PSTAGES, U_STAGE = C::U_STAGE,
+                  P_STAGE = C::P_STAGE, UNPACK_WARPS = C::UNPACK_WARPS, WARP_EPI0 = C::WARP_EPI0;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint8_t* uring = smem;                                          // USTAGES x (A 16 KiB | W 28 KiB)
+    uint8_t* uring = smem;                                          // USTAGES x (A 16 KiB | W rows)
     uint8_t* oring = uring + USTAGES * U_STAGE;                     // [EPI_WARPS][int32 | fp32] 32 x 32 blocks
     uint8_t* pring = oring + OUT_BYTES;                             // PSTAGES x (A | W packed)
     float4* colf = reinterpret_cast<float4*>(pring + PSTAGES * P_STAGE);   // [2][BN_MAX]
@@ -175,7 +265,12 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const int lane = threadIdx.x & 31;
     const int nk = (kw + BKW - 1) / BKW;
     const int tiles = tiles_m * tiles_n;
-    const uint32_t stage_tx = (uint32_t)(BM + bn) * P_ROW;
+    // Pair: CTA `rank` of cluster `cid` holds A rows 128 rank .. of the
+    // tile's 256 and W rows bn_cta rank .. of its bn; the even CTA leads.
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const int cid = (int)blockIdx.x / CTAS, ncl = (int)gridDim.x / CTAS;
+    const int bn_cta = bn / CTAS;
+    const uint32_t stage_tx = (uint32_t)(BM + bn_cta) * P_ROW;
 
     if (threadIdx.x == 0) {
         prefetch_tensormap(&tmA);
@@ -187,31 +282,29 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             mbar_init(&pempty[s], UNPACK_WARPS);
         }
         for (int s = 0; s < USTAGES; ++s) {
-            mbar_init(&ufull[s], UNPACK_WARPS);
+            mbar_init(&ufull[s], UNPACK_WARPS * CTAS);          // the leader's: every unpack warp of the group
             mbar_init(&uempty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&afull[b], 1);
-            mbar_init(&aempty[b], EPI_WARPS);
+            mbar_init(&aempty[b], EPI_WARPS * CTAS);            // the leader's: every epilogue warp of the group
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
-    if (warp == WARP_MMA) {
-        tmem_alloc(tmem_slot, TMEM_COLS);
-        tmem_relinquish();
-    }
+    if (warp == WARP_MMA) f4_tmem_alloc<PAIR>(tmem_slot, TMEM_COLS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     // Unit scale factors: each epilogue warp fills its 32 lanes of the 32
     // scale-factor columns, so whatever TMEM layout the MMA reads them in,
-    // every factor it finds is 2^0.
+    // every factor it finds is 2^0.  In a pair both CTAs fill theirs before
+    // the cluster barrier, which also publishes the barrier inits to the peer.
     if (warp >= WARP_EPI0) tmem_fill32(tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + SF_COL, SF_ONE);
     tc_fence_before();
-    __syncthreads();
+    if constexpr (PAIR) cluster_sync_all(); else __syncthreads();
     tc_fence_after();
 
     if (warp == WARP_PRODUCER) {
@@ -219,8 +312,9 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         if (lane == 0) {
             uint32_t g = 0, issued = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
-                const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * bn;
+            for (int t = cid; ok && t < tiles; t += ncl) {
+                const int m0 = (t / tiles_n) * (BM * CTAS) + BM * (int)rank;
+                const int n0 = (t % tiles_n) * bn + bn_cta * (int)rank;
                 for (int ks = 0; ks < nk; ++ks, ++g) {
                     const uint32_t s = g % (uint32_t)PSTAGES;
                     if (g >= (uint32_t)PSTAGES && !tc_wait(&pempty[s], ((g / PSTAGES) - 1) & 1, abort_flag)) {
@@ -239,14 +333,17 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
     } else if (warp == WARP_MMA) {
         // ------------------------------ MMA issuer ------------------------------
-        if (lane == 0) {
+        // One thread of the leading CTA; its commits arrive on the barrier of
+        // every CTA of the group whose shared or tensor memory they free.
+        if (lane == 0 && rank == 0) {
+            constexpr uint16_t all = PAIR ? 0x3 : 0x1;
             uint32_t g = 0;
             int lt = 0;
             bool ok = true;
             const uint32_t ubase = smem_u32(uring);
-            const uint32_t id = idesc(bn);
+            const uint32_t id = idesc(bn, CTAS);
             const uint32_t sfa = tmem_base + SFA_COL, sfb = tmem_base + SFB_COL;
-            for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++lt) {
+            for (int t = cid; ok && t < tiles; t += ncl, ++lt) {
                 const int b = lt & 1;
                 if (lt >= 2 && !tc_wait(&aempty[b], ((lt >> 1) - 1) & 1, abort_flag)) break;
                 tc_fence_after();
@@ -263,65 +360,76 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     #pragma unroll
                     for (int kk = 0; kk < BKE / UMMA_K; ++kk) {
                         // 32 bytes (64 elements) per K step inside the swizzle atom.
-                        mma_mxf4(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32), id, sfa,
-                                 sfb, (ks | kk) != 0 ? 1u : 0u);
+                        mma_mxf4<PAIR>(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32),
+                                       id, sfa, sfb, (ks | kk) != 0 ? 1u : 0u);
                     }
-                    mma_commit(&uempty[s]);
+                    f4_commit<PAIR>(&uempty[s], all);
                 }
-                if (ok) mma_commit(&afull[b]);
+                if (ok) f4_commit<PAIR>(&afull[b], all);
             }
-            mma_commit(drain);
+            f4_commit<PAIR>(drain, 0x1);
             mbar_wait_bounded(drain, 0);
         }
         __syncwarp();
     } else if (warp < WARP_EPI0) {
         // ------------------------------ unpack warps ------------------------------
-        // Thread u expands packed row u of the stage (A rows 0..127, then W
-        // rows 0..bn-1) into 128 bytes.  Rows are 32 bytes apart in the packed
+        // Thread u expands packed row u of the stage (A rows 0..127, then the
+        // CTA's W rows) into 128 bytes.  Rows are 32 bytes apart in the packed
         // stage, written by the TMA with the 32-byte swizzle: half h of row u
         // sits at 16 * (h ^ ((u >> 2) & 1)), so the eight lanes of a 16-byte
         // load phase hit distinct banks, while the words keep their order for
         // the conflict-free swizzled stores below.
-        const int u = threadIdx.x - WARP_UNPACK0 * 32;               // 0 .. BM + BN_MAX - 1
+        const int u = threadIdx.x - WARP_UNPACK0 * 32;
         const bool is_a = u < BM;
         const int r = is_a ? u : u - BM;
-        const bool active = is_a || r < bn;
+        const bool active = is_a || r < bn_cta;
         const int sw = r & 7;
         const int hsw = 16 * ((u >> 2) & 1);
-        uint32_t g = 0;
-        bool ok = true;
-        for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
-            for (int ks = 0; ks < nk; ++ks, ++g) {
-                const uint32_t ps = g % (uint32_t)PSTAGES, us = g % USTAGES;
-                const bool w1 = tc_wait(&pfull[ps], (g / PSTAGES) & 1, abort_flag);
-                const bool w2 = w1 && (g < USTAGES || tc_wait(&uempty[us], ((g / USTAGES) - 1) & 1, abort_flag));
-                if (!__all_sync(0xffffffffu, w1 && w2)) {
-                    ok = false;
-                    break;
-                }
-                uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;      // words 0..3 and 4..7 of the row
-                if (active) {
-                    const uint8_t* src = pring + ps * P_STAGE + u * P_ROW;
-                    lo = *reinterpret_cast<const uint4*>(src + hsw);
-                    hi = *reinterpret_cast<const uint4*>(src + (hsw ^ 16));
-                }
-                release_packed_stage(&pempty[ps], lane);
-                if (active) {
-                    // Chunk q of the row at (q ^ (r & 7)) * 16: the eight lanes of a
-                    // store phase (eight consecutive rows) hit distinct banks.
-                    uint8_t* row = uring + us * U_STAGE + (is_a ? 0 : U_A_BYTES) + r * ROW_BYTES;
-                    *reinterpret_cast<uint4*>(row + ((0 ^ sw) << 4)) = expand_word_e2m1(lo.x);
-                    *reinterpret_cast<uint4*>(row + ((1 ^ sw) << 4)) = expand_word_e2m1(lo.y);
-                    *reinterpret_cast<uint4*>(row + ((2 ^ sw) << 4)) = expand_word_e2m1(lo.z);
-                    *reinterpret_cast<uint4*>(row + ((3 ^ sw) << 4)) = expand_word_e2m1(lo.w);
-                    *reinterpret_cast<uint4*>(row + ((4 ^ sw) << 4)) = expand_word_e2m1(hi.x);
-                    *reinterpret_cast<uint4*>(row + ((5 ^ sw) << 4)) = expand_word_e2m1(hi.y);
-                    *reinterpret_cast<uint4*>(row + ((6 ^ sw) << 4)) = expand_word_e2m1(hi.z);
-                    *reinterpret_cast<uint4*>(row + ((7 ^ sw) << 4)) = expand_word_e2m1(hi.w);
-                }
-                fence_proxy_async_shared();                           // the bytes, visible to the tensor core
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&ufull[us]);
+        // The stages of all of this CTA's tiles form one sequence; the packed
+        // words of stage g + 1 are loaded as soon as stage g is stored, so when
+        // the MMAs free the next unpacked buffer the warp only expands.
+        const int my_tiles = cid < tiles ? (tiles - 1 - cid) / ncl + 1 : 0;
+        const uint32_t total = (uint32_t)my_tiles * (uint32_t)nk;
+        uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;              // words 0..3 and 4..7 of the row
+        auto load_packed = [&](uint32_t gg) -> bool {
+            const uint32_t ps = gg % (uint32_t)PSTAGES;
+            if (!__all_sync(0xffffffffu, tc_wait(&pfull[ps], (gg / PSTAGES) & 1, abort_flag))) return false;
+            if (active) {
+                const uint8_t* src = pring + ps * P_STAGE + u * P_ROW;
+                lo = *reinterpret_cast<const uint4*>(src + hsw);
+                hi = *reinterpret_cast<const uint4*>(src + (hsw ^ 16));
+            }
+            return true;
+        };
+        bool ok = total == 0 || load_packed(0);
+        for (uint32_t g = 0; ok && g < total; ++g) {
+            const uint32_t ps = g % (uint32_t)PSTAGES, us = g % USTAGES;
+            if (!__all_sync(0xffffffffu, g < USTAGES || tc_wait(&uempty[us], ((g / USTAGES) - 1) & 1, abort_flag)))
+                break;
+            if (active) {
+                // Chunk q of the row at (q ^ (r & 7)) * 16: the eight lanes of a
+                // store phase (eight consecutive rows) hit distinct banks.
+                uint8_t* row = uring + us * U_STAGE + (is_a ? 0 : U_A_BYTES) + r * ROW_BYTES;
+                *reinterpret_cast<uint4*>(row + ((0 ^ sw) << 4)) = expand_word_e2m1(lo.x);
+                *reinterpret_cast<uint4*>(row + ((1 ^ sw) << 4)) = expand_word_e2m1(lo.y);
+                *reinterpret_cast<uint4*>(row + ((2 ^ sw) << 4)) = expand_word_e2m1(lo.z);
+                *reinterpret_cast<uint4*>(row + ((3 ^ sw) << 4)) = expand_word_e2m1(lo.w);
+                *reinterpret_cast<uint4*>(row + ((4 ^ sw) << 4)) = expand_word_e2m1(hi.x);
+                *reinterpret_cast<uint4*>(row + ((5 ^ sw) << 4)) = expand_word_e2m1(hi.y);
+                *reinterpret_cast<uint4*>(row + ((6 ^ sw) << 4)) = expand_word_e2m1(hi.z);
+                *reinterpret_cast<uint4*>(row + ((7 ^ sw) << 4)) = expand_word_e2m1(hi.w);
+            }
+            if (g + 1 < total) ok = load_packed(g + 1);
+            // One proxy fence orders this thread's reads of the packed stage
+            // before its next TMA refill and its expanded bytes before the
+            // tensor core's reads; then the warp releases the one and hands
+            // the other to the MMA issuer (in the leading CTA).
+            fence_proxy_async_shared();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&pempty[ps]);
+                if (rank == 0) mbar_arrive(&ufull[us]);
+                else mbar_arrive_remote(&ufull[us], 0);
             }
         }
     } else {
@@ -354,9 +462,9 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const uint32_t sw = (uint32_t)(lane & 7);
         bool ok = true;
         int lt = 0;
-        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++lt) {
+        for (int t = cid; t < tiles; t += ncl, ++lt) {
             const int b = lt & 1;
-            const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * bn;
+            const int m0 = (t / tiles_n) * (BM * CTAS) + BM * (int)rank, n0 = (t % tiles_n) * bn;
             float4* cf = colf + b * BN_MAX;
             int2* ct = colt + b * BN_MAX;
             // Every warp finished tile lt - 2 (the last reader of this copy)
@@ -399,9 +507,13 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 uint32_t r[32];
                 tmem_ld32_sync(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * ACC_STRIDE + 32 * c), r);
                 if (c == chunks - 1) {
+                    // Whole accumulator read: hand it back to the MMA issuer.
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&aempty[b]);
+                    if (lane == 0) {
+                        if (rank == 0) mbar_arrive(&aempty[b]);
+                        else mbar_arrive_remote(&aempty[b], 0);
+                    }
                 }
                 const int nb = n0 + 32 * c;
                 if (nb >= N) {
@@ -505,11 +617,14 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
 
     // ------------------------------ teardown ------------------------------
+    // In a pair the leader's MMAs read the peer's shared and tensor memory
+    // and its commits arrive on the peer's barriers: neither CTA leaves (or
+    // frees its tensor memory) before both are done.
     tc_fence_before();
-    __syncthreads();
+    if constexpr (PAIR) cluster_sync_all(); else __syncthreads();
     if (warp == WARP_MMA) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        f4_tmem_dealloc<PAIR>(tmem_base, TMEM_COLS);
     }
 }
 
