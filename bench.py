@@ -492,6 +492,8 @@ def run_only_rows(args, torch, dist):
             dist.barrier()
 
     names = [n for n in args.only_rows.split(",") if n]
+    if args.square_shape:
+        _row_square.shape = tuple(int(v) for v in args.square_shape.split(","))
     for n in names:
         if n not in ROW_NAMES:
             raise SystemExit(f"unknown row {n!r}; choose from {ROW_NAMES}")
@@ -617,7 +619,8 @@ def _tensor_roofline(pk, macs_per_s, sustained, row=None, operand="int8", kernel
 
 def _row_square(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, clk_mhz, pk=None):
     # --- a2+a3+a6: square GEMM 8192^3, int32 + alpha-scaled fp32 outputs, both engines ---
-    sq = workloads.square()
+    shape = getattr(_row_square, "shape", None)
+    sq = workloads.square(*shape) if shape else workloads.square()
     Ad = sq.A.to(dev)
     A_p = bnn.empty_packed(sq.M, sq.K, dev)
     Wsq = bnn.empty_packed(sq.N, sq.K, dev)
@@ -648,7 +651,7 @@ def _row_square(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, cl
             kernel = "xnor_gemm_popc_kernel"
             label = "popcount (XOR + POPC, carry-save)"
         rows[name] = {
-            "workload": "M=N=K=8192 packed A x packed W^T, int32 s + alpha*s fp32 out",
+            "workload": f"M={sq.M} N={sq.N} K={sq.K} packed A x packed W^T, int32 s + alpha*s fp32 out",
             "engine": label,
             "kernel": kernel,
             "value": round(ws * mac_s / 1e9, 1), "unit": "binary GMAC/s", "tops": round(ws * 2 * mac_s / 1e12, 2),
@@ -1328,9 +1331,14 @@ def main():
     ap.add_argument("--only-rows", default=None,
                     help="comma-separated rows to time alone (no headline line); for profiling: "
                          + ",".join(ROW_NAMES))
+    ap.add_argument("--square-shape", default=None,
+                    help="M,N,K of the square_gemm row in an --only-rows run (a smaller case of the same "
+                         "kernel for profiling; default 8192,8192,8192)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.square_shape is not None and args.only_rows is None:
+        ap.error("--square-shape only applies to --only-rows runs")
 
     ws, rank, local = dist_env()
     if args.impl == "reference":

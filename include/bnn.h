@@ -217,7 +217,7 @@ bnn_status bnn_pack_conv3x3_weights(const void* w_oihw, bnn_dtype dt, int64_t co
                                     bnn_stream_t stream);
 
 /* Engine used by bnn_xnor_gemm, bnn_binary_linear_fused and
- * bnn_binary_conv3x3_fused.  Both engines return identical results (the
+ * bnn_binary_conv3x3_fused.  All engines return identical results (the
  * product is exact integer arithmetic):
  *   POPCOUNT: XOR + population count on the integer pipes, with carry-save
  *             compression (any shape).
