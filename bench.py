@@ -1057,6 +1057,31 @@ def _row_mlp(torch, bnn, workloads, dev, rows, timed, steps, ws, alu_peak, pk=No
 # CPU oracle timing (the baseline, never the product path)
 # ---------------------------------------------------------------------------
 
+def rows_summary(result: dict) -> dict:
+    """One compact entry per figure, placed last on the line so that a reader
+    of the line's end sees every row: [value, unit, roofline fraction,
+    microseconds per step]."""
+    out = {}
+    if "value" in result:
+        rf = result.get("roofline", {})
+        out["headline"] = [result["value"], result["unit"], rf.get("frac"), round(result["ms_per_step"] * 1e3, 3)]
+        for k in ("store_ordered", "dependent_chain", "gemv_default_flags", "e2e"):
+            v = result.get(k)
+            if isinstance(v, dict) and "value" in v:
+                out[k] = [v["value"], v["unit"], v.get("frac"), round(v["ms_per_step"] * 1e3, 3)]
+    for name, row in result.get("rows", {}).items():
+        if not isinstance(row, dict) or "value" not in row:
+            continue
+        rf = row.get("roofline", {})
+        ms = row.get("ms_per_step")
+        out[name] = [row["value"], row["unit"], rf.get("frac"), round(ms * 1e3, 3) if ms is not None else None]
+        dep = row.get("dependent_chain")
+        if isinstance(dep, dict) and "value" in dep:
+            out[name + ".dependent_chain"] = [dep["value"], dep["unit"], dep.get("frac"),
+                                              round(dep["ms_per_step"] * 1e3, 3)]
+    return out
+
+
 def cpu_model() -> str:
     try:
         for line in open("/proc/cpuinfo"):
@@ -1363,6 +1388,8 @@ def main():
         else:
             result = run_ours(args, torch, dist)
         if rank == 0:
+            if "rows" in result:
+                result["summary"] = rows_summary(result)
             print(json.dumps(result), flush=True)
     finally:
         if dist is not None:
