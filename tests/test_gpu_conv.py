@@ -12,7 +12,8 @@ from gpu_util import assert_affine_close, assert_no_device_error, assert_scaled_
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(params=[bnn.BNN_GEMM_ENGINE_POPCOUNT, bnn.BNN_GEMM_ENGINE_TENSOR], ids=["popcount", "tensor"])
+@pytest.fixture(params=[bnn.BNN_GEMM_ENGINE_POPCOUNT, bnn.BNN_GEMM_ENGINE_TENSOR, bnn.BNN_GEMM_ENGINE_TENSOR_I8],
+                ids=["popcount", "tensor", "tensor_i8"])
 def engine(request):
     """TENSOR runs the tcgen05 convolution where it applies (c <= 64,
     cout <= 256); other shapes stay on the popcount kernel."""
@@ -109,10 +110,13 @@ def test_conv_window_segments(n, c, h, w, cout):
     assert_no_device_error()
 
 
-def test_tensor_conv_full_output_repeated():
+@pytest.mark.parametrize("tensor_engine", [bnn.BNN_GEMM_ENGINE_TENSOR, bnn.BNN_GEMM_ENGINE_TENSOR_I8],
+                         ids=["tensor", "tensor_i8"])
+def test_tensor_conv_full_output_repeated(tensor_engine):
     """Races show up as a few wrong tiles in some launches only: the ResNet
-    layer runs 4 times on the tensor-core window kernel (INT32 output) and all
-    12.8M outputs are compared with the popcount kernel's."""
+    layer runs 4 times on the tensor-core window kernel (e2m1 and int8
+    operands; INT32 output) and all 12.8M outputs are compared with the
+    popcount kernel's."""
     cv = workloads.conv()
     d = dev()
     n, c, h, w = cv.X.shape
@@ -125,7 +129,7 @@ def test_tensor_conv_full_output_repeated():
     with bnn.gemm_engine(bnn.BNN_GEMM_ENGINE_POPCOUNT):
         bnn.bnn_binary_conv3x3_fused(Xb, c, Wp, ep, ref, 1, 1)
     out = torch.empty_like(ref)
-    with bnn.gemm_engine(bnn.BNN_GEMM_ENGINE_TENSOR):
+    with bnn.gemm_engine(tensor_engine):
         for r in range(4):
             out.fill_(0x5A5A5A5A)
             bnn.bnn_binary_conv3x3_fused(Xb, c, Wp, ep, out, 1, 1)

@@ -1175,14 +1175,14 @@ bnn_status bnn_binary_linear_fused(const uint32_t* A, int64_t lda, const uint32_
 // fit in shared memory next to the resident filters.  BNN_ERR_UNSUPPORTED
 // when a buffer cannot hold one tile's window.
 static bnn_status conv_window_plan(int64_t n, int64_t h, int64_t w, int64_t pad, int64_t cw, int64_t n_mma,
-                                   bnn::ConvWindow* g) {
+                                   bool f4, bnn::ConvWindow* g) {
     const int64_t Hp = h + 2 * pad, Wp = w + 2 * pad;
     const int64_t V = n * Hp * Wp;
     const int64_t halo = 2 * Wp + 2;
     if (V + 2 * halo + 256 > INT_MAX) return BNN_ERR_UNSUPPORTED;
     const int64_t tiles = ceil_div(V, (int64_t)bnn::ctw::BM);
-    const int64_t fixed = bnn::conv_tcw_smem_bytes((int)cw, (int)n_mma, 0);
-    int64_t rb = (227 * 1024 - fixed) / (2 * cw * 32);
+    const int64_t fixed = bnn::conv_tcw_smem_bytes((int)cw, (int)n_mma, 0, f4);
+    int64_t rb = (227 * 1024 - fixed) / (2 * bnn::conv_tcw_row_bytes((int)cw, f4));
     rb = std::min<int64_t>(rb, 16000) / 8 * 8;
     const int64_t grid = std::min<int64_t>(tiles, sm_count());
     const int64_t per_cta = ceil_div(tiles, grid);
@@ -1228,7 +1228,12 @@ bnn_status bnn_binary_conv3x3_fused(const uint32_t* X_nhwc_bits, int64_t n, int6
     bnn::ConvEpilogue ep{epi->mode, epi->alpha, epi->gamma, epi->beta, out_nchw};
     cudaStream_t s = as_cuda(stream);
     int engine = g_gemm_engine.load(std::memory_order_relaxed);
-    if (engine == BNN_GEMM_ENGINE_TENSOR_I8) engine = BNN_GEMM_ENGINE_TENSOR;   // the conv kernels are int8 only
+    // The window kernel runs on e2m1 operands where two words of K fit one
+    // MMA (cw even) and the scale factors fit beside the two accumulators,
+    // on int8 operands otherwise and under TENSOR_I8; the other tensor-core
+    // kernel is int8 only.
+    const bool i8_only = engine == BNN_GEMM_ENGINE_TENSOR_I8;
+    if (i8_only) engine = BNN_GEMM_ENGINE_TENSOR;
     const int64_t n_mma = std::max<int64_t>(16, ceil_div(cout, (int64_t)16) * 16);
     // Tensor cores, stride 1: the shifted-window kernel, when the resident
     // filters and two A buffers of at least one tile's window fit.  AUTO takes
@@ -1238,12 +1243,14 @@ bnn_status bnn_binary_conv3x3_fused(const uint32_t* X_nhwc_bits, int64_t n, int6
     const bool tc_window = engine == BNN_GEMM_ENGINE_TENSOR ||
                            (engine == BNN_GEMM_ENGINE_AUTO && cout >= 64 && cw <= 2 && npix >= 16384);
     if (tc_window && stride == 1 && cout <= bnn::ctc::MAX_N) {
+        const bool f4 = !i8_only && cw % 2 == 0 && 2 * ceil_div(n_mma, (int64_t)32) * 32 + 32 <= 512;
         bnn::ConvWindow g{};
-        const bnn_status st = conv_window_plan(n, h, w, pad, cw, n_mma, &g);
+        const bnn_status st = conv_window_plan(n, h, w, pad, cw, n_mma, f4, &g);
         if (st == BNN_OK) {
-            const int smem_w = bnn::conv_tcw_smem_bytes((int)cw, (int)n_mma, g.rb);
-            const uint32_t idesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n_mma >> 3) << 17) |
-                                   ((uint32_t)(bnn::ctw::BM >> 4) << 24);
+            const int smem_w = bnn::conv_tcw_smem_bytes((int)cw, (int)n_mma, g.rb, f4);
+            const uint32_t idesc = f4 ? bnn::f4::idesc((int)n_mma, 1)
+                                      : (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n_mma >> 3) << 17) |
+                                            ((uint32_t)(bnn::ctw::BM >> 4) << 24);
             const int grid = std::min(g.tiles, sm_count());
             auto launch_w = [&](auto kern) -> bnn_status {
                 if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_w) != cudaSuccess)
@@ -1252,6 +1259,8 @@ bnn_status bnn_binary_conv3x3_fused(const uint32_t* X_nhwc_bits, int64_t n, int6
                                                                        (int)n_mma, idesc, g, ep);
                 return launch_status();
             };
+            if (f4) return cw == 2 ? launch_w(bnn::xnor_conv3x3_tcw_kernel<2, true>)
+                                   : launch_w(bnn::xnor_conv3x3_tcw_kernel<4, true>);
             switch (cw) {
                 case 1: return launch_w(bnn::xnor_conv3x3_tcw_kernel<1>);
                 case 2: return launch_w(bnn::xnor_conv3x3_tcw_kernel<2>);

@@ -30,6 +30,7 @@
 #include "common.cuh"
 #include "conv.cuh"      // ConvEpilogue
 #include "gemm_tc.cuh"   // tcgen05 helpers, expand_word_pm1, umma_desc_sw128
+#include "gemm_f4.cuh"   // e2m1 expansion, kind::mxf4 MMA, unit scale factors
 
 namespace bnn {
 namespace ctc {
@@ -293,10 +294,18 @@ struct ConvWindow {
     int halo;        // 2 * Wp + 2
 };
 
+// Operand geometry of the window kernel.  int8 (+1/-1 bytes): an A row is
+// 32 bytes per packed word, a filter stage 128 elements.  e2m1 (+1/-1
+// nibbles, F4): 16 bytes per word, 256 elements per filter stage.
+__host__ __device__ constexpr int conv_tcw_row_bytes(int cw, bool f4) { return cw * (f4 ? 16 : 32); }
+__host__ __device__ constexpr int conv_tcw_b_stages(int cw, bool f4) {
+    return f4 ? (9 * cw + 7) / 8 : conv_tc_stages(cw);
+}
 // Shared-memory bytes for CW words per pixel, n_mma filter rows and rb rows
 // per A buffer.
-__host__ __device__ inline int conv_tcw_smem_bytes(int cw, int n_mma, int rb) {
-    return 1024 + conv_tc_stages(cw) * n_mma * 128 + 2 * rb * cw * 32 + 12 * n_mma + ctw::BAR_BYTES;
+__host__ __device__ inline int conv_tcw_smem_bytes(int cw, int n_mma, int rb, bool f4 = false) {
+    return 1024 + conv_tcw_b_stages(cw, f4) * n_mma * 128 + 2 * rb * conv_tcw_row_bytes(cw, f4) + 12 * n_mma +
+           ctw::BAR_BYTES;
 }
 
 // Non-swizzled K-major shared-memory descriptor: rows 16 B apart inside a
@@ -307,18 +316,23 @@ __device__ __forceinline__ uint64_t umma_desc_interleave(uint32_t smem_addr, uin
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1u << 46);
 }
 
-template <int CW>
+// F4: the same kernel on e2m1 operands (tcgen05.mma kind::mxf4 with unit
+// block scales, CW even): a pixel's word expands to 16 bytes instead of 32,
+// one K = 64 MMA covers two words, and the fp32 accumulators hold exact
+// integers (at most 9 * 32 * CW in magnitude).
+template <int CW, bool F4 = false>
 __global__ void __launch_bounds__(ctw::THREADS, 1)
 xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* __restrict__ Wp_,
                         int64_t ldw, int cout, int n_mma, uint32_t idesc, ConvWindow g, ConvEpilogue ep) {
     using namespace ctw;
+    static_assert(!F4 || CW % 2 == 0, "e2m1 MMAs take two words of K");
     constexpr int KW = 9 * CW;
-    constexpr int NS = conv_tc_stages(CW);
-    constexpr int KWP = 4 * NS;
+    constexpr int NS = conv_tcw_b_stages(CW, F4);
+    constexpr int KWP = (F4 ? 8 : 4) * NS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* bsm = smem;                                                   // NS x n_mma x 128 B, SW128
-    const int abuf_stride = g.rb * CW * 32;
+    const int abuf_stride = g.rb * conv_tcw_row_bytes(CW, F4);
     uint8_t* abuf = bsm + NS * n_mma * 128;                                // 2 x abuf_stride
     float* s_alpha = reinterpret_cast<float*>(abuf + 2 * abuf_stride);     // [n_mma]
     float* s_gamma = s_alpha + n_mma;
@@ -340,7 +354,10 @@ xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* _
     const int kt = te - tb;
     const int HpWp = g.Hp * g.Wp;
     const int acc_stride = (n_mma + 31) / 32 * 32;
-    const uint32_t tmem_cols = acc_stride <= 64 ? 128u : (acc_stride <= 128 ? 256u : 512u);
+    // e2m1: 32 columns of unit scale factors after the two accumulators.
+    const int used_cols = 2 * acc_stride + (F4 ? 32 : 0);
+    const uint32_t tmem_cols = used_cols <= 128 ? 128u : (used_cols <= 256 ? 256u : 512u);
+    const uint32_t sf_col = (uint32_t)(2 * acc_stride);
 
     for (int i = threadIdx.x; i < n_mma; i += blockDim.x) {
         const bool real = i < cout && ep.mode != BNN_OUT_INT32;
@@ -370,6 +387,15 @@ xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* _
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    if constexpr (F4) {
+        // The first four epilogue warps (one per TMEM lane quadrant) write
+        // the scale factors, all 2^0, before the first MMA.
+        if (warp >= WARP_EPI0 && warp < WARP_EPI0 + 4)
+            tmem_fill32(tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + sf_col, f4::SF_ONE);
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
 
     if (warp == WARP_MMA) {
         // ------------------------------ MMA issuer ------------------------------
@@ -395,21 +421,30 @@ xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* _
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(b * acc_stride);
                 const uint32_t a_tile = ad_lo + (uint32_t)(((seg & 1) * abuf_stride) >> 4) + (uint32_t)(ks * BM);
+                // One K step is 32 bytes of a row: two A planes (khalf apart)
+                // and two 16-byte chunks of a filter stage; int8 takes one
+                // word per step, e2m1 two.
+                constexpr int STEPS = F4 ? CW / 2 : CW;                  // K steps per tap
                 #pragma unroll
                 for (int tap = 0; tap < 9; ++tap) {
                     const uint32_t a_tap = a_tile + row_dy[tap / 3] + (uint32_t)(tap % 3);
                     #pragma unroll
-                    for (int j = 0; j < CW; ++j) {
-                        const int wk = tap * CW + j;
+                    for (int j = 0; j < STEPS; ++j) {
+                        const int wk = tap * STEPS + j;
                         const uint64_t ad = ((uint64_t)ad_hi << 32) | (a_tap + (uint32_t)j * khalf);
                         const uint64_t bd = ((uint64_t)bd_hi << 32) |
                                             (bd_lo + (uint32_t)(wk / 4) * bstage + (uint32_t)((wk % 4) * 2));
-                        asm volatile(
-                            "{\n\t.reg .pred p;\n\t"
-                            "setp.ne.b32 p, %4, 0;\n\t"
-                            "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-                            "l"(ad), "l"(bd), "r"(idesc), "r"(wk != 0 ? 1u : 0u)
-                            : "memory");
+                        if constexpr (F4) {
+                            mma_mxf4<false>(d_tmem, ad, bd, idesc, tmem_base + sf_col, tmem_base + sf_col + 16,
+                                            wk != 0 ? 1u : 0u);
+                        } else {
+                            asm volatile(
+                                "{\n\t.reg .pred p;\n\t"
+                                "setp.ne.b32 p, %4, 0;\n\t"
+                                "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+                                "l"(ad), "l"(bd), "r"(idesc), "r"(wk != 0 ? 1u : 0u)
+                                : "memory");
+                        }
                     }
                 }
                 mma_commit(&accfull[b]);
@@ -429,8 +464,14 @@ xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* _
             #pragma unroll
             for (int s = 0; s < NS; ++s) {
                 uint8_t* row = bsm + s * n_mma * 128 + fr * 128;
-                #pragma unroll
-                for (int q = 0; q < 4; ++q) expand_word_sw128(row, q, fr & 7, wd[4 * s + q]);
+                if constexpr (F4) {
+                    #pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        *reinterpret_cast<uint4*>(row + ((q ^ (fr & 7)) << 4)) = expand_word_e2m1(wd[8 * s + q]);
+                } else {
+                    #pragma unroll
+                    for (int q = 0; q < 4; ++q) expand_word_sw128(row, q, fr & 7, wd[4 * s + q]);
+                }
             }
         }
         for (int k = 0; k < kt; ++k) {
@@ -462,10 +503,14 @@ xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* _
                 }
                 #pragma unroll
                 for (int j = 0; j < CW; ++j) {
-                    uint4 c0, c1;
-                    expand_word_pm1(wd[j], c0, c1);
-                    *reinterpret_cast<uint4*>(ab + (2 * j) * g.rb * 16 + row * 16) = c0;
-                    *reinterpret_cast<uint4*>(ab + (2 * j + 1) * g.rb * 16 + row * 16) = c1;
+                    if constexpr (F4) {
+                        *reinterpret_cast<uint4*>(ab + j * g.rb * 16 + row * 16) = expand_word_e2m1(wd[j]);
+                    } else {
+                        uint4 c0, c1;
+                        expand_word_pm1(wd[j], c0, c1);
+                        *reinterpret_cast<uint4*>(ab + (2 * j) * g.rb * 16 + row * 16) = c0;
+                        *reinterpret_cast<uint4*>(ab + (2 * j + 1) * g.rb * 16 + row * 16) = c1;
+                    }
                 }
             }
             fence_proxy_async_shared();
@@ -506,6 +551,12 @@ xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* _
                     arrived = true;
                 }
                 if (!valid) continue;
+                if constexpr (F4) {
+                    // fp32 accumulators holding integers (|acc| < 2^22): read
+                    // them as the int32 values the int8 path produces.
+                    #pragma unroll
+                    for (int jj = 0; jj < EPI_COLS; ++jj) rr[jj] = (uint32_t)acc_to_int(rr[jj]);
+                }
                 if (ep.mode == BNN_OUT_INT32) {
                     int32_t* o = static_cast<int32_t*>(ep.out) + obase;
                     #pragma unroll
