@@ -895,11 +895,16 @@ def _row_multibit(torch, bnn, workloads, dev, pk, rows, timed, steps, ws):
     mac_s = macs * steps / (ms_g * 1e-3)
     pbytes = M * K + A.numel() * 4
     pack_gbs = pbytes * steps / (ms_p * 1e-3) / 1e9
-    roof = _tensor_roofline(pk, mac_s, sustained=False)
-    roof["traffic"] = recorded_traffic("bitserial_gemm", "xnor_gemm_tc_kernel<TC_PLANE_CODES>")
+    # Codes of up to two bits run on the e2m1 kernel (exact e2m1 values 0..3), wider ones on int8.
+    f4 = max(bs.a_bits, bs.w_bits) <= 2
+    kname = "xnor_gemm_f4_kernel" if f4 else "xnor_gemm_tc_kernel"
+    roof = _tensor_roofline(pk, mac_s, sustained=False, operand="e2m1" if f4 else "int8")
+    roof["traffic"] = recorded_traffic("bitserial_gemm", kname + ("<TC_PLANE_CODES>" if not f4 else ""))
     rows["bitserial_gemm"] = {
         "workload": f"DoReFa-style unsigned codes: a [{M}, {K}] {bs.a_bits}-bit x w [{N}, {K}] {bs.w_bits}-bit as bit "
-                    f"planes -> exact int32 sum_k a*w (planes folded to u8 codes, tcgen05 kind::i8 unsigned)",
+                    f"planes -> exact int32 sum_k a*w (planes folded to "
+                    + ("e2m1 code values, tcgen05 kind::mxf4, CTA pairs)" if f4 else "u8 codes, tcgen05 kind::i8)"),
+        "kernel": kname,
         "value": round(ws * mac_s / 1e9, 1), "unit": "code GMAC/s",
         "plane_pair_gmac_s": round(ws * mac_s * bs.a_bits * bs.w_bits / 1e9, 1),
         "ms_per_step": ms_g / steps, "roofline": roof,
@@ -926,13 +931,14 @@ def _row_multibit(torch, bnn, workloads, dev, pk, rows, timed, steps, ws):
     jp, ip = 1 << (J - 1).bit_length(), 1 << (I - 1).bit_length()
     bmacs = M * N * K * J * I
     bmac_s = bmacs * steps / (ms_b * 1e-3)
-    roof_b = _tensor_roofline(pk, bmac_s, sustained=False)
-    roof_b["traffic"] = recorded_traffic("binary_bases_gemm", "xnor_gemm_tc_kernel<TC_BASES>")
+    roof_b = _tensor_roofline(pk, bmac_s, sustained=False, operand="e2m1")
+    roof_b["traffic"] = recorded_traffic("binary_bases_gemm", "xnor_gemm_f4_kernel")
     roof_b["note"] = (f"{J} x {I} bases run as {jp} x {ip} (zero bases fill the power-of-two tile): "
                       f"the tensor pipe does {jp * ip / (J * I):.2f}x the algorithmic MACs")
     rows["binary_bases_gemm"] = {
         "workload": f"ABC-Net-style bases: {J} activation bases [{M}, {K}] x {I} weight bases [{N}, {K}], "
                     f"Y = sum_j sum_i beta_j alpha_i[n] (H_j B_i^T) fp32",
+        "kernel": "xnor_gemm_f4_kernel (bases mode, CTA pairs)",
         "value": round(ws * bmac_s / 1e9, 1), "unit": "binary GMAC/s (all base pairs)",
         "ms_per_step": ms_b / steps, "roofline": roof_b,
         "l2": f"{R} rotating activation-base / output sets"}

@@ -127,7 +127,12 @@ int gemm_f4_pairs_resident() {
     if (cudaFuncSetAttribute(bnn::xnor_gemm_f4_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C1::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(bnn::xnor_gemm_f4_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C2::SMEM_BYTES) != cudaSuccess)
+                             C2::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(bnn::xnor_gemm_f4_kernel<true, bnn::TC_PLANE_CODES>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bnn::f4::Cfg<true, bnn::TC_PLANE_CODES>::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(bnn::xnor_gemm_f4_kernel<true, bnn::TC_BASES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bnn::f4::Cfg<true, bnn::TC_BASES>::SMEM_BYTES) != cudaSuccess)
         return -1;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
@@ -283,6 +288,50 @@ F4Plan f4_plan(int64_t M, int64_t N, int64_t sms, int64_t pairs) {
     return best;
 }
 
+// Tile width of a CTA-pair e2m1 launch whose tiles hold bn / per_col output
+// columns: the multiple of 32 up to 224 that minimises (rounds of tiles over
+// the resident pairs) x (rows per stage, 128 + bn / 2).
+int f4_pair_tile_n(int64_t tiles_m, int64_t N, int per_col, int64_t pairs) {
+    int best = bnn::f4::BN_MAX;
+    int64_t best_cost = INT64_MAX;
+    for (int bn = bnn::f4::BN_MAX; bn >= 128; bn -= 32) {
+        const int64_t tiles = tiles_m * ceil_div(N, (int64_t)(bn / per_col));
+        const int64_t cost = ceil_div(tiles, pairs) * (bnn::f4::BM + bn / 2);
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = bn;
+        }
+    }
+    return best;
+}
+
+// One launch of the CTA-pair e2m1 kernel: clusters of two, as many as are
+// resident at once (the tiles are walked persistently).
+template <int MODE>
+bnn_status launch_f4_pairs(const CUtensorMap& tmA, const CUtensorMap& tmW, const CUtensorMap& tmCi,
+                           const CUtensorMap& tmCf, int64_t M, int64_t N, int64_t K, int64_t kw, int bn, int64_t tiles_m,
+                           int64_t tiles_n, int tma_out, const bnn::GemmEpilogue& e, const bnn::TcPlanes& pl,
+                           int pairs, cudaStream_t stream) {
+    using C = bnn::f4::Cfg<true, MODE>;
+    const int64_t clusters = std::min<int64_t>(tiles_m * tiles_n, pairs);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)(2 * clusters));
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, bnn::xnor_gemm_f4_kernel<true, MODE>, tmA, tmW, tmCi, tmCf, (int)M, (int)N, (int)K,
+                           (int)kw, bn, (int)tiles_m, (int)tiles_n, tma_out, e, pl) != cudaSuccess)
+        return BNN_ERR_CUDA;
+    return launch_status();
+}
+
 // The +1/-1 product on the tensor cores with e2m1 operands.  Callers check
 // K against MAX_KP (the exact-integer range of the fp32 accumulator).
 bnn_status launch_gemm_f4(const uint32_t* A, int64_t lda, const uint32_t* W, int64_t ldw, int64_t M, int64_t N,
@@ -312,27 +361,12 @@ bnn_status launch_gemm_f4(const uint32_t* A, int64_t lda, const uint32_t* W, int
     if (!plan.pair) {
         const int64_t grid = std::min<int64_t>(tiles_m * tiles_n, sms);
         bnn::xnor_gemm_f4_kernel<false><<<(unsigned)grid, Cfg<false>::THREADS, Cfg<false>::SMEM_BYTES, stream>>>(
-            tmA, tmW, tmCi, tmCf, (int)M, (int)N, (int)K, (int)kw, bn, (int)tiles_m, (int)tiles_n, tma_out, e);
+            tmA, tmW, tmCi, tmCf, (int)M, (int)N, (int)K, (int)kw, bn, (int)tiles_m, (int)tiles_n, tma_out, e,
+            bnn::TcPlanes{});
         return launch_status();
     }
-    // CTA pairs: clusters of two, as many as are resident at once.
-    const int64_t clusters = std::min<int64_t>(tiles_m * tiles_n, pairs);
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3((unsigned)(2 * clusters));
-    cfg.blockDim = dim3(Cfg<true>::THREADS);
-    cfg.dynamicSmemBytes = Cfg<true>::SMEM_BYTES;
-    cfg.stream = stream;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, bnn::xnor_gemm_f4_kernel<true>, tmA, tmW, tmCi, tmCf, (int)M, (int)N, (int)K,
-                           (int)kw, bn, (int)tiles_m, (int)tiles_n, tma_out, e) != cudaSuccess)
-        return BNN_ERR_CUDA;
-    return launch_status();
+    return launch_f4_pairs<bnn::TC_BINARY>(tmA, tmW, tmCi, tmCf, M, N, K, kw, bn, tiles_m, tiles_n, tma_out, e,
+                                           bnn::TcPlanes{}, pairs, stream);
 }
 
 // Padded K of the 4-bit kernel (whole 256-element stages).
@@ -345,15 +379,16 @@ inline int64_t f4_padded_k(int64_t K) {
 // box_planes, box_rows), no swizzle.  box_planes > planes reads the missing
 // planes as zero words.
 bool encode_plane_map(CUtensorMap* map, const uint32_t* base, int64_t kw, int64_t planes, int64_t rows, int64_t ld,
-                      int box_planes, int box_rows) {
+                      int box_planes, int box_rows, int box_words = bnn::tc::BKW,
+                      CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE) {
     auto enc = tensor_map_encoder();
     if (enc == nullptr) return false;
     cuuint64_t dims[3] = {(cuuint64_t)kw, (cuuint64_t)planes, (cuuint64_t)rows};
     cuuint64_t strides[2] = {(cuuint64_t)ld * 4u, (cuuint64_t)(planes * ld) * 4u};
-    cuuint32_t box[3] = {(cuuint32_t)bnn::tc::BKW, (cuuint32_t)box_planes, (cuuint32_t)box_rows};
+    cuuint32_t box[3] = {(cuuint32_t)box_words, (cuuint32_t)box_planes, (cuuint32_t)box_rows};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t*>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -864,6 +899,40 @@ bnn_status bnn_bitserial_gemm(const uint32_t* A, int64_t lda, int a_bits, const 
     if ((C_i32 && !aligned(C_i32, 4)) || (C_f32 && !aligned(C_f32, 4)) || (alpha && !aligned(alpha, 4)))
         return BNN_ERR_ALIGNMENT;
     if (M == 0 || N == 0) return BNN_OK;
+    {
+        // Codes of up to two bits are exact e2m1 values: the e2m1 kernel in
+        // CTA pairs, while every partial sum (at most 9 per element of the
+        // padded K) stays an integer the epilogue converts exactly.
+        const int engine = g_gemm_engine.load(std::memory_order_relaxed);
+        const int pairs = engine == BNN_GEMM_ENGINE_TENSOR_I8 ? -1 : gemm_f4_pairs_resident();
+        if (a_bits <= bnn::f4::MAX_F4_PLANES && w_bits <= bnn::f4::MAX_F4_PLANES && pairs > 0 && pairs < kNoPairs &&
+            M > bnn::f4::BM && 9 * f4_padded_k(K) < (int64_t(1) << 22)) {
+            const int bn = f4_pair_tile_n(ceil_div(M, (int64_t)2 * bnn::f4::BM), N, 1, pairs);
+            CUtensorMap fA, fW, fCi, fCf;
+            std::memset(&fCi, 0, sizeof(fCi));
+            std::memset(&fCf, 0, sizeof(fCf));
+            if (!encode_plane_map(&fA, A, kw, a_bits, M, lda, a_bits, bnn::f4::BM, bnn::f4::BKW,
+                                  CU_TENSOR_MAP_SWIZZLE_32B) ||
+                !encode_plane_map(&fW, W, kw, w_bits, N, ldw, w_bits, bn / 2, bnn::f4::BKW, CU_TENSOR_MAP_SWIZZLE_32B))
+                return BNN_ERR_CUDA;
+            bnn::GemmEpilogue e{};
+            e.c_i32 = C_i32;
+            e.ldc = ldc;
+            e.c_f32 = C_f32;
+            e.ldf = ldf;
+            e.alpha = alpha;
+            e.bits_words = packed_ld_words(N);
+            int tma_out = 0;
+            if (encode_output_map(&fCi, C_i32, CU_TENSOR_MAP_DATA_TYPE_INT32, N, M, ldc)) tma_out |= 1;
+            if (encode_output_map(&fCf, C_f32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, N, M, ldf)) tma_out |= 2;
+            bnn::TcPlanes pl{};
+            pl.ja = a_bits;
+            pl.jw = w_bits;
+            return launch_f4_pairs<bnn::TC_PLANE_CODES>(fA, fW, fCi, fCf, M, N, K, kw, bn,
+                                                        ceil_div(M, (int64_t)2 * bnn::f4::BM), ceil_div(N, bn),
+                                                        tma_out, e, pl, pairs, as_cuda(stream));
+        }
+    }
     CUtensorMap tmA, tmW;
     if (!encode_plane_map(&tmA, A, kw, a_bits, M, lda, a_bits, BM) ||
         !encode_plane_map(&tmW, W, kw, w_bits, N, ldw, w_bits, BN))
@@ -909,6 +978,35 @@ bnn_status bnn_binary_bases_gemm(const uint32_t* H, int64_t ldh, int J, const ui
     if (!aligned(beta, 4) || !aligned(alpha, 4) || !aligned(Y, 4)) return BNN_ERR_ALIGNMENT;
     if (M == 0 || N == 0) return BNN_OK;
     const int jp = pow2_at_least(J), ip = pow2_at_least(I);
+    {
+        // +1/-1 bases on the e2m1 kernel in CTA pairs: each CTA holds
+        // 128 / jp output rows (x jp bases) and half of the tile's bn / ip
+        // output columns (x ip bases).
+        const int engine = g_gemm_engine.load(std::memory_order_relaxed);
+        const int pairs = engine == BNN_GEMM_ENGINE_TENSOR_I8 ? -1 : gemm_f4_pairs_resident();
+        const int rows_cta = bnn::f4::BM / jp;
+        if (pairs > 0 && pairs < kNoPairs && M > rows_cta && f4_padded_k(K) <= bnn::f4::MAX_KP) {
+            const int64_t tiles_m = ceil_div(M, (int64_t)2 * rows_cta);
+            const int bn = f4_pair_tile_n(tiles_m, N, ip, pairs);
+            CUtensorMap fA, fW, fC;
+            std::memset(&fC, 0, sizeof(fC));
+            if (!encode_plane_map(&fA, H, kw, J, M, ldh, jp, rows_cta, bnn::f4::BKW, CU_TENSOR_MAP_SWIZZLE_32B) ||
+                !encode_plane_map(&fW, B, kw, I, N, ldb, ip, bn / 2 / ip, bnn::f4::BKW, CU_TENSOR_MAP_SWIZZLE_32B))
+                return BNN_ERR_CUDA;
+            bnn::TcPlanes pl{};
+            pl.ja = jp;
+            pl.jw = ip;
+            pl.j_real = J;
+            pl.i_real = I;
+            pl.beta = beta;
+            pl.alpha = alpha;
+            pl.lda_alpha = lda_alpha;
+            pl.y = Y;
+            pl.ldy = ldy;
+            return launch_f4_pairs<bnn::TC_BASES>(fA, fW, fC, fC, M, N, K, kw, bn, tiles_m, ceil_div(N, bn / ip), 0,
+                                                  bnn::GemmEpilogue{}, pl, pairs, as_cuda(stream));
+        }
+    }
     const int rows_per_tile = BM / jp, cols_per_tile = BN / ip;
     CUtensorMap tmA, tmW;
     if (!encode_plane_map(&tmA, H, kw, J, M, ldh, jp, rows_per_tile) ||

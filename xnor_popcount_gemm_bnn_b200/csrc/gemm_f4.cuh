@@ -69,6 +69,9 @@ static_assert(ACC_STRIDE + BN_MAX <= SF_COL, "accumulators overlap the scale fac
 static_assert(U_A_BYTES % 1024 == 0 && OUT_BLOCK % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 // Named barrier of the epilogue warps (id 0 is __syncthreads).
 constexpr int EPI_BAR = 1;
+// Bits per code in the plane-code mode: codes 0..3 are exact e2m1 values
+// (0x0, 0x2 = 1.0, 0x4 = 2.0, 0x5 = 3.0).
+constexpr int MAX_F4_PLANES = 2;
 // Largest padded K: partial sums stay integers of magnitude <= 2^20, exact
 // in fp32 and in the epilogue's float-to-int conversion (valid below 2^22).
 constexpr int64_t MAX_KP = int64_t(1) << 20;
@@ -79,14 +82,15 @@ constexpr int64_t MAX_KP = int64_t(1) << 20;
 // shared memory and its 128 x bn accumulator in its tensor memory, and the
 // even CTA issues the MMAs for both.  Per multiply-add the pair moves
 // (128 + bn / 2) instead of (128 + bn) rows through each SM's shared memory.
-template <bool PAIR>
+template <bool PAIR, int MODE = 0>
 struct Cfg {
     static constexpr int CTAS = PAIR ? 2 : 1;
     static constexpr int BN_CTA_MAX = BN_MAX / CTAS;            // W rows per CTA
     static constexpr int USTAGES = PAIR ? 4 : 3;                // unpacked ring
     static constexpr int U_B_BYTES = BN_CTA_MAX * ROW_BYTES;
     static constexpr int U_STAGE = U_A_BYTES + U_B_BYTES;
-    static constexpr int P_STAGE = (BM + BN_CTA_MAX) * P_ROW;
+    // Plane-code mode: every code row brings up to MAX_F4_PLANES packed planes.
+    static constexpr int P_STAGE = (BM + BN_CTA_MAX) * P_ROW * (MODE == 1 ? MAX_F4_PLANES : 1);
     static constexpr int UNPACK_WARPS = (BM + BN_CTA_MAX + 31) / 32;   // 11 single, 8 pair
     static constexpr int WARP_EPI0 = WARP_UNPACK0 + UNPACK_WARPS;
     static constexpr int THREADS = (WARP_EPI0 + EPI_WARPS) * 32;       // 544 single, 448 pair
@@ -228,19 +232,41 @@ __device__ __forceinline__ uint4 expand_word_e2m1(uint32_t w) {
     return make_uint4(((w << 3) & sign) | one, ((w << 2) & sign) | one, ((w << 1) & sign) | one, (w & sign) | one);
 }
 
+// Bit planes of unsigned codes (one or two planes: codes 0..3) -> e2m1
+// code values, 16 bytes per 32 codes, in expand_word_e2m1's element order
+// (word j, nibble i = element 4i + j).  With t0, t1 the two planes' bits at
+// bit 3 of each nibble: code 1 -> 0x2 (1.0), 2 -> 0x4 (2.0), 3 -> 0x5 (3.0),
+// 0 -> 0x0.
+__device__ __forceinline__ uint4 fold_planes_e2m1(uint32_t p0, uint32_t p1) {
+    constexpr uint32_t top = 0x88888888u;
+    uint32_t o[4];
+    #pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t t0 = (p0 << (3 - j)) & top, t1 = (p1 << (3 - j)) & top;
+        o[j] = (t1 >> 1) | ((t0 & ~t1) >> 2) | ((t0 & t1) >> 3);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // fp32 accumulator holding an integer of magnitude < 2^22 -> that integer
 // (adding 1.5 * 2^23 puts it in the low mantissa bits).
 __device__ __forceinline__ int32_t acc_to_int(uint32_t bits) {
     return __float_as_int(__uint_as_float(bits) + 12582912.0f) - 0x4B400000;
 }
 
-template <bool PAIR>
-__global__ void __launch_bounds__(f4::Cfg<PAIR>::THREADS, 1)
+// MODE (TcMode of gemm_tc.cuh): TC_BINARY the +1/-1 product; TC_PLANE_CODES
+// unsigned codes of one or two bit planes (3-D TMA boxes bring a code row's
+// planes together, the unpack folds them into e2m1 code values, pads are
+// code 0); TC_BASES +1/-1 binary bases, plane-interleaved so that
+// accumulator lane L holds base L mod ja of output row L / ja and column c
+// base c mod jw of output column c / jw, combined by the epilogue.
+template <bool PAIR, int MODE = TC_BINARY>
+__global__ void __launch_bounds__(f4::Cfg<PAIR, MODE>::THREADS, 1)
 xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW,
                     const __grid_constant__ CUtensorMap tmCi, const __grid_constant__ CUtensorMap tmCf, int M, int N,
-                    int K, int kw, int bn, int tiles_m, int tiles_n, int tma_out, GemmEpilogue ep) {
+                    int K, int kw, int bn, int tiles_m, int tiles_n, int tma_out, GemmEpilogue ep, TcPlanes pl) {
     using namespace f4;
-    using C = Cfg<PAIR>;
+    using C = Cfg<PAIR, MODE>;
     constexpr int CTAS = C::CTAS, USTAGES = C::USTAGES, PSTAGES = C::PSTAGES, U_STAGE = C::U_STAGE,
                   P_STAGE = C::P_STAGE, UNPACK_WARPS = C::UNPACK_WARPS, WARP_EPI0 = C::WARP_EPI0;
     extern __shared__ uint8_t smem_raw[];
@@ -270,7 +296,14 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
     const int cid = (int)blockIdx.x / CTAS, ncl = (int)gridDim.x / CTAS;
     const int bn_cta = bn / CTAS;
-    const uint32_t stage_tx = (uint32_t)(BM + bn_cta) * P_ROW;
+    // Planes per packed A / W row group (plane codes), output rows / columns
+    // per CTA and per tile (bases spend ja lanes on a row, jw columns on a column).
+    const int ja = MODE == TC_BINARY ? 1 : pl.ja, jw = MODE == TC_BINARY ? 1 : pl.jw;
+    const int rows_cta = MODE == TC_BASES ? BM / ja : BM;
+    const int cols_tile = MODE == TC_BASES ? bn / jw : bn;
+    const int pa_bytes = MODE == TC_PLANE_CODES ? BM * ja * P_ROW : P_A_BYTES;
+    const uint32_t stage_tx =
+        MODE == TC_PLANE_CODES ? (uint32_t)(BM * ja + bn_cta * jw) * P_ROW : (uint32_t)(BM + bn_cta) * P_ROW;
 
     if (threadIdx.x == 0) {
         prefetch_tensormap(&tmA);
@@ -312,9 +345,12 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         if (lane == 0) {
             uint32_t g = 0, issued = 0;
             bool ok = true;
+            // TMA coordinates in rows of the operand tensors (code or output
+            // rows; the 3-D boxes bring each row's planes along).
+            const int rows_w = MODE == TC_BASES ? bn_cta / jw : bn_cta;
             for (int t = cid; ok && t < tiles; t += ncl) {
-                const int m0 = (t / tiles_n) * (BM * CTAS) + BM * (int)rank;
-                const int n0 = (t % tiles_n) * bn + bn_cta * (int)rank;
+                const int m0 = (t / tiles_n) * (rows_cta * CTAS) + rows_cta * (int)rank;
+                const int n0 = (t % tiles_n) * cols_tile + rows_w * (int)rank;
                 for (int ks = 0; ks < nk; ++ks, ++g) {
                     const uint32_t s = g % (uint32_t)PSTAGES;
                     if (g >= (uint32_t)PSTAGES && !tc_wait(&pempty[s], ((g / PSTAGES) - 1) & 1, abort_flag)) {
@@ -323,8 +359,13 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     }
                     uint8_t* dst = pring + s * P_STAGE;
                     mbar_arrive_expect_tx(&pfull[s], stage_tx);
-                    tma_load_2d(dst, &tmA, ks * BKW, m0, &pfull[s]);
-                    tma_load_2d(dst + P_A_BYTES, &tmW, ks * BKW, n0, &pfull[s]);
+                    if constexpr (MODE == TC_BINARY) {
+                        tma_load_2d(dst, &tmA, ks * BKW, m0, &pfull[s]);
+                        tma_load_2d(dst + P_A_BYTES, &tmW, ks * BKW, n0, &pfull[s]);
+                    } else {
+                        tma_load_3d(dst, &tmA, ks * BKW, 0, m0, &pfull[s]);
+                        tma_load_3d(dst + pa_bytes, &tmW, ks * BKW, 0, n0, &pfull[s]);
+                    }
                     ++issued;
                 }
             }
@@ -391,13 +432,24 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const int my_tiles = cid < tiles ? (tiles - 1 - cid) / ncl + 1 : 0;
         const uint32_t total = (uint32_t)my_tiles * (uint32_t)nk;
         uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;              // words 0..3 and 4..7 of the row
+        uint4 lo1 = lo, hi1 = lo;                                     // plane codes: the second plane
+        // Plane codes: the row's planes are consecutive 32-byte slots, from
+        // slot s0 on (each slot's halves swizzled by its own index).
+        const int nplanes = MODE == TC_PLANE_CODES ? (is_a ? ja : jw) : 1;
+        const int s0 = MODE == TC_PLANE_CODES ? (is_a ? r * ja : BM * ja + r * jw) : u;
         auto load_packed = [&](uint32_t gg) -> bool {
             const uint32_t ps = gg % (uint32_t)PSTAGES;
             if (!__all_sync(0xffffffffu, tc_wait(&pfull[ps], (gg / PSTAGES) & 1, abort_flag))) return false;
             if (active) {
-                const uint8_t* src = pring + ps * P_STAGE + u * P_ROW;
-                lo = *reinterpret_cast<const uint4*>(src + hsw);
-                hi = *reinterpret_cast<const uint4*>(src + (hsw ^ 16));
+                const uint8_t* src = pring + ps * P_STAGE + s0 * P_ROW;
+                const int h0 = MODE == TC_PLANE_CODES ? 16 * ((s0 >> 2) & 1) : hsw;
+                lo = *reinterpret_cast<const uint4*>(src + h0);
+                hi = *reinterpret_cast<const uint4*>(src + (h0 ^ 16));
+                if (MODE == TC_PLANE_CODES && nplanes > 1) {
+                    const int h1 = 16 * (((s0 + 1) >> 2) & 1);
+                    lo1 = *reinterpret_cast<const uint4*>(src + P_ROW + h1);
+                    hi1 = *reinterpret_cast<const uint4*>(src + P_ROW + (h1 ^ 16));
+                }
             }
             return true;
         };
@@ -410,14 +462,25 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 // Chunk q of the row at (q ^ (r & 7)) * 16: the eight lanes of a
                 // store phase (eight consecutive rows) hit distinct banks.
                 uint8_t* row = uring + us * U_STAGE + (is_a ? 0 : U_A_BYTES) + r * ROW_BYTES;
-                *reinterpret_cast<uint4*>(row + ((0 ^ sw) << 4)) = expand_word_e2m1(lo.x);
-                *reinterpret_cast<uint4*>(row + ((1 ^ sw) << 4)) = expand_word_e2m1(lo.y);
-                *reinterpret_cast<uint4*>(row + ((2 ^ sw) << 4)) = expand_word_e2m1(lo.z);
-                *reinterpret_cast<uint4*>(row + ((3 ^ sw) << 4)) = expand_word_e2m1(lo.w);
-                *reinterpret_cast<uint4*>(row + ((4 ^ sw) << 4)) = expand_word_e2m1(hi.x);
-                *reinterpret_cast<uint4*>(row + ((5 ^ sw) << 4)) = expand_word_e2m1(hi.y);
-                *reinterpret_cast<uint4*>(row + ((6 ^ sw) << 4)) = expand_word_e2m1(hi.z);
-                *reinterpret_cast<uint4*>(row + ((7 ^ sw) << 4)) = expand_word_e2m1(hi.w);
+                if constexpr (MODE == TC_PLANE_CODES) {
+                    *reinterpret_cast<uint4*>(row + ((0 ^ sw) << 4)) = fold_planes_e2m1(lo.x, lo1.x);
+                    *reinterpret_cast<uint4*>(row + ((1 ^ sw) << 4)) = fold_planes_e2m1(lo.y, lo1.y);
+                    *reinterpret_cast<uint4*>(row + ((2 ^ sw) << 4)) = fold_planes_e2m1(lo.z, lo1.z);
+                    *reinterpret_cast<uint4*>(row + ((3 ^ sw) << 4)) = fold_planes_e2m1(lo.w, lo1.w);
+                    *reinterpret_cast<uint4*>(row + ((4 ^ sw) << 4)) = fold_planes_e2m1(hi.x, hi1.x);
+                    *reinterpret_cast<uint4*>(row + ((5 ^ sw) << 4)) = fold_planes_e2m1(hi.y, hi1.y);
+                    *reinterpret_cast<uint4*>(row + ((6 ^ sw) << 4)) = fold_planes_e2m1(hi.z, hi1.z);
+                    *reinterpret_cast<uint4*>(row + ((7 ^ sw) << 4)) = fold_planes_e2m1(hi.w, hi1.w);
+                } else {
+                    *reinterpret_cast<uint4*>(row + ((0 ^ sw) << 4)) = expand_word_e2m1(lo.x);
+                    *reinterpret_cast<uint4*>(row + ((1 ^ sw) << 4)) = expand_word_e2m1(lo.y);
+                    *reinterpret_cast<uint4*>(row + ((2 ^ sw) << 4)) = expand_word_e2m1(lo.z);
+                    *reinterpret_cast<uint4*>(row + ((3 ^ sw) << 4)) = expand_word_e2m1(lo.w);
+                    *reinterpret_cast<uint4*>(row + ((4 ^ sw) << 4)) = expand_word_e2m1(hi.x);
+                    *reinterpret_cast<uint4*>(row + ((5 ^ sw) << 4)) = expand_word_e2m1(hi.y);
+                    *reinterpret_cast<uint4*>(row + ((6 ^ sw) << 4)) = expand_word_e2m1(hi.z);
+                    *reinterpret_cast<uint4*>(row + ((7 ^ sw) << 4)) = expand_word_e2m1(hi.w);
+                }
             }
             if (g + 1 < total) ok = load_packed(g + 1);
             // One proxy fence orders this thread's reads of the packed stage
@@ -432,7 +495,7 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 else mbar_arrive_remote(&ufull[us], 0);
             }
         }
-    } else {
+    } else if constexpr (MODE != TC_BASES) {
         // ------------------------------ epilogue warps ------------------------------
         // Per tile the four warps stage the tile's column parameters in the
         // shared copy of this tile's parity (alpha/gamma/beta and the
@@ -455,7 +518,8 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const bool tma_i = (tma_out & 1) != 0 && ep.c_i32 != nullptr;
         const bool tma_f = (tma_out & 2) != 0 && ep.c_f32 != nullptr;
         const int kp = nk * BKE;                                      // padded K: acc = kp - 2 * popcount
-        const int pad = kp - K;
+        // +1/-1: each pad position adds (+1)(+1); plane codes: pads are code 0.
+        const int pad = MODE == TC_PLANE_CODES ? 0 : kp - K;
         const float padf = (float)pad;
         const bool affine = ep.gamma != nullptr;
         const int chunks = bn / 32;
@@ -614,6 +678,70 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         // be complete) before the CTA exits.
         if (lane == 0) bulk_wait_all();
         __syncwarp();
+    } else {
+        // ------------------------- epilogue warps, bases mode -------------------------
+        // Accumulator lane L holds base j = L mod ja of output row L / ja of
+        // this CTA; column c holds base i = c mod jw of output column c / jw.
+        // Each thread forms v = sum_i alpha_i[n] * s_ji for its base j, scales
+        // it by beta_j, and a butterfly over the ja lanes of the row adds the
+        // bases (every lane of the group ends with the total; lane o mod ja of
+        // the group stores output column o).  Padded bases have beta_j = 0 or
+        // alpha_i[n] = 0 and add exactly 0.  The per-tile alpha of every
+        // accumulator column sits in the shared double-buffered copy, behind
+        // the same named barrier as the other modes.
+        const int quad = warp & 3;
+        const int ew = warp - WARP_EPI0;
+        const int kp = nk * BKE;
+        const int pad = kp - K;
+        const int L = 32 * quad + lane;
+        const int jl = L & (ja - 1);
+        const float bj = jl < pl.j_real ? __ldg(pl.beta + jl) : 0.0f;
+        const int outs_per_chunk = 32 / jw;
+        const int chunks = bn / 32;
+        bool ok = true;
+        int lt = 0;
+        for (int t = cid; t < tiles; t += ncl, ++lt) {
+            const int b = lt & 1;
+            const int m0 = (t / tiles_n) * (rows_cta * CTAS) + rows_cta * (int)rank, n0 = (t % tiles_n) * cols_tile;
+            float* ca = reinterpret_cast<float*>(colf + b * BN_MAX);   // alpha of each accumulator column
+            for (int i = 32 * ew + lane; i < bn; i += 32 * EPI_WARPS) {
+                const int n = n0 + i / jw, ib = i & (jw - 1);
+                ca[i] = (n < N && ib < pl.i_real) ? __ldg(pl.alpha + (int64_t)ib * pl.lda_alpha + n) : 0.0f;
+            }
+            named_bar_sync(EPI_BAR, EPI_WARPS * 32);
+            ok = ok && __all_sync(0xffffffffu, tc_wait(&afull[b], (lt >> 1) & 1, abort_flag));
+            if (!ok) continue;
+            tc_fence_after();
+            const int m = m0 + L / ja;
+            #pragma unroll 1
+            for (int c = 0; c < chunks; ++c) {
+                uint32_t r[32];
+                tmem_ld32_sync(tmem_base + ((uint32_t)(32 * quad) << 16) + (uint32_t)(b * ACC_STRIDE + 32 * c), r);
+                if (c == chunks - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (rank == 0) mbar_arrive(&aempty[b]);
+                        else mbar_arrive_remote(&aempty[b], 0);
+                    }
+                }
+                const int nb = n0 + c * outs_per_chunk;
+                if (nb >= N) continue;                                // uniform across the warp
+                float v = 0.0f;
+                #pragma unroll
+                for (int col = 0; col < 32; ++col) {
+                    v = fmaf(ca[32 * c + col], (float)(acc_to_int(r[col]) - pad), v);
+                    if (((col + 1) & (jw - 1)) == 0) {
+                        float tsum = bj * v;
+                        for (int off = 1; off < ja; off <<= 1) tsum += __shfl_xor_sync(0xffffffffu, tsum, off);
+                        const int o = col / jw;
+                        const int n = nb + o;
+                        if ((o & (ja - 1)) == jl && m < M && n < N) pl.y[(int64_t)m * pl.ldy + n] = tsum;
+                        v = 0.0f;
+                    }
+                }
+            }
+        }
     }
 
     // ------------------------------ teardown ------------------------------
