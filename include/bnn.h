@@ -317,6 +317,31 @@ bnn_status bnn_xnor_gemv_ex(const uint32_t* W, int64_t ldw, const void* x, bnn_d
                             int64_t N, int64_t K, const float* alpha,
                             int32_t* y_i32, float* y_f32, uint32_t flags, bnn_stream_t stream);
 
+/* bnn_xnor_gemv_host -- bnn_xnor_gemv_ex for a caller whose x and y live in
+ * host memory: on `stream`, copies x (K elements) from host to device, runs
+ * the GEMV, and copies y (N fp32 values) back, one cudaMemcpyAsync each way.
+ *   Passage: as bnn_xnor_gemv ("First Principles ...", "Bandwidth math";
+ *   eq. (4), (6) and (1) of "Extreme Quantization ...").
+ *   W, ldw, alpha  device, as in bnn_xnor_gemv (W and alpha are the model's
+ *                  resident weights).
+ *   x_host   host memory, K elements of x_dt; pinned (page-locked) memory
+ *            makes the copy asynchronous, pageable memory is copied too but
+ *            the call may then block the host until the copy is done.
+ *   x_dev    device scratch for x, >= K elements of x_dt, 16-byte aligned,
+ *            owned by the caller (the library allocates nothing).
+ *   y_dev    device scratch for y, >= N fp32, 4-byte aligned.
+ *   y_host   host memory for the N fp32 outputs alpha[n] * s (pinned for an
+ *            asynchronous copy); valid once `stream` reaches the end of the
+ *            call's work (e.g. after cudaStreamSynchronize).
+ *   flags    BNN_GEMV_WEIGHTS_STATIC or 0 (x is written by the copy just
+ *            before the kernel, and y is read by the copy after it, so the
+ *            other flags do not apply).
+ *   Errors: INVALID_ARG (null pointer, bad size or flag), ALIGNMENT, and the
+ *   errors of bnn_xnor_gemv; BNN_ERR_CUDA when a copy cannot be enqueued. */
+bnn_status bnn_xnor_gemv_host(const uint32_t* W, int64_t ldw, const void* x_host, bnn_dtype x_dt, int64_t N,
+                              int64_t K, const float* alpha, void* x_dev, float* y_dev, float* y_host, uint32_t flags,
+                              bnn_stream_t stream);
+
 /* bnn_binary_weight_gemv -- binary weights times a REAL activation vector:
  *   y[n] = alpha[n] * sum_k sign(W[n,k]) * x[k]
  * ("Extreme Quantization: Binary, Ternary & 1-bit LLMs", Binary Neural

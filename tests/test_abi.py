@@ -158,6 +158,20 @@ def test_gemm_engine_setting_on_host():
     bnn.bnn_set_gemm_engine(prev)
 
 
+def test_gemv_host_entry_rejects_bad_arguments():
+    f = L.bnn_xnor_gemv_host
+    # W, ldw, x_host, dt, N, K, alpha, x_dev, y_dev, y_host, flags, stream
+    assert f(FAKE, 128, FAKE, 1, 8, 4096, FAKE, FAKE, FAKE, FAKE, 2, NULL) == bnn.BNN_ERR_INVALID_ARG    # inputs static
+    assert f(FAKE, 128, FAKE, 1, 8, 4096, FAKE, FAKE, FAKE, FAKE, 4, NULL) == bnn.BNN_ERR_INVALID_ARG    # output free
+    assert f(FAKE, 128, NULL, 1, 8, 4096, FAKE, FAKE, FAKE, FAKE, 0, NULL) == bnn.BNN_ERR_INVALID_ARG    # no x_host
+    assert f(FAKE, 128, FAKE, 1, 8, 4096, FAKE, NULL, FAKE, FAKE, 0, NULL) == bnn.BNN_ERR_INVALID_ARG    # no x_dev
+    assert f(FAKE, 128, FAKE, 1, 8, 4096, FAKE, FAKE, FAKE, NULL, 0, NULL) == bnn.BNN_ERR_INVALID_ARG    # no y_host
+    assert f(FAKE, 128, FAKE, 1, 8, 4096, NULL, FAKE, FAKE, FAKE, 0, NULL) == bnn.BNN_ERR_INVALID_ARG    # no alpha
+    assert f(FAKE, 128, FAKE, 7, 8, 4096, FAKE, FAKE, FAKE, FAKE, 0, NULL) == bnn.BNN_ERR_INVALID_ARG    # dtype
+    assert f(FAKE, 128, FAKE, 1, 8, 0, FAKE, FAKE, FAKE, FAKE, 0, NULL) == bnn.BNN_ERR_INVALID_ARG       # K < 1
+    assert f(FAKE, 128, FAKE, 1, 8, 4096, FAKE, FAKE_ODD, FAKE, FAKE, 0, NULL) == bnn.BNN_ERR_ALIGNMENT  # x_dev
+
+
 def test_binary_weight_gemv_rejects_bad_arguments():
     f = L.bnn_binary_weight_gemv
     assert f(FAKE, 4, FAKE, 0, 8, 32, FAKE, FAKE, 8, NULL) == bnn.BNN_ERR_INVALID_ARG       # unknown flag

@@ -275,3 +275,30 @@ def test_independent_gemvs_all_flags(use_graph):
         assert np.array_equal(stacked[l].cpu().numpy(), ref), f"stacked {l}"
         assert_scaled_close(yf[l], oracle.scaled(ref, oracle.alpha(Ws[l])))
     assert_no_device_error()
+
+
+@pytest.mark.parametrize("pinned", [True, False], ids=["pinned", "pageable"])
+def test_host_buffer_entry_matches_device_gemv(pinned):
+    """bnn_xnor_gemv_host (x and y in host memory, copies inside the call)
+    gives the same y as bnn_xnor_gemv on device buffers, bit for bit, on two
+    calls in a row with different x."""
+    N, K = 3000, 4096
+    d = dev()
+    W = workloads.normal((N, K), 0.02, 91)
+    W_p = bnn.empty_packed(N, K, d)
+    alpha = torch.empty(N, dtype=torch.float32, device=d)
+    bnn.bnn_pack_sign(W.to(d), W_p, alpha)
+    x_dev = torch.empty(K, dtype=torch.bfloat16, device=d)
+    y_dev = torch.empty(N, dtype=torch.float32, device=d)
+    for seed in (92, 93):
+        x = workloads.normal((K,), 1.0, seed, dtype=torch.bfloat16)
+        x_host = x.pin_memory() if pinned else x.clone()
+        y_host = torch.full((N,), float("nan"), dtype=torch.float32)
+        if pinned:
+            y_host = y_host.pin_memory()
+        bnn.bnn_xnor_gemv_host(W_p, x_host, K, alpha, x_dev, y_dev, y_host, flags=bnn.BNN_GEMV_WEIGHTS_STATIC)
+        torch.cuda.synchronize()
+        y_ref = torch.empty(N, dtype=torch.float32, device=d)
+        bnn.bnn_xnor_gemv(W_p, x.to(d), K, alpha, None, y_ref)
+        assert torch.equal(y_host, y_ref.cpu())
+    assert_no_device_error()

@@ -47,7 +47,7 @@ BNN_GEMM_ENGINE_TENSOR_I8 = 3
 EXPORTS = (
     "bnn_packed_ld_words", "bnn_conv3x3_ld_words", "bnn_status_string", "bnn_device_error",
     "bnn_pack_sign", "bnn_pack_sign_nchw", "bnn_pack_conv3x3_weights", "bnn_xnor_gemm",
-    "bnn_xnor_gemv", "bnn_xnor_gemv_ex", "bnn_binary_linear_fused", "bnn_binary_conv3x3_fused",
+    "bnn_xnor_gemv", "bnn_xnor_gemv_ex", "bnn_xnor_gemv_host", "bnn_binary_linear_fused", "bnn_binary_conv3x3_fused",
     "bnn_fold_bn_threshold", "bnn_set_gemm_engine", "bnn_get_gemm_engine", "bnn_selftest_wait_timeout",
     "bnn_binary_weight_gemv", "bnn_ternary_ld_words", "bnn_ternary_workspace_bytes", "bnn_ternary_pack",
     "bnn_ternary_gemv_i8", "bnn_ternary_pack_noalloc", "bnn_pack_sign_rsign", "bnn_pack_sign_nchw_rsign",
@@ -91,6 +91,7 @@ def _load() -> ctypes.CDLL:
         "bnn_xnor_gemm": (i32, [p, i64, p, i64, i64, i64, i64, p, p, i64, p, i64, p]),
         "bnn_xnor_gemv": (i32, [p, i64, p, i32, i64, i64, p, p, p, p]),
         "bnn_xnor_gemv_ex": (i32, [p, i64, p, i32, i64, i64, p, p, p, ctypes.c_uint32, p]),
+        "bnn_xnor_gemv_host": (i32, [p, i64, p, i32, i64, i64, p, p, p, p, ctypes.c_uint32, p]),
         "bnn_binary_weight_gemv": (i32, [p, i64, p, i32, i64, i64, p, p, ctypes.c_uint32, p]),
         "bnn_binary_linear_fused": (i32, [p, i64, p, i64, i64, i64, i64,
                                           ctypes.POINTER(bnn_epilogue), p, i64, p]),
@@ -313,6 +314,20 @@ def bnn_xnor_gemv_ex(W: torch.Tensor, x: torch.Tensor, K: Optional[int] = None,
     K = x.shape[-1] if K is None else int(K)
     _check("bnn_xnor_gemv_ex", _lib.bnn_xnor_gemv_ex(
         _ptr(W), _ld(W), _ptr(x), _dtype(x), N, K, _ptr(alpha), _ptr(y_i32), _ptr(y_f32),
+        int(flags), _stream(stream)))
+
+
+def bnn_xnor_gemv_host(W: torch.Tensor, x_host: torch.Tensor, K: Optional[int], alpha: torch.Tensor,
+                       x_dev: torch.Tensor, y_dev: torch.Tensor, y_host: torch.Tensor, flags: int = 0,
+                       N: Optional[int] = None, stream=None) -> None:
+    """The GEMV with x and y in host memory: copies x in, runs the GEMV, copies y (fp32) out, all on
+    `stream`; x_dev and y_dev are the caller's device scratch."""
+    assert not x_host.is_cuda and not y_host.is_cuda and x_dev.is_cuda and y_dev.is_cuda
+    N = W.shape[0] if N is None else N
+    K = x_host.shape[-1] if K is None else int(K)
+    assert x_dev.dtype == x_host.dtype and x_dev.numel() >= K and y_dev.numel() >= N and y_host.numel() >= N
+    _check("bnn_xnor_gemv_host", _lib.bnn_xnor_gemv_host(
+        _ptr(W), _ld(W), _ptr(x_host), _dtype(x_host), N, K, _ptr(alpha), _ptr(x_dev), _ptr(y_dev), _ptr(y_host),
         int(flags), _stream(stream)))
 
 

@@ -818,6 +818,25 @@ bnn_status bnn_xnor_gemv_ex(const uint32_t* W, int64_t ldw, const void* x, bnn_d
                      (flags & BNN_GEMV_INPUTS_STATIC) != 0, flags == kAll, stream);
 }
 
+bnn_status bnn_xnor_gemv_host(const uint32_t* W, int64_t ldw, const void* x_host, bnn_dtype x_dt, int64_t N,
+                              int64_t K, const float* alpha, void* x_dev, float* y_dev, float* y_host, uint32_t flags,
+                              bnn_stream_t stream) {
+    if (flags != 0 && flags != BNN_GEMV_WEIGHTS_STATIC) return BNN_ERR_INVALID_ARG;
+    if (x_host == nullptr || x_dev == nullptr || y_dev == nullptr || y_host == nullptr || alpha == nullptr)
+        return BNN_ERR_INVALID_ARG;
+    if (N < 0 || K < 1 || N > INT_MAX / 2 || K > INT_MAX / 2) return BNN_ERR_INVALID_ARG;
+    if (x_dt != BNN_F32 && x_dt != BNN_BF16) return BNN_ERR_INVALID_ARG;
+    if (!aligned(x_dev, 16) || !aligned(y_dev, 4)) return BNN_ERR_ALIGNMENT;
+    const size_t xbytes = (size_t)K * (x_dt == BNN_F32 ? 4 : 2), ybytes = (size_t)N * 4;
+    cudaStream_t s = as_cuda(stream);
+    if (cudaMemcpyAsync(x_dev, x_host, xbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return BNN_ERR_CUDA;
+    const bnn_status st = bnn_xnor_gemv_ex(W, ldw, x_dev, x_dt, N, K, alpha, nullptr, y_dev, flags, stream);
+    if (st != BNN_OK) return st;
+    if (N > 0 && cudaMemcpyAsync(y_host, y_dev, ybytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return BNN_ERR_CUDA;
+    return BNN_OK;
+}
+
 bnn_status bnn_binary_weight_gemv(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_dt, int64_t N,
                                   int64_t K, const float* alpha, float* y, uint32_t flags, bnn_stream_t stream) {
     constexpr uint32_t kAll = BNN_GEMV_WEIGHTS_STATIC | BNN_GEMV_INPUTS_STATIC | BNN_GEMV_OUTPUT_FREE;
