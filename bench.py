@@ -147,7 +147,8 @@ KERNEL_SOURCES = {
     "xnor_gemm_f4_kernel": ("gemm_f4.cuh", "gemm_tc.cuh", "gemm_popc.cuh", "common.cuh"),
     "xnor_gemm_popc_kernel": ("gemm_popc.cuh", "common.cuh"),
     "xnor_conv3x3_kernel": ("conv.cuh", "common.cuh"),
-    "xnor_conv3x3_tcw_kernel": ("conv_tc.cuh", "conv.cuh", "gemm_tc.cuh", "gemm_popc.cuh", "common.cuh"),
+    "xnor_conv3x3_tcw_kernel": ("conv_tc.cuh", "conv.cuh", "gemm_f4.cuh", "gemm_tc.cuh", "gemm_popc.cuh",
+                                "common.cuh"),
     "pack_sign_rows_kernel": ("pack.cuh", "common.cuh"),
     "pack_sign_nchw_kernel": ("pack.cuh", "common.cuh"),
     "pack_sign_nchw_tma_kernel": ("pack.cuh", "common.cuh"),
