@@ -551,7 +551,7 @@ xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* _
                     arrived = true;
                 }
                 if (!valid) continue;
-                if constexpr (F4) {
+                if (F4 && ep.mode == BNN_OUT_INT32) {
                     // fp32 accumulators holding integers (|acc| < 2^22): read
                     // them as the int32 values the int8 path produces.
                     #pragma unroll
@@ -576,7 +576,12 @@ xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* _
                         #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             const int co = c0 + j4 + q;
-                            float y = av[q] * (float)((int32_t)rr[j4 + q] - padc);
+                            // s = acc - pad exactly: an int32 subtraction, or for the
+                            // e2m1 accumulators one fp32 subtraction of two integers
+                            // below 2^22 (the same float as (float)s).
+                            const float sf = F4 ? __uint_as_float(rr[j4 + q]) - (float)padc
+                                                : (float)((int32_t)rr[j4 + q] - padc);
+                            float y = av[q] * sf;
                             if (affine) y = fmaf(gv[q], y, bv[q]);
                             if (co < cout) o[(int64_t)co * ohow] = y;
                         }
