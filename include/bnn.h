@@ -227,16 +227,17 @@ bnn_status bnn_pack_conv3x3_weights(const void* w_oihw, bnn_dtype dt, int64_t co
  *             accumulators holding exact integers) while K rounded up to a
  *             multiple of 256 is at most 2^20, as int8 bytes (kind::i8,
  *             int32 accumulators) beyond that; for large products.
- *   TENSOR_I8: the int8 tensor-core kernel at every K (the convolutions
- *             take it as TENSOR).
+ *   TENSOR_I8: the int8 tensor-core kernels at every K (GEMM, 3x3
+ *             convolution and the multi-bit products below).
  *   AUTO:     TENSOR when M >= 128, N >= 128 and K >= 512, else POPCOUNT
  *             (the default).  Convolutions: the stride-1 tensor-core kernel
  *             when cout >= 64, c <= 64 and n*oh*ow >= 16384, else POPCOUNT.
  * Under TENSOR the convolution uses the tensor cores where its shared memory
  * fits: stride 1 with cout <= 256 (the filters stay resident next to two
- * input buffers of at least one 128-pixel window); other strides with
- * c <= 64 and cout <= 256 when the filters and two gathered tiles fit.  Other
- * shapes use the popcount kernel. */
+ * input buffers of at least one 128-pixel window; e2m1 operands when the
+ * channels fill an even number of 32-bit words and cout <= 240, int8
+ * otherwise); other strides with c <= 64 and cout <= 256 when the filters and
+ * two gathered tiles fit (int8).  Other shapes use the popcount kernel. */
 typedef enum bnn_gemm_engine {
     BNN_GEMM_ENGINE_AUTO = 0,
     BNN_GEMM_ENGINE_POPCOUNT = 1,
@@ -596,9 +597,11 @@ bnn_status bnn_pack_bit_planes(const uint8_t* codes, int64_t rows, int64_t K, in
  * for codes 0 <= a < 2^a_bits and 0 <= w < 2^w_bits given as bit planes
  * (DoReFa-Net's bit-convolution, which a bit-serial kernel computes as
  * sum over plane pairs of 2^(b + b') * popcount(a_b AND w_b')).  The
- * tensor-core kernel folds each row's planes back into one unsigned byte per
- * element in shared memory and multiplies u8 x u8, so all plane pairs cost
- * one pass.
+ * tensor-core kernels fold each row's planes back into one code per element
+ * in shared memory, so all plane pairs cost one pass: codes of up to two bits
+ * as exact e2m1 values (0..3, kind::mxf4, CTA pairs, when M > 128 and
+ * 9 * K rounded up to 256 is below 2^22), wider codes -- and every code
+ * under BNN_GEMM_ENGINE_TENSOR_I8 -- as unsigned bytes (u8 x u8).
  *   A: plane-interleaved [M rows x a_bits planes], row stride lda words.
  *   W: plane-interleaved [N rows x w_bits planes], row stride ldw words.
  *   a_bits, w_bits: 1 .. 4.  K * (2^a_bits - 1) * (2^w_bits - 1) must fit in
@@ -618,6 +621,9 @@ bnn_status bnn_bitserial_gemm(const uint32_t* A, int64_t lda, int a_bits, const 
  * sum_i alpha_i[n] * s_ji is formed by fused multiply-adds in i order, then
  * beta_j * v_j, then the J terms are added pairwise (j, j^1), (j, j^2), ...;
  * |Y - Y_exact| <= (I + J + 2) * 2^-24 * sum_j sum_i |beta_j alpha_i[n] s_ji|.
+ * The products run on the e2m1 tensor-core kernel in CTA pairs (when M
+ * exceeds 128 / J' rows, J' = J rounded up to a power of two) and on the int8
+ * one otherwise or under BNN_GEMM_ENGINE_TENSOR_I8; both give the same s_ji.
  *   H: plane-interleaved +1/-1 bases [M rows x J planes], stride ldh words
  *   (base j of row m, packed as by bnn_pack_sign, at packed row m * J + j).
  *   B: plane-interleaved [N rows x I planes], stride ldb words.

@@ -14,11 +14,12 @@
 // and zero-filled words) are +1 in both operands and are subtracted as in
 // the int8 kernel.
 //
-// Roles (sm_100a, one persistent CTA per SM; 17 warps, 14 in the pair mode of
-// the Cfg comment below):
-//  * warp 0     : TMA producer, packed tiles of 128 A rows and bn W rows x 8
-//                 words (256 elements of K, 32-byte swizzle) into a ring.
-//  * warps 2-12 : unpack, one thread per packed row (128 + up to 224).  Each
+// Roles (sm_100a, one persistent CTA per SM; Cfg below gives the warp counts:
+// 11 unpack warps for single CTAs, 8 in a CTA pair):
+//  * warp 0     : TMA producer, packed tiles of 128 A rows and the CTA's W
+//                 rows x 8 words (256 elements of K, 32-byte swizzle) into a
+//                 ring.
+//  * warps 2 .. : unpack, one thread per packed row (128 + the W rows).  Each
 //                 word becomes 16 bytes: word j of the result is
 //                 ((w << (3 - j)) & 0x88888888) | 0x22222222, i.e. nibble i
 //                 holds element 4i + j -- a fixed permutation of the word's
@@ -29,7 +30,7 @@
 //                 accumulator 1 at 256, the scale factors at 480..511); one
 //                 thread issues 4 tcgen05.mma (M = 128, N = bn, K = 64) per
 //                 stage.
-//  * warps 13-16: epilogue: TMEM -> registers -> the fused output modes of
+//  * last 4     : epilogue: TMEM -> registers -> the fused output modes of
 //                 the int8 kernel; dense int32 / fp32 outputs leave as 32 x 32
 //                 blocks through swizzled shared memory and TMA tensor stores.
 //                 They also fill the scale-factor columns once before the
@@ -82,7 +83,7 @@ constexpr int64_t MAX_KP = int64_t(1) << 20;
 // shared memory and its 128 x bn accumulator in its tensor memory, and the
 // even CTA issues the MMAs for both.  Per multiply-add the pair moves
 // (128 + bn / 2) instead of (128 + bn) rows through each SM's shared memory.
-template <bool PAIR, int MODE = 0>
+template <bool PAIR, int MODE = TC_BINARY>
 struct Cfg {
     static constexpr int CTAS = PAIR ? 2 : 1;
     static constexpr int BN_CTA_MAX = BN_MAX / CTAS;            // W rows per CTA
@@ -90,7 +91,7 @@ struct Cfg {
     static constexpr int U_B_BYTES = BN_CTA_MAX * ROW_BYTES;
     static constexpr int U_STAGE = U_A_BYTES + U_B_BYTES;
     // Plane-code mode: every code row brings up to MAX_F4_PLANES packed planes.
-    static constexpr int P_STAGE = (BM + BN_CTA_MAX) * P_ROW * (MODE == 1 ? MAX_F4_PLANES : 1);
+    static constexpr int P_STAGE = (BM + BN_CTA_MAX) * P_ROW * (MODE == TC_PLANE_CODES ? MAX_F4_PLANES : 1);
     static constexpr int UNPACK_WARPS = (BM + BN_CTA_MAX + 31) / 32;   // 11 single, 8 pair
     static constexpr int WARP_EPI0 = WARP_UNPACK0 + UNPACK_WARPS;
     static constexpr int THREADS = (WARP_EPI0 + EPI_WARPS) * 32;       // 544 single, 448 pair
@@ -103,7 +104,9 @@ struct Cfg {
     static_assert(PSTAGES >= 4, "packed ring too shallow");
     static_assert(SMEM_BYTES <= tc::SMEM_LIMIT, "shared memory");
     static_assert(U_STAGE % 1024 == 0 && P_STAGE % 256 == 0, "stage alignment (128B / 32B swizzle)");
-    static_assert((WARP_EPI0 & 3) == 0 || EPI_WARPS == 4, "the epilogue warps cover the four TMEM lane quadrants");
+    // Four consecutive epilogue warps have four different (warp & 3): the
+    // four TMEM lane quadrants a warp may access.
+    static_assert(EPI_WARPS == 4, "one epilogue warp per TMEM lane quadrant");
 };
 // Block-scaled instruction descriptor: A and B e2m1 (format 1 of kind::mxf4)
 // at bits 7-9 and 10-12, both K-major, N >> 3 at bits 17-22, scale format
