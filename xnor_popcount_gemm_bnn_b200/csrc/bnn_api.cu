@@ -343,9 +343,13 @@ bnn_status launch_gemm_f4(const uint32_t* A, int64_t lda, const uint32_t* W, int
     if (pairs < 0) return BNN_ERR_CUDA;
     const F4Plan plan = f4_plan(M, N, sms, pairs);
     const int bn = plan.bn, ctas = plan.pair ? 2 : 1;
+    // Packed words per row per stage (two K atoms in CTA pairs) and the
+    // matching TMA swizzle of the packed rows (32 or 64 bytes).
+    const int sbkw = plan.pair ? Cfg<true>::S_BKW : Cfg<false>::S_BKW;
+    const CUtensorMapSwizzle psw = sbkw == 16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
     CUtensorMap tmA, tmW;
-    if (!encode_packed_map(&tmA, A, kw, M, lda, BM, BKW, CU_TENSOR_MAP_SWIZZLE_32B) ||
-        !encode_packed_map(&tmW, W, kw, N, ldw, bn / ctas, BKW, CU_TENSOR_MAP_SWIZZLE_32B))
+    if (!encode_packed_map(&tmA, A, kw, M, lda, BM, sbkw, psw) ||
+        !encode_packed_map(&tmW, W, kw, N, ldw, bn / ctas, sbkw, psw))
         return BNN_ERR_CUDA;
     const int64_t tiles_m = ceil_div(M, (int64_t)BM * ctas), tiles_n = ceil_div(N, bn);
     if (tiles_m * tiles_n > INT_MAX) return BNN_ERR_INVALID_ARG;
@@ -369,9 +373,11 @@ bnn_status launch_gemm_f4(const uint32_t* A, int64_t lda, const uint32_t* W, int
                                            bnn::TcPlanes{}, pairs, stream);
 }
 
-// Padded K of the 4-bit kernel (whole 256-element stages).
+// Padded K of the 4-bit kernel: K rounded up to whole stages, taken at the
+// largest stage (two K atoms, 512 elements) so that the bound holds for
+// every launch plan.
 inline int64_t f4_padded_k(int64_t K) {
-    return ceil_div(packed_ld_words(K), bnn::f4::BKW) * bnn::f4::BKE;
+    return ceil_div(packed_ld_words(K), (int64_t)2 * bnn::f4::BKW) * 2 * bnn::f4::BKE;
 }
 
 // 3-D map over a plane-interleaved packed matrix (plane p of row r is packed
@@ -930,6 +936,7 @@ bnn_status bnn_bitserial_gemm(const uint32_t* A, int64_t lda, int a_bits, const 
             CUtensorMap fA, fW, fCi, fCf;
             std::memset(&fCi, 0, sizeof(fCi));
             std::memset(&fCf, 0, sizeof(fCf));
+            static_assert(bnn::f4::Cfg<true, bnn::TC_PLANE_CODES>::S_BKW == bnn::f4::BKW, "codes stage one K atom");
             if (!encode_plane_map(&fA, A, kw, a_bits, M, lda, a_bits, bnn::f4::BM, bnn::f4::BKW,
                                   CU_TENSOR_MAP_SWIZZLE_32B) ||
                 !encode_plane_map(&fW, W, kw, w_bits, N, ldw, w_bits, bn / 2, bnn::f4::BKW, CU_TENSOR_MAP_SWIZZLE_32B))
@@ -1009,8 +1016,10 @@ bnn_status bnn_binary_bases_gemm(const uint32_t* H, int64_t ldh, int J, const ui
             const int bn = f4_pair_tile_n(tiles_m, N, ip, pairs);
             CUtensorMap fA, fW, fC;
             std::memset(&fC, 0, sizeof(fC));
-            if (!encode_plane_map(&fA, H, kw, J, M, ldh, jp, rows_cta, bnn::f4::BKW, CU_TENSOR_MAP_SWIZZLE_32B) ||
-                !encode_plane_map(&fW, B, kw, I, N, ldb, ip, bn / 2 / ip, bnn::f4::BKW, CU_TENSOR_MAP_SWIZZLE_32B))
+            constexpr int sbkw = bnn::f4::Cfg<true, bnn::TC_BASES>::S_BKW;   // two K atoms: 64-byte rows
+            static_assert(sbkw == 16, "bases pairs stage two K atoms");
+            if (!encode_plane_map(&fA, H, kw, J, M, ldh, jp, rows_cta, sbkw, CU_TENSOR_MAP_SWIZZLE_64B) ||
+                !encode_plane_map(&fW, B, kw, I, N, ldb, ip, bn / 2 / ip, sbkw, CU_TENSOR_MAP_SWIZZLE_64B))
                 return BNN_ERR_CUDA;
             bnn::TcPlanes pl{};
             pl.ja = jp;

@@ -87,11 +87,20 @@ template <bool PAIR, int MODE = TC_BINARY>
 struct Cfg {
     static constexpr int CTAS = PAIR ? 2 : 1;
     static constexpr int BN_CTA_MAX = BN_MAX / CTAS;            // W rows per CTA
-    static constexpr int USTAGES = PAIR ? 4 : 3;                // unpacked ring
-    static constexpr int U_B_BYTES = BN_CTA_MAX * ROW_BYTES;
-    static constexpr int U_STAGE = U_A_BYTES + U_B_BYTES;
+    // K atoms (128-byte swizzle atoms, 256 elements) per stage.  CTA pairs
+    // of +1/-1 rows take two: each hand-off between the unpack warps and the
+    // MMA issuer then covers 512 elements of K (8 MMAs), half as many
+    // hand-offs per product; the smaller per-CTA W tile leaves the room.
+    static constexpr int KATOMS = (PAIR && MODE != TC_PLANE_CODES) ? 2 : 1;
+    static constexpr int S_BKE = BKE * KATOMS;                  // elements of K per stage
+    static constexpr int S_BKW = BKW * KATOMS;                  // packed words per row per stage
+    static constexpr int S_PROW = P_ROW * KATOMS;               // packed bytes per row per stage
+    static constexpr int S_UA = U_A_BYTES * KATOMS;             // unpacked A bytes per stage: [atom][row][128 B]
+    static constexpr int USTAGES = PAIR ? (KATOMS == 2 ? 2 : 4) : 3;   // unpacked ring
+    static constexpr int U_B_BYTES = BN_CTA_MAX * ROW_BYTES * KATOMS;
+    static constexpr int U_STAGE = S_UA + U_B_BYTES;
     // Plane-code mode: every code row brings up to MAX_F4_PLANES packed planes.
-    static constexpr int P_STAGE = (BM + BN_CTA_MAX) * P_ROW * (MODE == TC_PLANE_CODES ? MAX_F4_PLANES : 1);
+    static constexpr int P_STAGE = (BM + BN_CTA_MAX) * S_PROW * (MODE == TC_PLANE_CODES ? MAX_F4_PLANES : 1);
     static constexpr int UNPACK_WARPS = (BM + BN_CTA_MAX + 31) / 32;   // 11 single, 8 pair
     static constexpr int WARP_EPI0 = WARP_UNPACK0 + UNPACK_WARPS;
     static constexpr int THREADS = (WARP_EPI0 + EPI_WARPS) * 32;       // 544 single, 448 pair
@@ -103,7 +112,9 @@ struct Cfg {
     static constexpr int SMEM_BYTES = SMEM_FIXED + PSTAGES * P_STAGE;
     static_assert(PSTAGES >= 4, "packed ring too shallow");
     static_assert(SMEM_BYTES <= tc::SMEM_LIMIT, "shared memory");
-    static_assert(U_STAGE % 1024 == 0 && P_STAGE % 256 == 0, "stage alignment (128B / 32B swizzle)");
+    static_assert(U_STAGE % 1024 == 0 && S_UA % 1024 == 0 && (BN_CTA_MAX * ROW_BYTES) % 1024 == 0,
+                  "unpacked atoms need 1024-byte alignment (128B swizzle)");
+    static_assert(P_STAGE % 512 == 0 && (BM * S_PROW) % 512 == 0, "packed stages: 32B / 64B swizzle alignment");
     // Four consecutive epilogue warps have four different (warp & 3): the
     // four TMEM lane quadrants a warp may access.
     static_assert(EPI_WARPS == 4, "one epilogue warp per TMEM lane quadrant");
@@ -272,6 +283,7 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     using C = Cfg<PAIR, MODE>;
     constexpr int CTAS = C::CTAS, USTAGES = C::USTAGES, PSTAGES = C::PSTAGES, U_STAGE = C::U_STAGE,
                   P_STAGE = C::P_STAGE, UNPACK_WARPS = C::UNPACK_WARPS, WARP_EPI0 = C::WARP_EPI0;
+    constexpr int KATOMS = C::KATOMS, S_BKE = C::S_BKE, S_BKW = C::S_BKW, S_PROW = C::S_PROW, S_UA = C::S_UA;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* uring = smem;                                          // USTAGES x (A 16 KiB | W rows)
@@ -292,7 +304,7 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int nk = (kw + BKW - 1) / BKW;
+    const int nk = (kw + S_BKW - 1) / S_BKW;
     const int tiles = tiles_m * tiles_n;
     // Pair: CTA `rank` of cluster `cid` holds A rows 128 rank .. of the
     // tile's 256 and W rows bn_cta rank .. of its bn; the even CTA leads.
@@ -304,9 +316,9 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const int ja = MODE == TC_BINARY ? 1 : pl.ja, jw = MODE == TC_BINARY ? 1 : pl.jw;
     const int rows_cta = MODE == TC_BASES ? BM / ja : BM;
     const int cols_tile = MODE == TC_BASES ? bn / jw : bn;
-    const int pa_bytes = MODE == TC_PLANE_CODES ? BM * ja * P_ROW : P_A_BYTES;
+    const int pa_bytes = MODE == TC_PLANE_CODES ? BM * ja * S_PROW : BM * S_PROW;
     const uint32_t stage_tx =
-        MODE == TC_PLANE_CODES ? (uint32_t)(BM * ja + bn_cta * jw) * P_ROW : (uint32_t)(BM + bn_cta) * P_ROW;
+        MODE == TC_PLANE_CODES ? (uint32_t)(BM * ja + bn_cta * jw) * S_PROW : (uint32_t)(BM + bn_cta) * S_PROW;
 
     if (threadIdx.x == 0) {
         prefetch_tensormap(&tmA);
@@ -363,11 +375,11 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     uint8_t* dst = pring + s * P_STAGE;
                     mbar_arrive_expect_tx(&pfull[s], stage_tx);
                     if constexpr (MODE == TC_BINARY) {
-                        tma_load_2d(dst, &tmA, ks * BKW, m0, &pfull[s]);
-                        tma_load_2d(dst + P_A_BYTES, &tmW, ks * BKW, n0, &pfull[s]);
+                        tma_load_2d(dst, &tmA, ks * S_BKW, m0, &pfull[s]);
+                        tma_load_2d(dst + pa_bytes, &tmW, ks * S_BKW, n0, &pfull[s]);
                     } else {
-                        tma_load_3d(dst, &tmA, ks * BKW, 0, m0, &pfull[s]);
-                        tma_load_3d(dst + pa_bytes, &tmW, ks * BKW, 0, n0, &pfull[s]);
+                        tma_load_3d(dst, &tmA, ks * S_BKW, 0, m0, &pfull[s]);
+                        tma_load_3d(dst + pa_bytes, &tmW, ks * S_BKW, 0, n0, &pfull[s]);
                     }
                     ++issued;
                 }
@@ -400,12 +412,15 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     }
                     tc_fence_after();
                     const uint32_t a_addr = ubase + s * U_STAGE;
-                    const uint32_t b_addr = a_addr + U_A_BYTES;
+                    const uint32_t b_addr = a_addr + S_UA;
                     #pragma unroll
-                    for (int kk = 0; kk < BKE / UMMA_K; ++kk) {
-                        // 32 bytes (64 elements) per K step inside the swizzle atom.
-                        mma_mxf4<PAIR>(d_tmem, umma_desc_sw128(a_addr + kk * 32), umma_desc_sw128(b_addr + kk * 32),
-                                       id, sfa, sfb, (ks | kk) != 0 ? 1u : 0u);
+                    for (int kk = 0; kk < S_BKE / UMMA_K; ++kk) {
+                        // 32 bytes (64 elements) per K step inside a swizzle atom;
+                        // atom kk / 4 of A (B) sits BM (BN_CTA_MAX) rows of 128 B on.
+                        const uint32_t ka = (uint32_t)(kk >> 2) * (BM * ROW_BYTES) + (uint32_t)(kk & 3) * 32;
+                        const uint32_t kb = (uint32_t)(kk >> 2) * (C::BN_CTA_MAX * ROW_BYTES) + (uint32_t)(kk & 3) * 32;
+                        mma_mxf4<PAIR>(d_tmem, umma_desc_sw128(a_addr + ka), umma_desc_sw128(b_addr + kb), id, sfa, sfb,
+                                       (ks | kk) != 0 ? 1u : 0u);
                     }
                     f4_commit<PAIR>(&uempty[s], all);
                 }
@@ -435,7 +450,8 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const int my_tiles = cid < tiles ? (tiles - 1 - cid) / ncl + 1 : 0;
         const uint32_t total = (uint32_t)my_tiles * (uint32_t)nk;
         uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;              // words 0..3 and 4..7 of the row
-        uint4 lo1 = lo, hi1 = lo;                                     // plane codes: the second plane
+        uint4 lo1 = lo, hi1 = lo;                                     // plane codes: the second plane;
+                                                                      // two K atoms: words 8..15
         // Plane codes: the row's planes are consecutive 32-byte slots, from
         // slot s0 on (each slot's halves swizzled by its own index).
         const int nplanes = MODE == TC_PLANE_CODES ? (is_a ? ja : jw) : 1;
@@ -444,14 +460,24 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const uint32_t ps = gg % (uint32_t)PSTAGES;
             if (!__all_sync(0xffffffffu, tc_wait(&pfull[ps], (gg / PSTAGES) & 1, abort_flag))) return false;
             if (active) {
-                const uint8_t* src = pring + ps * P_STAGE + s0 * P_ROW;
-                const int h0 = MODE == TC_PLANE_CODES ? 16 * ((s0 >> 2) & 1) : hsw;
-                lo = *reinterpret_cast<const uint4*>(src + h0);
-                hi = *reinterpret_cast<const uint4*>(src + (h0 ^ 16));
-                if (MODE == TC_PLANE_CODES && nplanes > 1) {
-                    const int h1 = 16 * (((s0 + 1) >> 2) & 1);
-                    lo1 = *reinterpret_cast<const uint4*>(src + P_ROW + h1);
-                    hi1 = *reinterpret_cast<const uint4*>(src + P_ROW + (h1 ^ 16));
+                const uint8_t* src = pring + ps * P_STAGE + s0 * S_PROW;
+                if constexpr (KATOMS == 2) {
+                    // 64-byte rows, written with the 64-byte swizzle: 16-byte
+                    // chunk c of slot s0 sits at (c ^ ((s0 >> 1) & 3)) * 16.
+                    const int x = (s0 >> 1) & 3;
+                    lo = *reinterpret_cast<const uint4*>(src + ((0 ^ x) << 4));
+                    hi = *reinterpret_cast<const uint4*>(src + ((1 ^ x) << 4));
+                    lo1 = *reinterpret_cast<const uint4*>(src + ((2 ^ x) << 4));
+                    hi1 = *reinterpret_cast<const uint4*>(src + ((3 ^ x) << 4));
+                } else {
+                    const int h0 = MODE == TC_PLANE_CODES ? 16 * ((s0 >> 2) & 1) : hsw;
+                    lo = *reinterpret_cast<const uint4*>(src + h0);
+                    hi = *reinterpret_cast<const uint4*>(src + (h0 ^ 16));
+                    if (MODE == TC_PLANE_CODES && nplanes > 1) {
+                        const int h1 = 16 * (((s0 + 1) >> 2) & 1);
+                        lo1 = *reinterpret_cast<const uint4*>(src + S_PROW + h1);
+                        hi1 = *reinterpret_cast<const uint4*>(src + S_PROW + (h1 ^ 16));
+                    }
                 }
             }
             return true;
@@ -464,7 +490,19 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             if (active) {
                 // Chunk q of the row at (q ^ (r & 7)) * 16: the eight lanes of a
                 // store phase (eight consecutive rows) hit distinct banks.
-                uint8_t* row = uring + us * U_STAGE + (is_a ? 0 : U_A_BYTES) + r * ROW_BYTES;
+                uint8_t* row = uring + us * U_STAGE + (is_a ? 0 : S_UA) + r * ROW_BYTES;
+                if constexpr (KATOMS == 2) {
+                    // Words 8..15 go to the second K atom, BM (or BN_CTA_MAX) rows on.
+                    uint8_t* row2 = row + (is_a ? BM : C::BN_CTA_MAX) * ROW_BYTES;
+                    *reinterpret_cast<uint4*>(row2 + ((0 ^ sw) << 4)) = expand_word_e2m1(lo1.x);
+                    *reinterpret_cast<uint4*>(row2 + ((1 ^ sw) << 4)) = expand_word_e2m1(lo1.y);
+                    *reinterpret_cast<uint4*>(row2 + ((2 ^ sw) << 4)) = expand_word_e2m1(lo1.z);
+                    *reinterpret_cast<uint4*>(row2 + ((3 ^ sw) << 4)) = expand_word_e2m1(lo1.w);
+                    *reinterpret_cast<uint4*>(row2 + ((4 ^ sw) << 4)) = expand_word_e2m1(hi1.x);
+                    *reinterpret_cast<uint4*>(row2 + ((5 ^ sw) << 4)) = expand_word_e2m1(hi1.y);
+                    *reinterpret_cast<uint4*>(row2 + ((6 ^ sw) << 4)) = expand_word_e2m1(hi1.z);
+                    *reinterpret_cast<uint4*>(row2 + ((7 ^ sw) << 4)) = expand_word_e2m1(hi1.w);
+                }
                 if constexpr (MODE == TC_PLANE_CODES) {
                     *reinterpret_cast<uint4*>(row + ((0 ^ sw) << 4)) = fold_planes_e2m1(lo.x, lo1.x);
                     *reinterpret_cast<uint4*>(row + ((1 ^ sw) << 4)) = fold_planes_e2m1(lo.y, lo1.y);
@@ -520,7 +558,7 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         uint8_t* obuf_f = obuf_i + OUT_BLOCK;                         // and fp32 block
         const bool tma_i = (tma_out & 1) != 0 && ep.c_i32 != nullptr;
         const bool tma_f = (tma_out & 2) != 0 && ep.c_f32 != nullptr;
-        const int kp = nk * BKE;                                      // padded K: acc = kp - 2 * popcount
+        const int kp = nk * S_BKE;                                    // padded K: acc = kp - 2 * popcount
         // +1/-1: each pad position adds (+1)(+1); plane codes: pads are code 0.
         const int pad = MODE == TC_PLANE_CODES ? 0 : kp - K;
         const float padf = (float)pad;
@@ -694,7 +732,7 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         // the same named barrier as the other modes.
         const int quad = warp & 3;
         const int ew = warp - WARP_EPI0;
-        const int kp = nk * BKE;
+        const int kp = nk * S_BKE;
         const int pad = kp - K;
         const int L = 32 * quad + lane;
         const int jl = L & (ja - 1);
