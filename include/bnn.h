@@ -599,8 +599,8 @@ bnn_status bnn_pack_bit_planes(const uint8_t* codes, int64_t rows, int64_t K, in
  * sum over plane pairs of 2^(b + b') * popcount(a_b AND w_b')).  The
  * tensor-core kernels fold each row's planes back into one code per element
  * in shared memory, so all plane pairs cost one pass: codes of up to two bits
- * as exact e2m1 values (0..3, kind::mxf4, CTA pairs, when M > 128 and
- * 9 * K rounded up to 256 is below 2^22), wider codes -- and every code
+ * as exact e2m1 values (code c as c / 2, kind::mxf4, CTA pairs, when
+ * M > 128 and 9 * K rounded up to 256 is below 2^22), wider codes -- and every code
  * under BNN_GEMM_ENGINE_TENSOR_I8 -- as unsigned bytes (u8 x u8).
  *   A: plane-interleaved [M rows x a_bits planes], row stride lda words.
  *   W: plane-interleaved [N rows x w_bits planes], row stride ldw words.

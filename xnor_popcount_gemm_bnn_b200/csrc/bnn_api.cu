@@ -925,9 +925,10 @@ bnn_status bnn_bitserial_gemm(const uint32_t* A, int64_t lda, int a_bits, const 
         return BNN_ERR_ALIGNMENT;
     if (M == 0 || N == 0) return BNN_OK;
     {
-        // Codes of up to two bits are exact e2m1 values: the e2m1 kernel in
-        // CTA pairs, while every partial sum (at most 9 per element of the
-        // padded K) stays an integer the epilogue converts exactly.
+        // Codes of up to two bits are exact e2m1 values (code c as the value
+        // c / 2): the e2m1 kernel in CTA pairs, while every partial sum times
+        // 4 (at most 9 per element of the padded K) stays an integer the
+        // epilogue converts exactly.
         const int engine = g_gemm_engine.load(std::memory_order_relaxed);
         const int pairs = engine == BNN_GEMM_ENGINE_TENSOR_I8 ? -1 : gemm_f4_pairs_resident();
         if (a_bits <= bnn::f4::MAX_F4_PLANES && w_bits <= bnn::f4::MAX_F4_PLANES && pairs > 0 && pairs < kNoPairs &&

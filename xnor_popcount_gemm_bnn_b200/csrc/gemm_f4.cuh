@@ -64,8 +64,11 @@ constexpr int MAX_PSTAGES = 8;
 constexpr int OUT_BLOCK = 32 * 32 * 4;
 constexpr int OUT_BYTES = EPI_WARPS * 2 * OUT_BLOCK;
 // Per-tile column parameters, one copy shared by the epilogue warps, double
-// buffered across tiles: float4 {alpha, gamma, beta, -} and int2 {c1, len2}.
-constexpr int COLP_BYTES = 2 * BN_MAX * (16 + 8);
+// buffered across tiles: five arrays [2][BN_MAX] of 4-byte values (alpha,
+// gamma, beta as fp32; c1, len2 as int32), so that an epilogue thread reads
+// four columns' worth of one parameter with one 16-byte load.
+constexpr int COLP_ARRAYS = 5;
+constexpr int COLP_BYTES = COLP_ARRAYS * 2 * BN_MAX * 4;
 static_assert(ACC_STRIDE + BN_MAX <= SF_COL, "accumulators overlap the scale factors");
 static_assert(U_A_BYTES % 1024 == 0 && OUT_BLOCK % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 // Named barrier of the epilogue warps (id 0 is __syncthreads).
@@ -247,25 +250,30 @@ __device__ __forceinline__ uint4 expand_word_e2m1(uint32_t w) {
 }
 
 // Bit planes of unsigned codes (one or two planes: codes 0..3) -> e2m1
-// code values, 16 bytes per 32 codes, in expand_word_e2m1's element order
-// (word j, nibble i = element 4i + j).  With t0, t1 the two planes' bits at
-// bit 3 of each nibble: code 1 -> 0x2 (1.0), 2 -> 0x4 (2.0), 3 -> 0x5 (3.0),
-// 0 -> 0x0.
+// values, 16 bytes per 32 codes, in expand_word_e2m1's element order (word
+// j, nibble i = element 4i + j).  The e2m1 nibble c (c = 0..3) is the value
+// c / 2 (0, 0.5 subnormal, 1.0, 1.5), so a code's nibble is the code itself:
+// plane 0 goes to bit 0 of the nibble, plane 1 to bit 1.  The MMA then sums
+// (a / 2)(w / 2), a quarter of the code product, and the epilogue scales the
+// fp32 accumulator by 4 (exact).
 __device__ __forceinline__ uint4 fold_planes_e2m1(uint32_t p0, uint32_t p1) {
-    constexpr uint32_t top = 0x88888888u;
-    uint32_t o[4];
-    #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const uint32_t t0 = (p0 << (3 - j)) & top, t1 = (p1 << (3 - j)) & top;
-        o[j] = (t1 >> 1) | ((t0 & ~t1) >> 2) | ((t0 & t1) >> 3);
-    }
-    return make_uint4(o[0], o[1], o[2], o[3]);
+    constexpr uint32_t b0 = 0x11111111u, b1 = 0x22222222u;
+    return make_uint4((p0 & b0) | ((p1 << 1) & b1), ((p0 >> 1) & b0) | (p1 & b1),
+                      ((p0 >> 2) & b0) | ((p1 >> 1) & b1), ((p0 >> 3) & b0) | ((p1 >> 2) & b1));
 }
 
 // fp32 accumulator holding an integer of magnitude < 2^22 -> that integer
 // (adding 1.5 * 2^23 puts it in the low mantissa bits).
 __device__ __forceinline__ int32_t acc_to_int(uint32_t bits) {
     return __float_as_int(__uint_as_float(bits) + 12582912.0f) - 0x4B400000;
+}
+
+// The same for an accumulator that holds the integer / scale (scale a power
+// of two; the fused multiply-add is exact).
+template <int SCALE>
+__device__ __forceinline__ int32_t acc_to_int_scaled(uint32_t bits) {
+    if constexpr (SCALE == 1) return acc_to_int(bits);
+    else return __float_as_int(fmaf(__uint_as_float(bits), (float)SCALE, 12582912.0f)) - 0x4B400000;
 }
 
 constexpr int log2_pow2(int v) { return v <= 1 ? 0 : 1 + log2_pow2(v >> 1); }
@@ -359,9 +367,8 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     uint8_t* uring = smem;                                          // USTAGES x (A 16 KiB | W rows)
     uint8_t* oring = uring + USTAGES * U_STAGE;                     // [EPI_WARPS][int32 | fp32] 32 x 32 blocks
     uint8_t* pring = oring + OUT_BYTES;                             // PSTAGES x (A | W packed)
-    float4* colf = reinterpret_cast<float4*>(pring + PSTAGES * P_STAGE);   // [2][BN_MAX]
-    int2* colt = reinterpret_cast<int2*>(colf + 2 * BN_MAX);               // [2][BN_MAX]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(colt + 2 * BN_MAX);
+    float* colp = reinterpret_cast<float*>(pring + PSTAGES * P_STAGE);     // COLP_ARRAYS x [2][BN_MAX]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(colp + COLP_ARRAYS * 2 * BN_MAX);
     uint64_t* pfull = bars;
     uint64_t* pempty = pfull + MAX_PSTAGES;
     uint64_t* ufull = pempty + MAX_PSTAGES;
@@ -632,6 +639,8 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         // +1/-1: each pad position adds (+1)(+1); plane codes: pads are code 0.
         const int pad = MODE == TC_PLANE_CODES ? 0 : kp - K;
         const float padf = (float)pad;
+        // Plane codes: the accumulator holds a quarter of the code product.
+        constexpr int ACC_SCALE = MODE == TC_PLANE_CODES ? 4 : 1;
         const bool affine = ep.gamma != nullptr;
         const int chunks = bn / 32;
         const uint32_t sw = (uint32_t)(lane & 7);
@@ -640,8 +649,11 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         for (int t = cid; t < tiles; t += ncl, ++lt) {
             const int b = lt & 1;
             const int m0 = (t / tiles_n) * (BM * CTAS) + BM * (int)rank, n0 = (t % tiles_n) * bn;
-            float4* cf = colf + b * BN_MAX;
-            int2* ct = colt + b * BN_MAX;
+            float* ca = colp + b * BN_MAX;                            // alpha
+            float* cg = ca + 2 * BN_MAX;                              // gamma
+            float* cb = cg + 2 * BN_MAX;                              // beta
+            int* c1 = reinterpret_cast<int*>(cb + 2 * BN_MAX);        // threshold range start
+            int* cl = c1 + 2 * BN_MAX;                                // and twice its length
             // Every warp finished tile lt - 2 (the last reader of this copy)
             // before it reached the barrier of tile lt - 1.
             for (int i = 32 * ew + lane; i < bn; i += 32 * EPI_WARPS) {
@@ -668,8 +680,11 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         th = make_int2((int)(uint32_t)(kp - 2 * lo), (int)(uint32_t)(2 * len));
                     }
                 }
-                cf[i] = f;
-                ct[i] = th;
+                ca[i] = f.x;
+                cg[i] = f.y;
+                cb[i] = f.z;
+                c1[i] = th.x;
+                cl[i] = th.y;
             }
             named_bar_sync(EPI_BAR, EPI_WARPS * 32);
             ok = ok && __all_sync(0xffffffffu, tc_wait(&afull[b], (lt >> 1) & 1, abort_flag));
@@ -700,9 +715,15 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 if (ep.c_bits != nullptr) {
                     uint32_t word = 0;
                     #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int2 q = ct[32 * c + j];
-                        word |= ((uint32_t)(q.x - acc_to_int(r[j])) < (uint32_t)q.y ? 1u : 0u) << j;
+                    for (int q = 0; q < 8; ++q) {
+                        const int4 lo = reinterpret_cast<const int4*>(c1 + 32 * c)[q];
+                        const int4 ln = reinterpret_cast<const int4*>(cl + 32 * c)[q];
+                        const int los[4] = {lo.x, lo.y, lo.z, lo.w}, lns[4] = {ln.x, ln.y, ln.z, ln.w};
+                        #pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const int j = 4 * q + k;
+                            word |= ((uint32_t)(los[k] - acc_to_int_scaled<ACC_SCALE>(r[j])) < (uint32_t)lns[k] ? 1u : 0u) << j;
+                        }
                     }
                     if (m < M && nb / 32 < ep.bits_words) ep.c_bits[(int64_t)m * ep.ldb + nb / 32] = word;
                 }
@@ -715,8 +736,10 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     #pragma unroll
                     for (int q = 0; q < 8; ++q)
                         *reinterpret_cast<int4*>(rowp + (((uint32_t)q ^ sw) << 4)) =
-                            make_int4(acc_to_int(r[4 * q]) - pad, acc_to_int(r[4 * q + 1]) - pad,
-                                      acc_to_int(r[4 * q + 2]) - pad, acc_to_int(r[4 * q + 3]) - pad);
+                            make_int4(acc_to_int_scaled<ACC_SCALE>(r[4 * q]) - pad,
+                                      acc_to_int_scaled<ACC_SCALE>(r[4 * q + 1]) - pad,
+                                      acc_to_int_scaled<ACC_SCALE>(r[4 * q + 2]) - pad,
+                                      acc_to_int_scaled<ACC_SCALE>(r[4 * q + 3]) - pad);
                     fence_proxy_async_shared();
                     __syncwarp();
                     if (lane == 0) {
@@ -728,8 +751,10 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     const bool vec = full_chunk && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0);
                     #pragma unroll
                     for (int j = 0; j < 32; j += 4) {
-                        const int4 o = make_int4(acc_to_int(r[j]) - pad, acc_to_int(r[j + 1]) - pad,
-                                                 acc_to_int(r[j + 2]) - pad, acc_to_int(r[j + 3]) - pad);
+                        const int4 o = make_int4(acc_to_int_scaled<ACC_SCALE>(r[j]) - pad,
+                                                 acc_to_int_scaled<ACC_SCALE>(r[j + 1]) - pad,
+                                                 acc_to_int_scaled<ACC_SCALE>(r[j + 2]) - pad,
+                                                 acc_to_int_scaled<ACC_SCALE>(r[j + 3]) - pad);
                         if (vec) {
                             *reinterpret_cast<int4*>(dst + j) = o;
                         } else {
@@ -741,8 +766,8 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     }
                 }
                 if (ep.c_f32 != nullptr && (tma_f || m < M)) {
-                    // acc - pad is an integer below 2^21: exact in fp32, so
-                    // f.x * (acc - pad) is alpha * (float)s.
+                    // ACC_SCALE * acc - pad is an integer below 2^22: exact
+                    // in fp32, so alpha times it is alpha * (float)s.
                     if (tma_f) {
                         if (lane == 0) { if (tma_i) bulk_wait_read<1>(); else bulk_wait_read<0>(); }
                         __syncwarp();
@@ -751,12 +776,19 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     const bool vec = full_chunk && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0);
                     #pragma unroll
                     for (int q = 0; q < 8; ++q) {
+                        const float4 a4 = reinterpret_cast<const float4*>(ca + 32 * c)[q];
+                        float4 g4 = make_float4(1.f, 1.f, 1.f, 1.f), b4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (affine) {
+                            g4 = reinterpret_cast<const float4*>(cg + 32 * c)[q];
+                            b4 = reinterpret_cast<const float4*>(cb + 32 * c)[q];
+                        }
+                        const float as[4] = {a4.x, a4.y, a4.z, a4.w}, gs[4] = {g4.x, g4.y, g4.z, g4.w},
+                                    bs[4] = {b4.x, b4.y, b4.z, b4.w};
                         float y[4];
                         #pragma unroll
                         for (int k = 0; k < 4; ++k) {
-                            const float4 f = cf[32 * c + 4 * q + k];
-                            float v = f.x * (__uint_as_float(r[4 * q + k]) - padf);
-                            if (affine) v = fmaf(f.y, v, f.z);
+                            float v = as[k] * fmaf(__uint_as_float(r[4 * q + k]), (float)ACC_SCALE, -padf);
+                            if (affine) v = fmaf(gs[k], v, bs[k]);
                             y[k] = v;
                         }
                         if (tma_f) {
@@ -815,7 +847,7 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         for (int t = cid; t < tiles; t += ncl, ++lt) {
             const int b = lt & 1;
             const int m0 = (t / tiles_n) * (rows_cta * CTAS) + rows_cta * (int)rank, n0 = (t % tiles_n) * cols_tile;
-            float* ca = reinterpret_cast<float*>(colf + b * BN_MAX);   // alpha of each accumulator column
+            float* ca = colp + b * BN_MAX;                             // alpha of each accumulator column
             for (int i = 32 * ew + lane; i < bn; i += 32 * EPI_WARPS) {
                 const int n = n0 + i / jw, ib = i & (jw - 1);
                 ca[i] = (n < N && ib < pl.i_real) ? __ldg(pl.alpha + (int64_t)ib * pl.lda_alpha + n) : 0.0f;
