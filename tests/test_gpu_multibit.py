@@ -70,7 +70,7 @@ SHAPES = [(1, 1, 1), (7, 5, 33), (130, 300, 1000), (257, 129, 4097), (64, 256, 1
 
 @pytest.mark.parametrize("a_bits,w_bits", [(1, 1), (2, 2), (1, 2), (2, 1), (3, 2), (4, 4), (4, 1), (2, 4)])
 @pytest.mark.parametrize("M,N,K", SHAPES)
-def test_bitserial_gemm(M, N, K, a_bits, w_bits):
+def test_bitserial_gemm(M, N, K, a_bits, w_bits, tc_engine):
     a = _codes(M, K, a_bits, 11 * M + K + a_bits)
     w = _codes(N, K, w_bits, 13 * N + K + w_bits)
     A = _pack_planes(a, a_bits, K)
@@ -182,9 +182,17 @@ def _bases_reference(h_real, b_real, alpha, beta):
     return y, mag
 
 
+@pytest.fixture(params=[bnn.BNN_GEMM_ENGINE_TENSOR, bnn.BNN_GEMM_ENGINE_TENSOR_I8], ids=["tensor", "tensor_i8"])
+def tc_engine(request):
+    """TENSOR: the e2m1 kernel in CTA pairs where M allows, else int8;
+    TENSOR_I8: the int8 kernel for every shape."""
+    with bnn.gemm_engine(request.param):
+        yield request.param
+
+
 @pytest.mark.parametrize("J,I", [(1, 1), (2, 3), (3, 3), (4, 2), (5, 8), (8, 1), (1, 4)])
 @pytest.mark.parametrize("M,N,K", [(1, 1, 1), (7, 5, 33), (130, 300, 1000), (70, 129, 4097)])
-def test_binary_bases_gemm(M, N, K, J, I):
+def test_binary_bases_gemm(M, N, K, J, I, tc_engine):
     h_real, b_real, alpha, beta = _bases_case(M, N, K, J, I, M + N + K + 10 * J + I)
     H = _pack_bases(h_real, J, M, K)
     B = _pack_bases(b_real, I, N, K)
@@ -197,6 +205,26 @@ def test_binary_bases_gemm(M, N, K, J, I):
     err = np.abs(got - y_ref)
     bound = (I + J + 2) * U * mag
     assert np.all(err <= bound), f"max err/bound {np.max(err / np.maximum(bound, 1e-300))}"
+    assert_no_device_error()
+
+
+@pytest.mark.parametrize("col0,ld", [(0, 304), (1, 304), (0, 303), (3, 311)])
+def test_binary_bases_strided_output(col0, ld, tc_engine):
+    """Y as a column window of a wider buffer: row strides and start columns
+    with and without 16-byte alignment (vector and scalar stores), and the
+    columns around the window left untouched."""
+    M, N, K, J, I = 300, 290, 700, 3, 2
+    h_real, b_real, alpha, beta = _bases_case(M, N, K, J, I, 31 + col0 + ld)
+    H, B = _pack_bases(h_real, J, M, K), _pack_bases(b_real, I, N, K)
+    big = torch.full((M, ld), -7.0, dtype=torch.float32, device=dev())
+    Y = big[:, col0:col0 + N]
+    bnn.bnn_binary_bases_gemm(H, J, B, I, K, beta.to(dev()), alpha.to(dev()), Y)
+    torch.cuda.synchronize()
+    y_ref, mag = _bases_reference(h_real, b_real, alpha, beta)
+    got = Y.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - y_ref) <= (I + J + 2) * U * mag)
+    rest = torch.cat([big[:, :col0].flatten(), big[:, col0 + N:].flatten()])
+    assert bool((rest == -7.0).all())
     assert_no_device_error()
 
 

@@ -276,75 +276,6 @@ __device__ __forceinline__ int32_t acc_to_int_scaled(uint32_t bits) {
     else return __float_as_int(fmaf(__uint_as_float(bits), (float)SCALE, 12582912.0f)) - 0x4B400000;
 }
 
-constexpr int log2_pow2(int v) { return v <= 1 ? 0 : 1 + log2_pow2(v >> 1); }
-
-// Binary bases, one 32-column accumulator chunk of one thread (lane jl of
-// the JA lanes of its output row; JW accumulator columns per output column,
-// so the chunk covers G = 32 / JW output columns).  acc holds s + pad for
-// each base pair (s the +1/-1 product, pad the +1 K padding): the fp32
-// difference is exact.  v_o = sum_i alpha_i[n_o] s_ji (fused multiply-adds
-// in i order), times beta_j; the JA lanes of the row then add their v by a
-// reduce-scatter, low lane bit first: at each step a lane keeps one half of
-// its values, hands the other half to its partner and adds the partner's
-// half of its own, so the adds pair up exactly as a butterfly would, but a
-// row's outputs end up spread over its lanes (P = G / JA consecutive ones
-// each) after G (1 - 1 / JA) shuffles instead of G log2 JA.  With G < JA the
-// last steps are a butterfly and the lowest lane of each group stores.
-// Shared-memory reads (the chunk's 32 alphas as eight broadcast 16-byte
-// loads) and shuffles share the shared-memory pipe with the unpack warps'
-// stores and the MMAs' operand reads, so the epilogue keeps both few.
-template <int JA, int JW>
-__device__ __forceinline__ void bases_combine_chunk(const uint32_t (&acc)[32], const float* ca, float padf, float bj,
-                                                    int jl, float* yrow, int nb, int N, bool vec) {
-    constexpr int G = 32 / JW;
-    constexpr int LOG_JA = log2_pow2(JA), LOG_G = log2_pow2(G);
-    constexpr int SCAT = LOG_JA < LOG_G ? LOG_JA : LOG_G;
-    constexpr int P = G >> SCAT;
-    float v[G];
-    #pragma unroll
-    for (int g = 0; g < G; ++g) v[g] = 0.0f;
-    #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        const float4 a = reinterpret_cast<const float4*>(ca)[q];
-        const float av[4] = {a.x, a.y, a.z, a.w};
-        #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int col = 4 * q + e;
-            v[col / JW] = fmaf(av[e], __uint_as_float(acc[col]) - padf, v[col / JW]);
-        }
-    }
-    #pragma unroll
-    for (int g = 0; g < G; ++g) v[g] *= bj;
-    int o0 = 0;                                       // first output column (of the chunk) this lane keeps
-    #pragma unroll
-    for (int s = 0; s < SCAT; ++s) {
-        const int half = G >> (s + 1);
-        const bool up = ((jl >> s) & 1) != 0;
-        #pragma unroll
-        for (int h = 0; h < half; ++h) {
-            const float send = up ? v[h] : v[h + half];
-            const float keep = up ? v[h + half] : v[h];
-            v[h] = keep + __shfl_xor_sync(0xffffffffu, send, 1 << s);
-        }
-        if (up) o0 += half;
-    }
-    #pragma unroll
-    for (int s = SCAT; s < LOG_JA; ++s) v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1 << s);
-    if ((jl >> SCAT) != 0 || yrow == nullptr) return;
-    const int n = nb + o0;
-    constexpr int VW = P < 4 ? P : 4;
-    if (vec && VW > 1 && n + P <= N && (n & (VW - 1)) == 0) {
-        #pragma unroll
-        for (int p = 0; p < P; p += VW) {
-            if constexpr (VW == 4) *reinterpret_cast<float4*>(yrow + n + p) = make_float4(v[p], v[p + 1], v[p + 2], v[p + 3]);
-            else if constexpr (VW == 2) *reinterpret_cast<float2*>(yrow + n + p) = make_float2(v[p], v[p + 1]);
-        }
-    } else {
-        #pragma unroll
-        for (int p = 0; p < P; ++p)
-            if (n + p < N) yrow[n + p] = v[p];
-    }
-}
 
 // MODE (TcMode of gemm_tc.cuh): TC_BINARY the +1/-1 product; TC_PLANE_CODES
 // unsigned codes of one or two bit planes (3-D TMA boxes bring a code row's
@@ -833,7 +764,7 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const int quad = warp & 3;
         const int ew = warp - WARP_EPI0;
         const int kp = nk * S_BKE;
-        const float padf = (float)(kp - K);
+        const int pad = kp - K;
         const int L = 32 * quad + lane;
         const int jl = L & (ja - 1);
         const float bj = jl < pl.j_real ? __ldg(pl.beta + jl) : 0.0f;
@@ -873,18 +804,7 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 if (nb >= N) continue;                                // uniform across the warp
                 const float* cc = ca + 32 * c;
                 float* yrow = m < M ? pl.y + (int64_t)m * pl.ldy : nullptr;
-                switch (shape) {                                      // uniform across the kernel
-#define BNN_BASES_CASE(LA, LW)                                                                   \
-    case (LA) * 4 + (LW):                                                                        \
-        bases_combine_chunk<1 << (LA), 1 << (LW)>(r, cc, padf, bj, jl, yrow, nb, N, vec);       \
-        break;
-                    BNN_BASES_CASE(0, 0) BNN_BASES_CASE(0, 1) BNN_BASES_CASE(0, 2) BNN_BASES_CASE(0, 3)
-                    BNN_BASES_CASE(1, 0) BNN_BASES_CASE(1, 1) BNN_BASES_CASE(1, 2) BNN_BASES_CASE(1, 3)
-                    BNN_BASES_CASE(2, 0) BNN_BASES_CASE(2, 1) BNN_BASES_CASE(2, 2) BNN_BASES_CASE(2, 3)
-                    BNN_BASES_CASE(3, 0) BNN_BASES_CASE(3, 1) BNN_BASES_CASE(3, 2) BNN_BASES_CASE(3, 3)
-#undef BNN_BASES_CASE
-                    default: break;
-                }
+                bases_combine<false>(shape, r, cc, pad, bj, jl, yrow, nb, N, vec);
             }
         }
     }

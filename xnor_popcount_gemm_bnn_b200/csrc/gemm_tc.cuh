@@ -192,6 +192,97 @@ __device__ __forceinline__ void tmem_ld16_sync(uint32_t taddr, uint32_t (&r)[16]
         : "memory");
 }
 
+constexpr int log2_pow2(int v) { return v <= 1 ? 0 : 1 + log2_pow2(v >> 1); }
+
+// Binary bases, one 32-column accumulator chunk of one thread (lane jl of
+// the JA lanes of its output row; JW accumulator columns per output column,
+// so the chunk covers G = 32 / JW output columns).  acc holds s + pad for
+// each base pair (s the +1/-1 product, pad the +1 K padding) as int32
+// (INT_ACC, the int8 kernel) or as an fp32 integer (the e2m1 kernel); s
+// is exact either way.  v_o = sum_i alpha_i[n_o] s_ji (fused multiply-adds
+// in i order), times beta_j; the JA lanes of the row then add their v by a
+// reduce-scatter, low lane bit first: at each step a lane keeps one half of
+// its values, hands the other half to its partner and adds the partner's
+// half of its own, so the adds pair up exactly as a butterfly would, but a
+// row's outputs end up spread over its lanes (P = G / JA consecutive ones
+// each) after G (1 - 1 / JA) shuffles instead of G log2 JA.  With G < JA the
+// last steps are a butterfly and the lowest lane of each group stores.
+// Shared-memory reads (the chunk's 32 alphas as eight broadcast 16-byte
+// loads) and shuffles share the shared-memory pipe with the unpack warps'
+// stores and the MMAs' operand reads, so the epilogue keeps both few.
+template <int JA, int JW, bool INT_ACC>
+__device__ __forceinline__ void bases_combine_chunk(const uint32_t (&acc)[32], const float* ca, int pad, float bj,
+                                                    int jl, float* yrow, int nb, int N, bool vec) {
+    constexpr int G = 32 / JW;
+    constexpr int LOG_JA = log2_pow2(JA), LOG_G = log2_pow2(G);
+    constexpr int SCAT = LOG_JA < LOG_G ? LOG_JA : LOG_G;
+    constexpr int P = G >> SCAT;
+    float v[G];
+    #pragma unroll
+    for (int g = 0; g < G; ++g) v[g] = 0.0f;
+    #pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const float4 a = reinterpret_cast<const float4*>(ca)[q];
+        const float av[4] = {a.x, a.y, a.z, a.w};
+        #pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int col = 4 * q + e;
+            const float s = INT_ACC ? (float)((int32_t)acc[col] - pad) : __uint_as_float(acc[col]) - (float)pad;
+            v[col / JW] = fmaf(av[e], s, v[col / JW]);
+        }
+    }
+    #pragma unroll
+    for (int g = 0; g < G; ++g) v[g] *= bj;
+    int o0 = 0;                                       // first output column (of the chunk) this lane keeps
+    #pragma unroll
+    for (int s = 0; s < SCAT; ++s) {
+        const int half = G >> (s + 1);
+        const bool up = ((jl >> s) & 1) != 0;
+        #pragma unroll
+        for (int h = 0; h < half; ++h) {
+            const float send = up ? v[h] : v[h + half];
+            const float keep = up ? v[h + half] : v[h];
+            v[h] = keep + __shfl_xor_sync(0xffffffffu, send, 1 << s);
+        }
+        if (up) o0 += half;
+    }
+    #pragma unroll
+    for (int s = SCAT; s < LOG_JA; ++s) v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1 << s);
+    if ((jl >> SCAT) != 0 || yrow == nullptr) return;
+    const int n = nb + o0;
+    constexpr int VW = P < 4 ? P : 4;
+    if (vec && VW > 1 && n + P <= N && (n & (VW - 1)) == 0) {
+        #pragma unroll
+        for (int p = 0; p < P; p += VW) {
+            if constexpr (VW == 4) *reinterpret_cast<float4*>(yrow + n + p) = make_float4(v[p], v[p + 1], v[p + 2], v[p + 3]);
+            else if constexpr (VW == 2) *reinterpret_cast<float2*>(yrow + n + p) = make_float2(v[p], v[p + 1]);
+        }
+    } else {
+        #pragma unroll
+        for (int p = 0; p < P; ++p)
+            if (n + p < N) yrow[n + p] = v[p];
+    }
+}
+
+// Dispatch of bases_combine_chunk over (log2 ja, log2 jw), both 0..3; the
+// shape is the same for the whole launch.
+template <bool INT_ACC>
+__device__ __forceinline__ void bases_combine(int shape, const uint32_t (&acc)[32], const float* ca, int pad, float bj,
+                                              int jl, float* yrow, int nb, int N, bool vec) {
+    switch (shape) {
+#define BNN_BASES_CASE(LA, LW)                                                                        \
+    case (LA) * 4 + (LW):                                                                             \
+        bases_combine_chunk<1 << (LA), 1 << (LW), INT_ACC>(acc, ca, pad, bj, jl, yrow, nb, N, vec);   \
+        break;
+        BNN_BASES_CASE(0, 0) BNN_BASES_CASE(0, 1) BNN_BASES_CASE(0, 2) BNN_BASES_CASE(0, 3)
+        BNN_BASES_CASE(1, 0) BNN_BASES_CASE(1, 1) BNN_BASES_CASE(1, 2) BNN_BASES_CASE(1, 3)
+        BNN_BASES_CASE(2, 0) BNN_BASES_CASE(2, 1) BNN_BASES_CASE(2, 2) BNN_BASES_CASE(2, 3)
+        BNN_BASES_CASE(3, 0) BNN_BASES_CASE(3, 1) BNN_BASES_CASE(3, 2) BNN_BASES_CASE(3, 3)
+#undef BNN_BASES_CASE
+        default: break;
+    }
+}
+
 // Bounded wait that also gives up as soon as another role of the CTA aborted.
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -589,11 +680,10 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     } else {
         // ------------------------- epilogue warps, bases mode -------------------------
         // Accumulator lane L holds base j = L mod ja of output row L / ja;
-        // column c holds base i = c mod jw of output column c / jw.  Each
-        // thread forms v = sum_i alpha_i[n] * s_ji for its base j, scales it by
-        // beta_j, and a butterfly over the ja lanes of the row adds the bases
-        // j (every lane of the group ends with the same total).  Padded bases
-        // have beta_j = 0 or alpha_i[n] = 0, so their products add exactly 0.
+        // column c holds base i = c mod jw of output column c / jw.
+        // bases_combine forms each output from its ja x jw accumulators.
+        // Padded bases have beta_j = 0 or alpha_i[n] = 0, so their products
+        // add exactly 0.
         const int quad = warp & 3;
         const int ja = pl.ja, jw = pl.jw;
         float* wcola = reinterpret_cast<float*>(colf + (warp - WARP_EPI0) * BN);   // alpha per column
@@ -603,6 +693,8 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const int jl = L & (ja - 1);
         const float bj = jl < pl.j_real ? __ldg(pl.beta + jl) : 0.0f;
         const int outs_per_chunk = 32 / jw;                           // output columns per 32 accumulator columns
+        const int shape = log2_pow2(ja) * 4 + log2_pow2(jw);
+        const bool vec = ((reinterpret_cast<uintptr_t>(pl.y) | ((uintptr_t)pl.ldy * 4u)) & 15u) == 0;
         int lt = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++lt) {
             const int b = lt & 1;
@@ -627,22 +719,8 @@ xnor_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 }
                 const int nb = n0 + c * outs_per_chunk;
                 if (nb >= N) continue;                                // uniform across the warp
-                // Columns in order; after the last base of each output column
-                // (every jw columns, the same for all lanes) the row total is
-                // formed and stored.  Register indices stay compile-time.
-                float v = 0.0f;
-                #pragma unroll
-                for (int col = 0; col < 32; ++col) {
-                    v = fmaf(wcola[32 * c + col], (float)((int32_t)r[col] - pad), v);
-                    if (((col + 1) & (jw - 1)) == 0) {
-                        float tsum = bj * v;
-                        for (int off = 1; off < ja; off <<= 1) tsum += __shfl_xor_sync(0xffffffffu, tsum, off);
-                        const int o = col / jw;
-                        const int n = nb + o;
-                        if ((o & (ja - 1)) == jl && m < M && n < N) pl.y[(int64_t)m * pl.ldy + n] = tsum;
-                        v = 0.0f;
-                    }
-                }
+                float* yrow = m < M ? pl.y + (int64_t)m * pl.ldy : nullptr;
+                bases_combine<true>(shape, r, wcola + 32 * c, pad, bj, jl, yrow, nb, N, vec);
             }
         }
     }
