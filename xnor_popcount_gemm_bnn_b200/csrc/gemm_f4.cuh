@@ -64,11 +64,8 @@ constexpr int MAX_PSTAGES = 8;
 constexpr int OUT_BLOCK = 32 * 32 * 4;
 constexpr int OUT_BYTES = EPI_WARPS * 2 * OUT_BLOCK;
 // Per-tile column parameters, one copy shared by the epilogue warps, double
-// buffered across tiles: five arrays [2][BN_MAX] of 4-byte values (alpha,
-// gamma, beta as fp32; c1, len2 as int32), so that an epilogue thread reads
-// four columns' worth of one parameter with one 16-byte load.
-constexpr int COLP_ARRAYS = 5;
-constexpr int COLP_BYTES = COLP_ARRAYS * 2 * BN_MAX * 4;
+// buffered across tiles: float4 {alpha, gamma, beta, -} and int2 {c1, len2}.
+constexpr int COLP_BYTES = 2 * BN_MAX * (16 + 8);
 static_assert(ACC_STRIDE + BN_MAX <= SF_COL, "accumulators overlap the scale factors");
 static_assert(U_A_BYTES % 1024 == 0 && OUT_BLOCK % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 // Named barrier of the epilogue warps (id 0 is __syncthreads).
@@ -298,8 +295,9 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     uint8_t* uring = smem;                                          // USTAGES x (A 16 KiB | W rows)
     uint8_t* oring = uring + USTAGES * U_STAGE;                     // [EPI_WARPS][int32 | fp32] 32 x 32 blocks
     uint8_t* pring = oring + OUT_BYTES;                             // PSTAGES x (A | W packed)
-    float* colp = reinterpret_cast<float*>(pring + PSTAGES * P_STAGE);     // COLP_ARRAYS x [2][BN_MAX]
-    uint64_t* bars = reinterpret_cast<uint64_t*>(colp + COLP_ARRAYS * 2 * BN_MAX);
+    float4* colf = reinterpret_cast<float4*>(pring + PSTAGES * P_STAGE);   // [2][BN_MAX]
+    int2* colt = reinterpret_cast<int2*>(colf + 2 * BN_MAX);               // [2][BN_MAX]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(colt + 2 * BN_MAX);
     uint64_t* pfull = bars;
     uint64_t* pempty = pfull + MAX_PSTAGES;
     uint64_t* ufull = pempty + MAX_PSTAGES;
@@ -580,11 +578,8 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         for (int t = cid; t < tiles; t += ncl, ++lt) {
             const int b = lt & 1;
             const int m0 = (t / tiles_n) * (BM * CTAS) + BM * (int)rank, n0 = (t % tiles_n) * bn;
-            float* ca = colp + b * BN_MAX;                            // alpha
-            float* cg = ca + 2 * BN_MAX;                              // gamma
-            float* cb = cg + 2 * BN_MAX;                              // beta
-            int* c1 = reinterpret_cast<int*>(cb + 2 * BN_MAX);        // threshold range start
-            int* cl = c1 + 2 * BN_MAX;                                // and twice its length
+            float4* cf = colf + b * BN_MAX;
+            int2* ct = colt + b * BN_MAX;
             // Every warp finished tile lt - 2 (the last reader of this copy)
             // before it reached the barrier of tile lt - 1.
             for (int i = 32 * ew + lane; i < bn; i += 32 * EPI_WARPS) {
@@ -611,11 +606,8 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         th = make_int2((int)(uint32_t)(kp - 2 * lo), (int)(uint32_t)(2 * len));
                     }
                 }
-                ca[i] = f.x;
-                cg[i] = f.y;
-                cb[i] = f.z;
-                c1[i] = th.x;
-                cl[i] = th.y;
+                cf[i] = f;
+                ct[i] = th;
             }
             named_bar_sync(EPI_BAR, EPI_WARPS * 32);
             ok = ok && __all_sync(0xffffffffu, tc_wait(&afull[b], (lt >> 1) & 1, abort_flag));
@@ -646,15 +638,9 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 if (ep.c_bits != nullptr) {
                     uint32_t word = 0;
                     #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const int4 lo = reinterpret_cast<const int4*>(c1 + 32 * c)[q];
-                        const int4 ln = reinterpret_cast<const int4*>(cl + 32 * c)[q];
-                        const int los[4] = {lo.x, lo.y, lo.z, lo.w}, lns[4] = {ln.x, ln.y, ln.z, ln.w};
-                        #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const int j = 4 * q + k;
-                            word |= ((uint32_t)(los[k] - acc_to_int_scaled<ACC_SCALE>(r[j])) < (uint32_t)lns[k] ? 1u : 0u) << j;
-                        }
+                    for (int j = 0; j < 32; ++j) {
+                        const int2 q = ct[32 * c + j];
+                        word |= ((uint32_t)(q.x - acc_to_int_scaled<ACC_SCALE>(r[j])) < (uint32_t)q.y ? 1u : 0u) << j;
                     }
                     if (m < M && nb / 32 < ep.bits_words) ep.c_bits[(int64_t)m * ep.ldb + nb / 32] = word;
                 }
@@ -707,19 +693,12 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     const bool vec = full_chunk && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0);
                     #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        const float4 a4 = reinterpret_cast<const float4*>(ca + 32 * c)[q];
-                        float4 g4 = make_float4(1.f, 1.f, 1.f, 1.f), b4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (affine) {
-                            g4 = reinterpret_cast<const float4*>(cg + 32 * c)[q];
-                            b4 = reinterpret_cast<const float4*>(cb + 32 * c)[q];
-                        }
-                        const float as[4] = {a4.x, a4.y, a4.z, a4.w}, gs[4] = {g4.x, g4.y, g4.z, g4.w},
-                                    bs[4] = {b4.x, b4.y, b4.z, b4.w};
                         float y[4];
                         #pragma unroll
                         for (int k = 0; k < 4; ++k) {
-                            float v = as[k] * fmaf(__uint_as_float(r[4 * q + k]), (float)ACC_SCALE, -padf);
-                            if (affine) v = fmaf(gs[k], v, bs[k]);
+                            const float4 f = cf[32 * c + 4 * q + k];
+                            float v = f.x * fmaf(__uint_as_float(r[4 * q + k]), (float)ACC_SCALE, -padf);
+                            if (affine) v = fmaf(f.y, v, f.z);
                             y[k] = v;
                         }
                         if (tma_f) {
@@ -778,7 +757,7 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         for (int t = cid; t < tiles; t += ncl, ++lt) {
             const int b = lt & 1;
             const int m0 = (t / tiles_n) * (rows_cta * CTAS) + rows_cta * (int)rank, n0 = (t % tiles_n) * cols_tile;
-            float* ca = colp + b * BN_MAX;                             // alpha of each accumulator column
+            float* ca = reinterpret_cast<float*>(colf + b * BN_MAX);   // alpha of each accumulator column
             for (int i = 32 * ew + lane; i < bn; i += 32 * EPI_WARPS) {
                 const int n = n0 + i / jw, ib = i & (jw - 1);
                 ca[i] = (n < N && ib < pl.i_real) ? __ldg(pl.alpha + (int64_t)ib * pl.lda_alpha + n) : 0.0f;
