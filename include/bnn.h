@@ -320,7 +320,14 @@ bnn_status bnn_xnor_gemv_ex(const uint32_t* W, int64_t ldw, const void* x, bnn_d
 
 /* bnn_xnor_gemv_host -- bnn_xnor_gemv_ex for a caller whose x and y live in
  * host memory: on `stream`, copies x (K elements) from host to device, runs
- * the GEMV, and copies y (N fp32 values) back, one cudaMemcpyAsync each way.
+ * the GEMV, and copies y (N fp32 values) back.  When both host buffers are
+ * pinned memory that the device can address (cudaHostAlloc / cudaMallocHost
+ * or cudaHostRegister, mapped into the unified address space), both buffers
+ * and y_dev are 16-byte aligned and both byte counts are multiples of 16, the
+ * copies are two small kernels whose loads and stores cross PCIe, chained to
+ * the GEMV by programmatic dependent launch (x is read before the wait for
+ * the previous work on the stream and written to x_dev after it).  Otherwise
+ * each copy is one cudaMemcpyAsync.
  *   Passage: as bnn_xnor_gemv ("First Principles ...", "Bandwidth math";
  *   eq. (4), (6) and (1) of "Extreme Quantization ...").
  *   W, ldw, alpha  device, as in bnn_xnor_gemv (W and alpha are the model's
@@ -330,7 +337,8 @@ bnn_status bnn_xnor_gemv_ex(const uint32_t* W, int64_t ldw, const void* x, bnn_d
  *            the call may then block the host until the copy is done.
  *   x_dev    device scratch for x, >= K elements of x_dt, 16-byte aligned,
  *            owned by the caller (the library allocates nothing).
- *   y_dev    device scratch for y, >= N fp32, 4-byte aligned.
+ *   y_dev    device scratch for y, >= N fp32, 4-byte aligned (16 for the
+ *            kernel copies).
  *   y_host   host memory for the N fp32 outputs alpha[n] * s (pinned for an
  *            asynchronous copy); valid once `stream` reaches the end of the
  *            call's work (e.g. after cudaStreamSynchronize).

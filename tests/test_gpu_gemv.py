@@ -277,28 +277,61 @@ def test_independent_gemvs_all_flags(use_graph):
     assert_no_device_error()
 
 
-@pytest.mark.parametrize("pinned", [True, False], ids=["pinned", "pageable"])
-def test_host_buffer_entry_matches_device_gemv(pinned):
+@pytest.mark.parametrize("pin_x,pin_y", [(True, True), (False, False), (True, False), (False, True)],
+                         ids=["pinned", "pageable", "pinned_x", "pinned_y"])
+@pytest.mark.parametrize("N,K,x_dt", [(3000, 4096, torch.bfloat16), (3001, 4095, torch.bfloat16),
+                                      (11008, 4096, torch.bfloat16), (517, 1000, torch.float32)])
+def test_host_buffer_entry_matches_device_gemv(pin_x, pin_y, N, K, x_dt):
     """bnn_xnor_gemv_host (x and y in host memory, copies inside the call)
     gives the same y as bnn_xnor_gemv on device buffers, bit for bit, on two
-    calls in a row with different x."""
-    N, K = 3000, 4096
+    calls in a row with different x.  Pinned x and y with 16-byte multiples
+    take the kernel copies over PCIe; pageable buffers, odd byte counts
+    (K = 4095 bf16, N = 3001 or 517) take the copy engines."""
     d = dev()
     W = workloads.normal((N, K), 0.02, 91)
     W_p = bnn.empty_packed(N, K, d)
     alpha = torch.empty(N, dtype=torch.float32, device=d)
     bnn.bnn_pack_sign(W.to(d), W_p, alpha)
-    x_dev = torch.empty(K, dtype=torch.bfloat16, device=d)
+    x_dev = torch.empty(K, dtype=x_dt, device=d)
     y_dev = torch.empty(N, dtype=torch.float32, device=d)
     for seed in (92, 93):
-        x = workloads.normal((K,), 1.0, seed, dtype=torch.bfloat16)
-        x_host = x.pin_memory() if pinned else x.clone()
+        x = workloads.normal((K,), 1.0, seed, dtype=x_dt)
+        x_host = x.pin_memory() if pin_x else x.clone()
         y_host = torch.full((N,), float("nan"), dtype=torch.float32)
-        if pinned:
+        if pin_y:
             y_host = y_host.pin_memory()
         bnn.bnn_xnor_gemv_host(W_p, x_host, K, alpha, x_dev, y_dev, y_host, flags=bnn.BNN_GEMV_WEIGHTS_STATIC)
         torch.cuda.synchronize()
         y_ref = torch.empty(N, dtype=torch.float32, device=d)
         bnn.bnn_xnor_gemv(W_p, x.to(d), K, alpha, None, y_ref)
         assert torch.equal(y_host, y_ref.cpu())
+    assert_no_device_error()
+
+
+def test_host_buffer_entry_chained_steps():
+    """Twelve host-buffer calls enqueued back to back with no host
+    synchronisation (the kernel copies chained by programmatic dependent
+    launch), each with its own pinned x and y and the shared device scratch:
+    every y equals the device GEMV of its own x, so no step's copy overtook
+    the previous step's use of the scratch."""
+    N, K, steps = 11008, 4096, 12
+    d = dev()
+    W = workloads.normal((N, K), 0.02, 95)
+    W_p = bnn.empty_packed(N, K, d)
+    alpha = torch.empty(N, dtype=torch.float32, device=d)
+    bnn.bnn_pack_sign(W.to(d), W_p, alpha)
+    xs = [workloads.normal((K,), 1.0, 200 + i, dtype=torch.bfloat16) for i in range(steps)]
+    x_hosts = [x.pin_memory() for x in xs]
+    y_hosts = [torch.full((N,), float("nan"), dtype=torch.float32).pin_memory() for _ in range(steps)]
+    x_dev = torch.empty(K, dtype=torch.bfloat16, device=d)
+    y_dev = torch.empty(N, dtype=torch.float32, device=d)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        bnn.bnn_xnor_gemv_host(W_p, x_hosts[i], K, alpha, x_dev, y_dev, y_hosts[i],
+                               flags=bnn.BNN_GEMV_WEIGHTS_STATIC)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        y_ref = torch.empty(N, dtype=torch.float32, device=d)
+        bnn.bnn_xnor_gemv(W_p, xs[i].to(d), K, alpha, None, y_ref)
+        assert torch.equal(y_hosts[i], y_ref.cpu()), f"step {i}"
     assert_no_device_error()

@@ -23,6 +23,7 @@
 #include "gemm_tc.cuh"
 #include "gemm_f4.cuh"
 #include "gemv.cuh"
+#include "hostio.cuh"
 #include "bwgemv.cuh"
 #include "bwgemv_i8.cuh"
 #include "pack.cuh"
@@ -531,6 +532,40 @@ bnn_status gemv_impl(const uint32_t* W, int64_t ldw, const void* x, bnn_dtype x_
                          weights_static, inputs_static, independent, as_cuda(stream));
 }
 
+// The device address of a host buffer that the device can access (pinned
+// memory from cudaHostAlloc / cudaMallocHost or cudaHostRegister, mapped
+// into the unified address space), else nullptr (pageable memory).
+void* mapped_host_view(const void* p) {
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return a.type == cudaMemoryTypeHost ? a.devicePointer : nullptr;
+}
+
+// copy16_kernel with programmatic dependent launch, enough blocks for one
+// pass of VEC vectors per thread (capped).
+template <bool SRC_EARLY>
+bnn_status launch_copy16(const void* src, void* dst, size_t n16, cudaStream_t stream) {
+    if (n16 == 0) return BNN_OK;
+    const int64_t per_block = (int64_t)bnn::hostio::THREADS * bnn::hostio::VEC;
+    const int64_t blocks = std::min<int64_t>(ceil_div((int64_t)n16, per_block), bnn::hostio::MAX_BLOCKS);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(bnn::hostio::THREADS);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, bnn::copy16_kernel<SRC_EARLY>, static_cast<const uint4*>(src),
+                           static_cast<uint4*>(dst), (int64_t)n16) != cudaSuccess)
+        return BNN_ERR_CUDA;
+    return BNN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -835,6 +870,20 @@ bnn_status bnn_xnor_gemv_host(const uint32_t* W, int64_t ldw, const void* x_host
     if (!aligned(x_dev, 16) || !aligned(y_dev, 4)) return BNN_ERR_ALIGNMENT;
     const size_t xbytes = (size_t)K * (x_dt == BNN_F32 ? 4 : 2), ybytes = (size_t)N * 4;
     cudaStream_t s = as_cuda(stream);
+    // Pinned host buffers that the device can address take the two copies as
+    // small kernels chained to the GEMV (hostio.cuh); other host memory, and
+    // sizes or alignments that 16-byte vectors do not fit, take the copy
+    // engines.
+    const void* x_map = mapped_host_view(x_host);
+    void* y_map = mapped_host_view(y_host);
+    if (x_map != nullptr && y_map != nullptr && aligned(x_map, 16) && aligned(y_map, 16) && aligned(y_dev, 16) &&
+        xbytes % 16 == 0 && ybytes % 16 == 0) {
+        bnn_status st = launch_copy16<true>(x_map, x_dev, xbytes / 16, s);
+        if (st != BNN_OK) return st;
+        if ((st = bnn_xnor_gemv_ex(W, ldw, x_dev, x_dt, N, K, alpha, nullptr, y_dev, flags, stream)) != BNN_OK)
+            return st;
+        return N > 0 ? launch_copy16<false>(y_dev, y_map, ybytes / 16, s) : BNN_OK;
+    }
     if (cudaMemcpyAsync(x_dev, x_host, xbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return BNN_ERR_CUDA;
     const bnn_status st = bnn_xnor_gemv_ex(W, ldw, x_dev, x_dt, N, K, alpha, nullptr, y_dev, flags, stream);
     if (st != BNN_OK) return st;
