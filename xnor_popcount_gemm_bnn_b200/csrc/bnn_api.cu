@@ -316,17 +316,21 @@ bnn_status launch_f4_pairs(const CUtensorMap& tmA, const CUtensorMap& tmW, const
     using C = bnn::f4::Cfg<true, MODE>;
     const int64_t clusters = std::min<int64_t>(tiles_m * tiles_n, pairs);
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // The kernel's set-up may overlap the previous kernel's last tiles; its
+    // loads and stores wait for that kernel (griddepcontrol.wait).
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3((unsigned)(2 * clusters));
     cfg.blockDim = dim3(C::THREADS);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = stream;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, bnn::xnor_gemm_f4_kernel<true, MODE>, tmA, tmW, tmCi, tmCf, (int)M, (int)N, (int)K,
                            (int)kw, bn, (int)tiles_m, (int)tiles_n, tma_out, e, pl) != cudaSuccess)
         return BNN_ERR_CUDA;

@@ -360,12 +360,21 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     tc_fence_before();
     if constexpr (PAIR) cluster_sync_all(); else __syncthreads();
     tc_fence_after();
+    // Programmatic dependent launch (CTA-pair launches carry the attribute):
+    // everything above -- barriers, tensor memory, scale factors -- ran while
+    // the previous kernel on the stream may still be finishing.  The reads of
+    // memory that kernel may write (the operand tiles, the epilogue's column
+    // parameters) and every global store come after griddepcontrol.wait in
+    // the producer and epilogue warps below.  All CTAs are resident, so the
+    // next launch may be scheduled now: its CTAs take SMs as these exit.
+    grid_dependents_launch();
 
     if (warp == WARP_PRODUCER) {
         // ------------------------------ TMA producer ------------------------------
         if (lane == 0) {
             uint32_t g = 0, issued = 0;
             bool ok = true;
+            grid_dependency_wait();
             // TMA coordinates in rows of the operand tensors (code or output
             // rows; the 3-D boxes bring each row's planes along).
             const int rows_w = MODE == TC_BASES ? bn_cta / jw : bn_cta;
@@ -558,6 +567,7 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         // tensor map are stored directly.  The barrier is reached the same
         // number of times by every warp, also after a failed wait (the warp
         // then skips the work), so it cannot hang.
+        grid_dependency_wait();
         const int quad = warp & 3;                                    // TMEM lanes 32*quad .. 32*quad + 31
         const int ew = warp - WARP_EPI0;                              // 0..3
         uint8_t* obuf_i = oring + ew * 2 * OUT_BLOCK;                 // this warp's int32 block
@@ -740,6 +750,7 @@ xnor_gemm_f4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         // Padded bases have beta_j = 0 or alpha_i[n] = 0 and add exactly 0.
         // The per-tile alpha of every accumulator column sits in the shared
         // double-buffered copy, behind the same named barrier as the other modes.
+        grid_dependency_wait();
         const int quad = warp & 3;
         const int ew = warp - WARP_EPI0;
         const int kp = nk * S_BKE;
