@@ -1435,8 +1435,21 @@ bnn_status bnn_binary_conv3x3_fused(const uint32_t* X_nhwc_bits, int64_t n, int6
             auto launch_w = [&](auto kern) -> bnn_status {
                 if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_w) != cudaSuccess)
                     return BNN_ERR_CUDA;
-                kern<<<(unsigned)grid, bnn::ctw::THREADS, smem_w, s>>>(X_nhwc_bits, (int)c, W_packed, ldw, (int)cout,
-                                                                       (int)n_mma, idesc, g, ep);
+                // Programmatic dependent launch: the kernel's set-up overlaps
+                // the previous kernel; its reads and stores wait for it.
+                cudaLaunchConfig_t cfg{};
+                cfg.gridDim = dim3((unsigned)grid);
+                cfg.blockDim = dim3(bnn::ctw::THREADS);
+                cfg.dynamicSmemBytes = (size_t)smem_w;
+                cfg.stream = s;
+                cudaLaunchAttribute attr[1];
+                attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+                attr[0].val.programmaticStreamSerializationAllowed = 1;
+                cfg.attrs = attr;
+                cfg.numAttrs = 1;
+                if (cudaLaunchKernelEx(&cfg, kern, X_nhwc_bits, (int)c, W_packed, ldw, (int)cout, (int)n_mma, idesc, g,
+                                       ep) != cudaSuccess)
+                    return BNN_ERR_CUDA;
                 return launch_status();
             };
             if (f4) return cw == 2 ? launch_w(bnn::xnor_conv3x3_tcw_kernel<2, true>)

@@ -359,12 +359,6 @@ xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* _
     const uint32_t tmem_cols = used_cols <= 128 ? 128u : (used_cols <= 256 ? 256u : 512u);
     const uint32_t sf_col = (uint32_t)(2 * acc_stride);
 
-    for (int i = threadIdx.x; i < n_mma; i += blockDim.x) {
-        const bool real = i < cout && ep.mode != BNN_OUT_INT32;
-        s_alpha[i] = real ? __ldg(ep.alpha + i) : 0.0f;
-        s_gamma[i] = real && ep.mode == BNN_OUT_AFFINE_F32 ? __ldg(ep.gamma + i) : 0.0f;
-        s_beta[i] = real && ep.mode == BNN_OUT_AFFINE_F32 ? __ldg(ep.beta + i) : 0.0f;
-    }
     if (threadIdx.x == 0) {
         for (int b = 0; b < AHEAD; ++b) {
             mbar_init(&afill[b], GATHER_WARPS);
@@ -396,6 +390,20 @@ xnor_conv3x3_tcw_kernel(const uint32_t* __restrict__ X, int c, const uint32_t* _
         __syncthreads();
         tc_fence_after();
     }
+    // Programmatic dependent launch: the set-up above ran while the previous
+    // kernel on the stream may still be finishing.  Every read of memory it
+    // may write (epilogue parameters, filters, the packed input) and every
+    // store come after this wait.  The grid is resident, so the next launch
+    // may be scheduled now; its CTAs take SMs as these exit.
+    grid_dependents_launch();
+    grid_dependency_wait();
+    for (int i = threadIdx.x; i < n_mma; i += blockDim.x) {
+        const bool real = i < cout && ep.mode != BNN_OUT_INT32;
+        s_alpha[i] = real ? __ldg(ep.alpha + i) : 0.0f;
+        s_gamma[i] = real && ep.mode == BNN_OUT_AFFINE_F32 ? __ldg(ep.gamma + i) : 0.0f;
+        s_beta[i] = real && ep.mode == BNN_OUT_AFFINE_F32 ? __ldg(ep.beta + i) : 0.0f;
+    }
+    __syncthreads();
 
     if (warp == WARP_MMA) {
         // ------------------------------ MMA issuer ------------------------------
