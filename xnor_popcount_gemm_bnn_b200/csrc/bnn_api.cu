@@ -1562,8 +1562,19 @@ bnn_status bnn_binary_conv1x1_fused(const uint32_t* X_nhwc_bits, int64_t n, int6
         if (smem > 48 * 1024 &&
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
             return BNN_ERR_CUDA;
-        kern<<<(unsigned)blocks, bnn::conv::THREADS, smem, s>>>(X_nhwc_bits, (int)n, (int)c, (int)h, (int)w, W_packed,
-                                                                ldw, (int)cout, (int)stride, (int)oh, (int)ow, ep);
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3((unsigned)blocks);
+        cfg.blockDim = dim3(bnn::conv::THREADS);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kern, X_nhwc_bits, (int)n, (int)c, (int)h, (int)w, W_packed, ldw, (int)cout,
+                               (int)stride, (int)oh, (int)ow, ep) != cudaSuccess)
+            return BNN_ERR_CUDA;
         return launch_status();
     };
     auto by_mode = [&](auto k_int, auto k_scaled, auto k_affine) -> bnn_status {

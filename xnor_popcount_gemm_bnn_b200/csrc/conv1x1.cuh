@@ -53,6 +53,12 @@ xnor_conv1x1_kernel(const uint32_t* __restrict__ X, int n, int c, int h, int w, 
     const int cw = (c + 31) / 32;
     float* ga = reinterpret_cast<float*>(ws1 + cout * KWP);
     float* be = ga + cout;
+    // Programmatic dependent launch: the next launch may be scheduled once
+    // every CTA of this grid has started (its CTAs then take SMs as these
+    // exit); every read of memory the previous kernel may write (filters,
+    // parameters, input) and every store follow the wait for that kernel.
+    grid_dependents_launch();
+    grid_dependency_wait();
     for (int i = threadIdx.x; i < cout * KWP; i += THREADS) {
         const int co = i / KWP, k = i % KWP;
         ws1[i] = (k < cw) ? Wp[(int64_t)co * ldw + k] : 0u;
