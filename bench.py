@@ -524,11 +524,13 @@ def e2e_gemv(torch, bnn, g, Ws, alpha, dev, steps, sync, max_over_ranks, ws):
     call = bnn._lib.bnn_xnor_gemv_host
     args = [(ctypes.c_void_p(W.data_ptr()), W.stride(0), ctypes.c_void_p(x_host.data_ptr()), bnn.BNN_BF16, g.N, g.K,
              ctypes.c_void_p(alpha.data_ptr()), ctypes.c_void_p(x_dev.data_ptr()), ctypes.c_void_p(y_dev.data_ptr()),
-             ctypes.c_void_p(y_host.data_ptr()), bnn.BNN_GEMV_WEIGHTS_STATIC, stream) for W in Ws]
+             ctypes.c_void_p(y_host.data_ptr()), bnn.BNN_GEMV_WEIGHTS_STATIC | bnn.BNN_GEMV_INPUTS_STATIC, stream)
+            for W in Ws]
     assert g.x.dtype == torch.bfloat16
 
     def one(i):
-        # x arrives by the copy inside the call: only the weights are static.
+        # x comes from the host buffer, which no device work writes (INPUTS_STATIC
+        # lets the copy-in read it early); the GEMV's x is written by that copy.
         st = call(*args[i % copies])
         if st != bnn.BNN_OK:
             raise bnn.BnnError("bnn_xnor_gemv_host", st, bnn._lib.bnn_status_string(st).decode())

@@ -325,9 +325,8 @@ bnn_status bnn_xnor_gemv_ex(const uint32_t* W, int64_t ldw, const void* x, bnn_d
  * or cudaHostRegister, mapped into the unified address space), both buffers
  * and y_dev are 16-byte aligned and both byte counts are multiples of 16, the
  * copies are two small kernels whose loads and stores cross PCIe, chained to
- * the GEMV by programmatic dependent launch (x is read before the wait for
- * the previous work on the stream and written to x_dev after it).  Otherwise
- * each copy is one cudaMemcpyAsync.
+ * the GEMV by programmatic dependent launch.  Otherwise each copy is one
+ * cudaMemcpyAsync.
  *   Passage: as bnn_xnor_gemv ("First Principles ...", "Bandwidth math";
  *   eq. (4), (6) and (1) of "Extreme Quantization ...").
  *   W, ldw, alpha  device, as in bnn_xnor_gemv (W and alpha are the model's
@@ -342,9 +341,14 @@ bnn_status bnn_xnor_gemv_ex(const uint32_t* W, int64_t ldw, const void* x, bnn_d
  *   y_host   host memory for the N fp32 outputs alpha[n] * s (pinned for an
  *            asynchronous copy); valid once `stream` reaches the end of the
  *            call's work (e.g. after cudaStreamSynchronize).
- *   flags    BNN_GEMV_WEIGHTS_STATIC or 0 (x is written by the copy just
- *            before the kernel, and y is read by the copy after it, so the
- *            other flags do not apply).
+ *   flags    0, BNN_GEMV_WEIGHTS_STATIC (as in bnn_xnor_gemv_ex) and/or
+ *            BNN_GEMV_INPUTS_STATIC, which here says that no earlier work on
+ *            the stream that may still be running writes x_host: the copy
+ *            kernel then reads x_host before waiting for that work (its PCIe
+ *            latency overlaps it) and writes x_dev after.  Without it the
+ *            read follows the wait, as a copy in stream order would.
+ *            BNN_GEMV_OUTPUT_FREE does not apply (y is read by the copy
+ *            after the kernel).
  *   Errors: INVALID_ARG (null pointer, bad size or flag), ALIGNMENT, and the
  *   errors of bnn_xnor_gemv; BNN_ERR_CUDA when a copy cannot be enqueued. */
 bnn_status bnn_xnor_gemv_host(const uint32_t* W, int64_t ldw, const void* x_host, bnn_dtype x_dt, int64_t N,

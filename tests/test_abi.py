@@ -161,7 +161,8 @@ def test_gemm_engine_setting_on_host():
 def test_gemv_host_entry_rejects_bad_arguments():
     f = L.bnn_xnor_gemv_host
     # W, ldw, x_host, dt, N, K, alpha, x_dev, y_dev, y_host, flags, stream
-    assert f(FAKE, 128, FAKE, 1, 8, 4096, FAKE, FAKE, FAKE, FAKE, 2, NULL) == bnn.BNN_ERR_INVALID_ARG    # inputs static
+    assert f(FAKE, 128, FAKE, 1, 8, 4096, FAKE, FAKE, FAKE, FAKE, 8, NULL) == bnn.BNN_ERR_INVALID_ARG    # unknown bit
+    assert f(FAKE, 128, FAKE, 1, 8, 4096, FAKE, FAKE, FAKE, FAKE, 7, NULL) == bnn.BNN_ERR_INVALID_ARG    # all three
     assert f(FAKE, 128, FAKE, 1, 8, 4096, FAKE, FAKE, FAKE, FAKE, 4, NULL) == bnn.BNN_ERR_INVALID_ARG    # output free
     assert f(FAKE, 128, NULL, 1, 8, 4096, FAKE, FAKE, FAKE, FAKE, 0, NULL) == bnn.BNN_ERR_INVALID_ARG    # no x_host
     assert f(FAKE, 128, FAKE, 1, 8, 4096, FAKE, NULL, FAKE, FAKE, 0, NULL) == bnn.BNN_ERR_INVALID_ARG    # no x_dev

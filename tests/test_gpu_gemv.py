@@ -281,7 +281,9 @@ def test_independent_gemvs_all_flags(use_graph):
                          ids=["pinned", "pageable", "pinned_x", "pinned_y"])
 @pytest.mark.parametrize("N,K,x_dt", [(3000, 4096, torch.bfloat16), (3001, 4095, torch.bfloat16),
                                       (11008, 4096, torch.bfloat16), (517, 1000, torch.float32)])
-def test_host_buffer_entry_matches_device_gemv(pin_x, pin_y, N, K, x_dt):
+@pytest.mark.parametrize("flags", [bnn.BNN_GEMV_WEIGHTS_STATIC,
+                                   bnn.BNN_GEMV_WEIGHTS_STATIC | bnn.BNN_GEMV_INPUTS_STATIC], ids=["w", "wx"])
+def test_host_buffer_entry_matches_device_gemv(pin_x, pin_y, N, K, x_dt, flags):
     """bnn_xnor_gemv_host (x and y in host memory, copies inside the call)
     gives the same y as bnn_xnor_gemv on device buffers, bit for bit, on two
     calls in a row with different x.  Pinned x and y with 16-byte multiples
@@ -300,7 +302,7 @@ def test_host_buffer_entry_matches_device_gemv(pin_x, pin_y, N, K, x_dt):
         y_host = torch.full((N,), float("nan"), dtype=torch.float32)
         if pin_y:
             y_host = y_host.pin_memory()
-        bnn.bnn_xnor_gemv_host(W_p, x_host, K, alpha, x_dev, y_dev, y_host, flags=bnn.BNN_GEMV_WEIGHTS_STATIC)
+        bnn.bnn_xnor_gemv_host(W_p, x_host, K, alpha, x_dev, y_dev, y_host, flags=flags)
         torch.cuda.synchronize()
         y_ref = torch.empty(N, dtype=torch.float32, device=d)
         bnn.bnn_xnor_gemv(W_p, x.to(d), K, alpha, None, y_ref)
@@ -308,7 +310,9 @@ def test_host_buffer_entry_matches_device_gemv(pin_x, pin_y, N, K, x_dt):
     assert_no_device_error()
 
 
-def test_host_buffer_entry_chained_steps():
+@pytest.mark.parametrize("flags", [bnn.BNN_GEMV_WEIGHTS_STATIC,
+                                   bnn.BNN_GEMV_WEIGHTS_STATIC | bnn.BNN_GEMV_INPUTS_STATIC], ids=["w", "wx"])
+def test_host_buffer_entry_chained_steps(flags):
     """Twelve host-buffer calls enqueued back to back with no host
     synchronisation (the kernel copies chained by programmatic dependent
     launch), each with its own pinned x and y and the shared device scratch:
@@ -327,8 +331,7 @@ def test_host_buffer_entry_chained_steps():
     y_dev = torch.empty(N, dtype=torch.float32, device=d)
     torch.cuda.synchronize()
     for i in range(steps):
-        bnn.bnn_xnor_gemv_host(W_p, x_hosts[i], K, alpha, x_dev, y_dev, y_hosts[i],
-                               flags=bnn.BNN_GEMV_WEIGHTS_STATIC)
+        bnn.bnn_xnor_gemv_host(W_p, x_hosts[i], K, alpha, x_dev, y_dev, y_hosts[i], flags=flags)
     torch.cuda.synchronize()
     for i in range(steps):
         y_ref = torch.empty(N, dtype=torch.float32, device=d)

@@ -866,7 +866,7 @@ bnn_status bnn_xnor_gemv_ex(const uint32_t* W, int64_t ldw, const void* x, bnn_d
 bnn_status bnn_xnor_gemv_host(const uint32_t* W, int64_t ldw, const void* x_host, bnn_dtype x_dt, int64_t N,
                               int64_t K, const float* alpha, void* x_dev, float* y_dev, float* y_host, uint32_t flags,
                               bnn_stream_t stream) {
-    if (flags != 0 && flags != BNN_GEMV_WEIGHTS_STATIC) return BNN_ERR_INVALID_ARG;
+    if ((flags & ~(uint32_t)(BNN_GEMV_WEIGHTS_STATIC | BNN_GEMV_INPUTS_STATIC)) != 0) return BNN_ERR_INVALID_ARG;
     if (x_host == nullptr || x_dev == nullptr || y_dev == nullptr || y_host == nullptr || alpha == nullptr)
         return BNN_ERR_INVALID_ARG;
     if (N < 0 || K < 1 || N > INT_MAX / 2 || K > INT_MAX / 2) return BNN_ERR_INVALID_ARG;
@@ -874,6 +874,8 @@ bnn_status bnn_xnor_gemv_host(const uint32_t* W, int64_t ldw, const void* x_host
     if (!aligned(x_dev, 16) || !aligned(y_dev, 4)) return BNN_ERR_ALIGNMENT;
     const size_t xbytes = (size_t)K * (x_dt == BNN_F32 ? 4 : 2), ybytes = (size_t)N * 4;
     cudaStream_t s = as_cuda(stream);
+    // x_dev is written just before the GEMV: only the weights may be static.
+    const uint32_t gemv_flags = flags & BNN_GEMV_WEIGHTS_STATIC;
     // Pinned host buffers that the device can address take the two copies as
     // small kernels chained to the GEMV (hostio.cuh); other host memory, and
     // sizes or alignments that 16-byte vectors do not fit, take the copy
@@ -882,14 +884,17 @@ bnn_status bnn_xnor_gemv_host(const uint32_t* W, int64_t ldw, const void* x_host
     void* y_map = mapped_host_view(y_host);
     if (x_map != nullptr && y_map != nullptr && aligned(x_map, 16) && aligned(y_map, 16) && aligned(y_dev, 16) &&
         xbytes % 16 == 0 && ybytes % 16 == 0) {
-        bnn_status st = launch_copy16<true>(x_map, x_dev, xbytes / 16, s);
+        // BNN_GEMV_INPUTS_STATIC: nothing in flight writes x_host, so the
+        // copy-in may read it before the previous work on the stream ends.
+        bnn_status st = (flags & BNN_GEMV_INPUTS_STATIC) ? launch_copy16<true>(x_map, x_dev, xbytes / 16, s)
+                                                          : launch_copy16<false>(x_map, x_dev, xbytes / 16, s);
         if (st != BNN_OK) return st;
-        if ((st = bnn_xnor_gemv_ex(W, ldw, x_dev, x_dt, N, K, alpha, nullptr, y_dev, flags, stream)) != BNN_OK)
+        if ((st = bnn_xnor_gemv_ex(W, ldw, x_dev, x_dt, N, K, alpha, nullptr, y_dev, gemv_flags, stream)) != BNN_OK)
             return st;
         return N > 0 ? launch_copy16<false>(y_dev, y_map, ybytes / 16, s) : BNN_OK;
     }
     if (cudaMemcpyAsync(x_dev, x_host, xbytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return BNN_ERR_CUDA;
-    const bnn_status st = bnn_xnor_gemv_ex(W, ldw, x_dev, x_dt, N, K, alpha, nullptr, y_dev, flags, stream);
+    const bnn_status st = bnn_xnor_gemv_ex(W, ldw, x_dev, x_dt, N, K, alpha, nullptr, y_dev, gemv_flags, stream);
     if (st != BNN_OK) return st;
     if (N > 0 && cudaMemcpyAsync(y_host, y_dev, ybytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return BNN_ERR_CUDA;
