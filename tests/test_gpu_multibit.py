@@ -208,6 +208,30 @@ def test_binary_bases_gemm(M, N, K, J, I, tc_engine):
     assert_no_device_error()
 
 
+@pytest.mark.parametrize("J", [1, 2, 4, 8])
+@pytest.mark.parametrize("I", [1, 2, 4, 8])
+_SHAPE_REFS = {}
+
+
+def test_binary_bases_every_combine_shape(J, I, tc_engine):
+    """Every (J', I') instance of the epilogue's per-shape combine (powers of
+    two up to 8 bases a side), at a shape with several row and column tiles
+    and ragged edges, against the oracle (computed once per (J, I))."""
+    M, N, K = 200, 160, 300
+    h_real, b_real, alpha, beta = _bases_case(M, N, K, J, I, 500 + 10 * J + I)
+    H, B = _pack_bases(h_real, J, M, K), _pack_bases(b_real, I, N, K)
+    Y = torch.full((M, N), float("nan"), dtype=torch.float32, device=dev())
+    bnn.bnn_binary_bases_gemm(H, J, B, I, K, beta.to(dev()), alpha.to(dev()), Y)
+    torch.cuda.synchronize()
+    if (J, I) not in _SHAPE_REFS:
+        _SHAPE_REFS[(J, I)] = _bases_reference(h_real, b_real, alpha, beta)
+    y_ref, mag = _SHAPE_REFS[(J, I)]
+    got = Y.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(got))
+    assert np.all(np.abs(got - y_ref) <= (I + J + 2) * U * mag)
+    assert_no_device_error()
+
+
 @pytest.mark.parametrize("col0,ld", [(0, 304), (1, 304), (0, 303), (3, 311)])
 def test_binary_bases_strided_output(col0, ld, tc_engine):
     """Y as a column window of a wider buffer: row strides and start columns
