@@ -208,11 +208,11 @@ def test_binary_bases_gemm(M, N, K, J, I, tc_engine):
     assert_no_device_error()
 
 
-@pytest.mark.parametrize("J", [1, 2, 4, 8])
-@pytest.mark.parametrize("I", [1, 2, 4, 8])
 _SHAPE_REFS = {}
 
 
+@pytest.mark.parametrize("J", [1, 2, 4, 8])
+@pytest.mark.parametrize("I", [1, 2, 4, 8])
 def test_binary_bases_every_combine_shape(J, I, tc_engine):
     """Every (J', I') instance of the epilogue's per-shape combine (powers of
     two up to 8 bases a side), at a shape with several row and column tiles
