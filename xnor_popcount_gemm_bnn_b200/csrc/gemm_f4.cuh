@@ -70,8 +70,8 @@ static_assert(ACC_STRIDE + BN_MAX <= SF_COL, "accumulators overlap the scale fac
 static_assert(U_A_BYTES % 1024 == 0 && OUT_BLOCK % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 // Named barrier of the epilogue warps (id 0 is __syncthreads).
 constexpr int EPI_BAR = 1;
-// Bits per code in the plane-code mode: codes 0..3 are exact e2m1 values
-// (0x0, 0x2 = 1.0, 0x4 = 2.0, 0x5 = 3.0).
+// Bits per code in the plane-code mode: a code c = 0..3 is the e2m1 nibble
+// c, the exact value c / 2 (0, 0.5, 1.0, 1.5); the epilogue scales by 4.
 constexpr int MAX_F4_PLANES = 2;
 // Largest padded K: partial sums stay integers of magnitude <= 2^20, exact
 // in fp32 and in the epilogue's float-to-int conversion (valid below 2^22).
