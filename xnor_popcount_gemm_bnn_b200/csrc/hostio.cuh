@@ -30,6 +30,9 @@ __global__ void __launch_bounds__(hostio::THREADS)
 copy16_kernel(const uint4* src, uint4* dst, int64_t n16) {
     using namespace hostio;
     const int64_t stride = (int64_t)gridDim.x * THREADS;
+    // The grid is a few resident blocks: the next kernel may be scheduled
+    // now and waits for this one itself.
+    grid_dependents_launch();
     if (!SRC_EARLY) grid_dependency_wait();
     for (int64_t base = (int64_t)blockIdx.x * THREADS + threadIdx.x; base < n16; base += stride * VEC) {
         uint4 v[VEC];
